@@ -1,0 +1,337 @@
+"""Benchmark: Falcon chunk-parallel forward, 8x12x2048x64 bf16 (chunk 64),
+Falcon-1 and Falcon-1A, on one or more B200s (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...
+
+One step = one chunk-parallel forward of Falcon-1 and one of Falcon-1A over
+the batch (B*L tokens each, all H heads), inputs resident in HBM.  L2 is
+flushed (a 256 MiB write) before every timed step; each step is timed with
+CUDA events on the launching stream and the job time is the max over ranks.
+Each rank runs the full batch (weak scaling, no collective on the data path).
+
+`--impl reference` times the fp64 CPU oracle (the only reference that exists
+for this method) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(name="falcon1-1A-chunk-bf16-8x12x2048x64", B=8, H=12, L=2048, dk=64, dv=64, chunk=64,
+                variants=("F1", "F1A"), seed=20260002)
+METRIC = "tokens/s for Falcon chunk-parallel fwd (H=12,d=64,L=2K) at 1 B200; % tensor/HBM peak"
+DECODE = dict(variant="F2A", N=64, H=16, dk=128, dv=128, lam=0.02, seed=20260005)
+
+
+def algorithmic_bytes_fwd(B, H, L, dk, dv, per_channel=False, elt=2):
+    """Bytes a chunk-parallel forward must move at least once: q, k, v, beta
+    and out in the input dtype plus the fp32 final state and lambda."""
+    tok = B * H * L
+    return tok * (2 * dk + dv + (dv if per_channel else 1) + dv) * elt + B * H * dv * dk * 4 + H * 4
+
+
+def algorithmic_bytes_decode(N, H, dk, dv, per_channel=True, elt=2):
+    """Per decode step: state read + write (fp32), x_prev read + write (fp32),
+    q, k, v, beta in, out."""
+    nh = N * H
+    return nh * (2 * dv * dk * 4 + 2 * dk * 4 + (2 * dk + dv + (dv if per_channel else 1) + dv) * elt) + H * 4
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def max_over_ranks(x, world):
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+class OracleSample:
+    """The fp64 oracle's chunk-parallel form on whole (b,h) units of the
+    workload (Falcon-1 and Falcon-1A), one batch of units per call, on all
+    host cores.  Inputs are drawn once, identical to the GPU run's."""
+
+    def __init__(self):
+        import oracle
+        from linear_attention_sequence_falcon_b200 import inputs as gen
+        w = WORKLOAD
+        oracle.build()
+        self.oracle = oracle
+        self.d = gen.draw("F1", w["B"], w["H"], w["L"], w["dk"], w["dv"], seed=w["seed"], dtype="bf16")
+        self.units = [(b, h) for b in range(w["B"]) for h in range(w["H"])]
+        self.ncores = os.cpu_count() or 1
+        self.next = 0
+        self.threads = 1
+
+    def step(self):
+        """One batch of min(cores, units) units through both variants;
+        returns (tokens, seconds)."""
+        import numpy as np
+        w = WORKLOAD
+        n = min(self.ncores, len(self.units))
+        batch = [self.units[(self.next + i) % len(self.units)] for i in range(n)]
+        self.next = (self.next + n) % len(self.units)
+        bs = [b for b, _ in batch]
+        hs = [h for _, h in batch]
+        # the selected units become the heads of one batch row, each with its own lambda
+        sel = lambda a: np.ascontiguousarray(a[bs, hs][None])  # noqa: E731
+        args = [sel(self.d[x]) for x in ("q_64", "k_64", "v_64", "beta_64")]
+        lam = np.asarray(self.d["lam_64"])[hs]
+        t0 = time.perf_counter()
+        for variant in w["variants"]:
+            _, _, self.threads = self.oracle.fwd(variant, "chunk", *args, lam, self.d["eps_64"], chunk=w["chunk"],
+                                                 nthreads=self.ncores, return_threads=True)
+        return len(w["variants"]) * n * w["L"], time.perf_counter() - t0
+
+
+def cpu_oracle_sample(budget_s=12.0):
+    """Oracle tokens/s over about budget_s of CPU wall time; returns
+    (tokens/s, threads, units done, seconds)."""
+    smp = OracleSample()
+    tokens, used, units = 0, 0.0, 0
+    while used < budget_s and units < len(smp.units):
+        t, s = smp.step()
+        tokens += t
+        used += s
+        units += min(smp.ncores, len(smp.units))
+    return tokens / used, smp.threads, units, used
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    smp = OracleSample()
+    for _ in range(args.warmup):
+        smp.step()
+    tokens, used = 0, 0.0
+    for _ in range(args.steps):
+        t, s = smp.step()
+        tokens += t
+        used += s
+    value = tokens / used
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": used / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.threads, "kind": "oracle",
+                             "sample": "each step: %d whole (b,h) units of the workload through the fp64 oracle's "
+                                       "chunk-parallel form, Falcon-1 and Falcon-1A" % min(smp.ncores, len(smp.units))},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config():
+    w = WORKLOAD
+    return {"workload": w["name"], "B": w["B"], "H": w["H"], "L": w["L"], "d_k": w["dk"], "d_v": w["dv"],
+            "chunk": w["chunk"], "variants": list(w["variants"]), "global_batch": w["B"], "seq_len": w["L"],
+            "l2": "flushed (256 MiB write) before every timed step", "parallelism": "replicas"}
+
+
+def run_ours(args):
+    import torch
+    import linear_attention_sequence_falcon_b200 as F
+    from linear_attention_sequence_falcon_b200 import build, inputs as gen
+    build.build()
+    F.load()
+    rank, world, local = dist_setup(args)
+    w = WORKLOAD
+    d = gen.draw("F1", w["B"], w["H"], w["L"], w["dk"], w["dv"], seed=w["seed"] + 1000 * rank, dtype="bf16")
+    q, k, v, beta, lam = (d[n].cuda() for n in ("q", "k", "v", "beta", "lam"))
+    outs = {var: torch.empty((w["B"], w["H"], w["L"], w["dv"]), dtype=torch.bfloat16, device="cuda")
+            for var in w["variants"]}
+    states = {var: torch.empty((w["B"], w["H"], w["dv"], w["dk"]), dtype=torch.float32, device="cuda")
+              for var in w["variants"]}
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        for var in w["variants"]:
+            if ev is not None:
+                ev[var][0].record(stream)
+            F.fwd(var, "chunk", q, k, v, beta, lam, d["eps"], chunk=w["chunk"], out=outs[var],
+                  final_state=states[var], stream=stream)
+            if ev is not None:
+                ev[var][1].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    barrier(world)
+    per_var = {var: [] for var in w["variants"]}
+    step_ms = []
+    with Clocks(local) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            ev = {var: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for var in w["variants"]}
+            step(ev)
+            torch.cuda.synchronize()
+            for var in w["variants"]:
+                per_var[var].append(ev[var][0].elapsed_time(ev[var][1]))
+            step_ms.append(sum(ev[var][0].elapsed_time(ev[var][1]) for var in w["variants"]))
+        barrier(world)
+    total_ms = max_over_ranks(sum(step_ms), world)
+    tokens_per_step = len(w["variants"]) * w["B"] * w["L"]
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+
+    # end to end through the C ABI from pinned host buffers
+    hq, hk, hv, hb = (d[n].pin_memory() for n in ("q", "k", "v", "beta"))
+    ho = {var: torch.empty_like(outs[var], device="cpu").pin_memory() for var in w["variants"]}
+    hs = {var: torch.empty_like(states[var], device="cpu").pin_memory() for var in w["variants"]}
+    e2e_ms = []
+    for i in range(max(args.warmup, 3) + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True); beta.copy_(hb, non_blocking=True)
+        step()
+        for var in w["variants"]:
+            ho[var].copy_(outs[var], non_blocking=True)
+            hs[var].copy_(states[var], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= max(args.warmup, 3):
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = max_over_ranks(sum(e2e_ms), world)
+    e2e_value = world * tokens_per_step * args.steps / (e2e_total / 1e3)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb))
+    d2h = sum(ho[var].numel() * ho[var].element_size() + hs[var].numel() * hs[var].element_size()
+              for var in w["variants"])
+
+    hbm, tflops, src = peaks()
+    f1_ms = statistics.mean(per_var["F1"])
+    ab = algorithmic_bytes_fwd(w["B"], w["H"], w["L"], w["dk"], w["dv"])
+    achieved = ab / (f1_ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "traffic": None, "kernel": "falcon chunk-parallel forward, Falcon-1", "peak_source": src,
+            "algorithmic_bytes_per_launch": ab, "launch_ms": f1_ms}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(), "roofline": roof,
+            "per_variant_ms": {var: statistics.mean(per_var[var]) for var in w["variants"]},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": len(w["variants"]) * args.steps, "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, threads, units, used = cpu_oracle_sample(budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": "fp64 oracle chunk-parallel form, Falcon-1 and Falcon-1A, %d whole (b,h) "
+                                          "units of the workload (%.1f s)" % (units, used)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,156 @@
+/*
+ * falcon.h -- C ABI of libfalcon.so: the Falcon family of normalised
+ * first-order fast-weight updates (Fast Weight Attention) on sm_100a.
+ *
+ * Method (web pages on arXiv 2608.27763, cited by title and section):
+ *   [EXPL] "Fast Weight Attention：用于持续学习的快速权重注意力", 核心方法 1-4
+ *   [SUMM] "Fast Weight Attention for Continual Learning", 方法
+ *   [NEWS] "借鉴40年前的设想！字节Seed提出快速权重注意力推进大模型持续学习", 02
+ *
+ * Per (batch b, head h) the state S is a d_v x d_k matrix, S_0 = 0.  With the
+ * prefix-aligned pair (x_t, y_t) = (phi(k_{t-1}), v_t) ([SUMM] 输入与状态定义),
+ * phi(k) = k/|k| (phi(0) = 0) and x_1 = 0:
+ *   n_t     = |x_t|^2  (Falcon-3/3A: sum of |x_i|^2 over the window W_t)
+ *   eta_t   = beta_t / (eps + n_t), 0 when n_t = 0   (NLMS step, [EXPL] 核心方法 2)
+ *   alpha_t = max(1 - eta_t * lambda_h, 2^-20)        (positive decay, [NEWS] 02 (1))
+ *   Falcon-1/2   S_t = alpha S_{t-1} + eta (y_t - S_{t-1} x_t) x_t^T
+ *   Falcon-1A/2A S_t = alpha S_{t-1} + eta y_t x_t^T
+ *   Falcon-3     S_t = alpha S_{t-1} + eta sum_{i in W_t} (y_i - S_{t-1} x_i) x_i^T
+ *   Falcon-3A    S_t = alpha S_{t-1} + eta sum_{i in W_t} y_i x_i^T
+ *   o_t = S_t q_t  (read after write)
+ * W_t = {max(1, t-window+1), ..., t}.  Falcon-2/2A take beta (hence eta and
+ * alpha) per value channel j, i.e. per row of S ([NEWS] 02 (2)).
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor arguments are DEVICE pointers to contiguous row-major arrays
+ *    owned by the caller; the library never frees or retains them.
+ *  - Calls only enqueue work on `stream` (0 = legacy default stream) and never
+ *    synchronise.  A non-zero return means nothing was enqueued, except
+ *    FALCON_ERR_LAUNCH, which reports cudaGetLastError() after a launch.
+ *    Faults inside a kernel surface asynchronously on the stream.
+ *  - Device values are not inspected by the host: lambda must lie in [0, 1)
+ *    and beta should be >= 0; other values give results but no error.
+ *  - Element types: falcon_dtype selects fp32 or bf16 for q, k, v, beta and
+ *    out.  lambda, the state, x_prev and the window carry are always fp32.
+ */
+#ifndef FALCON_H
+#define FALCON_H
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FALCON_F1 = 0,  /* regression, scalar NLMS step                      */
+    FALCON_F2 = 1,  /* regression, one step per value channel            */
+    FALCON_F3 = 2,  /* regression, sliding-window mini-batch of `window` */
+    FALCON_F1A = 3, /* inner product, scalar step                        */
+    FALCON_F2A = 4, /* inner product, per value channel                  */
+    FALCON_F3A = 5  /* inner product, sliding window                     */
+} falcon_variant;
+
+/* The three equivalent computation forms ([EXPL] 核心方法 3; [SUMM] 计算形式与数值稳定). */
+typedef enum {
+    FALCON_RECURRENT = 0, /* token-by-token state update                    */
+    FALCON_MASKED = 1,    /* all positions at once through a causal L x L mask */
+    FALCON_CHUNK = 2      /* parallel inside chunks, state passed between    */
+} falcon_form;
+
+typedef enum { FALCON_F32 = 0, FALCON_BF16 = 1 } falcon_dtype;
+
+/* Sample pairing: the prefix-aligned pair ([SUMM] 输入与状态定义) or the
+ * same-step pair (phi(k_t), v_t) ([EXPL] 核心方法 1, warning paragraph). */
+typedef enum { FALCON_PAIR_PREFIX = 0, FALCON_PAIR_SAME_STEP = 1 } falcon_pairing;
+
+/* Feature map: L2 normalisation, or the identity (for special-case checks). */
+typedef enum { FALCON_PHI_L2 = 0, FALCON_PHI_IDENTITY = 1 } falcon_phi;
+
+enum {
+    FALCON_OK = 0,
+    FALCON_ERR_NULL = -1,        /* a required pointer is NULL                      */
+    FALCON_ERR_ENUM = -2,        /* variant / form / dtype / pairing / phi invalid   */
+    FALCON_ERR_SHAPE = -3,       /* B,H,L < 0, or d_k, d_v not in {16,32,64,128}     */
+    FALCON_ERR_CHUNK = -4,       /* chunk not in {16,32,64} for the chunk form      */
+    FALCON_ERR_WINDOW = -6,      /* window < 1 or > 8 for Falcon-3/3A               */
+    FALCON_ERR_LAUNCH = -7,      /* a kernel launch failed (cudaGetLastError)       */
+    FALCON_ERR_ALLOC = -8,       /* stream-ordered scratch allocation failed        */
+    FALCON_ERR_UNSUPPORTED = -9  /* combination not supported (e.g. pairing+decode) */
+};
+
+/*
+ * falcon_fwd -- forward pass over whole sequences.
+ *
+ *   q, k     [B,H,L,d_k] dtype     queries and keys
+ *   v        [B,H,L,d_v] dtype     values (targets y_t = v_t)
+ *   beta     [B,H,L] dtype (Falcon-1/3/1A/3A) or [B,H,L,d_v] (Falcon-2/2A)
+ *   lambda   [H] fp32              forgetting strength per head, in [0,1)
+ *   eps      NLMS regulariser (>= 0)
+ *   window   B_w for Falcon-3/3A (1..8); ignored otherwise
+ *   chunk    chunk length for FALCON_CHUNK (16, 32 or 64); ignored otherwise
+ *   out      [B,H,L,d_v] dtype     o_t = S_t q_t (written)
+ *   final_state [B,H,d_v,d_k] fp32 S_L (written), may be NULL
+ * S_0 = 0.  L may be 0 (out untouched, final_state zeroed) and need not be a
+ * multiple of `chunk`.  FALCON_MASKED draws stream-ordered scratch
+ * (cudaMallocAsync/cudaFreeAsync on `stream`, about B*H*L*(window*d_v+2*d_v)
+ * floats) and returns FALCON_ERR_ALLOC if that fails.
+ */
+int falcon_fwd(falcon_variant variant, falcon_form form, falcon_dtype dtype,
+               const void *q, const void *k, const void *v, const void *beta,
+               const float *lambda, float eps, int window,
+               int B, int H, int L, int d_k, int d_v, int chunk,
+               void *out, float *final_state, cudaStream_t stream);
+
+/* falcon_fwd with the pairing and the feature map selectable. */
+int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype,
+                  falcon_pairing pairing, falcon_phi phi,
+                  const void *q, const void *k, const void *v, const void *beta,
+                  const float *lambda, float eps, int window,
+                  int B, int H, int L, int d_k, int d_v, int chunk,
+                  void *out, float *final_state, cudaStream_t stream);
+
+/*
+ * falcon_decode_step -- one recurrent step for N independent sequences
+ * ([EXPL] 核心方法 3: recurrent, O(d^2) per step, for inference).
+ *
+ *   q, k     [N,H,d_k] dtype, v [N,H,d_v] dtype, beta [N,H] or [N,H,d_v] dtype
+ *   lambda   [H] fp32; eps, window as in falcon_fwd
+ *   state    [N,H,d_v,d_k] fp32, in/out: S_{t-1} -> S_t
+ *   x_prev   [N,H,d_k] fp32, in/out: phi(k_{t-1}) -> phi(k_t); zeros before
+ *            the first token of a sequence
+ *   win      [N,H,window-1,d_k+d_v] fp32, in/out, Falcon-3/3A only (NULL
+ *            otherwise): the previous window-1 samples (x_i, y_i), oldest
+ *            first; zeros where the sequence has fewer samples
+ *   out      [N,H,d_v] dtype: o_t
+ * Prefix pairing and the L2 feature map.  Each (n,h) is read and written by
+ * exactly one thread block, so in-place carries are race-free.
+ */
+int falcon_decode_step(falcon_variant variant, falcon_dtype dtype,
+                       const void *q, const void *k, const void *v, const void *beta,
+                       const float *lambda, float eps, int window,
+                       int N, int H, int d_k, int d_v,
+                       float *state, float *x_prev, float *win, void *out,
+                       cudaStream_t stream);
+
+/*
+ * falcon_decode_carry_from_prefill -- the decode carry after a prefill of L
+ * tokens: x_prev = phi(k_L) and, for Falcon-3/3A, the samples (x_i, v_i),
+ * i = L-window+2 .. L (zeros for i < 1).  k [B,H,L,d_k], v [B,H,L,d_v] dtype;
+ * x_prev [B,H,d_k] and win [B,H,window-1,d_k+d_v] fp32 are written (win may
+ * be NULL when window <= 1 or the variant has no window).  The final state of
+ * the prefill comes from falcon_fwd's final_state.
+ */
+int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_dtype dtype,
+                                     const void *k, const void *v, int window,
+                                     int B, int H, int L, int d_k, int d_v,
+                                     float *x_prev, float *win, cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char *falcon_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FALCON_H */

@@ -1,0 +1,8 @@
+"""Falcon fast-weight updates (Fast Weight Attention) on B200 (sm_100a).
+
+The computation lives in libfalcon.so (C ABI in include/falcon.h, CUDA
+kernels in csrc/); this package is the thin ctypes binding plus the seeded
+synthetic-input generator.
+"""
+from ._lib import (DTYPES, EXPORTS, FORMS, LIB_PATH, VARIANTS, FalconError, carry_from_prefill,  # noqa: F401
+                   decode_step, fwd, load)

@@ -1,0 +1,130 @@
+"""ctypes binding of libfalcon.so (the C ABI declared in include/falcon.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  Tensors must already live on the GPU; the calls
+enqueue on torch's current stream (or the stream given) and return without
+synchronising.  There is no CPU fallback: if the library is missing or the
+device is not a CUDA GPU, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfalcon.so")
+
+VARIANTS = {"F1": 0, "F2": 1, "F3": 2, "F1A": 3, "F2A": 4, "F3A": 5}
+FORMS = {"recurrent": 0, "masked": 1, "chunk": 2}
+DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+PAIRINGS = {"prefix": 0, "same_step": 1}
+PHIS = {"l2": 0, "identity": 1}
+EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_decode_step", "falcon_decode_carry_from_prefill",
+           "falcon_status_string")
+
+_lib = None
+
+
+class FalconError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfalcon.so and declare the C signatures (raises if absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FalconError("libfalcon.so not built (run python -m linear_attention_sequence_falcon_b200.build)")
+    lib = ctypes.CDLL(path)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.falcon_fwd.argtypes = [I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, I, P, P, P]
+    lib.falcon_fwd.restype = I
+    lib.falcon_fwd_ex.argtypes = [I, I, I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, I, P, P, P]
+    lib.falcon_fwd_ex.restype = I
+    lib.falcon_decode_step.argtypes = [I, I, P, P, P, P, P, F, I, I, I, I, I, P, P, P, P, P]
+    lib.falcon_decode_step.restype = I
+    lib.falcon_decode_carry_from_prefill.argtypes = [I, I, P, P, I, I, I, I, I, I, P, P, P]
+    lib.falcon_decode_carry_from_prefill.restype = I
+    lib.falcon_status_string.argtypes = [I]
+    lib.falcon_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != 0:
+        msg = load().falcon_status_string(rc).decode()
+        raise FalconError("libfalcon status %d: %s" % (rc, msg))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise FalconError("tensor is not on a CUDA device (no CPU path exists)")
+    if not t.is_contiguous():
+        raise FalconError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def fwd(variant: str, form: str, q, k, v, beta, lam, eps: float, window: int = 1, chunk: int = 64,
+        out=None, final_state=None, pairing: str = "prefix", phi: str = "l2", stream=None,
+        want_state: bool = True):
+    """falcon_fwd_ex on CUDA tensors q,k [B,H,L,dk], v [B,H,L,dv], beta [B,H,L] or
+    [B,H,L,dv] (same dtype), lam [H] fp32.  Returns (out, final_state)."""
+    lib = load()
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in DTYPES or not (q.dtype == k.dtype == v.dtype == beta.dtype):
+        raise FalconError("q, k, v, beta must share one dtype, fp32 or bf16")
+    if lam.dtype != torch.float32:
+        raise FalconError("lambda must be fp32")
+    if out is None:
+        out = torch.empty((B, H, L, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and want_state:
+        final_state = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    rc = lib.falcon_fwd_ex(VARIANTS[variant], FORMS[form], DTYPES[q.dtype], PAIRINGS[pairing], PHIS[phi],
+                           _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(lam), float(eps), int(window),
+                           B, H, L, dk, dv, int(chunk), _ptr(out), _ptr(final_state), _stream(stream))
+    _check(rc)
+    return out, final_state
+
+
+def decode_step(variant: str, q, k, v, beta, lam, eps: float, window: int, state, x_prev, win=None,
+                out=None, stream=None):
+    """falcon_decode_step: q,k [N,H,dk], v [N,H,dv], beta [N,H] or [N,H,dv];
+    state [N,H,dv,dk], x_prev [N,H,dk], win [N,H,window-1,dk+dv] fp32 (in/out)."""
+    lib = load()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    rc = lib.falcon_decode_step(VARIANTS[variant], DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                _ptr(lam), float(eps), int(window), N, H, dk, dv, _ptr(state), _ptr(x_prev),
+                                _ptr(win), _ptr(out), _stream(stream))
+    _check(rc)
+    return out
+
+
+def carry_from_prefill(variant: str, k, v, window: int, x_prev=None, win=None, stream=None):
+    """falcon_decode_carry_from_prefill: returns (x_prev [B,H,dk], win [B,H,w-1,dk+dv])."""
+    lib = load()
+    B, H, L, dk = k.shape
+    dv = v.shape[-1]
+    w = window if variant in ("F3", "F3A") else 1
+    if x_prev is None:
+        x_prev = torch.empty((B, H, dk), dtype=torch.float32, device=k.device)
+    if win is None and w > 1:
+        win = torch.empty((B, H, w - 1, dk + dv), dtype=torch.float32, device=k.device)
+    rc = lib.falcon_decode_carry_from_prefill(VARIANTS[variant], DTYPES[k.dtype], _ptr(k), _ptr(v), int(window),
+                                              B, H, L, dk, dv, _ptr(x_prev), _ptr(win), _stream(stream))
+    _check(rc)
+    return x_prev, win

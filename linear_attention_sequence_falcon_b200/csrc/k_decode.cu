@@ -1,0 +1,213 @@
+// k_decode.cu -- one recurrent step per sequence (decode) and the decode carry
+// after a prefill ("recurrent: O(d^2) per step, for inference", page "Fast
+// Weight Attention：用于持续学习的快速权重注意力", 核心方法 3).
+//
+// The step is bound by streaming the fp32 state: every row of S is read once
+// and written once.  One thread block owns one (n,h): DK/4 lanes hold a row as
+// one float4 each (a 128-wide row is one fully coalesced 512-byte warp
+// access), four row passes are loaded before any is used to keep several
+// loads in flight per thread, and the two dot products a row needs (S_j.x_m
+// for every window sample, S_j.q) are reduced together by xor-shuffles.  The
+// read uses o_j = alpha (S_j.q) + eta sum_m e_m (x_m.q), so the updated row
+// is never re-read.  Because one block owns the (n,h), the carry (x_prev and
+// the window) is updated in place without races.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace falcon {
+
+template <typename T, int DK>
+__global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
+    constexpr int LPR = DK / 4;
+    constexpr int RPW = 32 / LPR;
+    constexpr int NW = 8;
+    constexpr int RPP = NW * RPW;  // rows per pass
+    constexpr int U = 4;           // passes in flight
+    __shared__ __align__(16) float xw[kMaxWindow][DK];
+    __shared__ float yw[kMaxWindow][128];
+    __shared__ __align__(16) float qv[DK];
+    __shared__ float kn[DK];
+    __shared__ float xq[kMaxWindow];
+    __shared__ float sqm[kMaxWindow];
+    __shared__ float knorm;
+
+    const VariantInfo vi = variant_info(p.variant, p.window);
+    const int w = vi.window;
+    const int nh = blockIdx.x;
+    const int h = nh % p.H;
+    const int dv = p.dv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
+    const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
+    const T *v = static_cast<const T *>(p.v) + (size_t)nh * dv;
+    const T *beta = static_cast<const T *>(p.beta) + (size_t)nh * (vi.per_channel ? dv : 1);
+    float *xp = p.x_prev + (size_t)nh * DK;
+    float *win = p.win ? p.win + (size_t)nh * (w - 1) * (DK + dv) : nullptr;
+
+    // stage the window (oldest first), the current sample (x_prev, v_t), q and k
+    for (int i = threadIdx.x; i < DK; i += blockDim.x) {
+        xw[w - 1][i] = xp[i];
+        qv[i] = to_f32(q[i]);
+        kn[i] = to_f32(k[i]);
+    }
+    for (int i = threadIdx.x; i < dv; i += blockDim.x) yw[w - 1][i] = to_f32(v[i]);
+    for (int i = threadIdx.x; i < (w - 1) * (DK + dv); i += blockDim.x) {
+        const int m = i / (DK + dv), c = i % (DK + dv);
+        const float val = win[i];
+        if (c < DK) xw[m][c] = val; else yw[m][c - DK] = val;
+    }
+    __syncthreads();
+    if (warp < w) {
+        float a = 0.f, b = 0.f;
+        for (int c = lane; c < DK; c += 32) {
+            a += xw[warp][c] * qv[c];
+            b += xw[warp][c] * xw[warp][c];
+        }
+        a = group_sum<32>(a);
+        b = group_sum<32>(b);
+        if (lane == 0) { xq[warp] = a; sqm[warp] = b; }
+    }
+    if (warp == NW - 1) {
+        float a = 0.f;
+        for (int c = lane; c < DK; c += 32) a += kn[c] * kn[c];
+        a = group_sum<32>(a);
+        if (lane == 0) knorm = a;
+    }
+    __syncthreads();
+    float n = 0.f;
+    for (int m = 0; m < w; ++m) n += sqm[m];
+    const float lam = p.lambda[h];
+    float eta_s = 0.f, alpha_s = 1.f;
+    if (!vi.per_channel) step_and_decay(to_f32(beta[0]), n, p.eps, lam, eta_s, alpha_s);
+
+    const int sl = lane % LPR;
+    const int rsub = warp * RPW + lane / LPR;
+    float4 xm[kMaxWindow];
+#pragma unroll
+    for (int m = 0; m < kMaxWindow; ++m)
+        if (m < w) xm[m] = *reinterpret_cast<const float4 *>(&xw[m][sl * 4]);
+    const float4 q4 = *reinterpret_cast<const float4 *>(&qv[sl * 4]);
+    float *S = p.state + (size_t)nh * dv * DK;
+    T *out = static_cast<T *>(p.out) + (size_t)nh * dv;
+
+    for (int base = 0; base < dv; base += RPP * U) {
+        float4 s4[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int row = base + u * RPP + rsub;
+            if (row < dv) s4[u] = *reinterpret_cast<const float4 *>(S + (size_t)row * DK + sl * 4);
+            else s4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int row = base + u * RPP + rsub;
+            const float4 s = s4[u];
+            float sq = s.x * q4.x + s.y * q4.y + s.z * q4.z + s.w * q4.w;
+            sq = group_sum<LPR>(sq);
+            float e[kMaxWindow];
+#pragma unroll
+            for (int m = 0; m < kMaxWindow; ++m) {
+                e[m] = 0.f;
+                if (m < w) {
+                    float d = 0.f;
+                    if (vi.regression) {
+                        d = s.x * xm[m].x + s.y * xm[m].y + s.z * xm[m].z + s.w * xm[m].w;
+                        d = group_sum<LPR>(d);
+                    }
+                    const float y = row < dv ? yw[m][row] : 0.f;
+                    e[m] = vi.regression ? y - d : y;
+                }
+            }
+            float eta = eta_s, alpha = alpha_s;
+            if (vi.per_channel && row < dv) step_and_decay(to_f32(beta[row]), n, p.eps, lam, eta, alpha);
+            float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
+            float gq = 0.f;
+#pragma unroll
+            for (int m = 0; m < kMaxWindow; ++m)
+                if (m < w) {
+                    g.x += e[m] * xm[m].x; g.y += e[m] * xm[m].y;
+                    g.z += e[m] * xm[m].z; g.w += e[m] * xm[m].w;
+                    gq += e[m] * xq[m];
+                }
+            if (row < dv) {
+                float4 r;
+                r.x = alpha * s.x + eta * g.x; r.y = alpha * s.y + eta * g.y;
+                r.z = alpha * s.z + eta * g.z; r.w = alpha * s.w + eta * g.w;
+                *reinterpret_cast<float4 *>(S + (size_t)row * DK + sl * 4) = r;
+                if (sl == 0) out[row] = from_f32<T>(alpha * sq + eta * gq);
+            }
+        }
+    }
+    // carry: x_prev <- phi(k_t); window drops its oldest sample, appends (x_prev, v_t)
+    const float inv = knorm > 0.f ? rsqrtf(knorm) : 0.f;
+    for (int i = threadIdx.x; i < DK; i += blockDim.x) xp[i] = kn[i] * inv;
+    if (w > 1) {
+        for (int i = threadIdx.x; i < (w - 1) * (DK + dv); i += blockDim.x) {
+            const int m = i / (DK + dv), c = i % (DK + dv);
+            win[i] = c < DK ? xw[m + 1][c] : yw[m + 1][c - DK];
+        }
+    }
+}
+
+template <typename T, int DK>
+__global__ void __launch_bounds__(128) carry_kernel(CarryParams p) {
+    const VariantInfo vi = variant_info(p.variant, p.window);
+    const int w = vi.window;
+    const int bh = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T *k = static_cast<const T *>(p.k) + (size_t)bh * p.L * DK;
+    const T *v = static_cast<const T *>(p.v) + (size_t)bh * p.L * p.dv;
+    // job 0: x_prev; jobs 1..w-1: window slots m = job-1
+    for (int job = warp; job < w; job += 4) {
+        const int m = job - 1;
+        const int i = job == 0 ? p.L : p.L - (w - 1) + m;  // sample index whose key is k_{i-1}
+        float *xdst = job == 0 ? p.x_prev + (size_t)bh * DK : p.win + ((size_t)bh * (w - 1) + m) * (DK + p.dv);
+        const int ki = i - 1;
+        float ss = 0.f;
+        for (int c = lane; c < DK; c += 32) {
+            const float x = (ki >= 0 && i >= 0) ? to_f32(k[(size_t)ki * DK + c]) : 0.f;
+            ss += x * x;
+        }
+        ss = group_sum<32>(ss);
+        const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+        for (int c = lane; c < DK; c += 32)
+            xdst[c] = (ki >= 0 && i >= 0) ? to_f32(k[(size_t)ki * DK + c]) * inv : 0.f;
+        if (job > 0)
+            for (int c = lane; c < p.dv; c += 32)
+                xdst[DK + c] = i >= 0 ? to_f32(v[(size_t)i * p.dv + c]) : 0.f;
+    }
+}
+
+template <typename T, int DK>
+static void launch_decode_dk(const DecodeParams &p, cudaStream_t s) {
+    decode_kernel<T, DK><<<p.N * p.H, 256, 0, s>>>(p);
+}
+
+template <typename T>
+int launch_decode(const DecodeParams &p, cudaStream_t s) {
+    switch (p.dk) {
+        case 16: launch_decode_dk<T, 16>(p, s); return 0;
+        case 32: launch_decode_dk<T, 32>(p, s); return 0;
+        case 64: launch_decode_dk<T, 64>(p, s); return 0;
+        case 128: launch_decode_dk<T, 128>(p, s); return 0;
+    }
+    return -3;
+}
+
+template <typename T>
+int launch_carry(const CarryParams &p, cudaStream_t s) {
+    switch (p.dk) {
+        case 16: carry_kernel<T, 16><<<p.B * p.H, 128, 0, s>>>(p); return 0;
+        case 32: carry_kernel<T, 32><<<p.B * p.H, 128, 0, s>>>(p); return 0;
+        case 64: carry_kernel<T, 64><<<p.B * p.H, 128, 0, s>>>(p); return 0;
+        case 128: carry_kernel<T, 128><<<p.B * p.H, 128, 0, s>>>(p); return 0;
+    }
+    return -3;
+}
+
+template int launch_decode<float>(const DecodeParams &, cudaStream_t);
+template int launch_decode<__nv_bfloat16>(const DecodeParams &, cudaStream_t);
+template int launch_carry<float>(const CarryParams &, cudaStream_t);
+template int launch_carry<__nv_bfloat16>(const CarryParams &, cudaStream_t);
+
+}  // namespace falcon

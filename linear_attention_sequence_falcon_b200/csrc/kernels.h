@@ -1,0 +1,51 @@
+// kernels.h -- internal launch interface between the C ABI (api.cu) and the
+// kernels.  Not installed; the public boundary is include/falcon.h.
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace falcon {
+
+struct FwdParams {
+    int variant, form, pairing, phi, window;
+    int B, H, L, dk, dv, chunk;
+    float eps;
+    const void *q, *k, *v, *beta;
+    const float *lambda;
+    void *out;
+    float *final_state;
+    // stream-ordered scratch for the masked-parallel form
+    float *ws_r, *ws_eta, *ws_gam;
+};
+
+struct DecodeParams {
+    int variant, window;
+    int N, H, dk, dv;
+    float eps;
+    const void *q, *k, *v, *beta;
+    const float *lambda;
+    float *state, *x_prev, *win;
+    void *out;
+};
+
+struct CarryParams {
+    int variant, window;
+    int B, H, L, dk, dv;
+    const void *k, *v;
+    float *x_prev, *win;
+};
+
+template <typename T> int launch_recurrent(const FwdParams &p, cudaStream_t s);
+template <typename T> int launch_span_chunk(const FwdParams &p, cudaStream_t s);
+template <typename T> int launch_span_masked(const FwdParams &p, cudaStream_t s);
+// bf16 chunk-parallel forward on tcgen05; returns 1 (nothing launched) for
+// shapes it does not cover, so the caller falls back to the span kernel.
+int launch_tc_chunk(const FwdParams &p, cudaStream_t s);
+template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
+template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
+
+// Scratch sizes (floats) of the masked-parallel form.
+size_t masked_ws_r_floats(const FwdParams &p);
+size_t masked_ws_eg_floats(const FwdParams &p);
+
+}  // namespace falcon

@@ -1,0 +1,246 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the fp64 oracle
+on the same seeded inputs.
+
+Error metric per tensor: max|gpu - oracle| / max|oracle| (max-norm relative).
+Bars: 1e-4 for fp32 inputs, 2e-2 for bf16 inputs with fp32 accumulation and
+state.  The oracle reference for every form is the recurrent definition.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_sequence_falcon_b200 import inputs as gen
+
+pytestmark = pytest.mark.gpu
+
+VARIANTS = ("F1", "F2", "F3", "F1A", "F2A", "F3A")
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+@pytest.fixture(scope="module")
+def F():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu tests")
+    from linear_attention_sequence_falcon_b200 import build
+    build.build()
+    import linear_attention_sequence_falcon_b200 as F
+    F.load()
+    return F
+
+
+def rel(gpu, ref):
+    ref = np.asarray(ref, dtype=np.float64)
+    den = max(np.abs(ref).max(), 1e-30)
+    return float(np.abs(np.asarray(gpu, dtype=np.float64) - ref).max() / den)
+
+
+def dev(d, name):
+    return d[name].cuda()
+
+
+def gpu_fwd(F, d, variant, form, chunk=64, window=1, pairing="prefix", phi="l2"):
+    out, S = F.fwd(variant, form, dev(d, "q"), dev(d, "k"), dev(d, "v"), dev(d, "beta"), dev(d, "lam"),
+                   d["eps"], window=window, chunk=chunk, pairing=pairing, phi=phi)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy(), S.double().cpu().numpy()
+
+
+def oracle_fwd(d, variant, window=1, units=None, pairing="prefix", phi="l2", form="recurrent", chunk=64):
+    q, k, v, b = d["q_64"], d["k_64"], d["v_64"], d["beta_64"]
+    lam = d["lam_64"]
+    if units is None:
+        return oracle.fwd(variant, form, q, k, v, b, lam, d["eps_64"], window=window, chunk=chunk,
+                          pairing=pairing, phi=phi)
+    outs, Ss = [], []
+    for (bb, hh) in units:
+        o, S = oracle.fwd(variant, form, q[bb:bb + 1, hh:hh + 1], k[bb:bb + 1, hh:hh + 1],
+                          v[bb:bb + 1, hh:hh + 1], b[bb:bb + 1, hh:hh + 1], lam[hh:hh + 1], d["eps_64"],
+                          window=window, chunk=chunk, pairing=pairing, phi=phi)
+        outs.append(o[0, 0])
+        Ss.append(S[0, 0])
+    return np.stack(outs), np.stack(Ss)
+
+
+def check(F, d, variant, form, chunk=64, window=1, units=None, pairing="prefix", phi="l2", tol=None):
+    go, gS = gpu_fwd(F, d, variant, form, chunk, window, pairing, phi)
+    oo, oS = oracle_fwd(d, variant, window, units, pairing, phi)
+    if units is not None:
+        go = np.stack([go[b, h] for b, h in units])
+        gS = np.stack([gS[b, h] for b, h in units])
+    tol = tol if tol is not None else TOL[d["dtype"]]
+    eo, eS = rel(go, oo), rel(gS, oS)
+    assert np.isfinite(go).all() and np.isfinite(gS).all()
+    assert eo <= tol and eS <= tol, f"{variant} {form} C={chunk}: out {eo:.3e} state {eS:.3e} (tol {tol})"
+    return eo, eS
+
+
+# --------------------------------------------------------------- small shapes, every combination
+
+@pytest.mark.parametrize("dk,dv", [(16, 16), (64, 64), (128, 128), (32, 64)])
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("form", ["recurrent", "masked", "chunk"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_parity_small(F, dtype, form, variant, dk, dv):
+    """B=2, H=3, L=150: several 64-token tiles and a ragged tail of 22."""
+    d = gen.draw(variant, 2, 3, 150, dk, dv, seed=1000 + dk + dv, dtype=dtype)
+    w = 4 if variant in ("F3", "F3A") else 1
+    check(F, d, variant, form, chunk=64, window=w)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_chunk_sizes(F, variant, chunk):
+    """Chunk-size invariance: every chunk length against the recurrent oracle."""
+    d = gen.draw(variant, 2, 2, 200, 64, 64, seed=77, dtype="bf16")
+    w = 3 if variant in ("F3", "F3A") else 1
+    check(F, d, variant, "chunk", chunk=chunk, window=w)
+
+
+@pytest.mark.parametrize("w", [1, 2, 5, 8])
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+@pytest.mark.parametrize("form", ["recurrent", "masked", "chunk"])
+def test_windows(F, variant, form, w):
+    d = gen.draw(variant, 1, 2, 130, 32, 32, seed=90 + w, dtype="f32")
+    check(F, d, variant, form, chunk=32, window=w)
+
+
+@pytest.mark.parametrize("pairing,phi", [("same_step", "l2"), ("prefix", "identity"), ("same_step", "identity")])
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("form", ["recurrent", "masked", "chunk"])
+def test_pairing_and_feature_map(F, variant, form, pairing, phi):
+    """The same-step pair and the identity feature map through falcon_fwd_ex."""
+    d = gen.draw(variant, 1, 2, 100, 16, 16, seed=5, dtype="f32", key_scale=0.25)
+    w = 3 if variant in ("F3", "F3A") else 1
+    check(F, d, variant, form, chunk=32, window=w, pairing=pairing, phi=phi)
+
+
+@pytest.mark.parametrize("L", [1, 2, 5, 63, 64, 65])
+@pytest.mark.parametrize("form", ["recurrent", "masked", "chunk"])
+def test_short_sequences(F, form, L):
+    for variant in VARIANTS:
+        d = gen.draw(variant, 1, 2, L, 64, 64, seed=L, dtype="f32")
+        w = 3 if variant in ("F3", "F3A") else 1
+        go, gS = gpu_fwd(F, d, variant, form, 64, w)
+        oo, oS = oracle_fwd(d, variant, w)
+        if L == 1:  # x_1 = 0: nothing is written
+            assert np.abs(go).max() == 0 and np.abs(gS).max() == 0
+        else:
+            assert rel(go, oo) <= 1e-4 and rel(gS, oS) <= 1e-4
+
+
+@pytest.mark.parametrize("form", ["recurrent", "masked", "chunk"])
+def test_empty_sequence_zeroes_state(F, form):
+    q = torch.zeros((2, 2, 0, 64), device="cuda", dtype=torch.bfloat16)
+    v = torch.zeros((2, 2, 0, 64), device="cuda", dtype=torch.bfloat16)
+    b = torch.zeros((2, 2, 0), device="cuda", dtype=torch.bfloat16)
+    lam = torch.zeros(2, device="cuda")
+    S = torch.full((2, 2, 64, 64), 7.0, device="cuda")
+    F.fwd("F1", form, q, q, v, b, lam, 1e-6, final_state=S)
+    torch.cuda.synchronize()
+    assert float(S.abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("form", ["recurrent", "masked", "chunk"])
+def test_zero_keys_write_nothing(F, form):
+    for variant in VARIANTS:
+        d = gen.draw(variant, 1, 2, 70, 32, 32, seed=3, dtype="bf16")
+        d["k"] = torch.zeros_like(d["k"])
+        go, gS = gpu_fwd(F, d, variant, form, 32, 3 if variant in ("F3", "F3A") else 1)
+        assert np.abs(go).max() == 0 and np.abs(gS).max() == 0
+
+
+def test_strong_forgetting_floor(F):
+    """lambda close to 1 with tiny keys under the identity map drives
+    1 - eta*lambda below zero; the positive-decay floor takes over."""
+    for variant in VARIANTS:
+        d = gen.draw(variant, 1, 2, 90, 16, 16, seed=8, dtype="f32", lam=0.9, key_scale=0.05)
+        w = 2 if variant in ("F3", "F3A") else 1
+        for form in ("recurrent", "masked", "chunk"):
+            check(F, d, variant, form, chunk=16, window=w, phi="identity")
+
+
+# --------------------------------------------------------------- the five benchmark workloads
+
+def test_workload1_falcon1_recurrent_fp32(F):
+    d = gen.workload_inputs(1, "F1")
+    check(F, d, "F1", "recurrent", tol=1e-4)
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_workload2_chunk_full(F, variant):
+    """8x12x2048x64 bf16, chunk 64, every (b,h) unit against the oracle."""
+    d = gen.workload_inputs(2, variant)
+    check(F, d, variant, "chunk", chunk=64)
+
+
+def test_workload3_falcon2_chunk_sampled(F):
+    """4x16x4096x128 bf16, per-channel beta; sampled units."""
+    d = gen.workload_inputs(3, "F2")
+    check(F, d, "F2", "chunk", chunk=64, units=[(0, 0), (1, 7), (3, 15)])
+
+
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+@pytest.mark.parametrize("form", ["masked", "chunk"])
+def test_workload4_window_full(F, variant, form):
+    d = gen.workload_inputs(4, variant)
+    check(F, d, variant, form, chunk=64, window=4, units=[(0, 0), (2, 5), (7, 11)])
+
+
+def test_workload4_masked_equals_chunk(F):
+    """The two parallel forms against each other on the full workload."""
+    for variant in ("F3", "F3A"):
+        d = gen.workload_inputs(4, variant)
+        om, Sm = gpu_fwd(F, d, variant, "masked", 64, 4)
+        oc, Sc = gpu_fwd(F, d, variant, "chunk", 64, 4)
+        assert rel(om, oc) <= 2e-2 and rel(Sm, Sc) <= 2e-2
+
+
+def test_workload5_prefill_sampled(F):
+    """2x16x32768x128 bf16 Falcon-2A prefill; sampled units."""
+    d = gen.workload_inputs(5, "F2A")
+    check(F, d, "F2A", "chunk", chunk=64, units=[(0, 0), (1, 15)])
+
+
+# --------------------------------------------------------------- decode
+
+def _decode_chain(F, variant, N, H, dk, dv, L0, steps, dtype, w):
+    d = gen.draw(variant, N, H, L0 + steps, dk, dv, seed=555, dtype=dtype, lam=0.02)
+    pre = {n: d[n][:, :, :L0].contiguous() for n in ("q", "k", "v", "beta")}
+    _, S = F.fwd(variant, "chunk", *(pre[n].cuda() for n in ("q", "k", "v", "beta")), d["lam"].cuda(), d["eps"],
+                 window=w, chunk=64)
+    x_prev, win = F.carry_from_prefill(variant, pre["k"].cuda(), pre["v"].cuda(), w)
+    torch.cuda.synchronize()
+    # carry parity
+    ox, ow = oracle.carry_from_prefill(variant, d["k_64"][:, :, :L0], d["v_64"][:, :, :L0], w)
+    assert rel(x_prev.double().cpu().numpy(), ox) <= 1e-6
+    if w > 1:
+        assert rel(win.double().cpu().numpy(), ow) <= 1e-6
+    outs = []
+    for t in range(L0, L0 + steps):
+        o = F.decode_step(variant, *(d[n][:, :, t].contiguous().cuda() for n in ("q", "k", "v", "beta")),
+                          d["lam"].cuda(), d["eps"], w, S, x_prev, win)
+        outs.append(o.double().cpu().numpy())
+    torch.cuda.synchronize()
+    return d, np.stack(outs, 2), S.double().cpu().numpy()
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_chain_matches_longer_prefill(F, variant, dtype):
+    """prefill(L0) -> carry -> decode steps == oracle over L0 + steps tokens."""
+    w = 4 if variant in ("F3", "F3A") else 1
+    L0, steps = 70, 9
+    d, outs, S = _decode_chain(F, variant, 3, 4, 64, 64, L0, steps, dtype, w)
+    oo, oS = oracle_fwd(d, variant, w)
+    tol = TOL[dtype]
+    assert rel(outs, oo[:, :, L0:]) <= tol
+    assert rel(S, oS) <= tol
+
+
+def test_decode_workload5_shape(F):
+    """N=64, H=16, 128x128 fp32 state: a few steps after a short prefill."""
+    d, outs, S = _decode_chain(F, "F2A", 64, 16, 128, 128, 40, 4, "bf16", 1)
+    oo, oS = oracle_fwd(d, "F2A", 1)
+    assert rel(outs, oo[:, :, 40:]) <= 2e-2
+    assert rel(S, oS) <= 2e-2
