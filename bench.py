@@ -245,6 +245,12 @@ def run_ours(args):
             if ev is not None:
                 ev[var][1].record(stream)
 
+    if args.profile:
+        # device step only, for profilers (which flush caches themselves)
+        for _ in range(args.warmup + args.steps):
+            step()
+        torch.cuda.synchronize()
+        return
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
         step()
@@ -326,6 +332,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run only warmup+steps device steps (no flush, e2e, clocks or JSON), for ncu")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
