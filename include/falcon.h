@@ -76,7 +76,9 @@ enum {
     FALCON_ERR_WINDOW = -6,      /* window < 1 or > 8 for Falcon-3/3A               */
     FALCON_ERR_LAUNCH = -7,      /* a kernel launch failed (cudaGetLastError)       */
     FALCON_ERR_ALLOC = -8,       /* stream-ordered scratch allocation failed        */
-    FALCON_ERR_UNSUPPORTED = -9  /* combination not supported (e.g. pairing+decode) */
+    FALCON_ERR_UNSUPPORTED = -9, /* combination not supported (e.g. pairing+decode) */
+    FALCON_ERR_SCRATCH = -10     /* problem needs more than the fixed scratch of
+                                    falcon_fwd_masked_noalloc                      */
 };
 
 /*
@@ -145,6 +147,38 @@ int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_dtype dtype,
                                      const void *k, const void *v, int window,
                                      int B, int H, int L, int d_k, int d_v,
                                      float *x_prev, float *win, cudaStream_t stream);
+
+/*
+ * falcon_fwd_masked_noalloc -- the masked-parallel forward (prefix pair, L2
+ * feature map) without any device allocation.  The paper has no counterpart;
+ * this entry point exists for callers that may not allocate device memory:
+ * a host that owns every device allocation and gives a plug-in only its
+ * input and output buffers, or a service running under a fixed, pre-planned
+ * memory budget.  falcon_fwd's masked form draws its scratch with
+ * cudaMallocAsync; this one uses a fixed array of
+ * FALCON_NOALLOC_SCRATCH_BYTES inside the library instead, which every GPU
+ * that loads the library holds until the process exits.  Arguments, layouts
+ * and results are those of falcon_fwd with form = FALCON_MASKED.
+ *  - The problem must fit: B*H*L*(window_eff*d_v + 2*d_v) floats, window_eff
+ *    = window for Falcon-3/3A and 1 otherwise, at most
+ *    FALCON_NOALLOC_SCRATCH_BYTES/4; larger problems return
+ *    FALCON_ERR_SCRATCH and enqueue nothing.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array: calls that may overlap on
+ *    the GPU (other streams, other host threads) race and must be serialised
+ *    by the caller.  No state carries over between calls (every scratch
+ *    element is written before it is read).
+ *  - Never calls cudaMalloc, cudaMallocAsync, cudaFree or any allocating
+ *    library routine.
+ */
+#define FALCON_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int falcon_fwd_masked_noalloc(falcon_variant variant, falcon_dtype dtype,
+                              const void *q, const void *k, const void *v, const void *beta,
+                              const float *lambda, float eps, int window,
+                              int B, int H, int L, int d_k, int d_v,
+                              void *out, float *final_state, cudaStream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char *falcon_status_string(int status);

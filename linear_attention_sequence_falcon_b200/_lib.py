@@ -22,7 +22,7 @@ DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PAIRINGS = {"prefix": 0, "same_step": 1}
 PHIS = {"l2": 0, "identity": 1}
 EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_decode_step", "falcon_decode_carry_from_prefill",
-           "falcon_status_string")
+           "falcon_fwd_masked_noalloc", "falcon_status_string")
 
 _lib = None
 
@@ -48,6 +48,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.falcon_decode_step.restype = I
     lib.falcon_decode_carry_from_prefill.argtypes = [I, I, P, P, I, I, I, I, I, I, P, P, P]
     lib.falcon_decode_carry_from_prefill.restype = I
+    lib.falcon_fwd_masked_noalloc.argtypes = [I, I, P, P, P, P, P, F, I, I, I, I, I, I, P, P, P]
+    lib.falcon_fwd_masked_noalloc.restype = I
     lib.falcon_status_string.argtypes = [I]
     lib.falcon_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -94,6 +96,27 @@ def fwd(variant: str, form: str, q, k, v, beta, lam, eps: float, window: int = 1
     rc = lib.falcon_fwd_ex(VARIANTS[variant], FORMS[form], DTYPES[q.dtype], PAIRINGS[pairing], PHIS[phi],
                            _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(lam), float(eps), int(window),
                            B, H, L, dk, dv, int(chunk), _ptr(out), _ptr(final_state), _stream(stream))
+    _check(rc)
+    return out, final_state
+
+
+def fwd_masked_noalloc(variant: str, q, k, v, beta, lam, eps: float, window: int = 1, out=None,
+                       final_state=None, stream=None):
+    """falcon_fwd_masked_noalloc: the masked-parallel forward for callers that
+    may not allocate device memory (a host that owns all device allocations,
+    a fixed memory budget).  Its scratch is a fixed array inside the library;
+    problems beyond it raise (FALCON_ERR_SCRATCH).  Calls sharing a device
+    must not overlap on the GPU.  Same results as fwd(..., form="masked")."""
+    lib = load()
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, L, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    rc = lib.falcon_fwd_masked_noalloc(VARIANTS[variant], DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                       _ptr(lam), float(eps), int(window), B, H, L, dk, dv, _ptr(out),
+                                       _ptr(final_state), _stream(stream))
     _check(rc)
     return out, final_state
 

@@ -141,6 +141,7 @@ extern "C" const char *falcon_status_string(int status) {
         case FALCON_ERR_LAUNCH: return "kernel launch failed";
         case FALCON_ERR_ALLOC: return "stream-ordered scratch allocation failed";
         case FALCON_ERR_UNSUPPORTED: return "unsupported combination";
+        case FALCON_ERR_SCRATCH: return "problem exceeds the fixed scratch of falcon_fwd_masked_noalloc";
     }
     return "unknown status";
 }
