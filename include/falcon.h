@@ -180,6 +180,16 @@ int falcon_fwd_masked_noalloc(falcon_variant variant, falcon_dtype dtype,
                               int B, int H, int L, int d_k, int d_v,
                               void *out, float *final_state, cudaStream_t stream);
 
+/*
+ * falcon_device_wait_timeouts -- diagnostic: how many thread blocks of the
+ * tensor-core kernels on the current device gave up on a bounded wait for
+ * their own tensor-core work (about 2 s per wait) since the library was
+ * loaded.  A block that gives up skips its remaining chunks, frees its tensor
+ * memory and exits, so the device stays usable; its outputs are then
+ * incomplete.  Synchronises with the device.  Returns 0 and writes *count.
+ */
+int falcon_device_wait_timeouts(unsigned int *count);
+
 /* Static description of a status code (never NULL). */
 const char *falcon_status_string(int status);
 

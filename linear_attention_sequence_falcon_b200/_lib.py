@@ -50,6 +50,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.falcon_decode_carry_from_prefill.restype = I
     lib.falcon_fwd_masked_noalloc.argtypes = [I, I, P, P, P, P, P, F, I, I, I, I, I, I, P, P, P]
     lib.falcon_fwd_masked_noalloc.restype = I
+    lib.falcon_device_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    lib.falcon_device_wait_timeouts.restype = I
     lib.falcon_status_string.argtypes = [I]
     lib.falcon_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -119,6 +121,13 @@ def fwd_masked_noalloc(variant: str, q, k, v, beta, lam, eps: float, window: int
                                        _ptr(final_state), _stream(stream))
     _check(rc)
     return out, final_state
+
+
+def wait_timeouts() -> int:
+    """Diagnostic counter of tensor-core thread blocks that gave up waiting."""
+    c = ctypes.c_uint(0)
+    _check(load().falcon_device_wait_timeouts(ctypes.byref(c)))
+    return int(c.value)
 
 
 def decode_step(variant: str, q, k, v, beta, lam, eps: float, window: int, state, x_prev, win=None,

@@ -130,6 +130,12 @@ extern "C" int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_d
     return launched(dtype == FALCON_BF16 ? launch_carry<__nv_bfloat16>(p, stream) : launch_carry<float>(p, stream));
 }
 
+extern "C" int falcon_device_wait_timeouts(unsigned int *count) {
+    if (!count) return FALCON_ERR_NULL;
+    *count = tc_wait_timeouts();
+    return cudaGetLastError() == cudaSuccess ? FALCON_OK : FALCON_ERR_LAUNCH;
+}
+
 extern "C" const char *falcon_status_string(int status) {
     switch (status) {
         case FALCON_OK: return "ok";

@@ -41,6 +41,8 @@ template <typename T> int launch_span_masked(const FwdParams &p, cudaStream_t s)
 // bf16 chunk-parallel forward on tcgen05; returns 1 (nothing launched) for
 // shapes it does not cover, so the caller falls back to the span kernel.
 int launch_tc_chunk(const FwdParams &p, cudaStream_t s);
+// Number of tensor-core chunk kernels that gave up on a bounded wait.
+unsigned int tc_wait_timeouts();
 template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
 
