@@ -30,9 +30,12 @@
 //   G4  A=[U0^T;W^T]      B=[P o Dm;(D_w X)^T] -> [O0^T | B] (lanes 0-63)
 //   G5  A=[S;0]           B=[Qt;-Phi'^T], accumulating onto G4
 //                                        -> [O^T | B - S Phi'] (lanes 0-63)
-// One thread block per (b,h), 128 threads; warp w reads tensor-memory lanes
-// 32w..32w+31.  The next chunk's q, k, v are prefetched with cp.async.
+// One thread block per (b,h), 256 threads; warp w reads tensor-memory lanes
+// 32(w%4)..32(w%4)+31, and the two warps of a lane quarter split the columns.  The next chunk's q, k, v are prefetched with cp.async.
+#include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -44,10 +47,11 @@ namespace {
 
 constexpr int CH = 64;  // chunk
 constexpr int DD = 64;  // d_k = d_v
-constexpr int NTH = 128;
+constexpr int NTH = 256;
 constexpr uint32_t TMEM_COLS = 512;
 // accumulator columns (each starts at a multiple of 128)
 constexpr uint32_t COL_G1 = 0, COL_G2 = 128, COL_G3 = 256, COL_G45 = 384;
+constexpr uint32_t COL_S = 64;  // fp32 state S, rows j in lanes 0-63
 
 // shared-memory byte offsets; operand tiles are 64 rows x 128 B (8 KB),
 // 1024-byte aligned, 128-row operands are two consecutive tiles
@@ -63,11 +67,14 @@ constexpr uint32_t OFF_SA = 13 * TILE;     // [S ; 0]
 constexpr uint32_t OFF_KR = 15 * TILE;     // raw keys (prefetch)
 constexpr uint32_t OFF_VR0 = 16 * TILE;    // raw values, buffer 0
 constexpr uint32_t OFF_VR1 = 17 * TILE;    // raw values, buffer 1
-constexpr uint32_t OFF_MF = 18 * TILE;     // fp32 M [64][65]
-constexpr uint32_t LDF = 65;
-constexpr uint32_t OFF_TF = OFF_MF + 64 * LDF * 4;  // fp32 T [64][65]
-constexpr uint32_t OFF_ZF = OFF_TF + 64 * LDF * 4;  // fp32 scratch [32][33]
-constexpr uint32_t OFF_VEC = OFF_ZF + 32 * 33 * 4;  // per-token vectors
+constexpr uint32_t OFF_MF = 18 * TILE;     // fp32 M [64][68]
+// row stride 68 floats: float4 row stores and the m16n8k8 fragment loads
+// below are both free of bank conflicts
+constexpr uint32_t LDF = 68;
+constexpr uint32_t OFF_TF = OFF_MF + 64 * LDF * 4;  // fp32 T [64][68]
+constexpr uint32_t LDZ = 36;
+constexpr uint32_t OFF_ZF = OFF_TF + 64 * LDF * 4;  // fp32 scratch [32][36]
+constexpr uint32_t OFF_VEC = OFF_ZF + 32 * LDZ * 4;  // per-token vectors
 constexpr uint32_t OFF_BAR = OFF_VEC + 8 * 64 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;  // + alignment slack
 
@@ -94,17 +101,6 @@ __device__ __forceinline__ void unpack8(uint4 u, float *f) {
     }
 }
 
-// one bf16 element (row r, column col) of a 128-byte-swizzled tile
-__device__ __forceinline__ void st_elem(uint8_t *tile, int r, int col, float x) {
-    *reinterpret_cast<__nv_bfloat16 *>(tile + tc::sw128(r, col >> 3) + (col & 7) * 2) = __float2bfloat16_rn(x);
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
@@ -124,10 +120,29 @@ __device__ float *g_dbg;
             __threadfence_system();                                    \
         }                                                              \
     } while (0)
+__device__ long long *g_tim;
+#define TIM(c, slot)                                                                \
+    do {                                                                            \
+        if (g_tim && blockIdx.x == 0 && threadIdx.x == 0 && (c) < 64)               \
+            g_tim[(c) * 16 + (slot)] = clock64();                                   \
+    } while (0)
+#define TIMT(c, slot, th)                                                           \
+    do {                                                                            \
+        if (g_tim && blockIdx.x == 0 && threadIdx.x == (th) && (c) < 64)            \
+            g_tim[(c) * 16 + (slot)] = clock64();                                   \
+    } while (0)
+#define TIMX(c, slot)                                                               \
+    do {                                                                            \
+        if ((c) == 5 && g_tim && blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == 64)) \
+            g_tim[64 * 16 + (threadIdx.x ? 32 : 0) + (slot)] = clock64();           \
+    } while (0)
 #define DBG_ON(c) (g_dbg != nullptr && blockIdx.x == 0 && (c) < 2)
 #define DBG(c, off) (g_dbg + (size_t)(c) * 50000 + (off))
 #else
 #define STAGE(sv)
+#define TIM(c, slot)
+#define TIMT(c, slot, th)
+#define TIMX(c, slot)
 #endif
 
 // Bounded wait on the MMA-completion barrier: about two seconds at most.
@@ -139,25 +154,20 @@ __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
-// Prefetch chunk c0's raw keys (row t <- key c0+t-1), queries and values.
-__device__ __forceinline__ void prefetch(const __nv_bfloat16 *kq, const __nv_bfloat16 *kk,
-                                         const __nv_bfloat16 *kv, int L, int c0, uint32_t base,
-                                         uint32_t off_q, uint32_t off_v) {
-    for (int i = threadIdx.x; i < 3 * 64 * 8; i += NTH) {
-        const int which = i / 512, r = (i / 8) % 64, c16 = i % 8;
-        const int tok = c0 + r;
-        if (which == 0) {
-            const int kt = tok - 1;
-            const bool ok = kt >= 0 && tok < L;
-            cp_async16(base + OFF_KR + tc::sw128(r, c16), kk + (size_t)(ok ? kt : 0) * DD + c16 * 8, ok);
-        } else {
-            const bool ok = tok < L;
-            const __nv_bfloat16 *src = which == 1 ? kq : kv;
-            cp_async16(base + (which == 1 ? off_q : off_v) + tc::sw128(r, c16),
-                       src + (size_t)(ok ? tok : 0) * DD + c16 * 8, ok);
-        }
-    }
-    cp_async_commit();
+// Tensor maps of q, k, v: 3-D [B*H][L][64] bf16, boxes of 64 x 64, 128-byte swizzle.
+struct TcMaps {
+    CUtensorMap q, k, v;
+};
+
+// TMA prefetch of chunk c0 (one thread): raw keys (row t <- key c0+t-1; the
+// key before the sequence start and rows past its end read as zeros),
+// queries and values, 24 KB completing on `bar`.
+__device__ __forceinline__ void prefetch_tma(const TcMaps &m, int bh, int c0, uint32_t base, uint32_t off_q,
+                                             uint32_t off_v, uint64_t *bar) {
+    tc::mbar_arrive_expect_tx(bar, 3 * TILE);
+    tc::tma_load_3d(base + OFF_KR, &m.k, 0, c0 - 1, bh, bar);
+    tc::tma_load_3d(base + off_q, &m.q, 0, c0, bh, bar);
+    tc::tma_load_3d(base + off_v, &m.v, 0, c0, bh, bar);
 }
 
 // D = A B^T over K = 64 (four K=16 slices), both operands K-major and
@@ -174,37 +184,40 @@ __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_saddr, ui
 }
 
 // 64 fp32 columns of this thread's tensor-memory lane.
-__device__ __forceinline__ void tmem_row64(uint32_t tbase, int warp, uint32_t col, float (&v)[64]) {
-    float a[32], b[32];
-    const uint32_t addr = tbase + ((uint32_t)(warp * 32) << 16) + col;
-    tc::tmem_ld32(addr, a);
-    tc::tmem_ld32(addr + 32, b);
-    tc::tmem_wait_ld();
+
+
+
+// One warp: C (16 x 8) = A (16 x K, rows of stride lda) * B (K x 8, rows of
+// stride ldb), K a multiple of 8, fp32 in shared memory, TF32 products.
+template <int K>
+__device__ __forceinline__ void warp_gemm_16x8(const float *A, int lda, const float *B, int ldb, float (&c)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    c[0] = c[1] = c[2] = c[3] = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        v[i] = a[i];
-        v[32 + i] = b[i];
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        uint32_t a[4], b[2];
+        a[0] = tc::f2tf32(A[g * lda + k0 + t]);
+        a[1] = tc::f2tf32(A[(g + 8) * lda + k0 + t]);
+        a[2] = tc::f2tf32(A[g * lda + k0 + t + 4]);
+        a[3] = tc::f2tf32(A[(g + 8) * lda + k0 + t + 4]);
+        b[0] = tc::f2tf32(B[(k0 + t) * ldb + g]);
+        b[1] = tc::f2tf32(B[(k0 + t + 4) * ldb + g]);
+        tc::mma_tf32(c, a, b);
     }
 }
 
-__device__ __forceinline__ void store_row_bf16(uint8_t *tile, int r, const float (&v)[64], float scale = 1.f) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        float t8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t8[e] = v[c * 8 + e] * scale;
-        *reinterpret_cast<uint4 *>(tile + tc::sw128(r, c)) = pack8(t8);
-    }
-}
-
-__device__ __forceinline__ void load_row_bf16(const uint8_t *tile, int r, float (&v)[64]) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) unpack8(*reinterpret_cast<const uint4 *>(tile + tc::sw128(r, c)), &v[c * 8]);
+// Write a 16 x 8 accumulator fragment (times `scale`) to C (row stride ldc).
+__device__ __forceinline__ void warp_store_16x8(float *C, int ldc, const float (&c)[4], float scale) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    C[g * ldc + 2 * t] = scale * c[0];
+    C[g * ldc + 2 * t + 1] = scale * c[1];
+    C[(g + 8) * ldc + 2 * t] = scale * c[2];
+    C[(g + 8) * ldc + 2 * t + 1] = scale * c[3];
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p) {
+__global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __grid_constant__ TcMaps maps) {
     extern __shared__ uint8_t smem_raw[];
     // align the operand tiles to 1024 bytes of the shared address space
     const uint32_t raw_s = tc::smem_u32(smem_raw);
@@ -216,17 +229,19 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p) {
     float *vec = reinterpret_cast<float *>(sm + OFF_VEC);
     float *v_sqn = vec, *v_eta = vec + 64, *v_G = vec + 128, *v_gm1 = vec + 192, *v_gt = vec + 256,
           *v_w = vec + 320, *v_beta = vec + 384;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);       // MMA completion
+    uint64_t *tbar = reinterpret_cast<uint64_t *>(sm + OFF_BAR + 16); // TMA arrival
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // tensor-memory lane quarter of this warp, and which half of a 64-column
+    // accumulator it handles (two warps share each lane quarter)
+    const int quarter = warp & 3, chalf = warp >> 2;
+    const int row = quarter * 32 + lane;  // accumulator row this thread reads
     const bool reg = p.variant == F1;
     const int bh = blockIdx.x, h = bh % p.H;
     const int L = p.L;
     const float lam = p.lambda[h];
-    const __nv_bfloat16 *kq = static_cast<const __nv_bfloat16 *>(p.q) + (size_t)bh * L * DD;
-    const __nv_bfloat16 *kk = static_cast<const __nv_bfloat16 *>(p.k) + (size_t)bh * L * DD;
-    const __nv_bfloat16 *kv = static_cast<const __nv_bfloat16 *>(p.v) + (size_t)bh * L * DD;
     const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(p.beta) + (size_t)bh * L;
     __nv_bfloat16 *ko = static_cast<__nv_bfloat16 *>(p.out) + (size_t)bh * L * DD;
 
@@ -239,27 +254,41 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p) {
         reinterpret_cast<uint4 *>(sm + OFF_XT + TILE)[i] = z;
         reinterpret_cast<uint4 *>(sm + OFF_B5 + TILE)[i] = z;
     }
+    // T's strictly-upper blocks are read as zeros by the block products
+    for (int i = tid; i < 64 * (int)LDF; i += NTH) Tf[i] = 0.f;
     if (tid == 0) {
         tc::mbar_init(bar, 1);
+        tc::mbar_init(tbar, 1);
         tc::fence_mbar_init();
     }
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, TMEM_COLS);
         tc::tmem_relinquish();
     }
-    prefetch(kq, kk, kv, L, 0, sbase, OFF_XQ0 + TILE, OFF_VR0);
+    __syncthreads();
+    if (tid == 0) prefetch_tma(maps, bh, 0, sbase, OFF_XQ0 + TILE, OFF_VR0, tbar);
+    bool tma_inflight = true;
+    float beta_next = (tid < 64 && tid < L) ? __bfloat162float(kb[tid]) : 0.f;
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = *tmem_slot;
+    const uint32_t tlane = tbase + ((uint32_t)(quarter * 32) << 16);  // this warp's lanes
     STAGE(1);
-
-    float Sreg[64];  // warps 0,1: row j = tid of S, fp32
+    if (quarter < 2) {  // S_0 = 0 (fp32 state, rows j in lanes 0-63)
+        float z16[16];
 #pragma unroll
-    for (int i = 0; i < 64; ++i) Sreg[i] = 0.f;
-    uint32_t phase = 0;
+        for (int i = 0; i < 16; ++i) z16[i] = 0.f;
+        tc::tmem_st16(tlane + COL_S + chalf * 32, z16);
+        tc::tmem_st16(tlane + COL_S + chalf * 32 + 16, z16);
+        tc::tmem_wait_st();
+    }
+
+    uint32_t phase = 0, tphase = 0;
     bool ok = true;
     const int nchunks = (L + CH - 1) / CH;
+    const float4 *G4 = reinterpret_cast<const float4 *>(v_G);
+    const float4 *E4 = reinterpret_cast<const float4 *>(v_eta);
 
     for (int c = 0; c < nchunks && ok; ++c) {
         const int c0 = c * CH;
@@ -268,87 +297,120 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p) {
         uint8_t *tX = sm + off_xq, *tQ = sm + off_xq + TILE;
         const uint8_t *tV = sm + (cur ? OFF_VR1 : OFF_VR0);
 
-        cp_async_wait_all();
-        __syncthreads();
+        ok = wait_mma(tbar, tphase);  // this chunk's q, k, v have landed
+        tphase ^= 1;
+        tma_inflight = false;
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
         STAGE(10 * c + 2);
+        TIM(c, 0);
 
-        // ---- samples x_t = phi(k_{t-1}): two threads per row t; Y^T from the raw values
-        const int r = tid >> 1, half = tid & 1;
-        float xr[32];
+        // ---- samples x_t = phi(k_{t-1}): four threads per row t
         {
+            const int r = tid >> 2, part = tid & 3;
+            float xr[16];
             float ss = 0.f;
 #pragma unroll
-            for (int c16 = 0; c16 < 4; ++c16) {
-                unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_KR + tc::sw128(r, half * 4 + c16)), &xr[c16 * 8]);
+            for (int c16 = 0; c16 < 2; ++c16) {
+                unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_KR + tc::sw128(r, part * 2 + c16)), &xr[c16 * 8]);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) ss += xr[c16 * 8 + e] * xr[c16 * 8 + e];
             }
             ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
             const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
             float sq = 0.f;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
+            for (int e = 0; e < 16; ++e) {
                 xr[e] *= inv;
                 sq += xr[e] * xr[e];
             }
             sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+            sq += __shfl_xor_sync(0xffffffffu, sq, 2);
 #pragma unroll
-            for (int c16 = 0; c16 < 4; ++c16)
-                *reinterpret_cast<uint4 *>(tX + tc::sw128(r, half * 4 + c16)) = pack8(&xr[c16 * 8]);
-            float yv[32];
-#pragma unroll
-            for (int c16 = 0; c16 < 4; ++c16)
-                unpack8(*reinterpret_cast<const uint4 *>(tV + tc::sw128(r, half * 4 + c16)), &yv[c16 * 8]);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) st_elem(sm + OFF_XT, half * 32 + e, r, yv[e]);  // Y^T
-            if (half == 0) {
-                v_sqn[r] = sq;
-                v_beta[r] = (c0 + r < L) ? __bfloat162float(kb[c0 + r]) : 0.f;
-            }
+            for (int c16 = 0; c16 < 2; ++c16)
+                *reinterpret_cast<uint4 *>(tX + tc::sw128(r, part * 2 + c16)) = pack8(&xr[c16 * 8]);
+            if (part == 0) v_sqn[r] = sq;
+            if (tid < 64) v_beta[tid] = beta_next;
         }
         __syncthreads();
-        // raw keys and values consumed: prefetch the next chunk
-        if (c + 1 < nchunks)
-            prefetch(kq, kk, kv, L, c0 + CH, sbase, (cur ? OFF_XQ0 : OFF_XQ1) + TILE, cur ? OFF_VR0 : OFF_VR1);
+        TIM(c, 1);
+        // raw keys consumed: prefetch the next chunk (beta into a register)
+        if (c + 1 < nchunks) {
+            if (tid == 0)
+                prefetch_tma(maps, bh, c0 + CH, sbase, (cur ? OFF_XQ0 : OFF_XQ1) + TILE, cur ? OFF_VR0 : OFF_VR1,
+                             tbar);
+            tma_inflight = true;
+            beta_next = (tid < 64 && c0 + CH + tid < L) ? __bfloat162float(kb[c0 + CH + tid]) : 0.f;
+        }
+        TIM(c, 10);
 
-        // ---- steps, log decays and their chunk-local cumulative sums
-        if (tid < 64) {
-            float eta, alpha;
-            step_and_decay(v_beta[tid], v_sqn[tid], p.eps, lam, eta, alpha);
-            float la = __logf(alpha);
+        // ---- steps, log decays and their chunk-local cumulative sums (warp 0,
+        //      tokens 2l and 2l+1 on lane l)
+        if (warp == 0) {
+            const int t0 = 2 * lane;
+            float eta0, eta1, al0, al1;
+            step_and_decay(v_beta[t0], v_sqn[t0], p.eps, lam, eta0, al0);
+            step_and_decay(v_beta[t0 + 1], v_sqn[t0 + 1], p.eps, lam, eta1, al1);
+            const float la0 = __logf(al0), la1 = __logf(al1);
+            float run = la0 + la1;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, la, o);
-                if (lane >= o) la += y;
+                const float y = __shfl_up_sync(0xffffffffu, run, o);
+                if (lane >= o) run += y;
             }
-            v_eta[tid] = eta;
-            v_G[tid] = la;
+            const float G1v = run, G0v = run - la1, Gm = run - la0 - la1;  // G_{t0+1}, G_{t0}, G_{t0-1}
+            const float GC = __shfl_sync(0xffffffffu, run, 31);
+            v_eta[t0] = eta0;
+            v_eta[t0 + 1] = eta1;
+            v_G[t0] = G0v;
+            v_G[t0 + 1] = G1v;
+            v_gm1[t0] = __expf(Gm);
+            v_gm1[t0 + 1] = __expf(G0v);
+            v_gt[t0] = __expf(G0v);
+            v_gt[t0 + 1] = __expf(G1v);
+            v_w[t0] = __expf(GC - G0v) * eta0;
+            v_w[t0 + 1] = __expf(GC - G1v) * eta1;
         }
         __syncthreads();
-        if (tid >= 32 && tid < 64) v_G[tid] += v_G[31];
-        __syncthreads();
-        if (tid < 64) {
-            const float G = v_G[tid];
-            v_gm1[tid] = __expf(tid > 0 ? v_G[tid - 1] : 0.f);
-            v_gt[tid] = __expf(G);
-            v_w[tid] = __expf(v_G[63] - G) * v_eta[tid];
-        }
-        __syncthreads();
-        const float gC = __expf(v_G[63]);
-
-        // ---- (D_a X)^T (regression) and (D_w X)^T, column r of each
+        // ---- transposed operand rows: Y^T, (D_a X)^T (regression), (D_w X)^T;
+        //      thread = (column n, 16 tokens)
         {
-            const float ws = v_w[r], ga = v_gm1[r];
+            const int n = tid >> 2, s0 = (tid & 3) * 16;
+            const int cn = n >> 3, en = (n & 7) * 2;
+            const float4 *W4 = reinterpret_cast<const float4 *>(v_w);
+            const float4 *A4 = reinterpret_cast<const float4 *>(v_gm1);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                st_elem(sm + OFF_A3 + TILE, half * 32 + e, r, xr[e] * ws);
-                if (reg) st_elem(sm + OFF_XT + TILE, half * 32 + e, r, xr[e] * ga);
+            for (int sb = 0; sb < 16; sb += 8) {
+                float xv[8], y8[8], a8[8], w8[8];
+                const float4 w0 = W4[(s0 + sb) / 4], w1 = W4[(s0 + sb) / 4 + 1];
+                const float4 a0 = A4[(s0 + sb) / 4], a1 = A4[(s0 + sb) / 4 + 1];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t off = tc::sw128(s0 + sb + i, cn) + en;
+                    xv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tX + off));
+                    y8[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tV + off));
+                }
+                const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    w8[i] = xv[i] * wv[i];
+                    a8[i] = xv[i] * av[i];
+                }
+                const int chunk = (s0 + sb) >> 3;
+                *reinterpret_cast<uint4 *>(sm + OFF_XT + tc::sw128(n, chunk)) = pack8(y8);
+                *reinterpret_cast<uint4 *>(sm + OFF_A3 + TILE + tc::sw128(n, chunk)) = pack8(w8);
+                if (reg) *reinterpret_cast<uint4 *>(sm + OFF_XT + TILE + tc::sw128(n, chunk)) = pack8(a8);
             }
         }
+        TIM(c, 14);
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
         STAGE(10 * c + 3);
+        TIM(c, 2);
+        const float gC = __expf(v_G[63]);
 
         // ---- G1: [X;Q] X^T -> A (lanes 0-63), P (lanes 64-127)
         if (tid == 0) {
@@ -362,103 +424,120 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p) {
         if (!ok) break;
         tc::fence_after_sync();
         STAGE(10 * c + 4);
+        TIM(c, 3);
         {
-            float v[64];
-            tmem_row64(tbase, warp, COL_G1, v);
-#ifdef FALCON_TC_DEBUG
-            if (DBG_ON(c)) for (int i = 0; i < 64; ++i) DBG(c, (warp < 2 ? 0 : 4096) + (tid & 63) * 64 + i)[0] = v[i];
-            if (DBG_ON(c) && tid < 64) for (int i = 0; i < 7; ++i) DBG(c, 49152 + i * 64 + tid)[0] = vec[i * 64 + tid];
-#endif
-            if (warp < 2) {
-                const int t = tid;
-                const float gp = t > 0 ? v_G[t - 1] : 0.f;
+            // rows 0-63: M[t][s] = (g_{t-1}/g_s) eta_s A[t][s] for s < t (fp32);
+            // rows 64-127: (P o Dm)[t][s] = (g_t/g_s) eta_s P[t][s] for s <= t (bf16).
+            // Branch-free: every exponent is computed (argument clamped to <= 0)
+            // and masked afterwards, so the 16 chains of a slice overlap.
+            const bool mrow = quarter < 2;
+            const int t = mrow ? row : row - 64;
+            const float gref = mrow ? (t > 0 ? v_G[t - 1] : 0.f) : v_G[t];
+            const int tlim = mrow ? t : t + 1;  // s < tlim
+            const bool active = mrow ? reg : true;
 #pragma unroll
-                for (int s = 0; s < 64; ++s)
-                    Mf[t * LDF + s] = (reg && s < t) ? __expf(gp - v_G[s]) * v_eta[s] * v[s] : 0.f;
-            } else {
-                const int t = tid - 64;
-                const float gt = v_G[t];
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int cs = chalf * 2 + k2;
+                float v[16], gs[16], es[16];
+                tc::tmem_ld16(tlane + COL_G1 + cs * 16, v);
 #pragma unroll
-                for (int s = 0; s < 64; ++s) v[s] = s <= t ? v[s] * __expf(gt - v_G[s]) * v_eta[s] : 0.f;
-                store_row_bf16(sm + OFF_A3, t, v);  // P o Dm
+                for (int q = 0; q < 4; ++q) {
+                    const float4 g = G4[cs * 4 + q], e = E4[cs * 4 + q];
+                    gs[q * 4 + 0] = g.x; gs[q * 4 + 1] = g.y; gs[q * 4 + 2] = g.z; gs[q * 4 + 3] = g.w;
+                    es[q * 4 + 0] = e.x; es[q * 4 + 1] = e.y; es[q * 4 + 2] = e.z; es[q * 4 + 3] = e.w;
+                }
+                tc::tmem_wait_ld();
+                float m[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float x = __expf(fminf(gref - gs[i], 0.f)) * es[i] * v[i];
+                    m[i] = (active && cs * 16 + i < tlim) ? x : 0.f;
+                }
+                if (mrow) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<float4 *>(Mf + t * LDF + cs * 16 + q * 4) =
+                            make_float4(m[q * 4], m[q * 4 + 1], m[q * 4 + 2], m[q * 4 + 3]);
+                } else {
+                    *reinterpret_cast<uint4 *>(sm + OFF_A3 + tc::sw128(t, cs * 2)) = pack8(&m[0]);
+                    *reinterpret_cast<uint4 *>(sm + OFF_A3 + tc::sw128(t, cs * 2 + 1)) = pack8(&m[8]);
+                }
             }
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
         STAGE(10 * c + 5);
+        TIM(c, 4);
 
         uint32_t a4 = sbase + OFF_XT;  // A of G4: [U0^T; W^T], or [Y^T; 0] for the A family
         if (reg) {
-            // ---- T = (I + M)^{-1}: 16x16 diagonal blocks by forward substitution
-            if (lane < 16) {
+            // ---- T = (I + M)^{-1}.  Diagonal 16x16 blocks by forward
+            //      substitution (warp b, lane = column); the off-diagonal
+            //      blocks by T_ij = -T_ii (M_i. T_.j) with TF32 warp MMAs.
+            if (warp < 4 && lane < 16) {
                 const int b0 = warp * 16, j = lane;
                 float tcol[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    float acc = (i == j) ? 1.f : 0.f;
+                    const float *mr = Mf + (b0 + i) * LDF + b0;
+                    float acc0 = (i == j) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-                    for (int s = 0; s < i; ++s) acc -= Mf[(b0 + i) * LDF + b0 + s] * tcol[s];
-                    tcol[i] = acc;
+                    for (int s = 0; s + 1 < i; s += 2) {
+                        acc0 -= mr[s] * tcol[s];
+                        acc1 -= mr[s + 1] * tcol[s + 1];
+                    }
+                    if (i & 1) acc0 -= mr[i - 1] * tcol[i - 1];
+                    tcol[i] = acc0 + acc1;
                 }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) Tf[(b0 + i) * LDF + b0 + j] = tcol[i];
             }
             __syncthreads();
-            // 16x16 off-diagonal blocks (1,0) and (3,2): T10 = -T11 (M10 T00)
-            for (int idx = tid; idx < 512; idx += NTH) {
-                const int pb = idx >> 8, i = (idx >> 4) & 15, j = idx & 15;
+            if (warp < 4) {  // blocks (1,0) [warps 0,1] and (3,2) [warps 2,3]; warp = 8 columns
+                const int pb = warp >> 1, nt = warp & 1;
                 const int r0 = pb ? 48 : 16, q0 = pb ? 32 : 0;
-                float acc = 0.f;
-                for (int s = j; s < 16; ++s) acc += Mf[(r0 + i) * LDF + q0 + s] * Tf[(q0 + s) * LDF + q0 + j];
-                Zf[(pb * 16 + i) * 33 + j] = acc;
+                float *zw = Zf + warp * 16 * 8;  // this warp's 16 x 8 scratch
+                float c4[4];
+                warp_gemm_16x8<16>(Mf + r0 * LDF + q0, LDF, Tf + q0 * LDF + q0 + nt * 8, LDF, c4);
+                warp_store_16x8(zw, 8, c4, 1.f);
+                __syncwarp();
+                warp_gemm_16x8<16>(Tf + r0 * LDF + r0, LDF, zw, 8, c4);
+                warp_store_16x8(Tf + r0 * LDF + q0 + nt * 8, LDF, c4, -1.f);
             }
             __syncthreads();
-            for (int idx = tid; idx < 512; idx += NTH) {
-                const int pb = idx >> 8, i = (idx >> 4) & 15, j = idx & 15;
-                const int r0 = pb ? 48 : 16, q0 = pb ? 32 : 0;
-                float acc = 0.f;
-                for (int s = 0; s <= i; ++s) acc += Tf[(r0 + i) * LDF + r0 + s] * Zf[(pb * 16 + s) * 33 + j];
-                Tf[(r0 + i) * LDF + q0 + j] = -acc;
+            // 32x32 block (rows 32-63, cols 0-31); warp = one 16x8 tile
+            const int rb = warp >> 2, cb = (warp >> 1) & 1, nt = warp & 1;
+            {   // Z = M_HL T_LL
+                float c4[4];
+                warp_gemm_16x8<32>(Mf + (32 + rb * 16) * LDF, LDF, Tf + cb * 16 + nt * 8, LDF, c4);
+                warp_store_16x8(Zf + rb * 16 * LDZ + cb * 16 + nt * 8, LDZ, c4, 1.f);
             }
             __syncthreads();
-            // 32x32 off-diagonal block: T_HL = -T_HH (M_HL T_LL)
-            for (int idx = tid; idx < 1024; idx += NTH) {
-                const int i = idx >> 5, j = idx & 31;
-                float acc = 0.f;
-                for (int s = j; s < 32; ++s) acc += Mf[(32 + i) * LDF + s] * Tf[s * LDF + j];
-                Zf[i * 33 + j] = acc;
+            {   // T_HL = -T_HH Z
+                float c4[4];
+                warp_gemm_16x8<32>(Tf + (32 + rb * 16) * LDF + 32, LDF, Zf + cb * 16 + nt * 8, LDZ, c4);
+                warp_store_16x8(Tf + (32 + rb * 16) * LDF + cb * 16 + nt * 8, LDF, c4, -1.f);
             }
             __syncthreads();
-            for (int idx = tid; idx < 1024; idx += NTH) {
-                const int i = idx >> 5, j = idx & 31;
-                float acc = 0.f;
-                for (int s = 0; s <= i; ++s) acc += Tf[(32 + i) * LDF + 32 + s] * Zf[s * 33 + j];
-                Tf[(32 + i) * LDF + j] = -acc;
-            }
-            __syncthreads();
-            {
-                float t8[8];
+            {   // T (lower triangle) to bf16: thread = (row, 16 columns)
+                const int r = tid >> 2, part = tid & 3;
 #pragma unroll
-                for (int c16 = 0; c16 < 4; ++c16) {
+                for (int c16 = 0; c16 < 2; ++c16) {
+                    float t8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int s = half * 32 + c16 * 8 + e;
+                        const int s = part * 16 + c16 * 8 + e;
                         t8[e] = s <= r ? Tf[r * LDF + s] : 0.f;
                     }
-                    *reinterpret_cast<uint4 *>(sm + OFF_TA + tc::sw128(r, half * 4 + c16)) = pack8(t8);
+                    *reinterpret_cast<uint4 *>(sm + OFF_TA + tc::sw128(r, part * 2 + c16)) = pack8(t8);
                 }
             }
-#ifdef FALCON_TC_DEBUG
-            if (DBG_ON(c)) for (int i = tid; i < 4096; i += NTH) {
-                DBG(c, 8192 + i)[0] = Mf[(i / 64) * LDF + i % 64];
-                DBG(c, 12288 + i)[0] = Tf[(i / 64) * LDF + i % 64];
-            }
-#endif
             tc::fence_proxy_async();
             tc::fence_before_sync();
             __syncthreads();
             STAGE(10 * c + 6);
+            TIM(c, 5);
 
             // ---- G2: [Y^T;(D_a X)^T] T^T -> U0^T (lanes 0-63), W^T (lanes 64-127)
             if (tid == 0) {
@@ -471,18 +550,20 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p) {
             ok = __syncthreads_and(ok);
             if (!ok) break;
             tc::fence_after_sync();
-            {
-                float v[64];
-                tmem_row64(tbase, warp, COL_G2, v);
-#ifdef FALCON_TC_DEBUG
-                if (DBG_ON(c)) for (int i = 0; i < 64; ++i) DBG(c, 16384 + tid * 64 + i)[0] = v[i];
-#endif
-                store_row_bf16(sm + OFF_WUT, tid, v);
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int cs = chalf * 2 + k2;
+                float v[16];
+                tc::tmem_ld16(tlane + COL_G2 + cs * 16, v);
+                tc::tmem_wait_ld();
+                *reinterpret_cast<uint4 *>(sm + OFF_WUT + tc::sw128(row, cs * 2)) = pack8(&v[0]);
+                *reinterpret_cast<uint4 *>(sm + OFF_WUT + tc::sw128(row, cs * 2 + 1)) = pack8(&v[8]);
             }
             tc::fence_proxy_async();
             tc::fence_before_sync();
             __syncthreads();
             STAGE(10 * c + 7);
+            TIM(c, 6);
 
             // ---- G3: [P o Dm;(D_w X)^T] W -> (P o Dm) W (lanes 0-63), Phi'^T (lanes 64-127)
             if (tid == 0) {
@@ -496,32 +577,50 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p) {
             if (!ok) break;
             tc::fence_after_sync();
             {
-                float v[64];
-                tmem_row64(tbase, warp, COL_G3, v);
-#ifdef FALCON_TC_DEBUG
-                if (DBG_ON(c)) for (int i = 0; i < 64; ++i) DBG(c, 24576 + tid * 64 + i)[0] = v[i];
-#endif
-                if (warp < 2) {  // Qt = D_g Q - (P o Dm) W
-                    float qrow[64];
-                    load_row_bf16(tQ, tid, qrow);
-                    const float g = v_gt[tid];
+                const bool qrow = quarter < 2;
+                const float g = qrow ? v_gt[row] : -1.f;
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) v[i] = g * qrow[i] - v[i];
-                    store_row_bf16(sm + OFF_B5, tid, v);
-                } else {  // -Phi'^T
-                    store_row_bf16(sm + OFF_B5 + TILE, tid - 64, v, -1.f);
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    const int cs = chalf * 2 + k2;
+                    float v[16];
+                    tc::tmem_ld16(tlane + COL_G3 + cs * 16, v);
+                    tc::tmem_wait_ld();
+                    if (qrow) {  // Qt = D_g Q - (P o Dm) W
+                        float q8[8];
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            unpack8(*reinterpret_cast<const uint4 *>(tQ + tc::sw128(row, cs * 2 + hh)), q8);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) v[hh * 8 + i] = g * q8[i] - v[hh * 8 + i];
+                        }
+                        *reinterpret_cast<uint4 *>(sm + OFF_B5 + tc::sw128(row, cs * 2)) = pack8(&v[0]);
+                        *reinterpret_cast<uint4 *>(sm + OFF_B5 + tc::sw128(row, cs * 2 + 1)) = pack8(&v[8]);
+                    } else {  // -Phi'^T
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = -v[i];
+                        *reinterpret_cast<uint4 *>(sm + OFF_B5 + TILE + tc::sw128(row - 64, cs * 2)) = pack8(&v[0]);
+                        *reinterpret_cast<uint4 *>(sm + OFF_B5 + TILE + tc::sw128(row - 64, cs * 2 + 1)) =
+                            pack8(&v[8]);
+                    }
                 }
             }
             a4 = sbase + OFF_WUT;
-        } else if (warp < 2) {  // inner-product family: Qt = D_g Q
-            float qrow[64];
-            load_row_bf16(tQ, tid, qrow);
-            store_row_bf16(sm + OFF_B5, tid, qrow, v_gt[tid]);
+        } else if (quarter < 2) {  // inner-product family: Qt = D_g Q
+            const float g = v_gt[row];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float q8[8];
+                unpack8(*reinterpret_cast<const uint4 *>(tQ + tc::sw128(row, chalf * 4 + cc)), q8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q8[i] *= g;
+                *reinterpret_cast<uint4 *>(sm + OFF_B5 + tc::sw128(row, chalf * 4 + cc)) = pack8(q8);
+            }
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
         STAGE(10 * c + 8);
+        TIM(c, 7);
 
         // ---- G4 then G5 (the chain) into one accumulator:
         //      [U0^T;W^T] [P o Dm;(D_w X)^T]^T + [S;0] [Qt;-Phi'^T]^T
@@ -536,47 +635,102 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p) {
         ok = __syncthreads_and(ok);
         if (!ok) break;
         tc::fence_after_sync();
-        {
-            float v[64], e[64];
-            tmem_row64(tbase, warp, COL_G45, v);       // O^T[j][t]
-            tmem_row64(tbase, warp, COL_G45 + 64, e);  // (B - S Phi')[j][k]
-#ifdef FALCON_TC_DEBUG
-            if (DBG_ON(c) && warp < 2) for (int i = 0; i < 64; ++i) {
-                DBG(c, 32768 + tid * 128 + i)[0] = v[i];
-                DBG(c, 32768 + tid * 128 + 64 + i)[0] = e[i];
-            }
-#endif
-            if (warp < 2) {
-                const int j = tid;
-                const int nt = min(CH, L - c0);
+        TIM(c, 8);
+        if (quarter < 2) {
+            const int j = row;
+            const int nt = min(CH, L - c0);
+            // outputs: O^T[j][t] -> out[c0 + t][j], this warp's 32 tokens
 #pragma unroll
-                for (int t = 0; t < 64; ++t)
-                    if (t < nt) ko[(size_t)(c0 + t) * DD + j] = __float2bfloat16_rn(v[t]);
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int cs = chalf * 2 + k2;
+                float v[16];
+                tc::tmem_ld16(tlane + COL_G45 + cs * 16, v);
+                tc::tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 64; ++i) Sreg[i] = gC * Sreg[i] + e[i];
-                store_row_bf16(sm + OFF_SA, j, Sreg);
+                for (int i = 0; i < 16; ++i)
+                    if (cs * 16 + i < nt) ko[(size_t)(c0 + cs * 16 + i) * DD + j] = __float2bfloat16_rn(v[i]);
             }
+            // state: S_end = g_C S + (B - S Phi'), fp32 in tensor memory, bf16 copy for the next chain MMA
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int cs = chalf * 2 + k2;
+                float ds[16], sv[16];
+                tc::tmem_ld16(tlane + COL_G45 + 64 + cs * 16, ds);
+                tc::tmem_ld16(tlane + COL_S + cs * 16, sv);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sv[i] = gC * sv[i] + ds[i];
+                tc::tmem_st16(tlane + COL_S + cs * 16, sv);
+                *reinterpret_cast<uint4 *>(sm + OFF_SA + tc::sw128(j, cs * 2)) = pack8(&sv[0]);
+                *reinterpret_cast<uint4 *>(sm + OFF_SA + tc::sw128(j, cs * 2 + 1)) = pack8(&sv[8]);
+            }
+            tc::tmem_wait_st();
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
         STAGE(10 * c + 9);
+        TIM(c, 9);
     }
 
     STAGE(ok ? 9999 : -2);
     if (!ok && tid == 0) atomicAdd(&g_tc_wait_timeouts, 1u);
-    if (ok && p.final_state && warp < 2) {
-        float *fs = p.final_state + ((size_t)bh * DD + tid) * DD;
+    if (ok && p.final_state && quarter < 2) {
+        float *fs = p.final_state + ((size_t)bh * DD + row) * DD;
+        tc::fence_after_sync();
 #pragma unroll
-        for (int c16 = 0; c16 < 16; ++c16)
-            *reinterpret_cast<float4 *>(fs + c16 * 4) =
-                make_float4(Sreg[c16 * 4], Sreg[c16 * 4 + 1], Sreg[c16 * 4 + 2], Sreg[c16 * 4 + 3]);
+        for (int k2 = 0; k2 < 2; ++k2) {
+            const int cs = chalf * 2 + k2;
+            float sv[16];
+            tc::tmem_ld16(tlane + COL_S + cs * 16, sv);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<float4 *>(fs + cs * 16 + q * 4) =
+                    make_float4(sv[q * 4], sv[q * 4 + 1], sv[q * 4 + 2], sv[q * 4 + 3]);
+        }
     }
-    cp_async_wait_all();
+    // a prefetch abandoned by an early exit must land before the block leaves
+    if (tma_inflight && !ok) (void)wait_mma(tbar, tphase);
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tbase, TMEM_COLS);
 }
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// [B*H][L][64] bf16 tensor, 64 x 64 boxes, 128-byte swizzle, zero fill outside.
+bool make_map(CUtensorMap *m, const void *base, int BH, int L) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)DD, (cuuint64_t)L, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)DD * 2, (cuuint64_t)L * DD * 2};
+    const cuuint32_t box[3] = {DD, CH, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
 
 int launch_tc_chunk(const FwdParams &p, cudaStream_t s) {
     const bool shape_ok = (p.variant == F1 || p.variant == F1A) && p.dk == DD && p.dv == DD && p.chunk == CH &&
@@ -585,8 +739,12 @@ int launch_tc_chunk(const FwdParams &p, cudaStream_t s) {
     if (!shape_ok || !al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.out) ||
         (p.final_state && !al16(p.final_state)))
         return 1;
+    TcMaps maps;
+    const int BH = p.B * p.H;
+    if (!make_map(&maps.q, p.q, BH, p.L) || !make_map(&maps.k, p.k, BH, p.L) || !make_map(&maps.v, p.v, BH, p.L))
+        return 1;
     cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    chunk_tc_kernel<<<p.B * p.H, NTH, SMEM_BYTES, s>>>(p);
+    chunk_tc_kernel<<<BH, NTH, SMEM_BYTES, s>>>(p, maps);
     return 0;
 }
 
@@ -598,6 +756,9 @@ extern "C" int *falcon_tc_debug_stage_alloc(int n) {
     if (cudaHostGetDevicePointer((void **)&d, h, 0) != cudaSuccess) return nullptr;
     if (cudaMemcpyToSymbol(g_stage, &d, sizeof(d)) != cudaSuccess) return nullptr;
     return h;
+}
+extern "C" int falcon_tc_debug_timer_set(long long *ptr) {
+    return cudaMemcpyToSymbol(g_tim, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;
 }
 extern "C" int falcon_tc_debug_set(float *ptr) {
     return cudaMemcpyToSymbol(g_dbg, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;
