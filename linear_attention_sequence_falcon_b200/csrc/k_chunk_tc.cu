@@ -22,8 +22,10 @@
 // factor is a difference of cumulative logs, hence <= 1.
 //
 // Every tcgen05 operand is K-major (rows of 128 bytes, 128-byte swizzle), so
-// each product is laid out as D = A B^T with both operands stored row-wise:
+// each product is laid out as D = A B^T with both operands stored row-wise;
+// the transposed operands are made by the tensor core itself (A = [.; I]):
 //   G1  A=[X;Q]           B=X            -> A (lanes 0-63), P (lanes 64-127)
+//   GT  A=[.;I] B=X -> X^T (lanes 64-127);  A=[I;.] B=Y -> Y^T (lanes 0-63)
 //       CUDA cores: M, P o Dm, T = (I+M)^{-1} (16x16 blocked inversion, fp32)
 //   G2  A=[Y^T;(D_a X)^T] B=T            -> U0^T (lanes 0-63), W^T (64-127)
 //   G3  A=[P o Dm;(D_w X)^T] B=W^T       -> (P o Dm)W (0-63), Phi'^T (64-127)
@@ -48,10 +50,12 @@ namespace {
 constexpr int CH = 64;  // chunk
 constexpr int DD = 64;  // d_k = d_v
 constexpr int NTH = 256;
+constexpr int ISSUER = 128;  // the thread that issues every tensor-core MMA (warp 4)
 constexpr uint32_t TMEM_COLS = 512;
 // accumulator columns (each starts at a multiple of 128)
 constexpr uint32_t COL_G1 = 0, COL_G2 = 128, COL_G3 = 256, COL_G45 = 384;
 constexpr uint32_t COL_S = 64;  // fp32 state S, rows j in lanes 0-63
+constexpr uint32_t COL_XT = 192, COL_YT = 320;  // X^T in lanes 64-127, Y^T in lanes 0-63
 
 // shared-memory byte offsets; operand tiles are 64 rows x 128 B (8 KB),
 // 1024-byte aligned, 128-row operands are two consecutive tiles
@@ -67,7 +71,8 @@ constexpr uint32_t OFF_SA = 13 * TILE;     // [S ; 0]
 constexpr uint32_t OFF_KR = 15 * TILE;     // raw keys (prefetch)
 constexpr uint32_t OFF_VR0 = 16 * TILE;    // raw values, buffer 0
 constexpr uint32_t OFF_VR1 = 17 * TILE;    // raw values, buffer 1
-constexpr uint32_t OFF_MF = 18 * TILE;     // fp32 M [64][68]
+constexpr uint32_t OFF_IDT = 18 * TILE;    // bf16 identity (the tile before it pads A to 128 rows)
+constexpr uint32_t OFF_MF = 19 * TILE;     // fp32 M [64][68]
 // row stride 68 floats: float4 row stores and the m16n8k8 fragment loads
 // below are both free of bank conflicts
 constexpr uint32_t LDF = 68;
@@ -254,6 +259,17 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
         reinterpret_cast<uint4 *>(sm + OFF_XT + TILE)[i] = z;
         reinterpret_cast<uint4 *>(sm + OFF_B5 + TILE)[i] = z;
     }
+    // identity operand (bf16 1.0 = 0x3F80 on the diagonal)
+    for (int i = tid; i < 64 * 8; i += NTH) {
+        const int r = i >> 3, c16 = i & 7;
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if ((r >> 3) == c16) {
+            const uint32_t one = 0x3F80u << (16 * (r & 1));
+            const int word = (r & 7) >> 1;
+            if (word == 0) u.x = one; else if (word == 1) u.y = one; else if (word == 2) u.z = one; else u.w = one;
+        }
+        *reinterpret_cast<uint4 *>(sm + OFF_IDT + tc::sw128(r, c16)) = u;
+    }
     // T's strictly-upper blocks are read as zeros by the block products
     for (int i = tid; i < 64 * (int)LDF; i += NTH) Tf[i] = 0.f;
     if (tid == 0) {
@@ -261,14 +277,22 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
         tc::mbar_init(tbar, 1);
         tc::fence_mbar_init();
     }
+    if (tid == NTH - 32) {
+        tc::prefetch_tmap(&maps.q);
+        tc::prefetch_tmap(&maps.k);
+        tc::prefetch_tmap(&maps.v);
+    }
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, TMEM_COLS);
         tc::tmem_relinquish();
     }
     __syncthreads();
-    if (tid == 0) prefetch_tma(maps, bh, 0, sbase, OFF_XQ0 + TILE, OFF_VR0, tbar);
+    if (tid == NTH - 32) prefetch_tma(maps, bh, 0, sbase, OFF_XQ0 + TILE, OFF_VR0, tbar);
     bool tma_inflight = true;
-    float beta_next = (tid < 64 && tid < L) ? __bfloat162float(kb[tid]) : 0.f;
+    // beta of the next chunk travels as raw bf16 and is converted only when it
+    // is stored a chunk later, so no warp waits on the global load
+    __nv_bfloat16 beta_next = __float2bfloat16_rn(0.f);
+    if (tid < 64 && tid < L) beta_next = kb[tid];
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -295,7 +319,6 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
         const int cur = c & 1;
         const uint32_t off_xq = cur ? OFF_XQ1 : OFF_XQ0;
         uint8_t *tX = sm + off_xq, *tQ = sm + off_xq + TILE;
-        const uint8_t *tV = sm + (cur ? OFF_VR1 : OFF_VR0);
 
         ok = wait_mma(tbar, tphase);  // this chunk's q, k, v have landed
         tphase ^= 1;
@@ -331,17 +354,31 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
             for (int c16 = 0; c16 < 2; ++c16)
                 *reinterpret_cast<uint4 *>(tX + tc::sw128(r, part * 2 + c16)) = pack8(&xr[c16 * 8]);
             if (part == 0) v_sqn[r] = sq;
-            if (tid < 64) v_beta[tid] = beta_next;
+            if (tid < 64) v_beta[tid] = __bfloat162float(beta_next);
         }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
         __syncthreads();
         TIM(c, 1);
+        // ---- G1 [X;Q] X^T -> A, P and GT [.;I] X^T, [.;I] Y^T -> X^T, Y^T; they
+        //      depend only on the samples and run while the steps are computed
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_gemm(tbase + COL_G1, sbase + off_xq, sbase + off_xq, 64, false);
+            issue_gemm(tbase + COL_XT, sbase + OFF_IDT - TILE, sbase + off_xq, 64, false);
+            issue_gemm(tbase + COL_YT, sbase + OFF_IDT, sbase + (cur ? OFF_VR1 : OFF_VR0), 64, false);
+            tc::mma_commit(bar);
+        }
+        TIMT(c, 12, ISSUER);
         // raw keys consumed: prefetch the next chunk (beta into a register)
         if (c + 1 < nchunks) {
-            if (tid == 0)
+            if (tid == NTH - 32)
                 prefetch_tma(maps, bh, c0 + CH, sbase, (cur ? OFF_XQ0 : OFF_XQ1) + TILE, cur ? OFF_VR0 : OFF_VR1,
                              tbar);
+            TIMT(c, 13, NTH - 32);
             tma_inflight = true;
-            beta_next = (tid < 64 && c0 + CH + tid < L) ? __bfloat162float(kb[c0 + CH + tid]) : 0.f;
+            beta_next = __float2bfloat16_rn(0.f);
+            if (tid < 64 && c0 + CH + tid < L) beta_next = kb[c0 + CH + tid];
         }
         TIM(c, 10);
 
@@ -349,9 +386,11 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
         //      tokens 2l and 2l+1 on lane l)
         if (warp == 0) {
             const int t0 = 2 * lane;
-            float eta0, eta1, al0, al1;
-            step_and_decay(v_beta[t0], v_sqn[t0], p.eps, lam, eta0, al0);
-            step_and_decay(v_beta[t0 + 1], v_sqn[t0 + 1], p.eps, lam, eta1, al1);
+            // eta = beta / (eps + n) (0 for an empty sample), alpha = max(1 - eta lambda, 2^-20)
+            const float n0 = v_sqn[t0], n1 = v_sqn[t0 + 1];
+            const float eta0 = n0 > 0.f ? __fdividef(v_beta[t0], p.eps + n0) : 0.f;
+            const float eta1 = n1 > 0.f ? __fdividef(v_beta[t0 + 1], p.eps + n1) : 0.f;
+            const float al0 = fmaxf(1.f - eta0 * lam, kAlphaFloor), al1 = fmaxf(1.f - eta1 * lam, kAlphaFloor);
             const float la0 = __logf(al0), la1 = __logf(al1);
             float run = la0 + la1;
 #pragma unroll
@@ -372,52 +411,12 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
             v_w[t0] = __expf(GC - G0v) * eta0;
             v_w[t0 + 1] = __expf(GC - G1v) * eta1;
         }
-        __syncthreads();
-        // ---- transposed operand rows: Y^T, (D_a X)^T (regression), (D_w X)^T;
-        //      thread = (column n, 16 tokens)
-        {
-            const int n = tid >> 2, s0 = (tid & 3) * 16;
-            const int cn = n >> 3, en = (n & 7) * 2;
-            const float4 *W4 = reinterpret_cast<const float4 *>(v_w);
-            const float4 *A4 = reinterpret_cast<const float4 *>(v_gm1);
-#pragma unroll
-            for (int sb = 0; sb < 16; sb += 8) {
-                float xv[8], y8[8], a8[8], w8[8];
-                const float4 w0 = W4[(s0 + sb) / 4], w1 = W4[(s0 + sb) / 4 + 1];
-                const float4 a0 = A4[(s0 + sb) / 4], a1 = A4[(s0 + sb) / 4 + 1];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t off = tc::sw128(s0 + sb + i, cn) + en;
-                    xv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tX + off));
-                    y8[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tV + off));
-                }
-                const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    w8[i] = xv[i] * wv[i];
-                    a8[i] = xv[i] * av[i];
-                }
-                const int chunk = (s0 + sb) >> 3;
-                *reinterpret_cast<uint4 *>(sm + OFF_XT + tc::sw128(n, chunk)) = pack8(y8);
-                *reinterpret_cast<uint4 *>(sm + OFF_A3 + TILE + tc::sw128(n, chunk)) = pack8(w8);
-                if (reg) *reinterpret_cast<uint4 *>(sm + OFF_XT + TILE + tc::sw128(n, chunk)) = pack8(a8);
-            }
-        }
-        TIM(c, 14);
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
+        TIMT(c, 11, 0);
         __syncthreads();
         STAGE(10 * c + 3);
         TIM(c, 2);
         const float gC = __expf(v_G[63]);
 
-        // ---- G1: [X;Q] X^T -> A (lanes 0-63), P (lanes 64-127)
-        if (tid == 0) {
-            tc::fence_after_sync();
-            issue_gemm(tbase + COL_G1, sbase + off_xq, sbase + off_xq, 64, false);
-            tc::mma_commit(bar);
-        }
         ok = wait_mma(bar, phase);
         phase ^= 1;
         ok = __syncthreads_and(ok);
@@ -458,9 +457,38 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
                     for (int q = 0; q < 4; ++q)
                         *reinterpret_cast<float4 *>(Mf + t * LDF + cs * 16 + q * 4) =
                             make_float4(m[q * 4], m[q * 4 + 1], m[q * 4 + 2], m[q * 4 + 3]);
+                    // Y^T row n = t -> XT[n]
+                    float yt[16];
+                    tc::tmem_ld16(tlane + COL_YT + cs * 16, yt);
+                    tc::tmem_wait_ld();
+                    *reinterpret_cast<uint4 *>(sm + OFF_XT + tc::sw128(t, cs * 2)) = pack8(&yt[0]);
+                    *reinterpret_cast<uint4 *>(sm + OFF_XT + tc::sw128(t, cs * 2 + 1)) = pack8(&yt[8]);
                 } else {
                     *reinterpret_cast<uint4 *>(sm + OFF_A3 + tc::sw128(t, cs * 2)) = pack8(&m[0]);
                     *reinterpret_cast<uint4 *>(sm + OFF_A3 + tc::sw128(t, cs * 2 + 1)) = pack8(&m[8]);
+                    // transposed rows n = t: (D_w X)^T -> A3[64+n], (D_a X)^T -> XT[64+n] (regression)
+                    float xt[16], ws[16], as[16];
+                    tc::tmem_ld16(tlane + COL_XT + cs * 16, xt);
+                    const float4 *W4 = reinterpret_cast<const float4 *>(v_w);
+                    const float4 *A4 = reinterpret_cast<const float4 *>(v_gm1);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 w = W4[cs * 4 + q], a = A4[cs * 4 + q];
+                        ws[q * 4 + 0] = w.x; ws[q * 4 + 1] = w.y; ws[q * 4 + 2] = w.z; ws[q * 4 + 3] = w.w;
+                        as[q * 4 + 0] = a.x; as[q * 4 + 1] = a.y; as[q * 4 + 2] = a.z; as[q * 4 + 3] = a.w;
+                    }
+                    tc::tmem_wait_ld();
+                    float o8[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o8[i] = xt[i] * ws[i];
+                    *reinterpret_cast<uint4 *>(sm + OFF_A3 + TILE + tc::sw128(t, cs * 2)) = pack8(&o8[0]);
+                    *reinterpret_cast<uint4 *>(sm + OFF_A3 + TILE + tc::sw128(t, cs * 2 + 1)) = pack8(&o8[8]);
+                    if (reg) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) o8[i] = xt[i] * as[i];
+                        *reinterpret_cast<uint4 *>(sm + OFF_XT + TILE + tc::sw128(t, cs * 2)) = pack8(&o8[0]);
+                        *reinterpret_cast<uint4 *>(sm + OFF_XT + TILE + tc::sw128(t, cs * 2 + 1)) = pack8(&o8[8]);
+                    }
                 }
             }
         }
@@ -540,7 +568,7 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
             TIM(c, 5);
 
             // ---- G2: [Y^T;(D_a X)^T] T^T -> U0^T (lanes 0-63), W^T (lanes 64-127)
-            if (tid == 0) {
+            if (tid == ISSUER) {
                 tc::fence_after_sync();
                 issue_gemm(tbase + COL_G2, sbase + OFF_XT, sbase + OFF_TA, 64, false);
                 tc::mma_commit(bar);
@@ -566,7 +594,7 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
             TIM(c, 6);
 
             // ---- G3: [P o Dm;(D_w X)^T] W -> (P o Dm) W (lanes 0-63), Phi'^T (lanes 64-127)
-            if (tid == 0) {
+            if (tid == ISSUER) {
                 tc::fence_after_sync();
                 issue_gemm(tbase + COL_G3, sbase + OFF_A3, sbase + OFF_WUT + TILE, 64, false);
                 tc::mma_commit(bar);
@@ -624,7 +652,7 @@ __global__ void __launch_bounds__(NTH, 1) chunk_tc_kernel(FwdParams p, const __g
 
         // ---- G4 then G5 (the chain) into one accumulator:
         //      [U0^T;W^T] [P o Dm;(D_w X)^T]^T + [S;0] [Qt;-Phi'^T]^T
-        if (tid == 0) {
+        if (tid == ISSUER) {
             tc::fence_after_sync();
             issue_gemm(tbase + COL_G45, a4, sbase + OFF_A3, 128, false);
             issue_gemm(tbase + COL_G45, sbase + OFF_SA, sbase + OFF_B5, 128, true);

@@ -64,6 +64,11 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int 
         : "memory");
 }
 
+// Pull a tensor map (kernel parameter) into the descriptor cache.
+__device__ __forceinline__ void prefetch_tmap(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
 // ---------------------------------------------------------------- fences
 
 // Make generic-proxy writes to shared memory visible to the async proxy
