@@ -262,6 +262,10 @@ def run_ours(args):
             step()
         torch.cuda.synchronize()
         return
+    if args.profile_decode:
+        args.steps = max(args.steps, 1)
+        measure_decode(F, gen, stream, flush, peaks()[0], args, profile=True)
+        return
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
         step()
@@ -316,6 +320,8 @@ def run_ours(args):
             "traffic": None, "kernel": "falcon chunk-parallel forward, Falcon-1", "peak_source": src,
             "algorithmic_bytes_per_launch": ab, "launch_ms": f1_ms}
 
+    decode = measure_decode(F, gen, stream, flush, hbm, args) if not args.no_decode else None
+
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -323,6 +329,8 @@ def run_ours(args):
             "per_variant_ms": {var: statistics.mean(per_var[var]) for var in w["variants"]},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": len(w["variants"]) * args.steps, "clocks": clk.summary()}
+    if decode is not None:
+        line["decode"] = decode
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, threads, units, used = cpu_oracle_sample(budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -335,6 +343,51 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def measure_decode(F, gen, stream, flush, hbm, args, profile=False):
+    """Decode row: one falcon_decode_step per step for N sequences (workload 5:
+    Falcon-2A, N=64, H=16, 128x128 fp32 state per head), L2 flushed before
+    every timed step (the 64 MiB state would otherwise stay in L2)."""
+    import torch
+    dd = DECODE
+    N, H, dk, dv = dd["N"], dd["H"], dd["dk"], dd["dv"]
+    pool = 16
+    d = gen.draw_decode(dd["variant"], N, H, dk, dv, pool, seed=dd["seed"], lam=dd["lam"])
+    q, k, v, beta = (d[n].cuda() for n in ("q", "k", "v", "beta"))
+    lam = d["lam"].cuda()
+    state = torch.zeros((N, H, dv, dk), dtype=torch.float32, device="cuda")
+    x_prev = torch.zeros((N, H, dk), dtype=torch.float32, device="cuda")
+    out = torch.empty((N, H, dv), dtype=torch.bfloat16, device="cuda")
+    steps = max(args.steps, 20)
+
+    def one(i):
+        F.decode_step(dd["variant"], q[i % pool], k[i % pool], v[i % pool], beta[i % pool], lam, d["eps"], 1,
+                      state, x_prev, out=out, stream=stream)
+
+    if profile:  # decode steps only, for profilers
+        for i in range(args.warmup + args.steps):
+            one(i)
+        torch.cuda.synchronize()
+        return None
+    for i in range(max(args.warmup, 3)):
+        one(i)
+    ms = []
+    for i in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        one(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    t = statistics.mean(ms)
+    ab = algorithmic_bytes_decode(N, H, dk, dv, per_channel=True)
+    gbs = ab / (t / 1e3) / 1e9
+    return {"workload": "falcon2A-decode-bf16-N64xH16-state128x128-fp32", "us_per_step": t * 1e3,
+            "tokens_per_s": N / (t / 1e3), "steps": steps, "l2": "flushed before every timed step",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "algorithmic_bytes_per_launch": ab, "traffic": None}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -343,6 +396,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--profile-decode", action="store_true",
+                    help="run only warmup+steps decode steps (no flush or JSON), for ncu")
     ap.add_argument("--profile", action="store_true",
                     help="run only warmup+steps device steps (no flush, e2e, clocks or JSON), for ncu")
     args = ap.parse_args()

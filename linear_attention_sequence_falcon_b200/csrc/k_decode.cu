@@ -149,6 +149,102 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
     }
 }
 
+// Window-1 variants (Falcon-1/2/1A/2A), the decode hot path.  A row of S is
+// held by LPR = min(8, DK/4) lanes, lane l owning float4 slots l, l+LPR, ...
+// (every load instruction reads LPR*16 contiguous bytes of a row), so a row's
+// dot products need only log2(LPR) shuffle steps; 1/(eps+n), beta and the
+// shared sample are staged once per block, never per row.
+template <typename T, int DK>
+__global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
+    constexpr int LPR = DK >= 32 ? 8 : DK / 4;
+    constexpr int NV4 = DK / (4 * LPR);  // float4 per lane per row
+    constexpr int RPW = 32 / LPR;        // rows per warp per pass
+    constexpr int NW = 8;
+    __shared__ __align__(16) float xs[DK];
+    __shared__ __align__(16) float qs[DK];
+    __shared__ float ks[DK];
+    __shared__ float ys[128];
+    __shared__ float bs[128];
+    __shared__ float red[3][NW];
+
+    const VariantInfo vi = variant_info(p.variant, 1);
+    const int nh = blockIdx.x, h = nh % p.H, dv = p.dv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
+    const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
+    const T *v = static_cast<const T *>(p.v) + (size_t)nh * dv;
+    const T *beta = static_cast<const T *>(p.beta) + (size_t)nh * (vi.per_channel ? dv : 1);
+    float *xp = p.x_prev + (size_t)nh * DK;
+
+    // stage the sample x = x_prev, q, k, v and beta; block sums of |x|^2, x.q, |k|^2
+    float px = 0.f, pq = 0.f, pk = 0.f;
+    for (int i = threadIdx.x; i < DK; i += blockDim.x) {
+        const float xv = xp[i], qv = to_f32(q[i]), kv = to_f32(k[i]);
+        xs[i] = xv;
+        qs[i] = qv;
+        ks[i] = kv;
+        px += xv * xv;
+        pq += xv * qv;
+        pk += kv * kv;
+    }
+    for (int i = threadIdx.x; i < dv; i += blockDim.x) {
+        ys[i] = to_f32(v[i]);
+        bs[i] = to_f32(beta[vi.per_channel ? i : 0]);
+    }
+    px = group_sum<32>(px);
+    pq = group_sum<32>(pq);
+    pk = group_sum<32>(pk);
+    if (lane == 0) { red[0][warp] = px; red[1][warp] = pq; red[2][warp] = pk; }
+    __syncthreads();
+    float n = 0.f, xq = 0.f, knorm = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) { n += red[0][w]; xq += red[1][w]; knorm += red[2][w]; }
+    const float inv_den = n > 0.f ? 1.f / (p.eps + n) : 0.f;  // eta = beta * inv_den
+    const float lam = p.lambda[h];
+
+    const int sl = lane % LPR, rsub = warp * RPW + lane / LPR;
+    float4 xr[NV4], qr[NV4];
+#pragma unroll
+    for (int i = 0; i < NV4; ++i) {
+        xr[i] = *reinterpret_cast<const float4 *>(&xs[4 * (sl + LPR * i)]);
+        qr[i] = *reinterpret_cast<const float4 *>(&qs[4 * (sl + LPR * i)]);
+    }
+    float *S = p.state + (size_t)nh * dv * DK;
+    T *out = static_cast<T *>(p.out) + (size_t)nh * dv;
+
+    for (int row = rsub; row < dv; row += NW * RPW) {
+        float4 s4[NV4];
+        float4 *Srow = reinterpret_cast<float4 *>(S + (size_t)row * DK);
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) s4[i] = Srow[sl + LPR * i];
+        float sq = 0.f, sx = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) {
+            sq += s4[i].x * qr[i].x + s4[i].y * qr[i].y + s4[i].z * qr[i].z + s4[i].w * qr[i].w;
+            sx += s4[i].x * xr[i].x + s4[i].y * xr[i].y + s4[i].z * xr[i].z + s4[i].w * xr[i].w;
+        }
+        sq = group_sum<LPR>(sq);
+        if (vi.regression) sx = group_sum<LPR>(sx);
+        const float eta = bs[row] * inv_den;
+        const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
+        const float e = vi.regression ? ys[row] - sx : ys[row];
+        const float ge = eta * e;
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) {
+            float4 r;
+            r.x = alpha * s4[i].x + ge * xr[i].x;
+            r.y = alpha * s4[i].y + ge * xr[i].y;
+            r.z = alpha * s4[i].z + ge * xr[i].z;
+            r.w = alpha * s4[i].w + ge * xr[i].w;
+            Srow[sl + LPR * i] = r;
+        }
+        if (sl == 0) out[row] = from_f32<T>(alpha * sq + ge * xq);
+    }
+    // carry: x_prev <- phi(k_t)
+    const float kinv = knorm > 0.f ? rsqrtf(knorm) : 0.f;
+    for (int i = threadIdx.x; i < DK; i += blockDim.x) xp[i] = ks[i] * kinv;
+}
+
 template <typename T, int DK>
 __global__ void __launch_bounds__(128) carry_kernel(CarryParams p) {
     const VariantInfo vi = variant_info(p.variant, p.window);
@@ -180,7 +276,10 @@ __global__ void __launch_bounds__(128) carry_kernel(CarryParams p) {
 
 template <typename T, int DK>
 static void launch_decode_dk(const DecodeParams &p, cudaStream_t s) {
-    decode_kernel<T, DK><<<p.N * p.H, 256, 0, s>>>(p);
+    if (variant_info(p.variant, p.window).window == 1)
+        decode1_kernel<T, DK><<<p.N * p.H, 256, 0, s>>>(p);
+    else
+        decode_kernel<T, DK><<<p.N * p.H, 256, 0, s>>>(p);
 }
 
 template <typename T>
