@@ -130,12 +130,19 @@ def dist_setup(args):
     return rank, world, local
 
 
+def _dist_device():
+    import torch
+    import torch.distributed as dist
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
 def max_over_ranks(x, world):
+    """The job's time is the slowest rank's (one all-reduce MAX, no data-path collective)."""
     import torch
     import torch.distributed as dist
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_dist_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -145,7 +152,15 @@ def barrier(world):
     import torch.distributed as dist
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def weak_scaling_value(world, tokens_per_step, steps, local_ms):
+    """Whole-job tokens/s: every rank processes its own full batch (weak
+    scaling), the job time is the max over ranks."""
+    total_ms = max_over_ranks(local_ms, world)
+    return world * tokens_per_step * steps / (total_ms / 1e3), total_ms
 
 
 class OracleSample:
@@ -283,9 +298,8 @@ def run_ours(args):
                 per_var[var].append(ev[var][0].elapsed_time(ev[var][1]))
             step_ms.append(sum(ev[var][0].elapsed_time(ev[var][1]) for var in w["variants"]))
         barrier(world)
-    total_ms = max_over_ranks(sum(step_ms), world)
     tokens_per_step = len(w["variants"]) * w["B"] * w["L"]
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value, total_ms = weak_scaling_value(world, tokens_per_step, args.steps, sum(step_ms))
 
     # end to end through the C ABI from pinned host buffers
     hq, hk, hv, hb = (d[n].pin_memory() for n in ("q", "k", "v", "beta"))
@@ -306,8 +320,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         if i >= max(args.warmup, 3):
             e2e_ms.append(e0.elapsed_time(e1))
-    e2e_total = max_over_ranks(sum(e2e_ms), world)
-    e2e_value = world * tokens_per_step * args.steps / (e2e_total / 1e3)
+    e2e_value, _ = weak_scaling_value(world, tokens_per_step, args.steps, sum(e2e_ms))
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb))
     d2h = sum(ho[var].numel() * ho[var].element_size() + hs[var].numel() * hs[var].element_size()
               for var in w["variants"])

@@ -190,6 +190,16 @@ int falcon_fwd_masked_noalloc(falcon_variant variant, falcon_dtype dtype,
  */
 int falcon_device_wait_timeouts(unsigned int *count);
 
+/*
+ * falcon_selftest_bounded_wait -- checks on the current device that the
+ * bounded waits the tensor-core kernels use give up instead of hanging: one
+ * block waits on a barrier phase that nothing completes, gives up after
+ * `timeout_us` microseconds and exits normally.  Synchronises; writes
+ * *gave_up = 1 when the wait gave up as it must (0 would mean it saw a
+ * completion, -1 that the kernel did not run).
+ */
+int falcon_selftest_bounded_wait(unsigned int timeout_us, int *gave_up);
+
 /* Static description of a status code (never NULL). */
 const char *falcon_status_string(int status);
 

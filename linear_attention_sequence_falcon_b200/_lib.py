@@ -22,7 +22,8 @@ DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PAIRINGS = {"prefix": 0, "same_step": 1}
 PHIS = {"l2": 0, "identity": 1}
 EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_decode_step", "falcon_decode_carry_from_prefill",
-           "falcon_fwd_masked_noalloc", "falcon_status_string")
+           "falcon_fwd_masked_noalloc", "falcon_device_wait_timeouts", "falcon_selftest_bounded_wait",
+           "falcon_status_string")
 
 _lib = None
 
@@ -52,6 +53,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.falcon_fwd_masked_noalloc.restype = I
     lib.falcon_device_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     lib.falcon_device_wait_timeouts.restype = I
+    lib.falcon_selftest_bounded_wait.argtypes = [ctypes.c_uint, ctypes.POINTER(ctypes.c_int)]
+    lib.falcon_selftest_bounded_wait.restype = I
     lib.falcon_status_string.argtypes = [I]
     lib.falcon_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -121,6 +124,13 @@ def fwd_masked_noalloc(variant: str, q, k, v, beta, lam, eps: float, window: int
                                        _ptr(final_state), _stream(stream))
     _check(rc)
     return out, final_state
+
+
+def selftest_bounded_wait(timeout_us: int = 2000) -> int:
+    """Runs the on-device bounded-wait check; returns 1 when the wait gave up."""
+    r = ctypes.c_int(-1)
+    _check(load().falcon_selftest_bounded_wait(int(timeout_us), ctypes.byref(r)))
+    return int(r.value)
 
 
 def wait_timeouts() -> int:

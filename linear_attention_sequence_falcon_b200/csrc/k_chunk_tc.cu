@@ -107,11 +107,6 @@ __device__ __forceinline__ void unpack8(uint4 u, float *f) {
 }
 
 
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
 
 __device__ unsigned int g_tc_wait_timeouts;
 
@@ -150,13 +145,9 @@ __device__ long long *g_tim;
 #define TIMX(c, slot)
 #endif
 
-// Bounded wait on the MMA-completion barrier: about two seconds at most.
+// Bounded wait on an MMA-completion or TMA-arrival barrier: two seconds at most.
 __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer();
-    while (!tc::mbar_try_wait(bar, parity)) {
-        if (globaltimer() - t0 > 2000000000ull) return false;
-    }
-    return true;
+    return tc::mbar_wait_timeout(bar, parity, 2000000000ull);
 }
 
 // Tensor maps of q, k, v: 3-D [B*H][L][64] bf16, boxes of 64 x 64, 128-byte swizzle.

@@ -36,12 +36,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Waits for the phase with the given parity to complete; gives up after
-// `limit` polls (each poll may itself suspend briefly) and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
+// `timeout_ns` nanoseconds and returns false (the caller records the
+// failure and leaves, so no wait can hang the device).
+__device__ __forceinline__ bool mbar_wait_timeout(uint64_t *bar, uint32_t parity, uint64_t timeout_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > timeout_ns) return false;
+    }
+    return true;
 }
 
 // The calling thread arrives on `bar` and adds `bytes` to the transaction
