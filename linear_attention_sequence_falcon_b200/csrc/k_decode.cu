@@ -153,70 +153,81 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
 // held by LPR = min(8, DK/4) lanes, lane l owning float4 slots l, l+LPR, ...
 // (every load instruction reads LPR*16 contiguous bytes of a row), so a row's
 // dot products need only log2(LPR) shuffle steps; 1/(eps+n), beta and the
-// shared sample are staged once per block, never per row.
+// shared sample are staged once per block, never per row.  A block serves
+// HPB (n,h) pairs so that the whole grid is resident at once (one wave).
 template <typename T, int DK>
 __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
+    constexpr int HPB = 2;
     constexpr int LPR = DK >= 32 ? 8 : DK / 4;
     constexpr int NV4 = DK / (4 * LPR);  // float4 per lane per row
     constexpr int RPW = 32 / LPR;        // rows per warp per pass
     constexpr int NW = 8;
-    __shared__ __align__(16) float xs[DK];
-    __shared__ __align__(16) float qs[DK];
-    __shared__ float ks[DK];
-    __shared__ float ys[128];
-    __shared__ float bs[128];
-    __shared__ float red[3][NW];
+    __shared__ __align__(16) float xs[HPB][DK];
+    __shared__ __align__(16) float qs[HPB][DK];
+    __shared__ float ks[HPB][DK];
+    __shared__ float ys[HPB][128];
+    __shared__ float bs[HPB][128];
+    __shared__ float red[HPB][3][NW];
+    __shared__ float hsc[HPB][4];  // inv_den, xq, lambda, |k|^2
 
     const VariantInfo vi = variant_info(p.variant, 1);
-    const int nh = blockIdx.x, h = nh % p.H, dv = p.dv;
+    const int nh_total = p.N * p.H, dv = p.dv;
+    const int nh0 = blockIdx.x * HPB;
+    const int nheads = min(HPB, nh_total - nh0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
-    const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
-    const T *v = static_cast<const T *>(p.v) + (size_t)nh * dv;
-    const T *beta = static_cast<const T *>(p.beta) + (size_t)nh * (vi.per_channel ? dv : 1);
-    float *xp = p.x_prev + (size_t)nh * DK;
 
-    // stage the sample x = x_prev, q, k, v and beta; block sums of |x|^2, x.q, |k|^2
-    float px = 0.f, pq = 0.f, pk = 0.f;
-    for (int i = threadIdx.x; i < DK; i += blockDim.x) {
-        const float xv = xp[i], qv = to_f32(q[i]), kv = to_f32(k[i]);
-        xs[i] = xv;
-        qs[i] = qv;
-        ks[i] = kv;
-        px += xv * xv;
-        pq += xv * qv;
-        pk += kv * kv;
+    // stage each pair's sample x = x_prev, q, k, v and beta
+    for (int hh = 0; hh < nheads; ++hh) {
+        const int nh = nh0 + hh;
+        const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
+        const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
+        const T *v = static_cast<const T *>(p.v) + (size_t)nh * dv;
+        const T *beta = static_cast<const T *>(p.beta) + (size_t)nh * (vi.per_channel ? dv : 1);
+        const float *xp = p.x_prev + (size_t)nh * DK;
+        float px = 0.f, pq = 0.f, pk = 0.f;
+        for (int i = threadIdx.x; i < DK; i += blockDim.x) {
+            const float xv = xp[i], qv = to_f32(q[i]), kv = to_f32(k[i]);
+            xs[hh][i] = xv;
+            qs[hh][i] = qv;
+            ks[hh][i] = kv;
+            px += xv * xv;
+            pq += xv * qv;
+            pk += kv * kv;
+        }
+        for (int i = threadIdx.x; i < dv; i += blockDim.x) {
+            ys[hh][i] = to_f32(v[i]);
+            bs[hh][i] = to_f32(beta[vi.per_channel ? i : 0]);
+        }
+        px = group_sum<32>(px);
+        pq = group_sum<32>(pq);
+        pk = group_sum<32>(pk);
+        if (lane == 0) { red[hh][0][warp] = px; red[hh][1][warp] = pq; red[hh][2][warp] = pk; }
     }
-    for (int i = threadIdx.x; i < dv; i += blockDim.x) {
-        ys[i] = to_f32(v[i]);
-        bs[i] = to_f32(beta[vi.per_channel ? i : 0]);
-    }
-    px = group_sum<32>(px);
-    pq = group_sum<32>(pq);
-    pk = group_sum<32>(pk);
-    if (lane == 0) { red[0][warp] = px; red[1][warp] = pq; red[2][warp] = pk; }
     __syncthreads();
-    float n = 0.f, xq = 0.f, knorm = 0.f;
+    if (threadIdx.x < nheads) {
+        const int hh = threadIdx.x;
+        float n = 0.f, xq = 0.f, knorm = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) { n += red[0][w]; xq += red[1][w]; knorm += red[2][w]; }
-    const float inv_den = n > 0.f ? 1.f / (p.eps + n) : 0.f;  // eta = beta * inv_den
-    const float lam = p.lambda[h];
+        for (int w = 0; w < NW; ++w) { n += red[hh][0][w]; xq += red[hh][1][w]; knorm += red[hh][2][w]; }
+        hsc[hh][0] = n > 0.f ? 1.f / (p.eps + n) : 0.f;  // eta = beta * inv_den
+        hsc[hh][1] = xq;
+        hsc[hh][2] = p.lambda[(nh0 + hh) % p.H];
+        hsc[hh][3] = knorm;
+    }
+    __syncthreads();
 
     const int sl = lane % LPR, rsub = warp * RPW + lane / LPR;
-    float4 xr[NV4], qr[NV4];
-#pragma unroll
-    for (int i = 0; i < NV4; ++i) {
-        xr[i] = *reinterpret_cast<const float4 *>(&xs[4 * (sl + LPR * i)]);
-        qr[i] = *reinterpret_cast<const float4 *>(&qs[4 * (sl + LPR * i)]);
-    }
-    float *S = p.state + (size_t)nh * dv * DK;
-    T *out = static_cast<T *>(p.out) + (size_t)nh * dv;
-
-    for (int row = rsub; row < dv; row += NW * RPW) {
-        float4 s4[NV4];
-        float4 *Srow = reinterpret_cast<float4 *>(S + (size_t)row * DK);
+    for (int r = rsub; r < nheads * dv; r += NW * RPW) {
+        const int hh = r / dv, row = r - hh * dv;  // uniform across a row's lanes
+        float4 xr[NV4], qr[NV4], s4[NV4];
+        float4 *Srow = reinterpret_cast<float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
 #pragma unroll
         for (int i = 0; i < NV4; ++i) s4[i] = Srow[sl + LPR * i];
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) {
+            xr[i] = *reinterpret_cast<const float4 *>(&xs[hh][4 * (sl + LPR * i)]);
+            qr[i] = *reinterpret_cast<const float4 *>(&qs[hh][4 * (sl + LPR * i)]);
+        }
         float sq = 0.f, sx = 0.f;
 #pragma unroll
         for (int i = 0; i < NV4; ++i) {
@@ -225,24 +236,29 @@ __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
         }
         sq = group_sum<LPR>(sq);
         if (vi.regression) sx = group_sum<LPR>(sx);
-        const float eta = bs[row] * inv_den;
-        const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
-        const float e = vi.regression ? ys[row] - sx : ys[row];
+        const float eta = bs[hh][row] * hsc[hh][0];
+        const float alpha = fmaxf(1.f - eta * hsc[hh][2], kAlphaFloor);
+        const float e = vi.regression ? ys[hh][row] - sx : ys[hh][row];
         const float ge = eta * e;
 #pragma unroll
         for (int i = 0; i < NV4; ++i) {
-            float4 r;
-            r.x = alpha * s4[i].x + ge * xr[i].x;
-            r.y = alpha * s4[i].y + ge * xr[i].y;
-            r.z = alpha * s4[i].z + ge * xr[i].z;
-            r.w = alpha * s4[i].w + ge * xr[i].w;
-            Srow[sl + LPR * i] = r;
+            float4 o;
+            o.x = alpha * s4[i].x + ge * xr[i].x;
+            o.y = alpha * s4[i].y + ge * xr[i].y;
+            o.z = alpha * s4[i].z + ge * xr[i].z;
+            o.w = alpha * s4[i].w + ge * xr[i].w;
+            Srow[sl + LPR * i] = o;
         }
-        if (sl == 0) out[row] = from_f32<T>(alpha * sq + ge * xq);
+        if (sl == 0)
+            static_cast<T *>(p.out)[(size_t)(nh0 + hh) * dv + row] = from_f32<T>(alpha * sq + ge * hsc[hh][1]);
     }
     // carry: x_prev <- phi(k_t)
-    const float kinv = knorm > 0.f ? rsqrtf(knorm) : 0.f;
-    for (int i = threadIdx.x; i < DK; i += blockDim.x) xp[i] = ks[i] * kinv;
+    for (int hh = 0; hh < nheads; ++hh) {
+        const float kn = hsc[hh][3];
+        const float kinv = kn > 0.f ? rsqrtf(kn) : 0.f;
+        float *xp = p.x_prev + (size_t)(nh0 + hh) * DK;
+        for (int i = threadIdx.x; i < DK; i += blockDim.x) xp[i] = ks[hh][i] * kinv;
+    }
 }
 
 template <typename T, int DK>
@@ -277,7 +293,7 @@ __global__ void __launch_bounds__(128) carry_kernel(CarryParams p) {
 template <typename T, int DK>
 static void launch_decode_dk(const DecodeParams &p, cudaStream_t s) {
     if (variant_info(p.variant, p.window).window == 1)
-        decode1_kernel<T, DK><<<p.N * p.H, 256, 0, s>>>(p);
+        decode1_kernel<T, DK><<<(p.N * p.H + 1) / 2, 256, 0, s>>>(p);
     else
         decode_kernel<T, DK><<<p.N * p.H, 256, 0, s>>>(p);
 }

@@ -244,3 +244,13 @@ def test_decode_workload5_shape(F):
     oo, oS = oracle_fwd(d, "F2A", 1)
     assert rel(outs, oo[:, :, 40:]) <= 2e-2
     assert rel(S, oS) <= 2e-2
+
+
+@pytest.mark.parametrize("variant", ["F1", "F2A"])
+@pytest.mark.parametrize("dk,dv", [(16, 32), (32, 16), (128, 64)])
+def test_decode_odd_pair_count(F, variant, dk, dv):
+    """An odd number of (n, h) pairs leaves the last decode block one pair short."""
+    d, outs, S = _decode_chain(F, variant, 3, 3, dk, dv, 20, 5, "f32", 1)
+    oo, oS = oracle_fwd(d, variant, 1)
+    assert rel(outs, oo[:, :, 20:]) <= 1e-4
+    assert rel(S, oS) <= 1e-4
