@@ -94,9 +94,13 @@ enum {
  *   out      [B,H,L,d_v] dtype     o_t = S_t q_t (written)
  *   final_state [B,H,d_v,d_k] fp32 S_L (written), may be NULL
  * S_0 = 0.  L may be 0 (out untouched, final_state zeroed) and need not be a
- * multiple of `chunk`.  FALCON_MASKED draws stream-ordered scratch
- * (cudaMallocAsync/cudaFreeAsync on `stream`, about B*H*L*(window*d_v+2*d_v)
- * floats) and returns FALCON_ERR_ALLOC if that fails.
+ * multiple of `chunk`.  Two paths draw stream-ordered scratch on `stream`
+ * from a memory pool the library owns (one per device, kept mapped between
+ * calls; see falcon_scratch_trim) and return FALCON_ERR_ALLOC if that fails:
+ * FALCON_MASKED (about B*H*L*(window*d_v+2*d_v) floats) and the bf16
+ * tensor-core chunk path, Falcon-1/1A with d_k = d_v = 64 and chunk 64
+ * (32 KiB + 4 bytes per (b, h, chunk): the chunk-local results that the
+ * second of its two kernels chains across chunks).
  */
 int falcon_fwd(falcon_variant variant, falcon_form form, falcon_dtype dtype,
                const void *q, const void *k, const void *v, const void *beta,
@@ -154,8 +158,8 @@ int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_dtype dtype,
  * this entry point exists for callers that may not allocate device memory:
  * a host that owns every device allocation and gives a plug-in only its
  * input and output buffers, or a service running under a fixed, pre-planned
- * memory budget.  falcon_fwd's masked form draws its scratch with
- * cudaMallocAsync; this one uses a fixed array of
+ * memory budget.  falcon_fwd's masked form draws its scratch from
+ * a stream-ordered pool; this one uses a fixed array of
  * FALCON_NOALLOC_SCRATCH_BYTES inside the library instead, which every GPU
  * that loads the library holds until the process exits.  Arguments, layouts
  * and results are those of falcon_fwd with form = FALCON_MASKED.
@@ -199,6 +203,14 @@ int falcon_device_wait_timeouts(unsigned int *count);
  * completion, -1 that the kernel did not run).
  */
 int falcon_selftest_bounded_wait(unsigned int timeout_us, int *gave_up);
+
+/*
+ * falcon_scratch_trim -- returns the unused memory of the current device's
+ * scratch pool (see falcon_fwd) to the driver.  Scratch still in use by
+ * enqueued work is kept.  The pool grows again on the next call that needs
+ * scratch.  Returns FALCON_OK, or FALCON_ERR_LAUNCH if the CUDA call fails.
+ */
+int falcon_scratch_trim(void);
 
 /* Static description of a status code (never NULL). */
 const char *falcon_status_string(int status);

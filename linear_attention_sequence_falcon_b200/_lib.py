@@ -23,7 +23,7 @@ PAIRINGS = {"prefix": 0, "same_step": 1}
 PHIS = {"l2": 0, "identity": 1}
 EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_decode_step", "falcon_decode_carry_from_prefill",
            "falcon_fwd_masked_noalloc", "falcon_device_wait_timeouts", "falcon_selftest_bounded_wait",
-           "falcon_status_string")
+           "falcon_scratch_trim", "falcon_status_string")
 
 _lib = None
 
@@ -55,6 +55,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.falcon_device_wait_timeouts.restype = I
     lib.falcon_selftest_bounded_wait.argtypes = [ctypes.c_uint, ctypes.POINTER(ctypes.c_int)]
     lib.falcon_selftest_bounded_wait.restype = I
+    lib.falcon_scratch_trim.argtypes = []
+    lib.falcon_scratch_trim.restype = I
     lib.falcon_status_string.argtypes = [I]
     lib.falcon_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -131,6 +133,11 @@ def selftest_bounded_wait(timeout_us: int = 2000) -> int:
     r = ctypes.c_int(-1)
     _check(load().falcon_selftest_bounded_wait(int(timeout_us), ctypes.byref(r)))
     return int(r.value)
+
+
+def scratch_trim() -> None:
+    """Return the unused memory of the current device's scratch pool."""
+    _check(load().falcon_scratch_trim())
 
 
 def wait_timeouts() -> int:

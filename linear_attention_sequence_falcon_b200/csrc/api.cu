@@ -62,15 +62,15 @@ extern "C" int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dt
         return launched(bf16 ? launch_recurrent<__nv_bfloat16>(p, stream) : launch_recurrent<float>(p, stream));
     if (form == FALCON_CHUNK) {
         if (bf16) {
-            const int tc = launch_tc_chunk(p, stream);
-            if (tc != 1) return launched(tc);  // 1: shape not covered by the tensor-core kernel
+            const int tc = launch_split_chunk(p, stream);
+            if (tc != 1) return launched(tc);  // 1: shape not covered by the tensor-core kernels
         }
         return launched(bf16 ? launch_span_chunk<__nv_bfloat16>(p, stream) : launch_span_chunk<float>(p, stream));
     }
     // masked-parallel: scratch for the solved unknowns, the steps and Gamma
     const size_t nr = masked_ws_r_floats(p), neg = masked_ws_eg_floats(p);
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, sizeof(float) * (nr + 2 * neg), stream) != cudaSuccess) {
+    if (scratch_alloc(&ws, sizeof(float) * (nr + 2 * neg), stream) != cudaSuccess) {
         cudaGetLastError();
         return FALCON_ERR_ALLOC;
     }
@@ -78,7 +78,7 @@ extern "C" int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dt
     p.ws_eta = p.ws_r + nr;
     p.ws_gam = p.ws_eta + neg;
     rc = launched(bf16 ? launch_span_masked<__nv_bfloat16>(p, stream) : launch_span_masked<float>(p, stream));
-    cudaFreeAsync(ws, stream);
+    scratch_free(ws, stream);
     return rc;
 }
 
@@ -132,8 +132,12 @@ extern "C" int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_d
 
 extern "C" int falcon_device_wait_timeouts(unsigned int *count) {
     if (!count) return FALCON_ERR_NULL;
-    *count = tc_wait_timeouts();
+    *count = tc_wait_timeouts() + split_wait_timeouts();
     return cudaGetLastError() == cudaSuccess ? FALCON_OK : FALCON_ERR_LAUNCH;
+}
+
+extern "C" int falcon_scratch_trim(void) {
+    return scratch_trim() == cudaSuccess ? FALCON_OK : FALCON_ERR_LAUNCH;
 }
 
 extern "C" const char *falcon_status_string(int status) {

@@ -43,8 +43,20 @@ template <typename T> int launch_span_masked(const FwdParams &p, cudaStream_t s)
 int launch_tc_chunk(const FwdParams &p, cudaStream_t s);
 // Number of tensor-core chunk kernels that gave up on a bounded wait.
 unsigned int tc_wait_timeouts();
+// The same forward as two kernels (every chunk's local part at once, then
+// the per-head chain) over a stream-ordered workspace; returns 1 for shapes
+// it does not cover, FALCON_ERR_ALLOC when the workspace cannot be had.
+int launch_split_chunk(const FwdParams &p, cudaStream_t s);
+size_t split_chunk_ws_bytes(const FwdParams &p);
+unsigned int split_wait_timeouts();
 template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
+
+// Stream-ordered scratch from the library's per-device pool (kept mapped
+// between calls); scratch_trim hands the pool's unused memory back.
+cudaError_t scratch_alloc(void **ptr, size_t bytes, cudaStream_t s);
+cudaError_t scratch_free(void *ptr, cudaStream_t s);
+cudaError_t scratch_trim();
 
 // Scratch sizes (floats) of the masked-parallel form.
 size_t masked_ws_r_floats(const FwdParams &p);

@@ -44,8 +44,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Waits for the phase with the given parity to complete; gives up after
 // `timeout_ns` nanoseconds and returns false (the caller records the
-// failure and leaves, so no wait can hang the device).
+// failure and leaves, so no wait can hang the device).  The timer is read
+// only once the first poll has failed: it is slow to read, and most waits
+// find their phase already complete.
 __device__ __forceinline__ bool mbar_wait_timeout(uint64_t *bar, uint32_t parity, uint64_t timeout_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (globaltimer_ns() - t0 > timeout_ns) return false;
@@ -71,6 +74,36 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int 
         "[%5];" ::"r"(dst),
         "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Untiled bulk copy global -> this CTA's shared memory (no multicast),
+// completing on `bar`; both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Untiled bulk copy shared -> global in the calling thread's bulk group.
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Wait until every committed bulk store of this thread has read its source
+// (the shared memory may then be reused; the global writes may still be in flight).
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Plain arrive (count 1) on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Barrier over `nthreads` threads (a multiple of 32) with hardware id `id` (1-15).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Pull a tensor map (kernel parameter) into the descriptor cache.
@@ -193,6 +226,27 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      smem_u32(bar))
+                 : "memory");
+}
+
+// ---------------------------------------------------------------- 8x8 b16 matrix moves
+
+// Four 8x8 b16 matrices, transposed on the way in: lanes 8m..8m+7 give the
+// row addresses of matrix m; thread t receives, for matrix m, the elements
+// (rows 2(t%4), 2(t%4)+1; column t/4) packed in r[m].
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+// Four 8x8 b16 matrices stored row-wise: lanes 8m..8m+7 give the row
+// addresses of matrix m; thread t supplies, for matrix m, row t/4, columns
+// 2(t%4), 2(t%4)+1 packed in r[m].
+__device__ __forceinline__ void stsm_x4(uint32_t addr, const uint32_t (&r)[4]) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
                  : "memory");
 }
 
