@@ -44,7 +44,14 @@ def _stale(target, deps):
 
 def build(force: bool = False, verbose: bool = False) -> str:
     deps = _deps()
-    if not force and not _stale(LIB, deps + [os.path.abspath(__file__)]):
+    # the library is also stale when the set of sources changed (one removed)
+    manifest = os.path.join(BUILD, "sources.txt")
+    listing = "\n".join(os.path.basename(x) for x in _sources())
+    try:
+        same_sources = open(manifest).read() == listing
+    except OSError:
+        same_sources = False
+    if not force and same_sources and not _stale(LIB, deps + [os.path.abspath(__file__)]):
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     headers = [d for d in deps if not d.endswith(".cu")]
@@ -68,6 +75,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = LIB + ".tmp%d" % os.getpid()
     run([NVCC] + ARCH + ["-shared", "-o", tmp] + objs)
     os.replace(tmp, LIB)
+    with open(manifest, "w") as fh:
+        fh.write(listing)
     return LIB
 
 

@@ -132,7 +132,7 @@ extern "C" int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_d
 
 extern "C" int falcon_device_wait_timeouts(unsigned int *count) {
     if (!count) return FALCON_ERR_NULL;
-    *count = tc_wait_timeouts() + split_wait_timeouts();
+    *count = split_wait_timeouts();
     return cudaGetLastError() == cudaSuccess ? FALCON_OK : FALCON_ERR_LAUNCH;
 }
 

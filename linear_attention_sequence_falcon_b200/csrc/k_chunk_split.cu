@@ -367,14 +367,9 @@ __global__ void __launch_bounds__(NTH1, 2)
             ss += __shfl_xor_sync(0xffffffffu, ss, 1);
             ss += __shfl_xor_sync(0xffffffffu, ss, 2);
             const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
-            float sq = 0.f;
+            const float sq = ss * inv * inv;  // |x_t|^2: 1 up to rounding, 0 for an empty sample
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                xr[e] *= inv;
-                sq += xr[e] * xr[e];
-            }
-            sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-            sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+            for (int e = 0; e < 16; ++e) xr[e] *= inv;
 #pragma unroll
             for (int c16 = 0; c16 < 2; ++c16)
                 *reinterpret_cast<uint4 *>(sm + oX + tc::sw128(r, part * 2 + c16)) = pack8(&xr[c16 * 8]);
@@ -526,15 +521,17 @@ __global__ void __launch_bounds__(NTH1, 2)
             float tcol[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const float *mr = Mf + (b0 + i) * LDF + b0;
-                float acc0 = (i == j) ? 1.f : 0.f, acc1 = 0.f;
+                // row i of the diagonal block, four float4 loads (broadcast across the lanes)
+                float mr[16];
 #pragma unroll
-                for (int s = 0; s + 1 < i; s += 2) {
-                    acc0 -= mr[s] * tcol[s];
-                    acc1 -= mr[s + 1] * tcol[s + 1];
+                for (int q = 0; q < 4; ++q) {
+                    const float4 m4 = *reinterpret_cast<const float4 *>(Mf + (b0 + i) * LDF + b0 + q * 4);
+                    mr[q * 4] = m4.x; mr[q * 4 + 1] = m4.y; mr[q * 4 + 2] = m4.z; mr[q * 4 + 3] = m4.w;
                 }
-                if (i & 1) acc0 -= mr[i - 1] * tcol[i - 1];
-                tcol[i] = acc0 + acc1;
+                float acc[4] = {(i == j) ? 1.f : 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int s = 0; s < i; ++s) acc[s & 3] -= mr[s] * tcol[s];
+                tcol[i] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
             __syncwarp(0x0000ffffu);  // every lane has read the block before any writes it
 #pragma unroll

@@ -38,16 +38,14 @@ struct CarryParams {
 template <typename T> int launch_recurrent(const FwdParams &p, cudaStream_t s);
 template <typename T> int launch_span_chunk(const FwdParams &p, cudaStream_t s);
 template <typename T> int launch_span_masked(const FwdParams &p, cudaStream_t s);
-// bf16 chunk-parallel forward on tcgen05; returns 1 (nothing launched) for
-// shapes it does not cover, so the caller falls back to the span kernel.
-int launch_tc_chunk(const FwdParams &p, cudaStream_t s);
-// Number of tensor-core chunk kernels that gave up on a bounded wait.
-unsigned int tc_wait_timeouts();
-// The same forward as two kernels (every chunk's local part at once, then
-// the per-head chain) over a stream-ordered workspace; returns 1 for shapes
-// it does not cover, FALCON_ERR_ALLOC when the workspace cannot be had.
+// bf16 chunk-parallel forward on tcgen05 as two kernels (every chunk's local
+// part at once, then the per-head chain) over a stream-ordered workspace;
+// returns 1 (nothing launched) for shapes it does not cover, so the caller
+// falls back to the span kernel, and FALCON_ERR_ALLOC when the workspace
+// cannot be had.
 int launch_split_chunk(const FwdParams &p, cudaStream_t s);
 size_t split_chunk_ws_bytes(const FwdParams &p);
+// Number of tensor-core thread blocks that gave up on a bounded wait.
 unsigned int split_wait_timeouts();
 template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
