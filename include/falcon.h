@@ -188,7 +188,8 @@ int falcon_fwd_masked_noalloc(falcon_variant variant, falcon_dtype dtype,
  * falcon_device_wait_timeouts -- diagnostic: how many thread blocks of the
  * tensor-core kernels on the current device gave up on a bounded wait for
  * their own tensor-core work (about 2 s per wait) since the library was
- * loaded.  A block that gives up skips its remaining chunks, frees its tensor
+ * loaded (each wait gives up after 4e9 SM cycles, 2-4 s).  A block that
+ * gives up skips its remaining chunks, frees its tensor
  * memory and exits, so the device stays usable; its outputs are then
  * incomplete.  Synchronises with the device.  Returns 0 and writes *count.
  */
@@ -198,7 +199,8 @@ int falcon_device_wait_timeouts(unsigned int *count);
  * falcon_selftest_bounded_wait -- checks on the current device that the
  * bounded waits the tensor-core kernels use give up instead of hanging: one
  * block waits on a barrier phase that nothing completes, gives up after
- * `timeout_us` microseconds and exits normally.  Synchronises; writes
+ * 2 * `timeout_us` thousand SM cycles (between 1 and 2 times `timeout_us`
+ * microseconds at SM clocks of 1-2 GHz) and exits normally.  Synchronises; writes
  * *gave_up = 1 when the wait gave up as it must (0 would mean it saw a
  * completion, -1 that the kernel did not run).
  */

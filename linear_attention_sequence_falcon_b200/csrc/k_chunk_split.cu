@@ -96,9 +96,9 @@ constexpr int NSA = 3;     // bf16 [S ; S] operand buffers (chunk index mod 3), 
 constexpr uint32_t S_SA = NST * IMG;
 constexpr uint32_t S_GC = S_SA + NSA * 2 * TILE;  // g_C per stage
 constexpr uint32_t S_BAR = S_GC + 64;
-constexpr uint32_t S_SMEM = S_BAR + 128 + 1024;
-// chain tensor memory: -S Phi' (64 columns), then O^T - O0^T in two buffers
-constexpr uint32_t C_DS = 0, C_O = 64;
+constexpr uint32_t S_SMEM = S_BAR + 256 + 1024;
+// chain tensor memory: two accumulators of 128 columns (chunk parity), each
+// [-S Phi' | O^T - O0^T] (the inner-product family uses the second half only)
 
 __device__ unsigned int g_split_wait_timeouts;
 
@@ -716,6 +716,8 @@ __global__ void __launch_bounds__(NTH1, 2)
     beta_raw = beta_next;
     lam_raw = lam_next;
     }  // units
+    // the chain kernel may be scheduled once every block has got this far
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (tid == 0) {
         tc::bulk_wait_read();  // the last images have been read out of shared memory
@@ -737,13 +739,13 @@ __global__ void __launch_bounds__(NTH1, 2)
 // One block per b*H + h.  Warps 0,1,4,5 (tensor-memory lanes 0-63) carry the
 // state, fp32 in registers (thread: row j, 32 of its columns); warps 2,3,6,7
 // (lanes 64-127) finish the outputs; warp 8 streams the images; warp 9
-// issues the products: for chunk c, -S_c Phi'_c (the only product on the
-// chain, committed on its own) and then the output product Qt_{c-1}
-// S_{c-1}^T of the previous chunk, which so runs while the state warps
-// compute S_{c+1}.  S_c sits in operand buffer c mod 3; the state warps
-// write S_{c+1} over S_{c-2} only after the -S Phi' completion of chunk c,
-// and that commit covers every earlier product of the issuing thread, the
-// output product of chunk c-2 included.
+// issues the products.  S_c sits, as a bf16 [S;S] operand, in buffer c mod 3.
+// Regression family: one product per chunk, [S;S] [-Phi'^T;Qt]^T into
+// accumulator c & 1, then the state warps form S_{c+1} in fp32, write its
+// copy and release the issuer through a named barrier.  Inner-product family:
+// no product is on the chain (S_{c+1} = g_C S_c + B_c); the state warps run
+// up to three chunks ahead, and each output product Qt_c S_c^T waits for its
+// S_c copy (sready) and frees its buffer on completion (sfree).
 namespace {
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
@@ -764,10 +766,11 @@ __global__ void __launch_bounds__(NTH2, 1)
     float *gcs = reinterpret_cast<float *>(sm + S_GC);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + S_BAR);  // [NST] image landed
     uint64_t *empty = full + NST;                                // [NST] image consumed (8 warps)
-    uint64_t *mma_s = empty + NST;                               // -S Phi' of the chunk done
-    uint64_t *mma_o = mma_s + 1;                                 // [2] Qt S^T done
+    uint64_t *mma_o = empty + NST;                               // [2] the chunk's product done
     uint64_t *accfree = mma_o + 2;                               // [2] outputs read (4 warps)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accfree + 2);
+    uint64_t *sready = accfree + 2;                              // [NSA] S copy written (inner product)
+    uint64_t *sfree = sready + NSA;                              // [NSA] S copy read (inner product)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfree + NSA);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -783,10 +786,13 @@ __global__ void __launch_bounds__(NTH2, 1)
             tc::mbar_init(&full[s], 1);
             tc::mbar_init(&empty[s], 8);
         }
-        tc::mbar_init(mma_s, 1);
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&mma_o[b], 1);
             tc::mbar_init(&accfree[b], 4);
+        }
+        for (int b = 0; b < NSA; ++b) {
+            tc::mbar_init(&sready[b], 128);
+            tc::mbar_init(&sfree[b], 1);
         }
         *abort_flag = 0;
         tc::fence_mbar_init();
@@ -804,6 +810,9 @@ __global__ void __launch_bounds__(NTH2, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = *tmem_slot;
+    // launched as a programmatic dependent of the local kernel: the set-up
+    // above overlaps its tail; its images are read only after it completed
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == 8) {
         // ---- producer: chunk images into NST stages
@@ -825,31 +834,50 @@ __global__ void __launch_bounds__(NTH2, 1)
         }
     } else if (warp == 9) {
         // ---- issuer
-        auto issue_out = [&](int co) {  // Qt S^T of chunk co into output buffer co & 1
+        auto issue_out = [&](int co) {  // Qt S^T of chunk co (inner product) into accumulator co & 1
             const uint32_t stage = sbase + (co % NST) * IMG, sa = sbase + S_SA + (uint32_t)(co % NSA) * 2 * TILE;
             bool go = true;
             if (co >= 2) go = wait_or_abort(&accfree[co & 1], ((co / 2) - 1) & 1, abort_flag);
-            if (go) issue_gemm(tbase + C_O + (co & 1) * 64, sa, stage + TILE, 64, false);
+            if (go) issue_gemm(tbase + (co & 1) * 128 + 64, sa, stage + TILE, 64, false);
             tc::mma_commit(&mma_o[co & 1]);
         };
-        for (int c = 0; c < nch; ++c) {
-            const int s = c % NST;
-            const uint32_t stage = sbase + s * IMG, sa = sbase + S_SA + (uint32_t)(c % NSA) * 2 * TILE;
-            bool go = true;
-            if (lane == 0) go = wait_or_abort(&full[s], (c / NST) & 1, abort_flag);
-            __syncwarp();
-            tc::named_sync(1, 160);  // S_c is in operand buffer c mod 3
-            if (lane == 0) {
+        if (reg) {
+            // one product per chunk: [S;S] [-Phi'^T ; Qt]^T -> [-S Phi' | O^T - O0^T]
+            for (int c = 0; c < nch; ++c) {
+                const int s = c % NST, b = c & 1;
+                const uint32_t stage = sbase + s * IMG, sa = sbase + S_SA + (uint32_t)(c % NSA) * 2 * TILE;
+                bool go = true;
+                if (lane == 0) {
+                    go = wait_or_abort(&full[s], (c / NST) & 1, abort_flag);
+                    if (go && c >= 2) go = wait_or_abort(&accfree[b], ((c / 2) - 1) & 1, abort_flag);
+                }
+                __syncwarp();
+                tc::named_sync(1, 160);  // S_c is in operand buffer c mod 3
+                if (lane == 0) {
+                    CTIM(c, 0);
+                    tc::fence_after_sync();
+                    if (go) issue_gemm(tbase + b * 128, sa, stage, 128, false);
+                    tc::mma_commit(&mma_o[b]);
+                    CTIM(c, 9);
+                }
+                __syncwarp();
+            }
+        } else if (lane == 0) {
+            // inner-product family: nothing on the chain is a product; the
+            // state warps run ahead and each output product waits for its S_c
+            for (int c = 0; c < nch; ++c) {
+                CTIM(c, 14);
+                bool go = wait_or_abort(&full[c % NST], (c / NST) & 1, abort_flag);
+                CTIM(c, 15);
+                if (go && c > 0) go = wait_or_abort(&sready[c % NSA], ((c - 1) / NSA) & 1, abort_flag);
                 CTIM(c, 0);
                 tc::fence_after_sync();
-                if (go && reg) issue_gemm(tbase + C_DS, sa, stage, 64, false);  // -S Phi'
-                tc::mma_commit(mma_s);
-                CTIM(c, 9);
-                if (c > 0) issue_out(c - 1);
+                issue_out(c);
+                tc::mma_commit(&sfree[c % NSA]);
+                CTIM(c, 13);
             }
-            __syncwarp();
         }
-        if (lane == 0 && nch > 0) issue_out(nch - 1);
+
         __syncwarp();
     } else {
         const int quarter = warp & 3, chalf = warp >> 2;
@@ -862,7 +890,7 @@ __global__ void __launch_bounds__(NTH2, 1)
             float S[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] = 0.f;
-            tc::named_sync(1, 160);  // S_0 is in operand buffer 0
+            if (reg) tc::named_sync(1, 160);  // S_0 is in operand buffer 0
             for (int c = 0; c < nch; ++c) {
                 const int s = c % NST;
                 const uint8_t *st = sm + s * IMG;
@@ -874,24 +902,27 @@ __global__ void __launch_bounds__(NTH2, 1)
                     unpack8(*reinterpret_cast<const uint4 *>(st + 3 * TILE + rowmajor8(j, chalf * 4 + g8)),
                             &bv[g8 * 8]);
                 const float g = gcs[s];
-                (void)wait_or_abort(mma_s, c & 1, abort_flag);
-                if (tid == 0) CTIM(c, 1);
-                tc::fence_after_sync();
                 if (reg) {
+                    (void)wait_or_abort(&mma_o[c & 1], (c / 2) & 1, abort_flag);
+                    if (tid == 0) CTIM(c, 1);
+                    tc::fence_after_sync();
                     float ds[32];
-                    tc::tmem_ld32(tl + C_DS + chalf * 32, ds);
+                    tc::tmem_ld32(tl + (c & 1) * 128 + chalf * 32, ds);
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) S[i] = g * S[i] + ds[i] + bv[i];
+                    tc::fence_before_sync();
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) S[i] = g * S[i] + bv[i];
                 }
-                tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&empty[s]);
                 if (c + 1 < nch) {
-                    // bf16 copy of S_{c+1} into both halves of operand buffer (c+1) mod 3
+                    // bf16 copy of S_{c+1} into both halves of operand buffer (c+1) mod 3,
+                    // over S_{c-2}: regression - covered by the -S Phi' commit of chunk c;
+                    // inner product - once the output product of chunk c-2 has read it
+                    if (!reg && c >= 2) (void)wait_or_abort(&sfree[(c + 1) % NSA], ((c - 2) / NSA) & 1, abort_flag);
                     uint8_t *sa = sm + S_SA + ((c + 1) % NSA) * 2 * TILE;
 #pragma unroll
                     for (int g8 = 0; g8 < 4; ++g8) {
@@ -901,7 +932,12 @@ __global__ void __launch_bounds__(NTH2, 1)
                     }
                     tc::fence_proxy_async();
                     if (tid == 0) CTIM(c, 2);
-                    tc::named_sync(1, 160);
+                    if (reg) {
+                        tc::named_sync(1, 160);
+                    } else {
+                        tc::fence_before_sync();
+                        tc::mbar_arrive(&sready[(c + 1) % NSA]);
+                    }
                 }
             }
             if (p.final_state && !*(volatile int *)abort_flag) {
@@ -926,7 +962,7 @@ __global__ void __launch_bounds__(NTH2, 1)
                 if (tid == 64) CTIM(c, 4);
                 tc::fence_after_sync();
                 float ov[32];
-                tc::tmem_ld32(tl + C_O + b * 64 + chalf * 32, ov);
+                tc::tmem_ld32(tl + b * 128 + 64 + chalf * 32, ov);
                 tc::tmem_wait_ld();
                 tc::fence_before_sync();
                 __syncwarp();
@@ -1023,10 +1059,29 @@ int launch_split_chunk(const FwdParams &p, cudaStream_t s) {
     }
     uint8_t *img = static_cast<uint8_t *>(ws);
     float *gc = reinterpret_cast<float *>(img + units * IMG);
-    cudaFuncSetAttribute(chunk_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L_SMEM);
-    cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_SMEM);
+    static bool attrs_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attrs_set[dev]) {
+        cudaFuncSetAttribute(chunk_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L_SMEM);
+        cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_SMEM);
+        if (dev >= 0 && dev < 64) attrs_set[dev] = true;
+    }
     chunk_local_kernel<<<(unsigned)std::min<size_t>(units, (size_t)2 * sm_count()), NTH1, L_SMEM, s>>>(p, maps, img, gc);
-    chunk_chain_kernel<<<BH, NTH2, S_SMEM, s>>>(p, img, gc);
+    // the chain kernel as a programmatic dependent launch (see griddepcontrol in both kernels)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(BH);
+    cfg.blockDim = dim3(NTH2);
+    cfg.dynamicSmemBytes = S_SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const uint8_t *cimg = img;
+    const float *cgc = gc;
+    cudaLaunchKernelEx(&cfg, chunk_chain_kernel, p, cimg, cgc);
     const cudaError_t e = cudaGetLastError();
     scratch_free(ws, s);
     return e == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH

@@ -44,14 +44,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Waits for the phase with the given parity to complete; gives up after
 // `timeout_ns` nanoseconds and returns false (the caller records the
-// failure and leaves, so no wait can hang the device).  The timer is read
-// only once the first poll has failed: it is slow to read, and most waits
-// find their phase already complete.
+// failure and leaves, so no wait can hang the device).  The bound is counted
+// in SM cycles at 2 cycles per nanosecond: the cycle counter is cheap to read
+// while the global timer is not, and at any SM clock between 1 and 2 GHz
+// the wait gives up between 1 and 2 times `timeout_ns`.
 __device__ __forceinline__ bool mbar_wait_timeout(uint64_t *bar, uint32_t parity, uint64_t timeout_ns) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const long long t0 = clock64();
+    const long long limit = (long long)(2 * timeout_ns);
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > timeout_ns) return false;
+        if (clock64() - t0 > limit) return false;
     }
     return true;
 }
