@@ -445,6 +445,45 @@ def measure_decode(F, gen, stream, flush, hbm, args, profile=False):
                          "algorithmic_bytes_per_launch": ab, "traffic": profiled_traffic("decode")}}
 
 
+def run_workloads(args):
+    """--workloads: one JSON line per (workload, variant, form) of the
+    workloads table (inputs.WORKLOADS): CUDA events around one falcon_fwd,
+    after a warm-up call, L2 flushed before each timed call; median of
+    --steps calls (at least 3, at most 20).  Not the contract line."""
+    import torch
+    import linear_attention_sequence_falcon_b200 as F
+    from linear_attention_sequence_falcon_b200 import build, inputs as gen
+    build.build()
+    F.load()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    cases = []
+    for n, w in gen.WORKLOADS.items():
+        forms = list(w["forms"])
+        if n == 2:
+            forms = ["chunk", "masked", "recurrent"]
+        for var in w["variants"]:
+            for form in forms:
+                cases.append((n, w, var, form))
+    for n, w, var, form in cases:
+        d = gen.workload_inputs(n, var)
+        args_ = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
+        out, S = F.fwd(var, form, *args_, d["eps"], window=w["window"], chunk=w["chunk"])
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(max(3, min(args.steps, 20))):
+            flush.zero_()
+            torch.cuda._sleep(HEAD_START_CYCLES)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            F.fwd(var, form, *args_, d["eps"], window=w["window"], chunk=w["chunk"], out=out, final_state=S)
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        t = statistics.median(ms)
+        print(json.dumps({"workload": n, "name": w["name"], "variant": var, "form": form, "dtype": w["dtype"],
+                          "ms": t, "tokens_per_s": w["B"] * w["L"] / (t / 1e3)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -456,10 +495,14 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--profile-decode", action="store_true",
                     help="run only warmup+steps decode steps (no flush or JSON), for ncu")
+    ap.add_argument("--workloads", action="store_true",
+                    help="time every workload and form of the workloads table, one JSON line each")
     ap.add_argument("--profile", action="store_true",
                     help="run only warmup+steps device steps (no flush, e2e, clocks or JSON), for ncu")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.workloads:
+        run_workloads(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
