@@ -263,9 +263,9 @@ __global__ void __launch_bounds__(NTH1, 2)
     const uint32_t sbase = tc::smem_u32(sm);
     float *Mf = reinterpret_cast<float *>(sm + L_MF);  // M, then T in place
     float *vec = reinterpret_cast<float *>(sm + L_VEC);
-    float *v_sqn = vec, *v_eta = vec + 64, *v_G = vec + 128, *v_gm1 = vec + 192, *v_gt = vec + 256,
-          *v_w = vec + 320, *v_beta = vec + 384, *v_a = vec + 448, *v_b = vec + 512, *v_c = vec + 576,
-          *v_sc = vec + 640;  // v_sc: lambda, factorised-decay flag
+    float *v_la = vec, *v_eta = vec + 64, *v_G = vec + 128, *v_gm1 = vec + 192, *v_gt = vec + 256,
+          *v_w = vec + 320, *v_lsc = vec + 384, *v_a = vec + 448, *v_b = vec + 512, *v_c = vec + 576,
+          *v_sc = vec + 640;  // v_sc[1]: factorised-decay flag; v_sc[8..15]: per-warp log-decay sums
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L_BAR);        // MMA completion
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L_BAR + 8);
     uint64_t *tbar = reinterpret_cast<uint64_t *>(sm + L_BAR + 16);  // [2] TMA arrival per input set
@@ -297,8 +297,11 @@ __global__ void __launch_bounds__(NTH1, 2)
         lraw = 0.f;
         if (u >= units) return;
         const int ubh = u / nch, uc0 = (u - ubh * nch) * CH;
-        if (tid < 64 && uc0 + tid < L) braw = static_cast<const __nv_bfloat16 *>(p.beta)[(size_t)ubh * L + uc0 + tid];
-        if (tid == 64) lraw = p.lambda[ubh % p.H];
+        // token t = tid / 4 on the first of the four threads of sample row t
+        if ((tid & 3) == 0) {
+            if (uc0 + (tid >> 2) < L) braw = static_cast<const __nv_bfloat16 *>(p.beta)[(size_t)ubh * L + uc0 + (tid >> 2)];
+            lraw = p.lambda[ubh % p.H];
+        }
     };
 
     int loads0 = 0, loads1 = 0;  // loads issued into each input set (thread 0)
@@ -353,7 +356,9 @@ __global__ void __launch_bounds__(NTH1, 2)
     if (!ok) break;
     LTIM(2);
     {
-        // ---- samples x_t = phi(k_{t-1}) in place: four threads per row t
+        // ---- samples x_t = phi(k_{t-1}) in place (four threads per row t), the
+        //      steps and log decays of the rows, and their cumulative sums
+        //      inside each warp (eight rows per warp)
         {
             const int r = tid >> 2, part = tid & 3;
             float xr[16];
@@ -373,61 +378,59 @@ __global__ void __launch_bounds__(NTH1, 2)
 #pragma unroll
             for (int c16 = 0; c16 < 2; ++c16)
                 *reinterpret_cast<uint4 *>(sm + oX + tc::sw128(r, part * 2 + c16)) = pack8(&xr[c16 * 8]);
-            if (part == 0) v_sqn[r] = sq;
-            if (tid < 64) v_beta[tid] = __bfloat162float(beta_raw);
-            if (tid == 64) v_sc[0] = lam_raw;
+            // eta = beta / (eps + n) (0 for an empty sample), alpha = max(1 - eta lambda, 2^-20)
+            const float beta_r = __shfl_sync(0xffffffffu, __bfloat162float(beta_raw), lane & ~3);
+            const float lam = __shfl_sync(0xffffffffu, lam_raw, lane & ~3);
+            const float eta = sq > 0.f ? __fdividef(beta_r, p.eps + sq) : 0.f;
+            const float la = __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
+            float run = la;  // inclusive sum over this warp's rows (lanes 4k hold row 8w+k)
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, run, o);
+                if (lane >= o) run += y;
+            }
+            if (part == 0) {
+                v_la[r] = la;
+                v_lsc[r] = run;
+                v_eta[r] = eta;
+            }
+            if (lane == 28) v_sc[8 + warp] = run;
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
         LTIM(3);
-        // ---- G1 [X;Q] X^T -> A (lanes 0-63), P (lanes 64-127), while the steps are computed
+        // ---- G1 [X;Q] X^T -> A (lanes 0-63), P (lanes 64-127), while the decays are formed
         if (tid == ISSUER1) {
             tc::fence_after_sync();
             issue_gemm(tbase + C_G1, sbase + oX, sbase + oX, 64, false);
             tc::mma_commit(bar);
         }
         __syncwarp();
-        if (warp == 0) {
-            // ---- steps, log decays and their chunk-local cumulative sums
-            //      (tokens 2l and 2l+1 on lane l)
-            const int t0 = 2 * lane;
-            // eta = beta / (eps + n) (0 for an empty sample), alpha = max(1 - eta lambda, 2^-20)
-            const float n0 = v_sqn[t0], n1 = v_sqn[t0 + 1];
-            const float eta0 = n0 > 0.f ? __fdividef(v_beta[t0], p.eps + n0) : 0.f;
-            const float eta1 = n1 > 0.f ? __fdividef(v_beta[t0 + 1], p.eps + n1) : 0.f;
-            const float lam = v_sc[0];
-            const float al0 = fmaxf(1.f - eta0 * lam, kAlphaFloor), al1 = fmaxf(1.f - eta1 * lam, kAlphaFloor);
-            const float la0 = __logf(al0), la1 = __logf(al1);
-            float run = la0 + la1;
-            LTIM(16);
+        if (tid < 64) {
+            // ---- token t: cumulative log decay G_t and the decay vectors
+            const int t = tid;
+            const float4 wa = *reinterpret_cast<const float4 *>(v_sc + 8);
+            const float4 wb = *reinterpret_cast<const float4 *>(v_sc + 12);
+            const float wt[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            float off = 0.f, GC = 0.f;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, run, o);
-                if (lane >= o) run += y;
+            for (int w = 0; w < 8; ++w) {
+                if (w < (t >> 3)) off += wt[w];
+                GC += wt[w];
             }
-            LTIM(17);
-            const float G1v = run, G0v = run - la1, Gm = run - la0 - la1;  // G_{t0+1}, G_{t0}, G_{t0-1}
-            const float GC = __shfl_sync(0xffffffffu, run, 31);
-            const float Gr = __shfl_sync(0xffffffffu, run, 15);  // G_31, the factorisation's reference
-            v_eta[t0] = eta0;
-            v_eta[t0 + 1] = eta1;
-            v_G[t0] = G0v;
-            v_G[t0 + 1] = G1v;
-            v_gm1[t0] = __expf(Gm);
-            v_gm1[t0 + 1] = __expf(G0v);
-            v_gt[t0] = __expf(G0v);
-            v_gt[t0 + 1] = __expf(G1v);
-            v_w[t0] = __expf(GC - G0v) * eta0;
-            v_w[t0 + 1] = __expf(GC - G1v) * eta1;
+            const float Gr = v_lsc[31] + (wt[0] + wt[1] + wt[2]);  // G_31, the factorisation's reference
+            const float Gt = v_lsc[t] + off, Gm = Gt - v_la[t];    // G_t, G_{t-1}
+            const float eta = v_eta[t];
+            v_G[t] = Gt;
+            v_gm1[t] = __expf(Gm);
+            v_gt[t] = __expf(Gt);
+            v_w[t] = __expf(GC - Gt) * eta;
             // e^{G_{t-1} - G_s} = a_t b_s / eta_s and e^{G_t - G_s} = c_t b_s / eta_s
-            v_a[t0] = __expf(Gm - Gr);
-            v_a[t0 + 1] = __expf(G0v - Gr);
-            v_c[t0] = __expf(G0v - Gr);
-            v_c[t0 + 1] = __expf(G1v - Gr);
-            v_b[t0] = eta0 * __expf(Gr - G0v);
-            v_b[t0 + 1] = eta1 * __expf(Gr - G1v);
-            if (lane == 31) {
+            v_a[t] = __expf(Gm - Gr);
+            v_c[t] = __expf(Gt - Gr);
+            v_b[t] = eta * __expf(Gr - Gt);
+            if (t == 0) {
                 gc_ws[u] = __expf(GC);
                 v_sc[1] = GC > kFactorMinLogDecay ? 1.f : 0.f;
             }
@@ -439,19 +442,19 @@ __global__ void __launch_bounds__(NTH1, 2)
             transpose4(sbase + oV, rb + 1, 0, sbase + L_XT, nullptr, 0, nullptr);
             transpose4(sbase + oV, rb + 1, 4, sbase + L_XT, nullptr, 0, nullptr);
         }
-        __syncthreads();
+        LTIM(16);
+        ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        phase ^= 1;
+        ok = __syncthreads_and(ok);
         LTIM(4);
+    }
+    if (ok) {
+        tc::fence_after_sync();
         // ---- (D_w X)^T -> A3 rows 64-127 and (D_a X)^T -> XT rows 64-127
         //      (regression), source row block = warp
         transpose4(sbase + oX, warp, 0, sbase + L_A3 + TILE, v_w, reg ? sbase + L_XT + TILE : 0, v_gm1);
         transpose4(sbase + oX, warp, 4, sbase + L_A3 + TILE, v_w, reg ? sbase + L_XT + TILE : 0, v_gm1);
-        ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
-        phase ^= 1;
-        ok = __syncthreads_and(ok);
         LTIM(5);
-    }
-    if (ok) {
-        tc::fence_after_sync();
         // rows 0-63: M[t][s] = (g_{t-1}/g_s) eta_s A[t][s] for s < t (fp32, regression only);
         // rows 64-127: (P o Dm)[t][s] = (g_t/g_s) eta_s P[t][s] for s <= t (bf16).
         const bool mrow = quarter < 2;
@@ -834,13 +837,6 @@ __global__ void __launch_bounds__(NTH2, 1)
         }
     } else if (warp == 9) {
         // ---- issuer
-        auto issue_out = [&](int co) {  // Qt S^T of chunk co (inner product) into accumulator co & 1
-            const uint32_t stage = sbase + (co % NST) * IMG, sa = sbase + S_SA + (uint32_t)(co % NSA) * 2 * TILE;
-            bool go = true;
-            if (co >= 2) go = wait_or_abort(&accfree[co & 1], ((co / 2) - 1) & 1, abort_flag);
-            if (go) issue_gemm(tbase + (co & 1) * 128 + 64, sa, stage + TILE, 64, false);
-            tc::mma_commit(&mma_o[co & 1]);
-        };
         if (reg) {
             // one product per chunk: [S;S] [-Phi'^T ; Qt]^T -> [-S Phi' | O^T - O0^T]
             for (int c = 0; c < nch; ++c) {
@@ -866,19 +862,18 @@ __global__ void __launch_bounds__(NTH2, 1)
             // inner-product family: nothing on the chain is a product; the
             // state warps run ahead and each output product waits for its S_c
             for (int c = 0; c < nch; ++c) {
-                CTIM(c, 14);
+                const int b = c & 1;
+                const uint32_t stage = sbase + (c % NST) * IMG, sa = sbase + S_SA + (uint32_t)(c % NSA) * 2 * TILE;
                 bool go = wait_or_abort(&full[c % NST], (c / NST) & 1, abort_flag);
-                CTIM(c, 15);
                 if (go && c > 0) go = wait_or_abort(&sready[c % NSA], ((c - 1) / NSA) & 1, abort_flag);
+                if (go && c >= 2) go = wait_or_abort(&accfree[b], ((c / 2) - 1) & 1, abort_flag);
                 CTIM(c, 0);
                 tc::fence_after_sync();
-                issue_out(c);
+                if (go) issue_gemm(tbase + b * 128 + 64, sa, stage + TILE, 64, false);
+                tc::mma_commit(&mma_o[b]);
                 tc::mma_commit(&sfree[c % NSA]);
-                CTIM(c, 13);
             }
         }
-
-        __syncwarp();
     } else {
         const int quarter = warp & 3, chalf = warp >> 2;
         const bool state_warp = quarter < 2;
