@@ -57,6 +57,8 @@ def _load():
         lib.oracle_decode_step.restype = I
         lib.oracle_carry_from_prefill.argtypes = [I, I, dp, dp, I, I, I, I, I, I, dp, dp]
         lib.oracle_carry_from_prefill.restype = I
+        lib.oracle_fwd_carry.argtypes = [I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, I, dp, dp, dp, dp, dp, I]
+        lib.oracle_fwd_carry.restype = I
         _lib = lib
     return _lib
 
@@ -124,3 +126,27 @@ def carry_from_prefill(variant, k, v, window, phi="l2"):
     if rc < 0:
         raise ValueError("oracle_carry_from_prefill rejected its arguments (code %d)" % rc)
     return x_prev, win
+
+
+def fwd_carry(variant, q, k, v, beta, lam, eps, window=1, S0=None, x_prev=None, win=None, phi="l2",
+              nthreads=0):
+    """Recurrent definition over a segment that continues a sequence: state
+    S0 [B,H,dv,dk] and the decode carry x_prev [B,H,dk], win [B,H,Bw-1,dk+dv]
+    (each None = zeros, the start of a sequence).  Prefix pairing.
+    Returns (out [B,H,L,dv], S_L [B,H,dv,dk])."""
+    lib = _load()
+    q, k, v, beta, lam = map(_f64, (q, k, v, beta, lam))
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    null = ctypes.POINTER(ctypes.c_double)()
+    carry = [_f64(a) if a is not None else None for a in (S0, x_prev, win)]
+    if carry[2] is not None and carry[2].size == 0:
+        carry[2] = None
+    ptrs = [_p(a) if a is not None else null for a in carry]
+    out = np.zeros((B, H, L, dv))
+    fs = np.zeros((B, H, dv, dk))
+    rc = lib.oracle_fwd_carry(VARIANTS[variant], PHIS[phi], _p(q), _p(k), _p(v), _p(beta), _p(lam),
+                              float(eps), int(window), B, H, L, dk, dv, *ptrs, _p(out), _p(fs), int(nthreads))
+    if rc < 0:
+        raise ValueError("oracle_fwd_carry rejected its arguments (code %d)" % rc)
+    return out, fs

@@ -37,8 +37,13 @@ def _samples(k, pairing, phi):
     return x
 
 
-def unit(variant, q, k, v, beta, lam, eps, window=1, pairing="prefix", phi="l2"):
+def unit(variant, q, k, v, beta, lam, eps, window=1, pairing="prefix", phi="l2", S0=None, x_prev=None,
+         carry=None):
     """One (b,h) unit: q,k [L,dk], v [L,dv], beta [L] or [L,dv], lam scalar.
+    A segment continuing a sequence starts from S0 [dv,dk] with x_1 = x_prev
+    [dk] (prefix pair) and, for Falcon-3/3A, the earlier samples `carry`
+    [Bw-1, dk+dv] (x then y, oldest first): then
+        S_t = S0 M_1 ... M_t + sum_s b_s M_{s+1} ... M_t.
     Returns (out [L,dv], S_L [dv,dk])."""
     q, k, v, beta = (np.asarray(a, dtype=np.float64) for a in (q, k, v, beta))
     L, dk = q.shape
@@ -46,7 +51,18 @@ def unit(variant, q, k, v, beta, lam, eps, window=1, pairing="prefix", phi="l2")
     reg = variant in ("F1", "F2", "F3")
     w = window if variant in ("F3", "F3A") else 1
     x = _samples(k, pairing, phi)
-    win = [list(range(max(0, t - w + 1), t + 1)) for t in range(L)]
+    if x_prev is not None:
+        x[0] = np.asarray(x_prev, dtype=np.float64)
+    # samples before the segment: index -m is row P - m of the carry (P = w - 1)
+    P = w - 1
+    xc = np.zeros((P, dk))
+    yc = np.zeros((P, dv))
+    if carry is not None and P > 0:
+        carry = np.asarray(carry, dtype=np.float64)
+        xc, yc = carry[:, :dk], carry[:, dk:]
+    x = np.concatenate([xc, x])
+    v = np.concatenate([yc, v])
+    win = [list(range(t - w + 1 + P, t + 1 + P)) for t in range(L)]
     energy = np.array([sum(float(x[i] @ x[i]) for i in win[t]) for t in range(L)])
     b2 = beta.reshape(L, -1)
     eta = np.where(energy[:, None] > 0, b2 / (eps + energy[:, None]), 0.0)
@@ -61,11 +77,15 @@ def unit(variant, q, k, v, beta, lam, eps, window=1, pairing="prefix", phi="l2")
     def bvec(s, j):
         return eta[s, j] * sum(v[i, j] * x[i] for i in win[s])
 
+    S0 = np.zeros((dv, dk)) if S0 is None else np.asarray(S0, dtype=np.float64)
     out = np.zeros((L, dv))
     S = np.zeros((dv, dk))
     for j in range(dv):
         for t in range(L):
-            row = np.zeros(dk)
+            P0 = eye.copy()
+            for r in range(t + 1):
+                P0 = P0 @ M(r, j)
+            row = S0[j] @ P0
             for s in range(t + 1):
                 P = eye.copy()
                 for r in range(s + 1, t + 1):

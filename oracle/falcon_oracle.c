@@ -363,6 +363,125 @@ int oracle_fwd(int variant, int form, int pairing, int phi,
 }
 
 /* ------------------------------------------------------------------ */
+/* Recurrent form continuing an earlier segment (initial state + carry). */
+/* ------------------------------------------------------------------ */
+
+/*
+ * A segment that continues a sequence: the state starts at S0 (zeros when
+ * NULL) and the samples before the segment are the decode carry (the same
+ * layout as oracle_decode_step): x_prev = phi(k) of the token before the
+ * segment, which is x_1 of the segment under the prefix pair, and for
+ * Falcon-3/3A the Bw-1 samples before it, win[m] = (x, y), oldest first.
+ * NULL carries are zeros, which is exactly the start of a sequence (R2: an
+ * all-zero sample adds no energy and no gradient).  The definition is the
+ * recurrent form above, run over the carried samples followed by the
+ * segment's; prefix pairing only.
+ */
+typedef struct {
+    int variant, phi, B, H, L, dk, dv, w;
+    double eps;
+    const double *q, *k, *v, *beta, *lambda, *S0, *x_prev, *win;
+    double *out, *final_state;
+} carry_job_t;
+
+static void carry_unit_run(const carry_job_t *C, int b, int h)
+{
+    const int L = C->L, dk = C->dk, dv = C->dv, w = C->w, P = w - 1;
+    const int nch = is_per_channel(C->variant) ? dv : 1;
+    const size_t bh = (size_t)b * C->H + h;
+    const double *k = C->k + bh * (size_t)L * dk, *v = C->v + bh * (size_t)L * dv;
+    const double *q = C->q + bh * (size_t)L * dk, *beta = C->beta + bh * (size_t)L * nch;
+    /* samples at positions -P .. L-1 (index i + P) */
+    double *X = (double *)calloc((size_t)(L + P) * dk, sizeof(double));
+    double *Y = (double *)calloc((size_t)(L + P) * dv, sizeof(double));
+    for (int m = 0; m < P && C->win; ++m) {
+        const double *wm = C->win + (bh * (size_t)P + m) * (size_t)(dk + dv);
+        memcpy(X + (size_t)m * dk, wm, sizeof(double) * dk);
+        memcpy(Y + (size_t)m * dv, wm + dk, sizeof(double) * dv);
+    }
+    for (int t = 0; t < L; ++t) {
+        double *xt = X + (size_t)(t + P) * dk;
+        if (t == 0) {
+            if (C->x_prev) memcpy(xt, C->x_prev + bh * (size_t)dk, sizeof(double) * dk);
+        } else {
+            apply_phi(C->phi, k + (size_t)(t - 1) * dk, dk, xt);
+        }
+        memcpy(Y + (size_t)(t + P) * dv, v + (size_t)t * dv, sizeof(double) * dv);
+    }
+    double *S = (double *)calloc((size_t)dv * dk, sizeof(double));
+    if (C->S0) memcpy(S, C->S0 + bh * (size_t)dv * dk, sizeof(double) * (size_t)dv * dk);
+    double *res = (double *)calloc((size_t)w * dv, sizeof(double));
+    double *out = C->out + bh * (size_t)L * dv;
+    const double lam = C->lambda[h];
+    for (int t = 0; t < L; ++t) {
+        /* window t-w+1 .. t, all present among the carried samples */
+        double n = 0.0;
+        for (int i = t - w + 1; i <= t; ++i) n += dot(X + (size_t)(i + P) * dk, X + (size_t)(i + P) * dk, dk);
+        for (int i = t - w + 1; i <= t; ++i) {
+            const double *xi = X + (size_t)(i + P) * dk, *yi = Y + (size_t)(i + P) * dv;
+            for (int j = 0; j < dv; ++j)
+                res[(size_t)(i - (t - w + 1)) * dv + j] =
+                    is_regression(C->variant) ? yi[j] - dot(S + (size_t)j * dk, xi, dk) : yi[j];
+        }
+        for (int j = 0; j < dv; ++j) {
+            const int ch = nch > 1 ? j : 0;
+            const double eta = n > 0.0 ? beta[(size_t)t * nch + ch] / (C->eps + n) : 0.0;
+            double a = 1.0 - eta * lam;
+            if (a < ALPHA_FLOOR) a = ALPHA_FLOOR;
+            double *Sj = S + (size_t)j * dk;
+            for (int c = 0; c < dk; ++c) {
+                double g = 0.0;
+                for (int i = t - w + 1; i <= t; ++i)
+                    g += res[(size_t)(i - (t - w + 1)) * dv + j] * X[(size_t)(i + P) * dk + c];
+                Sj[c] = a * Sj[c] + eta * g;
+            }
+        }
+        for (int j = 0; j < dv; ++j) out[(size_t)t * dv + j] = dot(S + (size_t)j * dk, q + (size_t)t * dk, dk);
+    }
+    if (C->final_state) memcpy(C->final_state + bh * (size_t)dv * dk, S, sizeof(double) * (size_t)dv * dk);
+    free(X); free(Y); free(S); free(res);
+}
+
+typedef struct {
+    const carry_job_t *C;
+    int tid, nthreads;
+} carry_worker_t;
+
+static void *carry_worker(void *arg)
+{
+    const carry_worker_t *W = (const carry_worker_t *)arg;
+    const int units = W->C->B * W->C->H;
+    for (int n = W->tid; n < units; n += W->nthreads) carry_unit_run(W->C, n / W->C->H, n % W->C->H);
+    return NULL;
+}
+
+/* Returns the number of threads used (>0) or a negative error. */
+int oracle_fwd_carry(int variant, int phi, const double *q, const double *k, const double *v, const double *beta,
+                     const double *lambda, double eps, int window, int B, int H, int L, int dk, int dv,
+                     const double *S0, const double *x_prev, const double *win,
+                     double *out, double *final_state, int nthreads)
+{
+    if (variant < 0 || variant > 5) return -2;
+    if (B < 0 || H < 0 || L < 0 || dk <= 0 || dv <= 0) return -3;
+    if (is_window(variant) && window < 1) return -6;
+    carry_job_t C = {variant, phi, B, H, L, dk, dv, is_window(variant) ? window : 1, eps,
+                     q, k, v, beta, lambda, S0, x_prev, win, out, final_state};
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    const int units = B * H;
+    if (nthreads > units) nthreads = units > 0 ? units : 1;
+    if (nthreads < 1) nthreads = 1;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
+    carry_worker_t *ws = (carry_worker_t *)malloc(sizeof(carry_worker_t) * nthreads);
+    for (int i = 0; i < nthreads; ++i) {
+        ws[i].C = &C; ws[i].tid = i; ws[i].nthreads = nthreads;
+        pthread_create(&th[i], NULL, carry_worker, &ws[i]);
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th); free(ws);
+    return nthreads;
+}
+
+/* ------------------------------------------------------------------ */
 /* Single-token recurrent step with its carry (decode).                 */
 /* ------------------------------------------------------------------ */
 

@@ -390,3 +390,67 @@ def test_edge_cases(oracle_mod):
         b = np.repeat(beta[..., None], 3, -1) if var in ("F2", "F2A") else beta
         o, S = oracle_mod.fwd(var, "recurrent", q, k, v, b, lam, 1e-6, window=wnd(var))
         assert np.all(o == 0) and np.all(S == 0)
+
+
+# ---------------------------------------------------------------- segments continuing a sequence
+
+def _carry_inputs(seed, B, H, dk, dv, variant):
+    rng = np.random.default_rng(seed)
+    S0 = rng.standard_normal((B, H, dv, dk)) * 0.5
+    xp = rng.standard_normal((B, H, dk))
+    xp /= np.linalg.norm(xp, axis=-1, keepdims=True)
+    w = wnd(variant)
+    win = rng.standard_normal((B, H, w - 1, dk + dv))
+    win[..., :dk] /= np.linalg.norm(win[..., :dk], axis=-1, keepdims=True)
+    return S0, xp, (win if w > 1 else None)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_carry_brute_force(oracle_mod, variant):
+    """A segment entered with state S0 and the samples before it: the oracle's
+    recurrence == the unrolled products S_t = S0 M_1...M_t + sum_s b_s
+    M_{s+1}...M_t of the same per-step updates ([EXPL] 核心方法 1)."""
+    L, dk, dv = 9, 4, 3
+    q, k, v, beta, lam = rnd(21, 1, 2, L, dk, dv, variant, lam_hi=0.3)
+    S0, xp, win = _carry_inputs(22, 1, 2, dk, dv, variant)
+    w = wnd(variant)
+    o, S = oracle_mod.fwd_carry(variant, q, k, v, beta, lam, 1e-6, window=w, S0=S0, x_prev=xp, win=win)
+    assert np.abs(o).max() > 1e-2
+    for h in range(2):
+        bo, bS = brute.unit(variant, q[0, h], k[0, h], v[0, h], beta[0, h], float(lam[h]), 1e-6, w,
+                            S0=S0[0, h], x_prev=xp[0, h], carry=None if win is None else win[0, h])
+        np.testing.assert_allclose(o[0, h], bo, rtol=1e-9, atol=1e-10)
+        np.testing.assert_allclose(S[0, h], bS, rtol=1e-9, atol=1e-10)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_carry_of_zeros_is_a_fresh_sequence(oracle_mod, variant):
+    """Zero state and zero carry are the start of a sequence (x_1 = 0 and
+    empty window samples add no energy and no gradient)."""
+    q, k, v, beta, lam = rnd(23, 2, 2, 30, 8, 4, variant)
+    w = wnd(variant)
+    o0, S0_ = oracle_mod.fwd(variant, "recurrent", q, k, v, beta, lam, 1e-6, window=w)
+    o1, S1 = oracle_mod.fwd_carry(variant, q, k, v, beta, lam, 1e-6, window=w)
+    np.testing.assert_allclose(o1, o0, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S1, S0_, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("split", [1, 17, 40])
+def test_continuation_equals_one_run(oracle_mod, variant, split):
+    """Running a sequence in two segments -- the second one entered with the
+    first one's final state and decode carry -- equals one run over the whole
+    sequence (chunk form for the whole run, recurrent for the segments)."""
+    L, dk, dv = 57, 8, 4
+    q, k, v, beta, lam = rnd(24, 2, 3, L, dk, dv, variant)
+    w = 3 if variant in ("F3", "F3A") else 1
+    o_all, S_all = oracle_mod.fwd(variant, "chunk", q, k, v, beta, lam, 1e-6, window=w, chunk=16)
+    a = slice(0, split)
+    b_ = slice(split, L)
+    o1, S1 = oracle_mod.fwd(variant, "recurrent", q[:, :, a], k[:, :, a], v[:, :, a], beta[:, :, a], lam,
+                            1e-6, window=w)
+    xp, win = oracle_mod.carry_from_prefill(variant, k[:, :, a], v[:, :, a], w)
+    o2, S2 = oracle_mod.fwd_carry(variant, q[:, :, b_], k[:, :, b_], v[:, :, b_], beta[:, :, b_], lam, 1e-6,
+                                  window=w, S0=S1, x_prev=xp, win=win)
+    np.testing.assert_allclose(np.concatenate([o1, o2], 2), o_all, rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(S2, S_all, rtol=1e-9, atol=1e-11)
