@@ -117,6 +117,35 @@ int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype,
                   void *out, float *final_state, cudaStream_t stream);
 
 /*
+ * falcon_fwd_carry -- falcon_fwd over a segment that continues a sequence:
+ * the recurrence picks up where an earlier segment (or a run of decode
+ * steps) left off.  Chunks already hand a fixed-size state from one to the
+ * next ([EXPL] 核心方法 3; [NEWS] 02 (2)); a segment boundary is the same
+ * hand-off, plus the samples that straddle it.
+ *
+ *   initial_state [B,H,d_v,d_k] fp32, or NULL: S_0 of the segment (zeros)
+ *   x_prev        [B,H,d_k] fp32, or NULL: phi(k) of the token before the
+ *                 segment, i.e. x_1 of the segment under the prefix pair
+ *                 (zeros: the start of a sequence)
+ *   win           [B,H,window-1,d_k+d_v] fp32, Falcon-3/3A, or NULL: the
+ *                 window-1 samples (x_i, y_i) before the segment, oldest
+ *                 first (zeros where the sequence has fewer)
+ * The carry has exactly the layout of the decode carry, so the final state of
+ * one segment and falcon_decode_carry_from_prefill of its keys and values
+ * continue it (or decode_step's in/out buffers after decoding).  Every other
+ * argument is as in falcon_fwd; prefix pairing, L2 feature map.  Forms:
+ * FALCON_RECURRENT and FALCON_CHUNK; FALCON_MASKED with a non-NULL carry
+ * returns FALCON_ERR_UNSUPPORTED (with all three NULL this is falcon_fwd).
+ * With L = 0 the final state is initial_state (or zeros).
+ */
+int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtype,
+                     const void *q, const void *k, const void *v, const void *beta,
+                     const float *lambda, float eps, int window,
+                     int B, int H, int L, int d_k, int d_v, int chunk,
+                     const float *initial_state, const float *x_prev, const float *win,
+                     void *out, float *final_state, cudaStream_t stream);
+
+/*
  * falcon_decode_step -- one recurrent step for N independent sequences
  * ([EXPL] 核心方法 3: recurrent, O(d^2) per step, for inference).
  *

@@ -21,7 +21,7 @@ FORMS = {"recurrent": 0, "masked": 1, "chunk": 2}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PAIRINGS = {"prefix": 0, "same_step": 1}
 PHIS = {"l2": 0, "identity": 1}
-EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_decode_step", "falcon_decode_carry_from_prefill",
+EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_fwd_carry", "falcon_decode_step", "falcon_decode_carry_from_prefill",
            "falcon_fwd_masked_noalloc", "falcon_device_wait_timeouts", "falcon_selftest_bounded_wait",
            "falcon_scratch_trim", "falcon_status_string")
 
@@ -45,6 +45,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.falcon_fwd.restype = I
     lib.falcon_fwd_ex.argtypes = [I, I, I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, I, P, P, P]
     lib.falcon_fwd_ex.restype = I
+    lib.falcon_fwd_carry.argtypes = [I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, I, P, P, P, P, P, P]
+    lib.falcon_fwd_carry.restype = I
     lib.falcon_decode_step.argtypes = [I, I, P, P, P, P, P, F, I, I, I, I, I, P, P, P, P, P]
     lib.falcon_decode_step.restype = I
     lib.falcon_decode_carry_from_prefill.argtypes = [I, I, P, P, I, I, I, I, I, I, P, P, P]
@@ -86,9 +88,12 @@ def _stream(stream):
 
 def fwd(variant: str, form: str, q, k, v, beta, lam, eps: float, window: int = 1, chunk: int = 64,
         out=None, final_state=None, pairing: str = "prefix", phi: str = "l2", stream=None,
-        want_state: bool = True):
+        want_state: bool = True, initial_state=None, x_prev=None, win=None):
     """falcon_fwd_ex on CUDA tensors q,k [B,H,L,dk], v [B,H,L,dv], beta [B,H,L] or
-    [B,H,L,dv] (same dtype), lam [H] fp32.  Returns (out, final_state)."""
+    [B,H,L,dv] (same dtype), lam [H] fp32.  Returns (out, final_state).
+    With initial_state [B,H,dv,dk], x_prev [B,H,dk] or win [B,H,window-1,dk+dv]
+    (fp32; the decode carry) it is falcon_fwd_carry: a segment continuing a
+    sequence (prefix pairing, L2 feature map)."""
     lib = load()
     B, H, L, dk = q.shape
     dv = v.shape[-1]
@@ -100,9 +105,21 @@ def fwd(variant: str, form: str, q, k, v, beta, lam, eps: float, window: int = 1
         out = torch.empty((B, H, L, dv), dtype=q.dtype, device=q.device)
     if final_state is None and want_state:
         final_state = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
-    rc = lib.falcon_fwd_ex(VARIANTS[variant], FORMS[form], DTYPES[q.dtype], PAIRINGS[pairing], PHIS[phi],
-                           _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(lam), float(eps), int(window),
-                           B, H, L, dk, dv, int(chunk), _ptr(out), _ptr(final_state), _stream(stream))
+    carry = (initial_state, x_prev, win)
+    if any(c is not None for c in carry):
+        if pairing != "prefix" or phi != "l2":
+            raise FalconError("a continued segment uses the prefix pairing and the L2 feature map")
+        for c in carry:
+            if c is not None and (c.dtype != torch.float32 or not c.is_contiguous()):
+                raise FalconError("initial_state, x_prev and win must be contiguous fp32")
+        rc = lib.falcon_fwd_carry(VARIANTS[variant], FORMS[form], DTYPES[q.dtype],
+                                  _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(lam), float(eps), int(window),
+                                  B, H, L, dk, dv, int(chunk), *(_ptr(c) if c is not None else None for c in carry),
+                                  _ptr(out), _ptr(final_state), _stream(stream))
+    else:
+        rc = lib.falcon_fwd_ex(VARIANTS[variant], FORMS[form], DTYPES[q.dtype], PAIRINGS[pairing], PHIS[phi],
+                               _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(lam), float(eps), int(window),
+                               B, H, L, dk, dv, int(chunk), _ptr(out), _ptr(final_state), _stream(stream))
     _check(rc)
     return out, final_state
 

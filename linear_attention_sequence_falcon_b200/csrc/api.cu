@@ -29,12 +29,12 @@ int launched(int rc) {
 
 }  // namespace
 
-extern "C" int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype,
-                             falcon_pairing pairing, falcon_phi phi,
-                             const void *q, const void *k, const void *v, const void *beta,
-                             const float *lambda, float eps, int window,
-                             int B, int H, int L, int d_k, int d_v, int chunk,
-                             void *out, float *final_state, cudaStream_t stream) {
+namespace {
+
+int fwd_impl(falcon_variant variant, falcon_form form, falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
+             const void *q, const void *k, const void *v, const void *beta, const float *lambda, float eps,
+             int window, int B, int H, int L, int d_k, int d_v, int chunk, const float *init_state,
+             const float *x_prev, const float *win, void *out, float *final_state, cudaStream_t stream) {
     int rc = validate_common(variant, dtype, window);
     if (rc) return rc;
     if (form < FALCON_RECURRENT || form > FALCON_CHUNK) return FALCON_ERR_ENUM;
@@ -49,10 +49,18 @@ extern "C" int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dt
     p.B = B; p.H = H; p.L = L; p.dk = d_k; p.dv = d_v; p.chunk = chunk; p.eps = eps;
     p.q = q; p.k = k; p.v = v; p.beta = beta; p.lambda = lambda;
     p.out = out; p.final_state = final_state;
+    p.init_state = init_state; p.x_prev = x_prev; p.win = p.window > 1 ? win : nullptr;
+    const bool carry = init_state || x_prev || p.win;
+    if (carry && form == FALCON_MASKED) return FALCON_ERR_UNSUPPORTED;
     if ((size_t)B * H == 0) return FALCON_OK;
     if (L == 0) {
         if (!final_state) return FALCON_OK;
-        const cudaError_t e = cudaMemsetAsync(final_state, 0, sizeof(float) * (size_t)B * H * d_v * d_k, stream);
+        cudaError_t e;
+        if (init_state)
+            e = cudaMemcpyAsync(final_state, init_state, sizeof(float) * (size_t)B * H * d_v * d_k,
+                                cudaMemcpyDeviceToDevice, stream);
+        else
+            e = cudaMemsetAsync(final_state, 0, sizeof(float) * (size_t)B * H * d_v * d_k, stream);
         return e == cudaSuccess ? FALCON_OK : FALCON_ERR_LAUNCH;
     }
     if (!q || !k || !v || !beta || !lambda || !out) return FALCON_ERR_NULL;
@@ -80,6 +88,28 @@ extern "C" int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dt
     rc = launched(bf16 ? launch_span_masked<__nv_bfloat16>(p, stream) : launch_span_masked<float>(p, stream));
     scratch_free(ws, stream);
     return rc;
+}
+
+}  // namespace
+
+extern "C" int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype,
+                             falcon_pairing pairing, falcon_phi phi,
+                             const void *q, const void *k, const void *v, const void *beta,
+                             const float *lambda, float eps, int window,
+                             int B, int H, int L, int d_k, int d_v, int chunk,
+                             void *out, float *final_state, cudaStream_t stream) {
+    return fwd_impl(variant, form, dtype, pairing, phi, q, k, v, beta, lambda, eps, window, B, H, L, d_k, d_v,
+                    chunk, nullptr, nullptr, nullptr, out, final_state, stream);
+}
+
+extern "C" int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtype,
+                                const void *q, const void *k, const void *v, const void *beta,
+                                const float *lambda, float eps, int window,
+                                int B, int H, int L, int d_k, int d_v, int chunk,
+                                const float *initial_state, const float *x_prev, const float *win,
+                                void *out, float *final_state, cudaStream_t stream) {
+    return fwd_impl(variant, form, dtype, FALCON_PAIR_PREFIX, FALCON_PHI_L2, q, k, v, beta, lambda, eps, window,
+                    B, H, L, d_k, d_v, chunk, initial_state, x_prev, win, out, final_state, stream);
 }
 
 extern "C" int falcon_fwd(falcon_variant variant, falcon_form form, falcon_dtype dtype,

@@ -361,17 +361,25 @@ __global__ void __launch_bounds__(NTH1, 2)
         //      inside each warp (eight rows per warp)
         {
             const int r = tid >> 2, part = tid & 3;
+            // x of a continued segment's first token is the carried phi(k), as given
+            const bool carried = r == 0 && p.x_prev != nullptr && u % nch == 0;
             float xr[16];
             float ss = 0.f;
 #pragma unroll
             for (int c16 = 0; c16 < 2; ++c16) {
-                unpack8(*reinterpret_cast<const uint4 *>(sm + oX + tc::sw128(r, part * 2 + c16)), &xr[c16 * 8]);
+                if (carried) {
+                    const float *xp = p.x_prev + (size_t)(u / nch) * DD + part * 16 + c16 * 8;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) xr[c16 * 8 + e] = xp[e];
+                } else {
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + oX + tc::sw128(r, part * 2 + c16)), &xr[c16 * 8]);
+                }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) ss += xr[c16 * 8 + e] * xr[c16 * 8 + e];
             }
             ss += __shfl_xor_sync(0xffffffffu, ss, 1);
             ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-            const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+            const float inv = carried ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
             const float sq = ss * inv * inv;  // |x_t|^2: 1 up to rounding, 0 for an empty sample
 #pragma unroll
             for (int e = 0; e < 16; ++e) xr[e] *= inv;
@@ -805,10 +813,6 @@ __global__ void __launch_bounds__(NTH2, 1)
         tc::tmem_alloc(tmem_slot, 256);
         tc::tmem_relinquish();
     }
-    // S_0 = 0: both halves of operand buffer 0
-    for (int i = tid; i < (int)(2 * TILE / 16); i += NTH2)
-        reinterpret_cast<uint4 *>(sm + S_SA)[i] = make_uint4(0, 0, 0, 0);
-    tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -865,7 +869,7 @@ __global__ void __launch_bounds__(NTH2, 1)
                 const int b = c & 1;
                 const uint32_t stage = sbase + (c % NST) * IMG, sa = sbase + S_SA + (uint32_t)(c % NSA) * 2 * TILE;
                 bool go = wait_or_abort(&full[c % NST], (c / NST) & 1, abort_flag);
-                if (go && c > 0) go = wait_or_abort(&sready[c % NSA], ((c - 1) / NSA) & 1, abort_flag);
+                if (go) go = wait_or_abort(&sready[c % NSA], (c / NSA) & 1, abort_flag);
                 if (go && c >= 2) go = wait_or_abort(&accfree[b], ((c / 2) - 1) & 1, abort_flag);
                 CTIM(c, 0);
                 tc::fence_after_sync();
@@ -882,10 +886,30 @@ __global__ void __launch_bounds__(NTH2, 1)
         __nv_bfloat16 *ko = static_cast<__nv_bfloat16 *>(p.out) + (size_t)bh * L * DD;
 
         if (state_warp) {
+            // S_0: the carried state of a continued segment, else zeros; its
+            // bf16 copy goes to both halves of operand buffer 0
             float S[32];
+            if (p.init_state) {
+                const float *s0 = p.init_state + ((size_t)bh * DD + j) * DD + chalf * 32;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) S[i] = 0.f;
-            if (reg) tc::named_sync(1, 160);  // S_0 is in operand buffer 0
+                for (int i = 0; i < 32; ++i) S[i] = s0[i];
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) S[i] = 0.f;
+            }
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+                const uint4 u4 = pack8(&S[g8 * 8]);
+                *reinterpret_cast<uint4 *>(sm + S_SA + tc::sw128(j, chalf * 4 + g8)) = u4;
+                *reinterpret_cast<uint4 *>(sm + S_SA + TILE + tc::sw128(j, chalf * 4 + g8)) = u4;
+            }
+            tc::fence_proxy_async();
+            if (reg) {
+                tc::named_sync(1, 160);  // S_0 is in operand buffer 0
+            } else {
+                tc::fence_before_sync();
+                tc::mbar_arrive(&sready[0]);
+            }
             for (int c = 0; c < nch; ++c) {
                 const int s = c % NST;
                 const uint8_t *st = sm + s * IMG;

@@ -48,17 +48,32 @@ __global__ void __launch_bounds__(128) recurrent_kernel(FwdParams p) {
     const T *kb = static_cast<const T *>(p.beta) + (size_t)bh * L * (vi.per_channel ? p.dv : 1);
     T *ko = static_cast<T *>(p.out) + (size_t)bh * L * p.dv;
 
+    // S_0: the carried state of a continued segment, else zeros
     float S[EPT];
 #pragma unroll
-    for (int e = 0; e < EPT; ++e) S[e] = 0.f;
+    for (int e = 0; e < EPT; ++e)
+        S[e] = (p.init_state && row_ok) ? p.init_state[((size_t)bh * p.dv + row) * DK + sl * EPT + e] : 0.f;
 
     for (int t0 = 0; t0 < L; t0 += TT) {
         const int nt = min(TT, L - t0);
-        // halo: the HALO samples before t0 (zeros before the sequence start)
+        // halo: the HALO samples before t0 -- at the segment start the carried
+        // window (the last window-1 slots), zeros before it
         if (t0 == 0) {
-            for (int i = threadIdx.x; i < HALO * DK; i += blockDim.x) xs[i] = 0.f;
-            for (int i = threadIdx.x; i < HALO * RPC; i += blockDim.x) ys[i] = 0.f;
-            for (int i = threadIdx.x; i < HALO; i += blockDim.x) sqn[i] = 0.f;
+            const int P = vi.window - 1;
+            for (int i = threadIdx.x; i < HALO * DK; i += blockDim.x) {
+                const int slot = i / DK, m = slot - (HALO - P);  // carried sample m, oldest first
+                xs[i] = (p.win && m >= 0) ? p.win[((size_t)bh * P + m) * (DK + p.dv) + i % DK] : 0.f;
+            }
+            for (int i = threadIdx.x; i < HALO * RPC; i += blockDim.x) {
+                const int slot = i / RPC, m = slot - (HALO - P), j = row0 + i % RPC;
+                ys[i] = (p.win && m >= 0 && j < p.dv) ? p.win[((size_t)bh * P + m) * (DK + p.dv) + DK + j] : 0.f;
+            }
+            __syncthreads();
+            for (int i = threadIdx.x; i < HALO; i += blockDim.x) {
+                float e = 0.f;
+                for (int c = 0; c < DK; ++c) e += xs[i * DK + c] * xs[i * DK + c];
+                sqn[i] = e;
+            }
         } else {
             for (int i = threadIdx.x; i < HALO * DK; i += blockDim.x) xs[i] = xs[TT * DK + i];
             for (int i = threadIdx.x; i < HALO * RPC; i += blockDim.x) ys[i] = ys[TT * RPC + i];
@@ -69,6 +84,8 @@ __global__ void __launch_bounds__(128) recurrent_kernel(FwdParams p) {
         for (int r = warp; r < nt; r += 4) {
             const int t = t0 + r;
             const int ki = p.pairing == 0 ? t - 1 : t;
+            // x of a continued segment's first token is the carried phi(k), as given
+            const bool carried = ki < 0 && p.x_prev != nullptr;
             float kv4[DK / 32 > 0 ? DK / 32 : 1];
             float ss = 0.f;
 #pragma unroll
@@ -76,11 +93,12 @@ __global__ void __launch_bounds__(128) recurrent_kernel(FwdParams p) {
                 const int c = lane + 32 * e;
                 float x = 0.f;
                 if (ki >= 0 && c < DK) x = to_f32(kk[(size_t)ki * DK + c]);
+                if (carried && c < DK) x = p.x_prev[(size_t)bh * DK + c];
                 kv4[e] = x;
                 ss += x * x;
             }
             ss = group_sum<32>(ss);
-            const float inv = (p.phi == 0) ? (ss > 0.f ? rsqrtf(ss) : 0.f) : 1.f;
+            const float inv = (p.phi == 0 && !carried) ? (ss > 0.f ? rsqrtf(ss) : 0.f) : 1.f;
             float sq = 0.f;
 #pragma unroll
             for (int e = 0; e < (DK >= 32 ? DK / 32 : 1); ++e) {

@@ -60,25 +60,33 @@ struct ChunkLayout {
 };
 
 // x_i for sample rows r in [0, nrows): sample index i = i0 + r; prefix pair
-// x_i = phi(k_{i-1}) (x_0 = 0), same-step x_i = phi(k_i); zeros for i < 0 or
-// i >= L (rows past the end are never read as real samples).  Also y_i for
-// the block's channel slice and |x_i|^2.
+// x_i = phi(k_{i-1}), same-step x_i = phi(k_i); zeros for i >= L (rows past
+// the end are never read as real samples).  Before the segment: x_0 (prefix
+// pair) is the carried phi(k) and the samples i < 0 the carried window of a
+// continued segment (zeros at the start of a sequence).  Also y_i for the
+// block's channel slice and |x_i|^2.
 template <typename T, int DK>
-__device__ void load_samples(const FwdParams &p, const T *kk, const T *kv, int L, int i0, int nrows,
+__device__ void load_samples(const FwdParams &p, int bh, const T *kk, const T *kv, int L, int i0, int nrows,
                              int j0, float *X, int LDX, float *Y, float *SQN) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int P = variant_info(p.variant, p.window).window - 1;
     for (int r = warp; r < nrows; r += kThreads / 32) {
         const int i = i0 + r;
         const int ki = p.pairing == 0 ? i - 1 : i;
         const bool ok = i >= 0 && i < L && ki >= 0;
+        // carried samples: the window before the segment, and x_0's phi(k)
+        const float *cw = (i < 0 && i >= -P && p.win) ? p.win + ((size_t)bh * P + (i + P)) * (DK + p.dv) : nullptr;
+        const bool cx = i == 0 && ki < 0 && p.x_prev != nullptr;
         float ss = 0.f;
         for (int c = lane; c < DK; c += 32) {
-            const float x = ok ? to_f32(kk[(size_t)ki * DK + c]) : 0.f;
+            float x = ok ? to_f32(kk[(size_t)ki * DK + c]) : 0.f;
+            if (cw) x = cw[c];
+            if (cx) x = p.x_prev[(size_t)bh * DK + c];
             X[r * LDX + c] = x;
             ss += x * x;
         }
         ss = group_sum<32>(ss);
-        const float inv = p.phi == 0 ? (ss > 0.f ? rsqrtf(ss) : 0.f) : 1.f;
+        const float inv = (p.phi == 0 && !cw && !cx) ? (ss > 0.f ? rsqrtf(ss) : 0.f) : 1.f;
         float sq = 0.f;
         for (int c = lane; c < DK; c += 32) {
             const float x = X[r * LDX + c] * inv;
@@ -89,7 +97,9 @@ __device__ void load_samples(const FwdParams &p, const T *kk, const T *kv, int L
         if (lane == 0) SQN[r] = sq;
         if (lane < VS) {
             const int j = j0 + lane;
-            Y[r * VS + lane] = (i >= 0 && i < L && j < p.dv) ? to_f32(kv[(size_t)i * p.dv + j]) : 0.f;
+            float y = (i >= 0 && i < L && j < p.dv) ? to_f32(kv[(size_t)i * p.dv + j]) : 0.f;
+            if (cw && j < p.dv) y = cw[DK + j];
+            Y[r * VS + lane] = y;
         }
     }
 }
@@ -159,13 +169,17 @@ __global__ void __launch_bounds__(kThreads) span_chunk_kernel(FwdParams p) {
     const T *kb = static_cast<const T *>(p.beta) + (size_t)bh * L * (vi.per_channel ? dv : 1);
     T *ko = static_cast<T *>(p.out) + (size_t)bh * L * dv;
 
-    for (int idx = threadIdx.x; idx < VS * LDX; idx += kThreads) S0[idx] = 0.f;
+    // S0: the carried state of a continued segment, else zeros
+    for (int idx = threadIdx.x; idx < VS * LDX; idx += kThreads) {
+        const int j = idx / LDX, c = idx % LDX;
+        S0[idx] = (p.init_state && c < DK && j0 + j < dv) ? p.init_state[((size_t)bh * dv + j0 + j) * DK + c] : 0.f;
+    }
 
     for (int c0 = 0; c0 < L; c0 += p.chunk) {
         const int n = min(p.chunk, L - c0);
         const int ns = n + w - 1;
         __syncthreads();
-        load_samples<T, DK>(p, kk, kv, L, c0 - (w - 1), ns, j0, X, LDX, Y, SQN);
+        load_samples<T, DK>(p, bh, kk, kv, L, c0 - (w - 1), ns, j0, X, LDX, Y, SQN);
         load_queries<T, DK>(kq, c0, n, Q, LDX);
         __syncthreads();
         steps_and_logdecay<T>(p, vi, kb, c0, n, j0, lam, SQN, ETA, G);
@@ -315,7 +329,7 @@ __global__ void __launch_bounds__(kThreads) span_masked_kernel(FwdParams p, int 
     for (int c0 = 0; c0 < L; c0 += C) {
         const int n = min(C, L - c0);
         __syncthreads();
-        load_samples<T, DK>(p, kk, kv, L, c0 - (w - 1), n + w - 1, j0, XI, LDX, Y, SQN);
+        load_samples<T, DK>(p, bh, kk, kv, L, c0 - (w - 1), n + w - 1, j0, XI, LDX, Y, SQN);
         __syncthreads();
         steps_and_logdecay<T>(p, vi, kb, c0, n, j0, lam, SQN, ETAI, GAMI);
         __syncthreads();
@@ -345,7 +359,7 @@ __global__ void __launch_bounds__(kThreads) span_masked_kernel(FwdParams p, int 
         const int n = min(C, L - c0);
         const int ns = n + w - 1;
         __syncthreads();
-        load_samples<T, DK>(p, kk, kv, L, c0 - (w - 1), ns, j0, XI, LDX, Y, SQN);
+        load_samples<T, DK>(p, bh, kk, kv, L, c0 - (w - 1), ns, j0, XI, LDX, Y, SQN);
         load_queries<T, DK>(kq, c0, n, QI, LDX);
         for (int idx = threadIdx.x; idx < n * VS; idx += kThreads) {
             const int tl = idx / VS, j = idx % VS;
@@ -365,7 +379,7 @@ __global__ void __launch_bounds__(kThreads) span_masked_kernel(FwdParams p, int 
         for (int cj = 0; cj < c0; cj += C) {
             const int nj = C;  // earlier blocks are always full
             __syncthreads();
-            load_samples<T, DK>(p, kk, kv, L, cj - (w - 1), nj + w - 1, j0, XJ, LDX, YJ, SQNJ);
+            load_samples<T, DK>(p, bh, kk, kv, L, cj - (w - 1), nj + w - 1, j0, XJ, LDX, YJ, SQNJ);
             for (int idx = threadIdx.x; idx < nj * VS; idx += kThreads) {
                 const int tl = idx / VS, j = idx % VS;
                 const bool ok = j0 + j < dv;

@@ -16,6 +16,10 @@ struct FwdParams {
     float *final_state;
     // stream-ordered scratch for the masked-parallel form
     float *ws_r, *ws_eta, *ws_gam;
+    // a segment continuing a sequence (NULL: zeros, the start of a sequence):
+    // initial state [B,H,dv,dk], x_prev [B,H,dk] (x of the first token) and
+    // the window-1 samples before the segment [B,H,window-1,dk+dv]
+    const float *init_state, *x_prev, *win;
 };
 
 struct DecodeParams {
