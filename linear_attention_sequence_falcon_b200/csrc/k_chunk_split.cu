@@ -281,13 +281,14 @@ __global__ void __launch_bounds__(NTH1, 2)
     LBLK(0);
     LTIM(0);
 
-    // loads of unit u into input set k: raw keys (row t <- key c0+t-1; the
-    // key before the sequence start and rows past its end read as zeros), q, v
+    // loads of unit u into input set k: raw keys (row t <- key c0+t-1 under
+    // the prefix pair, key c0+t under the same-step pair; the key before the
+    // sequence start and rows past its end read as zeros), q, v
     auto load_unit = [&](int u, int k) {
         const int ubh = u / nch, uc0 = (u - ubh * nch) * CH;
         const uint32_t o = sbase + (uint32_t)k * L_SET;
         tc::mbar_arrive_expect_tx(&tbar[k], 3 * TILE);
-        tc::tma_load_3d(o, &maps.k, 0, uc0 - 1, ubh, &tbar[k]);
+        tc::tma_load_3d(o, &maps.k, 0, p.pairing == 0 ? uc0 - 1 : uc0, ubh, &tbar[k]);
         tc::tma_load_3d(o + TILE, &maps.q, 0, uc0, ubh, &tbar[k]);
         tc::tma_load_3d(o + 2 * TILE, &maps.v, 0, uc0, ubh, &tbar[k]);
     };
@@ -379,7 +380,7 @@ __global__ void __launch_bounds__(NTH1, 2)
             }
             ss += __shfl_xor_sync(0xffffffffu, ss, 1);
             ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-            const float inv = carried ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
+            const float inv = (carried || p.phi != 0) ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
             const float sq = ss * inv * inv;  // |x_t|^2: 1 up to rounding, 0 for an empty sample
 #pragma unroll
             for (int e = 0; e < 16; ++e) xr[e] *= inv;
@@ -1059,8 +1060,7 @@ size_t split_chunk_ws_bytes(const FwdParams &p) {
 }
 
 int launch_split_chunk(const FwdParams &p, cudaStream_t s) {
-    const bool shape_ok = (p.variant == F1 || p.variant == F1A) && p.dk == DD && p.dv == DD && p.chunk == CH &&
-                          p.pairing == 0 && p.phi == 0;
+    const bool shape_ok = (p.variant == F1 || p.variant == F1A) && p.dk == DD && p.dv == DD && p.chunk == CH;
     auto al16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
     if (!shape_ok || !al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.out) ||
         (p.final_state && !al16(p.final_state)))

@@ -254,3 +254,31 @@ def test_decode_odd_pair_count(F, variant, dk, dv):
     oo, oS = oracle_fwd(d, variant, 1)
     assert rel(outs, oo[:, :, 20:]) <= 1e-4
     assert rel(S, oS) <= 1e-4
+
+
+# --------------------------------------------------------------- tensor-core path options and extremes
+
+@pytest.mark.parametrize("pairing,phi", [("same_step", "l2"), ("prefix", "identity"), ("same_step", "identity")])
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_tensor_core_pairing_and_feature_map(F, variant, pairing, phi):
+    """bf16, d = 64, chunk 64: the tensor-core chunk path with the same-step
+    pair and the identity feature map."""
+    d = gen.draw(variant, 2, 3, 150, 64, 64, seed=61, dtype="bf16", key_scale=0.125)
+    check(F, d, variant, "chunk", chunk=64, pairing=pairing, phi=phi)
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_tensor_core_strong_forgetting(F, variant):
+    """lambda = 0.999 on the tensor-core path: chunk log-decays around -45, so
+    the factorised decays use factors up to about e^22."""
+    d = gen.draw(variant, 1, 4, 200, 64, 64, seed=62, dtype="bf16", lam=0.999)
+    check(F, d, variant, "chunk", chunk=64)
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_tensor_core_decay_floor(F, variant):
+    """Tiny keys under the identity map with lambda = 0.9 put every alpha on
+    the 2^-20 floor: a chunk's log-decay is near -887, far below -80, so every
+    decay factor is taken as one exponential of a difference."""
+    d = gen.draw(variant, 1, 4, 200, 64, 64, seed=63, dtype="bf16", lam=0.9, key_scale=0.05)
+    check(F, d, variant, "chunk", chunk=64, phi="identity")
