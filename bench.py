@@ -458,6 +458,8 @@ def run_workloads(args):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     cases = []
     for n, w in gen.WORKLOADS.items():
+        if args.only and n != args.only:
+            continue
         forms = list(w["forms"])
         if n == 2:
             forms = ["chunk", "masked", "recurrent"]
@@ -497,6 +499,7 @@ def main():
                     help="run only warmup+steps decode steps (no flush or JSON), for ncu")
     ap.add_argument("--workloads", action="store_true",
                     help="time every workload and form of the workloads table, one JSON line each")
+    ap.add_argument("--only", type=int, default=0, help="with --workloads: just this workload number")
     ap.add_argument("--profile", action="store_true",
                     help="run only warmup+steps device steps (no flush, e2e, clocks or JSON), for ncu")
     args = ap.parse_args()

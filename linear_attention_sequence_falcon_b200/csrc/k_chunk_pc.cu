@@ -1,0 +1,588 @@
+// k_chunk_pc.cu -- chunk-parallel forward of Falcon-2A (inner product, one
+// step and decay per value channel) on the tcgen05 tensor cores, bf16
+// inputs, d_k = d_v = 128, chunk 64.
+//
+// Method: Falcon-2A takes eta and alpha per value channel j, i.e. per row of
+// S (page "借鉴40年前的设想！…", 02 (2)); the chunk form is parallel inside
+// chunks and hands a fixed-size state on (page "Fast Weight Attention：用于持
+// 续学习的快速权重注意力", 核心方法 3).  Per channel j, with the chunk-local
+// G_{t,j} = sum_{r<=t} log alpha_{r,j}, a chunk entered with S gives
+//   o_t[j]  = e^{G_{t,j}} (S q_t)[j] + sum_{s<=t} e^{G_{t,j}-G_{s,j}} eta_{s,j} y_{s,j} (x_s . q_t)
+//   S_end   = diag(e^{G_{C,j}}) S + dS,   dS[j][i] = sum_s e^{G_{C,j}-G_{s,j}} eta_{s,j} y_{s,j} x_s[i].
+// The inner-product family has no solve, and the state recursion is
+// elementwise in j (row j of S only ever scales by its own g_j), so the
+// forward is three fully parallel kernels:
+//   pc_delta_kernel  one block per (head, chunk): the decays and dS = W^T X
+//                    as one 128x128x64 product (W[s][j] = e^{G_C-G_s} eta y)
+//   pc_scan_kernel   one thread per (head, row j, 8 columns): S_c for every
+//                    chunk (written as the bf16 operand of the next kernel),
+//                    S_{c+1} = g_c S_c + dS_c in fp32, the final state
+//   pc_out_kernel    one block per (head, chunk): P = Q X^T, the intra-chunk
+//                    term as (P o mask) Yt with Yt[s][j] = e^{G_r-G_s} eta y
+//                    scaled by e^{G_t-G_r} (factorised around r = token 31
+//                    while every channel's log-decay stays above -80, else
+//                    one exponential per term on the CUDA cores), and the
+//                    carried term Q S_c^T scaled by e^{G_t}.
+// Every tcgen05 operand is K-major with 128-byte rows and the 128-byte
+// swizzle; d = 128 rows are two 64-column halves.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_sm100.cuh"
+
+namespace falcon {
+
+namespace {
+
+constexpr int CH = 64;    // chunk
+constexpr int DD = 128;   // d_k = d_v
+constexpr int NTH = 256;
+constexpr int ISSUER = 128;
+constexpr uint32_t TILE = 8192;                // 64 rows x 128 bytes
+constexpr uint32_t SIMG = 4 * TILE;            // bf16 S_c: two K halves of 128 rows x 64
+constexpr uint32_t DSIMG = DD * DD * 2;        // bf16 dS, row-major [j][i]
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr float kFactorMinLogDecay = -80.f;
+constexpr int LDG = DD + 1;                    // fp32 row stride of the G table (conflict-free columns)
+
+__device__ unsigned int g_pc_wait_timeouts;
+
+__device__ __forceinline__ uint4 pack8(const float *f) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(f[2], f[3]);
+    __nv_bfloat162 c = __floats2bfloat162_rn(f[4], f[5]);
+    __nv_bfloat162 d = __floats2bfloat162_rn(f[6], f[7]);
+    uint4 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    u.z = *reinterpret_cast<uint32_t *>(&c);
+    u.w = *reinterpret_cast<uint32_t *>(&d);
+    return u;
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float *f) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 t = __bfloat1622float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+// element (r, c) of a 64-row bf16 tile pair: two 64-column halves, the
+// second `hs` bytes after the first
+__device__ __forceinline__ uint32_t pair_off(int r, int c, uint32_t hs = TILE) {
+    return (uint32_t)(c >> 6) * hs + tc::sw128(r, (c & 63) >> 3) + (uint32_t)(c & 7) * 2;
+}
+
+// D (+)= A B^T over K = 64 * nk (4 K=16 slices per 64-column tile), both
+// operands K-major 128-byte-swizzled; the k-th K tile of A (B) starts
+// a_step (b_step) bytes after the previous one; M = 128.
+__device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a, uint32_t a_step, uint32_t b,
+                                           uint32_t b_step, int nk, int N) {
+    const uint32_t idesc = tc::idesc_bf16(128, N, 0, 0);
+    for (int kt = 0; kt < nk; ++kt)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = tc::sdesc_sw128(a + kt * a_step + kk * 32, 16, 1024);
+            const uint64_t bd = tc::sdesc_sw128(b + kt * b_step + kk * 32, 16, 1024);
+            tc::mma_bf16(d_tmem, ad, bd, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+        }
+}
+
+// Transposed copy of four 8x8 blocks of a 64-row bf16 tile (128-byte rows,
+// 128-byte swizzle): source row block rb, 16-byte chunks cb0..cb0+3 ->
+// destination rows 8*(cb0..cb0+3) (+ dst_row0), chunk rb.  Whole warp.
+__device__ __forceinline__ void transpose4(uint32_t src, int rb, int cb0, uint32_t dst, int dst_row0) {
+    const int lane = threadIdx.x & 31, m = lane >> 3, i = lane & 7;
+    uint32_t r[4];
+    tc::ldsm_x4_trans(src + (uint32_t)(rb * 8 + i) * 128u + ((uint32_t)((cb0 + m) ^ i) << 4), r);
+    const int drow = dst_row0 + (cb0 + m) * 8 + i;
+    tc::stsm_x4(dst + (uint32_t)drow * 128u + ((uint32_t)(rb ^ (drow & 7)) << 4), r);
+}
+
+// Transpose a 64 x 128 tile pair (rows s, two 64-column halves) into a
+// 128-row K-major tile (rows c, 64 columns s): 32 groups of 4 blocks over
+// the block's 8 warps.
+__device__ __forceinline__ void transpose_pair(uint32_t src_pair, uint32_t dst128) {
+    const int warp = threadIdx.x >> 5;
+    for (int g = warp; g < 32; g += NTH / 32) {
+        const int half = g >> 4, rb = (g >> 1) & 7, cb0 = (g & 1) * 4;
+        transpose4(src_pair + half * TILE, rb, cb0, dst128, half * 64);
+    }
+}
+
+struct PcMaps {
+    CUtensorMap q, k, v, beta;
+};
+
+// TMA: a 64-row x 128-column bf16 slab (rows y.., the two halves) into a tile pair
+__device__ __forceinline__ void load_pair(uint32_t dst, const CUtensorMap *m, int y, int bh, uint64_t *bar) {
+    tc::tma_load_3d(dst, m, 0, y, bh, bar);
+    tc::tma_load_3d(dst + TILE, m, 64, y, bh, bar);
+}
+
+// samples x_t = phi(k_{t-1}) in place over the raw-key tile pair (four
+// threads per row, 32 columns each), |x_t|^2 -> sqn[t].  The first token of
+// a continued segment takes the carried phi(k) as given.
+__device__ __forceinline__ void samples_pair(uint8_t *sm, uint32_t offx, uint32_t hs, const FwdParams &p, int bh,
+                                             bool first_chunk, float *sqn) {
+    const int tid = threadIdx.x, r = tid >> 2, part = tid & 3;
+    const bool carried = first_chunk && r == 0 && p.x_prev != nullptr && p.pairing == 0;
+    float xr[32];
+    float ss = 0.f;
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+        const int c = part * 32 + c8 * 8;
+        if (carried) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xr[c8 * 8 + e] = p.x_prev[(size_t)bh * DD + c + e];
+        } else {
+            unpack8(*reinterpret_cast<const uint4 *>(sm + offx + pair_off(r, c, hs)), &xr[c8 * 8]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss += xr[c8 * 8 + e] * xr[c8 * 8 + e];
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    const float inv = (carried || p.phi != 0) ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xr[c8 * 8 + e] *= inv;
+        *reinterpret_cast<uint4 *>(sm + offx + pair_off(r, part * 32 + c8 * 8, hs)) = pack8(&xr[c8 * 8]);
+    }
+    if (part == 0) sqn[r] = ss * inv * inv;
+}
+
+// bf16 element (r, c) of a tile pair
+__device__ __forceinline__ float pair_get(const uint8_t *sm, uint32_t off, int r, int c) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + off + pair_off(r, c)));
+}
+
+}  // namespace
+
+// ============================================================ dS kernel
+namespace {
+constexpr uint32_t D_X = 0;            // raw keys -> X (tile pair)
+constexpr uint32_t D_V = 2 * TILE;     // values (tile pair)
+constexpr uint32_t D_B = 4 * TILE;     // per-channel beta (tile pair)
+constexpr uint32_t D_W = 6 * TILE;     // W[s][j] = e^{G_C-G_s} eta y (tile pair)
+constexpr uint32_t D_WT = 8 * TILE;    // W^T: 128 rows j x 64 s
+constexpr uint32_t D_XT = 10 * TILE;   // X^T: 128 rows i x 64 s
+constexpr uint32_t D_VEC = 12 * TILE;  // |x_s|^2
+constexpr uint32_t D_BAR = D_VEC + 256;
+constexpr uint32_t D_SMEM = D_BAR + 64 + 1024;
+}  // namespace
+
+// One block per unit (b*H + h, chunk); blockIdx.x = bh * nchunks + c.
+__global__ void __launch_bounds__(NTH, 2)
+    pc_delta_kernel(FwdParams p, const __grid_constant__ PcMaps maps, __nv_bfloat16 *ds_ws, float *g_ws) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = tc::smem_u32(smem_raw);
+    uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = tc::smem_u32(sm);
+    float *sqn = reinterpret_cast<float *>(sm + D_VEC);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + D_BAR);
+    uint64_t *tbar = bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int L = p.L, nch = (L + CH - 1) / CH;
+    const int u = blockIdx.x, bh = u / nch, c0 = (u - bh * nch) * CH;
+
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::mbar_init(tbar, 1);
+        tc::fence_mbar_init();
+        tc::mbar_arrive_expect_tx(tbar, 6 * TILE);
+        load_pair(sbase + D_X, &maps.k, p.pairing == 0 ? c0 - 1 : c0, bh, tbar);
+        load_pair(sbase + D_V, &maps.v, c0, bh, tbar);
+        load_pair(sbase + D_B, &maps.beta, c0, bh, tbar);
+    }
+    __syncwarp();
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 128);
+        tc::tmem_relinquish();
+    }
+    const float lam = tid < DD ? p.lambda[bh % p.H] : 0.f;
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    bool ok = tc::mbar_wait_timeout(tbar, 0, kWaitNs);
+    ok = __syncthreads_and(ok);
+    if (ok) {
+        samples_pair(sm, D_X, TILE, p, bh, c0 == 0, sqn);
+        __syncthreads();
+        if (tid < DD) {
+            // channel j: eta_{s,j}, log alpha_{s,j} and their sum over the chunk, twice
+            const int j = tid;
+            float G = 0.f;
+            for (int s = 0; s < CH; ++s) {
+                const float n = sqn[s];
+                const float eta = n > 0.f ? __fdividef(pair_get(sm, D_B, s, j), p.eps + n) : 0.f;
+                G += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
+            }
+            const float GC = G;
+            G = 0.f;
+            for (int s = 0; s < CH; ++s) {
+                const float n = sqn[s];
+                const float eta = n > 0.f ? __fdividef(pair_get(sm, D_B, s, j), p.eps + n) : 0.f;
+                G += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
+                const float w = __expf(GC - G) * eta * pair_get(sm, D_V, s, j);  // GC - G <= 0
+                *reinterpret_cast<__nv_bfloat16 *>(sm + D_W + pair_off(s, j)) = __float2bfloat16_rn(w);
+            }
+            g_ws[(size_t)u * DD + j] = __expf(GC);
+        } else {
+            // X^T (warps 4-7)
+            for (int g = warp - 4; g < 32; g += 4) {
+                const int half = g >> 4, rb = (g >> 1) & 7, cb0 = (g & 1) * 4;
+                transpose4(sbase + D_X + half * TILE, rb, cb0, sbase + D_XT, half * 64);
+            }
+        }
+        __syncthreads();
+        transpose_pair(sbase + D_W, sbase + D_WT);
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        // dS[j][i] = sum_s W^T[j][s] X^T[i][s]
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_gemm(tbase, sbase + D_WT, 0, sbase + D_XT, 0, 1, 128);
+            tc::mma_commit(bar);
+        }
+        ok = tc::mbar_wait_timeout(bar, 0, kWaitNs);
+        ok = __syncthreads_and(ok);
+    }
+    if (ok) {
+        tc::fence_after_sync();
+        const int quarter = warp & 3, chalf = warp >> 2, j = quarter * 32 + lane;
+        const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
+        __nv_bfloat16 *dst = ds_ws + ((size_t)u * DD + j) * DD + chalf * 64;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+            float v[16];
+            tc::tmem_ld16(tl + chalf * 64 + k4 * 16, v);
+            tc::tmem_wait_ld();
+            *reinterpret_cast<uint4 *>(dst + k4 * 16) = pack8(&v[0]);
+            *reinterpret_cast<uint4 *>(dst + k4 * 16 + 8) = pack8(&v[8]);
+        }
+    } else {
+        if (tid == 0) atomicAdd(&g_pc_wait_timeouts, 1u);
+        (void)tc::mbar_wait_timeout(tbar, 0, kWaitNs);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 128);
+}
+
+// ============================================================ state scan
+// One thread per (b*H + h, row j, 8 columns): the state at every chunk start
+// (bf16, in the operand layout of pc_out_kernel: two K halves of 128 rows x
+// 128 bytes, swizzled), S_{c+1} = g_c S_c + dS_c in fp32, the final state.
+__global__ void __launch_bounds__(256)
+    pc_scan_kernel(FwdParams p, const __nv_bfloat16 *__restrict__ ds_ws, const float *__restrict__ g_ws,
+                   uint8_t *__restrict__ s_ws) {
+    const int nch = (p.L + CH - 1) / CH;
+    const size_t gidx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t rowid = gidx >> 4;  // bh * 128 + j
+    if (rowid >= (size_t)p.B * p.H * DD) return;
+    const int i8 = (int)(gidx & 15), j = (int)(rowid % DD);
+    const size_t bh = rowid / DD;
+    float S[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) S[e] = p.init_state ? p.init_state[rowid * DD + i8 * 8 + e] : 0.f;
+    const uint32_t soff = (uint32_t)(i8 >> 3) * (2 * TILE) + tc::sw128(j, i8 & 7);
+#pragma unroll 4
+    for (int c = 0; c < nch; ++c) {
+        const size_t u = bh * nch + c;
+        *reinterpret_cast<uint4 *>(s_ws + u * SIMG + soff) = pack8(S);
+        const uint4 d = *reinterpret_cast<const uint4 *>(ds_ws + (u * DD + j) * DD + i8 * 8);
+        const float g = g_ws[u * DD + j];
+        float dv[8];
+        unpack8(d, dv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) S[e] = g * S[e] + dv[e];
+    }
+    if (p.final_state) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) p.final_state[rowid * DD + i8 * 8 + e] = S[e];
+    }
+}
+
+// ============================================================ outputs
+namespace {
+constexpr uint32_t O_Q0 = 0, O_X0 = TILE, O_Q1 = 2 * TILE, O_X1 = 3 * TILE;  // [Q;X] per K half
+constexpr uint32_t O_V = 4 * TILE;     // values (tile pair)
+constexpr uint32_t O_B = 6 * TILE;     // per-channel beta (tile pair)
+constexpr uint32_t O_S = 8 * TILE;     // bf16 S_c: K half k at O_S + 2 TILE k (128 rows j)
+constexpr uint32_t O_Y = 12 * TILE;    // Yt[s][j] = e^{G_r-G_s} eta y (tile pair)
+constexpr uint32_t O_YT = 14 * TILE;   // Yt^T: 128 rows j x 64 s
+constexpr uint32_t O_PM = 16 * TILE;   // P o mask, rows t (the G table after it pads A to 128 rows)
+constexpr uint32_t O_G = 17 * TILE;    // fp32 G[t][j], row stride LDG
+constexpr uint32_t O_VEC = O_G + 64 * LDG * 4;  // |x_s|^2 [64], G_{r,j} [128]
+constexpr uint32_t O_BAR = O_VEC + (64 + 128 + 16) * 4;
+constexpr uint32_t O_SMEM = O_BAR + 64 + 1024;
+}  // namespace
+
+// One block per unit (b*H + h, chunk).  Tensor memory: [P;A] in columns
+// 0-63, then the intra-chunk product in 0-127; Q S_c^T in 128-255.
+__global__ void __launch_bounds__(NTH, 1)
+    pc_out_kernel(FwdParams p, const __grid_constant__ PcMaps maps, const uint8_t *s_ws) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = tc::smem_u32(smem_raw);
+    uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = tc::smem_u32(sm);
+    float *Gt = reinterpret_cast<float *>(sm + O_G);
+    float *sqn = reinterpret_cast<float *>(sm + O_VEC);
+    float *Gr = sqn + 64;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + O_BAR);
+    uint64_t *tbar = bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, chalf = warp >> 2, row = quarter * 32 + lane;
+    const int L = p.L, nch = (L + CH - 1) / CH;
+    const int u = blockIdx.x, bh = u / nch, c0 = (u - bh * nch) * CH, nt = min(CH, L - c0);
+
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::mbar_init(tbar, 1);
+        tc::fence_mbar_init();
+        const int krow = p.pairing == 0 ? c0 - 1 : c0;
+        tc::mbar_arrive_expect_tx(tbar, 8 * TILE + SIMG);
+        tc::tma_load_3d(sbase + O_Q0, &maps.q, 0, c0, bh, tbar);
+        tc::tma_load_3d(sbase + O_Q1, &maps.q, 64, c0, bh, tbar);
+        tc::tma_load_3d(sbase + O_X0, &maps.k, 0, krow, bh, tbar);
+        tc::tma_load_3d(sbase + O_X1, &maps.k, 64, krow, bh, tbar);
+        load_pair(sbase + O_V, &maps.v, c0, bh, tbar);
+        load_pair(sbase + O_B, &maps.beta, c0, bh, tbar);
+        tc::bulk_load(sbase + O_S, s_ws + (size_t)u * SIMG, SIMG, tbar);
+    }
+    __syncwarp();
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 256);
+        tc::tmem_relinquish();
+    }
+    const float lam = tid < DD ? p.lambda[bh % p.H] : 0.f;
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
+    bool ok = tc::mbar_wait_timeout(tbar, 0, kWaitNs);
+    ok = __syncthreads_and(ok);
+    bool unsafe = false;
+    if (ok) {
+        samples_pair(sm, O_X0, 2 * TILE, p, bh, c0 == 0, sqn);
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_gemm(tbase, sbase + O_Q0, 2 * TILE, sbase + O_X0, 2 * TILE, 2, 64);         // [P ; X X^T]
+            issue_gemm(tbase + 128, sbase + O_Q0, 2 * TILE, sbase + O_S, 2 * TILE, 2, 128);   // Q S_c^T
+            tc::mma_commit(bar);
+        }
+        bool local_unsafe = false;
+        if (tid < DD) {
+            // channel j: cumulative log decay G_{s,j} (table) and Yt[s][j]
+            const int j = tid;
+            float G = 0.f, Gref = 0.f;
+            for (int s = 0; s < CH; ++s) {
+                const float n = sqn[s];
+                const float eta = n > 0.f ? __fdividef(pair_get(sm, O_B, s, j), p.eps + n) : 0.f;
+                G += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
+                Gt[s * LDG + j] = G;
+                if (s == 31) Gref = G;
+            }
+            Gr[j] = Gref;
+            local_unsafe = G <= kFactorMinLogDecay;  // e^{G_r-G_s} could leave the fp32 range
+            for (int s = 0; s < CH; ++s) {
+                const float n = sqn[s];
+                const float eta = n > 0.f ? __fdividef(pair_get(sm, O_B, s, j), p.eps + n) : 0.f;
+                const float yt = local_unsafe ? 0.f : __expf(Gref - Gt[s * LDG + j]) * eta * pair_get(sm, O_V, s, j);
+                *reinterpret_cast<__nv_bfloat16 *>(sm + O_Y + pair_off(s, j)) = __float2bfloat16_rn(yt);
+            }
+        }
+        unsafe = __syncthreads_or(local_unsafe) != 0;
+        if (!unsafe) transpose_pair(sbase + O_Y, sbase + O_YT);
+        ok = tc::mbar_wait_timeout(bar, 0, kWaitNs);
+        ok = __syncthreads_and(ok);
+    }
+    if (ok) {
+        tc::fence_after_sync();
+        if (quarter < 2) {  // P o mask (s <= t) -> bf16, rows t
+            const int t = row;
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int cs = chalf * 2 + k2;
+                float v[16];
+                tc::tmem_ld16(tl + cs * 16, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = cs * 16 + i <= t ? v[i] : 0.f;
+                *reinterpret_cast<uint4 *>(sm + O_PM + tc::sw128(t, cs * 2)) = pack8(&v[0]);
+                *reinterpret_cast<uint4 *>(sm + O_PM + tc::sw128(t, cs * 2 + 1)) = pack8(&v[8]);
+            }
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (!unsafe) {
+            if (tid == ISSUER) {
+                tc::fence_after_sync();
+                issue_gemm(tbase, sbase + O_PM, 0, sbase + O_YT, 0, 1, 128);  // (P o mask) Yt
+                tc::mma_commit(bar);
+            }
+            ok = tc::mbar_wait_timeout(bar, 1, kWaitNs);
+            ok = __syncthreads_and(ok);
+        }
+    }
+    if (ok) {
+        tc::fence_after_sync();
+        if (quarter < 2) {
+            // o_t[j] = e^{G_t} (Q S_c^T)[t][j] + e^{G_t - G_r} ((P o mask) Yt)[t][j]
+            const int t = row;
+            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + ((size_t)bh * L + c0 + t) * DD;
+            float prow[CH];  // the fallback's P row
+            if (unsafe) {
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    float v[16];
+                    tc::tmem_ld16(tl + k4 * 16, v);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) prow[k4 * 16 + i] = v[i];
+                }
+            }
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int jj = chalf * 64 + k4 * 16;
+                float iv[16], av[16];
+                tc::tmem_ld16(tl + 128 + jj, iv);
+                if (!unsafe) tc::tmem_ld16(tl + jj, av);
+                tc::tmem_wait_ld();
+                float o[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int j = jj + i;
+                    const float gt = Gt[t * LDG + j];
+                    float intra;
+                    if (!unsafe) {
+                        intra = __expf(gt - Gr[j]) * av[i];
+                    } else {
+                        // one exponential per term, every exponent <= 0
+                        intra = 0.f;
+                        for (int s = 0; s <= t; ++s) {
+                            const float n = sqn[s];
+                            const float eta = n > 0.f ? __fdividef(pair_get(sm, O_B, s, j), p.eps + n) : 0.f;
+                            intra += prow[s] * __expf(gt - Gt[s * LDG + j]) * eta * pair_get(sm, O_V, s, j);
+                        }
+                    }
+                    o[i] = __expf(gt) * iv[i] + intra;
+                }
+                if (t < nt) {
+                    *reinterpret_cast<uint4 *>(dst + jj) = pack8(&o[0]);
+                    *reinterpret_cast<uint4 *>(dst + jj + 8) = pack8(&o[8]);
+                }
+            }
+        }
+    } else {
+        if (tid == 0) atomicAdd(&g_pc_wait_timeouts, 1u);
+        (void)tc::mbar_wait_timeout(tbar, 0, kWaitNs);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 256);
+}
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// [B*H][L][128] bf16 tensor, boxes of 64 rows x 64 columns (one 128-byte
+// swizzled half), zero fill outside.
+bool make_map(CUtensorMap *m, const void *base, int BH, int L) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)DD, (cuuint64_t)L, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)DD * 2, (cuuint64_t)L * DD * 2};
+    const cuuint32_t box[3] = {64, CH, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int launch_pc_chunk(const FwdParams &p, cudaStream_t s) {
+    const bool shape_ok = p.variant == F2A && p.dk == DD && p.dv == DD && p.chunk == CH;
+    auto al16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+    if (!shape_ok || !al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.beta) || !al16(p.out) ||
+        (p.final_state && !al16(p.final_state)))
+        return 1;
+    const int BH = p.B * p.H, nch = (p.L + CH - 1) / CH;
+    const size_t units = (size_t)BH * nch;
+    if (units > 0x7fffffffu) return 1;
+    PcMaps maps;
+    if (!make_map(&maps.q, p.q, BH, p.L) || !make_map(&maps.k, p.k, BH, p.L) || !make_map(&maps.v, p.v, BH, p.L) ||
+        !make_map(&maps.beta, p.beta, BH, p.L))
+        return 1;
+    void *ws = nullptr;
+    const size_t bytes = units * ((size_t)DSIMG + (size_t)DD * sizeof(float) + SIMG);
+    if (scratch_alloc(&ws, bytes, s) != cudaSuccess) {
+        cudaGetLastError();
+        return -8;  // FALCON_ERR_ALLOC
+    }
+    uint8_t *simg = static_cast<uint8_t *>(ws);
+    __nv_bfloat16 *ds = reinterpret_cast<__nv_bfloat16 *>(simg + units * SIMG);
+    float *g = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(ds) + units * DSIMG);
+    static bool attrs_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attrs_set[dev]) {
+        cudaFuncSetAttribute(pc_delta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)D_SMEM);
+        cudaFuncSetAttribute(pc_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)O_SMEM);
+        if (dev >= 0 && dev < 64) attrs_set[dev] = true;
+    }
+    pc_delta_kernel<<<(unsigned)units, NTH, D_SMEM, s>>>(p, maps, ds, g);
+    const size_t scan_threads = (size_t)BH * DD * 16;
+    pc_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, s>>>(p, ds, g, simg);
+    pc_out_kernel<<<(unsigned)units, NTH, O_SMEM, s>>>(p, maps, simg);
+    const cudaError_t e = cudaGetLastError();
+    scratch_free(ws, s);
+    return e == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
+}
+
+unsigned int pc_wait_timeouts() {
+    unsigned int v = 0;
+    cudaMemcpyFromSymbol(&v, g_pc_wait_timeouts, sizeof(v));
+    return v;
+}
+
+}  // namespace falcon

@@ -51,6 +51,11 @@ int launch_split_chunk(const FwdParams &p, cudaStream_t s);
 size_t split_chunk_ws_bytes(const FwdParams &p);
 // Number of tensor-core thread blocks that gave up on a bounded wait.
 unsigned int split_wait_timeouts();
+// bf16 Falcon-2A chunk-parallel forward, d_k = d_v = 128, chunk 64, on
+// tcgen05 (dS per chunk, state scan, outputs); returns 1 for shapes it does
+// not cover.
+int launch_pc_chunk(const FwdParams &p, cudaStream_t s);
+unsigned int pc_wait_timeouts();
 template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
 

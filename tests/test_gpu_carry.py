@@ -120,3 +120,7 @@ def test_empty_segment_keeps_the_state(F):
     _, S = F.fwd("F2A", "chunk", *(d[n].cuda() for n in ("q", "k", "v", "beta", "lam")), d["eps"], initial_state=S0)
     torch.cuda.synchronize()
     assert torch.equal(S, S0)
+
+
+def test_carry_falcon2a_d128_tensor_core_path(F):
+    check_segment(F, "F2A", "chunk", "bf16", 1, 3, 200, 128, 128, 64, 81)
