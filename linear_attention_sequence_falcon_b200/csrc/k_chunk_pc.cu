@@ -12,17 +12,17 @@
 // The inner-product family has no solve, and the state recursion is
 // elementwise in j (row j of S only ever scales by its own g_j), so the
 // forward is three fully parallel kernels:
-//   pc_delta_kernel  one block per (head, chunk): the decays and dS = W^T X
-//                    as one 128x128x64 product (W[s][j] = e^{G_C-G_s} eta y)
-//   pc_scan_kernel   one thread per (head, row j, 8 columns): S_c for every
-//                    chunk (written as the bf16 operand of the next kernel),
-//                    S_{c+1} = g_c S_c + dS_c in fp32, the final state
-//   pc_out_kernel    one block per (head, chunk): P = Q X^T, the intra-chunk
-//                    term as (P o mask) Yt with Yt[s][j] = e^{G_r-G_s} eta y
-//                    scaled by e^{G_t-G_r} (factorised around r = token 31
-//                    while every channel's log-decay stays above -80, else
-//                    one exponential per term on the CUDA cores), and the
-//                    carried term Q S_c^T scaled by e^{G_t}.
+//   pc_delta_kernel  one block per (head, chunk): the decays (one thread per
+//                    channel and half chunk), W[s][j] = e^{G_C-G_s} eta y,
+//                    dS = W^T X as one 128x128x64 product; hands on dS,
+//                    g = e^{G_C}, W^T and e^{G_t}
+//   pc_scan_kernel   one thread per (head, 16-byte column group): S_c for
+//                    every chunk (written as the bf16 operand of the next
+//                    kernel), S_{c+1} = g_c S_c + dS_c in fp32, the final state
+//   pc_out_kernel    one block per (head, chunk): P = Q X^T and Q S_c^T, then
+//                    (P o mask) W, and o = e^{G_t} (Q S_c^T + e^{-G_C} (P o mask) W)
+//                    while every channel's G_C stays above -80; below that the
+//                    intra-chunk terms are summed one exponential at a time.
 // Every tcgen05 operand is K-major with 128-byte rows and the 128-byte
 // swizzle; d = 128 rows are two 64-column halves.
 #include <cuda.h>
@@ -47,8 +47,6 @@ constexpr uint32_t TILE = 8192;                // 64 rows x 128 bytes
 constexpr uint32_t SIMG = 4 * TILE;            // bf16 S_c: two K halves of 128 rows x 64
 constexpr uint32_t DSIMG = DD * DD * 2;        // bf16 dS, row-major [j][i]
 constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr float kFactorMinLogDecay = -80.f;
-constexpr int LDG = DD + 1;                    // fp32 row stride of the G table (conflict-free columns)
 
 __device__ unsigned int g_pc_wait_timeouts;
 
@@ -132,7 +130,7 @@ __device__ __forceinline__ void load_pair(uint32_t dst, const CUtensorMap *m, in
 // threads per row, 32 columns each), |x_t|^2 -> sqn[t].  The first token of
 // a continued segment takes the carried phi(k) as given.
 __device__ __forceinline__ void samples_pair(uint8_t *sm, uint32_t offx, uint32_t hs, const FwdParams &p, int bh,
-                                             bool first_chunk, float *sqn) {
+                                             bool first_chunk, float *sqn, float *rinv = nullptr) {
     const int tid = threadIdx.x, r = tid >> 2, part = tid & 3;
     const bool carried = first_chunk && r == 0 && p.x_prev != nullptr && p.pairing == 0;
     float xr[32];
@@ -158,7 +156,11 @@ __device__ __forceinline__ void samples_pair(uint8_t *sm, uint32_t offx, uint32_
         for (int e = 0; e < 8; ++e) xr[c8 * 8 + e] *= inv;
         *reinterpret_cast<uint4 *>(sm + offx + pair_off(r, part * 32 + c8 * 8, hs)) = pack8(&xr[c8 * 8]);
     }
-    if (part == 0) sqn[r] = ss * inv * inv;
+    if (part == 0) {
+        const float n = ss * inv * inv;
+        sqn[r] = n;
+        if (rinv) rinv[r] = n > 0.f ? 1.f / (p.eps + n) : 0.f;  // eta_t = beta_t / (eps + |x_t|^2), 0 at x_t = 0
+    }
 }
 
 // bf16 element (r, c) of a tile pair
@@ -170,25 +172,48 @@ __device__ __forceinline__ float pair_get(const uint8_t *sm, uint32_t off, int r
 
 // ============================================================ dS kernel
 namespace {
-constexpr uint32_t D_X = 0;            // raw keys -> X (tile pair)
-constexpr uint32_t D_V = 2 * TILE;     // values (tile pair)
-constexpr uint32_t D_B = 4 * TILE;     // per-channel beta (tile pair)
-constexpr uint32_t D_W = 6 * TILE;     // W[s][j] = e^{G_C-G_s} eta y (tile pair)
-constexpr uint32_t D_WT = 8 * TILE;    // W^T: 128 rows j x 64 s
-constexpr uint32_t D_XT = 10 * TILE;   // X^T: 128 rows i x 64 s
-constexpr uint32_t D_VEC = 12 * TILE;  // |x_s|^2
-constexpr uint32_t D_BAR = D_VEC + 256;
+constexpr uint32_t D_X = 0;            // raw keys -> X (tile pair); with D_V the dS image after the product
+constexpr uint32_t D_V = 2 * TILE;     // values -> W[s][j] = e^{G_C-G_s} eta y in place (tile pair)
+constexpr uint32_t D_B = 4 * TILE;     // per-channel beta -> E[s][j] = e^{G_s} in place (tile pair)
+constexpr uint32_t D_WT = 6 * TILE;    // W^T: 128 rows j x 64 s
+constexpr uint32_t D_XT = 8 * TILE;    // X^T: 128 rows i x 64 s
+constexpr uint32_t D_VEC = 10 * TILE;  // |x_s|^2 [64], 1/(eps+|x_s|^2) [64], half-chunk log-decay sums [2][128]
+constexpr uint32_t D_BAR = D_VEC + (64 + 64 + 2 * DD) * 4;
 constexpr uint32_t D_SMEM = D_BAR + 64 + 1024;
+constexpr uint32_t WTIMG = 2 * TILE;   // W^T image handed to pc_out_kernel
+constexpr uint32_t EIMG = 2 * TILE;    // e^{G_t} tile pair handed to pc_out_kernel
+
+// per-unit workspace: S_c image, dS image, W^T image, e^{G_t} pair, g = e^{G_C}
+constexpr size_t WS_UNIT = (size_t)SIMG + DSIMG + WTIMG + EIMG + DD * sizeof(float);
+struct PcWs {
+    uint8_t *simg, *dsimg, *wt, *e;
+    float *g;
+};
+__host__ __device__ inline PcWs pc_ws(void *base, size_t units) {
+    uint8_t *b = static_cast<uint8_t *>(base);
+    PcWs w;
+    w.simg = b;
+    w.dsimg = w.simg + units * SIMG;
+    w.wt = w.dsimg + units * DSIMG;
+    w.e = w.wt + units * WTIMG;
+    w.g = reinterpret_cast<float *>(w.e + units * EIMG);
+    return w;
+}
 }  // namespace
 
 // One block per unit (b*H + h, chunk); blockIdx.x = bh * nchunks + c.
-__global__ void __launch_bounds__(NTH, 2)
-    pc_delta_kernel(FwdParams p, const __grid_constant__ PcMaps maps, __nv_bfloat16 *ds_ws, float *g_ws) {
+// The decays are taken by one thread per (channel j, half of the chunk):
+// 32 log-decays summed in registers, the two halves joined through shared
+// memory.  Outputs: dS (bf16 image, the layout of the state operand), g =
+// e^{G_C}, and for pc_out_kernel W^T (its intra-chunk operand) and e^{G_t}.
+__global__ void __launch_bounds__(NTH, 2) pc_delta_kernel(FwdParams p, const __grid_constant__ PcMaps maps, PcWs ws) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = tc::smem_u32(smem_raw);
     uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
     const uint32_t sbase = tc::smem_u32(sm);
     float *sqn = reinterpret_cast<float *>(sm + D_VEC);
+    float *rinv = sqn + 64;
+    float *hsum = rinv + 64;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + D_BAR);
     uint64_t *tbar = bar + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
@@ -211,7 +236,7 @@ __global__ void __launch_bounds__(NTH, 2)
         tc::tmem_alloc(tmem_slot, 128);
         tc::tmem_relinquish();
     }
-    const float lam = tid < DD ? p.lambda[bh % p.H] : 0.f;
+    const float lam = p.lambda[bh % p.H];
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -219,36 +244,46 @@ __global__ void __launch_bounds__(NTH, 2)
     bool ok = tc::mbar_wait_timeout(tbar, 0, kWaitNs);
     ok = __syncthreads_and(ok);
     if (ok) {
-        samples_pair(sm, D_X, TILE, p, bh, c0 == 0, sqn);
+        samples_pair(sm, D_X, TILE, p, bh, c0 == 0, sqn, rinv);
         __syncthreads();
-        if (tid < DD) {
-            // channel j: eta_{s,j}, log alpha_{s,j} and their sum over the chunk, twice
-            const int j = tid;
-            float G = 0.f;
-            for (int s = 0; s < CH; ++s) {
-                const float n = sqn[s];
-                const float eta = n > 0.f ? __fdividef(pair_get(sm, D_B, s, j), p.eps + n) : 0.f;
-                G += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
+        // channel j, tokens 32h .. 32h+31: the running sums of log alpha
+        const int h = tid >> 7, j = tid & (DD - 1);
+        float Gl[32];
+        {
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int s_ = h * 32 + i;
+                const float eta = pair_get(sm, D_B, s_, j) * rinv[s_];
+                acc += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
+                Gl[i] = acc;
             }
-            const float GC = G;
-            G = 0.f;
-            for (int s = 0; s < CH; ++s) {
-                const float n = sqn[s];
-                const float eta = n > 0.f ? __fdividef(pair_get(sm, D_B, s, j), p.eps + n) : 0.f;
-                G += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
-                const float w = __expf(GC - G) * eta * pair_get(sm, D_V, s, j);  // GC - G <= 0
-                *reinterpret_cast<__nv_bfloat16 *>(sm + D_W + pair_off(s, j)) = __float2bfloat16_rn(w);
-            }
-            g_ws[(size_t)u * DD + j] = __expf(GC);
-        } else {
-            // X^T (warps 4-7)
-            for (int g = warp - 4; g < 32; g += 4) {
-                const int half = g >> 4, rb = (g >> 1) & 7, cb0 = (g & 1) * 4;
-                transpose4(sbase + D_X + half * TILE, rb, cb0, sbase + D_XT, half * 64);
-            }
+            hsum[h * DD + j] = acc;
+        }
+        // X^T, four 8x8 groups per warp
+        for (int g = warp; g < 32; g += NTH / 32) {
+            const int half = g >> 4, rb = (g >> 1) & 7, cb0 = (g & 1) * 4;
+            transpose4(sbase + D_X + half * TILE, rb, cb0, sbase + D_XT, half * 64);
         }
         __syncthreads();
-        transpose_pair(sbase + D_W, sbase + D_WT);
+        {
+            // G_{s,j} = (h ? S0_j : 0) + Gl, G_C = S0_j + S1_j; every exponent below is <= 0
+            const float s0 = hsum[j], s1 = hsum[DD + j];
+            const float base = h ? s0 : 0.f, tail = h ? s1 : s0 + s1;  // G_C - base
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int s_ = h * 32 + i;
+                const uint32_t off = pair_off(s_, j);
+                __nv_bfloat16 *bp = reinterpret_cast<__nv_bfloat16 *>(sm + D_B + off);
+                __nv_bfloat16 *vp = reinterpret_cast<__nv_bfloat16 *>(sm + D_V + off);
+                const float eta = __bfloat162float(*bp) * rinv[s_];
+                *vp = __float2bfloat16_rn(__expf(tail - Gl[i]) * eta * __bfloat162float(*vp));
+                *bp = __float2bfloat16_rn(__expf(base + Gl[i]));
+            }
+            if (h == 0) ws.g[(size_t)u * DD + j] = __expf(s0 + s1);
+        }
+        __syncthreads();
+        transpose_pair(sbase + D_V, sbase + D_WT);
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
@@ -257,39 +292,49 @@ __global__ void __launch_bounds__(NTH, 2)
             tc::fence_after_sync();
             issue_gemm(tbase, sbase + D_WT, 0, sbase + D_XT, 0, 1, 128);
             tc::mma_commit(bar);
+            tc::bulk_store(ws.wt + (size_t)u * WTIMG, sbase + D_WT, WTIMG);
+            tc::bulk_store(ws.e + (size_t)u * EIMG, sbase + D_B, EIMG);
+            tc::bulk_commit();
         }
         ok = tc::mbar_wait_timeout(bar, 0, kWaitNs);
         ok = __syncthreads_and(ok);
     }
     if (ok) {
+        // dS -> bf16 image over X and W (both consumed by the product)
         tc::fence_after_sync();
         const int quarter = warp & 3, chalf = warp >> 2, j = quarter * 32 + lane;
         const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
-        __nv_bfloat16 *dst = ds_ws + ((size_t)u * DD + j) * DD + chalf * 64;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
             float v[16];
             tc::tmem_ld16(tl + chalf * 64 + k4 * 16, v);
             tc::tmem_wait_ld();
-            *reinterpret_cast<uint4 *>(dst + k4 * 16) = pack8(&v[0]);
-            *reinterpret_cast<uint4 *>(dst + k4 * 16 + 8) = pack8(&v[8]);
+            *reinterpret_cast<uint4 *>(sm + D_X + chalf * 2 * TILE + tc::sw128(j, k4 * 2)) = pack8(&v[0]);
+            *reinterpret_cast<uint4 *>(sm + D_X + chalf * 2 * TILE + tc::sw128(j, k4 * 2 + 1)) = pack8(&v[8]);
+        }
+        tc::fence_proxy_async();
+        __syncthreads();
+        if (tid == ISSUER) {
+            tc::bulk_store(ws.dsimg + (size_t)u * DSIMG, sbase + D_X, DSIMG);
+            tc::bulk_commit();
         }
     } else {
         if (tid == 0) atomicAdd(&g_pc_wait_timeouts, 1u);
         (void)tc::mbar_wait_timeout(tbar, 0, kWaitNs);
     }
+    if (tid == ISSUER) tc::bulk_wait_read();
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tbase, 128);
 }
 
 // ============================================================ state scan
-// One thread per (b*H + h, row j, 8 columns): the state at every chunk start
-// (bf16, in the operand layout of pc_out_kernel: two K halves of 128 rows x
-// 128 bytes, swizzled), S_{c+1} = g_c S_c + dS_c in fp32, the final state.
-__global__ void __launch_bounds__(256)
-    pc_scan_kernel(FwdParams p, const __nv_bfloat16 *__restrict__ ds_ws, const float *__restrict__ g_ws,
-                   uint8_t *__restrict__ s_ws) {
+// One thread per (b*H + h, 16-byte column group of the state image): the
+// state at every chunk start (bf16, in the operand layout of pc_out_kernel:
+// two K halves of 128 rows x 128 bytes, swizzled), S_{c+1} = g_c S_c + dS_c
+// in fp32 (dS in the same image layout), the final state.  Eight chunks'
+// loads are issued ahead of their use.
+__global__ void __launch_bounds__(256) pc_scan_kernel(FwdParams p, PcWs ws) {
     const int nch = (p.L + CH - 1) / CH;
     const size_t gidx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t rowid = gidx >> 4;  // bh * 128 + j
@@ -300,16 +345,27 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int e = 0; e < 8; ++e) S[e] = p.init_state ? p.init_state[rowid * DD + i8 * 8 + e] : 0.f;
     const uint32_t soff = (uint32_t)(i8 >> 3) * (2 * TILE) + tc::sw128(j, i8 & 7);
-#pragma unroll 4
-    for (int c = 0; c < nch; ++c) {
-        const size_t u = bh * nch + c;
-        *reinterpret_cast<uint4 *>(s_ws + u * SIMG + soff) = pack8(S);
-        const uint4 d = *reinterpret_cast<const uint4 *>(ds_ws + (u * DD + j) * DD + i8 * 8);
-        const float g = g_ws[u * DD + j];
-        float dv[8];
-        unpack8(d, dv);
+    constexpr int AHEAD = 8;
+    for (int c = 0; c < nch; c += AHEAD) {
+        uint4 d[AHEAD];
+        float g[AHEAD];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) S[e] = g * S[e] + dv[e];
+        for (int k = 0; k < AHEAD; ++k) {
+            const size_t u = bh * nch + min(c + k, nch - 1);
+            d[k] = __ldcs(reinterpret_cast<const uint4 *>(ws.dsimg + u * DSIMG + soff));
+            g[k] = ws.g[u * DD + j];
+        }
+#pragma unroll
+        for (int k = 0; k < AHEAD; ++k) {
+            if (c + k < nch) {
+                const size_t u = bh * nch + c + k;
+                *reinterpret_cast<uint4 *>(ws.simg + u * SIMG + soff) = pack8(S);
+                float dv[8];
+                unpack8(d[k], dv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) S[e] = g[k] * S[e] + dv[e];
+            }
+        }
     }
     if (p.final_state) {
 #pragma unroll
@@ -320,32 +376,40 @@ __global__ void __launch_bounds__(256)
 // ============================================================ outputs
 namespace {
 constexpr uint32_t O_Q0 = 0, O_X0 = TILE, O_Q1 = 2 * TILE, O_X1 = 3 * TILE;  // [Q;X] per K half
-constexpr uint32_t O_V = 4 * TILE;     // values (tile pair)
-constexpr uint32_t O_B = 6 * TILE;     // per-channel beta (tile pair)
-constexpr uint32_t O_S = 8 * TILE;     // bf16 S_c: K half k at O_S + 2 TILE k (128 rows j)
-constexpr uint32_t O_Y = 12 * TILE;    // Yt[s][j] = e^{G_r-G_s} eta y (tile pair)
-constexpr uint32_t O_YT = 14 * TILE;   // Yt^T: 128 rows j x 64 s
-constexpr uint32_t O_PM = 16 * TILE;   // P o mask, rows t (the G table after it pads A to 128 rows)
-constexpr uint32_t O_G = 17 * TILE;    // fp32 G[t][j], row stride LDG
-constexpr uint32_t O_VEC = O_G + 64 * LDG * 4;  // |x_s|^2 [64], G_{r,j} [128]
-constexpr uint32_t O_BAR = O_VEC + (64 + 128 + 16) * 4;
+constexpr uint32_t O_PM = 0;           // P o mask (rows t) over [Q;X] once the first products are done
+constexpr uint32_t O_S = 4 * TILE;     // bf16 S_c: K half k at O_S + 2 TILE k (128 rows j); fallback: fp32 G
+constexpr uint32_t O_WT = 8 * TILE;    // W^T image (128 rows j x 64 s); fallback: values (tile pair)
+constexpr uint32_t O_E = 10 * TILE;    // e^{G_t} (tile pair); fallback: per-channel beta (tile pair)
+constexpr uint32_t O_VEC = 12 * TILE;  // g [128], 1/g [128], |x_s|^2 [64]
+constexpr uint32_t O_BAR = O_VEC + (2 * DD + 64) * 4;
 constexpr uint32_t O_SMEM = O_BAR + 64 + 1024;
+// The factorised form scales the intra-chunk sum by e^{-G_C}: safe while every
+// channel keeps G_C > -80, i.e. g = e^{G_C} above e^{-80}.
+constexpr float kMinGain = 1.80485139e-35f;
+
+// the fallback's fp32 G table: row s, column j ^ (s mod 32) (conflict-free
+// along either index)
+__device__ __forceinline__ int gidx(int s, int j) { return s * DD + (j ^ (s & 31)); }
 }  // namespace
 
 // One block per unit (b*H + h, chunk).  Tensor memory: [P;A] in columns
-// 0-63, then the intra-chunk product in 0-127; Q S_c^T in 128-255.
-__global__ void __launch_bounds__(NTH, 1)
-    pc_out_kernel(FwdParams p, const __grid_constant__ PcMaps maps, const uint8_t *s_ws) {
+// 0-63, then the intra-chunk product in 0-127; Q S_c^T in 128-255.  With
+// W[s][j] = e^{G_C-G_s} eta y from pc_delta_kernel,
+//   o_t[j] = e^{G_t} ( (Q S_c^T)[t][j] + e^{-G_C} ((P o mask) W)[t][j] ).
+// A chunk where some channel decays below e^{-80} reloads values and
+// betas and sums the intra-chunk terms one exponential at a time.
+__global__ void __launch_bounds__(NTH, 2) pc_out_kernel(FwdParams p, const __grid_constant__ PcMaps maps, PcWs ws) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = tc::smem_u32(smem_raw);
     uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
     const uint32_t sbase = tc::smem_u32(sm);
-    float *Gt = reinterpret_cast<float *>(sm + O_G);
-    float *sqn = reinterpret_cast<float *>(sm + O_VEC);
-    float *Gr = sqn + 64;
+    float *gv = reinterpret_cast<float *>(sm + O_VEC);
+    float *rg = gv + DD;
+    float *sqn = rg + DD;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + O_BAR);
     uint64_t *tbar = bar + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
+    uint64_t *fbar = bar + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 3);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, chalf = warp >> 2, row = quarter * 32 + lane;
@@ -355,23 +419,24 @@ __global__ void __launch_bounds__(NTH, 1)
     if (tid == 0) {
         tc::mbar_init(bar, 1);
         tc::mbar_init(tbar, 1);
+        tc::mbar_init(fbar, 1);
         tc::fence_mbar_init();
         const int krow = p.pairing == 0 ? c0 - 1 : c0;
-        tc::mbar_arrive_expect_tx(tbar, 8 * TILE + SIMG);
+        tc::mbar_arrive_expect_tx(tbar, 4 * TILE + SIMG + WTIMG + EIMG + DD * 4);
         tc::tma_load_3d(sbase + O_Q0, &maps.q, 0, c0, bh, tbar);
         tc::tma_load_3d(sbase + O_Q1, &maps.q, 64, c0, bh, tbar);
         tc::tma_load_3d(sbase + O_X0, &maps.k, 0, krow, bh, tbar);
         tc::tma_load_3d(sbase + O_X1, &maps.k, 64, krow, bh, tbar);
-        load_pair(sbase + O_V, &maps.v, c0, bh, tbar);
-        load_pair(sbase + O_B, &maps.beta, c0, bh, tbar);
-        tc::bulk_load(sbase + O_S, s_ws + (size_t)u * SIMG, SIMG, tbar);
+        tc::bulk_load(sbase + O_S, ws.simg + (size_t)u * SIMG, SIMG, tbar);
+        tc::bulk_load(sbase + O_WT, ws.wt + (size_t)u * WTIMG, WTIMG, tbar);
+        tc::bulk_load(sbase + O_E, ws.e + (size_t)u * EIMG, EIMG, tbar);
+        tc::bulk_load(sbase + O_VEC, ws.g + (size_t)u * DD, DD * 4, tbar);
     }
     __syncwarp();
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, 256);
         tc::tmem_relinquish();
     }
-    const float lam = tid < DD ? p.lambda[bh % p.H] : 0.f;
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -379,45 +444,35 @@ __global__ void __launch_bounds__(NTH, 1)
     const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
     bool ok = tc::mbar_wait_timeout(tbar, 0, kWaitNs);
     ok = __syncthreads_and(ok);
-    bool unsafe = false;
+    bool unsafe = false, fb_loading = false;
     if (ok) {
         samples_pair(sm, O_X0, 2 * TILE, p, bh, c0 == 0, sqn);
+        bool low = false;
+        if (tid < DD) {
+            const float g = gv[tid];
+            low = !(g > kMinGain);
+            rg[tid] = 1.f / g;
+        }
         tc::fence_proxy_async();
         tc::fence_before_sync();
-        __syncthreads();
+        unsafe = __syncthreads_or(low) != 0;
         if (tid == ISSUER) {
             tc::fence_after_sync();
-            issue_gemm(tbase, sbase + O_Q0, 2 * TILE, sbase + O_X0, 2 * TILE, 2, 64);         // [P ; X X^T]
-            issue_gemm(tbase + 128, sbase + O_Q0, 2 * TILE, sbase + O_S, 2 * TILE, 2, 128);   // Q S_c^T
+            issue_gemm(tbase, sbase + O_Q0, 2 * TILE, sbase + O_X0, 2 * TILE, 2, 64);        // [P ; X X^T]
+            issue_gemm(tbase + 128, sbase + O_Q0, 2 * TILE, sbase + O_S, 2 * TILE, 2, 128);  // Q S_c^T
             tc::mma_commit(bar);
         }
-        bool local_unsafe = false;
-        if (tid < DD) {
-            // channel j: cumulative log decay G_{s,j} (table) and Yt[s][j]
-            const int j = tid;
-            float G = 0.f, Gref = 0.f;
-            for (int s = 0; s < CH; ++s) {
-                const float n = sqn[s];
-                const float eta = n > 0.f ? __fdividef(pair_get(sm, O_B, s, j), p.eps + n) : 0.f;
-                G += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
-                Gt[s * LDG + j] = G;
-                if (s == 31) Gref = G;
-            }
-            Gr[j] = Gref;
-            local_unsafe = G <= kFactorMinLogDecay;  // e^{G_r-G_s} could leave the fp32 range
-            for (int s = 0; s < CH; ++s) {
-                const float n = sqn[s];
-                const float eta = n > 0.f ? __fdividef(pair_get(sm, O_B, s, j), p.eps + n) : 0.f;
-                const float yt = local_unsafe ? 0.f : __expf(Gref - Gt[s * LDG + j]) * eta * pair_get(sm, O_V, s, j);
-                *reinterpret_cast<__nv_bfloat16 *>(sm + O_Y + pair_off(s, j)) = __float2bfloat16_rn(yt);
-            }
+        if (unsafe && tid == 0) {
+            // values and betas over W^T and e^{G_t}, which this path does not read
+            tc::mbar_arrive_expect_tx(fbar, 4 * TILE);
+            load_pair(sbase + O_WT, &maps.v, c0, bh, fbar);
+            load_pair(sbase + O_E, &maps.beta, c0, bh, fbar);
         }
-        unsafe = __syncthreads_or(local_unsafe) != 0;
-        if (!unsafe) transpose_pair(sbase + O_Y, sbase + O_YT);
+        fb_loading = unsafe;
         ok = tc::mbar_wait_timeout(bar, 0, kWaitNs);
         ok = __syncthreads_and(ok);
     }
-    if (ok) {
+    if (ok && !unsafe) {
         tc::fence_after_sync();
         if (quarter < 2) {  // P o mask (s <= t) -> bf16, rows t
             const int t = row;
@@ -436,24 +491,63 @@ __global__ void __launch_bounds__(NTH, 1)
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
-        if (!unsafe) {
-            if (tid == ISSUER) {
-                tc::fence_after_sync();
-                issue_gemm(tbase, sbase + O_PM, 0, sbase + O_YT, 0, 1, 128);  // (P o mask) Yt
-                tc::mma_commit(bar);
-            }
-            ok = tc::mbar_wait_timeout(bar, 1, kWaitNs);
-            ok = __syncthreads_and(ok);
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_gemm(tbase, sbase + O_PM, 0, sbase + O_WT, 0, 1, 128);  // (P o mask) W
+            tc::mma_commit(bar);
         }
-    }
-    if (ok) {
-        tc::fence_after_sync();
-        if (quarter < 2) {
-            // o_t[j] = e^{G_t} (Q S_c^T)[t][j] + e^{G_t - G_r} ((P o mask) Yt)[t][j]
+        ok = tc::mbar_wait_timeout(bar, 1, kWaitNs);
+        ok = __syncthreads_and(ok);
+        if (ok && quarter < 2) {
+            tc::fence_after_sync();
             const int t = row;
             __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + ((size_t)bh * L + c0 + t) * DD;
-            float prow[CH];  // the fallback's P row
-            if (unsafe) {
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int jj = chalf * 64 + k4 * 16;
+                float iv[16], av[16], ev[16];
+                tc::tmem_ld16(tl + 128 + jj, iv);
+                tc::tmem_ld16(tl + jj, av);
+                unpack8(*reinterpret_cast<const uint4 *>(sm + O_E + pair_off(t, jj)), &ev[0]);
+                unpack8(*reinterpret_cast<const uint4 *>(sm + O_E + pair_off(t, jj + 8)), &ev[8]);
+                tc::tmem_wait_ld();
+                float o[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] = ev[i] * fmaf(rg[jj + i], av[i], iv[i]);
+                if (t < nt) {
+                    *reinterpret_cast<uint4 *>(dst + jj) = pack8(&o[0]);
+                    *reinterpret_cast<uint4 *>(dst + jj + 8) = pack8(&o[8]);
+                }
+            }
+        }
+    } else if (ok) {
+        // fallback: o_t[j] = e^{G_t} (Q S_c^T)[t][j] + sum_{s<=t} P[t][s] e^{G_t-G_s} eta_s y_s
+        ok = tc::mbar_wait_timeout(fbar, 0, kWaitNs);
+        ok = __syncthreads_and(ok);
+        fb_loading = !ok;
+        if (ok) {
+            float *Gt = reinterpret_cast<float *>(sm + O_S);
+            const float lam = p.lambda[bh % p.H];
+            for (int e = tid; e < CH * DD; e += NTH) {
+                const int s_ = e >> 7, j = e & (DD - 1);
+                const float n = sqn[s_];
+                const float eta = n > 0.f ? __fdividef(pair_get(sm, O_E, s_, j), p.eps + n) : 0.f;
+                Gt[gidx(s_, j)] = __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
+            }
+            __syncthreads();
+            if (tid < DD) {
+                float G = 0.f;
+                for (int s_ = 0; s_ < CH; ++s_) {
+                    G += Gt[gidx(s_, tid)];
+                    Gt[gidx(s_, tid)] = G;
+                }
+            }
+            __syncthreads();
+            tc::fence_after_sync();
+            if (quarter < 2) {
+                const int t = row;
+                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + ((size_t)bh * L + c0 + t) * DD;
+                float prow[CH];
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
                     float v[16];
@@ -462,42 +556,35 @@ __global__ void __launch_bounds__(NTH, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) prow[k4 * 16 + i] = v[i];
                 }
-            }
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-                const int jj = chalf * 64 + k4 * 16;
-                float iv[16], av[16];
-                tc::tmem_ld16(tl + 128 + jj, iv);
-                if (!unsafe) tc::tmem_ld16(tl + jj, av);
-                tc::tmem_wait_ld();
-                float o[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int j = jj + i;
-                    const float gt = Gt[t * LDG + j];
-                    float intra;
-                    if (!unsafe) {
-                        intra = __expf(gt - Gr[j]) * av[i];
-                    } else {
-                        // one exponential per term, every exponent <= 0
-                        intra = 0.f;
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int jj = chalf * 64 + k4 * 16;
+                    float iv[16];
+                    tc::tmem_ld16(tl + 128 + jj, iv);
+                    tc::tmem_wait_ld();
+                    float o[16];
+                    for (int i = 0; i < 16; ++i) {
+                        const int j = jj + i;
+                        const float gt = Gt[gidx(t, j)];
+                        float intra = 0.f;  // one exponential per term, every exponent <= 0
                         for (int s = 0; s <= t; ++s) {
                             const float n = sqn[s];
-                            const float eta = n > 0.f ? __fdividef(pair_get(sm, O_B, s, j), p.eps + n) : 0.f;
-                            intra += prow[s] * __expf(gt - Gt[s * LDG + j]) * eta * pair_get(sm, O_V, s, j);
+                            const float eta = n > 0.f ? __fdividef(pair_get(sm, O_E, s, j), p.eps + n) : 0.f;
+                            intra += prow[s] * __expf(gt - Gt[gidx(s, j)]) * eta * pair_get(sm, O_WT, s, j);
                         }
+                        o[i] = __expf(gt) * iv[i] + intra;
                     }
-                    o[i] = __expf(gt) * iv[i] + intra;
-                }
-                if (t < nt) {
-                    *reinterpret_cast<uint4 *>(dst + jj) = pack8(&o[0]);
-                    *reinterpret_cast<uint4 *>(dst + jj + 8) = pack8(&o[8]);
+                    if (t < nt) {
+                        *reinterpret_cast<uint4 *>(dst + jj) = pack8(&o[0]);
+                        *reinterpret_cast<uint4 *>(dst + jj + 8) = pack8(&o[8]);
+                    }
                 }
             }
         }
-    } else {
+    }
+    if (!ok) {
         if (tid == 0) atomicAdd(&g_pc_wait_timeouts, 1u);
         (void)tc::mbar_wait_timeout(tbar, 0, kWaitNs);
+        if (fb_loading) (void)tc::mbar_wait_timeout(fbar, 0, kWaitNs);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -554,14 +641,11 @@ int launch_pc_chunk(const FwdParams &p, cudaStream_t s) {
         !make_map(&maps.beta, p.beta, BH, p.L))
         return 1;
     void *ws = nullptr;
-    const size_t bytes = units * ((size_t)DSIMG + (size_t)DD * sizeof(float) + SIMG);
-    if (scratch_alloc(&ws, bytes, s) != cudaSuccess) {
+    if (scratch_alloc(&ws, units * WS_UNIT, s) != cudaSuccess) {
         cudaGetLastError();
         return -8;  // FALCON_ERR_ALLOC
     }
-    uint8_t *simg = static_cast<uint8_t *>(ws);
-    __nv_bfloat16 *ds = reinterpret_cast<__nv_bfloat16 *>(simg + units * SIMG);
-    float *g = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(ds) + units * DSIMG);
+    const PcWs w = pc_ws(ws, units);
     static bool attrs_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -570,10 +654,10 @@ int launch_pc_chunk(const FwdParams &p, cudaStream_t s) {
         cudaFuncSetAttribute(pc_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)O_SMEM);
         if (dev >= 0 && dev < 64) attrs_set[dev] = true;
     }
-    pc_delta_kernel<<<(unsigned)units, NTH, D_SMEM, s>>>(p, maps, ds, g);
+    pc_delta_kernel<<<(unsigned)units, NTH, D_SMEM, s>>>(p, maps, w);
     const size_t scan_threads = (size_t)BH * DD * 16;
-    pc_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, s>>>(p, ds, g, simg);
-    pc_out_kernel<<<(unsigned)units, NTH, O_SMEM, s>>>(p, maps, simg);
+    pc_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, s>>>(p, w);
+    pc_out_kernel<<<(unsigned)units, NTH, O_SMEM, s>>>(p, maps, w);
     const cudaError_t e = cudaGetLastError();
     scratch_free(ws, s);
     return e == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
