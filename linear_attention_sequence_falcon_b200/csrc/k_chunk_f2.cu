@@ -1,0 +1,396 @@
+// k_chunk_f2.cu -- chunk-parallel forward of Falcon-2 (regression, one step
+// and decay per value channel) on the tcgen05 tensor cores, bf16 inputs,
+// d_k = d_v = 128, chunk 64.
+//
+// Method: Falcon-2 takes eta and alpha per value channel j, i.e. per row of S
+// (page "借鉴40年前的设想！…", 02 (2)); the chunk form is parallel inside a
+// chunk and recurrent across chunks (page "Fast Weight Attention：用于持续学
+// 习的快速权重注意力", 核心方法 3).  Row j of S runs its own normalised LMS
+// recursion s_j <- alpha s_j + eta (y_j - s_j.x) x^T.  Entering a chunk with
+// S_0, the errors E[t][j] = y_{t,j} - s_j^{(t-1)}.x_t solve, per channel, the
+// unit lower-triangular system
+//   E_t + sum_{s<t} e^{G_{t-1}-G_s} eta_s A[t,s] E_s = y_t - e^{G_{t-1}} (S_0 x_t)_j,   A = X X^T,
+// with chunk-local G_t = sum_{r<=t} log alpha_r, and then
+//   o_t[j]   = e^{G_t} (S_0 q_t)_j + sum_{s<=t} e^{G_t-G_s} eta_s E_s (x_s.q_t)
+//   S_end[j] = e^{G_C} S_0[j] + sum_s e^{G_C-G_s} eta_s E_s x_s.
+// In the weights of the state update, Z_s = e^{G_C-G_s} eta_s E_s, the
+// system reads
+//   Z_t = w_t (y_t - e^{G_{t-1}} (S_0 x_t)_j) - (eta_t/alpha_t) sum_{s<t} A[t,s] Z_s,
+//   w_t = e^{G_C-G_t} eta_t,
+// every coefficient inside the fp32 range, and both remaining sums are
+// tensor-core products:
+//   o_t[j] = e^{G_t} ((S_0 Q^T)[j][t] + e^{-G_C} (Z^T (P o mask)^T)[j][t]),  P = Q X^T,
+//   S_end  = diag(e^{G_C}) S_0 + Z^T X.
+// The output form needs G_C > -80 in every channel; a chunk below that
+// solves for eta_s E_s with one exponential per term instead.
+//
+// One block per (b, h) walks the chunks; S stays in fp32 registers (thread:
+// row j, 64 columns) with its bf16 copy in shared memory as the operand of
+// S_0 [X;Q]^T.  The per-channel systems are solved by forward substitution,
+// one thread per channel.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc128.cuh"
+#include "tc_sm100.cuh"
+
+namespace falcon {
+
+namespace {
+
+__device__ unsigned int g_f2_wait_timeouts;
+
+constexpr uint32_t F_IN = 0;          // [X;Q] per K half: half k at 2 TILE k, X rows 0-63, Q rows 64-127
+constexpr uint32_t F_V = 4 * TILE;    // values (tile pair)
+constexpr uint32_t F_B = 6 * TILE;    // per-channel beta (tile pair)
+constexpr uint32_t F_S = 8 * TILE;    // bf16 S_0: K half k at F_S + 2 TILE k (128 rows j)
+constexpr uint32_t F_XT = 12 * TILE;  // X^T: 128 rows i x 64 s
+constexpr uint32_t F_ZT = 14 * TILE;  // Z^T: 128 rows j x 64 s
+constexpr uint32_t F_PM = 16 * TILE;  // P o mask (s <= t): 64 rows t x 64 s
+constexpr uint32_t F_G = 17 * TILE;   // fp32 G[t][j] at gidx(t, j)
+constexpr int LDA = 68;               // fp32 row stride of A (16-byte rows, conflict-free stores)
+constexpr uint32_t F_A = F_G + CH * DD * 4;     // fp32 A[t][s] for s < t, zero above
+constexpr uint32_t F_VEC = F_A + CH * LDA * 4;  // |x|^2 [64], 1/(eps+|x|^2) [64], half sums [256], G_C [128]
+constexpr uint32_t F_BAR = F_VEC + (64 + 64 + 2 * DD + DD) * 4;
+constexpr uint32_t F_SMEM = F_BAR + 64 + 1024;
+// tensor memory (512 columns)
+constexpr uint32_t C_PA = 0;    // [X;Q] X^T: A rows t (lanes 0-63), P rows t (lanes 64-127); 64 columns
+constexpr uint32_t C_S = 64;    // S_0 [X;Q]^T: lanes j; (S_0 X^T)[j][t] in 0-63, (S_0 Q^T)[j][t] in 64-127
+constexpr uint32_t C_DS = 192;  // Z^T X: lanes j, columns i
+constexpr uint32_t C_I = 320;   // Z^T (P o mask)^T: lanes j, columns t
+constexpr float kMinLogDecay = -80.f;
+
+// fp32 G table: row t, column j ^ (t mod 32) (conflict-free along either index)
+__device__ __forceinline__ int gidx(int t, int j) { return t * DD + (j ^ (t & 31)); }
+
+__device__ __forceinline__ void store_state_image(uint8_t *sm, int j, int half, const float *S) {
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8)
+        *reinterpret_cast<uint4 *>(sm + F_S + half * 2 * TILE + tc::sw128(j, c8)) = pack8(&S[c8 * 8]);
+}
+
+// bf16 element (t, s) of the 64-row P o mask tile
+__device__ __forceinline__ float pm_get(const uint8_t *sm, int t, int s) {
+    return __bfloat162float(
+        *reinterpret_cast<const __nv_bfloat16 *>(sm + F_PM + tc::sw128(t, s >> 3) + (uint32_t)(s & 7) * 2));
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __grid_constant__ PcMaps maps) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = tc::smem_u32(smem_raw);
+    uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = tc::smem_u32(sm);
+    float *Gt = reinterpret_cast<float *>(sm + F_G);
+    float *At = reinterpret_cast<float *>(sm + F_A);
+    float *sqn = reinterpret_cast<float *>(sm + F_VEC);
+    float *rinv = sqn + 64;
+    float *hsum = rinv + 64;
+    float *gcv = hsum + 2 * DD;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + F_BAR);
+    uint64_t *tbar = bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, chalf = warp >> 2, row = quarter * 32 + lane;
+    const int bh = blockIdx.x, L = p.L, nch = (L + CH - 1) / CH;
+    const float lam = p.lambda[bh % p.H];
+
+    // keys (rows c0-1 .. under the prefix pair) and q as [X;Q] per K half, v, beta
+    auto load_chunk = [&](int c) {
+        const int c0 = c * CH, krow = p.pairing == 0 ? c0 - 1 : c0;
+        tc::mbar_arrive_expect_tx(tbar, 8 * TILE);
+        tc::tma_load_3d(sbase + F_IN, &maps.k, 0, krow, bh, tbar);
+        tc::tma_load_3d(sbase + F_IN + TILE, &maps.q, 0, c0, bh, tbar);
+        tc::tma_load_3d(sbase + F_IN + 2 * TILE, &maps.k, 64, krow, bh, tbar);
+        tc::tma_load_3d(sbase + F_IN + 3 * TILE, &maps.q, 64, c0, bh, tbar);
+        load_pair(sbase + F_V, &maps.v, c0, bh, tbar);
+        load_pair(sbase + F_B, &maps.beta, c0, bh, tbar);
+    };
+    int issued = 0;  // chunk loads issued (thread 0)
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::mbar_init(tbar, 1);
+        tc::fence_mbar_init();
+        if (nch > 0) {
+            load_chunk(0);
+            issued = 1;
+        }
+    }
+    __syncwarp();
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    // S in fp32 registers: thread = (row j, column half chalf)
+    float S[64];
+#pragma unroll
+    for (int e = 0; e < 64; ++e)
+        S[e] = p.init_state ? p.init_state[((size_t)bh * DD + row) * DD + chalf * 64 + e] : 0.f;
+    store_state_image(sm, row, chalf, S);
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
+
+    bool ok = true;
+    uint32_t phase = 0;
+    for (int c = 0; c < nch; ++c) {
+        const int c0 = c * CH, nt = min(CH, L - c0);
+        ok = tc::mbar_wait_timeout(tbar, (uint32_t)(c & 1), kWaitNs);
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        // ---- samples, then S_0 [X;Q]^T and [X;Q] X^T on the tensor core
+        samples_pair(sm, F_IN, 2 * TILE, p, bh, c == 0, sqn, rinv);
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_gemm(tbase + C_PA, sbase + F_IN, 2 * TILE, sbase + F_IN, 2 * TILE, 2, 64);
+            issue_gemm(tbase + C_S, sbase + F_S, 2 * TILE, sbase + F_IN, 2 * TILE, 2, 128);
+            tc::mma_commit(bar);
+        }
+        // ---- log decays: thread (half h, channel jj), 32 running sums in registers; X^T
+        {
+            const int h = tid >> 7, jj = tid & (DD - 1);
+            float Gl[32];
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int t = h * 32 + i;
+                const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
+                acc += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
+                Gl[i] = acc;
+            }
+            hsum[h * DD + jj] = acc;
+            for (int g = warp; g < 32; g += NTH / 32) {
+                const int half = g >> 4, rb = (g >> 1) & 7, cb0 = (g & 1) * 4;
+                transpose4(sbase + F_IN + half * 2 * TILE, rb, cb0, sbase + F_XT, half * 64);
+            }
+            __syncthreads();
+            const float base = h ? hsum[jj] : 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) Gt[gidx(h * 32 + i, jj)] = base + Gl[i];
+            if (h == 0) gcv[jj] = hsum[jj] + hsum[DD + jj];
+        }
+        __syncthreads();
+        const bool unsafe = __syncthreads_or(tid < DD && !(gcv[tid] > kMinLogDecay)) != 0;
+        ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        phase ^= 1;
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        tc::fence_after_sync();
+        // ---- A (lanes 0-63) -> fp32 rows t, s < t; P (lanes 64-127) -> bf16 P o mask rows t, s <= t
+        {
+            const int t = row & 63;
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int cs = chalf * 2 + k2;
+                float v[16];
+                tc::tmem_ld16(tl + C_PA + cs * 16, v);
+                tc::tmem_wait_ld();
+                if (quarter < 2) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = cs * 16 + i < t ? v[i] : 0.f;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<float4 *>(At + t * LDA + cs * 16 + q4 * 4) =
+                            make_float4(v[q4 * 4], v[q4 * 4 + 1], v[q4 * 4 + 2], v[q4 * 4 + 3]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = cs * 16 + i <= t ? v[i] : 0.f;
+                    *reinterpret_cast<uint4 *>(sm + F_PM + tc::sw128(t, cs * 2)) = pack8(&v[0]);
+                    *reinterpret_cast<uint4 *>(sm + F_PM + tc::sw128(t, cs * 2 + 1)) = pack8(&v[8]);
+                }
+            }
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        // ---- per-channel systems (warps 0-3, thread = channel jj = tensor-memory lane)
+        if (tid < DD) {
+            const int jj = tid;
+            const float gc = gcv[jj];
+            float Z[64];
+#pragma unroll
+            for (int s = 0; s < 64; ++s) Z[s] = 0.f;
+            if (!unsafe) {
+                float Gprev = 0.f;
+#pragma unroll
+                for (int tb = 0; tb < 4; ++tb) {
+                    float xs[16];
+                    tc::tmem_ld16(tl + C_S + tb * 16, xs);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int t = tb * 16 + i;
+                        const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
+                        const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
+                        const float G = Gt[gidx(t, jj)];
+                        const float r = __expf(gc - G) * eta * (pair_get(sm, F_V, t, jj) - __expf(Gprev) * xs[i]);
+                        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                        for (int s = 0; s < t; s += 4) {
+                            const float4 a = *reinterpret_cast<const float4 *>(At + t * LDA + s);
+                            a0 = fmaf(a.x, Z[s], a0);
+                            a1 = fmaf(a.y, Z[s + 1], a1);
+                            a2 = fmaf(a.z, Z[s + 2], a2);
+                            a3 = fmaf(a.w, Z[s + 3], a3);
+                        }
+                        Z[t] = r - __fdividef(eta, alpha) * ((a0 + a1) + (a2 + a3));
+                        Gprev = G;
+                    }
+                }
+            } else {
+                // F_s = eta_s E_s with one exponential per term (every exponent <= 0),
+                // the outputs from it, then Z_s = e^{G_C-G_s} F_s
+                float xs[64], F[64];
+#pragma unroll
+                for (int tb = 0; tb < 4; ++tb) {
+                    float v[16];
+                    tc::tmem_ld16(tl + C_S + tb * 16, v);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) xs[tb * 16 + i] = v[i];
+                }
+                float Gprev = 0.f;
+#pragma unroll 1
+                for (int t = 0; t < CH; ++t) {
+                    const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
+                    float a = 0.f;
+                    for (int s = 0; s < t; ++s) a += __expf(Gprev - Gt[gidx(s, jj)]) * At[t * LDA + s] * F[s];
+                    F[t] = eta * (pair_get(sm, F_V, t, jj) - __expf(Gprev) * xs[t] - a);
+                    Gprev = Gt[gidx(t, jj)];
+                }
+#pragma unroll
+                for (int tb = 0; tb < 4; ++tb) {
+                    float v[16];
+                    tc::tmem_ld16(tl + C_S + 64 + tb * 16, v);  // (S_0 Q^T)[j][t]
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) xs[tb * 16 + i] = v[i];
+                }
+#pragma unroll 1
+                for (int t = 0; t < nt; ++t) {
+                    const float G = Gt[gidx(t, jj)];
+                    float o = __expf(G) * xs[t];
+                    for (int s = 0; s <= t; ++s) o += __expf(G - Gt[gidx(s, jj)]) * pm_get(sm, t, s) * F[s];
+                    static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + jj] = __float2bfloat16_rn(o);
+                }
+#pragma unroll 1
+                for (int s = 0; s < CH; ++s) F[s] *= __expf(gc - Gt[gidx(s, jj)]);
+#pragma unroll
+                for (int s = 0; s < 64; ++s) Z[s] = F[s];
+            }
+            // Z^T row jj
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8)
+                *reinterpret_cast<uint4 *>(sm + F_ZT + tc::sw128(jj, c8)) = pack8(&Z[c8 * 8]);
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        // the chunk's inputs are consumed: the next chunk's loads run under the rest
+        if (tid == 0 && c + 1 < nch) {
+            load_chunk(c + 1);
+            ++issued;
+        }
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_gemm(tbase + C_DS, sbase + F_ZT, 0, sbase + F_XT, 0, 1, 128);                // Z^T X
+            if (!unsafe) issue_gemm(tbase + C_I, sbase + F_ZT, 0, sbase + F_PM, 0, 1, 64);    // Z^T (P o mask)^T
+            tc::mma_commit(bar);
+        }
+        ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        phase ^= 1;
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const float gcj = gcv[row];
+        if (!unsafe) {
+            // o_t[j] for t in 32 chalf .. 32 chalf + 31
+            const float ig = __expf(-gcj);
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int t0 = chalf * 32 + k2 * 16;
+                float iv[16], av[16];
+                tc::tmem_ld16(tl + C_S + 64 + t0, iv);
+                tc::tmem_ld16(tl + C_I + t0, av);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int t = t0 + i;
+                    const float o = __expf(Gt[gidx(t, row)]) * fmaf(ig, av[i], iv[i]);
+                    if (t < nt)
+                        static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + row] =
+                            __float2bfloat16_rn(o);
+                }
+            }
+        }
+        // S_end = diag(e^{G_C}) S_0 + Z^T X
+        {
+            const float g = __expf(gcj);
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                float dv[16];
+                tc::tmem_ld16(tl + C_DS + chalf * 64 + k4 * 16, dv);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) S[k4 * 16 + i] = fmaf(g, S[k4 * 16 + i], dv[i]);
+            }
+            store_state_image(sm, row, chalf, S);
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+    }
+    if (ok && p.final_state) {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) p.final_state[((size_t)bh * DD + row) * DD + chalf * 64 + e] = S[e];
+    }
+    if (!ok && tid == 0) {
+        atomicAdd(&g_f2_wait_timeouts, 1u);
+        // a load still in flight must land before the block leaves
+        if (issued > 0) (void)tc::mbar_wait_timeout(tbar, (uint32_t)((issued - 1) & 1), kWaitNs);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 512);
+}
+
+int launch_f2_chunk(const FwdParams &p, cudaStream_t s) {
+    const bool shape_ok = p.variant == F2 && p.dk == DD && p.dv == DD && p.chunk == CH;
+    auto al16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+    if (!shape_ok || !al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.beta) || !al16(p.out))
+        return 1;
+    const int BH = p.B * p.H;
+    if (BH <= 0 || p.L <= 0) return 1;
+    PcMaps maps;
+    if (!make_map(&maps.q, p.q, BH, p.L) || !make_map(&maps.k, p.k, BH, p.L) || !make_map(&maps.v, p.v, BH, p.L) ||
+        !make_map(&maps.beta, p.beta, BH, p.L))
+        return 1;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        cudaFuncSetAttribute(f2_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)F_SMEM);
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    f2_chunk_kernel<<<(unsigned)BH, NTH, F_SMEM, s>>>(p, maps);
+    return cudaGetLastError() == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
+}
+
+unsigned int f2_wait_timeouts() {
+    unsigned int v = 0;
+    cudaMemcpyFromSymbol(&v, g_f2_wait_timeouts, sizeof(v));
+    return v;
+}
+
+}  // namespace falcon

@@ -56,6 +56,11 @@ unsigned int split_wait_timeouts();
 // not cover.
 int launch_pc_chunk(const FwdParams &p, cudaStream_t s);
 unsigned int pc_wait_timeouts();
+// bf16 Falcon-2 chunk-parallel forward, d_k = d_v = 128, chunk 64, on tcgen05
+// (one block per head, per-channel forward substitution); returns 1 for
+// shapes it does not cover.
+int launch_f2_chunk(const FwdParams &p, cudaStream_t s);
+unsigned int f2_wait_timeouts();
 template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
 

@@ -124,3 +124,7 @@ def test_empty_segment_keeps_the_state(F):
 
 def test_carry_falcon2a_d128_tensor_core_path(F):
     check_segment(F, "F2A", "chunk", "bf16", 1, 3, 200, 128, 128, 64, 81)
+
+
+def test_carry_falcon2_d128_tensor_core_path(F):
+    check_segment(F, "F2", "chunk", "bf16", 1, 3, 200, 128, 128, 64, 91)

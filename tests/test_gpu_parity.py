@@ -312,3 +312,35 @@ def test_falcon2a_d128_decay_floor(F):
     decay factor is one exponential of a difference."""
     d = gen.draw("F2A", 1, 2, 130, 128, 128, seed=76, dtype="bf16", lam=0.9, key_scale=0.03)
     check(F, d, "F2A", "chunk", chunk=64, phi="identity")
+
+
+# --------------------------------------------------------------- the per-channel regression (Falcon-2, d = 128) tensor-core path
+
+@pytest.mark.parametrize("L", [64, 200, 513])
+def test_falcon2_d128_tensor_core_path(F, L):
+    """bf16 Falcon-2, d_k = d_v = 128, chunk 64: one block per head, the
+    per-channel systems by forward substitution, the products on tcgen05;
+    one chunk, a ragged tail, many chunks."""
+    d = gen.draw("F2", 2, 3, L, 128, 128, seed=80 + L, dtype="bf16", lam=0.02)
+    check(F, d, "F2", "chunk", chunk=64)
+
+
+@pytest.mark.parametrize("pairing,phi", [("same_step", "l2"), ("prefix", "identity")])
+def test_falcon2_d128_pairing_and_feature_map(F, pairing, phi):
+    d = gen.draw("F2", 1, 2, 150, 128, 128, seed=84, dtype="bf16", key_scale=0.09)
+    check(F, d, "F2", "chunk", chunk=64, pairing=pairing, phi=phi)
+
+
+def test_falcon2_d128_strong_forgetting(F):
+    """lambda = 0.999: per-channel chunk log-decays around -45, inside the
+    range of the factorised outputs."""
+    d = gen.draw("F2", 1, 3, 200, 128, 128, seed=85, dtype="bf16", lam=0.999)
+    check(F, d, "F2", "chunk", chunk=64)
+
+
+def test_falcon2_d128_decay_floor(F):
+    """Tiny keys under the identity map with lambda = 0.9: alpha sits on the
+    2^-20 floor, the chunk log-decay is far below -80, and the block solves
+    for eta E with one exponential per term."""
+    d = gen.draw("F2", 1, 2, 130, 128, 128, seed=86, dtype="bf16", lam=0.9, key_scale=0.03)
+    check(F, d, "F2", "chunk", chunk=64, phi="identity")
