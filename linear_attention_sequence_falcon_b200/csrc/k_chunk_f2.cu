@@ -42,6 +42,32 @@ namespace {
 
 __device__ unsigned int g_f2_wait_timeouts;
 
+#ifdef FALCON_TC_DEBUG
+// block 0, thread 0: SM cycles per phase summed over the chunks
+__device__ long long *g_f2_tim;
+#define F2T_INIT()                  \
+    long long f2t_acc_[8] = {0};    \
+    long long f2t_prev_ = clock64(); \
+    const bool f2t_on_ = blockIdx.x == 0 && threadIdx.x == 0
+#define F2T(k)                                      \
+    do {                                            \
+        if (f2t_on_) {                              \
+            const long long n_ = clock64();         \
+            f2t_acc_[k] += n_ - f2t_prev_;          \
+            f2t_prev_ = n_;                         \
+        }                                           \
+    } while (0)
+#define F2T_END()                                                             \
+    do {                                                                      \
+        if (f2t_on_ && g_f2_tim)                                              \
+            for (int i_ = 0; i_ < 8; ++i_) g_f2_tim[i_] = f2t_acc_[i_];        \
+    } while (0)
+#else
+#define F2T_INIT()
+#define F2T(k)
+#define F2T_END()
+#endif
+
 constexpr uint32_t F_IN = 0;          // [X;Q] per K half: half k at 2 TILE k, X rows 0-63, Q rows 64-127
 constexpr uint32_t F_V = 4 * TILE;    // values (tile pair)
 constexpr uint32_t F_B = 6 * TILE;    // per-channel beta (tile pair)
@@ -140,16 +166,19 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
 
     bool ok = true;
     uint32_t phase = 0;
+    F2T_INIT();
     for (int c = 0; c < nch; ++c) {
         const int c0 = c * CH, nt = min(CH, L - c0);
         ok = tc::mbar_wait_timeout(tbar, (uint32_t)(c & 1), kWaitNs);
         ok = __syncthreads_and(ok);
         if (!ok) break;
+        F2T(0);
         // ---- samples, then S_0 [X;Q]^T and [X;Q] X^T on the tensor core
         samples_pair(sm, F_IN, 2 * TILE, p, bh, c == 0, sqn, rinv);
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        F2T(1);
         if (tid == ISSUER) {
             tc::fence_after_sync();
             issue_gemm(tbase + C_PA, sbase + F_IN, 2 * TILE, sbase + F_IN, 2 * TILE, 2, 64);
@@ -181,10 +210,12 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
         }
         __syncthreads();
         const bool unsafe = __syncthreads_or(tid < DD && !(gcv[tid] > kMinLogDecay)) != 0;
+        F2T(2);
         ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
         phase ^= 1;
         ok = __syncthreads_and(ok);
         if (!ok) break;
+        F2T(3);
         tc::fence_after_sync();
         // ---- A (lanes 0-63) -> fp32 rows t, s < t; P (lanes 64-127) -> bf16 P o mask rows t, s <= t
         {
@@ -213,6 +244,7 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        F2T(4);
         tc::fence_after_sync();
         // ---- per-channel systems (warps 0-3, thread = channel jj = tensor-memory lane)
         if (tid < DD) {
@@ -297,6 +329,7 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        F2T(5);
         // the chunk's inputs are consumed: the next chunk's loads run under the rest
         if (tid == 0 && c + 1 < nch) {
             load_chunk(c + 1);
@@ -312,6 +345,7 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
         phase ^= 1;
         ok = __syncthreads_and(ok);
         if (!ok) break;
+        F2T(6);
         tc::fence_after_sync();
         const float gcj = gcv[row];
         if (!unsafe) {
@@ -350,7 +384,9 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        F2T(7);
     }
+    F2T_END();
     if (ok && p.final_state) {
 #pragma unroll
         for (int e = 0; e < 64; ++e) p.final_state[((size_t)bh * DD + row) * DD + chalf * 64 + e] = S[e];
@@ -386,6 +422,12 @@ int launch_f2_chunk(const FwdParams &p, cudaStream_t s) {
     f2_chunk_kernel<<<(unsigned)BH, NTH, F_SMEM, s>>>(p, maps);
     return cudaGetLastError() == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
 }
+
+#ifdef FALCON_TC_DEBUG
+extern "C" int falcon_f2_debug_timer_set(long long *ptr) {
+    return cudaMemcpyToSymbol(g_f2_tim, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 unsigned int f2_wait_timeouts() {
     unsigned int v = 0;
