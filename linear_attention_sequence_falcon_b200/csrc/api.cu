@@ -73,6 +73,7 @@ int fwd_impl(falcon_variant variant, falcon_form form, falcon_dtype dtype, falco
             int tc = launch_split_chunk(p, stream);
             if (tc == 1) tc = launch_pc_chunk(p, stream);
             if (tc == 1) tc = launch_f2_chunk(p, stream);
+            if (tc == 1) tc = launch_w_chunk(p, stream);
             if (tc != 1) return launched(tc);  // 1: shape not covered by the tensor-core kernels
         }
         return launched(bf16 ? launch_span_chunk<__nv_bfloat16>(p, stream) : launch_span_chunk<float>(p, stream));
@@ -164,7 +165,7 @@ extern "C" int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_d
 
 extern "C" int falcon_device_wait_timeouts(unsigned int *count) {
     if (!count) return FALCON_ERR_NULL;
-    *count = split_wait_timeouts() + pc_wait_timeouts() + f2_wait_timeouts();
+    *count = split_wait_timeouts() + pc_wait_timeouts() + f2_wait_timeouts() + w_wait_timeouts();
     return cudaGetLastError() == cudaSuccess ? FALCON_OK : FALCON_ERR_LAUNCH;
 }
 

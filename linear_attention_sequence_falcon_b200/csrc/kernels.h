@@ -61,6 +61,11 @@ unsigned int pc_wait_timeouts();
 // shapes it does not cover.
 int launch_f2_chunk(const FwdParams &p, cudaStream_t s);
 unsigned int f2_wait_timeouts();
+// bf16 Falcon-3/3A chunk-parallel forward, d_k = d_v = 64, chunk 64, window
+// 2..4, on tcgen05 (one block per head, the windowed system in token order);
+// returns 1 for shapes it does not cover.
+int launch_w_chunk(const FwdParams &p, cudaStream_t s);
+unsigned int w_wait_timeouts();
 template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
 

@@ -128,3 +128,10 @@ def test_carry_falcon2a_d128_tensor_core_path(F):
 
 def test_carry_falcon2_d128_tensor_core_path(F):
     check_segment(F, "F2", "chunk", "bf16", 1, 3, 200, 128, 128, 64, 91)
+
+
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+def test_carry_window_tensor_core_path(F, variant):
+    """window 3: the carried window samples (values included) and x_prev
+    enter the first chunk's sample rows."""
+    check_segment(F, variant, "chunk", "bf16", 1, 3, 200, 64, 64, 64, 141)

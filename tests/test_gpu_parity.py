@@ -344,3 +344,39 @@ def test_falcon2_d128_decay_floor(F):
     for eta E with one exponential per term."""
     d = gen.draw("F2", 1, 2, 130, 128, 128, seed=86, dtype="bf16", lam=0.9, key_scale=0.03)
     check(F, d, "F2", "chunk", chunk=64, phi="identity")
+
+
+# --------------------------------------------------------------- the windowed (Falcon-3/3A, d = 64) tensor-core path
+
+@pytest.mark.parametrize("w", [2, 3, 4])
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+@pytest.mark.parametrize("L", [1, 5, 64, 65, 200])
+def test_window_tensor_core_path(F, variant, w, L):
+    """bf16 Falcon-3/3A, d_k = d_v = 64, chunk 64: one block per head, the
+    windowed system in token order, the products on tcgen05; one chunk and a
+    ragged tail over several chunks."""
+    d = gen.draw(variant, 2, 3, L, 64, 64, seed=100 + 10 * w + L, dtype="bf16")
+    check(F, d, variant, "chunk", chunk=64, window=w)
+
+
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+def test_window_tensor_core_strong_forgetting(F, variant):
+    """lambda = 0.999 with a window of 4: chunk log-decays far below zero but
+    above -80, inside the factorised form."""
+    d = gen.draw(variant, 1, 3, 200, 64, 64, seed=131, dtype="bf16", lam=0.999)
+    check(F, d, variant, "chunk", chunk=64, window=4)
+
+
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+def test_window_tensor_core_decay_floor(F, variant):
+    """Tiny keys under the identity map with lambda = 0.9: alpha on the 2^-20
+    floor, chunk log-decays far below -80; those chunks run token by token."""
+    d = gen.draw(variant, 1, 2, 150, 64, 64, seed=132, dtype="bf16", lam=0.9, key_scale=0.03)
+    check(F, d, variant, "chunk", chunk=64, window=4, phi="identity")
+
+
+@pytest.mark.parametrize("pairing,phi", [("same_step", "l2"), ("prefix", "identity")])
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+def test_window_tensor_core_pairing_and_feature_map(F, variant, pairing, phi):
+    d = gen.draw(variant, 1, 2, 150, 64, 64, seed=133, dtype="bf16", key_scale=0.2)
+    check(F, d, variant, "chunk", chunk=64, window=4, pairing=pairing, phi=phi)
