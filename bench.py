@@ -37,8 +37,8 @@ DECODE = dict(variant="F2A", N=64, H=16, dk=128, dv=128, lam=0.02, seed=20260005
 CSRC = os.path.join(ROOT, "linear_attention_sequence_falcon_b200", "csrc")
 PROFILED = {
     "chunk": ("chunk_local_kernel_falcon1_8x12x2048x64.md", ("k_chunk_split.cu", "tc_sm100.cuh", "common.cuh",
-                                                               "kernels.h")),
-    "decode": ("decode1_kernel_falcon2A_64x16x128x128.md", ("k_decode.cu", "common.cuh", "kernels.h")),
+                                                               "params.h")),
+    "decode": ("decode1_kernel_falcon2A_64x16x128x128.md", ("k_decode.cu", "common.cuh", "params.h")),
 }
 # GPU spin (cycles) queued before every timed step, so the host has enqueued
 # the step's launches before its start event is reached

@@ -51,6 +51,32 @@ constexpr float kMinLogDecay = -80.f;
 
 __device__ unsigned int g_w_wait_timeouts;
 
+#ifdef FALCON_TC_DEBUG
+// block 0, thread 0: SM cycles per phase summed over the chunks
+__device__ long long *g_w_tim;
+#define WT_INIT()                    \
+    long long wt_acc_[8] = {0};      \
+    long long wt_prev_ = clock64();  \
+    const bool wt_on_ = blockIdx.x == 0 && threadIdx.x == 0
+#define WT(k)                                  \
+    do {                                       \
+        if (wt_on_) {                          \
+            const long long n_ = clock64();    \
+            wt_acc_[k] += n_ - wt_prev_;       \
+            wt_prev_ = n_;                     \
+        }                                      \
+    } while (0)
+#define WT_END()                                                         \
+    do {                                                                 \
+        if (wt_on_ && g_w_tim)                                           \
+            for (int i_ = 0; i_ < 8; ++i_) g_w_tim[i_] = wt_acc_[i_];     \
+    } while (0)
+#else
+#define WT_INIT()
+#define WT(k)
+#define WT_END()
+#endif
+
 // shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t W_XE = 0;            // sample rows x_r (128 rows; rows >= 64+B_w-1 zero up to NR)
 constexpr uint32_t W_VE = 2 * TILE;     // sample rows y_r (128 rows)
@@ -219,6 +245,7 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
 
     bool ok = true;
     uint32_t phase = 0;
+    WT_INIT();
     for (int c = 0; c < nch; ++c) {
         const int c0 = c * CH, nt = min(CH, L - c0);
         if (tid < CH) {
@@ -228,6 +255,7 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
         ok = tc::mbar_wait_timeout(tbar, (uint32_t)(c & 1), kWaitNs);
         ok = __syncthreads_and(ok);
         if (!ok) break;
+        WT(0);
         // ---- samples: rows r < MM normalised in place (four threads per row), rows MM..NR-1 zero
         for (int rr = tid >> 2; rr < NR; rr += NTH / 4) {  // a warp's lanes share the trip count
             const int part = tid & 3, i = c0 - BW + 1 + rr;
@@ -279,6 +307,7 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        WT(1);
         // ---- products: Gram and P over the sample rows, S_0 X^T, S_0 Q^T
         if (tid == ISSUER) {
             tc::fence_after_sync();
@@ -331,10 +360,12 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
         __syncthreads();
         const float GC = misc[2];
         const bool unsafe = !(GC > kMinLogDecay);
+        WT(2);
         ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
         phase ^= 1;
         ok = __syncthreads_and(ok);
         if (!ok) break;
+        WT(3);
         tc::fence_after_sync();
         if (!unsafe) {
             // ---- Gram rows r < 68 (lanes 0-79) -> fp32; P (lanes 0-63) -> P o (r <= t) bf16 and the band
@@ -388,6 +419,7 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
             tc::fence_proxy_async();
             tc::fence_before_sync();
             __syncthreads();
+            WT(4);
             tc::fence_after_sync();
             // ---- the chunk's system in token order (warps 0-1: thread = channel j = lane)
             if (tid < DD) {
@@ -450,6 +482,7 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
             tc::fence_proxy_async();
             tc::fence_before_sync();
             __syncthreads();
+            WT(5);
             if (tid == 0 && c + 1 < nch) {
                 load_chunk(c + 1);
                 ++issued;
@@ -464,6 +497,7 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
             phase ^= 1;
             ok = __syncthreads_and(ok);
             if (!ok) break;
+            WT(6);
             tc::fence_after_sync();
             if (sthr) {
                 const int j = row;
@@ -566,7 +600,9 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        WT(7);
     }
+    WT_END();
     if (ok && sthr && p.final_state) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) p.final_state[((size_t)bh * DD + row) * DD + chalf * 32 + e] = S[e];
@@ -644,6 +680,12 @@ int launch_w_chunk(const FwdParams &p, cudaStream_t s) {
         default: return launch_w<4>(p, maps, s);
     }
 }
+
+#ifdef FALCON_TC_DEBUG
+extern "C" int falcon_w_debug_timer_set(long long *ptr) {
+    return cudaMemcpyToSymbol(g_w_tim, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 unsigned int w_wait_timeouts() {
     unsigned int v = 0;
