@@ -47,12 +47,13 @@ __device__ unsigned int g_pc_wait_timeouts;
 
 // ============================================================ dS kernel
 namespace {
-constexpr uint32_t D_X = 0;            // raw keys -> X (tile pair); with D_V the dS image after the product
+constexpr uint32_t D_X = 0;            // raw keys -> X (tile pair) -> W^T (128 rows j x 64 s) once X^T is made;
+                                       // with D_V the dS image after the product
+constexpr uint32_t D_WT = D_X;
 constexpr uint32_t D_V = 2 * TILE;     // values -> W[s][j] = e^{G_C-G_s} eta y in place (tile pair)
 constexpr uint32_t D_B = 4 * TILE;     // per-channel beta -> E[s][j] = e^{G_s} in place (tile pair)
-constexpr uint32_t D_WT = 6 * TILE;    // W^T: 128 rows j x 64 s
-constexpr uint32_t D_XT = 8 * TILE;    // X^T: 128 rows i x 64 s
-constexpr uint32_t D_VEC = 10 * TILE;  // |x_s|^2 [64], 1/(eps+|x_s|^2) [64], half-chunk log-decay sums [2][128]
+constexpr uint32_t D_XT = 6 * TILE;    // X^T: 128 rows i x 64 s
+constexpr uint32_t D_VEC = 8 * TILE;   // |x_s|^2 [64], 1/(eps+|x_s|^2) [64], half-chunk log-decay sums [2][128]
 constexpr uint32_t D_BAR = D_VEC + (64 + 64 + 2 * DD) * 4;
 constexpr uint32_t D_SMEM = D_BAR + 64 + 1024;
 constexpr uint32_t WTIMG = 2 * TILE;   // W^T image handed to pc_out_kernel
@@ -81,7 +82,7 @@ __host__ __device__ inline PcWs pc_ws(void *base, size_t units) {
 // 32 log-decays summed in registers, the two halves joined through shared
 // memory.  Outputs: dS (bf16 image, the layout of the state operand), g =
 // e^{G_C}, and for pc_out_kernel W^T (its intra-chunk operand) and e^{G_t}.
-__global__ void __launch_bounds__(NTH, 2) pc_delta_kernel(FwdParams p, const __grid_constant__ PcMaps maps, PcWs ws) {
+__global__ void __launch_bounds__(NTH, 3) pc_delta_kernel(FwdParams p, const __grid_constant__ PcMaps maps, PcWs ws) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = tc::smem_u32(smem_raw);
     uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -172,10 +173,12 @@ __global__ void __launch_bounds__(NTH, 2) pc_delta_kernel(FwdParams p, const __g
             tc::bulk_commit();
         }
         ok = tc::mbar_wait_timeout(bar, 0, kWaitNs);
+        // the W^T image leaves shared memory before dS is staged over it
+        if (tid == ISSUER) tc::bulk_wait_read();
         ok = __syncthreads_and(ok);
     }
     if (ok) {
-        // dS -> bf16 image over X and W (both consumed by the product)
+        // dS -> bf16 image over W^T and W (both consumed by the product)
         tc::fence_after_sync();
         const int quarter = warp & 3, chalf = warp >> 2, j = quarter * 32 + lane;
         const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
