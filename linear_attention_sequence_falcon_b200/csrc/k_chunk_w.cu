@@ -421,49 +421,81 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
             __syncthreads();
             WT(4);
             tc::fence_after_sync();
-            // ---- the chunk's system in token order (warps 0-1: thread = channel j = lane)
+            // ---- the chunk's system in token order (warps 0-1: thread = channel j = lane),
+            //      in blocks of 8 tokens: the sums over rows final before a block are one
+            //      batch of independent dot products; only the rows the block itself
+            //      still adds to (t0 .. t0+7+BW-1, in registers) are walked token by token
             if (tid < DD) {
                 const int j = tid;
                 float *za = Za + j * LDZ;
                 const float *sx = SXt + j * LDZ;
+                constexpr int NB = 8, RB = NB + BW - 1;  // tokens and rows of a block
+                float zb[RB];                            // rows t0 .. t0+RB-1
+#pragma unroll
+                for (int k = 0; k < RB; ++k) zb[k] = 0.f;
 #pragma unroll 1
                 for (int tb = 0; tb < 4; ++tb) {
                     float bnd[16];
 #pragma unroll
-                    for (int ii = 0; ii < 16; ++ii) {
-                        const int t = tb * 16 + ii;
-                        const float wt = vw[t];
-                        float acc[BW];
+                    for (int hb = 0; hb < 2; ++hb) {
+                        const int t0 = tb * 16 + hb * NB;
+                        float cr[NB][BW];
 #pragma unroll
-                        for (int m = 0; m < BW; ++m) acc[m] = 0.f;
+                        for (int i = 0; i < NB; ++i)
+#pragma unroll
+                            for (int m = 0; m < BW; ++m) cr[i][m] = 0.f;
                         if (reg) {
-                            // rows r' < t + BW - 1 carry contributions of earlier tokens
-                            const int nq = (t + BW + 2) >> 2;
-#pragma unroll 2
-                            for (int q = 0; q < nq; ++q) {
+                            // rows r' < t0: final, in shared memory
+                            for (int q = 0; q < (t0 >> 2); ++q) {
                                 const float4 z4 = *reinterpret_cast<const float4 *>(za + q * 4);
 #pragma unroll
-                                for (int m = 0; m < BW; ++m) {
-                                    const float4 a4 = *reinterpret_cast<const float4 *>(At + (t + m) * LDA + q * 4);
-                                    acc[m] = fmaf(a4.x, z4.x, fmaf(a4.y, z4.y, fmaf(a4.z, z4.z, fmaf(a4.w, z4.w, acc[m]))));
+                                for (int rr = 0; rr < RB; ++rr) {
+                                    const float4 a4 = *reinterpret_cast<const float4 *>(At + (t0 + rr) * LDA + q * 4);
+                                    const float d = fmaf(a4.x, z4.x, fmaf(a4.y, z4.y, fmaf(a4.z, z4.z, a4.w * z4.w)));
+#pragma unroll
+                                    for (int i = 0; i < NB; ++i)
+#pragma unroll
+                                        for (int m = 0; m < BW; ++m)
+                                            if (i + m == rr) cr[i][m] += d;
                                 }
                             }
                         }
-                        const float gm = vgm1[t], kt = vkap[t];
 #pragma unroll
-                        for (int m = 0; m < BW; ++m) {
-                            const int r = t + m;
-                            const float y = tile_get(sm, W_VE, r, j);
-                            const float z = reg ? wt * (y - gm * sx[r]) - kt * acc[m] : wt * y;
-                            za[r] += z;
+                        for (int i = 0; i < NB; ++i) {
+                            const int t = t0 + i;
+                            const float wt = vw[t], gm = vgm1[t], kt = vkap[t];
+#pragma unroll
+                            for (int m = 0; m < BW; ++m) {
+                                float acc = cr[i][m];
+                                if (reg) {
+                                    // rows t0 .. t+BW-2 still accumulating: registers
+#pragma unroll
+                                    for (int k = 0; k < i + BW - 1; ++k)
+                                        acc = fmaf(At[(t + m) * LDA + t0 + k], zb[k], acc);
+                                }
+                                const int r = t + m;
+                                const float y = tile_get(sm, W_VE, r, j);
+                                cr[i][m] = reg ? wt * (y - gm * sx[r]) - kt * acc : wt * y;
+                            }
+                            // z_{t,m} lands on row t+m only after every slot of token t used the old sums
+#pragma unroll
+                            for (int m = 0; m < BW; ++m) zb[i + m] += cr[i][m];
+                            float bsum = 0.f;
+#pragma unroll
+                            for (int k = 1; k < BW; ++k) bsum = fmaf(pband[t * 4 + k], zb[i + k], bsum);
+                            bnd[hb * NB + i] = bsum;
                         }
-                        float b = 0.f;
+                        // rows t0 .. t0+7 are final; rows t0+8 .. carry into the next block
 #pragma unroll
-                        for (int k = 1; k < BW; ++k) b = fmaf(pband[t * 4 + k], za[t + k], b);
-                        bnd[ii] = b;
+                        for (int k = 0; k < NB; ++k) za[t0 + k] = zb[k];
+#pragma unroll
+                        for (int k = 0; k < RB; ++k) zb[k] = k + NB < RB ? zb[k + NB] : 0.f;
                     }
                     tc::tmem_st16(tl + C_G + tb * 16, bnd);
                 }
+                // rows 64 .. 64+BW-2 end the chunk in registers
+#pragma unroll
+                for (int k = 0; k < BW - 1; ++k) za[CH + k] = zb[k];
                 tc::tmem_wait_st();
                 // Zt^T row j
                 float zr[NR];
