@@ -236,7 +236,8 @@ class OracleSample:
         for variant in w["variants"]:
             _, _, self.threads = self.oracle.fwd(variant, "chunk", *args, lam, self.d["eps_64"], chunk=w["chunk"],
                                                  nthreads=self.ncores, return_threads=True)
-        return len(w["variants"]) * n * w["L"], time.perf_counter() - t0
+        # a token is one position of one sequence with all H heads: n units are n/H of a sequence
+        return len(w["variants"]) * n * w["L"] / w["H"], time.perf_counter() - t0
 
 
 def cpu_oracle_sample(budget_s=12.0):
@@ -271,7 +272,8 @@ def run_reference(args):
             "config": workload_config(),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.threads, "kind": "oracle",
                              "sample": "each step: %d whole (b,h) units of the workload through the fp64 oracle's "
-                                       "chunk-parallel form, Falcon-1 and Falcon-1A" % min(smp.ncores, len(smp.units))},
+                                       "chunk-parallel form, Falcon-1 and Falcon-1A; H units make one token of "
+                                       "the metric" % min(smp.ncores, len(smp.units))},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -382,14 +384,16 @@ def run_ours(args):
             "config": workload_config(), "roofline": roof,
             "per_variant_ms": {var: statistics.mean(per_var[var]) for var in w["variants"]},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": len(w["variants"]) * args.steps, "clocks": clk.summary()}
+            # every falcon_fwd of this shape is two kernels: chunk_local_kernel + chunk_chain_kernel
+            "gpu_launches": 2 * len(w["variants"]) * args.steps, "clocks": clk.summary()}
     if decode is not None:
         line["decode"] = decode
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, threads, units, used = cpu_oracle_sample(budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                 "sample": "fp64 oracle chunk-parallel form, Falcon-1 and Falcon-1A, %d whole (b,h) "
-                                          "units of the workload (%.1f s)" % (units, used)}
+                                          "units of the workload (%.1f s); H units make one token of the "
+                                          "metric" % (units, used)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -482,8 +486,42 @@ def run_workloads(args):
             torch.cuda.synchronize()
             ms.append(e0.elapsed_time(e1))
         t = statistics.median(ms)
-        print(json.dumps({"workload": n, "name": w["name"], "variant": var, "form": form, "dtype": w["dtype"],
-                          "ms": t, "tokens_per_s": w["B"] * w["L"] / (t / 1e3)}), flush=True)
+        elt = 2 if w["dtype"] == "bf16" else 4
+        ab = algorithmic_bytes_fwd(w["B"], w["H"], w["L"], w["dk"], w["dv"], per_channel=var in ("F2", "F2A"),
+                                   elt=elt)
+        gbs = ab / (t / 1e3) / 1e9
+        hbm, _, peak_src = peaks()
+        line = {"workload": n, "name": w["name"], "variant": var, "form": form, "dtype": w["dtype"],
+                "ms": t, "tokens_per_s": w["B"] * w["L"] / (t / 1e3),
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                             "peak_source": peak_src, "algorithmic_bytes_per_launch": ab}}
+        if not args.no_cpu_baseline:
+            line["cpu_oracle"] = workload_oracle_rate(d, var, form, w)
+        print(json.dumps(line), flush=True)
+
+
+def workload_oracle_rate(d, variant, form, w):
+    """The fp64 oracle's recurrent form (the definition, the same outputs as
+    every form at O(L d^2) per unit; its masked form is O(L^2)) on
+    min(cores, B*H) whole (b,h) units of the workload's inputs, all host
+    cores: tokens/s."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    units = [(b, h) for b in range(w["B"]) for h in range(w["H"])]
+    n = min(os.cpu_count() or 1, len(units))
+    bs = [b for b, _ in units[:n]]
+    hs = [h for _, h in units[:n]]
+    sel = lambda a: np.ascontiguousarray(a[bs, hs][None])  # noqa: E731
+    args = [sel(d[x]) for x in ("q_64", "k_64", "v_64", "beta_64")]
+    lam = np.asarray(d["lam_64"])[hs]
+    t0 = time.perf_counter()
+    _, _, threads = oracle.fwd(variant, "recurrent", *args, lam, d["eps_64"], window=w["window"],
+                               chunk=w["chunk"], nthreads=os.cpu_count() or 1, return_threads=True)
+    sec = time.perf_counter() - t0
+    # a token is one position of one sequence with all H heads
+    return {"value": n * w["L"] / w["H"] / sec, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": "fp64 recurrent form, %d whole (b,h) units, %.1f s" % (n, sec)}
 
 
 def main():
