@@ -112,16 +112,39 @@ __device__ void load_queries(const T *kq, int t0, int n, float *Q, int LDX) {
     }
 }
 
-// C[a][b] = sum_c U[a][c] V[b][c] for a < na, b < nb.
+// C[a][b] = sum_c U[a][c] V[b][c] for a < na, b < nb; each thread a 4x4
+// block of C (rows past na / columns past nb read row 0 and are not stored).
 template <int DK>
 __device__ void small_gemm_nt(const float *U, int ldu, int na, const float *V, int ldv, int nb,
                               float *C, int ldc) {
-    for (int idx = threadIdx.x; idx < na * nb; idx += kThreads) {
-        const int a = idx / nb, b = idx % nb;
-        float s = 0.f;
-#pragma unroll 8
-        for (int c = 0; c < DK; ++c) s += U[a * ldu + c] * V[b * ldv + c];
-        C[a * ldc + b] = s;
+    const int ta = (na + 3) >> 2, tb = (nb + 3) >> 2;
+    for (int idx = threadIdx.x; idx < ta * tb; idx += kThreads) {
+        const int a0 = (idx / tb) * 4, b0 = (idx % tb) * 4;
+        const float *u[4], *v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            u[i] = U + (a0 + i < na ? a0 + i : 0) * ldu;
+            v[i] = V + (b0 + i < nb ? b0 + i : 0) * ldv;
+        }
+        float acc[4][4] = {};
+#pragma unroll 4
+        for (int c = 0; c < DK; ++c) {
+            float x[4], y[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[i] = u[i][c];
+                y[i] = v[i][c];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc[i][k] = fmaf(x[i], y[k], acc[i][k]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (a0 + i < na && b0 + k < nb) C[(a0 + i) * ldc + b0 + k] = acc[i][k];
     }
 }
 
@@ -235,16 +258,20 @@ __global__ void __launch_bounds__(kThreads) span_chunk_kernel(FwdParams p) {
             }
             if (j0 + j < dv) ko[(size_t)(c0 + tl) * dv + j0 + j] = from_f32<T>(o);
         }
-        // state hand-off S0 <- S_{c1-1}
+        // state hand-off S0 <- S_{c1-1}; the weights e^{G_end - G_s} eta_s once per
+        // token (SX is free once the right-hand sides are formed)
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < n * VS; idx += kThreads)
+            SX[idx] = expf(G[(n - 1) * VS + idx % VS] - G[idx]) * ETA[idx];
+        __syncthreads();
         for (int idx = threadIdx.x; idx < VS * DK; idx += kThreads) {
             const int j = idx / DK, c = idx % DK;
             const float ge = G[(n - 1) * VS + j];
             float s = expf(ge) * S0[j * LDX + c];
             for (int sl = 0; sl < n; ++sl) {
-                const float coef = expf(ge - G[sl * VS + j]) * ETA[sl * VS + j];
                 float acc = 0.f;
                 for (int m = 0; m < w; ++m) acc += R[(sl * w + m) * VS + j] * X[(sl + m) * LDX + c];
-                s += coef * acc;
+                s += SX[sl * VS + j] * acc;
             }
             S0[j * LDX + c] = s;
         }
@@ -380,11 +407,15 @@ __global__ void __launch_bounds__(kThreads) span_masked_kernel(FwdParams p, int 
             const int nj = C;  // earlier blocks are always full
             __syncthreads();
             load_samples<T, DK>(p, bh, kk, kv, L, cj - (w - 1), nj + w - 1, j0, XJ, LDX, YJ, SQNJ);
+            // e^{Gamma_a - Gamma_s} for a in block I and s in block J < I splits at
+            // Gamma_{c0-1}, the end of the previous block, into two factors <= 1:
+            // ETAJ carries e^{Gamma_{c0-1} - Gamma_s} eta_s, the rows their own factor
             for (int idx = threadIdx.x; idx < nj * VS; idx += kThreads) {
                 const int tl = idx / VS, j = idx % VS;
                 const bool ok = j0 + j < dv;
-                ETAJ[idx] = ok ? weta[(size_t)(cj + tl) * dv + j0 + j] : 0.f;
-                GAMJ[idx] = ok ? wgam[(size_t)(cj + tl) * dv + j0 + j] : 0.f;
+                ETAJ[idx] = ok ? weta[(size_t)(cj + tl) * dv + j0 + j] *
+                                     expf(GPREV[j] - wgam[(size_t)(cj + tl) * dv + j0 + j])
+                               : 0.f;
             }
             for (int idx = threadIdx.x; idx < nj * w * VS; idx += kThreads) {
                 const int tl = idx / (w * VS), m = (idx / VS) % w, j = idx % VS;
@@ -400,12 +431,11 @@ __global__ void __launch_bounds__(kThreads) span_masked_kernel(FwdParams p, int 
                     const float gp = tl > 0 ? GAMI[(tl - 1) * VS + j] : GPREV[j];
                     float acc = 0.f;
                     for (int s = 0; s < nj; ++s) {
-                        const float coef = expf(gp - GAMJ[s * VS + j]) * ETAJ[s * VS + j];
                         float a2 = 0.f;
                         for (int m2 = 0; m2 < w; ++m2) a2 += A[(tl + m) * LDA + s + m2] * RJ[(s * w + m2) * VS + j];
-                        acc += coef * a2;
+                        acc += ETAJ[s * VS + j] * a2;
                     }
-                    RI[idx] -= acc;
+                    RI[idx] -= expf(gp - GPREV[j]) * acc;
                 }
             }
             for (int idx = threadIdx.x; idx < n * VS; idx += kThreads) {
@@ -413,12 +443,11 @@ __global__ void __launch_bounds__(kThreads) span_masked_kernel(FwdParams p, int 
                 const float gt = GAMI[idx];
                 float acc = 0.f;
                 for (int s = 0; s < nj; ++s) {
-                    const float coef = expf(gt - GAMJ[s * VS + j]) * ETAJ[s * VS + j];
                     float a2 = 0.f;
                     for (int m2 = 0; m2 < w; ++m2) a2 += P[tl * LDA + s + m2] * RJ[(s * w + m2) * VS + j];
-                    acc += coef * a2;
+                    acc += ETAJ[s * VS + j] * a2;
                 }
-                O[idx] += acc;
+                O[idx] += expf(gt - GPREV[j]) * acc;
             }
         }
         // the diagonal block
@@ -455,14 +484,17 @@ __global__ void __launch_bounds__(kThreads) span_masked_kernel(FwdParams p, int 
             const int tl = idx / (w * VS), m = (idx / VS) % w, j = idx % VS;
             if (j0 + j < dv) wr[((size_t)(c0 + tl) * w + m) * dv + j0 + j] = RI[idx];
         }
+        // the final state's weights e^{Gamma_L - Gamma_s} eta_s, once per token (GAMJ is free here)
+        for (int idx = threadIdx.x; idx < n * VS; idx += kThreads)
+            GAMJ[idx] = expf(GLAST[idx % VS] - GAMI[idx]) * ETAI[idx];
+        __syncthreads();
         for (int idx = threadIdx.x; idx < VS * DK; idx += kThreads) {
             const int j = idx / DK, c = idx % DK;
             float s = 0.f;
             for (int sl = 0; sl < n; ++sl) {
-                const float coef = expf(GLAST[j] - GAMI[sl * VS + j]) * ETAI[sl * VS + j];
                 float acc = 0.f;
                 for (int m = 0; m < w; ++m) acc += RI[(sl * w + m) * VS + j] * XI[(sl + m) * LDX + c];
-                s += coef * acc;
+                s += GAMJ[sl * VS + j] * acc;
             }
             S[j * LDX + c] += s;
         }
