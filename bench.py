@@ -500,6 +500,45 @@ def run_workloads(args):
         print(json.dumps(line), flush=True)
 
 
+def run_chunk_sweep(args):
+    """--chunk-sweep: the chunk-parallel forward of workload 2 (Falcon-1 and
+    Falcon-1A, 8x12x2048x64 bf16) at chunk 16, 32 and 64 under the prefix
+    pair, and at 64 under the same-step pair; CUDA events around one
+    falcon_fwd after a warm-up call, L2 flushed, median of --steps calls.
+    One JSON line each with the kernels that ran and the stream-ordered
+    workspace the call draws.  Not the contract line."""
+    import torch
+    import linear_attention_sequence_falcon_b200 as F
+    from linear_attention_sequence_falcon_b200 import build, inputs as gen
+    build.build()
+    F.load()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    w = gen.WORKLOADS[2]
+    units = w["B"] * w["H"] * ((w["L"] + 63) // 64)
+    for var in w["variants"]:
+        d = gen.workload_inputs(2, var)
+        args_ = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
+        for chunk, pairing in ((16, "prefix"), (32, "prefix"), (64, "prefix"), (64, "same_step")):
+            out, S = F.fwd(var, "chunk", *args_, d["eps"], chunk=chunk, pairing=pairing)
+            torch.cuda.synchronize()
+            ms = []
+            for _ in range(max(3, min(args.steps, 20))):
+                flush.zero_()
+                torch.cuda._sleep(HEAD_START_CYCLES)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                F.fwd(var, "chunk", *args_, d["eps"], chunk=chunk, pairing=pairing, out=out, final_state=S)
+                e1.record()
+                torch.cuda.synchronize()
+                ms.append(e0.elapsed_time(e1))
+            t = statistics.median(ms)
+            tc = chunk == 64
+            print(json.dumps({"sweep": "chunk", "workload": w["name"], "variant": var, "chunk": chunk,
+                              "pairing": pairing, "ms": t, "tokens_per_s": w["B"] * w["L"] / (t / 1e3),
+                              "kernels": "chunk_local_kernel + chunk_chain_kernel" if tc else "span_chunk_kernel",
+                              "workspace_bytes": units * 32 * 1024 + units * 4 if tc else 0}), flush=True)
+
+
 def workload_oracle_rate(d, variant, form, w):
     """The fp64 oracle in the row's own form -- the recurrent form for masked
     rows, whose O(L^2) oracle takes 7-80 s per (b,h) unit at L = 2048 -- on
@@ -542,9 +581,13 @@ def main():
     ap.add_argument("--workloads", action="store_true",
                     help="time every workload and form of the workloads table, one JSON line each")
     ap.add_argument("--only", type=int, default=0, help="with --workloads: just this workload number")
+    ap.add_argument("--chunk-sweep", action="store_true",
+                    help="the chunk form of workload 2 at chunk 16/32/64 and both pairings (one line each)")
     ap.add_argument("--profile", action="store_true",
                     help="run only warmup+steps device steps (no flush, e2e, clocks or JSON), for ncu")
     args = ap.parse_args()
+    if args.chunk_sweep:
+        return run_chunk_sweep(args)
     if args.workloads:
         run_workloads(args)
     elif args.impl == "reference":
