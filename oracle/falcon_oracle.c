@@ -578,3 +578,227 @@ int oracle_carry_from_prefill(int variant, int phi, const double *k, const doubl
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Reverse mode of the recurrent definition (the backward pass).        */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Gradients of a scalar loss L through the recurrent form, given dL/do_t
+ * (dout [B,H,L,dv]) and dL/dS_L (dstate [B,H,dv,dk], NULL for zero), for
+ * every variant, pairing and feature map, from S_0 = 0 (no carry).  The
+ * chunk form trains on the same function ([EXPL 核心方法 3], [NEWS 02 (2)]);
+ * this is its derivative taken step by step, latest step first:
+ *   o_t = S_t q_t                      dq_t = S_t^T do_t,   Gs += do_t q_t^T
+ *   S_t = alpha_t S_{t-1} + eta_t U_t  dalpha_t += <Gs, S_{t-1}>, deta_t += <Gs, U_t>
+ *   U_t = sum_{i in W_t} e_{t,i} x_i^T, e_{t,i} = y_i - S_{t-1} x_i (regression) or y_i
+ *                                      de_{t,i} = eta_t Gs x_i,  dx_i += eta_t Gs^T e_{t,i}
+ *                                      regression: dy_i += de, dx_i -= S_{t-1}^T de,
+ *                                                  Gs <- alpha_t Gs - sum_i de x_i^T
+ *                                      inner product: dy_i += de, Gs <- alpha_t Gs
+ * (row j with its own eta, alpha for Falcon-2/2A; the inner products above
+ * then stay within the row).  Then the steps (R3, R4):
+ *   alpha = max(1 - eta lambda, 2^-20): deta += -lambda dalpha, dlambda += -eta dalpha
+ *     where 1 - eta lambda > 2^-20; no gradient where the floor holds;
+ *   eta = beta / (eps + n) (0 when n = 0): dbeta = deta / (eps + n), dn += -deta beta / (eps + n)^2;
+ *   n = sum_{i in W_t} |x_i|^2: dx_i += 2 dn x_i;
+ *   x = k / |k| (R1): dk = (dx - x (x . dx)) / |k|, 0 at k = 0; identity: dk = dx.
+ * Outputs (all [B,H,...] like the inputs): dq, dk, dv, dbeta and dlambda [H]
+ * (summed over b).  The state history is kept whole: meant for small cases.
+ */
+typedef struct {
+    int variant, pairing, phi, B, H, L, dk, dv, w;
+    double eps;
+    const double *q, *k, *v, *beta, *lambda, *dout, *dstate;
+    double *dq, *dkk, *dvv, *dbeta, *dlam_bh;  /* dlam_bh [B*H], summed by the caller */
+} bwd_job_t;
+
+static void bwd_unit_run(const bwd_job_t *Bj, int b, int h)
+{
+    const int L = Bj->L, dk = Bj->dk, dv = Bj->dv, w = Bj->w;
+    const size_t bh = (size_t)b * Bj->H + h;
+    job_t J = {Bj->variant, FORM_RECURRENT, Bj->pairing, Bj->phi, Bj->B, Bj->H, L, dk, dv, w, 1, Bj->eps,
+               Bj->q, Bj->k, Bj->v, Bj->beta, Bj->lambda, NULL, NULL};
+    unit_t u;
+    prepare_unit(&J, b, h, &u);
+    const int nch = u.nch, reg = is_regression(Bj->variant);
+    const size_t SS = (size_t)dv * dk;
+    /* forward: the whole history S_0 .. S_L (S_0 = 0) */
+    double *hist = (double *)calloc((size_t)(L + 1) * SS, sizeof(double));
+    double *res = (double *)calloc((size_t)w * dv, sizeof(double));
+    for (int t = 0; t < L; ++t) {
+        const double *Sp = hist + (size_t)t * SS;
+        double *Sn = hist + (size_t)(t + 1) * SS;
+        int i0 = t - w + 1;
+        if (i0 < 0) i0 = 0;
+        for (int i = i0; i <= t; ++i)
+            for (int j = 0; j < dv; ++j)
+                res[(size_t)(i - i0) * dv + j] = reg ? u.y[(size_t)i * dv + j] - dot(Sp + (size_t)j * dk, u.x + (size_t)i * dk, dk)
+                                                     : u.y[(size_t)i * dv + j];
+        for (int j = 0; j < dv; ++j) {
+            const int ch = nch > 1 ? j : 0;
+            const double eta = u.eta[(size_t)t * nch + ch], a = u.alpha[(size_t)t * nch + ch];
+            for (int c = 0; c < dk; ++c) {
+                double g = 0.0;
+                for (int i = i0; i <= t; ++i) g += res[(size_t)(i - i0) * dv + j] * u.x[(size_t)i * dk + c];
+                Sn[(size_t)j * dk + c] = a * Sp[(size_t)j * dk + c] + eta * g;
+            }
+        }
+    }
+    /* backward */
+    double *Gs = (double *)calloc(SS, sizeof(double));
+    double *Gn = (double *)calloc(SS, sizeof(double));
+    double *dx = (double *)calloc((size_t)L * dk, sizeof(double));
+    double *deta = (double *)calloc((size_t)L * nch, sizeof(double));
+    double *dalpha = (double *)calloc((size_t)L * nch, sizeof(double));
+    double *de = (double *)calloc((size_t)w * dv, sizeof(double));
+    double *dq = Bj->dq + bh * (size_t)L * dk;
+    double *dvv = Bj->dvv + bh * (size_t)L * dv;
+    memset(dvv, 0, sizeof(double) * (size_t)L * dv);
+    if (Bj->dstate) memcpy(Gs, Bj->dstate + bh * SS, sizeof(double) * SS);
+    const double *dout = Bj->dout + bh * (size_t)L * dv;
+    for (int t = L - 1; t >= 0; --t) {
+        const double *St = hist + (size_t)(t + 1) * SS, *Sp = hist + (size_t)t * SS;
+        const double *qt = u.q + (size_t)t * dk, *dot_ = dout + (size_t)t * dv;
+        for (int c = 0; c < dk; ++c) {
+            double s = 0.0;
+            for (int j = 0; j < dv; ++j) s += St[(size_t)j * dk + c] * dot_[j];
+            dq[(size_t)t * dk + c] = s;
+        }
+        for (int j = 0; j < dv; ++j)
+            for (int c = 0; c < dk; ++c) Gs[(size_t)j * dk + c] += dot_[j] * qt[c];
+        int i0 = t - w + 1;
+        if (i0 < 0) i0 = 0;
+        for (int i = i0; i <= t; ++i)
+            for (int j = 0; j < dv; ++j)
+                res[(size_t)(i - i0) * dv + j] = reg ? u.y[(size_t)i * dv + j] - dot(Sp + (size_t)j * dk, u.x + (size_t)i * dk, dk)
+                                                     : u.y[(size_t)i * dv + j];
+        for (int j = 0; j < dv; ++j) {
+            const int ch = nch > 1 ? j : 0;
+            const double eta = u.eta[(size_t)t * nch + ch];
+            const double *Gj = Gs + (size_t)j * dk, *Spj = Sp + (size_t)j * dk;
+            dalpha[(size_t)t * nch + ch] += dot(Gj, Spj, dk);
+            for (int i = i0; i <= t; ++i) {
+                const double *xi = u.x + (size_t)i * dk;
+                const double e = res[(size_t)(i - i0) * dv + j];
+                const double gx = dot(Gj, xi, dk);
+                deta[(size_t)t * nch + ch] += e * gx;
+                de[(size_t)(i - i0) * dv + j] = eta * gx;
+                for (int c = 0; c < dk; ++c) dx[(size_t)i * dk + c] += eta * Gj[c] * e;
+            }
+        }
+        for (int i = i0; i <= t; ++i) {
+            for (int j = 0; j < dv; ++j) {
+                const double d = de[(size_t)(i - i0) * dv + j];
+                dvv[(size_t)i * dv + j] += d;
+                if (reg)
+                    for (int c = 0; c < dk; ++c) dx[(size_t)i * dk + c] -= Sp[(size_t)j * dk + c] * d;
+            }
+        }
+        /* dL/dS_{t-1} */
+        for (int j = 0; j < dv; ++j) {
+            const int ch = nch > 1 ? j : 0;
+            const double a = u.alpha[(size_t)t * nch + ch];
+            for (int c = 0; c < dk; ++c) {
+                double g = a * Gs[(size_t)j * dk + c];
+                if (reg)
+                    for (int i = i0; i <= t; ++i) g -= de[(size_t)(i - i0) * dv + j] * u.x[(size_t)i * dk + c];
+                Gn[(size_t)j * dk + c] = g;
+            }
+        }
+        memcpy(Gs, Gn, sizeof(double) * SS);
+    }
+    /* the steps, the normaliser, the feature map */
+    const double lam = Bj->lambda[h];
+    const double *beta = Bj->beta + bh * (size_t)L * nch;
+    double *dbeta = Bj->dbeta + bh * (size_t)L * nch;
+    double dlam = 0.0;
+    for (int t = 0; t < L; ++t) {
+        int i0 = t - w + 1;
+        if (i0 < 0) i0 = 0;
+        double n = 0.0;
+        for (int i = i0; i <= t; ++i) n += dot(u.x + (size_t)i * dk, u.x + (size_t)i * dk, dk);
+        double dn = 0.0;
+        for (int ch = 0; ch < nch; ++ch) {
+            const double eta = u.eta[(size_t)t * nch + ch];
+            double de_ = deta[(size_t)t * nch + ch];
+            if (1.0 - eta * lam > ALPHA_FLOOR) {
+                de_ += -lam * dalpha[(size_t)t * nch + ch];
+                dlam += -eta * dalpha[(size_t)t * nch + ch];
+            }
+            if (n > 0.0) {
+                const double bt = beta[(size_t)t * nch + ch];
+                dbeta[(size_t)t * nch + ch] = de_ / (Bj->eps + n);
+                dn += -de_ * bt / ((Bj->eps + n) * (Bj->eps + n));
+            } else {
+                dbeta[(size_t)t * nch + ch] = 0.0;
+            }
+        }
+        for (int i = i0; i <= t; ++i)
+            for (int c = 0; c < dk; ++c) dx[(size_t)i * dk + c] += 2.0 * dn * u.x[(size_t)i * dk + c];
+    }
+    double *dkk = Bj->dkk + bh * (size_t)L * dk;
+    memset(dkk, 0, sizeof(double) * (size_t)L * dk);
+    const double *kk = Bj->k + bh * (size_t)L * dk;
+    for (int i = 0; i < L; ++i) {
+        const int kr = Bj->pairing == PAIR_SAME_STEP ? i : i - 1;  /* x_i = phi(k_kr); x_0 = 0 under the prefix pair */
+        if (kr < 0) continue;
+        const double *xi = u.x + (size_t)i * dk, *dxi = dx + (size_t)i * dk, *ki = kk + (size_t)kr * dk;
+        if (Bj->phi == PHI_IDENTITY) {
+            for (int c = 0; c < dk; ++c) dkk[(size_t)kr * dk + c] += dxi[c];
+        } else {
+            const double nrm = sqrt(dot(ki, ki, dk));
+            if (nrm > 0.0) {
+                const double xd = dot(xi, dxi, dk);
+                for (int c = 0; c < dk; ++c) dkk[(size_t)kr * dk + c] += (dxi[c] - xi[c] * xd) / nrm;
+            }
+        }
+    }
+    Bj->dlam_bh[bh] = dlam;
+    free(hist); free(res); free(Gs); free(Gn); free(dx); free(deta); free(dalpha); free(de);
+    free_unit(&u);
+}
+
+typedef struct {
+    const bwd_job_t *J;
+    int tid, nthreads;
+} bwd_worker_t;
+
+static void *bwd_worker(void *arg)
+{
+    const bwd_worker_t *W = (const bwd_worker_t *)arg;
+    const int units = W->J->B * W->J->H;
+    for (int n = W->tid; n < units; n += W->nthreads) bwd_unit_run(W->J, n / W->J->H, n % W->J->H);
+    return NULL;
+}
+
+int oracle_bwd(int variant, int pairing, int phi, const double *q, const double *k, const double *v,
+               const double *beta, const double *lambda, double eps, int window, int B, int H, int L, int dk, int dv,
+               const double *dout, const double *dstate, double *dq, double *dkk, double *dvv, double *dbeta,
+               double *dlambda, int nthreads)
+{
+    if (variant < 0 || variant > 5) return -2;
+    if (B < 0 || H < 0 || L < 0 || dk <= 0 || dv <= 0) return -3;
+    if (is_window(variant) && window < 1) return -6;
+    double *dlam_bh = (double *)calloc((size_t)B * H + 1, sizeof(double));
+    bwd_job_t J = {variant, pairing, phi, B, H, L, dk, dv, is_window(variant) ? window : 1, eps,
+                   q, k, v, beta, lambda, dout, dstate, dq, dkk, dvv, dbeta, dlam_bh};
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    const int units = B * H;
+    if (nthreads > units) nthreads = units > 0 ? units : 1;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
+    bwd_worker_t *ws = (bwd_worker_t *)malloc(sizeof(bwd_worker_t) * nthreads);
+    for (int i = 0; i < nthreads; ++i) {
+        ws[i].J = &J; ws[i].tid = i; ws[i].nthreads = nthreads;
+        pthread_create(&th[i], NULL, bwd_worker, &ws[i]);
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    for (int hh = 0; hh < H; ++hh) {
+        double s = 0.0;
+        for (int bb = 0; bb < B; ++bb) s += dlam_bh[(size_t)bb * H + hh];
+        dlambda[hh] = s;
+    }
+    free(th); free(ws); free(dlam_bh);
+    return nthreads;
+}
