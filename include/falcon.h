@@ -146,6 +146,37 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
                      void *out, float *final_state, cudaStream_t stream);
 
 /*
+ * falcon_bwd -- the backward pass: gradients of a scalar loss with respect
+ * to q, k, v, beta and lambda, given dL/d(out) and dL/d(final_state), for a
+ * forward from S_0 = 0 with the same arguments.  The chunk form trains on the
+ * recurrent function ([EXPL] 核心方法 3); this is its derivative, taken in
+ * the recurrent form on the CUDA cores (fp32):
+ *   dq_t = S_t^T do_t;  Gs_t = do_t q_t^T + alpha_{t+1} Gs_{t+1};
+ *   dv_t = eta_t (Gs_t x_t);  the decays through dL/dG_t = do_t o_t - eta_t
+ *   y_t (Gs_t x_t) (+ <dL/dS_L, S_L> at the last token) summed from t
+ *   onwards (per value channel for Falcon-2A);
+ *   then alpha = max(1 - eta lambda, 2^-20) (no gradient on the floor),
+ *   eta = beta/(eps + |x|^2) and x = phi(k).
+ *
+ *   variant     FALCON_F1A or FALCON_F2A (others: FALCON_ERR_UNSUPPORTED)
+ *   dtype, q, k, v, beta, lambda, eps, B, H, L, pairing, phi: as in
+ *               falcon_fwd_ex; d_k = d_v in {32, 64, 128}
+ *   dout        [B,H,L,d_v] dtype: dL/d(out)
+ *   dstate      [B,H,d_v,d_k] fp32, or NULL (zero): dL/d(final_state)
+ *   dq, dk      [B,H,L,d_k] fp32, written
+ *   dv          [B,H,L,d_v] fp32, written
+ *   dbeta       [B,H,L] (Falcon-1A) or [B,H,L,d_v] (Falcon-2A) fp32, written
+ *   dlambda     [H] fp32, written (summed over b), or NULL
+ * Scratch: (2 L d + L + 5 L c) floats per (b,h), c = 1 or d_v, stream-ordered
+ * from the library's pool (FALCON_ERR_ALLOC if that fails).  Errors as in
+ * falcon_fwd.
+ */
+int falcon_bwd(falcon_variant variant, falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
+               const void *q, const void *k, const void *v, const void *beta, const float *lambda, float eps,
+               int B, int H, int L, int d_k, int d_v, const void *dout, const float *dstate,
+               float *dq, float *dk, float *dv, float *dbeta, float *dlambda, cudaStream_t stream);
+
+/*
  * falcon_decode_step -- one recurrent step for N independent sequences
  * ([EXPL] 核心方法 3: recurrent, O(d^2) per step, for inference).
  *

@@ -21,7 +21,7 @@ FORMS = {"recurrent": 0, "masked": 1, "chunk": 2}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PAIRINGS = {"prefix": 0, "same_step": 1}
 PHIS = {"l2": 0, "identity": 1}
-EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_fwd_carry", "falcon_decode_step", "falcon_decode_carry_from_prefill",
+EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_fwd_carry", "falcon_bwd", "falcon_decode_step", "falcon_decode_carry_from_prefill",
            "falcon_fwd_masked_noalloc", "falcon_device_wait_timeouts", "falcon_selftest_bounded_wait",
            "falcon_scratch_trim", "falcon_status_string")
 
@@ -47,6 +47,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.falcon_fwd_ex.restype = I
     lib.falcon_fwd_carry.argtypes = [I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, I, P, P, P, P, P, P]
     lib.falcon_fwd_carry.restype = I
+    lib.falcon_bwd.argtypes = [I, I, I, I, P, P, P, P, P, F, I, I, I, I, I, P, P, P, P, P, P, P, P]
+    lib.falcon_bwd.restype = I
     lib.falcon_decode_step.argtypes = [I, I, P, P, P, P, P, F, I, I, I, I, I, P, P, P, P, P]
     lib.falcon_decode_step.restype = I
     lib.falcon_decode_carry_from_prefill.argtypes = [I, I, P, P, I, I, I, I, I, I, P, P, P]
@@ -122,6 +124,32 @@ def fwd(variant: str, form: str, q, k, v, beta, lam, eps: float, window: int = 1
                                B, H, L, dk, dv, int(chunk), _ptr(out), _ptr(final_state), _stream(stream))
     _check(rc)
     return out, final_state
+
+
+def bwd(variant: str, q, k, v, beta, lam, eps: float, dout, dstate=None, pairing: str = "prefix",
+        phi: str = "l2", stream=None):
+    """falcon_bwd: gradients of a loss with respect to q, k, v, beta and lambda
+    of a forward from S_0 = 0, given dout = dL/d(out) (dtype of q) and dstate =
+    dL/d(final_state) (fp32, or None).  Falcon-1A and Falcon-2A, d_k = d_v in
+    {32, 64, 128}.  Returns a dict of fp32 tensors dq, dk, dv, dbeta, dlambda."""
+    lib = load()
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in DTYPES or not (q.dtype == k.dtype == v.dtype == beta.dtype == dout.dtype):
+        raise FalconError("q, k, v, beta, dout must share one dtype, fp32 or bf16")
+    if lam.dtype != torch.float32 or (dstate is not None and dstate.dtype != torch.float32):
+        raise FalconError("lambda and dstate must be fp32")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"dq": torch.empty((B, H, L, dk), **f32), "dk": torch.empty((B, H, L, dk), **f32),
+         "dv": torch.empty((B, H, L, dv), **f32), "dbeta": torch.empty(tuple(beta.shape), **f32),
+         "dlambda": torch.zeros((H,), **f32)}
+    rc = lib.falcon_bwd(VARIANTS[variant], DTYPES[q.dtype], PAIRINGS[pairing], PHIS[phi],
+                        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(lam), float(eps), B, H, L, dk, dv,
+                        _ptr(dout), _ptr(dstate) if dstate is not None else None,
+                        _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dbeta"]), _ptr(g["dlambda"]),
+                        _stream(stream))
+    _check(rc)
+    return g
 
 
 def fwd_masked_noalloc(variant: str, q, k, v, beta, lam, eps: float, window: int = 1, out=None,

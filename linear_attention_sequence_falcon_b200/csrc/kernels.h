@@ -37,6 +37,9 @@ unsigned int f2_wait_timeouts();
 int launch_w_chunk(const FwdParams &p, cudaStream_t s);
 unsigned int w_wait_timeouts();
 template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
+// Backward pass of Falcon-1A / Falcon-2A (recurrent form, fp32), d_k = d_v in
+// {32, 64, 128}; the arguments are validated by the caller.
+template <typename T> int launch_bwd(const BwdParams &p, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
 
 // Stream-ordered scratch from the library's per-device pool (kept mapped

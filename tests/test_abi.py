@@ -66,3 +66,25 @@ def test_validation_codes(lib):
     assert lib.falcon_decode_step(0, 1, P, P, P, P, P, 1e-6, 1, 4, 2, 64, 100, P, P, None, P, None) == -3
     assert lib.falcon_decode_carry_from_prefill(9, 1, P, P, 1, 1, 1, 4, 64, 64, P, None, None) == -2
     assert lib.falcon_decode_carry_from_prefill(2, 1, P, P, 4, 1, 1, 4, 64, 64, P, None, None) == -1
+
+
+def _bwd(lib, variant=3, dtype=1, pairing=0, phi=0, B=1, H=1, L=8, dk=64, dv=64, ptr=1, dlam=True):
+    P = ctypes.c_void_p(ptr) if ptr else None
+    return lib.falcon_bwd(variant, dtype, pairing, phi, P, P, P, P, P, 1e-6, B, H, L, dk, dv, P, None,
+                          P, P, P, P, P if dlam else None, None)
+
+
+def test_backward_validation_codes(lib):
+    lib.falcon_bwd.restype = ctypes.c_int
+    assert _bwd(lib, variant=9) == -2
+    assert _bwd(lib, dtype=4) == -2
+    assert _bwd(lib, pairing=2) == -2
+    assert _bwd(lib, phi=3) == -2
+    assert _bwd(lib, dk=48) == -3
+    assert _bwd(lib, variant=0) == -9   # regression family: not in the backward kernel
+    assert _bwd(lib, variant=5) == -9   # windows: not in the backward kernel
+    assert _bwd(lib, dk=64, dv=32) == -9
+    assert _bwd(lib, dk=16, dv=16) == -9
+    assert _bwd(lib, ptr=0) == -1
+    assert _bwd(lib, B=0) == 0
+    assert _bwd(lib, L=0, dlam=False) == 0
