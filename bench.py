@@ -539,6 +539,68 @@ def run_chunk_sweep(args):
                               "workspace_bytes": units * 32 * 1024 + units * 4 if tc else 0}), flush=True)
 
 
+def run_backward(args):
+    """--backward: falcon_bwd (the backward pass of Falcon-1A / Falcon-2A) on
+    workload 2 (Falcon-1A, 8x12x2048x64 bf16) and on workload 5's prefill
+    (Falcon-2A, 2x16x32768x128 bf16): CUDA events around one call after a
+    warm-up call, L2 flushed, median of --steps calls (3..10); an HBM
+    roofline on the algorithmic bytes (q, k, v, beta, dout read; dq, dk, dv,
+    dbeta written in fp32) and the fp64 oracle's reverse mode on whole (b,h)
+    units (workload 2 only: its state history at L = 32768, d = 128 would
+    take 4 GB per unit).  Not the contract line."""
+    import numpy as np
+    import torch
+    import linear_attention_sequence_falcon_b200 as F
+    from linear_attention_sequence_falcon_b200 import build, inputs as gen
+    build.build()
+    F.load()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    hbm, _, peak_src = peaks()
+    for n, var in ((2, "F1A"), (5, "F2A")):
+        w = gen.WORKLOADS[n]
+        d = gen.workload_inputs(n, var)
+        B, H, L, dk, dv = w["B"], w["H"], w["L"], w["dk"], w["dv"]
+        rng = np.random.default_rng(20260100 + n)
+        do = torch.from_numpy(rng.standard_normal((B, H, L, dv)).astype(np.float32)).to(torch.bfloat16).cuda()
+        ds = torch.from_numpy(rng.standard_normal((B, H, dv, dk)).astype(np.float32)).cuda()
+        a = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
+        F.bwd(var, *a, d["eps"], do, ds)
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush.zero_()
+            torch.cuda._sleep(HEAD_START_CYCLES)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            F.bwd(var, *a, d["eps"], do, ds)
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        t = statistics.median(ms)
+        nb = dv if var == "F2A" else 1
+        tok = B * H * L
+        ab = tok * (dk + dk + dv + nb + dv) * 2 + tok * (dk + dk + dv + nb) * 4 + B * H * dv * dk * 4
+        gbs = ab / (t / 1e3) / 1e9
+        line = {"backward": var, "workload": w["name"], "ms": t, "tokens_per_s": B * L / (t / 1e3),
+                "kernels": "bwd_prep_kernel + bwd_sweep_kernel + bwd_decay_kernel + bwd_key_kernel",
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                             "peak_source": peak_src, "algorithmic_bytes_per_launch": ab}}
+        if n == 2 and not args.no_cpu_baseline:
+            import oracle
+            oracle.build()
+            units = [(b, h) for b in range(B) for h in range(H)][:min(os.cpu_count() or 1, B * H)]
+            bs, hs = [u[0] for u in units], [u[1] for u in units]
+            sel = lambda x: np.ascontiguousarray(x[bs, hs][None])  # noqa: E731
+            t0 = time.perf_counter()
+            oracle.bwd(var, *(sel(d[k]) for k in ("q_64", "k_64", "v_64", "beta_64")), np.asarray(d["lam_64"])[hs],
+                       d["eps_64"], sel(do.double().cpu().numpy()), sel(ds.double().cpu().numpy()))
+            sec = time.perf_counter() - t0
+            line["cpu_oracle"] = {"value": len(units) * L / H / sec, "unit": "tokens/s", "cores": os.cpu_count(),
+                                  "kind": "oracle", "sample": "fp64 reverse mode, %d whole (b,h) units, %.1f s"
+                                  % (len(units), sec)}
+        print(json.dumps(line), flush=True)
+
+
 def workload_oracle_rate(d, variant, form, w):
     """The fp64 oracle in the row's own form -- the recurrent form for masked
     rows, whose O(L^2) oracle takes 7-80 s per (b,h) unit at L = 2048 -- on
@@ -581,6 +643,8 @@ def main():
     ap.add_argument("--workloads", action="store_true",
                     help="time every workload and form of the workloads table, one JSON line each")
     ap.add_argument("--only", type=int, default=0, help="with --workloads: just this workload number")
+    ap.add_argument("--backward", action="store_true",
+                    help="time falcon_bwd on workload 2 (Falcon-1A) and workload 5's prefill (Falcon-2A)")
     ap.add_argument("--chunk-sweep", action="store_true",
                     help="the chunk form of workload 2 at chunk 16/32/64 and both pairings (one line each)")
     ap.add_argument("--profile", action="store_true",
@@ -588,6 +652,8 @@ def main():
     args = ap.parse_args()
     if args.chunk_sweep:
         return run_chunk_sweep(args)
+    if args.backward:
+        return run_backward(args)
     if args.workloads:
         run_workloads(args)
     elif args.impl == "reference":
