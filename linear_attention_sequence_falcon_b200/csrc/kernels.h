@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include "params.h"
+#include "params_bwd.h"
 
 namespace falcon {
 

@@ -30,15 +30,6 @@ struct DecodeParams {
     void *out;
 };
 
-struct BwdParams {
-    int variant, pairing, phi;
-    int B, H, L, dk, dv;
-    float eps;
-    const void *q, *k, *v, *beta, *dout;
-    const float *lambda, *dstate;
-    float *dq, *dk_out, *dv_out, *dbeta, *dlambda;
-};
-
 struct CarryParams {
     int variant, window;
     int B, H, L, dk, dv;
