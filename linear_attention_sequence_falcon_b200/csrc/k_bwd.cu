@@ -19,10 +19,10 @@
 // beta / (eps + |x|^2) (0 at x = 0) and x = k / |k| (or k) take it to beta,
 // lambda and k.
 //
-// Three kernels: per-token samples and steps (a warp per token), the two
+// Four kernels: per-token samples and steps (a warp per token), the two
 // sweeps per head (a block per (b, h); S, then Gs, in shared memory; tokens
-// staged 32 at a time), and the decay chain (a reverse scan per (b, h,
-// channel), then a warp per token for the feature map).
+// staged 32 at a time), the decay chain (a block-wide reverse scan per (b, h,
+// channel)) and a warp per token for the feature map.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -219,35 +219,83 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
     }
 }
 
-// decay chain per (b, h, channel): dlog alpha_t = sum_{t'>=t} (ga - gb)_t',
-// then alpha and eta; writes dbeta, the total deta (for |x|^2), dlambda
+// decay chain: one block per (b, h, channel).  dlog alpha_t = sum_{t'>=t}
+// (ga - gb)_t' as a block-wide reverse scan over tiles of 2048 tokens (eight
+// per thread, latest tile first, the sum of the later tiles carried), then
+// alpha and eta per token; writes dbeta, each channel's share of dL/d|x|^2
+// (over deta) and dlambda.
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float *ns, const float *etas,
                                                        const float *alphas, const float *dga, const float *dgb,
                                                        float *deta) {
+    constexpr int PER = 8, TS = 256 * PER;
+    __shared__ float wsum[8];
+    __shared__ float wlam[8];
     const int nch = p.variant == F2A ? p.dv : 1;
-    const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= (size_t)p.B * p.H * nch) return;
-    const size_t bh = gid / nch;
-    const int ch = (int)(gid % nch), L = p.L;
+    const size_t bh = blockIdx.x / nch;
+    const int ch = (int)(blockIdx.x % nch), L = p.L, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float lam = p.lambda[bh % p.H];
     const T *beta = static_cast<const T *>(p.beta) + bh * (size_t)L * nch;
-    float run = 0.f, dlam = 0.f;
-    for (int t = L - 1; t >= 0; --t) {
-        const size_t i = (bh * L + t) * nch + ch;
-        run += dga[i] - dgb[i];
-        const float a = alphas[i], eta = etas[i], n = ns[bh * L + t];
-        const float dalpha = run / a;
-        float d = deta[i];
-        if (1.f - eta * lam > kAlphaFloor) {
-            d -= lam * dalpha;
-            dlam -= eta * dalpha;
+    float carry = 0.f, dlam = 0.f;
+    for (int t1 = L; t1 > 0; t1 -= TS) {
+        const int t0 = max(0, t1 - TS), base = t0 + tid * PER;
+        float v[PER], sfx[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int t = base + k;
+            const size_t i = (bh * L + t) * nch + ch;
+            v[k] = t < t1 ? dga[i] - dgb[i] : 0.f;
         }
-        p.dbeta[i] = n > 0.f ? d / (p.eps + n) : 0.f;
-        // dL/dn_t share of this channel
-        deta[i] = n > 0.f ? -d * ld(beta, (size_t)t * nch + ch) / ((p.eps + n) * (p.eps + n)) : 0.f;
+        float run = 0.f;
+#pragma unroll
+        for (int k = PER - 1; k >= 0; --k) {
+            run += v[k];
+            sfx[k] = run;  // sum over this thread's tokens >= base + k
+        }
+        // suffix sums over the later threads of the warp, then over the later warps
+        float x = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, x, o);
+            if (lane + o < 32) x += y;
+        }
+        if (lane == 0) wsum[warp] = x;
+        __syncthreads();
+        float later = x - run;
+        float tile = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            if (w > warp) later += wsum[w];
+            tile += wsum[w];
+        }
+        later += carry;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int t = base + k;
+            if (t >= t1) continue;
+            const size_t i = (bh * L + t) * nch + ch;
+            const float dlog = sfx[k] + later;
+            const float a = alphas[i], eta = etas[i], n = ns[bh * L + t];
+            const float dalpha = dlog / a;
+            float d = deta[i];
+            if (1.f - eta * lam > kAlphaFloor) {
+                d -= lam * dalpha;
+                dlam -= eta * dalpha;
+            }
+            p.dbeta[i] = n > 0.f ? d / (p.eps + n) : 0.f;
+            deta[i] = n > 0.f ? -d * ld(beta, (size_t)t * nch + ch) / ((p.eps + n) * (p.eps + n)) : 0.f;
+        }
+        carry += tile;
+        __syncthreads();
     }
-    if (p.dlambda) atomicAdd(&p.dlambda[bh % p.H], dlam);
+    dlam = group_sum<32>(dlam);
+    if (lane == 0) wlam[warp] = dlam;
+    __syncthreads();
+    if (tid == 0 && p.dlambda) {
+        float s = 0.f;
+        for (int w = 0; w < 8; ++w) s += wlam[w];
+        atomicAdd(&p.dlambda[bh % p.H], s);
+    }
 }
 
 // a warp per (b, h, t): dx_t += 2 dn_t x_t, then dk of the key x_t came from
@@ -324,7 +372,7 @@ int launch_bwd(const BwdParams &p, cudaStream_t s) {
                      : launch_sweep<T, 128>(p, xs, etas, alphas, dga, dgb, deta, dx, s);
     const size_t chans = (size_t)p.B * p.H * nch;
     if (p.dlambda) cudaMemsetAsync(p.dlambda, 0, sizeof(float) * p.H, s);
-    bwd_decay_kernel<T><<<(unsigned)((chans + 255) / 256), 256, 0, s>>>(p, ns, etas, alphas, dga, dgb, deta);
+    bwd_decay_kernel<T><<<(unsigned)chans, 256, 0, s>>>(p, ns, etas, alphas, dga, dgb, deta);
     bwd_key_kernel<T><<<wblocks, 256, 0, s>>>(p, xs, deta, dx);
     const cudaError_t e = cudaGetLastError();
     scratch_free(ws, s);
