@@ -158,7 +158,8 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
  *   then alpha = max(1 - eta lambda, 2^-20) (no gradient on the floor),
  *   eta = beta/(eps + |x|^2) and x = phi(k).
  *
- *   variant     FALCON_F1A or FALCON_F2A (others: FALCON_ERR_UNSUPPORTED)
+ *   variant     FALCON_F1, FALCON_F2, FALCON_F1A or FALCON_F2A (the windowed
+ *               variants: FALCON_ERR_UNSUPPORTED)
  *   dtype, q, k, v, beta, lambda, eps, B, H, L, pairing, phi: as in
  *               falcon_fwd_ex; d_k = d_v in {32, 64, 128}
  *   dout        [B,H,L,d_v] dtype: dL/d(out)
@@ -167,9 +168,12 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
  *   dv          [B,H,L,d_v] fp32, written
  *   dbeta       [B,H,L] (Falcon-1A) or [B,H,L,d_v] (Falcon-2A) fp32, written
  *   dlambda     [H] fp32, written (summed over b), or NULL
- * Scratch: (2 L d + L + 5 L c) floats per (b,h), c = 1 or d_v, stream-ordered
- * from the library's pool (FALCON_ERR_ALLOC if that fails).  Errors as in
- * falcon_fwd.
+ * The regression family's derivative needs S_{t-1} at every step: the
+ * forward sweep keeps S every 32 tokens and the reverse sweep recomputes
+ * each 32-token stretch from it.
+ * Scratch: (2 L d + L + 5 L c) floats per (b,h), c = 1 or d_v, plus
+ * (ceil(L/32) + 32) d^2 for the regression family, stream-ordered from the
+ * library's pool (FALCON_ERR_ALLOC if that fails).  Errors as in falcon_fwd.
  */
 int falcon_bwd(falcon_variant variant, falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
                const void *q, const void *k, const void *v, const void *beta, const float *lambda, float eps,

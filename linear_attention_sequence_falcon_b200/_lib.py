@@ -130,8 +130,8 @@ def bwd(variant: str, q, k, v, beta, lam, eps: float, dout, dstate=None, pairing
         phi: str = "l2", stream=None):
     """falcon_bwd: gradients of a loss with respect to q, k, v, beta and lambda
     of a forward from S_0 = 0, given dout = dL/d(out) (dtype of q) and dstate =
-    dL/d(final_state) (fp32, or None).  Falcon-1A and Falcon-2A, d_k = d_v in
-    {32, 64, 128}.  Returns a dict of fp32 tensors dq, dk, dv, dbeta, dlambda."""
+    dL/d(final_state) (fp32, or None).  Falcon-1/2 and Falcon-1A/2A, d_k = d_v
+    in {32, 64, 128}.  Returns a dict of fp32 tensors dq, dk, dv, dbeta, dlambda."""
     lib = load()
     B, H, L, dk = q.shape
     dv = v.shape[-1]

@@ -172,7 +172,7 @@ extern "C" int falcon_bwd(falcon_variant variant, falcon_dtype dtype, falcon_pai
     if (pairing != FALCON_PAIR_PREFIX && pairing != FALCON_PAIR_SAME_STEP) return FALCON_ERR_ENUM;
     if (phi != FALCON_PHI_L2 && phi != FALCON_PHI_IDENTITY) return FALCON_ERR_ENUM;
     if (B < 0 || H < 0 || L < 0 || !dim_ok(d_k) || !dim_ok(d_v)) return FALCON_ERR_SHAPE;
-    if (variant != FALCON_F1A && variant != FALCON_F2A) return FALCON_ERR_UNSUPPORTED;
+    if (variant == FALCON_F3 || variant == FALCON_F3A) return FALCON_ERR_UNSUPPORTED;
     if (d_k != d_v || d_k < 32) return FALCON_ERR_UNSUPPORTED;
     if ((size_t)B * H == 0) return FALCON_OK;
     if (L == 0) {

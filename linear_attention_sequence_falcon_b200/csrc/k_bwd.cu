@@ -1,7 +1,8 @@
-// k_bwd.cu -- backward pass of the inner-product family (Falcon-1A and
-// Falcon-2A, one sample per update) in the recurrent form, fp32 on the CUDA
-// cores: the gradients of a loss with respect to q, k, v, beta and lambda,
-// given dL/do (and dL/dS_L).
+// k_bwd.cu -- backward pass of Falcon-1/2 and Falcon-1A/2A (one sample per
+// update) in the recurrent form, fp32 on the CUDA cores: the gradients of a
+// loss with respect to q, k, v, beta and lambda, given dL/do (and dL/dS_L).
+// The inner-product family is described first; the regression family's sweep
+// (bwd_sweep_reg_kernel) follows it.
 //
 // The chunk form trains on the recurrent function (page "Fast Weight
 // Attention：用于持续学习的快速权重注意力", 核心方法 3); its derivative, with
@@ -60,7 +61,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdParams p, float *xs, f
     for (int c = lane; c < D; c += 32) xs[gw * D + c] = kr >= 0 ? ld(k, (size_t)kr * D + c) * inv : 0.f;
     const float n = ss * inv * inv;
     if (lane == 0) ns[gw] = n;
-    const int nch = p.variant == F2A ? p.dv : 1;
+    const int nch = (p.variant == F2A || p.variant == F2) ? p.dv : 1;
     const float lam = p.lambda[bh % p.H];
     const T *beta = static_cast<const T *>(p.beta) + bh * (size_t)p.L * nch;
     for (int ch = lane; ch < nch; ch += 32) {
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
     float *ta_next = ta + TT * D;                   // alpha of the token after the tile ([D])
     const int tid = threadIdx.x, L = p.L;
     const size_t bh = blockIdx.x;
-    const int nch = p.variant == F2A ? D : 1;
+    const int nch = (p.variant == F2A || p.variant == F2) ? D : 1;
     const T *q = static_cast<const T *>(p.q) + bh * (size_t)L * D;
     const T *v = static_cast<const T *>(p.v) + bh * (size_t)L * D;
     const T *dout = static_cast<const T *>(p.dout) + bh * (size_t)L * D;
@@ -219,6 +220,193 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
     }
 }
 
+// The regression family (Falcon-1 / Falcon-2): S_t = alpha_t S_{t-1} +
+// eta_t (y_t - S_{t-1} x_t) x_t^T.  Its derivative needs S_{t-1} at every
+// step of the reverse sweep: the forward sweep keeps S at the start of every
+// tile of TT tokens (ck), and the reverse sweep recomputes a tile's states
+// from its checkpoint (ts, global scratch of the block) before walking it
+// backwards.  Per step, with Gs = dL/dS_t (do_t q_t^T added):
+//   e = y - S_{t-1} x,  de = eta (Gs x),  dalpha = <Gs, S_{t-1}> (per row),
+//   deta = e . (Gs x) (per row),  dy = de,
+//   dx = Gs^T (eta o e) - S_{t-1}^T de,  Gs <- alpha o Gs - de x^T.
+// dalpha is written straight into dga (the scan is not needed here).
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, const float *xs, const float *etas,
+                                                              const float *alphas, float *dga, float *deta, float *dx,
+                                                              float *ck, float *ts) {
+    constexpr int NT = 256, LD = D + 1, RPT = NT / D, SEG = D / RPT;
+    extern __shared__ float sm[];
+    float *S = sm;                                  // [D][LD]: S, then Gs
+    float *tq = S + D * LD, *tdo = tq + TT * D;
+    float *ty = tdo + TT * D, *tx = ty + TT * D;
+    float *te = tx + TT * D, *ta = te + TT * D;
+    float *ve = ta + TT * D, *vde = ve + D;         // [D] e_j and de_j of the current step
+    float *vsum = vde + D;                          // [3 * D] row sums for the Falcon-1 totals
+    const int tid = threadIdx.x, L = p.L;
+    const size_t bh = blockIdx.x;
+    const int nch = p.variant == F2 ? D : 1;
+    const T *q = static_cast<const T *>(p.q) + bh * (size_t)L * D;
+    const T *v = static_cast<const T *>(p.v) + bh * (size_t)L * D;
+    const T *dout = static_cast<const T *>(p.dout) + bh * (size_t)L * D;
+    const float *x = xs + bh * (size_t)L * D;
+    const float *et = etas + bh * (size_t)L * nch, *al = alphas + bh * (size_t)L * nch;
+    float *dq = p.dq + bh * (size_t)L * D, *dv = p.dv_out + bh * (size_t)L * D;
+    float *ga = dga + bh * (size_t)L * nch, *de = deta + bh * (size_t)L * nch;
+    float *dxo = dx + bh * (size_t)L * D;
+    const int ntile = (L + TT - 1) / TT;
+    float *cks = ck + bh * (size_t)ntile * D * D;   // S before each tile
+    float *tss = ts + bh * (size_t)TT * D * D;      // S before each token of the tile being walked
+
+    auto stage = [&](int t0, int n) {
+        for (int e = tid; e < TT * D; e += NT) {
+            const int i = e / D, c = e % D, t = t0 + i;
+            const bool in = i < n;
+            tq[e] = in ? ld(q, (size_t)t * D + c) : 0.f;
+            tdo[e] = in ? ld(dout, (size_t)t * D + c) : 0.f;
+            ty[e] = in ? ld(v, (size_t)t * D + c) : 0.f;
+            tx[e] = in ? x[(size_t)t * D + c] : 0.f;
+            te[e] = in ? et[(size_t)t * nch + (nch > 1 ? c : 0)] : 0.f;
+            ta[e] = in ? al[(size_t)t * nch + (nch > 1 ? c : 0)] : 1.f;
+        }
+    };
+    const int rj = tid / RPT, rp = tid % RPT;
+    // one regression step on the state in S with token i of the staged tile
+    auto step = [&](int i) {
+        float r = 0.f;  // (S x)_rj
+#pragma unroll 8
+        for (int s = 0; s < SEG; ++s) {
+            const int c = rp * SEG + s;
+            r = fmaf(S[rj * LD + c], tx[i * D + c], r);
+        }
+#pragma unroll
+        for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o2);
+        if (rp == 0) ve[rj] = ty[i * D + rj] - r;
+        __syncthreads();
+        for (int e = tid; e < D * D; e += NT) {
+            const int j = e / D, c = e % D;
+            S[j * LD + c] = ta[i * D + j] * S[j * LD + c] + te[i * D + j] * ve[j] * tx[i * D + c];
+        }
+        __syncthreads();
+    };
+
+    // ---- forward sweep: checkpoints, S_t, dq_t = S_t^T do_t
+    for (int e = tid; e < D * LD; e += NT) S[e] = 0.f;
+    for (int tb = 0; tb < ntile; ++tb) {
+        const int t0 = tb * TT, n = min(TT, L - t0);
+        __syncthreads();
+        stage(t0, n);
+        for (int e = tid; e < D * D; e += NT) cks[(size_t)tb * D * D + e] = S[(e / D) * LD + e % D];
+        __syncthreads();
+        for (int i = 0; i < n; ++i) {
+            step(i);
+            float g = 0.f;
+#pragma unroll 8
+            for (int s = 0; s < SEG; ++s) {
+                const int c = rp * SEG + s;
+                g = fmaf(S[c * LD + rj], tdo[i * D + c], g);
+            }
+#pragma unroll
+            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) g += __shfl_xor_sync(0xffffffffu, g, o2);
+            if (rp == 0) dq[(size_t)(t0 + i) * D + rj] = g;
+        }
+    }
+    // ---- reverse sweep, tile by tile; Gs = dL/dS in S between tiles
+    __syncthreads();
+    for (int e = tid; e < D * D; e += NT) {
+        const int j = e / D, c = e % D;
+        S[j * LD + c] = p.dstate ? p.dstate[(bh * D + j) * D + c] : 0.f;  // dL/dS_L
+    }
+    for (int tb = ntile - 1; tb >= 0; --tb) {
+        const int t0 = tb * TT, n = min(TT, L - t0);
+        float *ckt = cks + (size_t)tb * D * D;
+        __syncthreads();
+        stage(t0, n);
+        // swap Gs and the tile's checkpoint (each element by one thread)
+        for (int e = tid; e < D * D; e += NT) {
+            const int j = e / D, c = e % D;
+            const float sv = ckt[e];
+            ckt[e] = S[j * LD + c];
+            S[j * LD + c] = sv;
+        }
+        __syncthreads();
+        // recompute the tile: tss[i] = S before token t0 + i
+        for (int i = 0; i < n; ++i) {
+            for (int e = tid; e < D * D; e += NT) tss[(size_t)i * D * D + e] = S[(e / D) * LD + e % D];
+            step(i);
+        }
+        for (int e = tid; e < D * D; e += NT) S[(e / D) * LD + e % D] = ckt[e];
+        __syncthreads();
+        for (int i = n - 1; i >= 0; --i) {
+            const int t = t0 + i;
+            const float *Sp = tss + (size_t)i * D * D;
+            for (int e = tid; e < D * D; e += NT) {
+                const int j = e / D, c = e % D;
+                S[j * LD + c] += tdo[i * D + j] * tq[i * D + c];
+            }
+            __syncthreads();
+            float sx = 0.f, gx = 0.f, gs = 0.f;  // row rj: (S_{t-1} x), (Gs x), <Gs, S_{t-1}>
+#pragma unroll 8
+            for (int s2 = 0; s2 < SEG; ++s2) {
+                const int c = rp * SEG + s2;
+                const float sp = Sp[(size_t)rj * D + c], g = S[rj * LD + c];
+                sx = fmaf(sp, tx[i * D + c], sx);
+                gx = fmaf(g, tx[i * D + c], gx);
+                gs = fmaf(g, sp, gs);
+            }
+#pragma unroll
+            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
+                sx += __shfl_xor_sync(0xffffffffu, sx, o2);
+                gx += __shfl_xor_sync(0xffffffffu, gx, o2);
+                gs += __shfl_xor_sync(0xffffffffu, gs, o2);
+            }
+            if (rp == 0) {
+                const float eta = te[i * D + rj], e = ty[i * D + rj] - sx, d = eta * gx;
+                ve[rj] = eta * e;
+                vde[rj] = d;
+                dv[(size_t)t * D + rj] = d;
+                if (nch > 1) {
+                    ga[(size_t)t * D + rj] = gs;
+                    de[(size_t)t * D + rj] = e * gx;
+                } else {
+                    vsum[rj] = gs;
+                    vsum[D + rj] = e * gx;
+                }
+            }
+            __syncthreads();
+            float dxc = 0.f;  // column rj: sum_j (eta e)_j Gs[j][c] - de_j S_{t-1}[j][c]
+#pragma unroll 8
+            for (int s2 = 0; s2 < SEG; ++s2) {
+                const int j = rp * SEG + s2;
+                dxc = fmaf(ve[j], S[j * LD + rj], dxc);
+                dxc = fmaf(-vde[j], Sp[(size_t)j * D + rj], dxc);
+            }
+#pragma unroll
+            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) dxc += __shfl_xor_sync(0xffffffffu, dxc, o2);
+            if (rp == 0) dxo[(size_t)t * D + rj] = dxc;
+            if (nch == 1 && tid < 32) {
+                float a = 0.f, b = 0.f;
+                for (int j = tid; j < D; j += 32) {
+                    a += vsum[j];
+                    b += vsum[D + j];
+                }
+                a = group_sum<32>(a);
+                b = group_sum<32>(b);
+                if (tid == 0) {
+                    ga[t] = a;
+                    de[t] = b;
+                }
+            }
+            __syncthreads();
+            // Gs <- alpha o Gs - de x^T (dL/dS_{t-1})
+            for (int e = tid; e < D * D; e += NT) {
+                const int j = e / D, c = e % D;
+                S[j * LD + c] = ta[i * D + j] * S[j * LD + c] - vde[j] * tx[i * D + c];
+            }
+            __syncthreads();
+        }
+    }
+}
+
 // decay chain: one block per (b, h, channel).  dlog alpha_t = sum_{t'>=t}
 // (ga - gb)_t' as a block-wide reverse scan over tiles of 2048 tokens (eight
 // per thread, latest tile first, the sum of the later tiles carried), then
@@ -231,9 +419,10 @@ __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float
     constexpr int PER = 8, TS = 256 * PER;
     __shared__ float wsum[8];
     __shared__ float wlam[8];
-    const int nch = p.variant == F2A ? p.dv : 1;
+    const int nch = (p.variant == F2A || p.variant == F2) ? p.dv : 1;
     const size_t bh = blockIdx.x / nch;
     const int ch = (int)(blockIdx.x % nch), L = p.L, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool reg = p.variant == F1 || p.variant == F2;
     const float lam = p.lambda[bh % p.H];
     const T *beta = static_cast<const T *>(p.beta) + bh * (size_t)L * nch;
     float carry = 0.f, dlam = 0.f;
@@ -244,7 +433,7 @@ __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float
         for (int k = 0; k < PER; ++k) {
             const int t = base + k;
             const size_t i = (bh * L + t) * nch + ch;
-            v[k] = t < t1 ? dga[i] - dgb[i] : 0.f;
+            v[k] = (t < t1 && !reg) ? dga[i] - dgb[i] : 0.f;
         }
         float run = 0.f;
 #pragma unroll
@@ -274,9 +463,9 @@ __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float
             const int t = base + k;
             if (t >= t1) continue;
             const size_t i = (bh * L + t) * nch + ch;
-            const float dlog = sfx[k] + later;
             const float a = alphas[i], eta = etas[i], n = ns[bh * L + t];
-            const float dalpha = dlog / a;
+            // the regression family's sweep gives dL/dalpha directly
+            const float dalpha = reg ? dga[i] : (sfx[k] + later) / a;
             float d = deta[i];
             if (1.f - eta * lam > kAlphaFloor) {
                 d -= lam * dalpha;
@@ -306,7 +495,7 @@ __global__ void __launch_bounds__(256) bwd_key_kernel(BwdParams p, const float *
     if (gw >= (size_t)p.B * p.H * p.L) return;
     const int D = p.dk, L = p.L, t = (int)(gw % L);
     const size_t bh = gw / L;
-    const int nch = p.variant == F2A ? p.dv : 1;
+    const int nch = (p.variant == F2A || p.variant == F2) ? p.dv : 1;
     float dn = 0.f;
     for (int ch = lane; ch < nch; ch += 32) dn += dnc[gw * nch + ch];
     dn = group_sum<32>(dn);
@@ -341,7 +530,13 @@ __global__ void __launch_bounds__(256) bwd_key_kernel(BwdParams p, const float *
 
 template <typename T, int D>
 int launch_sweep(const BwdParams &p, const float *xs, const float *etas, const float *alphas, float *dga, float *dgb,
-                 float *deta, float *dx, cudaStream_t s) {
+                 float *deta, float *dx, float *ck, float *ts, cudaStream_t s) {
+    if (p.variant == F1 || p.variant == F2) {
+        const size_t bytes = ((size_t)D * (D + 1) + 6 * TT * D + 5 * D) * sizeof(float);
+        cudaFuncSetAttribute(bwd_sweep_reg_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        bwd_sweep_reg_kernel<T, D><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
+        return 0;
+    }
     const size_t bytes = ((size_t)D * (D + 1) + 6 * TT * D + D) * sizeof(float);
     cudaFuncSetAttribute(bwd_sweep_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     bwd_sweep_kernel<T, D><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
@@ -352,11 +547,15 @@ int launch_sweep(const BwdParams &p, const float *xs, const float *etas, const f
 
 template <typename T>
 int launch_bwd(const BwdParams &p, cudaStream_t s) {
-    const int D = p.dk, nch = p.variant == F2A ? D : 1;
+    const int D = p.dk, nch = (p.variant == F2A || p.variant == F2) ? D : 1;
+    const bool reg = p.variant == F1 || p.variant == F2;
     const size_t rows = (size_t)p.B * p.H * p.L;
     if (rows == 0) return 0;
-    // scratch: x, |x|^2, eta, alpha, the two decay-gradient halves, deta, dx
-    const size_t nf = rows * D * 2 + rows + rows * nch * 5;
+    // scratch: x, |x|^2, eta, alpha, the two decay-gradient halves, deta, dx;
+    // the regression family adds the tile checkpoints and one tile of states per head
+    const size_t BH = (size_t)p.B * p.H, ntile = (p.L + TT - 1) / TT;
+    const size_t nreg = reg ? BH * (ntile + TT) * D * D : 0;
+    const size_t nf = rows * D * 2 + rows + rows * nch * 5 + nreg;
     void *ws = nullptr;
     if (scratch_alloc(&ws, nf * sizeof(float), s) != cudaSuccess) {
         cudaGetLastError();
@@ -365,11 +564,12 @@ int launch_bwd(const BwdParams &p, cudaStream_t s) {
     float *xs = static_cast<float *>(ws), *dx = xs + rows * D, *ns = dx + rows * D;
     float *etas = ns + rows, *alphas = etas + rows * nch, *dga = alphas + rows * nch, *dgb = dga + rows * nch;
     float *deta = dgb + rows * nch;
+    float *ck = deta + rows * nch, *ts = ck + BH * ntile * D * D;
     const unsigned wblocks = (unsigned)((rows * 32 + 255) / 256);
     bwd_prep_kernel<T><<<wblocks, 256, 0, s>>>(p, xs, ns, etas, alphas);
-    int rc = D == 32 ? launch_sweep<T, 32>(p, xs, etas, alphas, dga, dgb, deta, dx, s)
-           : D == 64 ? launch_sweep<T, 64>(p, xs, etas, alphas, dga, dgb, deta, dx, s)
-                     : launch_sweep<T, 128>(p, xs, etas, alphas, dga, dgb, deta, dx, s);
+    int rc = D == 32 ? launch_sweep<T, 32>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
+           : D == 64 ? launch_sweep<T, 64>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
+                     : launch_sweep<T, 128>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s);
     const size_t chans = (size_t)p.B * p.H * nch;
     if (p.dlambda) cudaMemsetAsync(p.dlambda, 0, sizeof(float) * p.H, s);
     bwd_decay_kernel<T><<<(unsigned)chans, 256, 0, s>>>(p, ns, etas, alphas, dga, dgb, deta);

@@ -81,8 +81,8 @@ def test_backward_validation_codes(lib):
     assert _bwd(lib, pairing=2) == -2
     assert _bwd(lib, phi=3) == -2
     assert _bwd(lib, dk=48) == -3
-    assert _bwd(lib, variant=0) == -9   # regression family: not in the backward kernel
-    assert _bwd(lib, variant=5) == -9   # windows: not in the backward kernel
+    assert _bwd(lib, variant=2) == -9   # windows: not in the backward kernels
+    assert _bwd(lib, variant=5) == -9
     assert _bwd(lib, dk=64, dv=32) == -9
     assert _bwd(lib, dk=16, dv=16) == -9
     assert _bwd(lib, ptr=0) == -1

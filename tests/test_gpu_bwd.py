@@ -1,4 +1,4 @@
-"""GPU parity of falcon_bwd (the backward pass of Falcon-1A / Falcon-2A)
+"""GPU parity of falcon_bwd (the backward pass of Falcon-1/2 and Falcon-1A/2A)
 against the fp64 oracle's reverse mode of the recurrent definition
 (oracle.bwd, pinned by finite differences in test_oracle_bwd.py), on the same
 seeded inputs.
@@ -73,7 +73,7 @@ def check(got, ref, tol=TOL):
         assert e <= tol, f"{n}: {e:.3e} (tol {tol})"
 
 
-@pytest.mark.parametrize("variant", ["F1A", "F2A"])
+@pytest.mark.parametrize("variant", ["F1", "F2", "F1A", "F2A"])
 @pytest.mark.parametrize("d", [32, 64, 128])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("L", [1, 37, 100])
@@ -83,14 +83,14 @@ def test_backward_parity(F, variant, d, dtype, L):
     check(got, ref)
 
 
-@pytest.mark.parametrize("variant", ["F1A", "F2A"])
+@pytest.mark.parametrize("variant", ["F1", "F2", "F1A", "F2A"])
 @pytest.mark.parametrize("pairing,phi", [("same_step", "l2"), ("prefix", "identity"), ("same_step", "identity")])
 def test_backward_pairing_and_feature_map(F, variant, pairing, phi):
     got, ref = grads_case(F, variant, 1, 2, 70, 64, "f32", seed=231, pairing=pairing, phi=phi, key_scale=0.3)
     check(got, ref)
 
 
-@pytest.mark.parametrize("variant", ["F1A", "F2A"])
+@pytest.mark.parametrize("variant", ["F1", "F2", "F1A", "F2A"])
 def test_backward_without_state_gradient_and_with_clamped_decay(F, variant):
     """dstate = NULL, and lambda = 0.9 with tiny keys under the identity map:
     eta = beta/(eps+|x|^2) is large, alpha sits on its 2^-20 floor for most
@@ -111,15 +111,16 @@ def test_backward_empty_sequence(F):
     assert torch.count_nonzero(g["dlambda"]) == 0
 
 
-@pytest.mark.parametrize("variant", ["F1A"])
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
 def test_backward_workload2_sampled(F, variant):
     """The workload-2 shape (8x12x2048x64 bf16): three sampled (b, h) units."""
     got, ref = grads_case(F, variant, 8, 12, 2048, 64, "bf16", seed=20260002, units=[(0, 0), (3, 7), (7, 11)])
     check(got, ref)
 
 
-def test_backward_rejects_other_variants(F):
-    d_ = gen.draw("F1", 1, 1, 8, 64, 64, seed=2, dtype="f32")
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+def test_backward_rejects_the_windowed_variants(F, variant):
+    d_ = gen.draw(variant, 1, 1, 8, 64, 64, seed=2, dtype="f32")
     with pytest.raises(F.FalconError):
-        F.bwd("F1", *(d_[n].cuda() for n in ("q", "k", "v", "beta", "lam")), d_["eps"],
+        F.bwd(variant, *(d_[n].cuda() for n in ("q", "k", "v", "beta", "lam")), d_["eps"],
               torch.zeros((1, 1, 8, 64), device="cuda"))
