@@ -540,9 +540,9 @@ def run_chunk_sweep(args):
 
 
 def run_backward(args):
-    """--backward: falcon_bwd (the backward pass of Falcon-1A / Falcon-2A) on
-    workload 2 (Falcon-1A, 8x12x2048x64 bf16) and on workload 5's prefill
-    (Falcon-2A, 2x16x32768x128 bf16): CUDA events around one call after a
+    """--backward: falcon_bwd on workload 2 (Falcon-1 and Falcon-1A,
+    8x12x2048x64 bf16), workload 3 (Falcon-2, 4x16x4096x128) and workload 5's
+    prefill (Falcon-2A, 2x16x32768x128 bf16): CUDA events around one call after a
     warm-up call, L2 flushed, median of --steps calls (3..10); an HBM
     roofline on the algorithmic bytes (q, k, v, beta, dout read; dq, dk, dv,
     dbeta written in fp32) and the fp64 oracle's reverse mode on whole (b,h)
@@ -556,7 +556,7 @@ def run_backward(args):
     F.load()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     hbm, _, peak_src = peaks()
-    for n, var in ((2, "F1A"), (5, "F2A")):
+    for n, var in ((2, "F1"), (2, "F1A"), (3, "F2"), (5, "F2A")):
         w = gen.WORKLOADS[n]
         d = gen.workload_inputs(n, var)
         B, H, L, dk, dv = w["B"], w["H"], w["L"], w["dk"], w["dv"]
@@ -577,7 +577,7 @@ def run_backward(args):
             torch.cuda.synchronize()
             ms.append(e0.elapsed_time(e1))
         t = statistics.median(ms)
-        nb = dv if var == "F2A" else 1
+        nb = dv if var in ("F2", "F2A") else 1
         tok = B * H * L
         ab = tok * (dk + dk + dv + nb + dv) * 2 + tok * (dk + dk + dv + nb) * 4 + B * H * dv * dk * 4
         gbs = ab / (t / 1e3) / 1e9
@@ -644,7 +644,7 @@ def main():
                     help="time every workload and form of the workloads table, one JSON line each")
     ap.add_argument("--only", type=int, default=0, help="with --workloads: just this workload number")
     ap.add_argument("--backward", action="store_true",
-                    help="time falcon_bwd on workload 2 (Falcon-1A) and workload 5's prefill (Falcon-2A)")
+                    help="time falcon_bwd on workloads 2 (Falcon-1, -1A), 3 (Falcon-2) and 5's prefill (Falcon-2A)")
     ap.add_argument("--chunk-sweep", action="store_true",
                     help="the chunk form of workload 2 at chunk 16/32/64 and both pairings (one line each)")
     ap.add_argument("--profile", action="store_true",
