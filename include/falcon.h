@@ -150,7 +150,8 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
  * to q, k, v, beta and lambda, given dL/d(out) and dL/d(final_state), for a
  * forward from S_0 = 0 with the same arguments.  The chunk form trains on the
  * recurrent function ([EXPL] 核心方法 3); this is its derivative, taken in
- * the recurrent form on the CUDA cores (fp32):
+ * the recurrent form on the CUDA cores (fp32); shown here for one sample per
+ * update (a window sums the same terms over its samples):
  *   dq_t = S_t^T do_t;  Gs_t = do_t q_t^T + alpha_{t+1} Gs_{t+1};
  *   dv_t = eta_t (Gs_t x_t);  the decays through dL/dG_t = do_t o_t - eta_t
  *   y_t (Gs_t x_t) (+ <dL/dS_L, S_L> at the last token) summed from t
@@ -158,10 +159,10 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
  *   then alpha = max(1 - eta lambda, 2^-20) (no gradient on the floor),
  *   eta = beta/(eps + |x|^2) and x = phi(k).
  *
- *   variant     FALCON_F1, FALCON_F2, FALCON_F1A or FALCON_F2A (the windowed
- *               variants: FALCON_ERR_UNSUPPORTED)
+ *   variant     any; window as in falcon_fwd (1..8 for Falcon-3/3A)
  *   dtype, q, k, v, beta, lambda, eps, B, H, L, pairing, phi: as in
- *               falcon_fwd_ex; d_k = d_v in {32, 64, 128}
+ *               falcon_fwd_ex; d_k = d_v in {32, 64, 128} (other shapes:
+ *               FALCON_ERR_UNSUPPORTED)
  *   dout        [B,H,L,d_v] dtype: dL/d(out)
  *   dstate      [B,H,d_v,d_k] fp32, or NULL (zero): dL/d(final_state)
  *   dq, dk      [B,H,L,d_k] fp32, written
@@ -177,7 +178,7 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
  */
 int falcon_bwd(falcon_variant variant, falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
                const void *q, const void *k, const void *v, const void *beta, const float *lambda, float eps,
-               int B, int H, int L, int d_k, int d_v, const void *dout, const float *dstate,
+               int window, int B, int H, int L, int d_k, int d_v, const void *dout, const float *dstate,
                float *dq, float *dk, float *dv, float *dbeta, float *dlambda, cudaStream_t stream);
 
 /*

@@ -47,7 +47,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.falcon_fwd_ex.restype = I
     lib.falcon_fwd_carry.argtypes = [I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, I, P, P, P, P, P, P]
     lib.falcon_fwd_carry.restype = I
-    lib.falcon_bwd.argtypes = [I, I, I, I, P, P, P, P, P, F, I, I, I, I, I, P, P, P, P, P, P, P, P]
+    lib.falcon_bwd.argtypes = [I, I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, P, P, P, P, P, P, P, P]
     lib.falcon_bwd.restype = I
     lib.falcon_decode_step.argtypes = [I, I, P, P, P, P, P, F, I, I, I, I, I, P, P, P, P, P]
     lib.falcon_decode_step.restype = I
@@ -126,12 +126,12 @@ def fwd(variant: str, form: str, q, k, v, beta, lam, eps: float, window: int = 1
     return out, final_state
 
 
-def bwd(variant: str, q, k, v, beta, lam, eps: float, dout, dstate=None, pairing: str = "prefix",
+def bwd(variant: str, q, k, v, beta, lam, eps: float, dout, dstate=None, window: int = 1, pairing: str = "prefix",
         phi: str = "l2", stream=None):
     """falcon_bwd: gradients of a loss with respect to q, k, v, beta and lambda
     of a forward from S_0 = 0, given dout = dL/d(out) (dtype of q) and dstate =
-    dL/d(final_state) (fp32, or None).  Falcon-1/2 and Falcon-1A/2A, d_k = d_v
-    in {32, 64, 128}.  Returns a dict of fp32 tensors dq, dk, dv, dbeta, dlambda."""
+    dL/d(final_state) (fp32, or None).  Every variant (window for Falcon-3/3A),
+    d_k = d_v in {32, 64, 128}.  Returns a dict of fp32 tensors dq, dk, dv, dbeta, dlambda."""
     lib = load()
     B, H, L, dk = q.shape
     dv = v.shape[-1]
@@ -144,7 +144,7 @@ def bwd(variant: str, q, k, v, beta, lam, eps: float, dout, dstate=None, pairing
          "dv": torch.empty((B, H, L, dv), **f32), "dbeta": torch.empty(tuple(beta.shape), **f32),
          "dlambda": torch.zeros((H,), **f32)}
     rc = lib.falcon_bwd(VARIANTS[variant], DTYPES[q.dtype], PAIRINGS[pairing], PHIS[phi],
-                        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(lam), float(eps), B, H, L, dk, dv,
+                        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(lam), float(eps), int(window), B, H, L, dk, dv,
                         _ptr(dout), _ptr(dstate) if dstate is not None else None,
                         _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dbeta"]), _ptr(g["dlambda"]),
                         _stream(stream))

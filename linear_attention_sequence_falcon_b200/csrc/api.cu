@@ -165,15 +165,16 @@ extern "C" int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_d
 
 extern "C" int falcon_bwd(falcon_variant variant, falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
                           const void *q, const void *k, const void *v, const void *beta, const float *lambda,
-                          float eps, int B, int H, int L, int d_k, int d_v, const void *dout, const float *dstate,
-                          float *dq, float *dk, float *dv, float *dbeta, float *dlambda, cudaStream_t stream) {
-    int rc = validate_common(variant, dtype, 1);
+                          float eps, int window, int B, int H, int L, int d_k, int d_v, const void *dout,
+                          const float *dstate, float *dq, float *dk, float *dv, float *dbeta, float *dlambda,
+                          cudaStream_t stream) {
+    int rc = validate_common(variant, dtype, window);
     if (rc) return rc;
     if (pairing != FALCON_PAIR_PREFIX && pairing != FALCON_PAIR_SAME_STEP) return FALCON_ERR_ENUM;
     if (phi != FALCON_PHI_L2 && phi != FALCON_PHI_IDENTITY) return FALCON_ERR_ENUM;
     if (B < 0 || H < 0 || L < 0 || !dim_ok(d_k) || !dim_ok(d_v)) return FALCON_ERR_SHAPE;
-    if (variant == FALCON_F3 || variant == FALCON_F3A) return FALCON_ERR_UNSUPPORTED;
     if (d_k != d_v || d_k < 32) return FALCON_ERR_UNSUPPORTED;
+    const bool has_window = variant == FALCON_F3 || variant == FALCON_F3A;
     if ((size_t)B * H == 0) return FALCON_OK;
     if (L == 0) {
         if (!dlambda) return FALCON_OK;
@@ -182,7 +183,7 @@ extern "C" int falcon_bwd(falcon_variant variant, falcon_dtype dtype, falcon_pai
     }
     if (!q || !k || !v || !beta || !lambda || !dout || !dq || !dk || !dv || !dbeta) return FALCON_ERR_NULL;
     BwdParams p{};
-    p.variant = variant; p.pairing = pairing; p.phi = phi;
+    p.variant = variant; p.pairing = pairing; p.phi = phi; p.window = has_window ? window : 1;
     p.B = B; p.H = H; p.L = L; p.dk = d_k; p.dv = d_v; p.eps = eps;
     p.q = q; p.k = k; p.v = v; p.beta = beta; p.dout = dout; p.lambda = lambda; p.dstate = dstate;
     p.dq = dq; p.dk_out = dk; p.dv_out = dv; p.dbeta = dbeta; p.dlambda = dlambda;

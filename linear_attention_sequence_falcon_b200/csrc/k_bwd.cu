@@ -1,29 +1,37 @@
-// k_bwd.cu -- backward pass of Falcon-1/2 and Falcon-1A/2A (one sample per
-// update) in the recurrent form, fp32 on the CUDA cores: the gradients of a
-// loss with respect to q, k, v, beta and lambda, given dL/do (and dL/dS_L).
-// The inner-product family is described first; the regression family's sweep
-// (bwd_sweep_reg_kernel) follows it.
+// k_bwd.cu -- backward pass of every Falcon variant in the recurrent form,
+// fp32 on the CUDA cores: the gradients of a loss with respect to q, k, v,
+// beta and lambda, given dL/do (and dL/dS_L), from S_0 = 0.
 //
 // The chunk form trains on the recurrent function (page "Fast Weight
-// Attention：用于持续学习的快速权重注意力", 核心方法 3); its derivative, with
-// S_t = alpha_t o S_{t-1} + (eta_t o y_t) x_t^T (per value channel j for
-// Falcon-2A; page "借鉴40年前的设想！…", 02 (2)) and o_t = S_t q_t:
-//   dq_t = S_t^T do_t,
-//   Gs_t = dL/dS_t = do_t q_t^T + alpha_{t+1} o Gs_{t+1}   (Gs_L = dL/dS_L),
-//   dy_t = eta_t o (Gs_t x_t),  deta_t = y_t o (Gs_t x_t),  dx_t = Gs_t^T (eta_t o y_t).
-// The decays need no stored past state: with G_t = sum_{r<=t} log alpha_r,
-//   dL/dG_t = do_t o o_t - (eta_t o y_t) o (Gs_t x_t)      (per channel),
+// Attention：用于持续学习的快速权重注意力", 核心方法 3).  Each update uses the
+// B_w most recent samples (B_w = 1 outside Falcon-3/3A; page "借鉴40年前的设
+// 想！…", 02 (2)), with one step per value channel j for Falcon-2/2A:
+//   S_t = alpha_t o S_{t-1} + eta_t o sum_m e_{t,m} x_{t-m}^T,   o_t = S_t q_t,
+//   e_{t,m} = y_{t-m}                    (inner-product family)
+//   e_{t,m} = y_{t-m} - S_{t-1} x_{t-m}  (regression family).
+// Its derivative, latest step first, with Gs = dL/dS_t:
+//   dq_t = S_t^T do_t,   Gs_t = do_t q_t^T + alpha_{t+1} o Gs_{t+1} (- sum de x^T, regression),
+//   de_{t,m} = eta_t o (Gs_t x_{t-m}),  dy_{t-m} += de_{t,m},
+//   dx_{t-m} += Gs_t^T (eta_t o e_{t,m})  (- S_{t-1}^T de_{t,m}, regression),
+//   deta_t = sum_m e_{t,m} o (Gs_t x_{t-m}).
+// The inner-product family needs no past state for the decays: with G_t =
+// sum_{r<=t} log alpha_r,
+//   dL/dG_t = do_t o o_t - sum_m (eta_t o y_{t-m}) o (Gs_t x_{t-m})  (per channel),
 // plus <dL/dS_L, S_L> (per row) at the last token, whose G the final state
-// carries as well,
-//   dL/dlog alpha_t = sum_{t'>=t} dL/dG_t',
-// then alpha = max(1 - eta lambda, 2^-20) (no gradient on the floor), eta =
-// beta / (eps + |x|^2) (0 at x = 0) and x = k / |k| (or k) take it to beta,
-// lambda and k.
+// carries as well, and dL/dlog alpha_t = sum_{t'>=t} dL/dG_t'.  The
+// regression family takes dalpha_t = <Gs_t, S_{t-1}> directly: its forward
+// sweep keeps S at the start of every tile of TT tokens, and the reverse sweep
+// recomputes a tile's states from that checkpoint before walking it back.
+// Then alpha = max(1 - eta lambda, 2^-20) (no gradient on the floor), eta =
+// beta / (eps + n), n the window's energy (0 at n = 0), and x = k / |k| (or
+// k) take it to beta, lambda and k.
 //
-// Four kernels: per-token samples and steps (a warp per token), the two
-// sweeps per head (a block per (b, h); S, then Gs, in shared memory; tokens
-// staged 32 at a time), the decay chain (a block-wide reverse scan per (b, h,
-// channel)) and a warp per token for the feature map.
+// Kernels: per-token samples and steps (a warp per token), the sweeps per
+// head (a block per (b, h); S, then Gs, in shared memory; tokens staged 32 at
+// a time with the B_w - 1 samples before them; each sample's dy and dx
+// gathered over the B_w steps that use it in a sliding register window), the
+// decay chain (a block per (b, h, channel)) and a warp per token for the
+// feature map.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -33,14 +41,20 @@ namespace falcon {
 
 namespace {
 
-constexpr int TT = 32;  // tokens staged per tile
+constexpr int TT = 32;             // tokens staged per tile
+constexpr int MAXW = 8;            // window bound (the forward's kMaxWindow)
+constexpr int TW = TT + MAXW - 1;  // sample rows staged per tile
 
 template <typename T>
 __device__ __forceinline__ float ld(const T *p, size_t i) {
     return to_f32(p[i]);
 }
 
-// per token: x_t (fp32), |x_t|^2, eta_t, alpha_t; a warp per (b, h, t)
+__host__ __device__ __forceinline__ int channels(const BwdParams &p) {
+    return (p.variant == F2A || p.variant == F2) ? p.dv : 1;
+}
+
+// per token: x_t (fp32), the window energy n_t, eta_t, alpha_t; a warp per (b, h, t)
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdParams p, float *xs, float *ns, float *etas, float *alphas) {
     const size_t gw = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -49,19 +63,27 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdParams p, float *xs, f
     if (gw >= rows) return;
     const int D = p.dk, t = (int)(gw % p.L);
     const size_t bh = gw / p.L;
-    const int kr = p.pairing == 0 ? t - 1 : t;
     const T *k = static_cast<const T *>(p.k) + bh * (size_t)p.L * D;
-    float ss = 0.f;
-    for (int c = lane; c < D; c += 32) {
-        const float v = kr >= 0 ? ld(k, (size_t)kr * D + c) : 0.f;
-        ss += v * v;
+    float n = 0.f;
+    for (int m = 0; m < p.window; ++m) {
+        const int sidx = t - m, kr = p.pairing == 0 ? sidx - 1 : sidx;
+        if (sidx < 0 || kr < 0) break;
+        float ss = 0.f;
+        for (int c = lane; c < D; c += 32) {
+            const float v = ld(k, (size_t)kr * D + c);
+            ss += v * v;
+        }
+        ss = group_sum<32>(ss);
+        const float inv = p.phi != 0 ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
+        n += ss * inv * inv;
+        if (m == 0)
+            for (int c = lane; c < D; c += 32) xs[gw * D + c] = ld(k, (size_t)kr * D + c) * inv;
     }
-    ss = group_sum<32>(ss);
-    const float inv = p.phi != 0 ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
-    for (int c = lane; c < D; c += 32) xs[gw * D + c] = kr >= 0 ? ld(k, (size_t)kr * D + c) * inv : 0.f;
-    const float n = ss * inv * inv;
+    const int kr0 = p.pairing == 0 ? t - 1 : t;
+    if (kr0 < 0)
+        for (int c = lane; c < D; c += 32) xs[gw * D + c] = 0.f;
     if (lane == 0) ns[gw] = n;
-    const int nch = (p.variant == F2A || p.variant == F2) ? p.dv : 1;
+    const int nch = channels(p);
     const float lam = p.lambda[bh % p.H];
     const T *beta = static_cast<const T *>(p.beta) + bh * (size_t)p.L * nch;
     for (int ch = lane; ch < nch; ch += 32) {
@@ -72,21 +94,52 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdParams p, float *xs, f
     }
 }
 
-// The two sweeps of one (b, h).  S (then Gs) in shared memory, D x (D+1).
+// Shared-memory tiles of one sweep: q, do, eta, alpha of TT tokens (eta and
+// alpha per channel; scalars repeated), and x, y of the TW samples from
+// t0 - (MAXW - 1): token i's window slot m is sample row i + MAXW - 1 - m.
+template <typename T, int D>
+struct Tiles {
+    float *tq, *tdo, *te, *ta, *tx, *ty;
+    __device__ Tiles(float *base) {
+        tq = base; tdo = tq + TT * D; te = tdo + TT * D; ta = te + TT * D; tx = ta + TT * D; ty = tx + TW * D;
+    }
+    static constexpr size_t floats = 4 * TT * D + 2 * TW * D;
+    __device__ void stage(const BwdParams &p, const T *q, const T *dout, const T *v, const float *x, const float *et,
+                          const float *al, int t0, int n, int nch) {
+        const int L = p.L;
+        for (int e = threadIdx.x; e < TT * D; e += blockDim.x) {
+            const int i = e / D, c = e % D, t = t0 + i;
+            const bool in = i < n;
+            tq[e] = in ? ld(q, (size_t)t * D + c) : 0.f;
+            tdo[e] = in ? ld(dout, (size_t)t * D + c) : 0.f;
+            te[e] = in ? et[(size_t)t * nch + (nch > 1 ? c : 0)] : 0.f;
+            ta[e] = in ? al[(size_t)t * nch + (nch > 1 ? c : 0)] : 1.f;
+        }
+        for (int e = threadIdx.x; e < TW * D; e += blockDim.x) {
+            const int r = e / D, c = e % D, sidx = t0 - (MAXW - 1) + r;
+            const bool in = r < n + MAXW - 1 && sidx >= 0 && sidx < L;
+            tx[e] = in ? x[(size_t)sidx * D + c] : 0.f;
+            ty[e] = in ? ld(v, (size_t)sidx * D + c) : 0.f;
+        }
+    }
+    __device__ float x(int i, int m, int c) const { return tx[(i + MAXW - 1 - m) * D + c]; }
+    __device__ float y(int i, int m, int j) const { return ty[(i + MAXW - 1 - m) * D + j]; }
+};
+
+// The sweeps of one (b, h) for the inner-product family (Falcon-1A/2A/3A).
 template <typename T, int D>
 __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const float *xs, const float *etas,
                                                           const float *alphas, float *dga, float *dgb, float *deta,
                                                           float *dx) {
     constexpr int NT = 256, LD = D + 1, RPT = NT / D, SEG = D / RPT;
     extern __shared__ float sm[];
-    float *S = sm;                                  // [D][LD]
-    float *tq = S + D * LD, *tdo = tq + TT * D;     // [TT][D] staged q, do
-    float *ty = tdo + TT * D, *tx = ty + TT * D;    // staged y, x
-    float *te = tx + TT * D, *ta = te + TT * D;     // staged eta, alpha (per channel; scalars repeat)
-    float *ta_next = ta + TT * D;                   // alpha of the token after the tile ([D])
-    const int tid = threadIdx.x, L = p.L;
+    float *S = sm;                          // [D][LD]: S, then Gs
+    Tiles<T, D> tl(S + D * LD);
+    float *ta_next = tl.ty + TW * D;        // [D] alpha of the token after the tile
+    float *vsum = ta_next + D;              // [D] per-row terms summed for the scalar variants
+    const int tid = threadIdx.x, L = p.L, w = p.window;
     const size_t bh = blockIdx.x;
-    const int nch = (p.variant == F2A || p.variant == F2) ? D : 1;
+    const int nch = channels(p);
     const T *q = static_cast<const T *>(p.q) + bh * (size_t)L * D;
     const T *v = static_cast<const T *>(p.v) + bh * (size_t)L * D;
     const T *dout = static_cast<const T *>(p.dout) + bh * (size_t)L * D;
@@ -95,50 +148,38 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
     float *dq = p.dq + bh * (size_t)L * D, *dv = p.dv_out + bh * (size_t)L * D;
     float *ga = dga + bh * (size_t)L * nch, *gb = dgb + bh * (size_t)L * nch, *de = deta + bh * (size_t)L * nch;
     float *dxo = dx + bh * (size_t)L * D;
-
-    auto stage = [&](int t0, int n) {
-        for (int e = tid; e < TT * D; e += NT) {
-            const int i = e / D, c = e % D, t = t0 + i;
-            const bool in = i < n;
-            tq[e] = in ? ld(q, (size_t)t * D + c) : 0.f;
-            tdo[e] = in ? ld(dout, (size_t)t * D + c) : 0.f;
-            ty[e] = in ? ld(v, (size_t)t * D + c) : 0.f;
-            tx[e] = in ? x[(size_t)t * D + c] : 0.f;
-            te[e] = in ? et[(size_t)t * nch + (nch > 1 ? c : 0)] : 0.f;
-            ta[e] = in ? al[(size_t)t * nch + (nch > 1 ? c : 0)] : 1.f;
-        }
-    };
-    // row / column of this thread in the reductions
     const int rj = tid / RPT, rp = tid % RPT;
 
-    // ---- forward sweep: S_t, then dq_t = S_t^T do_t and do_t o o_t
+    // ---- forward sweep: S_t, dq_t = S_t^T do_t and do_t o o_t (+ <dS_L, S_L> at the end)
     for (int e = tid; e < D * LD; e += NT) S[e] = 0.f;
     for (int t0 = 0; t0 < L; t0 += TT) {
         const int n = min(TT, L - t0);
         __syncthreads();
-        stage(t0, n);
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
         __syncthreads();
         for (int i = 0; i < n; ++i) {
             const int t = t0 + i;
             for (int e = tid; e < D * D; e += NT) {
                 const int j = e / D, c = e % D;
-                S[j * LD + c] = ta[i * D + j] * S[j * LD + c] + te[i * D + j] * ty[i * D + j] * tx[i * D + c];
+                float u = 0.f;
+#pragma unroll
+                for (int m = 0; m < MAXW; ++m)
+                    if (m < w) u = fmaf(tl.y(i, m, j), tl.x(i, m, c), u);
+                S[j * LD + c] = tl.ta[i * D + j] * S[j * LD + c] + tl.te[i * D + j] * u;
             }
             __syncthreads();
             float o = 0.f, g = 0.f, f = 0.f;  // row rj: (S q)_j; column rj: (S^T do)_c
 #pragma unroll 8
             for (int s = 0; s < SEG; ++s) {
                 const int c = rp * SEG + s;
-                o = fmaf(S[rj * LD + c], tq[i * D + c], o);
-                g = fmaf(S[c * LD + rj], tdo[i * D + c], g);
+                o = fmaf(S[rj * LD + c], tl.tq[i * D + c], o);
+                g = fmaf(S[c * LD + rj], tl.tdo[i * D + c], g);
             }
-            // the final state is e^{G_{L-1}} (...) too: dL/dG_{L-1} also takes <dS_L, S_L> (row rj)
-            if (t == L - 1 && p.dstate) {
+            if (t == L - 1 && p.dstate)
                 for (int s = 0; s < SEG; ++s) {
                     const int c = rp * SEG + s;
                     f = fmaf(S[rj * LD + c], p.dstate[(bh * D + rj) * D + c], f);
                 }
-            }
 #pragma unroll
             for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
                 o += __shfl_xor_sync(0xffffffffu, o, o2);
@@ -147,104 +188,125 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
             }
             if (rp == 0) {
                 dq[(size_t)t * D + rj] = g;
-                const float a = tdo[i * D + rj] * o + f;
+                const float a = tl.tdo[i * D + rj] * o + f;
                 if (nch > 1) ga[(size_t)t * D + rj] = a;
-                else tx[i * D + rj] = a;  // x of this token is no longer needed: reuse it
+                else vsum[rj] = a;
             }
             __syncthreads();
             if (nch == 1 && tid < 32) {
                 float a = 0.f;
-                for (int j = tid; j < D; j += 32) a += tx[i * D + j];
+                for (int j = tid; j < D; j += 32) a += vsum[j];
                 a = group_sum<32>(a);
                 if (tid == 0) ga[t] = a;
             }
         }
     }
-    // ---- reverse sweep: Gs_t, dy_t, deta_t, dx_t and (eta y) o (Gs x)
+    // ---- reverse sweep: Gs_t; dy and dx of the window's samples; deta_t; the key-side dG
     __syncthreads();
     for (int e = tid; e < D * D; e += NT) {
         const int j = e / D, c = e % D;
         S[j * LD + c] = p.dstate ? p.dstate[(bh * D + j) * D + c] : 0.f;
     }
     for (int e = tid; e < D; e += NT) ta_next[e] = 1.f;  // no step after the last token
+    float acc_dy[MAXW], acc_dx[MAXW];  // samples t - m: row rj of dy, column rj of dx
+#pragma unroll
+    for (int m = 0; m < MAXW; ++m) acc_dy[m] = acc_dx[m] = 0.f;
     const int ntile = (L + TT - 1) / TT;
     for (int tb = ntile - 1; tb >= 0; --tb) {
         const int t0 = tb * TT, n = min(TT, L - t0);
         __syncthreads();
-        stage(t0, n);
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
         __syncthreads();
         for (int i = n - 1; i >= 0; --i) {
             const int t = t0 + i;
-            const float *anext = i + 1 < n ? ta + (i + 1) * D : ta_next;
+            const float *anext = i + 1 < n ? tl.ta + (i + 1) * D : ta_next;
             for (int e = tid; e < D * D; e += NT) {
                 const int j = e / D, c = e % D;
-                S[j * LD + c] = anext[j] * S[j * LD + c] + tdo[i * D + j] * tq[i * D + c];
+                S[j * LD + c] = anext[j] * S[j * LD + c] + tl.tdo[i * D + j] * tl.tq[i * D + c];
             }
             __syncthreads();
-            float gx = 0.f, dxc = 0.f;  // row rj: (Gs x)_j; column rj: (Gs^T (eta o y))_c
-#pragma unroll 8
+            float gx[MAXW], dxm[MAXW];  // row rj: (Gs x_{t-m})_j; column rj: (Gs^T (eta o y_{t-m}))_c
+#pragma unroll
+            for (int m = 0; m < MAXW; ++m) gx[m] = dxm[m] = 0.f;
             for (int s = 0; s < SEG; ++s) {
                 const int c = rp * SEG + s;
-                gx = fmaf(S[rj * LD + c], tx[i * D + c], gx);
-                dxc = fmaf(S[c * LD + rj], te[i * D + c] * ty[i * D + c], dxc);
-            }
+                const float gr = S[rj * LD + c], gc = S[c * LD + rj], ec = tl.te[i * D + c];
 #pragma unroll
-            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
-                gx += __shfl_xor_sync(0xffffffffu, gx, o2);
-                dxc += __shfl_xor_sync(0xffffffffu, dxc, o2);
+                for (int m = 0; m < MAXW; ++m)
+                    if (m < w) {
+                        gx[m] = fmaf(gr, tl.x(i, m, c), gx[m]);
+                        dxm[m] = fmaf(gc, ec * tl.y(i, m, c), dxm[m]);
+                    }
             }
+            float sy = 0.f;  // sum_m y_{t-m,j} (Gs x_{t-m})_j
+            const float eta = tl.te[i * D + rj];
+#pragma unroll
+            for (int m = 0; m < MAXW; ++m)
+                if (m < w) {
+#pragma unroll
+                    for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
+                        gx[m] += __shfl_xor_sync(0xffffffffu, gx[m], o2);
+                        dxm[m] += __shfl_xor_sync(0xffffffffu, dxm[m], o2);
+                    }
+                    acc_dy[m] += eta * gx[m];
+                    acc_dx[m] += dxm[m];
+                    sy = fmaf(tl.y(i, m, rj), gx[m], sy);
+                }
             if (rp == 0) {
-                const float eta = te[i * D + rj], y = ty[i * D + rj];
-                dv[(size_t)t * D + rj] = eta * gx;
-                dxo[(size_t)t * D + rj] = dxc;
+                dv[(size_t)t * D + rj] = acc_dy[0];  // sample t: every step that uses it is done
+                dxo[(size_t)t * D + rj] = acc_dx[0];
                 if (nch > 1) {
-                    de[(size_t)t * D + rj] = y * gx;
-                    gb[(size_t)t * D + rj] = eta * y * gx;
+                    de[(size_t)t * D + rj] = sy;
+                    gb[(size_t)t * D + rj] = eta * sy;
                 } else {
-                    tdo[i * D + rj] = y * gx;  // do of this token is no longer needed: reuse it
+                    vsum[rj] = sy;
                 }
             }
+#pragma unroll
+            for (int m = 0; m < MAXW - 1; ++m) {
+                acc_dy[m] = acc_dy[m + 1];
+                acc_dx[m] = acc_dx[m + 1];
+            }
+            acc_dy[MAXW - 1] = acc_dx[MAXW - 1] = 0.f;
             __syncthreads();
             if (nch == 1 && tid < 32) {
                 float a = 0.f;
-                for (int j = tid; j < D; j += 32) a += tdo[i * D + j];
+                for (int j = tid; j < D; j += 32) a += vsum[j];
                 a = group_sum<32>(a);
                 if (tid == 0) {
                     de[t] = a;
-                    gb[t] = te[i * D] * a;
+                    gb[t] = tl.te[i * D] * a;
                 }
             }
         }
         __syncthreads();
-        for (int e = tid; e < D; e += NT) ta_next[e] = ta[e];  // alpha of this tile's first token
+        for (int e = tid; e < D; e += NT) ta_next[e] = tl.ta[e];  // alpha of this tile's first token
     }
 }
 
-// The regression family (Falcon-1 / Falcon-2): S_t = alpha_t S_{t-1} +
-// eta_t (y_t - S_{t-1} x_t) x_t^T.  Its derivative needs S_{t-1} at every
-// step of the reverse sweep: the forward sweep keeps S at the start of every
-// tile of TT tokens (ck), and the reverse sweep recomputes a tile's states
-// from its checkpoint (ts, global scratch of the block) before walking it
-// backwards.  Per step, with Gs = dL/dS_t (do_t q_t^T added):
-//   e = y - S_{t-1} x,  de = eta (Gs x),  dalpha = <Gs, S_{t-1}> (per row),
-//   deta = e . (Gs x) (per row),  dy = de,
-//   dx = Gs^T (eta o e) - S_{t-1}^T de,  Gs <- alpha o Gs - de x^T.
-// dalpha is written straight into dga (the scan is not needed here).
+// The sweeps of one (b, h) for the regression family (Falcon-1/2/3).  The
+// forward sweep keeps S before every tile (ck); the reverse sweep swaps Gs
+// with the tile's checkpoint, recomputes the tile's states S_{t-1} into the
+// block's scratch (ts), puts Gs back and walks the tile:
+//   e_m = y_{t-m} - S_{t-1} x_{t-m},  de_m = eta (Gs x_{t-m}),
+//   dalpha = <Gs, S_{t-1}>,  deta = sum_m e_m (Gs x_{t-m})  (per row),
+//   dy_{t-m} += de_m,  dx_{t-m} += Gs^T (eta e_m) - S_{t-1}^T de_m,
+//   Gs <- alpha o Gs - sum_m de_m x_{t-m}^T.
+// dalpha goes straight into dga (no scan).
 template <typename T, int D>
 __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, const float *xs, const float *etas,
                                                               const float *alphas, float *dga, float *deta, float *dx,
                                                               float *ck, float *ts) {
     constexpr int NT = 256, LD = D + 1, RPT = NT / D, SEG = D / RPT;
     extern __shared__ float sm[];
-    float *S = sm;                                  // [D][LD]: S, then Gs
-    float *tq = S + D * LD, *tdo = tq + TT * D;
-    float *ty = tdo + TT * D, *tx = ty + TT * D;
-    float *te = tx + TT * D, *ta = te + TT * D;
-    float *ve = ta + TT * D, *vde = ve + D;         // [D] e_j and de_j of the current step
-    float *vsum = vde + D;                          // [3 * D] row sums for the Falcon-1 totals
-    const int tid = threadIdx.x, L = p.L;
+    float *S = sm;                          // [D][LD]: S, then Gs
+    Tiles<T, D> tl(S + D * LD);
+    float *ve = tl.ty + TW * D;             // [MAXW][D] e (forward) or eta e (reverse) of the window
+    float *vde = ve + MAXW * D;             // [MAXW][D] de of the window
+    float *vsum = vde + MAXW * D;           // [2][D] per-row terms summed for the scalar variants
+    const int tid = threadIdx.x, L = p.L, w = p.window;
     const size_t bh = blockIdx.x;
-    const int nch = p.variant == F2 ? D : 1;
+    const int nch = channels(p);
     const T *q = static_cast<const T *>(p.q) + bh * (size_t)L * D;
     const T *v = static_cast<const T *>(p.v) + bh * (size_t)L * D;
     const T *dout = static_cast<const T *>(p.dout) + bh * (size_t)L * D;
@@ -256,35 +318,35 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
     const int ntile = (L + TT - 1) / TT;
     float *cks = ck + bh * (size_t)ntile * D * D;   // S before each tile
     float *tss = ts + bh * (size_t)TT * D * D;      // S before each token of the tile being walked
-
-    auto stage = [&](int t0, int n) {
-        for (int e = tid; e < TT * D; e += NT) {
-            const int i = e / D, c = e % D, t = t0 + i;
-            const bool in = i < n;
-            tq[e] = in ? ld(q, (size_t)t * D + c) : 0.f;
-            tdo[e] = in ? ld(dout, (size_t)t * D + c) : 0.f;
-            ty[e] = in ? ld(v, (size_t)t * D + c) : 0.f;
-            tx[e] = in ? x[(size_t)t * D + c] : 0.f;
-            te[e] = in ? et[(size_t)t * nch + (nch > 1 ? c : 0)] : 0.f;
-            ta[e] = in ? al[(size_t)t * nch + (nch > 1 ? c : 0)] : 1.f;
-        }
-    };
     const int rj = tid / RPT, rp = tid % RPT;
-    // one regression step on the state in S with token i of the staged tile
+
+    // one step of the recurrence on S with token i of the staged tile
     auto step = [&](int i) {
-        float r = 0.f;  // (S x)_rj
-#pragma unroll 8
+        float r[MAXW];
+#pragma unroll
+        for (int m = 0; m < MAXW; ++m) r[m] = 0.f;
         for (int s = 0; s < SEG; ++s) {
             const int c = rp * SEG + s;
-            r = fmaf(S[rj * LD + c], tx[i * D + c], r);
+            const float sv = S[rj * LD + c];
+#pragma unroll
+            for (int m = 0; m < MAXW; ++m)
+                if (m < w) r[m] = fmaf(sv, tl.x(i, m, c), r[m]);
         }
 #pragma unroll
-        for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o2);
-        if (rp == 0) ve[rj] = ty[i * D + rj] - r;
+        for (int m = 0; m < MAXW; ++m)
+            if (m < w) {
+#pragma unroll
+                for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) r[m] += __shfl_xor_sync(0xffffffffu, r[m], o2);
+                if (rp == 0) ve[m * D + rj] = tl.y(i, m, rj) - r[m];
+            }
         __syncthreads();
         for (int e = tid; e < D * D; e += NT) {
             const int j = e / D, c = e % D;
-            S[j * LD + c] = ta[i * D + j] * S[j * LD + c] + te[i * D + j] * ve[j] * tx[i * D + c];
+            float u = 0.f;
+#pragma unroll
+            for (int m = 0; m < MAXW; ++m)
+                if (m < w) u = fmaf(ve[m * D + j], tl.x(i, m, c), u);
+            S[j * LD + c] = tl.ta[i * D + j] * S[j * LD + c] + tl.te[i * D + j] * u;
         }
         __syncthreads();
     };
@@ -294,7 +356,7 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
     for (int tb = 0; tb < ntile; ++tb) {
         const int t0 = tb * TT, n = min(TT, L - t0);
         __syncthreads();
-        stage(t0, n);
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
         for (int e = tid; e < D * D; e += NT) cks[(size_t)tb * D * D + e] = S[(e / D) * LD + e % D];
         __syncthreads();
         for (int i = 0; i < n; ++i) {
@@ -303,7 +365,7 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
 #pragma unroll 8
             for (int s = 0; s < SEG; ++s) {
                 const int c = rp * SEG + s;
-                g = fmaf(S[c * LD + rj], tdo[i * D + c], g);
+                g = fmaf(S[c * LD + rj], tl.tdo[i * D + c], g);
             }
 #pragma unroll
             for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) g += __shfl_xor_sync(0xffffffffu, g, o2);
@@ -316,11 +378,14 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
         const int j = e / D, c = e % D;
         S[j * LD + c] = p.dstate ? p.dstate[(bh * D + j) * D + c] : 0.f;  // dL/dS_L
     }
+    float acc_dy[MAXW], acc_dx[MAXW];  // samples t - m: row rj of dy, column rj of dx
+#pragma unroll
+    for (int m = 0; m < MAXW; ++m) acc_dy[m] = acc_dx[m] = 0.f;
     for (int tb = ntile - 1; tb >= 0; --tb) {
         const int t0 = tb * TT, n = min(TT, L - t0);
         float *ckt = cks + (size_t)tb * D * D;
         __syncthreads();
-        stage(t0, n);
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
         // swap Gs and the tile's checkpoint (each element by one thread)
         for (int e = tid; e < D * D; e += NT) {
             const int j = e / D, c = e % D;
@@ -341,48 +406,81 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
             const float *Sp = tss + (size_t)i * D * D;
             for (int e = tid; e < D * D; e += NT) {
                 const int j = e / D, c = e % D;
-                S[j * LD + c] += tdo[i * D + j] * tq[i * D + c];
+                S[j * LD + c] += tl.tdo[i * D + j] * tl.tq[i * D + c];
             }
             __syncthreads();
-            float sx = 0.f, gx = 0.f, gs = 0.f;  // row rj: (S_{t-1} x), (Gs x), <Gs, S_{t-1}>
-#pragma unroll 8
-            for (int s2 = 0; s2 < SEG; ++s2) {
-                const int c = rp * SEG + s2;
+            float sx[MAXW], gx[MAXW], gs = 0.f;  // row rj: (S_{t-1} x_{t-m}), (Gs x_{t-m}), <Gs, S_{t-1}>
+#pragma unroll
+            for (int m = 0; m < MAXW; ++m) sx[m] = gx[m] = 0.f;
+            for (int s = 0; s < SEG; ++s) {
+                const int c = rp * SEG + s;
                 const float sp = Sp[(size_t)rj * D + c], g = S[rj * LD + c];
-                sx = fmaf(sp, tx[i * D + c], sx);
-                gx = fmaf(g, tx[i * D + c], gx);
                 gs = fmaf(g, sp, gs);
+#pragma unroll
+                for (int m = 0; m < MAXW; ++m)
+                    if (m < w) {
+                        const float xv = tl.x(i, m, c);
+                        sx[m] = fmaf(sp, xv, sx[m]);
+                        gx[m] = fmaf(g, xv, gx[m]);
+                    }
             }
 #pragma unroll
-            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
-                sx += __shfl_xor_sync(0xffffffffu, sx, o2);
-                gx += __shfl_xor_sync(0xffffffffu, gx, o2);
-                gs += __shfl_xor_sync(0xffffffffu, gs, o2);
-            }
+            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o2);
+            const float eta = tl.te[i * D + rj];
+            float dterm = 0.f;
+#pragma unroll
+            for (int m = 0; m < MAXW; ++m)
+                if (m < w) {
+#pragma unroll
+                    for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
+                        sx[m] += __shfl_xor_sync(0xffffffffu, sx[m], o2);
+                        gx[m] += __shfl_xor_sync(0xffffffffu, gx[m], o2);
+                    }
+                    const float e = tl.y(i, m, rj) - sx[m], d = eta * gx[m];
+                    acc_dy[m] += d;
+                    dterm = fmaf(e, gx[m], dterm);
+                    if (rp == 0) {
+                        ve[m * D + rj] = eta * e;
+                        vde[m * D + rj] = d;
+                    }
+                }
             if (rp == 0) {
-                const float eta = te[i * D + rj], e = ty[i * D + rj] - sx, d = eta * gx;
-                ve[rj] = eta * e;
-                vde[rj] = d;
-                dv[(size_t)t * D + rj] = d;
                 if (nch > 1) {
                     ga[(size_t)t * D + rj] = gs;
-                    de[(size_t)t * D + rj] = e * gx;
+                    de[(size_t)t * D + rj] = dterm;
                 } else {
                     vsum[rj] = gs;
-                    vsum[D + rj] = e * gx;
+                    vsum[D + rj] = dterm;
                 }
             }
             __syncthreads();
-            float dxc = 0.f;  // column rj: sum_j (eta e)_j Gs[j][c] - de_j S_{t-1}[j][c]
-#pragma unroll 8
-            for (int s2 = 0; s2 < SEG; ++s2) {
-                const int j = rp * SEG + s2;
-                dxc = fmaf(ve[j], S[j * LD + rj], dxc);
-                dxc = fmaf(-vde[j], Sp[(size_t)j * D + rj], dxc);
+            float dxm[MAXW];  // column rj: sum_j (eta e_m)_j Gs[j][c] - de_{m,j} S_{t-1}[j][c]
+#pragma unroll
+            for (int m = 0; m < MAXW; ++m) dxm[m] = 0.f;
+            for (int s = 0; s < SEG; ++s) {
+                const int j = rp * SEG + s;
+                const float gc = S[j * LD + rj], sc = Sp[(size_t)j * D + rj];
+#pragma unroll
+                for (int m = 0; m < MAXW; ++m)
+                    if (m < w) dxm[m] = fmaf(ve[m * D + j], gc, fmaf(-vde[m * D + j], sc, dxm[m]));
             }
 #pragma unroll
-            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) dxc += __shfl_xor_sync(0xffffffffu, dxc, o2);
-            if (rp == 0) dxo[(size_t)t * D + rj] = dxc;
+            for (int m = 0; m < MAXW; ++m)
+                if (m < w) {
+#pragma unroll
+                    for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) dxm[m] += __shfl_xor_sync(0xffffffffu, dxm[m], o2);
+                    acc_dx[m] += dxm[m];
+                }
+            if (rp == 0) {
+                dv[(size_t)t * D + rj] = acc_dy[0];  // sample t: every step that uses it is done
+                dxo[(size_t)t * D + rj] = acc_dx[0];
+            }
+#pragma unroll
+            for (int m = 0; m < MAXW - 1; ++m) {
+                acc_dy[m] = acc_dy[m + 1];
+                acc_dx[m] = acc_dx[m + 1];
+            }
+            acc_dy[MAXW - 1] = acc_dx[MAXW - 1] = 0.f;
             if (nch == 1 && tid < 32) {
                 float a = 0.f, b = 0.f;
                 for (int j = tid; j < D; j += 32) {
@@ -397,10 +495,14 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
                 }
             }
             __syncthreads();
-            // Gs <- alpha o Gs - de x^T (dL/dS_{t-1})
+            // Gs <- alpha o Gs - sum_m de_m x_{t-m}^T  (dL/dS_{t-1})
             for (int e = tid; e < D * D; e += NT) {
                 const int j = e / D, c = e % D;
-                S[j * LD + c] = ta[i * D + j] * S[j * LD + c] - vde[j] * tx[i * D + c];
+                float u = 0.f;
+#pragma unroll
+                for (int m = 0; m < MAXW; ++m)
+                    if (m < w) u = fmaf(vde[m * D + j], tl.x(i, m, c), u);
+                S[j * LD + c] = tl.ta[i * D + j] * S[j * LD + c] - u;
             }
             __syncthreads();
         }
@@ -422,7 +524,7 @@ __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float
     const int nch = (p.variant == F2A || p.variant == F2) ? p.dv : 1;
     const size_t bh = blockIdx.x / nch;
     const int ch = (int)(blockIdx.x % nch), L = p.L, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool reg = p.variant == F1 || p.variant == F2;
+    const bool reg = p.variant == F1 || p.variant == F2 || p.variant == F3;
     const float lam = p.lambda[bh % p.H];
     const T *beta = static_cast<const T *>(p.beta) + bh * (size_t)L * nch;
     float carry = 0.f, dlam = 0.f;
@@ -487,7 +589,8 @@ __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float
     }
 }
 
-// a warp per (b, h, t): dx_t += 2 dn_t x_t, then dk of the key x_t came from
+// a warp per (b, h, t): sample t's normaliser share (the windows of tokens
+// t .. t+B_w-1 hold it) gives dx_t += 2 dn x_t; then dk of the key x_t came from
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_key_kernel(BwdParams p, const float *xs, const float *dnc, const float *dx) {
     const size_t gw = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -495,9 +598,10 @@ __global__ void __launch_bounds__(256) bwd_key_kernel(BwdParams p, const float *
     if (gw >= (size_t)p.B * p.H * p.L) return;
     const int D = p.dk, L = p.L, t = (int)(gw % L);
     const size_t bh = gw / L;
-    const int nch = (p.variant == F2A || p.variant == F2) ? p.dv : 1;
+    const int nch = channels(p);
     float dn = 0.f;
-    for (int ch = lane; ch < nch; ch += 32) dn += dnc[gw * nch + ch];
+    for (int m = 0; m < p.window && t + m < L; ++m)
+        for (int ch = lane; ch < nch; ch += 32) dn += dnc[(gw + m) * nch + ch];
     dn = group_sum<32>(dn);
     // the key row this token's sample was made from; under the prefix pair the
     // last key feeds no sample and the first sample is zero
@@ -528,16 +632,19 @@ __global__ void __launch_bounds__(256) bwd_key_kernel(BwdParams p, const float *
     }
 }
 
+__host__ __device__ bool regression(int v) { return v == F1 || v == F2 || v == F3; }
+
 template <typename T, int D>
 int launch_sweep(const BwdParams &p, const float *xs, const float *etas, const float *alphas, float *dga, float *dgb,
                  float *deta, float *dx, float *ck, float *ts, cudaStream_t s) {
-    if (p.variant == F1 || p.variant == F2) {
-        const size_t bytes = ((size_t)D * (D + 1) + 6 * TT * D + 5 * D) * sizeof(float);
+    constexpr size_t base = (size_t)D * (D + 1) + Tiles<T, D>::floats;
+    if (regression(p.variant)) {
+        const size_t bytes = (base + 2 * MAXW * D + 2 * D) * sizeof(float);
         cudaFuncSetAttribute(bwd_sweep_reg_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         bwd_sweep_reg_kernel<T, D><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
         return 0;
     }
-    const size_t bytes = ((size_t)D * (D + 1) + 6 * TT * D + D) * sizeof(float);
+    const size_t bytes = (base + 2 * D) * sizeof(float);
     cudaFuncSetAttribute(bwd_sweep_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     bwd_sweep_kernel<T, D><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
     return 0;
@@ -547,12 +654,12 @@ int launch_sweep(const BwdParams &p, const float *xs, const float *etas, const f
 
 template <typename T>
 int launch_bwd(const BwdParams &p, cudaStream_t s) {
-    const int D = p.dk, nch = (p.variant == F2A || p.variant == F2) ? D : 1;
-    const bool reg = p.variant == F1 || p.variant == F2;
+    const int D = p.dk, nch = channels(p);
+    const bool reg = regression(p.variant);
     const size_t rows = (size_t)p.B * p.H * p.L;
     if (rows == 0) return 0;
-    // scratch: x, |x|^2, eta, alpha, the two decay-gradient halves, deta, dx;
-    // the regression family adds the tile checkpoints and one tile of states per head
+    // scratch: x, |x|^2 (window energy), eta, alpha, the two decay-gradient halves,
+    // deta, dx; the regression family adds the tile checkpoints and one tile of states per head
     const size_t BH = (size_t)p.B * p.H, ntile = (p.L + TT - 1) / TT;
     const size_t nreg = reg ? BH * (ntile + TT) * D * D : 0;
     const size_t nf = rows * D * 2 + rows + rows * nch * 5 + nreg;

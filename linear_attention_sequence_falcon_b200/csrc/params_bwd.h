@@ -5,7 +5,7 @@
 namespace falcon {
 
 struct BwdParams {
-    int variant, pairing, phi;
+    int variant, pairing, phi, window;
     int B, H, L, dk, dv;
     float eps;
     const void *q, *k, *v, *beta, *dout;

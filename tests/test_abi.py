@@ -68,9 +68,9 @@ def test_validation_codes(lib):
     assert lib.falcon_decode_carry_from_prefill(2, 1, P, P, 4, 1, 1, 4, 64, 64, P, None, None) == -1
 
 
-def _bwd(lib, variant=3, dtype=1, pairing=0, phi=0, B=1, H=1, L=8, dk=64, dv=64, ptr=1, dlam=True):
+def _bwd(lib, variant=3, dtype=1, pairing=0, phi=0, window=1, B=1, H=1, L=8, dk=64, dv=64, ptr=1, dlam=True):
     P = ctypes.c_void_p(ptr) if ptr else None
-    return lib.falcon_bwd(variant, dtype, pairing, phi, P, P, P, P, P, 1e-6, B, H, L, dk, dv, P, None,
+    return lib.falcon_bwd(variant, dtype, pairing, phi, P, P, P, P, P, 1e-6, window, B, H, L, dk, dv, P, None,
                           P, P, P, P, P if dlam else None, None)
 
 
@@ -81,8 +81,8 @@ def test_backward_validation_codes(lib):
     assert _bwd(lib, pairing=2) == -2
     assert _bwd(lib, phi=3) == -2
     assert _bwd(lib, dk=48) == -3
-    assert _bwd(lib, variant=2) == -9   # windows: not in the backward kernels
-    assert _bwd(lib, variant=5) == -9
+    assert _bwd(lib, variant=2, window=0) == -6
+    assert _bwd(lib, variant=5, window=9) == -6
     assert _bwd(lib, dk=64, dv=32) == -9
     assert _bwd(lib, dk=16, dv=16) == -9
     assert _bwd(lib, ptr=0) == -1

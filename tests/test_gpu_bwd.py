@@ -1,4 +1,4 @@
-"""GPU parity of falcon_bwd (the backward pass of Falcon-1/2 and Falcon-1A/2A)
+"""GPU parity of falcon_bwd (the backward pass of every variant)
 against the fp64 oracle's reverse mode of the recurrent definition
 (oracle.bwd, pinned by finite differences in test_oracle_bwd.py), on the same
 seeded inputs.
@@ -37,19 +37,21 @@ def rel(gpu, ref):
 
 
 def grads_case(F, variant, B, H, L, d, dtype, seed, pairing="prefix", phi="l2", with_dstate=True, lam=None,
-               key_scale=1.0, units=None):
+               key_scale=1.0, units=None, window=None):
+    if window is None:
+        window = 3 if variant in ("F3", "F3A") else 1
     d_ = gen.draw(variant, B, H, L, d, d, seed=seed, dtype=dtype, lam=lam, key_scale=key_scale)
     rng = np.random.default_rng(seed + 1)
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     do = torch.from_numpy(rng.standard_normal((B, H, L, d)).astype(np.float32)).to(tdt)
     ds = torch.from_numpy(rng.standard_normal((B, H, d, d)).astype(np.float32)) if with_dstate else None
     g = F.bwd(variant, *(d_[n].cuda() for n in ("q", "k", "v", "beta", "lam")), d_["eps"], do.cuda(),
-              None if ds is None else ds.cuda(), pairing=pairing, phi=phi)
+              None if ds is None else ds.cuda(), window=window, pairing=pairing, phi=phi)
     torch.cuda.synchronize()
     if units is None:
         args = [d_[n] for n in ("q_64", "k_64", "v_64", "beta_64")]
         ref = oracle.bwd(variant, *args, d_["lam_64"], d_["eps_64"], do.double().numpy(),
-                         None if ds is None else ds.double().numpy(), pairing=pairing, phi=phi)
+                         None if ds is None else ds.double().numpy(), window=window, pairing=pairing, phi=phi)
         got = {n: g[n].double().cpu().numpy() for n in NAMES}
         return got, ref
     # sampled (b, h) units of a large case: each through the oracle as a batch of one
@@ -59,7 +61,7 @@ def grads_case(F, variant, B, H, L, d, dtype, seed, pairing="prefix", phi="l2", 
         one = lambda a: np.ascontiguousarray(a[b:b + 1, h:h + 1])  # noqa: E731
         r = oracle.bwd(variant, *(one(d_[n]) for n in ("q_64", "k_64", "v_64", "beta_64")),
                        np.asarray(d_["lam_64"])[h:h + 1], d_["eps_64"], one(do.double().numpy()),
-                       None if ds is None else one(ds.double().numpy()), pairing=pairing, phi=phi)
+                       None if ds is None else one(ds.double().numpy()), window=window, pairing=pairing, phi=phi)
         for n in got:
             got[n].append(g[n][b, h].double().cpu().numpy())
             ref[n].append(r[n][0, 0])
@@ -73,7 +75,7 @@ def check(got, ref, tol=TOL):
         assert e <= tol, f"{n}: {e:.3e} (tol {tol})"
 
 
-@pytest.mark.parametrize("variant", ["F1", "F2", "F1A", "F2A"])
+@pytest.mark.parametrize("variant", ["F1", "F2", "F3", "F1A", "F2A", "F3A"])
 @pytest.mark.parametrize("d", [32, 64, 128])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("L", [1, 37, 100])
@@ -83,14 +85,14 @@ def test_backward_parity(F, variant, d, dtype, L):
     check(got, ref)
 
 
-@pytest.mark.parametrize("variant", ["F1", "F2", "F1A", "F2A"])
+@pytest.mark.parametrize("variant", ["F1", "F2", "F3", "F1A", "F2A", "F3A"])
 @pytest.mark.parametrize("pairing,phi", [("same_step", "l2"), ("prefix", "identity"), ("same_step", "identity")])
 def test_backward_pairing_and_feature_map(F, variant, pairing, phi):
     got, ref = grads_case(F, variant, 1, 2, 70, 64, "f32", seed=231, pairing=pairing, phi=phi, key_scale=0.3)
     check(got, ref)
 
 
-@pytest.mark.parametrize("variant", ["F1", "F2", "F1A", "F2A"])
+@pytest.mark.parametrize("variant", ["F1", "F2", "F3", "F1A", "F2A", "F3A"])
 def test_backward_without_state_gradient_and_with_clamped_decay(F, variant):
     """dstate = NULL, and lambda = 0.9 with tiny keys under the identity map:
     eta = beta/(eps+|x|^2) is large, alpha sits on its 2^-20 floor for most
@@ -118,9 +120,17 @@ def test_backward_workload2_sampled(F, variant):
     check(got, ref)
 
 
+@pytest.mark.parametrize("w", [2, 4, 8])
 @pytest.mark.parametrize("variant", ["F3", "F3A"])
-def test_backward_rejects_the_windowed_variants(F, variant):
-    d_ = gen.draw(variant, 1, 1, 8, 64, 64, seed=2, dtype="f32")
+def test_backward_windows(F, variant, w):
+    """Windows of 2, 4 and 8 samples (the staged tile carries the 7 samples
+    before it; each sample's gradient gathers the w steps that use it)."""
+    got, ref = grads_case(F, variant, 1, 2, 75, 64, "f32", seed=250 + w, window=w)
+    check(got, ref)
+
+
+def test_backward_rejects_an_unsupported_shape(F):
+    d_ = gen.draw("F1", 1, 1, 8, 64, 32, seed=2, dtype="f32")
     with pytest.raises(F.FalconError):
-        F.bwd(variant, *(d_[n].cuda() for n in ("q", "k", "v", "beta", "lam")), d_["eps"],
-              torch.zeros((1, 1, 8, 64), device="cuda"))
+        F.bwd("F1", *(d_[n].cuda() for n in ("q", "k", "v", "beta", "lam")), d_["eps"],
+              torch.zeros((1, 1, 8, 32), device="cuda"))
