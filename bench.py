@@ -541,12 +541,13 @@ def run_chunk_sweep(args):
 
 def run_backward(args):
     """--backward: falcon_bwd on workload 2 (Falcon-1 and Falcon-1A,
-    8x12x2048x64 bf16), workload 3 (Falcon-2, 4x16x4096x128) and workload 5's
-    prefill (Falcon-2A, 2x16x32768x128 bf16): CUDA events around one call after a
+    8x12x2048x64 bf16), workload 3 (Falcon-2, 4x16x4096x128), workload 4
+    (Falcon-3 and Falcon-3A, window 4) and workload 5's prefill (Falcon-2A,
+    2x16x32768x128 bf16): CUDA events around one call after a
     warm-up call, L2 flushed, median of --steps calls (3..10); an HBM
     roofline on the algorithmic bytes (q, k, v, beta, dout read; dq, dk, dv,
     dbeta written in fp32) and the fp64 oracle's reverse mode on whole (b,h)
-    units (workload 2 only: its state history at L = 32768, d = 128 would
+    units (workloads 2 and 4: its state history at L = 32768, d = 128 would
     take 4 GB per unit).  Not the contract line."""
     import numpy as np
     import torch
@@ -556,7 +557,7 @@ def run_backward(args):
     F.load()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     hbm, _, peak_src = peaks()
-    for n, var in ((2, "F1"), (2, "F1A"), (3, "F2"), (5, "F2A")):
+    for n, var in ((2, "F1"), (2, "F1A"), (3, "F2"), (4, "F3"), (4, "F3A"), (5, "F2A")):
         w = gen.WORKLOADS[n]
         d = gen.workload_inputs(n, var)
         B, H, L, dk, dv = w["B"], w["H"], w["L"], w["dk"], w["dv"]
@@ -564,7 +565,7 @@ def run_backward(args):
         do = torch.from_numpy(rng.standard_normal((B, H, L, dv)).astype(np.float32)).to(torch.bfloat16).cuda()
         ds = torch.from_numpy(rng.standard_normal((B, H, dv, dk)).astype(np.float32)).cuda()
         a = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
-        F.bwd(var, *a, d["eps"], do, ds)
+        F.bwd(var, *a, d["eps"], do, ds, window=w["window"])
         torch.cuda.synchronize()
         ms = []
         for _ in range(max(3, min(args.steps, 10))):
@@ -572,7 +573,7 @@ def run_backward(args):
             torch.cuda._sleep(HEAD_START_CYCLES)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            F.bwd(var, *a, d["eps"], do, ds)
+            F.bwd(var, *a, d["eps"], do, ds, window=w["window"])
             e1.record()
             torch.cuda.synchronize()
             ms.append(e0.elapsed_time(e1))
@@ -585,7 +586,7 @@ def run_backward(args):
                 "kernels": "bwd_prep_kernel + bwd_sweep_kernel + bwd_decay_kernel + bwd_key_kernel",
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                              "peak_source": peak_src, "algorithmic_bytes_per_launch": ab}}
-        if n == 2 and not args.no_cpu_baseline:
+        if n in (2, 4) and not args.no_cpu_baseline:
             import oracle
             oracle.build()
             units = [(b, h) for b in range(B) for h in range(H)][:min(os.cpu_count() or 1, B * H)]
@@ -593,7 +594,7 @@ def run_backward(args):
             sel = lambda x: np.ascontiguousarray(x[bs, hs][None])  # noqa: E731
             t0 = time.perf_counter()
             oracle.bwd(var, *(sel(d[k]) for k in ("q_64", "k_64", "v_64", "beta_64")), np.asarray(d["lam_64"])[hs],
-                       d["eps_64"], sel(do.double().cpu().numpy()), sel(ds.double().cpu().numpy()))
+                       d["eps_64"], sel(do.double().cpu().numpy()), sel(ds.double().cpu().numpy()), window=w["window"])
             sec = time.perf_counter() - t0
             line["cpu_oracle"] = {"value": len(units) * L / H / sec, "unit": "tokens/s", "cores": os.cpu_count(),
                                   "kind": "oracle", "sample": "fp64 reverse mode, %d whole (b,h) units, %.1f s"

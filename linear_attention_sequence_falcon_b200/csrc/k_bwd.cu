@@ -43,7 +43,6 @@ namespace {
 
 constexpr int TT = 32;             // tokens staged per tile
 constexpr int MAXW = 8;            // window bound (the forward's kMaxWindow)
-constexpr int TW = TT + MAXW - 1;  // sample rows staged per tile
 
 template <typename T>
 __device__ __forceinline__ float ld(const T *p, size_t i) {
@@ -96,9 +95,12 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdParams p, float *xs, f
 
 // Shared-memory tiles of one sweep: q, do, eta, alpha of TT tokens (eta and
 // alpha per channel; scalars repeated), and x, y of the TW samples from
-// t0 - (MAXW - 1): token i's window slot m is sample row i + MAXW - 1 - m.
-template <typename T, int D>
+// t0 - (MW - 1): token i's window slot m is sample row i + MW - 1 - m.  MW is
+// the number of window slots the kernel is built for (1, or MAXW for the
+// windowed variants).
+template <typename T, int D, int MW>
 struct Tiles {
+    static constexpr int TW = TT + MW - 1;  // sample rows staged per tile
     float *tq, *tdo, *te, *ta, *tx, *ty;
     __device__ Tiles(float *base) {
         tq = base; tdo = tq + TT * D; te = tdo + TT * D; ta = te + TT * D; tx = ta + TT * D; ty = tx + TW * D;
@@ -116,26 +118,26 @@ struct Tiles {
             ta[e] = in ? al[(size_t)t * nch + (nch > 1 ? c : 0)] : 1.f;
         }
         for (int e = threadIdx.x; e < TW * D; e += blockDim.x) {
-            const int r = e / D, c = e % D, sidx = t0 - (MAXW - 1) + r;
-            const bool in = r < n + MAXW - 1 && sidx >= 0 && sidx < L;
+            const int r = e / D, c = e % D, sidx = t0 - (MW - 1) + r;
+            const bool in = r < n + MW - 1 && sidx >= 0 && sidx < L;
             tx[e] = in ? x[(size_t)sidx * D + c] : 0.f;
             ty[e] = in ? ld(v, (size_t)sidx * D + c) : 0.f;
         }
     }
-    __device__ float x(int i, int m, int c) const { return tx[(i + MAXW - 1 - m) * D + c]; }
-    __device__ float y(int i, int m, int j) const { return ty[(i + MAXW - 1 - m) * D + j]; }
+    __device__ float x(int i, int m, int c) const { return tx[(i + MW - 1 - m) * D + c]; }
+    __device__ float y(int i, int m, int j) const { return ty[(i + MW - 1 - m) * D + j]; }
 };
 
 // The sweeps of one (b, h) for the inner-product family (Falcon-1A/2A/3A).
-template <typename T, int D>
+template <typename T, int D, int MW>
 __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const float *xs, const float *etas,
                                                           const float *alphas, float *dga, float *dgb, float *deta,
                                                           float *dx) {
     constexpr int NT = 256, LD = D + 1, RPT = NT / D, SEG = D / RPT;
     extern __shared__ float sm[];
     float *S = sm;                          // [D][LD]: S, then Gs
-    Tiles<T, D> tl(S + D * LD);
-    float *ta_next = tl.ty + TW * D;        // [D] alpha of the token after the tile
+    Tiles<T, D, MW> tl(S + D * LD);
+    float *ta_next = tl.ty + Tiles<T, D, MW>::TW * D;        // [D] alpha of the token after the tile
     float *vsum = ta_next + D;              // [D] per-row terms summed for the scalar variants
     const int tid = threadIdx.x, L = p.L, w = p.window;
     const size_t bh = blockIdx.x;
@@ -163,7 +165,7 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
                 const int j = e / D, c = e % D;
                 float u = 0.f;
 #pragma unroll
-                for (int m = 0; m < MAXW; ++m)
+                for (int m = 0; m < MW; ++m)
                     if (m < w) u = fmaf(tl.y(i, m, j), tl.x(i, m, c), u);
                 S[j * LD + c] = tl.ta[i * D + j] * S[j * LD + c] + tl.te[i * D + j] * u;
             }
@@ -208,9 +210,9 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
         S[j * LD + c] = p.dstate ? p.dstate[(bh * D + j) * D + c] : 0.f;
     }
     for (int e = tid; e < D; e += NT) ta_next[e] = 1.f;  // no step after the last token
-    float acc_dy[MAXW], acc_dx[MAXW];  // samples t - m: row rj of dy, column rj of dx
+    float acc_dy[MW], acc_dx[MW];  // samples t - m: row rj of dy, column rj of dx
 #pragma unroll
-    for (int m = 0; m < MAXW; ++m) acc_dy[m] = acc_dx[m] = 0.f;
+    for (int m = 0; m < MW; ++m) acc_dy[m] = acc_dx[m] = 0.f;
     const int ntile = (L + TT - 1) / TT;
     for (int tb = ntile - 1; tb >= 0; --tb) {
         const int t0 = tb * TT, n = min(TT, L - t0);
@@ -225,14 +227,14 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
                 S[j * LD + c] = anext[j] * S[j * LD + c] + tl.tdo[i * D + j] * tl.tq[i * D + c];
             }
             __syncthreads();
-            float gx[MAXW], dxm[MAXW];  // row rj: (Gs x_{t-m})_j; column rj: (Gs^T (eta o y_{t-m}))_c
+            float gx[MW], dxm[MW];  // row rj: (Gs x_{t-m})_j; column rj: (Gs^T (eta o y_{t-m}))_c
 #pragma unroll
-            for (int m = 0; m < MAXW; ++m) gx[m] = dxm[m] = 0.f;
+            for (int m = 0; m < MW; ++m) gx[m] = dxm[m] = 0.f;
             for (int s = 0; s < SEG; ++s) {
                 const int c = rp * SEG + s;
                 const float gr = S[rj * LD + c], gc = S[c * LD + rj], ec = tl.te[i * D + c];
 #pragma unroll
-                for (int m = 0; m < MAXW; ++m)
+                for (int m = 0; m < MW; ++m)
                     if (m < w) {
                         gx[m] = fmaf(gr, tl.x(i, m, c), gx[m]);
                         dxm[m] = fmaf(gc, ec * tl.y(i, m, c), dxm[m]);
@@ -241,7 +243,7 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
             float sy = 0.f;  // sum_m y_{t-m,j} (Gs x_{t-m})_j
             const float eta = tl.te[i * D + rj];
 #pragma unroll
-            for (int m = 0; m < MAXW; ++m)
+            for (int m = 0; m < MW; ++m)
                 if (m < w) {
 #pragma unroll
                     for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
@@ -263,11 +265,11 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
                 }
             }
 #pragma unroll
-            for (int m = 0; m < MAXW - 1; ++m) {
+            for (int m = 0; m < MW - 1; ++m) {
                 acc_dy[m] = acc_dy[m + 1];
                 acc_dx[m] = acc_dx[m + 1];
             }
-            acc_dy[MAXW - 1] = acc_dx[MAXW - 1] = 0.f;
+            acc_dy[MW - 1] = acc_dx[MW - 1] = 0.f;
             __syncthreads();
             if (nch == 1 && tid < 32) {
                 float a = 0.f;
@@ -293,17 +295,17 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
 //   dy_{t-m} += de_m,  dx_{t-m} += Gs^T (eta e_m) - S_{t-1}^T de_m,
 //   Gs <- alpha o Gs - sum_m de_m x_{t-m}^T.
 // dalpha goes straight into dga (no scan).
-template <typename T, int D>
+template <typename T, int D, int MW>
 __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, const float *xs, const float *etas,
                                                               const float *alphas, float *dga, float *deta, float *dx,
                                                               float *ck, float *ts) {
     constexpr int NT = 256, LD = D + 1, RPT = NT / D, SEG = D / RPT;
     extern __shared__ float sm[];
     float *S = sm;                          // [D][LD]: S, then Gs
-    Tiles<T, D> tl(S + D * LD);
-    float *ve = tl.ty + TW * D;             // [MAXW][D] e (forward) or eta e (reverse) of the window
-    float *vde = ve + MAXW * D;             // [MAXW][D] de of the window
-    float *vsum = vde + MAXW * D;           // [2][D] per-row terms summed for the scalar variants
+    Tiles<T, D, MW> tl(S + D * LD);
+    float *ve = tl.ty + Tiles<T, D, MW>::TW * D;             // [MW][D] e (forward) or eta e (reverse) of the window
+    float *vde = ve + MW * D;             // [MW][D] de of the window
+    float *vsum = vde + MW * D;           // [2][D] per-row terms summed for the scalar variants
     const int tid = threadIdx.x, L = p.L, w = p.window;
     const size_t bh = blockIdx.x;
     const int nch = channels(p);
@@ -322,18 +324,18 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
 
     // one step of the recurrence on S with token i of the staged tile
     auto step = [&](int i) {
-        float r[MAXW];
+        float r[MW];
 #pragma unroll
-        for (int m = 0; m < MAXW; ++m) r[m] = 0.f;
+        for (int m = 0; m < MW; ++m) r[m] = 0.f;
         for (int s = 0; s < SEG; ++s) {
             const int c = rp * SEG + s;
             const float sv = S[rj * LD + c];
 #pragma unroll
-            for (int m = 0; m < MAXW; ++m)
+            for (int m = 0; m < MW; ++m)
                 if (m < w) r[m] = fmaf(sv, tl.x(i, m, c), r[m]);
         }
 #pragma unroll
-        for (int m = 0; m < MAXW; ++m)
+        for (int m = 0; m < MW; ++m)
             if (m < w) {
 #pragma unroll
                 for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) r[m] += __shfl_xor_sync(0xffffffffu, r[m], o2);
@@ -344,7 +346,7 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
             const int j = e / D, c = e % D;
             float u = 0.f;
 #pragma unroll
-            for (int m = 0; m < MAXW; ++m)
+            for (int m = 0; m < MW; ++m)
                 if (m < w) u = fmaf(ve[m * D + j], tl.x(i, m, c), u);
             S[j * LD + c] = tl.ta[i * D + j] * S[j * LD + c] + tl.te[i * D + j] * u;
         }
@@ -378,9 +380,9 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
         const int j = e / D, c = e % D;
         S[j * LD + c] = p.dstate ? p.dstate[(bh * D + j) * D + c] : 0.f;  // dL/dS_L
     }
-    float acc_dy[MAXW], acc_dx[MAXW];  // samples t - m: row rj of dy, column rj of dx
+    float acc_dy[MW], acc_dx[MW];  // samples t - m: row rj of dy, column rj of dx
 #pragma unroll
-    for (int m = 0; m < MAXW; ++m) acc_dy[m] = acc_dx[m] = 0.f;
+    for (int m = 0; m < MW; ++m) acc_dy[m] = acc_dx[m] = 0.f;
     for (int tb = ntile - 1; tb >= 0; --tb) {
         const int t0 = tb * TT, n = min(TT, L - t0);
         float *ckt = cks + (size_t)tb * D * D;
@@ -409,15 +411,15 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
                 S[j * LD + c] += tl.tdo[i * D + j] * tl.tq[i * D + c];
             }
             __syncthreads();
-            float sx[MAXW], gx[MAXW], gs = 0.f;  // row rj: (S_{t-1} x_{t-m}), (Gs x_{t-m}), <Gs, S_{t-1}>
+            float sx[MW], gx[MW], gs = 0.f;  // row rj: (S_{t-1} x_{t-m}), (Gs x_{t-m}), <Gs, S_{t-1}>
 #pragma unroll
-            for (int m = 0; m < MAXW; ++m) sx[m] = gx[m] = 0.f;
+            for (int m = 0; m < MW; ++m) sx[m] = gx[m] = 0.f;
             for (int s = 0; s < SEG; ++s) {
                 const int c = rp * SEG + s;
                 const float sp = Sp[(size_t)rj * D + c], g = S[rj * LD + c];
                 gs = fmaf(g, sp, gs);
 #pragma unroll
-                for (int m = 0; m < MAXW; ++m)
+                for (int m = 0; m < MW; ++m)
                     if (m < w) {
                         const float xv = tl.x(i, m, c);
                         sx[m] = fmaf(sp, xv, sx[m]);
@@ -429,7 +431,7 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
             const float eta = tl.te[i * D + rj];
             float dterm = 0.f;
 #pragma unroll
-            for (int m = 0; m < MAXW; ++m)
+            for (int m = 0; m < MW; ++m)
                 if (m < w) {
 #pragma unroll
                     for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
@@ -454,18 +456,18 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
                 }
             }
             __syncthreads();
-            float dxm[MAXW];  // column rj: sum_j (eta e_m)_j Gs[j][c] - de_{m,j} S_{t-1}[j][c]
+            float dxm[MW];  // column rj: sum_j (eta e_m)_j Gs[j][c] - de_{m,j} S_{t-1}[j][c]
 #pragma unroll
-            for (int m = 0; m < MAXW; ++m) dxm[m] = 0.f;
+            for (int m = 0; m < MW; ++m) dxm[m] = 0.f;
             for (int s = 0; s < SEG; ++s) {
                 const int j = rp * SEG + s;
                 const float gc = S[j * LD + rj], sc = Sp[(size_t)j * D + rj];
 #pragma unroll
-                for (int m = 0; m < MAXW; ++m)
+                for (int m = 0; m < MW; ++m)
                     if (m < w) dxm[m] = fmaf(ve[m * D + j], gc, fmaf(-vde[m * D + j], sc, dxm[m]));
             }
 #pragma unroll
-            for (int m = 0; m < MAXW; ++m)
+            for (int m = 0; m < MW; ++m)
                 if (m < w) {
 #pragma unroll
                     for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) dxm[m] += __shfl_xor_sync(0xffffffffu, dxm[m], o2);
@@ -476,11 +478,11 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
                 dxo[(size_t)t * D + rj] = acc_dx[0];
             }
 #pragma unroll
-            for (int m = 0; m < MAXW - 1; ++m) {
+            for (int m = 0; m < MW - 1; ++m) {
                 acc_dy[m] = acc_dy[m + 1];
                 acc_dx[m] = acc_dx[m + 1];
             }
-            acc_dy[MAXW - 1] = acc_dx[MAXW - 1] = 0.f;
+            acc_dy[MW - 1] = acc_dx[MW - 1] = 0.f;
             if (nch == 1 && tid < 32) {
                 float a = 0.f, b = 0.f;
                 for (int j = tid; j < D; j += 32) {
@@ -500,7 +502,7 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
                 const int j = e / D, c = e % D;
                 float u = 0.f;
 #pragma unroll
-                for (int m = 0; m < MAXW; ++m)
+                for (int m = 0; m < MW; ++m)
                     if (m < w) u = fmaf(vde[m * D + j], tl.x(i, m, c), u);
                 S[j * LD + c] = tl.ta[i * D + j] * S[j * LD + c] - u;
             }
@@ -634,20 +636,29 @@ __global__ void __launch_bounds__(256) bwd_key_kernel(BwdParams p, const float *
 
 __host__ __device__ bool regression(int v) { return v == F1 || v == F2 || v == F3; }
 
-template <typename T, int D>
-int launch_sweep(const BwdParams &p, const float *xs, const float *etas, const float *alphas, float *dga, float *dgb,
-                 float *deta, float *dx, float *ck, float *ts, cudaStream_t s) {
-    constexpr size_t base = (size_t)D * (D + 1) + Tiles<T, D>::floats;
+template <typename T, int D, int MW>
+int launch_sweep_w(const BwdParams &p, const float *xs, const float *etas, const float *alphas, float *dga, float *dgb,
+                   float *deta, float *dx, float *ck, float *ts, cudaStream_t s) {
+    constexpr size_t base = (size_t)D * (D + 1) + Tiles<T, D, MW>::floats;
     if (regression(p.variant)) {
-        const size_t bytes = (base + 2 * MAXW * D + 2 * D) * sizeof(float);
-        cudaFuncSetAttribute(bwd_sweep_reg_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-        bwd_sweep_reg_kernel<T, D><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
+        const size_t bytes = (base + 2 * MW * D + 2 * D) * sizeof(float);
+        cudaFuncSetAttribute(bwd_sweep_reg_kernel<T, D, MW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        bwd_sweep_reg_kernel<T, D, MW>
+            <<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
         return 0;
     }
     const size_t bytes = (base + 2 * D) * sizeof(float);
-    cudaFuncSetAttribute(bwd_sweep_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    bwd_sweep_kernel<T, D><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
+    cudaFuncSetAttribute(bwd_sweep_kernel<T, D, MW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    bwd_sweep_kernel<T, D, MW><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
     return 0;
+}
+
+// one window slot for the single-sample variants, MAXW for Falcon-3/3A
+template <typename T, int D>
+int launch_sweep(const BwdParams &p, const float *xs, const float *etas, const float *alphas, float *dga, float *dgb,
+                 float *deta, float *dx, float *ck, float *ts, cudaStream_t s) {
+    if (p.window > 1) return launch_sweep_w<T, D, MAXW>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s);
+    return launch_sweep_w<T, D, 1>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s);
 }
 
 }  // namespace
