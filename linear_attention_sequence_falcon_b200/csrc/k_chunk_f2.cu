@@ -254,6 +254,8 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
 #pragma unroll
             for (int s = 0; s < 64; ++s) Z[s] = 0.f;
             if (!unsafe) {
+                // in blocks of 8 tokens: the sums over the rows before a block are one
+                // batch of independent dot products, the rows inside it a short walk
                 float Gprev = 0.f;
 #pragma unroll
                 for (int tb = 0; tb < 4; ++tb) {
@@ -261,23 +263,35 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
                     tc::tmem_ld16(tl + C_S + tb * 16, xs);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int t = tb * 16 + i;
-                        const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
-                        const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
-                        const float G = Gt[gidx(t, jj)];
-                        const float r = __expf(gc - G) * eta * (pair_get(sm, F_V, t, jj) - __expf(Gprev) * xs[i]);
-                        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                    for (int hb = 0; hb < 2; ++hb) {
+                        const int t0 = tb * 16 + hb * 8;
+                        float r[8], kap[8], cr[8];
 #pragma unroll
-                        for (int s = 0; s < t; s += 4) {
-                            const float4 a = *reinterpret_cast<const float4 *>(At + t * LDA + s);
-                            a0 = fmaf(a.x, Z[s], a0);
-                            a1 = fmaf(a.y, Z[s + 1], a1);
-                            a2 = fmaf(a.z, Z[s + 2], a2);
-                            a3 = fmaf(a.w, Z[s + 3], a3);
+                        for (int i = 0; i < 8; ++i) {
+                            const int t = t0 + i;
+                            const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
+                            const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
+                            const float G = Gt[gidx(t, jj)];
+                            r[i] = __expf(gc - G) * eta * (pair_get(sm, F_V, t, jj) - __expf(Gprev) * xs[hb * 8 + i]);
+                            kap[i] = __fdividef(eta, alpha);
+                            cr[i] = 0.f;
+                            Gprev = G;
                         }
-                        Z[t] = r - __fdividef(eta, alpha) * ((a0 + a1) + (a2 + a3));
-                        Gprev = G;
+#pragma unroll
+                        for (int s = 0; s < t0; s += 4) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float4 a = *reinterpret_cast<const float4 *>(At + (t0 + i) * LDA + s);
+                                cr[i] = fmaf(a.x, Z[s], fmaf(a.y, Z[s + 1], fmaf(a.z, Z[s + 2], fmaf(a.w, Z[s + 3], cr[i]))));
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float acc = cr[i];
+#pragma unroll
+                            for (int s = t0; s < t0 + i; ++s) acc = fmaf(At[(t0 + i) * LDA + s], Z[s], acc);
+                            Z[t0 + i] = r[i] - kap[i] * acc;
+                        }
                     }
                 }
             } else {
