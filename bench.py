@@ -342,29 +342,26 @@ def run_ours(args):
     tokens_per_step = len(w["variants"]) * w["B"] * w["L"]
     value, total_ms = weak_scaling_value(world, tokens_per_step, args.steps, sum(step_ms))
 
-    # end to end through the C ABI from pinned host buffers
-    hq, hk, hv, hb = (d[n].pin_memory() for n in ("q", "k", "v", "beta"))
-    ho = {var: torch.empty_like(outs[var], device="cpu").pin_memory() for var in w["variants"]}
-    hs = {var: torch.empty_like(states[var], device="cpu").pin_memory() for var in w["variants"]}
+    # end to end through the C ABI on pinned host buffers: falcon_fwd_host
+    # copies the inputs in, runs both variants and copies outputs and states
+    # back, the batch cut into slices so that copies and compute overlap
+    hq, hk, hv, hb, hl = (d[n].pin_memory() for n in ("q", "k", "v", "beta", "lam"))
+    ho = [torch.empty_like(outs[var], device="cpu").pin_memory() for var in w["variants"]]
+    hs = [torch.empty_like(states[var], device="cpu").pin_memory() for var in w["variants"]]
     e2e_ms = []
     for i in range(max(args.warmup, 3) + args.steps):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True); beta.copy_(hb, non_blocking=True)
-        step()
-        for var in w["variants"]:
-            ho[var].copy_(outs[var], non_blocking=True)
-            hs[var].copy_(states[var], non_blocking=True)
+        F.fwd_host(w["variants"], "chunk", hq, hk, hv, hb, hl, d["eps"], chunk=w["chunk"], out=ho,
+                   final_state=hs, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize()
         if i >= max(args.warmup, 3):
             e2e_ms.append(e0.elapsed_time(e1))
     e2e_value, _ = weak_scaling_value(world, tokens_per_step, args.steps, sum(e2e_ms))
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb))
-    d2h = sum(ho[var].numel() * ho[var].element_size() + hs[var].numel() * hs[var].element_size()
-              for var in w["variants"])
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb, hl))
+    d2h = sum(t.numel() * t.element_size() for t in ho + hs)
 
     hbm, tflops, src = peaks()
     f1_ms = statistics.mean(per_var["F1"])

@@ -117,6 +117,45 @@ int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype,
                   void *out, float *final_state, cudaStream_t stream);
 
 /*
+ * falcon_fwd_host -- falcon_fwd_ex for inputs and outputs in HOST memory,
+ * for one or several variants over the same inputs.  The library copies the
+ * inputs to the device, runs the forward and copies the results back.  The
+ * batch is cut into `slices` runs of whole batch rows; slice i's inputs go
+ * host->device on a library-owned copy stream while slice i-1 computes on
+ * `stream` and slice i-2's outputs go device->host on a second copy stream.
+ *
+ *   n_variants   1..6 entries of `variants`, all with the same beta layout
+ *                (all per value channel, Falcon-2/2A, or none): every one is
+ *                computed from the same inputs (FALCON_ERR_UNSUPPORTED
+ *                otherwise, and for n_variants outside 1..6 or slices < 0)
+ *   q, k, v, beta, lambda   as in falcon_fwd_ex, in host memory (page-locked
+ *                memory lets the copies run asynchronously and overlap;
+ *                pageable memory gives the same results without overlap)
+ *   out          array of n_variants host pointers, out[i] [B,H,L,d_v] dtype
+ *   final_state  NULL, or an array of n_variants host pointers (entries may
+ *                be NULL), final_state[i] [B,H,d_v,d_k] fp32
+ *   slices       number of slices, clamped to [1, min(B, 64)]; 0 lets the
+ *                library choose (about one per 4 MiB of input, at most 8)
+ *   every other argument as in falcon_fwd_ex.
+ * The call returns once the work is enqueued.  The host buffers must stay
+ * valid, and the inputs unchanged, until `stream` has passed the call's work;
+ * the outputs are complete then (cudaStreamSynchronize(stream)).  The device
+ * buffers (inputs, lambda, outputs and states: about the inputs' size plus
+ * n_variants times the outputs') are one stream-ordered block from the
+ * library's pool, freed on `stream` at the end of the call's work.  Argument
+ * errors return before anything is enqueued.  An error after the first copy
+ * (FALCON_ERR_LAUNCH, or a status of the per-slice forward) stops further
+ * slices; the streams are still joined into `stream` and the block freed,
+ * and the outputs are then incomplete.
+ */
+int falcon_fwd_host(int n_variants, const falcon_variant *variants, falcon_form form, falcon_dtype dtype,
+                    falcon_pairing pairing, falcon_phi phi,
+                    const void *q, const void *k, const void *v, const void *beta,
+                    const float *lambda, float eps, int window,
+                    int B, int H, int L, int d_k, int d_v, int chunk,
+                    void *const *out, float *const *final_state, int slices, cudaStream_t stream);
+
+/*
  * falcon_fwd_carry -- falcon_fwd over a segment that continues a sequence:
  * the recurrence picks up where an earlier segment (or a run of decode
  * steps) left off.  Chunks already hand a fixed-size state from one to the
@@ -167,7 +206,7 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
  *   dstate      [B,H,d_v,d_k] fp32, or NULL (zero): dL/d(final_state)
  *   dq, dk      [B,H,L,d_k] fp32, written
  *   dv          [B,H,L,d_v] fp32, written
- *   dbeta       [B,H,L] (Falcon-1A) or [B,H,L,d_v] (Falcon-2A) fp32, written
+ *   dbeta       [B,H,L] (Falcon-1/3/1A/3A) or [B,H,L,d_v] (Falcon-2/2A) fp32, written
  *   dlambda     [H] fp32, written (summed over b), or NULL
  * The regression family's derivative needs S_{t-1} at every step: the
  * forward sweep keeps S every 32 tokens and the reverse sweep recomputes

@@ -21,7 +21,7 @@ FORMS = {"recurrent": 0, "masked": 1, "chunk": 2}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PAIRINGS = {"prefix": 0, "same_step": 1}
 PHIS = {"l2": 0, "identity": 1}
-EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_fwd_carry", "falcon_bwd", "falcon_decode_step", "falcon_decode_carry_from_prefill",
+EXPORTS = ("falcon_fwd", "falcon_fwd_ex", "falcon_fwd_host", "falcon_fwd_carry", "falcon_bwd", "falcon_decode_step", "falcon_decode_carry_from_prefill",
            "falcon_fwd_masked_noalloc", "falcon_device_wait_timeouts", "falcon_selftest_bounded_wait",
            "falcon_scratch_trim", "falcon_status_string")
 
@@ -45,6 +45,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.falcon_fwd.restype = I
     lib.falcon_fwd_ex.argtypes = [I, I, I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, I, P, P, P]
     lib.falcon_fwd_ex.restype = I
+    lib.falcon_fwd_host.argtypes = [I, P, I, I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, I, P, P, I, P]
+    lib.falcon_fwd_host.restype = I
     lib.falcon_fwd_carry.argtypes = [I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, I, P, P, P, P, P, P]
     lib.falcon_fwd_carry.restype = I
     lib.falcon_bwd.argtypes = [I, I, I, I, P, P, P, P, P, F, I, I, I, I, I, I, P, P, P, P, P, P, P, P]
@@ -122,6 +124,59 @@ def fwd(variant: str, form: str, q, k, v, beta, lam, eps: float, window: int = 1
         rc = lib.falcon_fwd_ex(VARIANTS[variant], FORMS[form], DTYPES[q.dtype], PAIRINGS[pairing], PHIS[phi],
                                _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(lam), float(eps), int(window),
                                B, H, L, dk, dv, int(chunk), _ptr(out), _ptr(final_state), _stream(stream))
+    _check(rc)
+    return out, final_state
+
+
+def _host_ptr(t):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise FalconError("fwd_host takes host (CPU) tensors")
+    if not t.is_contiguous():
+        raise FalconError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def fwd_host(variants, form: str, q, k, v, beta, lam, eps: float, window: int = 1, chunk: int = 64,
+             out=None, final_state=None, pairing: str = "prefix", phi: str = "l2", slices: int = 0,
+             want_state: bool = True, stream=None):
+    """falcon_fwd_host: the forward of one or several variants over the same
+    inputs in host memory (CPU tensors; pinned memory lets the library overlap
+    the copies of one batch slice with the compute of the next).  q,k
+    [B,H,L,dk], v [B,H,L,dv], beta [B,H,L] or [B,H,L,dv] (same dtype), lam [H]
+    fp32.  Returns (outs, states): lists of CPU tensors, one per variant
+    (pinned when allocated here).  The call only enqueues; synchronise the
+    stream before reading the results."""
+    lib = load()
+    if isinstance(variants, str):
+        variants = [variants]
+    n = len(variants)
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in DTYPES or not (q.dtype == k.dtype == v.dtype == beta.dtype):
+        raise FalconError("q, k, v, beta must share one dtype, fp32 or bf16")
+    if lam.dtype != torch.float32:
+        raise FalconError("lambda must be fp32")
+    pin = torch.cuda.is_available()
+    if out is None:
+        out = [torch.empty((B, H, L, dv), dtype=q.dtype, pin_memory=pin) for _ in range(n)]
+    if final_state is None and want_state:
+        final_state = [torch.empty((B, H, dv, dk), dtype=torch.float32, pin_memory=pin) for _ in range(n)]
+    if len(out) != n or (final_state is not None and len(final_state) != n):
+        raise FalconError("one output (and one state) per variant")
+    vids = (ctypes.c_int * n)(*(VARIANTS[x] for x in variants))
+    outs = (ctypes.c_void_p * n)(*(_host_ptr(o) for o in out))
+    states = None
+    if final_state is not None:
+        for st in final_state:
+            if st is not None and st.dtype != torch.float32:
+                raise FalconError("final states are fp32")
+        states = (ctypes.c_void_p * n)(*(_host_ptr(st) for st in final_state))
+    hp = lambda t: ctypes.c_void_p(_host_ptr(t))  # noqa: E731
+    rc = lib.falcon_fwd_host(n, vids, FORMS[form], DTYPES[q.dtype], PAIRINGS[pairing], PHIS[phi],
+                             hp(q), hp(k), hp(v), hp(beta), hp(lam), float(eps), int(window),
+                             B, H, L, dk, dv, int(chunk), outs, states, int(slices), _stream(stream))
     _check(rc)
     return out, final_state
 

@@ -29,19 +29,30 @@ int launched(int rc) {
 
 }  // namespace
 
-namespace {
+namespace falcon {
 
-int fwd_impl(falcon_variant variant, falcon_form form, falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
-             const void *q, const void *k, const void *v, const void *beta, const float *lambda, float eps,
-             int window, int B, int H, int L, int d_k, int d_v, int chunk, const float *init_state,
-             const float *x_prev, const float *win, void *out, float *final_state, cudaStream_t stream) {
-    int rc = validate_common(variant, dtype, window);
+int validate_fwd(int variant, int form, int dtype, int pairing, int phi, int window, int B, int H, int L, int d_k,
+                 int d_v, int chunk) {
+    const int rc = validate_common(variant, dtype, window);
     if (rc) return rc;
     if (form < FALCON_RECURRENT || form > FALCON_CHUNK) return FALCON_ERR_ENUM;
     if (pairing != FALCON_PAIR_PREFIX && pairing != FALCON_PAIR_SAME_STEP) return FALCON_ERR_ENUM;
     if (phi != FALCON_PHI_L2 && phi != FALCON_PHI_IDENTITY) return FALCON_ERR_ENUM;
     if (B < 0 || H < 0 || L < 0 || !dim_ok(d_k) || !dim_ok(d_v)) return FALCON_ERR_SHAPE;
     if (form == FALCON_CHUNK && !(chunk == 16 || chunk == 32 || chunk == 64)) return FALCON_ERR_CHUNK;
+    return FALCON_OK;
+}
+
+}  // namespace falcon
+
+namespace {
+
+int fwd_impl(falcon_variant variant, falcon_form form, falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
+             const void *q, const void *k, const void *v, const void *beta, const float *lambda, float eps,
+             int window, int B, int H, int L, int d_k, int d_v, int chunk, const float *init_state,
+             const float *x_prev, const float *win, void *out, float *final_state, cudaStream_t stream) {
+    int rc = validate_fwd(variant, form, dtype, pairing, phi, window, B, H, L, d_k, d_v, chunk);
+    if (rc) return rc;
     const bool has_window = variant == FALCON_F3 || variant == FALCON_F3A;
     FwdParams p{};
     p.variant = variant; p.form = form; p.pairing = pairing; p.phi = phi;

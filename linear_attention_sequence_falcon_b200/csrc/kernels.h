@@ -38,7 +38,7 @@ unsigned int f2_wait_timeouts();
 int launch_w_chunk(const FwdParams &p, cudaStream_t s);
 unsigned int w_wait_timeouts();
 template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
-// Backward pass of Falcon-1A / Falcon-2A (recurrent form, fp32), d_k = d_v in
+// Backward pass of every variant (recurrent form, fp32), d_k = d_v in
 // {32, 64, 128}; the arguments are validated by the caller.
 template <typename T> int launch_bwd(const BwdParams &p, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
@@ -48,6 +48,11 @@ template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
 cudaError_t scratch_alloc(void **ptr, size_t bytes, cudaStream_t s);
 cudaError_t scratch_free(void *ptr, cudaStream_t s);
 cudaError_t scratch_trim();
+
+// The argument checks of falcon_fwd_ex (FALCON_OK or the status it returns
+// for them); nothing is enqueued.
+int validate_fwd(int variant, int form, int dtype, int pairing, int phi, int window, int B, int H, int L, int d_k,
+                 int d_v, int chunk);
 
 // Scratch sizes (floats) of the masked-parallel form.
 size_t masked_ws_r_floats(const FwdParams &p);

@@ -88,3 +88,31 @@ def test_backward_validation_codes(lib):
     assert _bwd(lib, ptr=0) == -1
     assert _bwd(lib, B=0) == 0
     assert _bwd(lib, L=0, dlam=False) == 0
+
+
+def _host(lib, variants=(0, 3), form=2, dtype=1, window=1, B=1, H=1, L=8, dk=64, dv=64, chunk=64, ptr=1,
+          outs=(1, 1), slices=0, vnull=False):
+    P = ctypes.c_void_p(ptr) if ptr else None
+    n = len(variants)
+    vids = None if vnull else (ctypes.c_int * max(n, 1))(*variants)
+    out = (ctypes.c_void_p * max(len(outs), 1))(*outs)
+    return lib.falcon_fwd_host(n, vids, form, dtype, 0, 0, P, P, P, P, P, 1e-6, window, B, H, L, dk, dv, chunk,
+                               out, None, slices, None)
+
+
+def test_host_validation_codes(lib):
+    """falcon_fwd_host answers argument errors before any copy or launch."""
+    lib.falcon_fwd_host.restype = ctypes.c_int
+    assert _host(lib, variants=()) == -9
+    assert _host(lib, variants=(0,) * 7, outs=(1,) * 7) == -9
+    assert _host(lib, slices=-1) == -9
+    assert _host(lib, vnull=True) == -1
+    assert _host(lib, variants=(0, 9)) == -2
+    assert _host(lib, variants=(0, 1)) == -9  # scalar and per-channel beta in one call
+    assert _host(lib, variants=(1, 4), B=0) == 0  # Falcon-2 and Falcon-2A share the per-channel layout
+    assert _host(lib, chunk=100) == -4
+    assert _host(lib, dk=48) == -3
+    assert _host(lib, variants=(2,), outs=(1,), window=0) == -6
+    assert _host(lib, ptr=0) == -1
+    assert _host(lib, outs=(1, 0)) == -1
+    assert _host(lib, B=0) == 0
