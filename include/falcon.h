@@ -22,8 +22,9 @@
  * alpha) per value channel j, i.e. per row of S ([NEWS] 02 (2)).
  *
  * Conventions shared by every entry point:
- *  - All tensor arguments are DEVICE pointers to contiguous row-major arrays
- *    owned by the caller; the library never frees or retains them.
+ *  - All tensor arguments are DEVICE pointers (HOST pointers for
+ *    falcon_fwd_host) to contiguous row-major arrays owned by the caller;
+ *    the library never frees or retains them.
  *  - Calls only enqueue work on `stream` (0 = legacy default stream) and never
  *    synchronise.  A non-zero return means nothing was enqueued, except
  *    FALCON_ERR_LAUNCH, which reports cudaGetLastError() after a launch.
@@ -130,7 +131,8 @@ int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype,
  *                otherwise, and for n_variants outside 1..6 or slices < 0)
  *   q, k, v, beta, lambda   as in falcon_fwd_ex, in host memory (page-locked
  *                memory lets the copies run asynchronously and overlap;
- *                pageable memory gives the same results without overlap)
+ *                pageable memory gives the same results without overlap,
+ *                and its copies may block the calling thread)
  *   out          array of n_variants host pointers, out[i] [B,H,L,d_v] dtype
  *   final_state  NULL, or an array of n_variants host pointers (entries may
  *                be NULL), final_state[i] [B,H,d_v,d_k] fp32
