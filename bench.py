@@ -555,6 +555,8 @@ def run_backward(args):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     hbm, _, peak_src = peaks()
     for n, var in ((2, "F1"), (2, "F1A"), (3, "F2"), (4, "F3"), (4, "F3A"), (5, "F2A")):
+        if args.only and n != args.only:
+            continue
         w = gen.WORKLOADS[n]
         d = gen.workload_inputs(n, var)
         B, H, L, dk, dv = w["B"], w["H"], w["L"], w["dk"], w["dv"]
@@ -640,7 +642,7 @@ def main():
                     help="run only warmup+steps decode steps (no flush or JSON), for ncu")
     ap.add_argument("--workloads", action="store_true",
                     help="time every workload and form of the workloads table, one JSON line each")
-    ap.add_argument("--only", type=int, default=0, help="with --workloads: just this workload number")
+    ap.add_argument("--only", type=int, default=0, help="with --workloads or --backward: just this workload number")
     ap.add_argument("--backward", action="store_true",
                     help="time falcon_bwd on workloads 2 (Falcon-1, -1A), 3 (Falcon-2) and 5's prefill (Falcon-2A)")
     ap.add_argument("--chunk-sweep", action="store_true",
