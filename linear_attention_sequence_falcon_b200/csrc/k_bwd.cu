@@ -286,6 +286,229 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
     }
 }
 
+// The sweeps of one (b, h) for the inner-product family with one sample per
+// update (Falcon-1A, Falcon-2A; Falcon-3A with a window of 1), S and then Gs
+// held in registers.  Warp w owns rows [w D/8, (w+1) D/8); lane (rg, cg) =
+// (lane / 8, lane % 8) owns NR = D/32 of them and the NC = D/8 columns from
+// cg NC.  A row sum adds the 8 lanes of a row group (shuffles); a column sum
+// adds the 4 row groups (shuffles), then the 8 warps through shared memory,
+// double-buffered by token parity so that each token needs one barrier.
+// Same arithmetic as bwd_sweep_kernel, with the summation order of the
+// reductions changed.
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 1) bwd_sweep_rs_kernel(BwdParams p, const float *xs, const float *etas,
+                                                             const float *alphas, float *dga, float *dgb,
+                                                             float *deta, float *dx) {
+    constexpr int NR = D / 32, NC = D / 8, NW = 8;
+    extern __shared__ float sm[];
+    Tiles<T, D, 1> tl(sm);
+    float *ta_next = tl.ty + Tiles<T, D, 1>::TW * D;  // [D] alpha of the token after the tile
+    float *red = ta_next + D;                         // [2][NW][D] column partials of each warp
+    float *red1 = red + 2 * NW * D;                   // [2][NW] scalar partials of each warp
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rg = lane >> 3, cg = lane & 7;
+    const int j0 = warp * (D / NW) + rg * NR, c0 = cg * NC;  // this lane's first row and column
+    const int L = p.L;
+    const size_t bh = blockIdx.x;
+    const int nch = channels(p);
+    const T *q = static_cast<const T *>(p.q) + bh * (size_t)L * D;
+    const T *v = static_cast<const T *>(p.v) + bh * (size_t)L * D;
+    const T *dout = static_cast<const T *>(p.dout) + bh * (size_t)L * D;
+    const float *x = xs + bh * (size_t)L * D;
+    const float *et = etas + bh * (size_t)L * nch, *al = alphas + bh * (size_t)L * nch;
+    float *dq = p.dq + bh * (size_t)L * D, *dv = p.dv_out + bh * (size_t)L * D;
+    float *ga = dga + bh * (size_t)L * nch, *gb = dgb + bh * (size_t)L * nch, *de = deta + bh * (size_t)L * nch;
+    float *dxo = dx + bh * (size_t)L * D;
+    const float *dst = p.dstate ? p.dstate + bh * (size_t)D * D : nullptr;
+
+    auto load_cols = [&](const float *row, float (&f)[NC]) {
+#pragma unroll
+        for (int k = 0; k < NC; k += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(row + c0 + k);
+            f[k] = a.x; f[k + 1] = a.y; f[k + 2] = a.z; f[k + 3] = a.w;
+        }
+    };
+    // column sums: over this lane's rows (done by the caller), the 4 row groups,
+    // then (after the barrier) the 8 warps
+    auto put_cols = [&](float (&f)[NC], float *rb) {
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+            f[k] += __shfl_xor_sync(0xffffffffu, f[k], 8);
+            f[k] += __shfl_xor_sync(0xffffffffu, f[k], 16);
+        }
+        if (rg == 0)
+#pragma unroll
+            for (int k = 0; k < NC; k += 4)
+                *reinterpret_cast<float4 *>(rb + warp * D + c0 + k) = make_float4(f[k], f[k + 1], f[k + 2], f[k + 3]);
+    };
+    auto row_sum = [&](float s) {
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        return s;
+    };
+    auto warp_rows_sum = [&](float s) {  // over the 4 row groups (each row counted once)
+        s += __shfl_xor_sync(0xffffffffu, s, 8);
+        s += __shfl_xor_sync(0xffffffffu, s, 16);
+        return s;
+    };
+
+    float Sr[NR][NC];
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int k = 0; k < NC; ++k) Sr[r][k] = 0.f;
+    int par = 0;
+
+    // ---- forward sweep: S_t, dq_t = S_t^T do_t and do_t o o_t (+ <dS_L, S_L> at the end)
+    for (int t0 = 0; t0 < L; t0 += TT) {
+        const int n = min(TT, L - t0);
+        __syncthreads();
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
+        __syncthreads();
+        for (int i = 0; i < n; ++i, par ^= 1) {
+            const int t = t0 + i;
+            float xc[NC], qc[NC], orow[NR], dj[NR], frow[NR];
+            load_cols(tl.tx + i * D, xc);
+            load_cols(tl.tq + i * D, qc);
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const int j = j0 + r;
+                const float a = tl.ta[i * D + j], u = tl.te[i * D + j] * tl.ty[i * D + j];
+                float o = 0.f;
+#pragma unroll
+                for (int k = 0; k < NC; ++k) {
+                    Sr[r][k] = fmaf(a, Sr[r][k], u * xc[k]);
+                    o = fmaf(Sr[r][k], qc[k], o);
+                }
+                orow[r] = o;
+                dj[r] = tl.tdo[i * D + j];
+                frow[r] = 0.f;
+            }
+            if (t == L - 1 && dst) {  // the same for every thread
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    float f = 0.f;
+#pragma unroll
+                    for (int k = 0; k < NC; ++k) f = fmaf(Sr[r][k], dst[(size_t)(j0 + r) * D + c0 + k], f);
+                    frow[r] = row_sum(f);
+                }
+            }
+            float gcol[NC];
+#pragma unroll
+            for (int k = 0; k < NC; ++k) {
+                float g = 0.f;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) g = fmaf(Sr[r][k], dj[r], g);
+                gcol[k] = g;
+            }
+            float *rb = red + par * NW * D;
+            put_cols(gcol, rb);
+            float asum = 0.f;
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const float a = dj[r] * row_sum(orow[r]) + frow[r];
+                if (nch > 1 && cg == 0) ga[(size_t)t * D + j0 + r] = a;
+                asum += a;
+            }
+            if (nch == 1) {
+                asum = warp_rows_sum(asum);
+                if (lane == 0) red1[par * NW + warp] = asum;
+            }
+            __syncthreads();
+            if (tid < D) {
+                float g = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) g += rb[w * D + tid];
+                dq[(size_t)t * D + tid] = g;
+            }
+            if (nch == 1 && tid == 255) {
+                float a = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) a += red1[par * NW + w];
+                ga[t] = a;
+            }
+        }
+    }
+    // ---- reverse sweep: Gs_t; dy_t and dx_t; deta_t; the key-side dG
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int k = 0; k < NC; ++k) Sr[r][k] = dst ? dst[(size_t)(j0 + r) * D + c0 + k] : 0.f;
+    __syncthreads();
+    for (int e = tid; e < D; e += blockDim.x) ta_next[e] = 1.f;  // no step after the last token
+    const int ntile = (L + TT - 1) / TT;
+    for (int tb = ntile - 1; tb >= 0; --tb) {
+        const int t0 = tb * TT, n = min(TT, L - t0);
+        __syncthreads();
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
+        __syncthreads();
+        for (int i = n - 1; i >= 0; --i, par ^= 1) {
+            const int t = t0 + i;
+            const float *anext = i + 1 < n ? tl.ta + (i + 1) * D : ta_next;
+            float xc[NC], qc[NC], gx[NR], ey[NR];
+            load_cols(tl.tx + i * D, xc);
+            load_cols(tl.tq + i * D, qc);
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const int j = j0 + r;
+                const float an = anext[j], dj = tl.tdo[i * D + j];
+                float g = 0.f;
+#pragma unroll
+                for (int k = 0; k < NC; ++k) {
+                    Sr[r][k] = fmaf(an, Sr[r][k], dj * qc[k]);
+                    g = fmaf(Sr[r][k], xc[k], g);
+                }
+                gx[r] = g;
+                ey[r] = tl.te[i * D + j] * tl.ty[i * D + j];
+            }
+            float dcol[NC];
+#pragma unroll
+            for (int k = 0; k < NC; ++k) {
+                float s = 0.f;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) s = fmaf(Sr[r][k], ey[r], s);
+                dcol[k] = s;
+            }
+            float *rb = red + par * NW * D;
+            put_cols(dcol, rb);
+            float ssum = 0.f;
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const int j = j0 + r;
+                const float g = row_sum(gx[r]), eta = tl.te[i * D + j], sy = tl.ty[i * D + j] * g;
+                if (cg == 0) {
+                    dv[(size_t)t * D + j] = eta * g;
+                    if (nch > 1) {
+                        de[(size_t)t * D + j] = sy;
+                        gb[(size_t)t * D + j] = eta * sy;
+                    }
+                }
+                ssum += sy;
+            }
+            if (nch == 1) {
+                ssum = warp_rows_sum(ssum);
+                if (lane == 0) red1[par * NW + warp] = ssum;
+            }
+            __syncthreads();
+            if (tid < D) {
+                float s = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) s += rb[w * D + tid];
+                dxo[(size_t)t * D + tid] = s;
+            }
+            if (nch == 1 && tid == 255) {
+                float a = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) a += red1[par * NW + w];
+                de[t] = a;
+                gb[t] = tl.te[i * D] * a;
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < D; e += blockDim.x) ta_next[e] = tl.ta[e];  // alpha of this tile's first token
+    }
+}
+
 // The sweeps of one (b, h) for the regression family (Falcon-1/2/3).  The
 // forward sweep keeps S before every tile (ck); the reverse sweep swaps Gs
 // with the tile's checkpoint, recomputes the tile's states S_{t-1} into the
@@ -647,9 +870,15 @@ int launch_sweep_w(const BwdParams &p, const float *xs, const float *etas, const
             <<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
         return 0;
     }
-    const size_t bytes = (base + 2 * D) * sizeof(float);
-    cudaFuncSetAttribute(bwd_sweep_kernel<T, D, MW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    bwd_sweep_kernel<T, D, MW><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
+    if constexpr (MW == 1) {  // one sample per update: S in registers
+        const size_t bytes = (Tiles<T, D, 1>::floats + D + 2 * 8 * D + 2 * 8) * sizeof(float);
+        cudaFuncSetAttribute(bwd_sweep_rs_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        bwd_sweep_rs_kernel<T, D><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
+    } else {
+        const size_t bytes = (base + 2 * D) * sizeof(float);
+        cudaFuncSetAttribute(bwd_sweep_kernel<T, D, MW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        bwd_sweep_kernel<T, D, MW><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
+    }
     return 0;
 }
 

@@ -120,11 +120,12 @@ def test_backward_workload2_sampled(F, variant):
     check(got, ref)
 
 
-@pytest.mark.parametrize("w", [2, 4, 8])
+@pytest.mark.parametrize("w", [1, 2, 4, 8])
 @pytest.mark.parametrize("variant", ["F3", "F3A"])
 def test_backward_windows(F, variant, w):
-    """Windows of 2, 4 and 8 samples (the staged tile carries the 7 samples
-    before it; each sample's gradient gathers the w steps that use it)."""
+    """Windows of 1, 2, 4 and 8 samples (the staged tile carries the 7 samples
+    before it; each sample's gradient gathers the w steps that use it; a
+    window of 1 runs the single-sample sweeps)."""
     got, ref = grads_case(F, variant, 1, 2, 75, 64, "f32", seed=250 + w, window=w)
     check(got, ref)
 
