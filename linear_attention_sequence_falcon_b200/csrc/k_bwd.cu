@@ -509,6 +509,243 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_rs_kernel(BwdParams p, const
     }
 }
 
+// The sweeps of one (b, h) for the regression family with one sample per
+// update (Falcon-1, Falcon-2; Falcon-3 with a window of 1), S, Gs and the
+// walked state S_{t-1} held in registers with the lane layout of
+// bwd_sweep_rs_kernel.  The forward sweep keeps S before every tile (ck); the
+// reverse sweep recomputes a tile's states S_{t-1} from that checkpoint into
+// the head's scratch (ts) and walks the tile back:
+//   Gs += do q^T;  e = y - S_{t-1} x,  de = eta o (Gs x),
+//   dalpha = <Gs, S_{t-1}>,  deta = e o (Gs x)  (per row),
+//   dy_t = de,  dx_t = Gs^T (eta o e) - S_{t-1}^T de,  Gs <- alpha o Gs - de x^T.
+// Every lane reads back only the checkpoint and state elements it wrote.
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 1) bwd_sweep_reg_rs_kernel(BwdParams p, const float *xs, const float *etas,
+                                                                 const float *alphas, float *dga, float *deta,
+                                                                 float *dx, float *ck, float *ts) {
+    constexpr int NR = D / 32, NC = D / 8, NW = 8;
+    extern __shared__ float sm[];
+    Tiles<T, D, 1> tl(sm);
+    float *red = tl.ty + Tiles<T, D, 1>::TW * D;  // [2][NW][D] column partials of each warp
+    float *red1 = red + 2 * NW * D;               // [2][NW][2] scalar partials (dalpha, deta) of each warp
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rg = lane >> 3, cg = lane & 7;
+    const int j0 = warp * (D / NW) + rg * NR, c0 = cg * NC;
+    const int L = p.L;
+    const size_t bh = blockIdx.x;
+    const int nch = channels(p);
+    const T *q = static_cast<const T *>(p.q) + bh * (size_t)L * D;
+    const T *v = static_cast<const T *>(p.v) + bh * (size_t)L * D;
+    const T *dout = static_cast<const T *>(p.dout) + bh * (size_t)L * D;
+    const float *x = xs + bh * (size_t)L * D;
+    const float *et = etas + bh * (size_t)L * nch, *al = alphas + bh * (size_t)L * nch;
+    float *dq = p.dq + bh * (size_t)L * D, *dv = p.dv_out + bh * (size_t)L * D;
+    float *ga = dga + bh * (size_t)L * nch, *de = deta + bh * (size_t)L * nch;
+    float *dxo = dx + bh * (size_t)L * D;
+    const int ntile = (L + TT - 1) / TT;
+    float *cks = ck + bh * (size_t)ntile * D * D;  // S before each tile
+    float *tss = ts + bh * (size_t)TT * D * D;     // S before each token of the tile being walked
+    const float *dst = p.dstate ? p.dstate + bh * (size_t)D * D : nullptr;
+
+    auto load_cols = [&](const float *row, float (&f)[NC]) {
+#pragma unroll
+        for (int k = 0; k < NC; k += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(row + c0 + k);
+            f[k] = a.x; f[k + 1] = a.y; f[k + 2] = a.z; f[k + 3] = a.w;
+        }
+    };
+    auto store_img = [&](float *img, const float (&A)[NR][NC]) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+            for (int k = 0; k < NC; k += 4)
+                *reinterpret_cast<float4 *>(img + (size_t)(j0 + r) * D + c0 + k) =
+                    make_float4(A[r][k], A[r][k + 1], A[r][k + 2], A[r][k + 3]);
+    };
+    auto load_img = [&](const float *img, float (&A)[NR][NC]) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+            for (int k = 0; k < NC; k += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(img + (size_t)(j0 + r) * D + c0 + k);
+                A[r][k] = a.x; A[r][k + 1] = a.y; A[r][k + 2] = a.z; A[r][k + 3] = a.w;
+            }
+    };
+    auto put_cols = [&](float (&f)[NC], float *rb) {
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+            f[k] += __shfl_xor_sync(0xffffffffu, f[k], 8);
+            f[k] += __shfl_xor_sync(0xffffffffu, f[k], 16);
+        }
+        if (rg == 0)
+#pragma unroll
+            for (int k = 0; k < NC; k += 4)
+                *reinterpret_cast<float4 *>(rb + warp * D + c0 + k) = make_float4(f[k], f[k + 1], f[k + 2], f[k + 3]);
+    };
+    auto row_sum = [&](float s) {
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        return s;
+    };
+    auto warp_rows_sum = [&](float s) {
+        s += __shfl_xor_sync(0xffffffffu, s, 8);
+        s += __shfl_xor_sync(0xffffffffu, s, 16);
+        return s;
+    };
+    // one step of the recurrence on A = S with token i of the staged tile
+    auto step = [&](float (&A)[NR][NC], int i, const float (&xc)[NC]) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            const int j = j0 + r;
+            float s = 0.f;
+#pragma unroll
+            for (int k = 0; k < NC; ++k) s = fmaf(A[r][k], xc[k], s);
+            const float u = tl.te[i * D + j] * (tl.ty[i * D + j] - row_sum(s)), a = tl.ta[i * D + j];
+#pragma unroll
+            for (int k = 0; k < NC; ++k) A[r][k] = fmaf(a, A[r][k], u * xc[k]);
+        }
+    };
+
+    float A[NR][NC];  // S (forward), Gs (reverse)
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int k = 0; k < NC; ++k) A[r][k] = 0.f;
+    int par = 0;
+
+    // ---- forward sweep: checkpoints, S_t, dq_t = S_t^T do_t
+    for (int tb = 0; tb < ntile; ++tb) {
+        const int t0 = tb * TT, n = min(TT, L - t0);
+        __syncthreads();
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
+        __syncthreads();
+        store_img(cks + (size_t)tb * D * D, A);
+        for (int i = 0; i < n; ++i, par ^= 1) {
+            float xc[NC];
+            load_cols(tl.tx + i * D, xc);
+            step(A, i, xc);
+            float dj[NR], gcol[NC];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) dj[r] = tl.tdo[i * D + j0 + r];
+#pragma unroll
+            for (int k = 0; k < NC; ++k) {
+                float g = 0.f;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) g = fmaf(A[r][k], dj[r], g);
+                gcol[k] = g;
+            }
+            float *rb = red + par * NW * D;
+            put_cols(gcol, rb);
+            __syncthreads();
+            if (tid < D) {
+                float g = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) g += rb[w * D + tid];
+                dq[(size_t)(t0 + i) * D + tid] = g;
+            }
+        }
+    }
+    // ---- reverse sweep, tile by tile
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int k = 0; k < NC; ++k) A[r][k] = dst ? dst[(size_t)(j0 + r) * D + c0 + k] : 0.f;  // dL/dS_L
+    for (int tb = ntile - 1; tb >= 0; --tb) {
+        const int t0 = tb * TT, n = min(TT, L - t0);
+        __syncthreads();
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
+        __syncthreads();
+        {   // the tile's states S_{t-1}, recomputed from its checkpoint
+            float P[NR][NC];
+            load_img(cks + (size_t)tb * D * D, P);
+            for (int i = 0; i < n; ++i) {
+                store_img(tss + (size_t)i * D * D, P);
+                float xc[NC];
+                load_cols(tl.tx + i * D, xc);
+                step(P, i, xc);
+            }
+        }
+        for (int i = n - 1; i >= 0; --i, par ^= 1) {
+            const int t = t0 + i;
+            float P[NR][NC], xc[NC], qc[NC];
+            load_img(tss + (size_t)i * D * D, P);
+            load_cols(tl.tx + i * D, xc);
+            load_cols(tl.tq + i * D, qc);
+            float ve[NR], vd[NR], gsum = 0.f, dsum = 0.f;
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const int j = j0 + r;
+                const float dj = tl.tdo[i * D + j];
+                float sx = 0.f, gx = 0.f, gs = 0.f;
+#pragma unroll
+                for (int k = 0; k < NC; ++k) {
+                    A[r][k] = fmaf(dj, qc[k], A[r][k]);
+                    sx = fmaf(P[r][k], xc[k], sx);
+                    gx = fmaf(A[r][k], xc[k], gx);
+                    gs = fmaf(A[r][k], P[r][k], gs);
+                }
+                sx = row_sum(sx);
+                gx = row_sum(gx);
+                gs = row_sum(gs);
+                const float eta = tl.te[i * D + j], e = tl.ty[i * D + j] - sx, d = eta * gx, dterm = e * gx;
+                ve[r] = eta * e;
+                vd[r] = d;
+                if (cg == 0) {
+                    dv[(size_t)t * D + j] = d;
+                    if (nch > 1) {
+                        ga[(size_t)t * D + j] = gs;
+                        de[(size_t)t * D + j] = dterm;
+                    }
+                }
+                gsum += gs;
+                dsum += dterm;
+            }
+            float dcol[NC];  // Gs^T (eta o e) - S_{t-1}^T de
+#pragma unroll
+            for (int k = 0; k < NC; ++k) {
+                float s = 0.f;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) s = fmaf(ve[r], A[r][k], fmaf(-vd[r], P[r][k], s));
+                dcol[k] = s;
+            }
+            float *rb = red + par * NW * D;
+            put_cols(dcol, rb);
+            if (nch == 1) {
+                gsum = warp_rows_sum(gsum);
+                dsum = warp_rows_sum(dsum);
+                if (lane == 0) {
+                    red1[(par * NW + warp) * 2] = gsum;
+                    red1[(par * NW + warp) * 2 + 1] = dsum;
+                }
+            }
+            // Gs <- alpha o Gs - de x^T  (dL/dS_{t-1})
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const float a = tl.ta[i * D + j0 + r];
+#pragma unroll
+                for (int k = 0; k < NC; ++k) A[r][k] = fmaf(a, A[r][k], -vd[r] * xc[k]);
+            }
+            __syncthreads();
+            if (tid < D) {
+                float s = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) s += rb[w * D + tid];
+                dxo[(size_t)t * D + tid] = s;
+            }
+            if (nch == 1 && tid == 255) {
+                float a = 0.f, b = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) {
+                    a += red1[(par * NW + w) * 2];
+                    b += red1[(par * NW + w) * 2 + 1];
+                }
+                ga[t] = a;
+                de[t] = b;
+            }
+        }
+    }
+}
+
 // The sweeps of one (b, h) for the regression family (Falcon-1/2/3).  The
 // forward sweep keeps S before every tile (ck); the reverse sweep swaps Gs
 // with the tile's checkpoint, recomputes the tile's states S_{t-1} into the
@@ -864,10 +1101,19 @@ int launch_sweep_w(const BwdParams &p, const float *xs, const float *etas, const
                    float *deta, float *dx, float *ck, float *ts, cudaStream_t s) {
     constexpr size_t base = (size_t)D * (D + 1) + Tiles<T, D, MW>::floats;
     if (regression(p.variant)) {
-        const size_t bytes = (base + 2 * MW * D + 2 * D) * sizeof(float);
-        cudaFuncSetAttribute(bwd_sweep_reg_kernel<T, D, MW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-        bwd_sweep_reg_kernel<T, D, MW>
-            <<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
+        if constexpr (MW == 1) {  // one sample per update: S, Gs and S_{t-1} in registers
+            const size_t bytes = (Tiles<T, D, 1>::floats + 2 * 8 * D + 2 * 8 * 2) * sizeof(float);
+            cudaFuncSetAttribute(bwd_sweep_reg_rs_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)bytes);
+            bwd_sweep_reg_rs_kernel<T, D>
+                <<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
+        } else {
+            const size_t bytes = (base + 2 * MW * D + 2 * D) * sizeof(float);
+            cudaFuncSetAttribute(bwd_sweep_reg_kernel<T, D, MW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)bytes);
+            bwd_sweep_reg_kernel<T, D, MW>
+                <<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
+        }
         return 0;
     }
     if constexpr (MW == 1) {  // one sample per update: S in registers
@@ -902,7 +1148,9 @@ int launch_bwd(const BwdParams &p, cudaStream_t s) {
     // deta, dx; the regression family adds the tile checkpoints and one tile of states per head
     const size_t BH = (size_t)p.B * p.H, ntile = (p.L + TT - 1) / TT;
     const size_t nreg = reg ? BH * (ntile + TT) * D * D : 0;
-    const size_t nf = rows * D * 2 + rows + rows * nch * 5 + nreg;
+    // the checkpoints start on a 256-byte boundary (the sweeps move them in 16-byte pieces)
+    const size_t off_ck = (rows * D * 2 + rows + rows * nch * 5 + 63) & ~static_cast<size_t>(63);
+    const size_t nf = off_ck + nreg;
     void *ws = nullptr;
     if (scratch_alloc(&ws, nf * sizeof(float), s) != cudaSuccess) {
         cudaGetLastError();
@@ -911,7 +1159,7 @@ int launch_bwd(const BwdParams &p, cudaStream_t s) {
     float *xs = static_cast<float *>(ws), *dx = xs + rows * D, *ns = dx + rows * D;
     float *etas = ns + rows, *alphas = etas + rows * nch, *dga = alphas + rows * nch, *dgb = dga + rows * nch;
     float *deta = dgb + rows * nch;
-    float *ck = deta + rows * nch, *ts = ck + BH * ntile * D * D;
+    float *ck = xs + off_ck, *ts = ck + BH * ntile * D * D;
     const unsigned wblocks = (unsigned)((rows * 32 + 255) / 256);
     bwd_prep_kernel<T><<<wblocks, 256, 0, s>>>(p, xs, ns, etas, alphas);
     int rc = D == 32 ? launch_sweep<T, 32>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
