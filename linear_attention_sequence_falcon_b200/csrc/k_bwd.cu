@@ -27,11 +27,12 @@
 // k) take it to beta, lambda and k.
 //
 // Kernels: per-token samples and steps (a warp per token), the sweeps per
-// head (a block per (b, h); S, then Gs, in shared memory; tokens staged 32 at
-// a time with the B_w - 1 samples before them; each sample's dy and dx
-// gathered over the B_w steps that use it in a sliding register window), the
-// decay chain (a block per (b, h, channel)) and a warp per token for the
-// feature map.
+// head (a block per (b, h); tokens staged 32 at a time; with one sample per
+// update S, then Gs, live in registers; with a window they live in shared
+// memory, each tile is staged with the B_w - 1 samples before it and each
+// sample's dy and dx are gathered over the B_w steps that use it in a
+// sliding register window), the decay chain (a block per (b, h, channel))
+// and a warp per token for the feature map.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
