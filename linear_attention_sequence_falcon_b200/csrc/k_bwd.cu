@@ -27,11 +27,10 @@
 // k) take it to beta, lambda and k.
 //
 // Kernels: per-token samples and steps (a warp per token), the sweeps per
-// head (a block per (b, h); tokens staged 32 at a time; with one sample per
-// update S, then Gs, live in registers; with a window they live in shared
-// memory, each tile is staged with the B_w - 1 samples before it and each
-// sample's dy and dx are gathered over the B_w steps that use it in a
-// sliding register window), the decay chain (a block per (b, h, channel))
+// head (a block per (b, h); S, then Gs, in registers spread over the block;
+// tokens staged 32 at a time, with the B_w - 1 samples before them for a
+// window, each sample's dy and dx gathered over the B_w steps that use it in
+// sliding register windows), the decay chain (a block per (b, h, channel))
 // and a warp per token for the feature map.
 #include <cuda_bf16.h>
 
@@ -129,164 +128,6 @@ struct Tiles {
     __device__ float y(int i, int m, int j) const { return ty[(i + MW - 1 - m) * D + j]; }
 };
 
-// The sweeps of one (b, h) for the inner-product family (Falcon-1A/2A/3A).
-template <typename T, int D, int MW>
-__global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const float *xs, const float *etas,
-                                                          const float *alphas, float *dga, float *dgb, float *deta,
-                                                          float *dx) {
-    constexpr int NT = 256, LD = D + 1, RPT = NT / D, SEG = D / RPT;
-    extern __shared__ float sm[];
-    float *S = sm;                          // [D][LD]: S, then Gs
-    Tiles<T, D, MW> tl(S + D * LD);
-    float *ta_next = tl.ty + Tiles<T, D, MW>::TW * D;        // [D] alpha of the token after the tile
-    float *vsum = ta_next + D;              // [D] per-row terms summed for the scalar variants
-    const int tid = threadIdx.x, L = p.L, w = p.window;
-    const size_t bh = blockIdx.x;
-    const int nch = channels(p);
-    const T *q = static_cast<const T *>(p.q) + bh * (size_t)L * D;
-    const T *v = static_cast<const T *>(p.v) + bh * (size_t)L * D;
-    const T *dout = static_cast<const T *>(p.dout) + bh * (size_t)L * D;
-    const float *x = xs + bh * (size_t)L * D;
-    const float *et = etas + bh * (size_t)L * nch, *al = alphas + bh * (size_t)L * nch;
-    float *dq = p.dq + bh * (size_t)L * D, *dv = p.dv_out + bh * (size_t)L * D;
-    float *ga = dga + bh * (size_t)L * nch, *gb = dgb + bh * (size_t)L * nch, *de = deta + bh * (size_t)L * nch;
-    float *dxo = dx + bh * (size_t)L * D;
-    const int rj = tid / RPT, rp = tid % RPT;
-
-    // ---- forward sweep: S_t, dq_t = S_t^T do_t and do_t o o_t (+ <dS_L, S_L> at the end)
-    for (int e = tid; e < D * LD; e += NT) S[e] = 0.f;
-    for (int t0 = 0; t0 < L; t0 += TT) {
-        const int n = min(TT, L - t0);
-        __syncthreads();
-        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
-        __syncthreads();
-        for (int i = 0; i < n; ++i) {
-            const int t = t0 + i;
-            for (int e = tid; e < D * D; e += NT) {
-                const int j = e / D, c = e % D;
-                float u = 0.f;
-#pragma unroll
-                for (int m = 0; m < MW; ++m)
-                    if (m < w) u = fmaf(tl.y(i, m, j), tl.x(i, m, c), u);
-                S[j * LD + c] = tl.ta[i * D + j] * S[j * LD + c] + tl.te[i * D + j] * u;
-            }
-            __syncthreads();
-            float o = 0.f, g = 0.f, f = 0.f;  // row rj: (S q)_j; column rj: (S^T do)_c
-#pragma unroll 8
-            for (int s = 0; s < SEG; ++s) {
-                const int c = rp * SEG + s;
-                o = fmaf(S[rj * LD + c], tl.tq[i * D + c], o);
-                g = fmaf(S[c * LD + rj], tl.tdo[i * D + c], g);
-            }
-            if (t == L - 1 && p.dstate)
-                for (int s = 0; s < SEG; ++s) {
-                    const int c = rp * SEG + s;
-                    f = fmaf(S[rj * LD + c], p.dstate[(bh * D + rj) * D + c], f);
-                }
-#pragma unroll
-            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
-                o += __shfl_xor_sync(0xffffffffu, o, o2);
-                g += __shfl_xor_sync(0xffffffffu, g, o2);
-                f += __shfl_xor_sync(0xffffffffu, f, o2);
-            }
-            if (rp == 0) {
-                dq[(size_t)t * D + rj] = g;
-                const float a = tl.tdo[i * D + rj] * o + f;
-                if (nch > 1) ga[(size_t)t * D + rj] = a;
-                else vsum[rj] = a;
-            }
-            __syncthreads();
-            if (nch == 1 && tid < 32) {
-                float a = 0.f;
-                for (int j = tid; j < D; j += 32) a += vsum[j];
-                a = group_sum<32>(a);
-                if (tid == 0) ga[t] = a;
-            }
-        }
-    }
-    // ---- reverse sweep: Gs_t; dy and dx of the window's samples; deta_t; the key-side dG
-    __syncthreads();
-    for (int e = tid; e < D * D; e += NT) {
-        const int j = e / D, c = e % D;
-        S[j * LD + c] = p.dstate ? p.dstate[(bh * D + j) * D + c] : 0.f;
-    }
-    for (int e = tid; e < D; e += NT) ta_next[e] = 1.f;  // no step after the last token
-    float acc_dy[MW], acc_dx[MW];  // samples t - m: row rj of dy, column rj of dx
-#pragma unroll
-    for (int m = 0; m < MW; ++m) acc_dy[m] = acc_dx[m] = 0.f;
-    const int ntile = (L + TT - 1) / TT;
-    for (int tb = ntile - 1; tb >= 0; --tb) {
-        const int t0 = tb * TT, n = min(TT, L - t0);
-        __syncthreads();
-        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
-        __syncthreads();
-        for (int i = n - 1; i >= 0; --i) {
-            const int t = t0 + i;
-            const float *anext = i + 1 < n ? tl.ta + (i + 1) * D : ta_next;
-            for (int e = tid; e < D * D; e += NT) {
-                const int j = e / D, c = e % D;
-                S[j * LD + c] = anext[j] * S[j * LD + c] + tl.tdo[i * D + j] * tl.tq[i * D + c];
-            }
-            __syncthreads();
-            float gx[MW], dxm[MW];  // row rj: (Gs x_{t-m})_j; column rj: (Gs^T (eta o y_{t-m}))_c
-#pragma unroll
-            for (int m = 0; m < MW; ++m) gx[m] = dxm[m] = 0.f;
-            for (int s = 0; s < SEG; ++s) {
-                const int c = rp * SEG + s;
-                const float gr = S[rj * LD + c], gc = S[c * LD + rj], ec = tl.te[i * D + c];
-#pragma unroll
-                for (int m = 0; m < MW; ++m)
-                    if (m < w) {
-                        gx[m] = fmaf(gr, tl.x(i, m, c), gx[m]);
-                        dxm[m] = fmaf(gc, ec * tl.y(i, m, c), dxm[m]);
-                    }
-            }
-            float sy = 0.f;  // sum_m y_{t-m,j} (Gs x_{t-m})_j
-            const float eta = tl.te[i * D + rj];
-#pragma unroll
-            for (int m = 0; m < MW; ++m)
-                if (m < w) {
-#pragma unroll
-                    for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
-                        gx[m] += __shfl_xor_sync(0xffffffffu, gx[m], o2);
-                        dxm[m] += __shfl_xor_sync(0xffffffffu, dxm[m], o2);
-                    }
-                    acc_dy[m] += eta * gx[m];
-                    acc_dx[m] += dxm[m];
-                    sy = fmaf(tl.y(i, m, rj), gx[m], sy);
-                }
-            if (rp == 0) {
-                dv[(size_t)t * D + rj] = acc_dy[0];  // sample t: every step that uses it is done
-                dxo[(size_t)t * D + rj] = acc_dx[0];
-                if (nch > 1) {
-                    de[(size_t)t * D + rj] = sy;
-                    gb[(size_t)t * D + rj] = eta * sy;
-                } else {
-                    vsum[rj] = sy;
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < MW - 1; ++m) {
-                acc_dy[m] = acc_dy[m + 1];
-                acc_dx[m] = acc_dx[m + 1];
-            }
-            acc_dy[MW - 1] = acc_dx[MW - 1] = 0.f;
-            __syncthreads();
-            if (nch == 1 && tid < 32) {
-                float a = 0.f;
-                for (int j = tid; j < D; j += 32) a += vsum[j];
-                a = group_sum<32>(a);
-                if (tid == 0) {
-                    de[t] = a;
-                    gb[t] = tl.te[i * D] * a;
-                }
-            }
-        }
-        __syncthreads();
-        for (int e = tid; e < D; e += NT) ta_next[e] = tl.ta[e];  // alpha of this tile's first token
-    }
-}
-
 // The sweeps of one (b, h) for the inner-product family with one sample per
 // update (Falcon-1A, Falcon-2A; Falcon-3A with a window of 1), S and then Gs
 // held in registers.  Warp w owns rows [w D/8, (w+1) D/8); lane (rg, cg) =
@@ -294,8 +135,6 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_kernel(BwdParams p, const fl
 // cg NC.  A row sum adds the 8 lanes of a row group (shuffles); a column sum
 // adds the 4 row groups (shuffles), then the 8 warps through shared memory,
 // double-buffered by token parity so that each token needs one barrier.
-// Same arithmetic as bwd_sweep_kernel, with the summation order of the
-// reductions changed.
 template <typename T, int D>
 __global__ void __launch_bounds__(256, 1) bwd_sweep_rs_kernel(BwdParams p, const float *xs, const float *etas,
                                                              const float *alphas, float *dga, float *dgb,
@@ -747,27 +586,292 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_rs_kernel(BwdParams p, c
     }
 }
 
-// The sweeps of one (b, h) for the regression family (Falcon-1/2/3).  The
-// forward sweep keeps S before every tile (ck); the reverse sweep swaps Gs
-// with the tile's checkpoint, recomputes the tile's states S_{t-1} into the
-// block's scratch (ts), puts Gs back and walks the tile:
-//   e_m = y_{t-m} - S_{t-1} x_{t-m},  de_m = eta (Gs x_{t-m}),
-//   dalpha = <Gs, S_{t-1}>,  deta = sum_m e_m (Gs x_{t-m})  (per row),
-//   dy_{t-m} += de_m,  dx_{t-m} += Gs^T (eta e_m) - S_{t-1}^T de_m,
-//   Gs <- alpha o Gs - sum_m de_m x_{t-m}^T.
-// dalpha goes straight into dga (no scan).
-template <typename T, int D, int MW>
-__global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, const float *xs, const float *etas,
-                                                              const float *alphas, float *dga, float *deta, float *dx,
-                                                              float *ck, float *ts) {
-    constexpr int NT = 256, LD = D + 1, RPT = NT / D, SEG = D / RPT;
+// bwd_sweep_rs_kernel for a window of up to MAXW samples per update
+// (Falcon-3A): the tile carries the MAXW - 1 samples before it, and each
+// sample's dy (rows, on the lanes) and dx (columns, on the threads that
+// finish the column sums) gather the steps that use it in sliding register
+// windows, written once the reverse sweep passes the sample.
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 1) bwd_sweep_rsw_kernel(BwdParams p, const float *xs, const float *etas,
+                                                              const float *alphas, float *dga, float *dgb,
+                                                              float *deta, float *dx) {
+    constexpr int NR = D / 32, NC = D / 8, NW = 8, MW = MAXW;
     extern __shared__ float sm[];
-    float *S = sm;                          // [D][LD]: S, then Gs
-    Tiles<T, D, MW> tl(S + D * LD);
-    float *ve = tl.ty + Tiles<T, D, MW>::TW * D;             // [MW][D] e (forward) or eta e (reverse) of the window
-    float *vde = ve + MW * D;             // [MW][D] de of the window
-    float *vsum = vde + MW * D;           // [2][D] per-row terms summed for the scalar variants
-    const int tid = threadIdx.x, L = p.L, w = p.window;
+    Tiles<T, D, MW> tl(sm);
+    float *ta_next = tl.ty + Tiles<T, D, MW>::TW * D;  // [D] alpha of the token after the tile
+    float *red = ta_next + D;                          // [2][MW][NW][D] column partials of each warp
+    float *red1 = red + 2 * MW * NW * D;               // [2][NW] scalar partials of each warp
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rg = lane >> 3, cg = lane & 7;
+    const int j0 = warp * (D / NW) + rg * NR, c0 = cg * NC;
+    const int L = p.L, w = p.window;
+    const size_t bh = blockIdx.x;
+    const int nch = channels(p);
+    const T *q = static_cast<const T *>(p.q) + bh * (size_t)L * D;
+    const T *v = static_cast<const T *>(p.v) + bh * (size_t)L * D;
+    const T *dout = static_cast<const T *>(p.dout) + bh * (size_t)L * D;
+    const float *x = xs + bh * (size_t)L * D;
+    const float *et = etas + bh * (size_t)L * nch, *al = alphas + bh * (size_t)L * nch;
+    float *dq = p.dq + bh * (size_t)L * D, *dv = p.dv_out + bh * (size_t)L * D;
+    float *ga = dga + bh * (size_t)L * nch, *gb = dgb + bh * (size_t)L * nch, *de = deta + bh * (size_t)L * nch;
+    float *dxo = dx + bh * (size_t)L * D;
+    const float *dst = p.dstate ? p.dstate + bh * (size_t)D * D : nullptr;
+
+    auto load_cols = [&](const float *row, float (&f)[NC]) {
+#pragma unroll
+        for (int k = 0; k < NC; k += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(row + c0 + k);
+            f[k] = a.x; f[k + 1] = a.y; f[k + 2] = a.z; f[k + 3] = a.w;
+        }
+    };
+    auto put_cols = [&](float (&f)[NC], float *rb) {
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+            f[k] += __shfl_xor_sync(0xffffffffu, f[k], 8);
+            f[k] += __shfl_xor_sync(0xffffffffu, f[k], 16);
+        }
+        if (rg == 0)
+#pragma unroll
+            for (int k = 0; k < NC; k += 4)
+                *reinterpret_cast<float4 *>(rb + warp * D + c0 + k) = make_float4(f[k], f[k + 1], f[k + 2], f[k + 3]);
+    };
+    auto row_sum = [&](float s) {
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        return s;
+    };
+    auto warp_rows_sum = [&](float s) {
+        s += __shfl_xor_sync(0xffffffffu, s, 8);
+        s += __shfl_xor_sync(0xffffffffu, s, 16);
+        return s;
+    };
+    // sample row of token i's window slot m in the staged tile
+    auto srow = [&](int i, int m) { return (i + MW - 1 - m) * D; };
+
+    float Sr[NR][NC];
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int k = 0; k < NC; ++k) Sr[r][k] = 0.f;
+    int par = 0;
+
+    // ---- forward sweep: S_t, dq_t = S_t^T do_t and do_t o o_t (+ <dS_L, S_L> at the end)
+    for (int t0 = 0; t0 < L; t0 += TT) {
+        const int n = min(TT, L - t0);
+        __syncthreads();
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
+        __syncthreads();
+        for (int i = 0; i < n; ++i, par ^= 1) {
+            const int t = t0 + i;
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const float a = tl.ta[i * D + j0 + r];
+#pragma unroll
+                for (int k = 0; k < NC; ++k) Sr[r][k] *= a;
+            }
+#pragma unroll
+            for (int m = 0; m < MW; ++m)
+                if (m < w) {
+                    float xc[NC];
+                    load_cols(tl.tx + srow(i, m), xc);
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) {
+                        const float u = tl.te[i * D + j0 + r] * tl.ty[srow(i, m) + j0 + r];
+#pragma unroll
+                        for (int k = 0; k < NC; ++k) Sr[r][k] = fmaf(u, xc[k], Sr[r][k]);
+                    }
+                }
+            float qc[NC], orow[NR], dj[NR], frow[NR];
+            load_cols(tl.tq + i * D, qc);
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                float o = 0.f;
+#pragma unroll
+                for (int k = 0; k < NC; ++k) o = fmaf(Sr[r][k], qc[k], o);
+                orow[r] = o;
+                dj[r] = tl.tdo[i * D + j0 + r];
+                frow[r] = 0.f;
+            }
+            if (t == L - 1 && dst) {
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    float f = 0.f;
+#pragma unroll
+                    for (int k = 0; k < NC; ++k) f = fmaf(Sr[r][k], dst[(size_t)(j0 + r) * D + c0 + k], f);
+                    frow[r] = row_sum(f);
+                }
+            }
+            float gcol[NC];
+#pragma unroll
+            for (int k = 0; k < NC; ++k) {
+                float g = 0.f;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) g = fmaf(Sr[r][k], dj[r], g);
+                gcol[k] = g;
+            }
+            float *rb = red + par * MW * NW * D;
+            put_cols(gcol, rb);
+            float asum = 0.f;
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const float a = dj[r] * row_sum(orow[r]) + frow[r];
+                if (nch > 1 && cg == 0) ga[(size_t)t * D + j0 + r] = a;
+                asum += a;
+            }
+            if (nch == 1) {
+                asum = warp_rows_sum(asum);
+                if (lane == 0) red1[par * NW + warp] = asum;
+            }
+            __syncthreads();
+            if (tid < D) {
+                float g = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < NW; ++ww) g += rb[ww * D + tid];
+                dq[(size_t)t * D + tid] = g;
+            }
+            if (nch == 1 && tid == 255) {
+                float a = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < NW; ++ww) a += red1[par * NW + ww];
+                ga[t] = a;
+            }
+        }
+    }
+    // ---- reverse sweep: Gs_t; dy and dx of the window's samples; deta_t; the key-side dG
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int k = 0; k < NC; ++k) Sr[r][k] = dst ? dst[(size_t)(j0 + r) * D + c0 + k] : 0.f;
+    __syncthreads();
+    for (int e = tid; e < D; e += blockDim.x) ta_next[e] = 1.f;
+    float acc_dy[MW][NR];  // this lane's rows of dy of samples t - m
+    float acc_dx[MW];      // column tid of dx of samples t - m (threads tid < D)
+#pragma unroll
+    for (int m = 0; m < MW; ++m) {
+        acc_dx[m] = 0.f;
+#pragma unroll
+        for (int r = 0; r < NR; ++r) acc_dy[m][r] = 0.f;
+    }
+    const int ntile = (L + TT - 1) / TT;
+    for (int tb = ntile - 1; tb >= 0; --tb) {
+        const int t0 = tb * TT, n = min(TT, L - t0);
+        __syncthreads();
+        tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
+        __syncthreads();
+        for (int i = n - 1; i >= 0; --i, par ^= 1) {
+            const int t = t0 + i;
+            const float *anext = i + 1 < n ? tl.ta + (i + 1) * D : ta_next;
+            {
+                float qc[NC];
+                load_cols(tl.tq + i * D, qc);
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    const float an = anext[j0 + r], dj = tl.tdo[i * D + j0 + r];
+#pragma unroll
+                    for (int k = 0; k < NC; ++k) Sr[r][k] = fmaf(an, Sr[r][k], dj * qc[k]);
+                }
+            }
+            float sy[NR];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) sy[r] = 0.f;
+            float *rb = red + par * MW * NW * D;
+#pragma unroll
+            for (int m = 0; m < MW; ++m)
+                if (m < w) {
+                    float xc[NC], dcol[NC], ey[NR];
+                    load_cols(tl.tx + srow(i, m), xc);
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) {
+                        const int j = j0 + r;
+                        float g = 0.f;
+#pragma unroll
+                        for (int k = 0; k < NC; ++k) g = fmaf(Sr[r][k], xc[k], g);
+                        g = row_sum(g);
+                        const float eta = tl.te[i * D + j], y = tl.ty[srow(i, m) + j];
+                        acc_dy[m][r] += eta * g;
+                        sy[r] = fmaf(y, g, sy[r]);
+                        ey[r] = eta * y;
+                    }
+#pragma unroll
+                    for (int k = 0; k < NC; ++k) {
+                        float s = 0.f;
+#pragma unroll
+                        for (int r = 0; r < NR; ++r) s = fmaf(Sr[r][k], ey[r], s);
+                        dcol[k] = s;
+                    }
+                    put_cols(dcol, rb + m * NW * D);
+                }
+            float ssum = 0.f;
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const int j = j0 + r;
+                const float eta = tl.te[i * D + j];
+                if (cg == 0) {
+                    dv[(size_t)t * D + j] = acc_dy[0][r];  // sample t: every step that uses it is done
+                    if (nch > 1) {
+                        de[(size_t)t * D + j] = sy[r];
+                        gb[(size_t)t * D + j] = eta * sy[r];
+                    }
+                }
+                ssum += sy[r];
+            }
+#pragma unroll
+            for (int m = 0; m < MW - 1; ++m)
+#pragma unroll
+                for (int r = 0; r < NR; ++r) acc_dy[m][r] = acc_dy[m + 1][r];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) acc_dy[MW - 1][r] = 0.f;
+            if (nch == 1) {
+                ssum = warp_rows_sum(ssum);
+                if (lane == 0) red1[par * NW + warp] = ssum;
+            }
+            __syncthreads();
+            if (tid < D) {
+#pragma unroll
+                for (int m = 0; m < MW; ++m)
+                    if (m < w) {
+                        float s = 0.f;
+#pragma unroll
+                        for (int ww = 0; ww < NW; ++ww) s += rb[(m * NW + ww) * D + tid];
+                        acc_dx[m] += s;
+                    }
+                dxo[(size_t)t * D + tid] = acc_dx[0];
+#pragma unroll
+                for (int m = 0; m < MW - 1; ++m) acc_dx[m] = acc_dx[m + 1];
+                acc_dx[MW - 1] = 0.f;
+            }
+            if (nch == 1 && tid == 255) {
+                float a = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < NW; ++ww) a += red1[par * NW + ww];
+                de[t] = a;
+                gb[t] = tl.te[i * D] * a;
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < D; e += blockDim.x) ta_next[e] = tl.ta[e];
+    }
+}
+
+// bwd_sweep_reg_rs_kernel for a window of up to MAXW samples per update
+// (Falcon-3): every sample's error is taken at S_{t-1},
+//   e_m = y_{t-m} - S_{t-1} x_{t-m},  de_m = eta o (Gs x_{t-m}),
+//   dalpha = <Gs, S_{t-1}>,  deta = sum_m e_m o (Gs x_{t-m}),
+//   dy_{t-m} += de_m,  dx_{t-m} += Gs^T (eta o e_m) - S_{t-1}^T de_m,
+//   Gs <- alpha o Gs - sum_m de_m x_{t-m}^T,
+// with the sliding register windows of bwd_sweep_rsw_kernel for dy and dx.
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 1) bwd_sweep_reg_rsw_kernel(BwdParams p, const float *xs, const float *etas,
+                                                                  const float *alphas, float *dga, float *deta,
+                                                                  float *dx, float *ck, float *ts) {
+    constexpr int NR = D / 32, NC = D / 8, NW = 8, MW = MAXW;
+    extern __shared__ float sm[];
+    Tiles<T, D, MW> tl(sm);
+    float *red = tl.ty + Tiles<T, D, MW>::TW * D;  // [2][MW][NW][D] column partials of each warp
+    float *red1 = red + 2 * MW * NW * D;           // [2][NW][2] scalar partials (dalpha, deta) of each warp
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, rg = lane >> 3, cg = lane & 7;
+    const int j0 = warp * (D / NW) + rg * NR, c0 = cg * NC;
+    const int L = p.L, w = p.window;
     const size_t bh = blockIdx.x;
     const int nch = channels(p);
     const T *q = static_cast<const T *>(p.q) + bh * (size_t)L * D;
@@ -779,195 +883,278 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_kernel(BwdParams p, cons
     float *ga = dga + bh * (size_t)L * nch, *de = deta + bh * (size_t)L * nch;
     float *dxo = dx + bh * (size_t)L * D;
     const int ntile = (L + TT - 1) / TT;
-    float *cks = ck + bh * (size_t)ntile * D * D;   // S before each tile
-    float *tss = ts + bh * (size_t)TT * D * D;      // S before each token of the tile being walked
-    const int rj = tid / RPT, rp = tid % RPT;
+    float *cks = ck + bh * (size_t)ntile * D * D;
+    float *tss = ts + bh * (size_t)TT * D * D;
+    const float *dst = p.dstate ? p.dstate + bh * (size_t)D * D : nullptr;
 
-    // one step of the recurrence on S with token i of the staged tile
-    auto step = [&](int i) {
-        float r[MW];
+    auto load_cols = [&](const float *row, float (&f)[NC]) {
 #pragma unroll
-        for (int m = 0; m < MW; ++m) r[m] = 0.f;
-        for (int s = 0; s < SEG; ++s) {
-            const int c = rp * SEG + s;
-            const float sv = S[rj * LD + c];
+        for (int k = 0; k < NC; k += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(row + c0 + k);
+            f[k] = a.x; f[k + 1] = a.y; f[k + 2] = a.z; f[k + 3] = a.w;
+        }
+    };
+    auto store_img = [&](float *img, const float (&A)[NR][NC]) {
 #pragma unroll
-            for (int m = 0; m < MW; ++m)
-                if (m < w) r[m] = fmaf(sv, tl.x(i, m, c), r[m]);
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+            for (int k = 0; k < NC; k += 4)
+                *reinterpret_cast<float4 *>(img + (size_t)(j0 + r) * D + c0 + k) =
+                    make_float4(A[r][k], A[r][k + 1], A[r][k + 2], A[r][k + 3]);
+    };
+    auto load_img = [&](const float *img, float (&A)[NR][NC]) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+            for (int k = 0; k < NC; k += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(img + (size_t)(j0 + r) * D + c0 + k);
+                A[r][k] = a.x; A[r][k + 1] = a.y; A[r][k + 2] = a.z; A[r][k + 3] = a.w;
+            }
+    };
+    auto put_cols = [&](float (&f)[NC], float *rb) {
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+            f[k] += __shfl_xor_sync(0xffffffffu, f[k], 8);
+            f[k] += __shfl_xor_sync(0xffffffffu, f[k], 16);
+        }
+        if (rg == 0)
+#pragma unroll
+            for (int k = 0; k < NC; k += 4)
+                *reinterpret_cast<float4 *>(rb + warp * D + c0 + k) = make_float4(f[k], f[k + 1], f[k + 2], f[k + 3]);
+    };
+    auto row_sum = [&](float s) {
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        return s;
+    };
+    auto warp_rows_sum = [&](float s) {
+        s += __shfl_xor_sync(0xffffffffu, s, 8);
+        s += __shfl_xor_sync(0xffffffffu, s, 16);
+        return s;
+    };
+    auto srow = [&](int i, int m) { return (i + MW - 1 - m) * D; };
+    // one step of the recurrence on A = S with token i of the staged tile:
+    // every sample's error at S_{t-1} first, then the update
+    auto step = [&](float (&A)[NR][NC], int i) {
+        float u[MW][NR];
+#pragma unroll
+        for (int m = 0; m < MW; ++m)
+            if (m < w) {
+                float xc[NC];
+                load_cols(tl.tx + srow(i, m), xc);
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    float s = 0.f;
+#pragma unroll
+                    for (int k = 0; k < NC; ++k) s = fmaf(A[r][k], xc[k], s);
+                    u[m][r] = tl.te[i * D + j0 + r] * (tl.ty[srow(i, m) + j0 + r] - row_sum(s));
+                }
+            }
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            const float a = tl.ta[i * D + j0 + r];
+#pragma unroll
+            for (int k = 0; k < NC; ++k) A[r][k] *= a;
         }
 #pragma unroll
         for (int m = 0; m < MW; ++m)
             if (m < w) {
+                float xc[NC];
+                load_cols(tl.tx + srow(i, m), xc);
 #pragma unroll
-                for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) r[m] += __shfl_xor_sync(0xffffffffu, r[m], o2);
-                if (rp == 0) ve[m * D + rj] = tl.y(i, m, rj) - r[m];
+                for (int r = 0; r < NR; ++r)
+#pragma unroll
+                    for (int k = 0; k < NC; ++k) A[r][k] = fmaf(u[m][r], xc[k], A[r][k]);
             }
-        __syncthreads();
-        for (int e = tid; e < D * D; e += NT) {
-            const int j = e / D, c = e % D;
-            float u = 0.f;
-#pragma unroll
-            for (int m = 0; m < MW; ++m)
-                if (m < w) u = fmaf(ve[m * D + j], tl.x(i, m, c), u);
-            S[j * LD + c] = tl.ta[i * D + j] * S[j * LD + c] + tl.te[i * D + j] * u;
-        }
-        __syncthreads();
     };
 
+    float A[NR][NC];  // S (forward), Gs (reverse)
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int k = 0; k < NC; ++k) A[r][k] = 0.f;
+    int par = 0;
+
     // ---- forward sweep: checkpoints, S_t, dq_t = S_t^T do_t
-    for (int e = tid; e < D * LD; e += NT) S[e] = 0.f;
     for (int tb = 0; tb < ntile; ++tb) {
         const int t0 = tb * TT, n = min(TT, L - t0);
         __syncthreads();
         tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
-        for (int e = tid; e < D * D; e += NT) cks[(size_t)tb * D * D + e] = S[(e / D) * LD + e % D];
         __syncthreads();
-        for (int i = 0; i < n; ++i) {
-            step(i);
-            float g = 0.f;
-#pragma unroll 8
-            for (int s = 0; s < SEG; ++s) {
-                const int c = rp * SEG + s;
-                g = fmaf(S[c * LD + rj], tl.tdo[i * D + c], g);
-            }
+        store_img(cks + (size_t)tb * D * D, A);
+        for (int i = 0; i < n; ++i, par ^= 1) {
+            step(A, i);
+            float dj[NR], gcol[NC];
 #pragma unroll
-            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) g += __shfl_xor_sync(0xffffffffu, g, o2);
-            if (rp == 0) dq[(size_t)(t0 + i) * D + rj] = g;
+            for (int r = 0; r < NR; ++r) dj[r] = tl.tdo[i * D + j0 + r];
+#pragma unroll
+            for (int k = 0; k < NC; ++k) {
+                float g = 0.f;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) g = fmaf(A[r][k], dj[r], g);
+                gcol[k] = g;
+            }
+            float *rb = red + par * MW * NW * D;
+            put_cols(gcol, rb);
+            __syncthreads();
+            if (tid < D) {
+                float g = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < NW; ++ww) g += rb[ww * D + tid];
+                dq[(size_t)(t0 + i) * D + tid] = g;
+            }
         }
     }
-    // ---- reverse sweep, tile by tile; Gs = dL/dS in S between tiles
-    __syncthreads();
-    for (int e = tid; e < D * D; e += NT) {
-        const int j = e / D, c = e % D;
-        S[j * LD + c] = p.dstate ? p.dstate[(bh * D + j) * D + c] : 0.f;  // dL/dS_L
-    }
-    float acc_dy[MW], acc_dx[MW];  // samples t - m: row rj of dy, column rj of dx
+    // ---- reverse sweep, tile by tile
 #pragma unroll
-    for (int m = 0; m < MW; ++m) acc_dy[m] = acc_dx[m] = 0.f;
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int k = 0; k < NC; ++k) A[r][k] = dst ? dst[(size_t)(j0 + r) * D + c0 + k] : 0.f;  // dL/dS_L
+    float acc_dy[MW][NR];  // this lane's rows of dy of samples t - m
+    float acc_dx[MW];      // column tid of dx of samples t - m (threads tid < D)
+#pragma unroll
+    for (int m = 0; m < MW; ++m) {
+        acc_dx[m] = 0.f;
+#pragma unroll
+        for (int r = 0; r < NR; ++r) acc_dy[m][r] = 0.f;
+    }
     for (int tb = ntile - 1; tb >= 0; --tb) {
         const int t0 = tb * TT, n = min(TT, L - t0);
-        float *ckt = cks + (size_t)tb * D * D;
         __syncthreads();
         tl.stage(p, q, dout, v, x, et, al, t0, n, nch);
-        // swap Gs and the tile's checkpoint (each element by one thread)
-        for (int e = tid; e < D * D; e += NT) {
-            const int j = e / D, c = e % D;
-            const float sv = ckt[e];
-            ckt[e] = S[j * LD + c];
-            S[j * LD + c] = sv;
-        }
         __syncthreads();
-        // recompute the tile: tss[i] = S before token t0 + i
-        for (int i = 0; i < n; ++i) {
-            for (int e = tid; e < D * D; e += NT) tss[(size_t)i * D * D + e] = S[(e / D) * LD + e % D];
-            step(i);
-        }
-        for (int e = tid; e < D * D; e += NT) S[(e / D) * LD + e % D] = ckt[e];
-        __syncthreads();
-        for (int i = n - 1; i >= 0; --i) {
-            const int t = t0 + i;
-            const float *Sp = tss + (size_t)i * D * D;
-            for (int e = tid; e < D * D; e += NT) {
-                const int j = e / D, c = e % D;
-                S[j * LD + c] += tl.tdo[i * D + j] * tl.tq[i * D + c];
+        {   // the tile's states S_{t-1}, recomputed from its checkpoint
+            float P[NR][NC];
+            load_img(cks + (size_t)tb * D * D, P);
+            for (int i = 0; i < n; ++i) {
+                store_img(tss + (size_t)i * D * D, P);
+                step(P, i);
             }
-            __syncthreads();
-            float sx[MW], gx[MW], gs = 0.f;  // row rj: (S_{t-1} x_{t-m}), (Gs x_{t-m}), <Gs, S_{t-1}>
+        }
+        for (int i = n - 1; i >= 0; --i, par ^= 1) {
+            const int t = t0 + i;
+            float P[NR][NC];
+            load_img(tss + (size_t)i * D * D, P);
+            float gs[NR], dterm[NR], vd[MW][NR];
+            {
+                float qc[NC];
+                load_cols(tl.tq + i * D, qc);
 #pragma unroll
-            for (int m = 0; m < MW; ++m) sx[m] = gx[m] = 0.f;
-            for (int s = 0; s < SEG; ++s) {
-                const int c = rp * SEG + s;
-                const float sp = Sp[(size_t)rj * D + c], g = S[rj * LD + c];
-                gs = fmaf(g, sp, gs);
+                for (int r = 0; r < NR; ++r) {
+                    const float dj = tl.tdo[i * D + j0 + r];
+                    float g = 0.f;
+#pragma unroll
+                    for (int k = 0; k < NC; ++k) {
+                        A[r][k] = fmaf(dj, qc[k], A[r][k]);
+                        g = fmaf(A[r][k], P[r][k], g);
+                    }
+                    gs[r] = row_sum(g);
+                    dterm[r] = 0.f;
+                }
+            }
+            float *rb = red + par * MW * NW * D;
+#pragma unroll
+            for (int m = 0; m < MW; ++m)
+                if (m < w) {
+                    float xc[NC], dcol[NC], ve[NR];
+                    load_cols(tl.tx + srow(i, m), xc);
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) {
+                        const int j = j0 + r;
+                        float sx = 0.f, gx = 0.f;
+#pragma unroll
+                        for (int k = 0; k < NC; ++k) {
+                            sx = fmaf(P[r][k], xc[k], sx);
+                            gx = fmaf(A[r][k], xc[k], gx);
+                        }
+                        sx = row_sum(sx);
+                        gx = row_sum(gx);
+                        const float eta = tl.te[i * D + j], e = tl.ty[srow(i, m) + j] - sx, d = eta * gx;
+                        acc_dy[m][r] += d;
+                        dterm[r] = fmaf(e, gx, dterm[r]);
+                        ve[r] = eta * e;
+                        vd[m][r] = d;
+                    }
+#pragma unroll
+                    for (int k = 0; k < NC; ++k) {
+                        float s = 0.f;
+#pragma unroll
+                        for (int r = 0; r < NR; ++r) s = fmaf(ve[r], A[r][k], fmaf(-vd[m][r], P[r][k], s));
+                        dcol[k] = s;
+                    }
+                    put_cols(dcol, rb + m * NW * D);
+                }
+            float gsum = 0.f, dsum = 0.f;
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const int j = j0 + r;
+                if (cg == 0) {
+                    dv[(size_t)t * D + j] = acc_dy[0][r];  // sample t: every step that uses it is done
+                    if (nch > 1) {
+                        ga[(size_t)t * D + j] = gs[r];
+                        de[(size_t)t * D + j] = dterm[r];
+                    }
+                }
+                gsum += gs[r];
+                dsum += dterm[r];
+            }
+#pragma unroll
+            for (int m = 0; m < MW - 1; ++m)
+#pragma unroll
+                for (int r = 0; r < NR; ++r) acc_dy[m][r] = acc_dy[m + 1][r];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) acc_dy[MW - 1][r] = 0.f;
+            if (nch == 1) {
+                gsum = warp_rows_sum(gsum);
+                dsum = warp_rows_sum(dsum);
+                if (lane == 0) {
+                    red1[(par * NW + warp) * 2] = gsum;
+                    red1[(par * NW + warp) * 2 + 1] = dsum;
+                }
+            }
+            // Gs <- alpha o Gs - sum_m de_m x_{t-m}^T  (dL/dS_{t-1})
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const float a = tl.ta[i * D + j0 + r];
+#pragma unroll
+                for (int k = 0; k < NC; ++k) A[r][k] *= a;
+            }
+#pragma unroll
+            for (int m = 0; m < MW; ++m)
+                if (m < w) {
+                    float xc[NC];
+                    load_cols(tl.tx + srow(i, m), xc);
+#pragma unroll
+                    for (int r = 0; r < NR; ++r)
+#pragma unroll
+                        for (int k = 0; k < NC; ++k) A[r][k] = fmaf(-vd[m][r], xc[k], A[r][k]);
+                }
+            __syncthreads();
+            if (tid < D) {
 #pragma unroll
                 for (int m = 0; m < MW; ++m)
                     if (m < w) {
-                        const float xv = tl.x(i, m, c);
-                        sx[m] = fmaf(sp, xv, sx[m]);
-                        gx[m] = fmaf(g, xv, gx[m]);
+                        float s = 0.f;
+#pragma unroll
+                        for (int ww = 0; ww < NW; ++ww) s += rb[(m * NW + ww) * D + tid];
+                        acc_dx[m] += s;
                     }
+                dxo[(size_t)t * D + tid] = acc_dx[0];
+#pragma unroll
+                for (int m = 0; m < MW - 1; ++m) acc_dx[m] = acc_dx[m + 1];
+                acc_dx[MW - 1] = 0.f;
             }
-#pragma unroll
-            for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o2);
-            const float eta = tl.te[i * D + rj];
-            float dterm = 0.f;
-#pragma unroll
-            for (int m = 0; m < MW; ++m)
-                if (m < w) {
-#pragma unroll
-                    for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) {
-                        sx[m] += __shfl_xor_sync(0xffffffffu, sx[m], o2);
-                        gx[m] += __shfl_xor_sync(0xffffffffu, gx[m], o2);
-                    }
-                    const float e = tl.y(i, m, rj) - sx[m], d = eta * gx[m];
-                    acc_dy[m] += d;
-                    dterm = fmaf(e, gx[m], dterm);
-                    if (rp == 0) {
-                        ve[m * D + rj] = eta * e;
-                        vde[m * D + rj] = d;
-                    }
-                }
-            if (rp == 0) {
-                if (nch > 1) {
-                    ga[(size_t)t * D + rj] = gs;
-                    de[(size_t)t * D + rj] = dterm;
-                } else {
-                    vsum[rj] = gs;
-                    vsum[D + rj] = dterm;
-                }
-            }
-            __syncthreads();
-            float dxm[MW];  // column rj: sum_j (eta e_m)_j Gs[j][c] - de_{m,j} S_{t-1}[j][c]
-#pragma unroll
-            for (int m = 0; m < MW; ++m) dxm[m] = 0.f;
-            for (int s = 0; s < SEG; ++s) {
-                const int j = rp * SEG + s;
-                const float gc = S[j * LD + rj], sc = Sp[(size_t)j * D + rj];
-#pragma unroll
-                for (int m = 0; m < MW; ++m)
-                    if (m < w) dxm[m] = fmaf(ve[m * D + j], gc, fmaf(-vde[m * D + j], sc, dxm[m]));
-            }
-#pragma unroll
-            for (int m = 0; m < MW; ++m)
-                if (m < w) {
-#pragma unroll
-                    for (int o2 = RPT / 2; o2 > 0; o2 >>= 1) dxm[m] += __shfl_xor_sync(0xffffffffu, dxm[m], o2);
-                    acc_dx[m] += dxm[m];
-                }
-            if (rp == 0) {
-                dv[(size_t)t * D + rj] = acc_dy[0];  // sample t: every step that uses it is done
-                dxo[(size_t)t * D + rj] = acc_dx[0];
-            }
-#pragma unroll
-            for (int m = 0; m < MW - 1; ++m) {
-                acc_dy[m] = acc_dy[m + 1];
-                acc_dx[m] = acc_dx[m + 1];
-            }
-            acc_dy[MW - 1] = acc_dx[MW - 1] = 0.f;
-            if (nch == 1 && tid < 32) {
+            if (nch == 1 && tid == 255) {
                 float a = 0.f, b = 0.f;
-                for (int j = tid; j < D; j += 32) {
-                    a += vsum[j];
-                    b += vsum[D + j];
-                }
-                a = group_sum<32>(a);
-                b = group_sum<32>(b);
-                if (tid == 0) {
-                    ga[t] = a;
-                    de[t] = b;
-                }
-            }
-            __syncthreads();
-            // Gs <- alpha o Gs - sum_m de_m x_{t-m}^T  (dL/dS_{t-1})
-            for (int e = tid; e < D * D; e += NT) {
-                const int j = e / D, c = e % D;
-                float u = 0.f;
 #pragma unroll
-                for (int m = 0; m < MW; ++m)
-                    if (m < w) u = fmaf(vde[m * D + j], tl.x(i, m, c), u);
-                S[j * LD + c] = tl.ta[i * D + j] * S[j * LD + c] - u;
+                for (int ww = 0; ww < NW; ++ww) {
+                    a += red1[(par * NW + ww) * 2];
+                    b += red1[(par * NW + ww) * 2 + 1];
+                }
+                ga[t] = a;
+                de[t] = b;
             }
-            __syncthreads();
         }
     }
 }
@@ -1100,7 +1287,6 @@ __host__ __device__ bool regression(int v) { return v == F1 || v == F2 || v == F
 template <typename T, int D, int MW>
 int launch_sweep_w(const BwdParams &p, const float *xs, const float *etas, const float *alphas, float *dga, float *dgb,
                    float *deta, float *dx, float *ck, float *ts, cudaStream_t s) {
-    constexpr size_t base = (size_t)D * (D + 1) + Tiles<T, D, MW>::floats;
     if (regression(p.variant)) {
         if constexpr (MW == 1) {  // one sample per update: S, Gs and S_{t-1} in registers
             const size_t bytes = (Tiles<T, D, 1>::floats + 2 * 8 * D + 2 * 8 * 2) * sizeof(float);
@@ -1108,11 +1294,11 @@ int launch_sweep_w(const BwdParams &p, const float *xs, const float *etas, const
                                  (int)bytes);
             bwd_sweep_reg_rs_kernel<T, D>
                 <<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
-        } else {
-            const size_t bytes = (base + 2 * MW * D + 2 * D) * sizeof(float);
-            cudaFuncSetAttribute(bwd_sweep_reg_kernel<T, D, MW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        } else {  // a window: the same, with sliding register windows for dy and dx
+            const size_t bytes = (Tiles<T, D, MW>::floats + 2 * MW * 8 * D + 2 * 8 * 2) * sizeof(float);
+            cudaFuncSetAttribute(bwd_sweep_reg_rsw_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)bytes);
-            bwd_sweep_reg_kernel<T, D, MW>
+            bwd_sweep_reg_rsw_kernel<T, D>
                 <<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, deta, dx, ck, ts);
         }
         return 0;
@@ -1122,9 +1308,9 @@ int launch_sweep_w(const BwdParams &p, const float *xs, const float *etas, const
         cudaFuncSetAttribute(bwd_sweep_rs_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         bwd_sweep_rs_kernel<T, D><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
     } else {
-        const size_t bytes = (base + 2 * D) * sizeof(float);
-        cudaFuncSetAttribute(bwd_sweep_kernel<T, D, MW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-        bwd_sweep_kernel<T, D, MW><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
+        const size_t bytes = (Tiles<T, D, MW>::floats + D + 2 * MW * 8 * D + 2 * 8) * sizeof(float);
+        cudaFuncSetAttribute(bwd_sweep_rsw_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        bwd_sweep_rsw_kernel<T, D><<<(unsigned)(p.B * p.H), 256, bytes, s>>>(p, xs, etas, alphas, dga, dgb, deta, dx);
     }
     return 0;
 }
