@@ -214,8 +214,9 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
  * forward sweep keeps S every 32 tokens and the reverse sweep recomputes
  * each 32-token stretch from it.
  * Scratch: (2 L d + L + 5 L c) floats per (b,h), c = 1 or d_v, plus
- * (ceil(L/32) + 32) d^2 for the regression family, stream-ordered from the
- * library's pool (FALCON_ERR_ALLOC if that fails).  Errors as in falcon_fwd.
+ * (ceil(L/32) + 32) d^2 for the regression family (and under 64 floats of
+ * alignment), stream-ordered from the library's pool (FALCON_ERR_ALLOC if
+ * that fails).  Errors as in falcon_fwd.
  */
 int falcon_bwd(falcon_variant variant, falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
                const void *q, const void *k, const void *v, const void *beta, const float *lambda, float eps,
