@@ -34,17 +34,21 @@ def test_algorithmic_bytes_of_the_bench_workload(bench):
 
 
 def test_profiled_traffic_follows_the_sources(bench, monkeypatch, tmp_path):
-    """The committed summaries match the committed sources; a change to a
-    source the capture was built from withdraws the figure."""
-    for key in bench.PROFILED:
-        assert isinstance(bench.profiled_traffic(key), int), key
+    """A summary's traffic figure counts while the captured kernel's sources
+    hash to the value it records, and not after any of them changes."""
     name, files = bench.PROFILED["chunk"]
-    fake = tmp_path / "csrc"
-    fake.mkdir()
+    (tmp_path / "profiles").mkdir()
+    csrc = tmp_path / "csrc"
+    csrc.mkdir()
     for f in files:
-        src = open(os.path.join(bench.CSRC, f)).read()
-        (fake / f).write_text(src + ("\n// edited\n" if f == files[0] else ""))
-    monkeypatch.setattr(bench, "CSRC", str(fake))
+        (csrc / f).write_text(open(os.path.join(bench.CSRC, f)).read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "CSRC", str(csrc))
+    assert bench.profiled_traffic("chunk") is None  # no summary
+    (tmp_path / "profiles" / name).write_text(
+        "source sha256: %s\n\ntraffic per launch: 123456 B\n" % bench.source_hash(files))
+    assert bench.profiled_traffic("chunk") == 123456
+    (csrc / files[-1]).write_text((csrc / files[-1]).read_text() + "\n// edited\n")
     assert bench.profiled_traffic("chunk") is None
 
 
