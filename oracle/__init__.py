@@ -54,11 +54,11 @@ def _load():
         I, D = ctypes.c_int, ctypes.c_double
         lib.oracle_fwd.argtypes = [I, I, I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, I, I, dp, dp, I]
         lib.oracle_fwd.restype = I
-        lib.oracle_decode_step.argtypes = [I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, dp, dp, dp, dp]
+        lib.oracle_decode_step.argtypes = [I, I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, dp, dp, dp, dp]
         lib.oracle_decode_step.restype = I
-        lib.oracle_carry_from_prefill.argtypes = [I, I, dp, dp, I, I, I, I, I, I, dp, dp]
+        lib.oracle_carry_from_prefill.argtypes = [I, I, I, dp, dp, I, I, I, I, I, I, dp, dp]
         lib.oracle_carry_from_prefill.restype = I
-        lib.oracle_fwd_carry.argtypes = [I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, I, dp, dp, dp, dp, dp, I]
+        lib.oracle_fwd_carry.argtypes = [I, I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, I, dp, dp, dp, dp, dp, I]
         lib.oracle_fwd_carry.restype = I
         lib.oracle_bwd.argtypes = [I, I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, I, dp, dp, dp, dp, dp, dp, dp, I]
         lib.oracle_bwd.restype = I
@@ -98,24 +98,26 @@ def fwd(variant, form, q, k, v, beta, lam, eps, window=1, chunk=64,
     return out, fs
 
 
-def decode_step(variant, q, k, v, beta, lam, eps, window, state, x_prev, win, phi="l2"):
-    """One decode step on fp64 arrays; state, x_prev and win are updated in place."""
+def decode_step(variant, q, k, v, beta, lam, eps, window, state, x_prev, win, phi="l2", pairing="prefix"):
+    """One decode step on fp64 arrays; state, x_prev and win are updated in
+    place (x_prev may be None under the same-step pair)."""
     lib = _load()
     q, k, v, beta, lam = map(_f64, (q, k, v, beta, lam))
     for a in (state, x_prev, win):
-        assert a.dtype == np.float64 and a.flags.c_contiguous
+        assert a is None or (a.dtype == np.float64 and a.flags.c_contiguous)
     N, H, dk = q.shape
     dv = v.shape[-1]
     out = np.zeros((N, H, dv))
-    rc = lib.oracle_decode_step(VARIANTS[variant], PHIS[phi], _p(q), _p(k), _p(v), _p(beta),
+    null = ctypes.POINTER(ctypes.c_double)()
+    rc = lib.oracle_decode_step(VARIANTS[variant], PAIRINGS[pairing], PHIS[phi], _p(q), _p(k), _p(v), _p(beta),
                                 _p(lam), float(eps), int(window), N, H, dk, dv,
-                                _p(state), _p(x_prev), _p(win), _p(out))
+                                _p(state), _p(x_prev) if x_prev is not None else null, _p(win), _p(out))
     if rc < 0:
         raise ValueError("oracle_decode_step rejected its arguments (code %d)" % rc)
     return out
 
 
-def carry_from_prefill(variant, k, v, window, phi="l2"):
+def carry_from_prefill(variant, k, v, window, phi="l2", pairing="prefix"):
     """Decode carry (x_prev [B,H,dk], win [B,H,max(Bw-1,0),dk+dv]) after a prefill."""
     lib = _load()
     k, v = _f64(k), _f64(v)
@@ -124,7 +126,7 @@ def carry_from_prefill(variant, k, v, window, phi="l2"):
     w = window if variant in ("F3", "F3A") else 1
     x_prev = np.zeros((B, H, dk))
     win = np.zeros((B, H, max(w - 1, 0), dk + dv))
-    rc = lib.oracle_carry_from_prefill(VARIANTS[variant], PHIS[phi], _p(k), _p(v), int(window),
+    rc = lib.oracle_carry_from_prefill(VARIANTS[variant], PAIRINGS[pairing], PHIS[phi], _p(k), _p(v), int(window),
                                        B, H, L, dk, dv, _p(x_prev), _p(win))
     if rc < 0:
         raise ValueError("oracle_carry_from_prefill rejected its arguments (code %d)" % rc)
@@ -132,11 +134,11 @@ def carry_from_prefill(variant, k, v, window, phi="l2"):
 
 
 def fwd_carry(variant, q, k, v, beta, lam, eps, window=1, S0=None, x_prev=None, win=None, phi="l2",
-              nthreads=0):
+              nthreads=0, pairing="prefix"):
     """Recurrent definition over a segment that continues a sequence: state
     S0 [B,H,dv,dk] and the decode carry x_prev [B,H,dk], win [B,H,Bw-1,dk+dv]
-    (each None = zeros, the start of a sequence).  Prefix pairing.
-    Returns (out [B,H,L,dv], S_L [B,H,dv,dk])."""
+    (each None = zeros, the start of a sequence; x_prev is not read under the
+    same-step pair).  Returns (out [B,H,L,dv], S_L [B,H,dv,dk])."""
     lib = _load()
     q, k, v, beta, lam = map(_f64, (q, k, v, beta, lam))
     B, H, L, dk = q.shape
@@ -148,7 +150,7 @@ def fwd_carry(variant, q, k, v, beta, lam, eps, window=1, S0=None, x_prev=None, 
     ptrs = [_p(a) if a is not None else null for a in carry]
     out = np.zeros((B, H, L, dv))
     fs = np.zeros((B, H, dv, dk))
-    rc = lib.oracle_fwd_carry(VARIANTS[variant], PHIS[phi], _p(q), _p(k), _p(v), _p(beta), _p(lam),
+    rc = lib.oracle_fwd_carry(VARIANTS[variant], PAIRINGS[pairing], PHIS[phi], _p(q), _p(k), _p(v), _p(beta), _p(lam),
                               float(eps), int(window), B, H, L, dk, dv, *ptrs, _p(out), _p(fs), int(nthreads))
     if rc < 0:
         raise ValueError("oracle_fwd_carry rejected its arguments (code %d)" % rc)

@@ -375,10 +375,12 @@ int oracle_fwd(int variant, int form, int pairing, int phi,
  * NULL carries are zeros, which is exactly the start of a sequence (R2: an
  * all-zero sample adds no energy and no gradient).  The definition is the
  * recurrent form above, run over the carried samples followed by the
- * segment's; prefix pairing only.
+ * segment's.  Under the same-step pair ([EXPL 核心方法 1] warning paragraph)
+ * the segment's samples are (phi(k_t), v_t), so x_prev is not read, and the
+ * window carry holds the same-step samples before the segment.
  */
 typedef struct {
-    int variant, phi, B, H, L, dk, dv, w;
+    int variant, pairing, phi, B, H, L, dk, dv, w;
     double eps;
     const double *q, *k, *v, *beta, *lambda, *S0, *x_prev, *win;
     double *out, *final_state;
@@ -401,7 +403,9 @@ static void carry_unit_run(const carry_job_t *C, int b, int h)
     }
     for (int t = 0; t < L; ++t) {
         double *xt = X + (size_t)(t + P) * dk;
-        if (t == 0) {
+        if (C->pairing == PAIR_SAME_STEP) {
+            apply_phi(C->phi, k + (size_t)t * dk, dk, xt); /* the segment's own key */
+        } else if (t == 0) {
             if (C->x_prev) memcpy(xt, C->x_prev + bh * (size_t)dk, sizeof(double) * dk);
         } else {
             apply_phi(C->phi, k + (size_t)(t - 1) * dk, dk, xt);
@@ -456,15 +460,15 @@ static void *carry_worker(void *arg)
 }
 
 /* Returns the number of threads used (>0) or a negative error. */
-int oracle_fwd_carry(int variant, int phi, const double *q, const double *k, const double *v, const double *beta,
-                     const double *lambda, double eps, int window, int B, int H, int L, int dk, int dv,
-                     const double *S0, const double *x_prev, const double *win,
+int oracle_fwd_carry(int variant, int pairing, int phi, const double *q, const double *k, const double *v,
+                     const double *beta, const double *lambda, double eps, int window, int B, int H, int L, int dk,
+                     int dv, const double *S0, const double *x_prev, const double *win,
                      double *out, double *final_state, int nthreads)
 {
-    if (variant < 0 || variant > 5) return -2;
+    if (variant < 0 || variant > 5 || pairing < 0 || pairing > 1) return -2;
     if (B < 0 || H < 0 || L < 0 || dk <= 0 || dv <= 0) return -3;
     if (is_window(variant) && window < 1) return -6;
-    carry_job_t C = {variant, phi, B, H, L, dk, dv, is_window(variant) ? window : 1, eps,
+    carry_job_t C = {variant, pairing, phi, B, H, L, dk, dv, is_window(variant) ? window : 1, eps,
                      q, k, v, beta, lambda, S0, x_prev, win, out, final_state};
     if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
     const int units = B * H;
@@ -491,15 +495,19 @@ int oracle_fwd_carry(int variant, int phi, const double *q, const double *k, con
  * token, R2) and, for Falcon-3/3A, the previous Bw-1 samples win[m] =
  * (x, y), oldest first (zeros where the sequence had fewer samples, which
  * contribute nothing: an all-zero x adds no energy and no gradient).
+ * Under the same-step pair ([EXPL 核心方法 1] warning paragraph) the step's
+ * sample is (phi(k_t), v_t) and x_prev is not read (it may be NULL; when
+ * given it is still set to phi(k_t)).
  * Layouts: state [N,H,dv,dk]; x_prev [N,H,dk]; win [N,H,Bw-1,dk+dv];
  * q,k [N,H,dk]; v,out [N,H,dv]; beta [N,H] or [N,H,dv].
  */
-int oracle_decode_step(int variant, int phi, const double *q, const double *k, const double *v,
+int oracle_decode_step(int variant, int pairing, int phi, const double *q, const double *k, const double *v,
                        const double *beta, const double *lambda, double eps, int window,
                        int N, int H, int dk, int dv, double *state, double *x_prev, double *win,
                        double *out)
 {
-    if (variant < 0 || variant > 5) return -2;
+    if (variant < 0 || variant > 5 || pairing < 0 || pairing > 1) return -2;
+    if (pairing == PAIR_PREFIX && !x_prev) return -1;
     const int w = is_window(variant) ? window : 1;
     if (w < 1) return -6;
     const int nch = is_per_channel(variant) ? dv : 1;
@@ -515,7 +523,10 @@ int oracle_decode_step(int variant, int phi, const double *q, const double *k, c
             memcpy(xs + (size_t)m * dk, slot, sizeof(double) * dk);
             memcpy(ys + (size_t)m * dv, slot + dk, sizeof(double) * dv);
         }
-        memcpy(xs + (size_t)(w - 1) * dk, x_prev + (size_t)nh * dk, sizeof(double) * dk);
+        if (pairing == PAIR_SAME_STEP)
+            apply_phi(phi, k + (size_t)nh * dk, dk, xs + (size_t)(w - 1) * dk);
+        else
+            memcpy(xs + (size_t)(w - 1) * dk, x_prev + (size_t)nh * dk, sizeof(double) * dk);
         memcpy(ys + (size_t)(w - 1) * dv, v + (size_t)nh * dv, sizeof(double) * dv);
         double n = 0.0;
         for (int m = 0; m < w; ++m) n += dot(xs + (size_t)m * dk, xs + (size_t)m * dk, dk);
@@ -546,22 +557,24 @@ int oracle_decode_step(int variant, int phi, const double *q, const double *k, c
             memcpy(slot, xs + (size_t)(w - 1) * dk, sizeof(double) * dk);
             memcpy(slot + dk, ys + (size_t)(w - 1) * dv, sizeof(double) * dv);
         }
-        apply_phi(phi, k + (size_t)nh * dk, dk, x_prev + (size_t)nh * dk);
+        if (x_prev) apply_phi(phi, k + (size_t)nh * dk, dk, x_prev + (size_t)nh * dk);
     }
     free(xs); free(ys); free(res);
     return 0;
 }
 
 /*
- * Decode carry after a prefill of L tokens (prefix pair): x_prev = phi(k_L)
- * and the window holds the samples (x_i, y_i) for i = L-Bw+2..L, oldest
- * first, zeros for i < 1.
+ * Decode carry after a prefill of L tokens: x_prev = phi(k_L) and the window
+ * holds the samples (x_i, y_i) for i = L-Bw+2..L, oldest first, zeros for
+ * i < 1; x_i = phi(k_{i-1}) under the prefix pair, phi(k_i) under the
+ * same-step pair.
  */
-int oracle_carry_from_prefill(int variant, int phi, const double *k, const double *v, int window,
+int oracle_carry_from_prefill(int variant, int pairing, int phi, const double *k, const double *v, int window,
                               int B, int H, int L, int dk, int dv, double *x_prev, double *win)
 {
     const int w = is_window(variant) ? window : 1;
     if (w < 1) return -6;
+    if (pairing < 0 || pairing > 1) return -2;
     for (int bh = 0; bh < B * H; ++bh) {
         const double *kb = k + (size_t)bh * L * dk;
         const double *vb = v + (size_t)bh * L * dv;
@@ -572,7 +585,8 @@ int oracle_carry_from_prefill(int variant, int phi, const double *k, const doubl
             const int i = L - (w - 1) + m; /* 0-based sample index */
             memset(slot, 0, sizeof(double) * (dk + dv));
             if (i < 0) continue;
-            if (i >= 1) apply_phi(phi, kb + (size_t)(i - 1) * dk, dk, slot);
+            if (pairing == PAIR_SAME_STEP) apply_phi(phi, kb + (size_t)i * dk, dk, slot);
+            else if (i >= 1) apply_phi(phi, kb + (size_t)(i - 1) * dk, dk, slot);
             memcpy(slot + dk, vb + (size_t)i * dv, sizeof(double) * dv);
         }
     }

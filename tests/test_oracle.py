@@ -336,40 +336,48 @@ def test_window_one_and_uniform_channels_reduce_to_falcon1(oracle_mod):
 
 # ---------------------------------------------------------------- decode
 
+@pytest.mark.parametrize("pairing", ["prefix", "same_step"])
 @pytest.mark.parametrize("variant", VARIANTS)
-def test_decode_chain_equals_prefill(oracle_mod, variant):
+def test_decode_chain_equals_prefill(oracle_mod, variant, pairing):
     """prefill(L0) -> carry -> n decode steps == prefill(L0 + n): the fixed-size
     state plus the carry is the whole memory ([SUMM] 计算形式与数值稳定: the
-    recurrent form for autoregressive inference)."""
+    recurrent form for autoregressive inference), under either pairing (the
+    same-step pair of [EXPL] 核心方法 1, warning paragraph, takes phi(k_t) as
+    the step's own sample; the full run's samples come from the forward's
+    pairing rule, written independently of the decode step)."""
     L0, n, dk, dv = 9, 7, 6, 4
     w = 3 if variant in ("F3", "F3A") else 1
     q, k, v, beta, lam = rnd(43, 2, 3, L0 + n, dk, dv, variant)
-    o_full, S_full = oracle_mod.fwd(variant, "recurrent", q, k, v, beta, lam, 1e-6, window=w)
+    o_full, S_full = oracle_mod.fwd(variant, "recurrent", q, k, v, beta, lam, 1e-6, window=w, pairing=pairing)
     _, S0 = oracle_mod.fwd(variant, "recurrent", q[:, :, :L0], k[:, :, :L0], v[:, :, :L0],
-                           beta[:, :, :L0], lam, 1e-6, window=w)
-    x_prev, win = oracle_mod.carry_from_prefill(variant, k[:, :, :L0], v[:, :, :L0], w)
+                           beta[:, :, :L0], lam, 1e-6, window=w, pairing=pairing)
+    x_prev, win = oracle_mod.carry_from_prefill(variant, k[:, :, :L0], v[:, :, :L0], w, pairing=pairing)
+    if pairing == "same_step":
+        x_prev = None  # not read by the same-step step
     state = np.ascontiguousarray(S0)
     for t in range(L0, L0 + n):
         o = oracle_mod.decode_step(variant, q[:, :, t], k[:, :, t], v[:, :, t], beta[:, :, t],
-                                   lam, 1e-6, w, state, x_prev, win)
+                                   lam, 1e-6, w, state, x_prev, win, pairing=pairing)
         np.testing.assert_allclose(o, o_full[:, :, t], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(state, S_full, rtol=1e-10, atol=1e-12)
 
 
+@pytest.mark.parametrize("pairing", ["prefix", "same_step"])
 @pytest.mark.parametrize("variant", VARIANTS)
-def test_decode_from_zero_carry(oracle_mod, variant):
+def test_decode_from_zero_carry(oracle_mod, variant, pairing):
     """Decode from S=0 and an all-zero carry reproduces the sequence from its
-    first token (x_1 = 0: the first step writes nothing)."""
+    first token (prefix pair: x_1 = 0, the first step writes nothing; the
+    same-step pair writes with phi(k_1) from the first step on)."""
     L, dk, dv = 8, 4, 3
     w = 3 if variant in ("F3", "F3A") else 1
     q, k, v, beta, lam = rnd(47, 1, 2, L, dk, dv, variant)
-    o_full, S_full = oracle_mod.fwd(variant, "recurrent", q, k, v, beta, lam, 1e-6, window=w)
+    o_full, S_full = oracle_mod.fwd(variant, "recurrent", q, k, v, beta, lam, 1e-6, window=w, pairing=pairing)
     state = np.zeros((1, 2, dv, dk))
     x_prev = np.zeros((1, 2, dk))
     win = np.zeros((1, 2, max(w - 1, 0), dk + dv))
     for t in range(L):
         o = oracle_mod.decode_step(variant, q[:, :, t], k[:, :, t], v[:, :, t], beta[:, :, t],
-                                   lam, 1e-6, w, state, x_prev, win)
+                                   lam, 1e-6, w, state, x_prev, win, pairing=pairing)
         np.testing.assert_allclose(o, o_full[:, :, t], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(state, S_full, rtol=1e-10, atol=1e-12)
 
@@ -435,22 +443,26 @@ def test_carry_of_zeros_is_a_fresh_sequence(oracle_mod, variant):
     np.testing.assert_allclose(S1, S0_, rtol=1e-12, atol=1e-13)
 
 
+@pytest.mark.parametrize("pairing", ["prefix", "same_step"])
 @pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("split", [1, 17, 40])
-def test_continuation_equals_one_run(oracle_mod, variant, split):
+def test_continuation_equals_one_run(oracle_mod, variant, split, pairing):
     """Running a sequence in two segments -- the second one entered with the
     first one's final state and decode carry -- equals one run over the whole
-    sequence (chunk form for the whole run, recurrent for the segments)."""
+    sequence (chunk form for the whole run, recurrent for the segments),
+    under either pairing."""
     L, dk, dv = 57, 8, 4
     q, k, v, beta, lam = rnd(24, 2, 3, L, dk, dv, variant)
     w = 3 if variant in ("F3", "F3A") else 1
-    o_all, S_all = oracle_mod.fwd(variant, "chunk", q, k, v, beta, lam, 1e-6, window=w, chunk=16)
+    o_all, S_all = oracle_mod.fwd(variant, "chunk", q, k, v, beta, lam, 1e-6, window=w, chunk=16, pairing=pairing)
     a = slice(0, split)
     b_ = slice(split, L)
     o1, S1 = oracle_mod.fwd(variant, "recurrent", q[:, :, a], k[:, :, a], v[:, :, a], beta[:, :, a], lam,
-                            1e-6, window=w)
-    xp, win = oracle_mod.carry_from_prefill(variant, k[:, :, a], v[:, :, a], w)
+                            1e-6, window=w, pairing=pairing)
+    xp, win = oracle_mod.carry_from_prefill(variant, k[:, :, a], v[:, :, a], w, pairing=pairing)
+    if pairing == "same_step":
+        xp = None  # the segment's first sample is its own phi(k)
     o2, S2 = oracle_mod.fwd_carry(variant, q[:, :, b_], k[:, :, b_], v[:, :, b_], beta[:, :, b_], lam, 1e-6,
-                                  window=w, S0=S1, x_prev=xp, win=win)
+                                  window=w, S0=S1, x_prev=xp, win=win, pairing=pairing)
     np.testing.assert_allclose(np.concatenate([o1, o2], 2), o_all, rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(S2, S_all, rtol=1e-9, atol=1e-11)
