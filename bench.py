@@ -325,6 +325,9 @@ def run_ours(args):
         flush.zero_()
         step()
     barrier(world)
+    # blocks that gave up on a bounded wait leave incomplete outputs while the
+    # call returns OK: the counter must not move over the measured steps
+    timeouts_before = F.wait_timeouts()
     per_var = {var: [] for var in w["variants"]}
     step_ms = []
     with Clocks(local) as clk:
@@ -374,6 +377,12 @@ def run_ours(args):
             "algorithmic_bytes_per_launch": ab, "launch_ms": f1_ms}
 
     decode = measure_decode(F, gen, stream, flush, hbm, args) if not args.no_decode else None
+    timeouts_delta = int(max_over_ranks(float(F.wait_timeouts() - timeouts_before), world))
+    if timeouts_delta != 0:
+        print(json.dumps({"metric": METRIC, "error": "%d tensor-core thread blocks gave up on a bounded wait "
+                          "during the measured steps: outputs incomplete, no value reported" % timeouts_delta}),
+              flush=True)
+        sys.exit(3)
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -382,9 +391,17 @@ def run_ours(args):
             "per_variant_ms": {var: statistics.mean(per_var[var]) for var in w["variants"]},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             # every falcon_fwd of this shape is two kernels: chunk_local_kernel + chunk_chain_kernel
-            "gpu_launches": 2 * len(w["variants"]) * args.steps, "clocks": clk.summary()}
+            "gpu_launches": 2 * len(w["variants"]) * args.steps, "clocks": clk.summary(),
+            "wait_timeouts_delta": timeouts_delta}
     if decode is not None:
         line["decode"] = decode
+        # the window path (Falcon-3, window 4) and d = 64 decode, same batch and heads
+        line["decode_more"] = [measure_decode(F, gen, stream, flush, hbm, args, variant="F3", window=4),
+                               measure_decode(F, gen, stream, flush, hbm, args, variant="F1", dk=64)]
+    if not args.no_extras:
+        # the chunk-length sweep and the backward on the same workload (extra keys, not the headline)
+        line["chunk_sweep"] = chunk_sweep_rows(F, gen, flush, args.steps)
+        line["backward"] = backward_rows(F, gen, flush, args.steps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, threads, units, used = cpu_oracle_sample(budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -398,27 +415,33 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def measure_decode(F, gen, stream, flush, hbm, args, profile=False):
-    """Decode row: one falcon_decode_step per step for N sequences (Falcon-2A,
-    N=64, H=16, 128x128 fp32 state per head, 64 MiB of state).  Steps rotate
-    over four independent sets of states and carries (256 MiB in all, twice
-    L2), so no step finds its state in L2; the dirty lines a step leaves are
-    written back during later steps, as in steady-state serving."""
+def measure_decode(F, gen, stream, flush, hbm, args, profile=False, variant=None, dk=None, window=1):
+    """Decode row: one falcon_decode_step per step for N sequences (by
+    default Falcon-2A, N=64, H=16, 128x128 fp32 state per head, 64 MiB of
+    state).  Steps rotate over four independent sets of states and carries
+    (256 MiB in all at d = 128, twice L2), so no step finds its state in L2;
+    the dirty lines a step leaves are written back during later steps, as in
+    steady-state serving."""
     import torch
     dd = DECODE
-    N, H, dk, dv = dd["N"], dd["H"], dd["dk"], dd["dv"]
-    pool, sets = 16, 4
-    d = gen.draw_decode(dd["variant"], N, H, dk, dv, pool, seed=dd["seed"], lam=dd["lam"])
+    variant = variant or dd["variant"]
+    N, H = dd["N"], dd["H"]
+    dk = dv = dk or dd["dk"]
+    pool = 16
+    sets = 4 if dk == 128 else 16  # at least twice L2 of states in rotation
+    d = gen.draw_decode(variant, N, H, dk, dv, pool, seed=dd["seed"], lam=dd["lam"])
     q, k, v, beta = (d[n].cuda() for n in ("q", "k", "v", "beta"))
     lam = d["lam"].cuda()
     state = [torch.zeros((N, H, dv, dk), dtype=torch.float32, device="cuda") for _ in range(sets)]
     x_prev = [torch.zeros((N, H, dk), dtype=torch.float32, device="cuda") for _ in range(sets)]
+    win = [torch.zeros((N, H, window - 1, dk + dv), dtype=torch.float32, device="cuda") if window > 1 else None
+           for _ in range(sets)]
     out = torch.empty((N, H, dv), dtype=torch.bfloat16, device="cuda")
     steps = max(args.steps, 20)
 
     def one(i):
-        F.decode_step(dd["variant"], q[i % pool], k[i % pool], v[i % pool], beta[i % pool], lam, d["eps"], 1,
-                      state[i % sets], x_prev[i % sets], out=out, stream=stream)
+        F.decode_step(variant, q[i % pool], k[i % pool], v[i % pool], beta[i % pool], lam, d["eps"], window,
+                      state[i % sets], x_prev[i % sets], win[i % sets], out=out, stream=stream)
 
     if profile:  # decode steps only, for profilers
         for i in range(args.warmup + args.steps):
@@ -437,13 +460,96 @@ def measure_decode(F, gen, stream, flush, hbm, args, profile=False):
         torch.cuda.synchronize()
         ms.append(e0.elapsed_time(e1))
     t = statistics.mean(ms)
-    ab = algorithmic_bytes_decode(N, H, dk, dv, per_channel=True)
+    per_channel = variant in ("F2", "F2A")
+    ab = algorithmic_bytes_decode(N, H, dk, dv, per_channel=per_channel)
+    if window > 1:  # the window carry is read and written too
+        ab += N * H * (window - 1) * (dk + dv) * 4 * 2
     gbs = ab / (t / 1e3) / 1e9
-    return {"workload": "falcon2A-decode-bf16-N64xH16-state128x128-fp32", "us_per_step": t * 1e3,
-            "tokens_per_s": N / (t / 1e3), "steps": steps,
-            "l2": "4 rotating sets of states and carries (256 MiB, 2x L2); no flush",
+    kernel = "decode1_kernel" if window == 1 else "decode_kernel"
+    return {"workload": "%s-decode-bf16-N%dxH%d-state%dx%d-fp32%s" % (
+                variant.replace("F", "falcon"), N, H, dv, dk, "-window%d" % window if window > 1 else ""),
+            "kernel": kernel, "us_per_step": t * 1e3, "tokens_per_s": N / (t / 1e3), "steps": steps,
+            "l2": "%d rotating sets of states and carries (%d MiB, over 2x L2); no flush"
+                  % (sets, sets * N * H * dv * dk * 4 >> 20),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                         "algorithmic_bytes_per_launch": ab, "traffic": profiled_traffic("decode")}}
+                         "algorithmic_bytes_per_launch": ab,
+                         "traffic": profiled_traffic("decode") if (variant, dk, window) == (dd["variant"], 128, 1)
+                         else None}}
+
+
+def time_call(fn, flush, steps, stream=None):
+    """Median CUDA-event time (ms) of fn() over `steps` calls (3..20), L2
+    flushed and a GPU head start queued before each, after one warm-up call."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(max(3, min(steps, 20))):
+        flush.zero_()
+        torch.cuda._sleep(HEAD_START_CYCLES)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    return statistics.median(ms)
+
+
+SWEEP_KERNELS = {16: "seq_chunk_kernel<16>", 32: "seq_chunk_kernel<32>", 64: "chunk_local_kernel + chunk_chain_kernel",
+                 128: "seq_chunk_kernel<128>"}
+
+
+def chunk_sweep_rows(F, gen, flush, steps):
+    """The chunk-parallel forward of workload 2 (Falcon-1 and Falcon-1A,
+    8x12x2048x64 bf16) at chunk 16, 32, 64 and 128 under the prefix pair and
+    at 64 under the same-step pair; every point on the tensor cores."""
+    import torch
+    w = gen.WORKLOADS[2]
+    rows = []
+    for var in w["variants"]:
+        d = gen.workload_inputs(2, var)
+        a = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
+        out = torch.empty((w["B"], w["H"], w["L"], w["dv"]), dtype=torch.bfloat16, device="cuda")
+        S = torch.empty((w["B"], w["H"], w["dv"], w["dk"]), dtype=torch.float32, device="cuda")
+        for chunk, pairing in ((16, "prefix"), (32, "prefix"), (64, "prefix"), (128, "prefix"), (64, "same_step")):
+            need = F.fwd_workspace_size(var, "chunk", torch.bfloat16, w["B"], w["H"], w["L"], w["dk"], w["dv"],
+                                        chunk=chunk, pairing=pairing)
+            ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+            t = time_call(lambda: F.fwd(var, "chunk", *a, d["eps"], chunk=chunk, pairing=pairing, out=out,
+                                        final_state=S, workspace=ws), flush, steps)
+            rows.append({"variant": var, "chunk": chunk, "pairing": pairing, "ms": t,
+                         "tokens_per_s": w["B"] * w["L"] / (t / 1e3), "kernels": SWEEP_KERNELS[chunk],
+                         "workspace_bytes": need})
+    return rows
+
+
+def backward_rows(F, gen, flush, steps, variants=("F1", "F1A"), forms=("chunk", "recurrent")):
+    """falcon_bwd_ex on workload 2 (8x12x2048x64 bf16): the chunk-parallel
+    backward and the recurrent one, each against the algorithmic bytes
+    (q, k, v, beta, dout read in bf16; dq, dk, dv, dbeta written in fp32)."""
+    import numpy as np
+    import torch
+    w = gen.WORKLOADS[2]
+    B, H, L, dk, dv = w["B"], w["H"], w["L"], w["dk"], w["dv"]
+    hbm, _, src = peaks()
+    rng = np.random.default_rng(20260102)
+    do = torch.from_numpy(rng.standard_normal((B, H, L, dv)).astype(np.float32)).to(torch.bfloat16).cuda()
+    ds = torch.from_numpy(rng.standard_normal((B, H, dv, dk)).astype(np.float32)).cuda()
+    tok = B * H * L
+    ab = tok * (dk + dk + dv + 1 + dv) * 2 + tok * (dk + dk + dv + 1) * 4 + B * H * dv * dk * 4
+    out = {}
+    for var in variants:
+        d = gen.workload_inputs(2, var)
+        a = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
+        for form in forms:
+            t = time_call(lambda: F.bwd(var, *a, d["eps"], do, ds, form=form), flush, steps)
+            gbs = ab / (t / 1e3) / 1e9
+            out["%s_%s" % (var, form)] = {"ms": t, "tokens_per_s": B * L / (t / 1e3),
+                                          "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                                       "frac": gbs / hbm, "peak_source": src,
+                                                       "algorithmic_bytes_per_launch": ab}}
+    return out
 
 
 def run_workloads(args):
@@ -498,42 +604,15 @@ def run_workloads(args):
 
 
 def run_chunk_sweep(args):
-    """--chunk-sweep: the chunk-parallel forward of workload 2 (Falcon-1 and
-    Falcon-1A, 8x12x2048x64 bf16) at chunk 16, 32 and 64 under the prefix
-    pair, and at 64 under the same-step pair; CUDA events around one
-    falcon_fwd after a warm-up call, L2 flushed, median of --steps calls.
-    One JSON line each with the kernels that ran and the stream-ordered
-    workspace the call draws.  Not the contract line."""
+    """--chunk-sweep: chunk_sweep_rows as one JSON line each.  Not the contract line."""
     import torch
     import linear_attention_sequence_falcon_b200 as F
     from linear_attention_sequence_falcon_b200 import build, inputs as gen
     build.build()
     F.load()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-    w = gen.WORKLOADS[2]
-    units = w["B"] * w["H"] * ((w["L"] + 63) // 64)
-    for var in w["variants"]:
-        d = gen.workload_inputs(2, var)
-        args_ = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
-        for chunk, pairing in ((16, "prefix"), (32, "prefix"), (64, "prefix"), (64, "same_step")):
-            out, S = F.fwd(var, "chunk", *args_, d["eps"], chunk=chunk, pairing=pairing)
-            torch.cuda.synchronize()
-            ms = []
-            for _ in range(max(3, min(args.steps, 20))):
-                flush.zero_()
-                torch.cuda._sleep(HEAD_START_CYCLES)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                F.fwd(var, "chunk", *args_, d["eps"], chunk=chunk, pairing=pairing, out=out, final_state=S)
-                e1.record()
-                torch.cuda.synchronize()
-                ms.append(e0.elapsed_time(e1))
-            t = statistics.median(ms)
-            tc = chunk == 64
-            print(json.dumps({"sweep": "chunk", "workload": w["name"], "variant": var, "chunk": chunk,
-                              "pairing": pairing, "ms": t, "tokens_per_s": w["B"] * w["L"] / (t / 1e3),
-                              "kernels": "chunk_local_kernel + chunk_chain_kernel" if tc else "span_chunk_kernel",
-                              "workspace_bytes": units * 32 * 1024 + units * 4 if tc else 0}), flush=True)
+    for row in chunk_sweep_rows(F, gen, flush, args.steps):
+        print(json.dumps(dict(sweep="chunk", workload=gen.WORKLOADS[2]["name"], **row)), flush=True)
 
 
 def run_backward(args):
@@ -638,6 +717,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="leave out the chunk sweep and backward keys")
     ap.add_argument("--profile-decode", action="store_true",
                     help="run only warmup+steps decode steps (no flush or JSON), for ncu")
     ap.add_argument("--workloads", action="store_true",

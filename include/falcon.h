@@ -25,6 +25,15 @@
  *  - All tensor arguments are DEVICE pointers (HOST pointers for
  *    falcon_fwd_host) to contiguous row-major arrays owned by the caller;
  *    the library never frees or retains them.
+ *  - Memory: the *_ws entry points run in a workspace the caller allocates
+ *    (its size from the matching *_workspace_size query, 256-byte aligned)
+ *    and allocate nothing.  The other entry points that need a workspace
+ *    draw it stream-ordered (cudaMallocAsync) from the device's current
+ *    memory pool and free it on the same stream; the library keeps no pool
+ *    of its own, so what stays mapped between calls is the pool owner's
+ *    choice (its release threshold).  Library-owned device memory is limited
+ *    to a few diagnostic counters and the fixed array of
+ *    falcon_fwd_masked_noalloc.
  *  - Calls only enqueue work on `stream` (0 = legacy default stream) and never
  *    synchronise.  A non-zero return means nothing was enqueued, except
  *    FALCON_ERR_LAUNCH, which reports cudaGetLastError() after a launch.
@@ -38,6 +47,7 @@
 #define FALCON_H
 
 #include <cuda_runtime_api.h>
+#include <stddef.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -78,8 +88,10 @@ enum {
     FALCON_ERR_LAUNCH = -7,      /* a kernel launch failed (cudaGetLastError)       */
     FALCON_ERR_ALLOC = -8,       /* stream-ordered scratch allocation failed        */
     FALCON_ERR_UNSUPPORTED = -9, /* combination not supported (e.g. pairing+decode) */
-    FALCON_ERR_SCRATCH = -10     /* problem needs more than the fixed scratch of
+    FALCON_ERR_SCRATCH = -10,    /* problem needs more than the fixed scratch of
                                     falcon_fwd_masked_noalloc                      */
+    FALCON_ERR_WORKSPACE = -11   /* the caller's workspace is NULL, smaller than its
+                                    size query or not 256-byte aligned              */
 };
 
 /*
@@ -95,13 +107,14 @@ enum {
  *   out      [B,H,L,d_v] dtype     o_t = S_t q_t (written)
  *   final_state [B,H,d_v,d_k] fp32 S_L (written), may be NULL
  * S_0 = 0.  L may be 0 (out untouched, final_state zeroed) and need not be a
- * multiple of `chunk`.  Two paths draw stream-ordered scratch on `stream`
- * from a memory pool the library owns (one per device, kept mapped between
- * calls; see falcon_scratch_trim) and return FALCON_ERR_ALLOC if that fails:
- * FALCON_MASKED (about B*H*L*(window*d_v+2*d_v) floats) and the bf16
- * tensor-core chunk path, Falcon-1/1A with d_k = d_v = 64 and chunk 64
+ * multiple of `chunk`.  Three paths need a workspace, drawn stream-ordered
+ * on `stream` from the device's current memory pool (FALCON_ERR_ALLOC if
+ * that fails; falcon_fwd_ws takes it from the caller instead):
+ * FALCON_MASKED (about B*H*L*(window*d_v+2*d_v) floats), the bf16
+ * tensor-core chunk path of Falcon-1/1A with d_k = d_v = 64 and chunk 64
  * (32 KiB + 4 bytes per (b, h, chunk): the chunk-local results that the
- * second of its two kernels chains across chunks).
+ * second of its two kernels chains across chunks) and that of Falcon-2A
+ * with d_k = d_v = 128 and chunk 64 (96.5 KiB per (b, h, chunk)).
  */
 int falcon_fwd(falcon_variant variant, falcon_form form, falcon_dtype dtype,
                const void *q, const void *k, const void *v, const void *beta,
@@ -116,6 +129,39 @@ int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype,
                   const float *lambda, float eps, int window,
                   int B, int H, int L, int d_k, int d_v, int chunk,
                   void *out, float *final_state, cudaStream_t stream);
+
+/*
+ * falcon_fwd_workspace_size -- bytes of device workspace a forward with
+ * these arguments needs (0 when its kernels need none).  A host-only query:
+ * nothing is enqueued.  Argument errors as in falcon_fwd_ex; *bytes is 0
+ * then.
+ */
+int falcon_fwd_workspace_size(falcon_variant variant, falcon_form form, falcon_dtype dtype,
+                              falcon_pairing pairing, falcon_phi phi, int window,
+                              int B, int H, int L, int d_k, int d_v, int chunk, size_t *bytes);
+
+/*
+ * falcon_fwd_ws -- the forward (every form, pairing and feature map, with or
+ * without the carry of falcon_fwd_carry_ex) in a workspace the caller owns:
+ * the library allocates nothing.
+ *   workspace        device memory, 256-byte aligned, at least the bytes
+ *                    falcon_fwd_workspace_size gives for the same arguments
+ *                    (may be NULL when that is 0); its contents on entry do
+ *                    not matter, and it may be reused once `stream` has
+ *                    passed the call's work
+ *   workspace_bytes  its size; too small, misaligned or NULL when needed:
+ *                    FALCON_ERR_WORKSPACE, nothing enqueued
+ *   initial_state, x_prev, win   the carry of falcon_fwd_carry_ex, or NULL
+ * Every other argument, and the results, as in falcon_fwd_carry_ex.
+ */
+int falcon_fwd_ws(falcon_variant variant, falcon_form form, falcon_dtype dtype,
+                  falcon_pairing pairing, falcon_phi phi,
+                  const void *q, const void *k, const void *v, const void *beta,
+                  const float *lambda, float eps, int window,
+                  int B, int H, int L, int d_k, int d_v, int chunk,
+                  const float *initial_state, const float *x_prev, const float *win,
+                  void *out, float *final_state, void *workspace, size_t workspace_bytes,
+                  cudaStream_t stream);
 
 /*
  * falcon_fwd_host -- falcon_fwd_ex for inputs and outputs in HOST memory,
@@ -143,9 +189,10 @@ int falcon_fwd_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype,
  * valid, and the inputs unchanged, until `stream` has passed the call's work;
  * the outputs are complete then (cudaStreamSynchronize(stream)).  The device
  * buffers (inputs, lambda, outputs and states: about the inputs' size plus
- * n_variants times the outputs') are one stream-ordered block from the
- * library's pool, freed on `stream` at the end of the call's work.  Argument
- * errors return before anything is enqueued.  An error after the first copy
+ * n_variants times the outputs', and the per-slice forward's workspace) are
+ * one stream-ordered block from the device's current memory pool, freed on
+ * `stream` at the end of the call's work (falcon_fwd_host_ws: the caller's
+ * block instead).  Argument errors return before anything is enqueued.  An error after the first copy
  * (FALCON_ERR_LAUNCH, or a status of the per-slice forward) stops further
  * slices; the streams are still joined into `stream` and the block freed,
  * and the outputs are then incomplete.
@@ -156,6 +203,26 @@ int falcon_fwd_host(int n_variants, const falcon_variant *variants, falcon_form 
                     const float *lambda, float eps, int window,
                     int B, int H, int L, int d_k, int d_v, int chunk,
                     void *const *out, float *const *final_state, int slices, cudaStream_t stream);
+
+/*
+ * falcon_fwd_host_workspace_size / falcon_fwd_host_ws -- falcon_fwd_host in
+ * a device workspace the caller owns (256-byte aligned; the library then
+ * allocates nothing).  The size depends on the arguments of the size query,
+ * with_state != 0 when final states are wanted for every variant (a call
+ * that wants fewer needs no more).  Too small, misaligned or NULL:
+ * FALCON_ERR_WORKSPACE, nothing enqueued.  Everything else as falcon_fwd_host.
+ */
+int falcon_fwd_host_workspace_size(int n_variants, const falcon_variant *variants, falcon_form form,
+                                   falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi, int window,
+                                   int B, int H, int L, int d_k, int d_v, int chunk, int with_state, int slices,
+                                   size_t *bytes);
+int falcon_fwd_host_ws(int n_variants, const falcon_variant *variants, falcon_form form, falcon_dtype dtype,
+                       falcon_pairing pairing, falcon_phi phi,
+                       const void *q, const void *k, const void *v, const void *beta,
+                       const float *lambda, float eps, int window,
+                       int B, int H, int L, int d_k, int d_v, int chunk,
+                       void *const *out, float *const *final_state, int slices,
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * falcon_fwd_carry -- falcon_fwd over a segment that continues a sequence:
@@ -187,6 +254,23 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
                      void *out, float *final_state, cudaStream_t stream);
 
 /*
+ * falcon_fwd_carry_ex -- falcon_fwd_carry with the pairing and the feature
+ * map selectable.  Under the same-step pair ([EXPL] 核心方法 1, warning
+ * paragraph) the segment's first sample is (phi(k_1), v_1) of the segment
+ * itself, so x_prev is not read (it may be NULL); `win` holds the window-1
+ * same-step samples before the segment, as falcon_decode_carry_from_prefill_ex
+ * and falcon_decode_step_ex leave them.  phi applies to the segment's keys;
+ * carried samples are used as given.
+ */
+int falcon_fwd_carry_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype,
+                        falcon_pairing pairing, falcon_phi phi,
+                        const void *q, const void *k, const void *v, const void *beta,
+                        const float *lambda, float eps, int window,
+                        int B, int H, int L, int d_k, int d_v, int chunk,
+                        const float *initial_state, const float *x_prev, const float *win,
+                        void *out, float *final_state, cudaStream_t stream);
+
+/*
  * falcon_bwd -- the backward pass: gradients of a scalar loss with respect
  * to q, k, v, beta and lambda, given dL/d(out) and dL/d(final_state), for a
  * forward from S_0 = 0 with the same arguments.  The chunk form trains on the
@@ -213,15 +297,58 @@ int falcon_fwd_carry(falcon_variant variant, falcon_form form, falcon_dtype dtyp
  * The regression family's derivative needs S_{t-1} at every step: the
  * forward sweep keeps S every 32 tokens and the reverse sweep recomputes
  * each 32-token stretch from it.
- * Scratch: (2 L d + L + 5 L c) floats per (b,h), c = 1 or d_v, plus
+ * Workspace: (2 L d + L + 5 L c) floats per (b,h), c = 1 or d_v, plus
  * (ceil(L/32) + 32) d^2 for the regression family (and under 64 floats of
- * alignment), stream-ordered from the library's pool (FALCON_ERR_ALLOC if
- * that fails).  Errors as in falcon_fwd.
+ * alignment), stream-ordered from the device's current memory pool
+ * (FALCON_ERR_ALLOC if that fails).  Errors as in falcon_fwd.
  */
 int falcon_bwd(falcon_variant variant, falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
                const void *q, const void *k, const void *v, const void *beta, const float *lambda, float eps,
                int window, int B, int H, int L, int d_k, int d_v, const void *dout, const float *dstate,
                float *dq, float *dk, float *dv, float *dbeta, float *dlambda, cudaStream_t stream);
+
+/*
+ * falcon_bwd_ex -- falcon_bwd with the form of the forward whose derivative
+ * is taken.
+ *   form  FALCON_RECURRENT: as falcon_bwd (every variant and shape above).
+ *         FALCON_CHUNK: the chunk-parallel backward ([NEWS] 02 (2), the
+ *         paragraph after the variant list: every variant trains in the
+ *         chunk-parallel form), for Falcon-1 and Falcon-1A with bf16 inputs,
+ *         d_k = d_v = 64 and chunk 64 (FALCON_ERR_UNSUPPORTED for other
+ *         variants, dtypes or sizes; FALCON_ERR_CHUNK for another chunk; the
+ *         recurrent form covers them).  The chunk-parallel forward (tensor
+ *         cores) runs first and keeps the state entering every chunk; a
+ *         reverse chain per head then carries dL/dS across chunk boundaries,
+ *         G_c = g_C G_{c+1} - G_{c+1} Phi'_c^T + dO_c^T Qt_c, with the
+ *         forward's per-chunk operators; every chunk's gradients then come at
+ *         once from its inputs, its entering state and G_{c+1} (matrix form,
+ *         TF32 tensor-core products, fp32 accumulation).  The inputs must be
+ *         16-byte aligned (FALCON_ERR_UNSUPPORTED otherwise).
+ *         FALCON_MASKED: FALCON_ERR_UNSUPPORTED.
+ *   chunk 64 for FALCON_CHUNK; ignored otherwise
+ * Every other argument and the results as in falcon_bwd; the workspace is
+ * drawn stream-ordered from the device's current memory pool.
+ */
+int falcon_bwd_ex(falcon_variant variant, falcon_form form, falcon_dtype dtype, falcon_pairing pairing,
+                  falcon_phi phi, const void *q, const void *k, const void *v, const void *beta,
+                  const float *lambda, float eps, int window, int B, int H, int L, int d_k, int d_v, int chunk,
+                  const void *dout, const float *dstate, float *dq, float *dk, float *dv, float *dbeta,
+                  float *dlambda, cudaStream_t stream);
+
+/*
+ * falcon_bwd_workspace_size / falcon_bwd_ws -- falcon_bwd_ex in a workspace
+ * the caller owns (256-byte aligned, at least the queried bytes; the library
+ * then allocates nothing; FALCON_ERR_WORKSPACE when it is too small,
+ * misaligned or NULL).  Everything else as falcon_bwd_ex.
+ */
+int falcon_bwd_workspace_size(falcon_variant variant, falcon_form form, falcon_dtype dtype, falcon_pairing pairing,
+                              falcon_phi phi, int window, int B, int H, int L, int d_k, int d_v, int chunk,
+                              size_t *bytes);
+int falcon_bwd_ws(falcon_variant variant, falcon_form form, falcon_dtype dtype, falcon_pairing pairing,
+                  falcon_phi phi, const void *q, const void *k, const void *v, const void *beta,
+                  const float *lambda, float eps, int window, int B, int H, int L, int d_k, int d_v, int chunk,
+                  const void *dout, const float *dstate, float *dq, float *dk, float *dv, float *dbeta,
+                  float *dlambda, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * falcon_decode_step -- one recurrent step for N independent sequences
@@ -247,6 +374,20 @@ int falcon_decode_step(falcon_variant variant, falcon_dtype dtype,
                        cudaStream_t stream);
 
 /*
+ * falcon_decode_step_ex -- falcon_decode_step with the pairing selectable.
+ * Under the same-step pair ([EXPL] 核心方法 1, warning paragraph) the
+ * step's sample is (phi(k_t), v_t): x_prev is not read and may be NULL (when
+ * given it is still set to phi(k_t)); the window carry then holds the
+ * previous window-1 same-step samples and receives (phi(k_t), v_t).
+ */
+int falcon_decode_step_ex(falcon_variant variant, falcon_dtype dtype, falcon_pairing pairing,
+                          const void *q, const void *k, const void *v, const void *beta,
+                          const float *lambda, float eps, int window,
+                          int N, int H, int d_k, int d_v,
+                          float *state, float *x_prev, float *win, void *out,
+                          cudaStream_t stream);
+
+/*
  * falcon_decode_carry_from_prefill -- the decode carry after a prefill of L
  * tokens: x_prev = phi(k_L) and, for Falcon-3/3A, the samples (x_i, v_i),
  * i = L-window+2 .. L (zeros for i < 1).  k [B,H,L,d_k], v [B,H,L,d_v] dtype;
@@ -258,6 +399,17 @@ int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_dtype dtype,
                                      const void *k, const void *v, int window,
                                      int B, int H, int L, int d_k, int d_v,
                                      float *x_prev, float *win, cudaStream_t stream);
+
+/*
+ * falcon_decode_carry_from_prefill_ex -- the same with the pairing
+ * selectable.  Under the same-step pair the window holds the samples
+ * (phi(k_i), v_i), i = L-window+2 .. L (zeros for i < 1), and x_prev (which
+ * the same-step decode does not read) may be NULL; when given it is phi(k_L).
+ */
+int falcon_decode_carry_from_prefill_ex(falcon_variant variant, falcon_dtype dtype, falcon_pairing pairing,
+                                        const void *k, const void *v, int window,
+                                        int B, int H, int L, int d_k, int d_v,
+                                        float *x_prev, float *win, cudaStream_t stream);
 
 /*
  * falcon_fwd_masked_noalloc -- the masked-parallel forward (prefix pair, L2
@@ -276,7 +428,11 @@ int falcon_decode_carry_from_prefill(falcon_variant variant, falcon_dtype dtype,
  *    FALCON_ERR_SCRATCH and enqueue nothing.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.
+ *    before any stream capture.  With lazy module loading the array itself is
+ *    materialised when the library's device code is first loaded on that
+ *    device, possibly during that first call: make it part of set-up, before
+ *    a memory budget is fixed (a lookup that runs out of memory returns
+ *    FALCON_ERR_ALLOC).
  *  - Every call on a device shares the one array: calls that may overlap on
  *    the GPU (other streams, other host threads) race and must be serialised
  *    by the caller.  No state carries over between calls (every scratch
@@ -315,9 +471,10 @@ int falcon_selftest_bounded_wait(unsigned int timeout_us, int *gave_up);
 
 /*
  * falcon_scratch_trim -- returns the unused memory of the current device's
- * scratch pool (see falcon_fwd) to the driver.  Scratch still in use by
- * enqueued work is kept.  The pool grows again on the next call that needs
- * scratch.  Returns FALCON_OK, or FALCON_ERR_LAUNCH if the CUDA call fails.
+ * current memory pool, from which the allocating entry points draw their
+ * workspace (see falcon_fwd), to the driver (cudaMemPoolTrimTo(pool, 0)).
+ * Memory still in use by enqueued work is kept.  Returns FALCON_OK, or
+ * FALCON_ERR_LAUNCH if the CUDA call fails.
  */
 int falcon_scratch_trim(void);
 

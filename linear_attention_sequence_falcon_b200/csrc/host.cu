@@ -4,9 +4,12 @@
 // outputs go device -> host on a copy-out stream, so that the copies of one
 // slice overlap the compute and the opposite-direction copies of its
 // neighbours.  Events order the three streams; the device buffers are one
-// stream-ordered block of the library's pool, freed on the caller's stream
-// once every copy has been joined back into it.
+// block: the caller's workspace (falcon_fwd_host_ws), or stream-ordered
+// memory freed on the caller's stream once every copy has been joined back
+// into it (falcon_fwd_host).
 #include <cuda_runtime.h>
+
+#include <stdint.h>
 
 #include <algorithm>
 #include <mutex>
@@ -75,11 +78,22 @@ struct Events {
 
 }  // namespace
 
-extern "C" int falcon_fwd_host(int n_variants, const falcon_variant *variants, falcon_form form, falcon_dtype dtype,
-                               falcon_pairing pairing, falcon_phi phi, const void *q, const void *k, const void *v,
-                               const void *beta, const float *lambda, float eps, int window, int B, int H, int L,
-                               int d_k, int d_v, int chunk, void *const *out, float *const *final_state, int slices,
-                               cudaStream_t stream) {
+namespace {
+
+// Device layout of one falcon_fwd_host call: the inputs, lambda, and each
+// variant's outputs and states (each array on a 256-byte boundary), then the
+// workspace of the per-slice forward, which every slice and variant reuses in
+// stream order.
+struct HostLayout {
+    size_t bq, bv, bb, bs;  // bytes per batch row
+    size_t o_k, o_v, o_b, o_l, o_out[kMaxVariants], o_st[kMaxVariants];
+    size_t o_inner, inner, total;
+    int ns;
+};
+
+int host_layout(int n_variants, const falcon_variant *variants, falcon_form form, falcon_dtype dtype,
+                falcon_pairing pairing, falcon_phi phi, int window, int B, int H, int L, int d_k, int d_v, int chunk,
+                bool with_state, const bool *states, int slices, HostLayout *lay) {
     if (n_variants < 1 || n_variants > kMaxVariants || slices < 0) return FALCON_ERR_UNSUPPORTED;
     if (!variants) return FALCON_ERR_NULL;
     for (int i = 0; i < n_variants; ++i) {
@@ -87,30 +101,65 @@ extern "C" int falcon_fwd_host(int n_variants, const falcon_variant *variants, f
         if (rc) return rc;
         if (per_channel(variants[i]) != per_channel(variants[0])) return FALCON_ERR_UNSUPPORTED;
     }
+    HostLayout &y = *lay;
+    const size_t es = dtype == FALCON_BF16 ? 2 : 4;
+    y.bq = (size_t)H * L * d_k * es;
+    y.bv = (size_t)H * L * d_v * es;
+    y.bb = (size_t)H * L * (per_channel(variants[0]) ? d_v : 1) * es;
+    y.bs = (size_t)H * d_v * d_k * sizeof(float);
+    y.o_k = align256((size_t)B * y.bq);
+    y.o_v = y.o_k + align256((size_t)B * y.bq);
+    y.o_b = y.o_v + align256((size_t)B * y.bv);
+    y.o_l = y.o_b + align256((size_t)B * y.bb);
+    size_t total = y.o_l + align256((size_t)H * sizeof(float));
+    for (int i = 0; i < n_variants; ++i) {
+        y.o_out[i] = total;
+        total += align256((size_t)B * y.bv);
+        y.o_st[i] = total;
+        if (with_state && states[i]) total += align256((size_t)B * y.bs);
+    }
+    int ns = slices > 0 ? std::min(slices, B) : default_slices((size_t)B * (2 * y.bq + y.bv + y.bb), B);
+    y.ns = std::max(1, std::min(ns, kMaxSlices));
+    int rows = 0;  // the largest slice
+    for (int i = 0; i < y.ns; ++i)
+        rows = std::max(rows, (int)((long long)(i + 1) * B / y.ns) - (int)((long long)i * B / y.ns));
+    y.inner = 0;
+    for (int i = 0; i < n_variants; ++i) {
+        size_t need = 0;
+        const int rc = falcon_fwd_workspace_size(variants[i], form, dtype, pairing, phi, window, rows, H, L, d_k,
+                                                 d_v, chunk, &need);
+        if (rc) return rc;
+        y.inner = std::max(y.inner, need);
+    }
+    y.o_inner = total;
+    y.total = total + align256(y.inner);
+    return FALCON_OK;
+}
+
+int fwd_host_impl(int n_variants, const falcon_variant *variants, falcon_form form, falcon_dtype dtype,
+                  falcon_pairing pairing, falcon_phi phi, const void *q, const void *k, const void *v,
+                  const void *beta, const float *lambda, float eps, int window, int B, int H, int L, int d_k,
+                  int d_v, int chunk, void *const *out, float *const *final_state, int slices, int ws_given,
+                  void *ws_ptr, size_t ws_bytes, cudaStream_t stream) {
+    bool states[kMaxVariants] = {false};
+    if (n_variants >= 1 && n_variants <= kMaxVariants && final_state)
+        for (int i = 0; i < n_variants; ++i) states[i] = final_state[i] != nullptr;
+    HostLayout lay;
+    int lrc = host_layout(n_variants, variants, form, dtype, pairing, phi, window, B, H, L, d_k, d_v, chunk,
+                          final_state != nullptr, states, slices, &lay);
+    if (lrc) return lrc;
     if ((size_t)B * H == 0) return FALCON_OK;
     if (L > 0) {
         if (!q || !k || !v || !beta || !lambda || !out) return FALCON_ERR_NULL;
         for (int i = 0; i < n_variants; ++i)
             if (!out[i]) return FALCON_ERR_NULL;
     }
-
-    // bytes per batch row of every array, and the device block's layout
-    const size_t es = dtype == FALCON_BF16 ? 2 : 4;
-    const size_t bq = (size_t)H * L * d_k * es, bv = (size_t)H * L * d_v * es;
-    const size_t bb = (size_t)H * L * (per_channel(variants[0]) ? d_v : 1) * es;
-    const size_t bs = (size_t)H * d_v * d_k * sizeof(float);
-    const size_t o_k = align256((size_t)B * bq), o_v = o_k + align256((size_t)B * bq);
-    const size_t o_b = o_v + align256((size_t)B * bv), o_l = o_b + align256((size_t)B * bb);
-    size_t o_out[kMaxVariants], o_st[kMaxVariants];
-    size_t total = o_l + align256((size_t)H * sizeof(float));
-    for (int i = 0; i < n_variants; ++i) {
-        o_out[i] = total;
-        total += align256((size_t)B * bv);
-        o_st[i] = total;
-        if (final_state && final_state[i]) total += align256((size_t)B * bs);
-    }
-    int ns = slices > 0 ? std::min(slices, B) : default_slices((size_t)B * (2 * bq + bv + bb), B);
-    ns = std::min(ns, kMaxSlices);
+    const size_t bq = lay.bq, bv = lay.bv, bb = lay.bb, bs = lay.bs;
+    const size_t o_k = lay.o_k, o_v = lay.o_v, o_b = lay.o_b, o_l = lay.o_l;
+    const size_t *o_out = lay.o_out, *o_st = lay.o_st;
+    const int ns = lay.ns;
+    if (ws_given && (!ws_ptr || ws_bytes < lay.total || (reinterpret_cast<uintptr_t>(ws_ptr) & 255u) != 0))
+        return FALCON_ERR_WORKSPACE;
 
     cudaStream_t s_in, s_out;
     if (copy_streams(&s_in, &s_out) != cudaSuccess) {
@@ -123,10 +172,9 @@ extern "C" int falcon_fwd_host(int n_variants, const falcon_variant *variants, f
         return FALCON_ERR_LAUNCH;
     }
     void *ws = nullptr;
-    if (scratch_alloc(&ws, total, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return FALCON_ERR_ALLOC;
-    }
+    bool owned = false;
+    lrc = ws_acquire(ws_given, ws_ptr, ws_bytes, lay.total, stream, &ws, &owned);
+    if (lrc) return lrc;
     uint8_t *dev = static_cast<uint8_t *>(ws);
     cudaEvent_t ev_start = evs.ev[2 * ns], ev_done = evs.ev[2 * ns + 1], ev_in_tail = evs.ev[2 * ns + 2];
 
@@ -160,11 +208,12 @@ extern "C" int falcon_fwd_host(int n_variants, const falcon_variant *variants, f
         if (rc == FALCON_OK) ok(cudaStreamWaitEvent(stream, ev_in, 0));
         for (int j = 0; j < n_variants && rc == FALCON_OK; ++j) {
             const bool st = final_state && final_state[j];
-            const int r = falcon_fwd_ex(variants[j], form, dtype, pairing, phi, dev + b0 * bq, dev + o_k + b0 * bq,
+            const int r = falcon_fwd_ws(variants[j], form, dtype, pairing, phi, dev + b0 * bq, dev + o_k + b0 * bq,
                                         dev + o_v + b0 * bv, dev + o_b + b0 * bb,
                                         reinterpret_cast<const float *>(dev + o_l), eps, window, nb, H, L, d_k, d_v,
-                                        chunk, dev + o_out[j] + b0 * bv,
-                                        st ? reinterpret_cast<float *>(dev + o_st[j] + b0 * bs) : nullptr, stream);
+                                        chunk, nullptr, nullptr, nullptr, dev + o_out[j] + b0 * bv,
+                                        st ? reinterpret_cast<float *>(dev + o_st[j] + b0 * bs) : nullptr,
+                                        dev + lay.o_inner, lay.inner, stream);
             if (r != FALCON_OK) rc = r;
         }
         if (rc == FALCON_OK) ok(cudaEventRecord(ev_comp, stream));
@@ -189,7 +238,44 @@ extern "C" int falcon_fwd_host(int n_variants, const falcon_variant *variants, f
         cudaStreamSynchronize(stream);
         if (rc == FALCON_OK) rc = FALCON_ERR_LAUNCH;
     }
-    scratch_free(ws, stream);
+    ws_release(ws, owned, stream);
     if (rc != FALCON_OK) cudaGetLastError();
     return rc;
+}
+
+}  // namespace
+
+extern "C" int falcon_fwd_host(int n_variants, const falcon_variant *variants, falcon_form form, falcon_dtype dtype,
+                               falcon_pairing pairing, falcon_phi phi, const void *q, const void *k, const void *v,
+                               const void *beta, const float *lambda, float eps, int window, int B, int H, int L,
+                               int d_k, int d_v, int chunk, void *const *out, float *const *final_state, int slices,
+                               cudaStream_t stream) {
+    return fwd_host_impl(n_variants, variants, form, dtype, pairing, phi, q, k, v, beta, lambda, eps, window, B, H,
+                         L, d_k, d_v, chunk, out, final_state, slices, 0, nullptr, 0, stream);
+}
+
+extern "C" int falcon_fwd_host_workspace_size(int n_variants, const falcon_variant *variants, falcon_form form,
+                                              falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi,
+                                              int window, int B, int H, int L, int d_k, int d_v, int chunk,
+                                              int with_state, int slices, size_t *bytes) {
+    if (!bytes) return FALCON_ERR_NULL;
+    *bytes = 0;
+    bool states[kMaxVariants];
+    for (int i = 0; i < kMaxVariants; ++i) states[i] = with_state != 0;
+    HostLayout lay;
+    const int rc = host_layout(n_variants, variants, form, dtype, pairing, phi, window, B, H, L, d_k, d_v, chunk,
+                               with_state != 0, states, slices, &lay);
+    if (rc) return rc;
+    *bytes = (size_t)B * H == 0 ? 0 : lay.total;
+    return FALCON_OK;
+}
+
+extern "C" int falcon_fwd_host_ws(int n_variants, const falcon_variant *variants, falcon_form form,
+                                  falcon_dtype dtype, falcon_pairing pairing, falcon_phi phi, const void *q,
+                                  const void *k, const void *v, const void *beta, const float *lambda, float eps,
+                                  int window, int B, int H, int L, int d_k, int d_v, int chunk, void *const *out,
+                                  float *const *final_state, int slices, void *workspace, size_t workspace_bytes,
+                                  cudaStream_t stream) {
+    return fwd_host_impl(n_variants, variants, form, dtype, pairing, phi, q, k, v, beta, lambda, eps, window, B, H,
+                         L, d_k, d_v, chunk, out, final_state, slices, 1, workspace, workspace_bytes, stream);
 }

@@ -1167,14 +1167,17 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_rsw_kernel(BwdParams p, 
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float *ns, const float *etas,
                                                        const float *alphas, const float *dga, const float *dgb,
-                                                       float *deta) {
+                                                       const float *dgx, float *deta) {
     constexpr int PER = 8, TS = 256 * PER;
     __shared__ float wsum[8];
     __shared__ float wlam[8];
     const int nch = (p.variant == F2A || p.variant == F2) ? p.dv : 1;
     const size_t bh = blockIdx.x / nch;
     const int ch = (int)(blockIdx.x % nch), L = p.L, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool reg = p.variant == F1 || p.variant == F2 || p.variant == F3;
+    // the regression family's recurrent sweeps give dL/dalpha directly; the
+    // chunk-parallel backward (dgx != NULL) gives dL/dlog alpha whole in dga
+    const bool direct = dgx != nullptr;
+    const bool reg = (p.variant == F1 || p.variant == F2 || p.variant == F3) && !direct;
     const float lam = p.lambda[bh % p.H];
     const T *beta = static_cast<const T *>(p.beta) + bh * (size_t)L * nch;
     float carry = 0.f, dlam = 0.f;
@@ -1185,7 +1188,7 @@ __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float
         for (int k = 0; k < PER; ++k) {
             const int t = base + k;
             const size_t i = (bh * L + t) * nch + ch;
-            v[k] = (t < t1 && !reg) ? dga[i] - dgb[i] : 0.f;
+            v[k] = (t < t1 && !reg && !direct) ? dga[i] - dgb[i] : 0.f;
         }
         float run = 0.f;
 #pragma unroll
@@ -1217,7 +1220,7 @@ __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float
             const size_t i = (bh * L + t) * nch + ch;
             const float a = alphas[i], eta = etas[i], n = ns[bh * L + t];
             // the regression family's sweep gives dL/dalpha directly
-            const float dalpha = reg ? dga[i] : (sfx[k] + later) / a;
+            const float dalpha = reg ? dga[i] : direct ? dga[i] / a : (sfx[k] + later) / a;
             float d = deta[i];
             if (1.f - eta * lam > kAlphaFloor) {
                 d -= lam * dalpha;
@@ -1325,40 +1328,70 @@ int launch_sweep(const BwdParams &p, const float *xs, const float *etas, const f
 
 }  // namespace
 
+namespace {
+
+// Workspace layout (floats): x, dx ([rows][D] each), |x|^2 (window energy)
+// [rows], eta, alpha, the two decay-gradient halves and deta ([rows][nch]
+// each); the regression family adds, from a 256-byte boundary (the sweeps
+// move them in 16-byte pieces), the tile checkpoints [BH][ntile][D][D] and
+// one tile of states per head [BH][TT][D][D].
+size_t bwd_ck_offset(const BwdParams &p) {
+    const size_t rows = (size_t)p.B * p.H * p.L;
+    return (rows * p.dk * 2 + rows + rows * channels(p) * 5 + 63) & ~static_cast<size_t>(63);
+}
+
+}  // namespace
+
+size_t bwd_ws_bytes(const BwdParams &p) {
+    const size_t BH = (size_t)p.B * p.H, ntile = (p.L + TT - 1) / TT;
+    if (BH * p.L == 0) return 0;
+    if (bwd_chunk_covers(p))  // the per-token arrays, dgx, then the chunk path's own
+        return bwd_ck_offset(p) * sizeof(float) + ((BH * p.L * sizeof(float) + 255) & ~static_cast<size_t>(255)) +
+               bwd_chunk_ws_bytes(p);
+    const size_t nreg = regression(p.variant) ? BH * (ntile + TT) * p.dk * p.dk : 0;
+    return (bwd_ck_offset(p) + nreg) * sizeof(float);
+}
+
 template <typename T>
 int launch_bwd(const BwdParams &p, cudaStream_t s) {
     const int D = p.dk, nch = channels(p);
-    const bool reg = regression(p.variant);
     const size_t rows = (size_t)p.B * p.H * p.L;
     if (rows == 0) return 0;
-    // scratch: x, |x|^2 (window energy), eta, alpha, the two decay-gradient halves,
-    // deta, dx; the regression family adds the tile checkpoints and one tile of states per head
     const size_t BH = (size_t)p.B * p.H, ntile = (p.L + TT - 1) / TT;
-    const size_t nreg = reg ? BH * (ntile + TT) * D * D : 0;
-    // the checkpoints start on a 256-byte boundary (the sweeps move them in 16-byte pieces)
-    const size_t off_ck = (rows * D * 2 + rows + rows * nch * 5 + 63) & ~static_cast<size_t>(63);
-    const size_t nf = off_ck + nreg;
+    const size_t off_ck = bwd_ck_offset(p);
     void *ws = nullptr;
-    if (scratch_alloc(&ws, nf * sizeof(float), s) != cudaSuccess) {
-        cudaGetLastError();
-        return -8;  // FALCON_ERR_ALLOC
-    }
+    bool owned = false;
+    const int wrc = ws_acquire(p.ws_given, p.ws, p.ws_bytes, bwd_ws_bytes(p), s, &ws, &owned);
+    if (wrc) return wrc;
     float *xs = static_cast<float *>(ws), *dx = xs + rows * D, *ns = dx + rows * D;
     float *etas = ns + rows, *alphas = etas + rows * nch, *dga = alphas + rows * nch, *dgb = dga + rows * nch;
     float *deta = dgb + rows * nch;
     float *ck = xs + off_ck, *ts = ck + BH * ntile * D * D;
     const unsigned wblocks = (unsigned)((rows * 32 + 255) / 256);
     bwd_prep_kernel<T><<<wblocks, 256, 0, s>>>(p, xs, ns, etas, alphas);
-    int rc = D == 32 ? launch_sweep<T, 32>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
+    float *dgx = nullptr;
+    int rc;
+    if (bwd_chunk_covers(p)) {
+        // chunk-parallel: dgx after the per-token arrays, then the chunk path's workspace
+        dgx = xs + off_ck;
+        uint8_t *cws = reinterpret_cast<uint8_t *>(dgx) + ((rows * sizeof(float) + 255) & ~static_cast<size_t>(255));
+        rc = launch_bwd_chunk(p, cws, xs, etas, alphas, dga, dgb, dgx, deta, dx, s);
+        if (rc == 1) rc = -9;  // FALCON_ERR_UNSUPPORTED: the forward's tensor-core path refused the pointers
+    } else {
+        rc = D == 32 ? launch_sweep<T, 32>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
            : D == 64 ? launch_sweep<T, 64>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
                      : launch_sweep<T, 128>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s);
+    }
+    if (rc != 0) {
+        ws_release(ws, owned, s);
+        return rc;
+    }
     const size_t chans = (size_t)p.B * p.H * nch;
     if (p.dlambda) cudaMemsetAsync(p.dlambda, 0, sizeof(float) * p.H, s);
-    bwd_decay_kernel<T><<<(unsigned)chans, 256, 0, s>>>(p, ns, etas, alphas, dga, dgb, deta);
+    bwd_decay_kernel<T><<<(unsigned)chans, 256, 0, s>>>(p, ns, etas, alphas, dga, dgb, dgx, deta);
     bwd_key_kernel<T><<<wblocks, 256, 0, s>>>(p, xs, deta, dx);
     const cudaError_t e = cudaGetLastError();
-    scratch_free(ws, s);
-    if (rc != 0) return rc;
+    ws_release(ws, owned, s);
     return e == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
 }
 

@@ -470,24 +470,28 @@ __global__ void __launch_bounds__(NTH, 2) pc_out_kernel(FwdParams p, const __gri
 }
 
 
+bool pc_chunk_covers(const FwdParams &p) {
+    if (!(p.variant == F2A && p.dk == DD && p.dv == DD && p.chunk == CH)) return false;
+    return (size_t)p.B * p.H * ((p.L + CH - 1) / CH) <= 0x7fffffffu;
+}
+
+size_t pc_chunk_ws_bytes(const FwdParams &p) { return (size_t)p.B * p.H * ((p.L + CH - 1) / CH) * WS_UNIT; }
+
 int launch_pc_chunk(const FwdParams &p, cudaStream_t s) {
-    const bool shape_ok = p.variant == F2A && p.dk == DD && p.dv == DD && p.chunk == CH;
     auto al16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
-    if (!shape_ok || !al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.beta) || !al16(p.out) ||
+    if (!pc_chunk_covers(p) || !al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.beta) || !al16(p.out) ||
         (p.final_state && !al16(p.final_state)))
         return 1;
     const int BH = p.B * p.H, nch = (p.L + CH - 1) / CH;
     const size_t units = (size_t)BH * nch;
-    if (units > 0x7fffffffu) return 1;
     PcMaps maps;
     if (!make_map(&maps.q, p.q, BH, p.L) || !make_map(&maps.k, p.k, BH, p.L) || !make_map(&maps.v, p.v, BH, p.L) ||
         !make_map(&maps.beta, p.beta, BH, p.L))
         return 1;
     void *ws = nullptr;
-    if (scratch_alloc(&ws, units * WS_UNIT, s) != cudaSuccess) {
-        cudaGetLastError();
-        return -8;  // FALCON_ERR_ALLOC
-    }
+    bool owned = false;
+    const int wrc = ws_acquire(p.ws_given, p.ws, p.ws_bytes, pc_chunk_ws_bytes(p), s, &ws, &owned);
+    if (wrc) return wrc;
     const PcWs w = pc_ws(ws, units);
     static bool attrs_set[64] = {false};
     int dev = 0;
@@ -502,7 +506,7 @@ int launch_pc_chunk(const FwdParams &p, cudaStream_t s) {
     pc_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, s>>>(p, w);
     pc_out_kernel<<<(unsigned)units, NTH, O_SMEM, s>>>(p, maps, w);
     const cudaError_t e = cudaGetLastError();
-    scratch_free(ws, s);
+    ws_release(ws, owned, s);
     return e == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
 }
 

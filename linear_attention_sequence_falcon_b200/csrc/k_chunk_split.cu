@@ -914,6 +914,13 @@ __global__ void __launch_bounds__(NTH2, 1)
             for (int c = 0; c < nch; ++c) {
                 const int s = c % NST;
                 const uint8_t *st = sm + s * IMG;
+                if (p.states_out) {  // the state entering chunk c, for the backward
+                    float *so = p.states_out + (((size_t)bh * nch + c) * DD + j) * DD + chalf * 32;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<float4 *>(so + q * 4) =
+                            make_float4(S[q * 4], S[q * 4 + 1], S[q * 4 + 2], S[q * 4 + 3]);
+                }
                 // B row j (this thread's 32 columns) and g_C while the product runs
                 (void)wait_or_abort(&full[s], (c / NST) & 1, abort_flag);
                 float bv[32];
@@ -1054,28 +1061,30 @@ int sm_count() {
     return counts[dev];
 }
 
+bool split_chunk_covers(const FwdParams &p) {
+    if (!((p.variant == F1 || p.variant == F1A) && p.dk == DD && p.dv == DD && p.chunk == CH)) return false;
+    return (size_t)p.B * p.H * ((p.L + CH - 1) / CH) <= 0x7fffffffu;
+}
+
 size_t split_chunk_ws_bytes(const FwdParams &p) {
     const size_t units = (size_t)p.B * p.H * ((p.L + CH - 1) / CH);
     return units * IMG + units * sizeof(float);
 }
 
 int launch_split_chunk(const FwdParams &p, cudaStream_t s) {
-    const bool shape_ok = (p.variant == F1 || p.variant == F1A) && p.dk == DD && p.dv == DD && p.chunk == CH;
     auto al16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
-    if (!shape_ok || !al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.out) ||
+    if (!split_chunk_covers(p) || !al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.out) ||
         (p.final_state && !al16(p.final_state)))
         return 1;
     const int BH = p.B * p.H, nch = (p.L + CH - 1) / CH;
-    if ((size_t)BH * nch > 0x7fffffffu) return 1;
     SplitMaps maps;
     if (!make_map(&maps.q, p.q, BH, p.L) || !make_map(&maps.k, p.k, BH, p.L) || !make_map(&maps.v, p.v, BH, p.L))
         return 1;
     void *ws = nullptr;
+    bool owned = false;
     const size_t units = (size_t)BH * nch;
-    if (scratch_alloc(&ws, split_chunk_ws_bytes(p), s) != cudaSuccess) {
-        cudaGetLastError();
-        return -8;  // FALCON_ERR_ALLOC
-    }
+    const int wrc = ws_acquire(p.ws_given, p.ws, p.ws_bytes, split_chunk_ws_bytes(p), s, &ws, &owned);
+    if (wrc) return wrc;
     uint8_t *img = static_cast<uint8_t *>(ws);
     float *gc = reinterpret_cast<float *>(img + units * IMG);
     static bool attrs_set[64] = {false};
@@ -1102,7 +1111,7 @@ int launch_split_chunk(const FwdParams &p, cudaStream_t s) {
     const float *cgc = gc;
     cudaLaunchKernelEx(&cfg, chunk_chain_kernel, p, cimg, cgc);
     const cudaError_t e = cudaGetLastError();
-    scratch_free(ws, s);
+    ws_release(ws, owned, s);
     return e == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
 }
 

@@ -41,12 +41,13 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
     const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
     const T *v = static_cast<const T *>(p.v) + (size_t)nh * dv;
     const T *beta = static_cast<const T *>(p.beta) + (size_t)nh * (vi.per_channel ? dv : 1);
-    float *xp = p.x_prev + (size_t)nh * DK;
+    const bool same = p.pairing != 0;  // same-step pair: the current sample is (phi(k_t), v_t)
+    float *xp = p.x_prev ? p.x_prev + (size_t)nh * DK : nullptr;
     float *win = p.win ? p.win + (size_t)nh * (w - 1) * (DK + dv) : nullptr;
 
     // stage the window (oldest first), the current sample (x_prev, v_t), q and k
     for (int i = threadIdx.x; i < DK; i += blockDim.x) {
-        xw[w - 1][i] = xp[i];
+        xw[w - 1][i] = same ? 0.f : xp[i];
         qv[i] = to_f32(q[i]);
         kn[i] = to_f32(k[i]);
     }
@@ -57,6 +58,18 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
         if (c < DK) xw[m][c] = val; else yw[m][c - DK] = val;
     }
     __syncthreads();
+    if (same) {  // the current sample is phi(k_t): its norm first
+        if (warp == 0) {
+            float a = 0.f;
+            for (int c = lane; c < DK; c += 32) a += kn[c] * kn[c];
+            a = group_sum<32>(a);
+            if (lane == 0) knorm = a;
+        }
+        __syncthreads();
+        const float inv = knorm > 0.f ? rsqrtf(knorm) : 0.f;
+        for (int i = threadIdx.x; i < DK; i += blockDim.x) xw[w - 1][i] = kn[i] * inv;
+        __syncthreads();
+    }
     if (warp < w) {
         float a = 0.f, b = 0.f;
         for (int c = lane; c < DK; c += 32) {
@@ -138,9 +151,11 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
             }
         }
     }
-    // carry: x_prev <- phi(k_t); window drops its oldest sample, appends (x_prev, v_t)
+    // carry: x_prev <- phi(k_t); the window drops its oldest sample and
+    // appends the current one (x_prev or phi(k_t), v_t)
     const float inv = knorm > 0.f ? rsqrtf(knorm) : 0.f;
-    for (int i = threadIdx.x; i < DK; i += blockDim.x) xp[i] = kn[i] * inv;
+    if (xp)
+        for (int i = threadIdx.x; i < DK; i += blockDim.x) xp[i] = kn[i] * inv;
     if (w > 1) {
         for (int i = threadIdx.x; i < (w - 1) * (DK + dv); i += blockDim.x) {
             const int m = i / (DK + dv), c = i % (DK + dv);
@@ -168,7 +183,7 @@ __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
     __shared__ float ys[HPB][128];
     __shared__ float bs[HPB][128];
     __shared__ float red[HPB][3][NW];
-    __shared__ float hsc[HPB][4];  // inv_den, xq, lambda, |k|^2
+    __shared__ float hsc[HPB][5];  // inv_den, xq, lambda, |k|^2, 1/|k| (same-step pair)
 
     const VariantInfo vi = variant_info(p.variant, 1);
     const int nh_total = p.N * p.H, dv = p.dv;
@@ -176,17 +191,19 @@ __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
     const int nheads = min(HPB, nh_total - nh0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // stage each pair's sample x = x_prev, q, k, v and beta
+    // stage each pair's sample x = x_prev (prefix pair) or k, normalised
+    // below (same-step pair), q, k, v and beta
+    const bool same = p.pairing != 0;
     for (int hh = 0; hh < nheads; ++hh) {
         const int nh = nh0 + hh;
         const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
         const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
         const T *v = static_cast<const T *>(p.v) + (size_t)nh * dv;
         const T *beta = static_cast<const T *>(p.beta) + (size_t)nh * (vi.per_channel ? dv : 1);
-        const float *xp = p.x_prev + (size_t)nh * DK;
+        const float *xp = same ? nullptr : p.x_prev + (size_t)nh * DK;
         float px = 0.f, pq = 0.f, pk = 0.f;
         for (int i = threadIdx.x; i < DK; i += blockDim.x) {
-            const float xv = xp[i], qv = to_f32(q[i]), kv = to_f32(k[i]);
+            const float qv = to_f32(q[i]), kv = to_f32(k[i]), xv = same ? kv : xp[i];
             xs[hh][i] = xv;
             qs[hh][i] = qv;
             ks[hh][i] = kv;
@@ -209,20 +226,43 @@ __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
         float n = 0.f, xq = 0.f, knorm = 0.f;
 #pragma unroll
         for (int w = 0; w < NW; ++w) { n += red[hh][0][w]; xq += red[hh][1][w]; knorm += red[hh][2][w]; }
+        if (same) {  // x = k / |k|: its energy and its product with q
+            const float inv = knorm > 0.f ? rsqrtf(knorm) : 0.f;
+            n *= inv * inv;
+            xq *= inv;
+            hsc[hh][4] = inv;
+        }
         hsc[hh][0] = n > 0.f ? 1.f / (p.eps + n) : 0.f;  // eta = beta * inv_den
         hsc[hh][1] = xq;
         hsc[hh][2] = p.lambda[(nh0 + hh) % p.H];
         hsc[hh][3] = knorm;
     }
     __syncthreads();
+    if (same) {
+        for (int hh = 0; hh < nheads; ++hh)
+            for (int i = threadIdx.x; i < DK; i += blockDim.x) xs[hh][i] *= hsc[hh][4];
+        __syncthreads();
+    }
 
     const int sl = lane % LPR, rsub = warp * RPW + lane / LPR;
-    for (int r = rsub; r < nheads * dv; r += NW * RPW) {
-        const int hh = r / dv, row = r - hh * dv;  // uniform across a row's lanes
-        float4 xr[NV4], qr[NV4], s4[NV4];
-        float4 *Srow = reinterpret_cast<float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
+    const int total = nheads * dv, stride = NW * RPW;
+    // the next row's state is loaded before this row is reduced, so two rows'
+    // loads are in flight per lane (the step waits on HBM, not on issue)
+    float4 cur[NV4], nxt[NV4];
+    auto load_row = [&](int r, float4(&dst)[NV4]) {
+        if (r < total) {
+            const int hh = r / dv, row = r - hh * dv;
+            const float4 *Srow = reinterpret_cast<const float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
 #pragma unroll
-        for (int i = 0; i < NV4; ++i) s4[i] = Srow[sl + LPR * i];
+            for (int i = 0; i < NV4; ++i) dst[i] = Srow[sl + LPR * i];
+        }
+    };
+    load_row(rsub, cur);
+    for (int r = rsub; r < total; r += stride) {
+        load_row(r + stride, nxt);
+        const int hh = r / dv, row = r - hh * dv;  // uniform across a row's lanes
+        float4 xr[NV4], qr[NV4];
+        float4 *Srow = reinterpret_cast<float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
 #pragma unroll
         for (int i = 0; i < NV4; ++i) {
             xr[i] = *reinterpret_cast<const float4 *>(&xs[hh][4 * (sl + LPR * i)]);
@@ -231,8 +271,8 @@ __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
         float sq = 0.f, sx = 0.f;
 #pragma unroll
         for (int i = 0; i < NV4; ++i) {
-            sq += s4[i].x * qr[i].x + s4[i].y * qr[i].y + s4[i].z * qr[i].z + s4[i].w * qr[i].w;
-            sx += s4[i].x * xr[i].x + s4[i].y * xr[i].y + s4[i].z * xr[i].z + s4[i].w * xr[i].w;
+            sq += cur[i].x * qr[i].x + cur[i].y * qr[i].y + cur[i].z * qr[i].z + cur[i].w * qr[i].w;
+            sx += cur[i].x * xr[i].x + cur[i].y * xr[i].y + cur[i].z * xr[i].z + cur[i].w * xr[i].w;
         }
         sq = group_sum<LPR>(sq);
         if (vi.regression) sx = group_sum<LPR>(sx);
@@ -243,17 +283,19 @@ __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
 #pragma unroll
         for (int i = 0; i < NV4; ++i) {
             float4 o;
-            o.x = alpha * s4[i].x + ge * xr[i].x;
-            o.y = alpha * s4[i].y + ge * xr[i].y;
-            o.z = alpha * s4[i].z + ge * xr[i].z;
-            o.w = alpha * s4[i].w + ge * xr[i].w;
+            o.x = alpha * cur[i].x + ge * xr[i].x;
+            o.y = alpha * cur[i].y + ge * xr[i].y;
+            o.z = alpha * cur[i].z + ge * xr[i].z;
+            o.w = alpha * cur[i].w + ge * xr[i].w;
             Srow[sl + LPR * i] = o;
         }
         if (sl == 0)
             static_cast<T *>(p.out)[(size_t)(nh0 + hh) * dv + row] = from_f32<T>(alpha * sq + ge * hsc[hh][1]);
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) cur[i] = nxt[i];
     }
-    // carry: x_prev <- phi(k_t)
-    for (int hh = 0; hh < nheads; ++hh) {
+    // carry: x_prev <- phi(k_t) (the same-step pair may leave it out)
+    for (int hh = 0; hh < nheads && p.x_prev; ++hh) {
         const float kn = hsc[hh][3];
         const float kinv = kn > 0.f ? rsqrtf(kn) : 0.f;
         float *xp = p.x_prev + (size_t)(nh0 + hh) * DK;
@@ -269,12 +311,15 @@ __global__ void __launch_bounds__(128) carry_kernel(CarryParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const T *k = static_cast<const T *>(p.k) + (size_t)bh * p.L * DK;
     const T *v = static_cast<const T *>(p.v) + (size_t)bh * p.L * p.dv;
-    // job 0: x_prev; jobs 1..w-1: window slots m = job-1
+    // job 0: x_prev = phi(k_L); jobs 1..w-1: window slots m = job-1, the
+    // samples i = L-w+1+m (0-based) whose key is k_{i-1} (prefix pair) or k_i
+    // (same-step pair)
     for (int job = warp; job < w; job += 4) {
+        if (job == 0 && !p.x_prev) continue;
         const int m = job - 1;
-        const int i = job == 0 ? p.L : p.L - (w - 1) + m;  // sample index whose key is k_{i-1}
+        const int i = job == 0 ? p.L : p.L - (w - 1) + m;
         float *xdst = job == 0 ? p.x_prev + (size_t)bh * DK : p.win + ((size_t)bh * (w - 1) + m) * (DK + p.dv);
-        const int ki = i - 1;
+        const int ki = (job > 0 && p.pairing != 0) ? i : i - 1;
         float ss = 0.f;
         for (int c = lane; c < DK; c += 32) {
             const float x = (ki >= 0 && i >= 0) ? to_f32(k[(size_t)ki * DK + c]) : 0.f;

@@ -19,6 +19,8 @@ template <typename T> int launch_span_masked(const FwdParams &p, cudaStream_t s)
 // falls back to the span kernel, and FALCON_ERR_ALLOC when the workspace
 // cannot be had.
 int launch_split_chunk(const FwdParams &p, cudaStream_t s);
+// true when the shape is one the split kernels take (pointer alignment aside)
+bool split_chunk_covers(const FwdParams &p);
 size_t split_chunk_ws_bytes(const FwdParams &p);
 // Number of tensor-core thread blocks that gave up on a bounded wait.
 unsigned int split_wait_timeouts();
@@ -26,6 +28,8 @@ unsigned int split_wait_timeouts();
 // tcgen05 (dS per chunk, state scan, outputs); returns 1 for shapes it does
 // not cover.
 int launch_pc_chunk(const FwdParams &p, cudaStream_t s);
+bool pc_chunk_covers(const FwdParams &p);
+size_t pc_chunk_ws_bytes(const FwdParams &p);
 unsigned int pc_wait_timeouts();
 // bf16 Falcon-2 chunk-parallel forward, d_k = d_v = 128, chunk 64, on tcgen05
 // (one block per head, per-channel forward substitution); returns 1 for
@@ -37,17 +41,41 @@ unsigned int f2_wait_timeouts();
 // returns 1 for shapes it does not cover.
 int launch_w_chunk(const FwdParams &p, cudaStream_t s);
 unsigned int w_wait_timeouts();
+// bf16 Falcon-1/1A chunk-parallel forward, d_k = d_v = 64, chunk 16, 32 or
+// 128 (TF32 warp MMAs, one block per head); returns 1 for shapes it does not
+// cover.
+int launch_seq_chunk(const FwdParams &p, cudaStream_t s);
+bool seq_chunk_covers(const FwdParams &p);
 template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
 // Backward pass of every variant (recurrent form, fp32), d_k = d_v in
 // {32, 64, 128}; the arguments are validated by the caller.
 template <typename T> int launch_bwd(const BwdParams &p, cudaStream_t s);
+size_t bwd_ws_bytes(const BwdParams &p);
+// The chunk-parallel backward (k_bwd_chunk.cu): the shapes it takes, its
+// share of the workspace, and its launch (forward with chunk states, reverse
+// chain, per-chunk gradients) over the per-token arrays of launch_bwd.
+bool bwd_chunk_covers(const BwdParams &p);
+size_t bwd_chunk_ws_bytes(const BwdParams &p);
+int launch_bwd_chunk(const BwdParams &p, void *ws, const float *xs, const float *etas, const float *alphas,
+                     float *dga, float *dgb, float *dgx, float *deta, float *dx, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
 
-// Stream-ordered scratch from the library's per-device pool (kept mapped
-// between calls); scratch_trim hands the pool's unused memory back.
+// Stream-ordered scratch from the device's current memory pool
+// (cudaMallocAsync); scratch_trim hands that pool's unused memory back.
 cudaError_t scratch_alloc(void **ptr, size_t bytes, cudaStream_t s);
 cudaError_t scratch_free(void *ptr, cudaStream_t s);
 cudaError_t scratch_trim();
+
+// Status codes the launchers return (the values of include/falcon.h).
+constexpr int kErrAlloc = -8;
+constexpr int kErrWorkspace = -11;
+// The workspace of one call: the caller's block when `given` (checked to be
+// at least `need` bytes and 256-byte aligned, else kErrWorkspace; nothing is
+// allocated), else `need` bytes drawn stream-ordered on `s` (kErrAlloc if
+// that fails).  *owned tells ws_release whether to free it on `s`.
+int ws_acquire(int given, void *given_ptr, size_t given_bytes, size_t need, cudaStream_t s, void **ptr,
+               bool *owned);
+void ws_release(void *ptr, bool owned, cudaStream_t s);
 
 // The argument checks of falcon_fwd_ex (FALCON_OK or the status it returns
 // for them); nothing is enqueued.

@@ -12,12 +12,17 @@
 // below and makes no allocation of any kind.
 //
 // The array is a file-scope __device__ variable, so every GPU that loads the
-// library holds its kNoAllocScratchBytes until the process exits.  Host code
-// may not use the array's name as a device address (on the host it names a
-// stand-in object), so the device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, on the first call that
-// runs on it; that first call should therefore come before any stream
-// capture.  All calls on a device share the one array: calls that overlap on
+// library's device code holds its kNoAllocScratchBytes until the process
+// exits.  With lazy module loading (the CUDA 12 default) the array is
+// materialised when the module is first loaded on a device, which may be
+// inside this entry point's first call there: a caller on a fixed budget
+// should make that first call during set-up, before the budget is fixed.
+// Host code may not use the array's name as a device address (on the host it
+// names a stand-in object), so the device address is looked up once per
+// device with cudaGetSymbolAddress, with that device current, on the first
+// call that runs on it; that first call should therefore come before any
+// stream capture.  A lookup that fails for lack of memory returns
+// FALCON_ERR_ALLOC.  All calls on a device share the one array: calls that overlap on
 // the GPU (different streams, or several host threads) race on it and must
 // be serialised by the caller.  The kernel writes every scratch element
 // before reading it, so nothing needs clearing between calls.
@@ -52,9 +57,10 @@ int scratch_address(float **out) {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_addr[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) {
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+        if (e != cudaSuccess || !p) {
             cudaGetLastError();
-            return FALCON_ERR_LAUNCH;
+            return e == cudaErrorMemoryAllocation ? FALCON_ERR_ALLOC : FALCON_ERR_LAUNCH;
         }
         g_addr[dev] = static_cast<float *>(p);
     }

@@ -2,6 +2,8 @@
 // Not installed; the public boundary is include/falcon.h.
 #pragma once
 
+#include <stddef.h>
+
 namespace falcon {
 
 struct FwdParams {
@@ -18,10 +20,19 @@ struct FwdParams {
     // initial state [B,H,dv,dk], x_prev [B,H,dk] (x of the first token) and
     // the window-1 samples before the segment [B,H,window-1,dk+dv]
     const float *init_state, *x_prev, *win;
+    // the call's workspace: the caller's block (ws_given, ws_bytes long) or,
+    // when not given, stream-ordered memory drawn by the launcher itself
+    void *ws;
+    size_t ws_bytes;
+    int ws_given;
+    // optional: the state entering every chunk, [B,H,nchunks,dv,dk] fp32
+    // (written by the Falcon-1/1A tensor-core path for the chunk-parallel
+    // backward)
+    float *states_out;
 };
 
 struct DecodeParams {
-    int variant, window;
+    int variant, window, pairing;
     int N, H, dk, dv;
     float eps;
     const void *q, *k, *v, *beta;
@@ -31,7 +42,7 @@ struct DecodeParams {
 };
 
 struct CarryParams {
-    int variant, window;
+    int variant, window, pairing;
     int B, H, L, dk, dv;
     const void *k, *v;
     float *x_prev, *win;

@@ -135,3 +135,84 @@ def test_backward_rejects_an_unsupported_shape(F):
     with pytest.raises(F.FalconError):
         F.bwd("F1", *(d_[n].cuda() for n in ("q", "k", "v", "beta", "lam")), d_["eps"],
               torch.zeros((1, 1, 8, 32), device="cuda"))
+
+
+# --------------------------------------------------------------- the chunk-parallel backward (Falcon-1/1A, bf16, d = 64)
+
+def _check_chunk(F, variant, B, H, L, seed, with_state=True, pairing="prefix", phi="l2", lam=None, key_scale=1.0,
+                 units=None, tol=2e-2):
+    kw = dict(dtype="bf16", key_scale=key_scale)
+    if lam is not None:
+        kw["lam"] = lam
+    d = gen.draw(variant, B, H, L, 64, 64, seed=seed, **kw)
+    rng = np.random.default_rng(seed + 1)
+    do = torch.from_numpy(rng.standard_normal((B, H, L, 64)).astype(np.float32)).to(torch.bfloat16)
+    ds = torch.from_numpy(rng.standard_normal((B, H, 64, 64)).astype(np.float32)) if with_state else None
+    a = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
+    g = F.bwd(variant, *a, d["eps"], do.cuda(), ds.cuda() if ds is not None else None, pairing=pairing, phi=phi,
+              form="chunk", chunk=64)
+    torch.cuda.synchronize()
+    sel = (lambda x: x) if units is None else (lambda x: np.stack([x[b, h] for b, h in units]))
+    if units is None:
+        ref = oracle.bwd(variant, d["q_64"], d["k_64"], d["v_64"], d["beta_64"], d["lam_64"], d["eps_64"],
+                         do.double().numpy(), None if ds is None else ds.double().numpy(), pairing=pairing, phi=phi)
+    else:
+        parts = []
+        for (b, h) in units:
+            s_ = lambda x: x[b:b + 1, h:h + 1]  # noqa: E731
+            parts.append(oracle.bwd(variant, s_(d["q_64"]), s_(d["k_64"]), s_(d["v_64"]), s_(d["beta_64"]),
+                                    d["lam_64"][h:h + 1], d["eps_64"], s_(do.double().numpy()),
+                                    None if ds is None else s_(ds.double().numpy()), pairing=pairing, phi=phi))
+        ref = {n: np.stack([p_[n][0, 0] for p_ in parts]) for n in ("dq", "dk", "dv", "dbeta")}
+    for n in ("dq", "dk", "dv", "dbeta"):
+        got = sel(g[n].double().cpu().numpy())
+        e = rel(got, ref[n])
+        assert np.isfinite(got).all() and e <= tol, (variant, n, e)
+    if units is None:
+        assert rel(g["dlambda"].double().cpu().numpy(), ref["dlambda"]) <= tol, variant
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+@pytest.mark.parametrize("L", [1, 64, 100, 257])
+def test_chunk_backward_matches_oracle(F, variant, L):
+    """One chunk, a ragged tail, several chunks: every gradient of the
+    chunk-parallel backward against the reverse mode of the fp64 recurrence."""
+    _check_chunk(F, variant, 2, 3, L, seed=900 + L)
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_chunk_backward_without_state_gradient(F, variant):
+    _check_chunk(F, variant, 1, 2, 200, seed=911, with_state=False)
+
+
+@pytest.mark.parametrize("pairing,phi", [("same_step", "l2"), ("prefix", "identity")])
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_chunk_backward_pairing_and_feature_map(F, variant, pairing, phi):
+    _check_chunk(F, variant, 1, 2, 150, seed=913, pairing=pairing, phi=phi, key_scale=0.125)
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_chunk_backward_strong_forgetting(F, variant):
+    """lambda = 0.999: chunk log-decays around -45."""
+    _check_chunk(F, variant, 1, 3, 200, seed=915, lam=0.999)
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_chunk_backward_workload2_shape(F, variant):
+    """8 x 12 x 2048 x 64 bf16, 32 chunks per head; three sampled heads
+    against the oracle's reverse mode."""
+    _check_chunk(F, variant, 8, 12, 2048, seed=917, units=[(0, 0), (3, 7), (7, 11)])
+
+
+def test_chunk_backward_matches_recurrent_backward(F):
+    """The two forms' gradients on the GPU agree (same function, two
+    computations)."""
+    d = gen.draw("F1", 2, 2, 300, 64, 64, seed=919, dtype="bf16")
+    a = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
+    do = torch.randn((2, 2, 300, 64), device="cuda").to(torch.bfloat16)
+    ds = torch.randn((2, 2, 64, 64), device="cuda")
+    g1 = F.bwd("F1", *a, d["eps"], do, ds, form="chunk")
+    g2 = F.bwd("F1", *a, d["eps"], do, ds, form="recurrent")
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "dbeta", "dlambda"):
+        assert rel(g1[n].double().cpu().numpy(), g2[n].double().cpu().numpy()) <= 2e-2, n

@@ -97,6 +97,30 @@ def test_chunk_sizes(F, variant, chunk):
     check(F, d, variant, "chunk", chunk=chunk, window=w)
 
 
+@pytest.mark.parametrize("chunk", [16, 32, 128])
+@pytest.mark.parametrize("L", [1, 15, 100, 128, 129, 513])
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_tensor_core_chunk_lengths(F, variant, L, chunk):
+    """bf16 Falcon-1/1A at d = 64 with chunk 16, 32 and 128 (the tensor-core
+    path that walks a head's chunks): one token, ragged tails, exact
+    multiples and many chunks."""
+    d = gen.draw(variant, 2, 3, L, 64, 64, seed=300 + L + chunk, dtype="bf16")
+    check(F, d, variant, "chunk", chunk=chunk)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 128])
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_tensor_core_chunk_lengths_options(F, variant, chunk):
+    """The same path with the same-step pair, the identity map, strong
+    forgetting and the decay floor."""
+    d = gen.draw(variant, 1, 2, 150, 64, 64, seed=310 + chunk, dtype="bf16", key_scale=0.125)
+    check(F, d, variant, "chunk", chunk=chunk, pairing="same_step", phi="identity")
+    d = gen.draw(variant, 1, 3, 200, 64, 64, seed=311 + chunk, dtype="bf16", lam=0.999)
+    check(F, d, variant, "chunk", chunk=chunk)
+    d = gen.draw(variant, 1, 2, 200, 64, 64, seed=312 + chunk, dtype="bf16", lam=0.9, key_scale=0.05)
+    check(F, d, variant, "chunk", chunk=chunk, phi="identity")
+
+
 @pytest.mark.parametrize("w", [1, 2, 5, 8])
 @pytest.mark.parametrize("variant", ["F3", "F3A"])
 @pytest.mark.parametrize("form", ["recurrent", "masked", "chunk"])
@@ -204,44 +228,70 @@ def test_workload5_prefill_sampled(F):
 
 # --------------------------------------------------------------- decode
 
-def _decode_chain(F, variant, N, H, dk, dv, L0, steps, dtype, w):
-    d = gen.draw(variant, N, H, L0 + steps, dk, dv, seed=555, dtype=dtype, lam=0.02)
+def _decode_chain(F, variant, N, H, dk, dv, L0, steps, dtype, w, pairing="prefix", lam=0.02, seed=555):
+    d = gen.draw(variant, N, H, L0 + steps, dk, dv, seed=seed, dtype=dtype, lam=lam)
     pre = {n: d[n][:, :, :L0].contiguous() for n in ("q", "k", "v", "beta")}
     _, S = F.fwd(variant, "chunk", *(pre[n].cuda() for n in ("q", "k", "v", "beta")), d["lam"].cuda(), d["eps"],
-                 window=w, chunk=64)
-    x_prev, win = F.carry_from_prefill(variant, pre["k"].cuda(), pre["v"].cuda(), w)
+                 window=w, chunk=64, pairing=pairing)
+    x_prev, win = F.carry_from_prefill(variant, pre["k"].cuda(), pre["v"].cuda(), w, pairing=pairing)
     torch.cuda.synchronize()
     # carry parity
-    ox, ow = oracle.carry_from_prefill(variant, d["k_64"][:, :, :L0], d["v_64"][:, :, :L0], w)
+    ox, ow = oracle.carry_from_prefill(variant, d["k_64"][:, :, :L0], d["v_64"][:, :, :L0], w, pairing=pairing)
     assert rel(x_prev.double().cpu().numpy(), ox) <= 1e-6
     if w > 1:
         assert rel(win.double().cpu().numpy(), ow) <= 1e-6
-    outs = []
-    for t in range(L0, L0 + steps):
-        o = F.decode_step(variant, *(d[n][:, :, t].contiguous().cuda() for n in ("q", "k", "v", "beta")),
-                          d["lam"].cuda(), d["eps"], w, S, x_prev, win)
-        outs.append(o.double().cpu().numpy())
+    # every step's token vectors as one contiguous [steps, N, H, ...] block on the device
+    tok = {n: d[n][:, :, L0:].movedim(2, 0).contiguous().cuda() for n in ("q", "k", "v", "beta")}
+    lam_d = d["lam"].cuda()
+    outs = torch.empty((steps,) + (N, H, dv), dtype=d["q"].dtype, device="cuda")
+    for i in range(steps):
+        F.decode_step(variant, tok["q"][i], tok["k"][i], tok["v"][i], tok["beta"][i], lam_d, d["eps"], w, S,
+                      None if pairing == "same_step" else x_prev, win, out=outs[i], pairing=pairing)
     torch.cuda.synchronize()
-    return d, np.stack(outs, 2), S.double().cpu().numpy()
+    return d, outs.movedim(0, 2).double().cpu().numpy(), S.double().cpu().numpy()
 
 
+@pytest.mark.parametrize("pairing", ["prefix", "same_step"])
 @pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_decode_chain_matches_longer_prefill(F, variant, dtype):
-    """prefill(L0) -> carry -> decode steps == oracle over L0 + steps tokens."""
+def test_decode_chain_matches_longer_prefill(F, variant, dtype, pairing):
+    """prefill(L0) -> carry -> decode steps == oracle over L0 + steps tokens,
+    under the prefix pair and the same-step pair (whose decode reads phi(k_t)
+    itself and no x_prev)."""
     w = 4 if variant in ("F3", "F3A") else 1
     L0, steps = 70, 9
-    d, outs, S = _decode_chain(F, variant, 3, 4, 64, 64, L0, steps, dtype, w)
-    oo, oS = oracle_fwd(d, variant, w)
+    d, outs, S = _decode_chain(F, variant, 3, 4, 64, 64, L0, steps, dtype, w, pairing=pairing)
+    oo, oS = oracle_fwd(d, variant, w, pairing=pairing)
     tol = TOL[dtype]
     assert rel(outs, oo[:, :, L0:]) <= tol
     assert rel(S, oS) <= tol
 
 
-def test_decode_workload5_shape(F):
+@pytest.mark.parametrize("variant,dk,w,dtype", [("F2A", 128, 1, "bf16"), ("F2A", 128, 1, "f32"),
+                                                ("F1", 64, 1, "bf16"), ("F3", 64, 4, "bf16"),
+                                                ("F1", 64, 1, "f32")])
+def test_decode_chain_4096_steps(F, variant, dk, w, dtype):
+    """The decode length of the long-sequence workload: 4,096 decode steps
+    after a 64-token prefill, fp32 state (N = 2, H = 2, lambda = 0.02).  Every
+    step's output and the final state against the fp64 recurrence over all
+    4,160 tokens: fp32 state drift over thousands of updates stays within the
+    tolerance."""
+    L0, steps = 64, 4096
+    d, outs, S = _decode_chain(F, variant, 2, 2, dk, dk, L0, steps, dtype, w, seed=5050)
+    oo, oS = oracle_fwd(d, variant, w)
+    tol = TOL[dtype]
+    eo, eS = rel(outs, oo[:, :, L0:]), rel(S, oS)
+    # per-step check on a spread of steps, so that a late drift cannot hide behind early large outputs
+    for t in (0, 1, 1023, 2047, 3071, steps - 1):
+        assert rel(outs[:, :, t], oo[:, :, L0 + t]) <= tol, (t, rel(outs[:, :, t], oo[:, :, L0 + t]))
+    assert eo <= tol and eS <= tol, (eo, eS)
+
+
+@pytest.mark.parametrize("pairing", ["prefix", "same_step"])
+def test_decode_workload5_shape(F, pairing):
     """N=64, H=16, 128x128 fp32 state: a few steps after a short prefill."""
-    d, outs, S = _decode_chain(F, "F2A", 64, 16, 128, 128, 40, 4, "bf16", 1)
-    oo, oS = oracle_fwd(d, "F2A", 1)
+    d, outs, S = _decode_chain(F, "F2A", 64, 16, 128, 128, 40, 4, "bf16", 1, pairing=pairing)
+    oo, oS = oracle_fwd(d, "F2A", 1, pairing=pairing)
     assert rel(outs, oo[:, :, 40:]) <= 2e-2
     assert rel(S, oS) <= 2e-2
 
