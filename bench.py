@@ -372,7 +372,7 @@ def run_ours(args):
     achieved = ab / (f1_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
             "traffic": profiled_traffic("chunk"),
-            "kernel": "one Falcon-1 chunk-parallel forward (chunk_local_kernel + chunk_chain_kernel)",
+            "kernel": "one Falcon-1 chunk-parallel forward (chunk_local_kernel<true>: local part and chain step fused)",
             "peak_source": src,
             "algorithmic_bytes_per_launch": ab, "launch_ms": f1_ms}
 
@@ -390,8 +390,9 @@ def run_ours(args):
             "config": workload_config(), "roofline": roof,
             "per_variant_ms": {var: statistics.mean(per_var[var]) for var in w["variants"]},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            # every falcon_fwd of this shape is two kernels: chunk_local_kernel + chunk_chain_kernel
-            "gpu_launches": 2 * len(w["variants"]) * args.steps, "clocks": clk.summary(),
+            # every falcon_fwd of this shape is one kernel (chunk_local_kernel<true>) after a
+            # memset of its ticket counter and head counts
+            "gpu_launches": len(w["variants"]) * args.steps, "clocks": clk.summary(),
             "wait_timeouts_delta": timeouts_delta}
     if decode is not None:
         line["decode"] = decode
@@ -496,7 +497,7 @@ def time_call(fn, flush, steps, stream=None):
     return statistics.median(ms)
 
 
-SWEEP_KERNELS = {16: "seq_chunk_kernel<16>", 32: "seq_chunk_kernel<32>", 64: "chunk_local_kernel + chunk_chain_kernel",
+SWEEP_KERNELS = {16: "seq_chunk_kernel<16>", 32: "seq_chunk_kernel<32>", 64: "chunk_local_kernel<true> (fused)",
                  128: "seq_chunk_kernel<128>"}
 
 
@@ -636,6 +637,8 @@ def run_backward(args):
     for n, var in ((2, "F1"), (2, "F1A"), (3, "F2"), (4, "F3"), (4, "F3A"), (5, "F2A")):
         if args.only and n != args.only:
             continue
+        if args.bwd_form == "chunk" and var not in ("F1", "F1A"):
+            continue  # the chunk-parallel backward covers Falcon-1/1A (bf16, d = 64)
         w = gen.WORKLOADS[n]
         d = gen.workload_inputs(n, var)
         B, H, L, dk, dv = w["B"], w["H"], w["L"], w["dk"], w["dv"]
@@ -643,7 +646,7 @@ def run_backward(args):
         do = torch.from_numpy(rng.standard_normal((B, H, L, dv)).astype(np.float32)).to(torch.bfloat16).cuda()
         ds = torch.from_numpy(rng.standard_normal((B, H, dv, dk)).astype(np.float32)).cuda()
         a = [d[k].cuda() for k in ("q", "k", "v", "beta", "lam")]
-        F.bwd(var, *a, d["eps"], do, ds, window=w["window"])
+        F.bwd(var, *a, d["eps"], do, ds, window=w["window"], form=args.bwd_form)
         torch.cuda.synchronize()
         ms = []
         for _ in range(max(3, min(args.steps, 10))):
@@ -651,7 +654,7 @@ def run_backward(args):
             torch.cuda._sleep(HEAD_START_CYCLES)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            F.bwd(var, *a, d["eps"], do, ds, window=w["window"])
+            F.bwd(var, *a, d["eps"], do, ds, window=w["window"], form=args.bwd_form)
             e1.record()
             torch.cuda.synchronize()
             ms.append(e0.elapsed_time(e1))
@@ -660,8 +663,11 @@ def run_backward(args):
         tok = B * H * L
         ab = tok * (dk + dk + dv + nb + dv) * 2 + tok * (dk + dk + dv + nb) * 4 + B * H * dv * dk * 4
         gbs = ab / (t / 1e3) / 1e9
-        line = {"backward": var, "workload": w["name"], "ms": t, "tokens_per_s": B * L / (t / 1e3),
-                "kernels": "bwd_prep_kernel + bwd_sweep_kernel + bwd_decay_kernel + bwd_key_kernel",
+        kern = ("bwd_prep_kernel + chunk_local_kernel + chunk_chain_kernel + bwd_rchain_kernel + bwd_chunk_kernel"
+                " + bwd_decay_kernel + bwd_key_kernel" if args.bwd_form == "chunk" else
+                "bwd_prep_kernel + bwd_sweep_kernel + bwd_decay_kernel + bwd_key_kernel")
+        line = {"backward": var, "form": args.bwd_form, "workload": w["name"], "ms": t,
+                "tokens_per_s": B * L / (t / 1e3), "kernels": kern,
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                              "peak_source": peak_src, "algorithmic_bytes_per_launch": ab}}
         if n in (2, 4) and not args.no_cpu_baseline:
@@ -725,6 +731,8 @@ def main():
     ap.add_argument("--only", type=int, default=0, help="with --workloads or --backward: just this workload number")
     ap.add_argument("--backward", action="store_true",
                     help="time falcon_bwd on workloads 2 (Falcon-1, -1A), 3 (Falcon-2) and 5's prefill (Falcon-2A)")
+    ap.add_argument("--bwd-form", default="recurrent", choices=["recurrent", "chunk"],
+                    help="with --backward: the form whose derivative is taken")
     ap.add_argument("--chunk-sweep", action="store_true",
                     help="the chunk form of workload 2 at chunk 16/32/64 and both pairings (one line each)")
     ap.add_argument("--profile", action="store_true",

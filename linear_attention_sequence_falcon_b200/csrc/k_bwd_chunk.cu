@@ -457,7 +457,7 @@ size_t bwd_chunk_ws_bytes(const BwdParams &p) {
     const size_t rows = BH * p.L;
     FwdParams f{};
     f.variant = p.variant; f.B = p.B; f.H = p.H; f.L = p.L; f.dk = DD; f.dv = DD; f.chunk = CC;
-    return al256(split_chunk_ws_bytes(f))         // the forward's images and g_C
+    return al256(split_chunk_images_ws_bytes(f))  // the forward's images and g_C
            + al256(units * DD * DD * 4) * 2       // states entering each chunk; G^ leaving each chunk
            + al256(rows * DD * 2)                 // the forward's outputs (unused)
            + al256(BH * DD * DD * 4);             // the forward's final state
@@ -473,7 +473,7 @@ int launch_bwd_chunk(const BwdParams &p, void *ws, const float *xs, const float 
     f.B = p.B; f.H = p.H; f.L = p.L; f.dk = DD; f.dv = DD; f.chunk = CC; f.eps = p.eps;
     f.q = p.q; f.k = p.k; f.v = p.v; f.beta = p.beta; f.lambda = p.lambda;
     size_t off = 0;
-    f.ws = base; f.ws_bytes = split_chunk_ws_bytes(f); f.ws_given = 1;
+    f.ws = base; f.ws_bytes = split_chunk_images_ws_bytes(f); f.ws_given = 1;
     const uint8_t *img = base;
     const float *gc = reinterpret_cast<const float *>(base + units * IMG_B);
     off += al256(f.ws_bytes);
