@@ -60,7 +60,7 @@ def _load():
         lib.oracle_carry_from_prefill.restype = I
         lib.oracle_fwd_carry.argtypes = [I, I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, I, dp, dp, dp, dp, dp, I]
         lib.oracle_fwd_carry.restype = I
-        lib.oracle_bwd.argtypes = [I, I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, I, dp, dp, dp, dp, dp, dp, dp, I]
+        lib.oracle_bwd.argtypes = [I, I, I, dp, dp, dp, dp, dp, D, I, I, I, I, I, I, dp, dp, dp, dp, dp, dp, dp, I, dp]
         lib.oracle_bwd.restype = I
         _lib = lib
     return _lib
@@ -160,17 +160,18 @@ def fwd_carry(variant, q, k, v, beta, lam, eps, window=1, S0=None, x_prev=None, 
 def bwd(variant, q, k, v, beta, lam, eps, dout, dstate=None, window=1, pairing="prefix", phi="l2", nthreads=0):
     """Reverse mode of the recurrent definition (S_0 = 0): given dL/dout
     [B,H,L,dv] and dL/dS_L [B,H,dv,dk] (None: zero), returns dq, dk, dv
-    (shapes of q, k, v), dbeta (shape of beta) and dlambda [H]."""
+    (shapes of q, k, v), dbeta (shape of beta), dlambda [H] and
+    dlambda_l1 [H], the sum of the magnitudes of the terms dlambda adds up."""
     lib = _load()
     q, k, v, beta, lam, dout = map(_f64, (q, k, v, beta, lam, dout))
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     dq, dkk, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
-    dbeta, dlam = np.zeros_like(beta), np.zeros(H)
+    dbeta, dlam, dlam_l1 = np.zeros_like(beta), np.zeros(H), np.zeros(H)
     ds = None if dstate is None else _f64(dstate)
     rc = lib.oracle_bwd(VARIANTS[variant], PAIRINGS[pairing], PHIS[phi], _p(q), _p(k), _p(v), _p(beta), _p(lam),
                         float(eps), int(window), B, H, L, dk, dv, _p(dout), None if ds is None else _p(ds),
-                        _p(dq), _p(dkk), _p(dvv), _p(dbeta), _p(dlam), int(nthreads))
+                        _p(dq), _p(dkk), _p(dvv), _p(dbeta), _p(dlam), int(nthreads), _p(dlam_l1))
     if rc < 0:
         raise ValueError("oracle_bwd rejected its arguments (code %d)" % rc)
-    return {"dq": dq, "dk": dkk, "dv": dvv, "dbeta": dbeta, "dlambda": dlam}
+    return {"dq": dq, "dk": dkk, "dv": dvv, "dbeta": dbeta, "dlambda": dlam, "dlambda_l1": dlam_l1}

@@ -625,6 +625,7 @@ typedef struct {
     double eps;
     const double *q, *k, *v, *beta, *lambda, *dout, *dstate;
     double *dq, *dkk, *dvv, *dbeta, *dlam_bh;  /* dlam_bh [B*H], summed by the caller */
+    double *dlam_l1_bh;                        /* [B*H]: sum of |eta_t dL/dalpha_t| over the dlambda terms */
 } bwd_job_t;
 
 static void bwd_unit_run(const bwd_job_t *Bj, int b, int h)
@@ -726,7 +727,7 @@ static void bwd_unit_run(const bwd_job_t *Bj, int b, int h)
     const double lam = Bj->lambda[h];
     const double *beta = Bj->beta + bh * (size_t)L * nch;
     double *dbeta = Bj->dbeta + bh * (size_t)L * nch;
-    double dlam = 0.0;
+    double dlam = 0.0, dlam_l1 = 0.0;
     for (int t = 0; t < L; ++t) {
         int i0 = t - w + 1;
         if (i0 < 0) i0 = 0;
@@ -739,6 +740,7 @@ static void bwd_unit_run(const bwd_job_t *Bj, int b, int h)
             if (1.0 - eta * lam > ALPHA_FLOOR) {
                 de_ += -lam * dalpha[(size_t)t * nch + ch];
                 dlam += -eta * dalpha[(size_t)t * nch + ch];
+                dlam_l1 += fabs(eta * dalpha[(size_t)t * nch + ch]);
             }
             if (n > 0.0) {
                 const double bt = beta[(size_t)t * nch + ch];
@@ -769,6 +771,7 @@ static void bwd_unit_run(const bwd_job_t *Bj, int b, int h)
         }
     }
     Bj->dlam_bh[bh] = dlam;
+    Bj->dlam_l1_bh[bh] = dlam_l1;
     free(hist); free(res); free(Gs); free(Gn); free(dx); free(deta); free(dalpha); free(de);
     free_unit(&u);
 }
@@ -786,17 +789,20 @@ static void *bwd_worker(void *arg)
     return NULL;
 }
 
+/* dlambda_l1 (optional, [H]): the sum over b and t of |eta_t dL/dalpha_t|,
+ * the mass of the terms dlambda sums (the scale of its rounding error). */
 int oracle_bwd(int variant, int pairing, int phi, const double *q, const double *k, const double *v,
                const double *beta, const double *lambda, double eps, int window, int B, int H, int L, int dk, int dv,
                const double *dout, const double *dstate, double *dq, double *dkk, double *dvv, double *dbeta,
-               double *dlambda, int nthreads)
+               double *dlambda, int nthreads, double *dlambda_l1)
 {
     if (variant < 0 || variant > 5) return -2;
     if (B < 0 || H < 0 || L < 0 || dk <= 0 || dv <= 0) return -3;
     if (is_window(variant) && window < 1) return -6;
     double *dlam_bh = (double *)calloc((size_t)B * H + 1, sizeof(double));
+    double *dlam_l1_bh = (double *)calloc((size_t)B * H + 1, sizeof(double));
     bwd_job_t J = {variant, pairing, phi, B, H, L, dk, dv, is_window(variant) ? window : 1, eps,
-                   q, k, v, beta, lambda, dout, dstate, dq, dkk, dvv, dbeta, dlam_bh};
+                   q, k, v, beta, lambda, dout, dstate, dq, dkk, dvv, dbeta, dlam_bh, dlam_l1_bh};
     if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
     if (nthreads < 1) nthreads = 1;
     const int units = B * H;
@@ -809,10 +815,14 @@ int oracle_bwd(int variant, int pairing, int phi, const double *q, const double 
     }
     for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
     for (int hh = 0; hh < H; ++hh) {
-        double s = 0.0;
-        for (int bb = 0; bb < B; ++bb) s += dlam_bh[(size_t)bb * H + hh];
+        double s = 0.0, a = 0.0;
+        for (int bb = 0; bb < B; ++bb) {
+            s += dlam_bh[(size_t)bb * H + hh];
+            a += dlam_l1_bh[(size_t)bb * H + hh];
+        }
         dlambda[hh] = s;
+        if (dlambda_l1) dlambda_l1[hh] = a;
     }
-    free(th); free(ws); free(dlam_bh);
+    free(th); free(ws); free(dlam_bh); free(dlam_l1_bh);
     return nthreads;
 }

@@ -169,7 +169,13 @@ def _check_chunk(F, variant, B, H, L, seed, with_state=True, pairing="prefix", p
         e = rel(got, ref[n])
         assert np.isfinite(got).all() and e <= tol, (variant, n, e)
     if units is None:
-        assert rel(g["dlambda"].double().cpu().numpy(), ref["dlambda"]) <= tol, variant
+        # dlambda is a sum over every token of -eta_t dL/dalpha_t; a sum whose
+        # terms carry a relative error e is accurate to e times the mass of
+        # its terms, which the oracle reports per head (terms of both signs
+        # cancel under strong forgetting, so the sum itself can be far smaller)
+        dl = g["dlambda"].double().cpu().numpy()
+        assert np.all(np.abs(dl - ref["dlambda"]) <= tol * ref["dlambda_l1"]), (variant, dl, ref["dlambda"],
+                                                                              ref["dlambda_l1"])
 
 
 @pytest.mark.parametrize("variant", ["F1", "F1A"])
@@ -214,5 +220,12 @@ def test_chunk_backward_matches_recurrent_backward(F):
     g1 = F.bwd("F1", *a, d["eps"], do, ds, form="chunk")
     g2 = F.bwd("F1", *a, d["eps"], do, ds, form="recurrent")
     torch.cuda.synchronize()
-    for n in ("dq", "dk", "dv", "dbeta", "dlambda"):
+    for n in ("dq", "dk", "dv", "dbeta"):
         assert rel(g1[n].double().cpu().numpy(), g2[n].double().cpu().numpy()) <= 2e-2, n
+    # dlambda sums terms of both signs over every token: the two forms may
+    # differ by the per-term error times the mass of the terms, which the
+    # oracle reports for these inputs
+    ref = oracle.bwd("F1", d["q_64"], d["k_64"], d["v_64"], d["beta_64"], d["lam_64"], d["eps_64"],
+                     do.double().cpu().numpy(), ds.double().cpu().numpy())
+    dl1, dl2 = (g["dlambda"].double().cpu().numpy() for g in (g1, g2))
+    assert np.all(np.abs(dl1 - dl2) <= 2e-2 * ref["dlambda_l1"]), (dl1, dl2, ref["dlambda_l1"])

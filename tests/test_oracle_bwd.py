@@ -105,9 +105,27 @@ def test_backward_closed_form_without_forgetting():
     assert np.abs(g["dlambda"]).max() > 0  # lambda = 0 is not clamped: its gradient is -sum eta dalpha
 
 
+def test_dlambda_term_mass():
+    """dlambda_l1 is the mass of the terms dlambda sums: |dlambda| <= mass,
+    with equality for a single token (one term), and the mass of a batch is
+    the sum of its rows' masses."""
+    rng = np.random.default_rng(7)
+    q, k, v, beta, lam = draw("F1", rng, L=40, B=3)
+    do = rng.standard_normal(v.shape)
+    g = oracle.bwd("F1", q, k, v, beta, lam, 1e-6, do)
+    assert np.all(np.abs(g["dlambda"]) <= g["dlambda_l1"] + 1e-12) and np.all(g["dlambda_l1"] > 0)
+    parts = [oracle.bwd("F1", q[b:b + 1], k[b:b + 1], v[b:b + 1], beta[b:b + 1], lam, 1e-6, do[b:b + 1])
+             for b in range(3)]
+    np.testing.assert_allclose(sum(p["dlambda_l1"] for p in parts), g["dlambda_l1"], rtol=1e-12)
+    # two tokens under the prefix pair: x_1 = 0, so only token 2 steps: one term
+    q2, k2, v2, b2, l2 = (a[:1, :, :2] if a.ndim > 1 else a for a in (q, k, v, beta, lam))
+    g2 = oracle.bwd("F1", q2, k2, v2, b2, lam, 1e-6, do[:1, :, :2])
+    np.testing.assert_allclose(np.abs(g2["dlambda"]), g2["dlambda_l1"], rtol=1e-12)
+
+
 def test_backward_of_an_empty_sequence():
     rng = np.random.default_rng(3)
     q, k, v, beta, lam = draw("F2A", rng, L=0)
     g = oracle.bwd("F2A", q, k, v, beta, lam, 1e-6, np.zeros(v.shape))
-    assert all(a.size == 0 for key, a in g.items() if key != "dlambda")
-    assert np.all(g["dlambda"] == 0)
+    assert all(a.size == 0 for key, a in g.items() if key not in ("dlambda", "dlambda_l1"))
+    assert np.all(g["dlambda"] == 0) and np.all(g["dlambda_l1"] == 0)
