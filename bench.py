@@ -372,7 +372,7 @@ def run_ours(args):
     achieved = ab / (f1_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
             "traffic": profiled_traffic("chunk"),
-            "kernel": "one Falcon-1 chunk-parallel forward (chunk_local_kernel<true>: local part and chain step fused)",
+            "kernel": "one Falcon-1 chunk-parallel forward (chunk_local_kernel + chunk_chain_kernel)",
             "peak_source": src,
             "algorithmic_bytes_per_launch": ab, "launch_ms": f1_ms}
 
@@ -390,9 +390,8 @@ def run_ours(args):
             "config": workload_config(), "roofline": roof,
             "per_variant_ms": {var: statistics.mean(per_var[var]) for var in w["variants"]},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            # every falcon_fwd of this shape is one kernel (chunk_local_kernel<true>) after a
-            # memset of its ticket counter and head counts
-            "gpu_launches": len(w["variants"]) * args.steps, "clocks": clk.summary(),
+            # every falcon_fwd of this shape is two kernels: chunk_local_kernel + chunk_chain_kernel
+            "gpu_launches": 2 * len(w["variants"]) * args.steps, "clocks": clk.summary(),
             "wait_timeouts_delta": timeouts_delta}
     if decode is not None:
         line["decode"] = decode
@@ -497,7 +496,7 @@ def time_call(fn, flush, steps, stream=None):
     return statistics.median(ms)
 
 
-SWEEP_KERNELS = {16: "seq_chunk_kernel<16>", 32: "seq_chunk_kernel<32>", 64: "chunk_local_kernel<true> (fused)",
+SWEEP_KERNELS = {16: "seq_chunk_kernel<16>", 32: "seq_chunk_kernel<32>", 64: "chunk_local_kernel + chunk_chain_kernel",
                  128: "seq_chunk_kernel<128>"}
 
 

@@ -83,7 +83,7 @@ enum {
     FALCON_ERR_NULL = -1,        /* a required pointer is NULL                      */
     FALCON_ERR_ENUM = -2,        /* variant / form / dtype / pairing / phi invalid   */
     FALCON_ERR_SHAPE = -3,       /* B,H,L < 0, or d_k, d_v not in {16,32,64,128}     */
-    FALCON_ERR_CHUNK = -4,       /* chunk not in {16,32,64} for the chunk form      */
+    FALCON_ERR_CHUNK = -4,       /* chunk not in {16,32,64} (or 128 where taken)     */
     FALCON_ERR_WINDOW = -6,      /* window < 1 or > 8 for Falcon-3/3A               */
     FALCON_ERR_LAUNCH = -7,      /* a kernel launch failed (cudaGetLastError)       */
     FALCON_ERR_ALLOC = -8,       /* stream-ordered scratch allocation failed        */
@@ -103,7 +103,8 @@ enum {
  *   lambda   [H] fp32              forgetting strength per head, in [0,1)
  *   eps      NLMS regulariser (>= 0)
  *   window   B_w for Falcon-3/3A (1..8); ignored otherwise
- *   chunk    chunk length for FALCON_CHUNK (16, 32 or 64); ignored otherwise
+ *   chunk    chunk length for FALCON_CHUNK (16, 32 or 64; 128 for Falcon-1/1A
+ *            with bf16 inputs and d_k = d_v in {32, 64}); ignored otherwise
  *   out      [B,H,L,d_v] dtype     o_t = S_t q_t (written)
  *   final_state [B,H,d_v,d_k] fp32 S_L (written), may be NULL
  * S_0 = 0.  L may be 0 (out untouched, final_state zeroed) and need not be a

@@ -40,9 +40,9 @@ int validate_fwd(int variant, int form, int dtype, int pairing, int phi, int win
     if (phi != FALCON_PHI_L2 && phi != FALCON_PHI_IDENTITY) return FALCON_ERR_ENUM;
     if (B < 0 || H < 0 || L < 0 || !dim_ok(d_k) || !dim_ok(d_v)) return FALCON_ERR_SHAPE;
     if (form == FALCON_CHUNK && !(chunk == 16 || chunk == 32 || chunk == 64)) {
-        // chunk 128: the tensor-core path of Falcon-1/1A with bf16 inputs and d = 64 only
+        // chunk 128: the tensor-core path of Falcon-1/1A with bf16 inputs and d_k = d_v <= 64 only
         const bool c128 = chunk == 128 && (variant == FALCON_F1 || variant == FALCON_F1A) &&
-                          dtype == FALCON_BF16 && d_k == 64 && d_v == 64;
+                          dtype == FALCON_BF16 && d_k == d_v && (d_k == 32 || d_k == 64);
         if (!c128) return FALCON_ERR_CHUNK;
     }
     return FALCON_OK;
@@ -379,7 +379,7 @@ extern "C" const char *falcon_status_string(int status) {
         case FALCON_ERR_ENUM: return "invalid variant, form, dtype, pairing or feature map";
         case FALCON_ERR_SHAPE: return "unsupported shape: B,H,L must be >= 0 and d_k,d_v in {16,32,64,128}";
         case FALCON_ERR_CHUNK:
-            return "chunk must be 16, 32 or 64 for the chunk-parallel form (128: Falcon-1/1A, bf16, d = 64)";
+            return "chunk must be 16, 32 or 64 for the chunk-parallel form (128: Falcon-1/1A, bf16, d = 32 or 64)";
         case FALCON_ERR_WINDOW: return "window must be in [1,8] for Falcon-3/3A";
         case FALCON_ERR_LAUNCH: return "kernel launch failed";
         case FALCON_ERR_ALLOC: return "stream-ordered scratch allocation failed";

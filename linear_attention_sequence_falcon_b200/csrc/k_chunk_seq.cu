@@ -1,6 +1,8 @@
 // k_chunk_seq.cu -- chunk-parallel forward of Falcon-1 and Falcon-1A (bf16
-// inputs, d_k = d_v = 64) for chunk lengths 16, 32 and 128, on the tensor
-// cores (TF32 warp MMAs on fp32 shared-memory tiles, fp32 accumulation).
+// inputs, d_k = d_v = d in {32, 64, 128}) for the chunk lengths the fused
+// kernel (d = 64, chunk 64) does not take: 16, 32, 64 and 128 (chunk 128 for
+// d <= 64), on the tensor cores (TF32 warp MMAs on fp32 shared-memory tiles,
+// fp32 accumulation).
 //
 // The chunk length is the pages' latency/memory knob ("start at chunk = 512
 // and measure the curve at 128/256/512/1024", page "Fast Weight Attention：
@@ -29,18 +31,18 @@ namespace falcon {
 
 namespace {
 
-constexpr int DD = 64;
-constexpr int LDX = 68;   // fp32 row stride of the C x 64 tiles
 constexpr int NTHS = 256;
 
-template <int C>
+template <int C, int DD>
 struct SeqLayout {
-    static constexpr int LDM = C + 4;  // row stride of the C x C tile
-    // X, Q, E (C x 64); MP: P o Dm in the lower triangle (diagonal included)
+    static constexpr int LDX = DD + 4;  // fp32 row stride of the C x d and d x d tiles
+    static constexpr int LDM = C + 4;   // row stride of the C x C tile
+    // X, Q, E (C x d); MP: P o Dm in the lower triangle (diagonal included)
     // and M transposed in the strict upper triangle (M[t][s] at [s][t]); S0
-    // (64 x 64); per-token vectors
+    // (d x d); per-token vectors
     static constexpr size_t X = 0, Q = X + (size_t)C * LDX, E = Q + (size_t)C * LDX, MP = E + (size_t)C * LDX,
                             S0 = MP + (size_t)C * LDM, VEC = S0 + (size_t)DD * LDX, total = VEC + 4 * C + 64;
+    static constexpr size_t bytes = total * sizeof(float);
 };
 
 // c (16 x 8 at rows r0, columns n0) += sum_{k < K} op(A)(r, k) op(B)(k, n),
@@ -75,10 +77,10 @@ __device__ __forceinline__ void each16x8(int r0, int n0, const float (&c)[4], Fn
 
 }  // namespace
 
-template <int C>
+template <int C, int DD>
 __global__ void __launch_bounds__(NTHS, 1) seq_chunk_kernel(FwdParams p) {
-    using Lo = SeqLayout<C>;
-    constexpr int LDM = Lo::LDM;
+    using Lo = SeqLayout<C, DD>;
+    constexpr int LDM = Lo::LDM, LDX = Lo::LDX, EPL = DD / 32;  // elements of a row per lane
     extern __shared__ float sm[];
     float *X = sm + Lo::X, *Q = sm + Lo::Q, *E = sm + Lo::E, *MP = sm + Lo::MP, *S0 = sm + Lo::S0;
     float *vG = sm + Lo::VEC, *veta = vG + C, *vw = veta + C, *vla = vw + C, *vsc = vla + C;
@@ -106,26 +108,29 @@ __global__ void __launch_bounds__(NTHS, 1) seq_chunk_kernel(FwdParams p) {
         for (int r = warp; r < C; r += NTHS / 32) {
             const int t = c0 + r, ki = p.pairing == 0 ? t - 1 : t;
             const bool carried = r < n && ki < 0 && p.x_prev != nullptr;  // x of a continued segment's first token
-            float x0 = 0.f, x1 = 0.f;
-            if (carried) {
-                x0 = p.x_prev[bh * DD + lane];
-                x1 = p.x_prev[bh * DD + lane + 32];
-            } else if (r < n && ki >= 0) {
-                x0 = __bfloat162float(kk[(size_t)ki * DD + lane]);
-                x1 = __bfloat162float(kk[(size_t)ki * DD + lane + 32]);
-            }
-            const float ss = group_sum<32>(x0 * x0 + x1 * x1);
-            const float inv = (p.phi != 0 || carried) ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
-            x0 *= inv;
-            x1 *= inv;
-            X[r * LDX + lane] = x0;
-            X[r * LDX + lane + 32] = x1;
-            const float sq = group_sum<32>(x0 * x0 + x1 * x1);
             const bool in = r < n;
-            Q[r * LDX + lane] = in ? __bfloat162float(kq[(size_t)t * DD + lane]) : 0.f;
-            Q[r * LDX + lane + 32] = in ? __bfloat162float(kq[(size_t)t * DD + lane + 32]) : 0.f;
-            E[r * LDX + lane] = in ? __bfloat162float(kv[(size_t)t * DD + lane]) : 0.f;
-            E[r * LDX + lane + 32] = in ? __bfloat162float(kv[(size_t)t * DD + lane + 32]) : 0.f;
+            float xv[EPL];
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+                const int cc = lane + 32 * e;
+                xv[e] = carried ? p.x_prev[bh * DD + cc]
+                                : (in && ki >= 0 ? __bfloat162float(kk[(size_t)ki * DD + cc]) : 0.f);
+                ss += xv[e] * xv[e];
+            }
+            ss = group_sum<32>(ss);
+            const float inv = (p.phi != 0 || carried) ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
+            float sq = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+                const int cc = lane + 32 * e;
+                const float x = xv[e] * inv;
+                sq += x * x;
+                X[r * LDX + cc] = x;
+                Q[r * LDX + cc] = in ? __bfloat162float(kq[(size_t)t * DD + cc]) : 0.f;
+                E[r * LDX + cc] = in ? __bfloat162float(kv[(size_t)t * DD + cc]) : 0.f;
+            }
+            sq = group_sum<32>(sq);
             if (lane == 0) {
                 float eta = 0.f, alpha = 1.f;
                 if (in) step_and_decay(__bfloat162float(kb[t]), sq, p.eps, lam, eta, alpha);
@@ -160,13 +165,13 @@ __global__ void __launch_bounds__(NTHS, 1) seq_chunk_kernel(FwdParams p) {
                 const int r0 = (tt / (C / 8)) * 16, n0 = (tt % (C / 8)) * 8;
                 if (n0 > r0 + 15) continue;  // strictly above the diagonal: masked out
                 float c[4] = {0.f, 0.f, 0.f, 0.f};
-                mma16x8<false, true>(Q, LDX, X, LDX, r0, n0, 64, c);
+                mma16x8<false, true>(Q, LDX, X, LDX, r0, n0, DD, c);
                 each16x8(r0, n0, c, [&](int t, int s, float v) {
                     if (s <= t) MP[t * LDM + s] = __expf(vG[t] - vG[s]) * veta[s] * v;
                 });
                 if (reg) {
                     float a[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma16x8<false, true>(X, LDX, X, LDX, r0, n0, 64, a);
+                    mma16x8<false, true>(X, LDX, X, LDX, r0, n0, DD, a);
                     each16x8(r0, n0, a, [&](int t, int s, float v) {
                         if (s < t) MP[s * LDM + t] = __expf(Gm1(t) - vG[s]) * veta[s] * v;
                     });
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(NTHS, 1) seq_chunk_kernel(FwdParams p) {
                 for (int tt = warp; tt < NXT; tt += NTHS / 32) {
                     const int r0 = (tt / (DD / 8)) * 16, n0 = (tt % (DD / 8)) * 8;
                     float c[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma16x8<false, true>(X, LDX, S0, LDX, r0, n0, 64, c);
+                    mma16x8<false, true>(X, LDX, S0, LDX, r0, n0, DD, c);
                     // E holds Y; every element read and written by this lane only
                     each16x8(r0, n0, c, [&](int t, int j, float v) { E[t * LDX + j] -= __expf(Gm1(t)) * v; });
                 }
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(NTHS, 1) seq_chunk_kernel(FwdParams p) {
             for (int tt = warp; tt < NOT; tt += NTHS / 32) {
                 const int r0 = (tt / (DD / 8)) * 16, n0 = (tt % (DD / 8)) * 8;
                 float c[4] = {0.f, 0.f, 0.f, 0.f};
-                mma16x8<false, true>(Q, LDX, S0, LDX, r0, n0, 64, c);
+                mma16x8<false, true>(Q, LDX, S0, LDX, r0, n0, DD, c);
                 const int lane_g = lane >> 2;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) c[e] *= __expf(vG[r0 + lane_g + (e >> 1) * 8]);
@@ -230,12 +235,13 @@ __global__ void __launch_bounds__(NTHS, 1) seq_chunk_kernel(FwdParams p) {
         }
         if (tid < C) vw[tid] = __expf(GC - vG[tid]) * veta[tid];
         __syncthreads();
-        // ---- S_end = e^{G_C} S0 + E^T D_w X (64 x 64, K = C)
+        // ---- S_end = e^{G_C} S0 + E^T D_w X (d x d, K = C)
         {
-            float c[4][4];
+            constexpr int NST = (DD / 16) * (DD / 8), PER = NST / (NTHS / 32);  // 16 x 8 tiles, per warp
+            float c[PER][4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int tt = warp * 4 + q, r0 = (tt / 8) * 16, n0 = (tt % 8) * 8;
+            for (int q = 0; q < PER; ++q) {
+                const int tt = warp * PER + q, r0 = (tt / (DD / 8)) * 16, n0 = (tt % (DD / 8)) * 8;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) c[q][e] = 0.f;
                 // A(j, s) = E[s][j] w_s: scale X's rows by w instead (B(s, i) = w_s X[s][i])
@@ -254,8 +260,8 @@ __global__ void __launch_bounds__(NTHS, 1) seq_chunk_kernel(FwdParams p) {
             __syncthreads();  // every warp has read S0 for O
             const float gc = __expf(GC);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int tt = warp * 4 + q, r0 = (tt / 8) * 16, n0 = (tt % 8) * 8;
+            for (int q = 0; q < PER; ++q) {
+                const int tt = warp * PER + q, r0 = (tt / (DD / 8)) * 16, n0 = (tt % (DD / 8)) * 8;
                 each16x8(r0, n0, c[q], [&](int j, int i, float v) { S0[j * LDX + i] = gc * S0[j * LDX + i] + v; });
             }
         }
@@ -266,34 +272,48 @@ __global__ void __launch_bounds__(NTHS, 1) seq_chunk_kernel(FwdParams p) {
 }
 
 bool seq_chunk_covers(const FwdParams &p) {
-    return (p.variant == F1 || p.variant == F1A) && p.dk == DD && p.dv == DD &&
-           (p.chunk == 16 || p.chunk == 32 || p.chunk == 128);
+    if (!(p.variant == F1 || p.variant == F1A) || p.dk != p.dv) return false;
+    if (!(p.dk == 32 || p.dk == 64 || p.dk == 128)) return false;
+    if (!(p.chunk == 16 || p.chunk == 32 || p.chunk == 64 || p.chunk == 128)) return false;
+    return !(p.chunk == 128 && p.dk == 128);  // 338 KB of shared memory
 }
 
 namespace {
 
-template <int C>
+template <int C, int DD>
 int launch_c(const FwdParams &p, cudaStream_t s) {
-    const size_t bytes = SeqLayout<C>::total * sizeof(float);
+    constexpr size_t bytes = SeqLayout<C, DD>::bytes;
+    static_assert(bytes <= 227 * 1024, "shared memory of one block");
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr[dev]) {
-        cudaFuncSetAttribute(seq_chunk_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        cudaFuncSetAttribute(seq_chunk_kernel<C, DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (dev >= 0 && dev < 64) attr[dev] = true;
     }
-    seq_chunk_kernel<C><<<(unsigned)(p.B * p.H), NTHS, bytes, s>>>(p);
+    seq_chunk_kernel<C, DD><<<(unsigned)(p.B * p.H), NTHS, bytes, s>>>(p);
     return 0;
+}
+
+template <int DD>
+int launch_d(const FwdParams &p, cudaStream_t s) {
+    switch (p.chunk) {
+        case 16: return launch_c<16, DD>(p, s);
+        case 32: return launch_c<32, DD>(p, s);
+        case 64: return launch_c<64, DD>(p, s);
+    }
+    return 1;
 }
 
 }  // namespace
 
 int launch_seq_chunk(const FwdParams &p, cudaStream_t s) {
     if (!seq_chunk_covers(p)) return 1;
-    switch (p.chunk) {
-        case 16: return launch_c<16>(p, s);
-        case 32: return launch_c<32>(p, s);
-        case 128: return launch_c<128>(p, s);
+    if (p.chunk == 128) return p.dk == 32 ? launch_c<128, 32>(p, s) : launch_c<128, 64>(p, s);
+    switch (p.dk) {
+        case 32: return launch_d<32>(p, s);
+        case 64: return launch_d<64>(p, s);
+        case 128: return launch_d<128>(p, s);
     }
     return 1;
 }

@@ -256,56 +256,10 @@ __device__ __forceinline__ void transpose4(uint32_t src, int rb, int cb0, uint32
 
 }  // namespace
 
-// The fused forward's hand-off between blocks (chunk_local_kernel<true>): a
-// ticket counter that hands units out in chunk-major order, per head the
-// number of chunks whose outgoing state is published (kPoison once a block
-// gave up), and a two-slot ring of fp32 states per head.
-struct ChainRing {
-    unsigned *ticket;
-    unsigned *done;
-    float *slots;  // [B*H][2][64][64]
-};
-constexpr unsigned kPoison = 0x80000000u;
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Waits until *done >= need; false when the head was poisoned or the wait
-// ran out (kWaitNs), which the caller turns into a give-up of its own.
-__device__ __noinline__ bool wait_done(const unsigned *done, unsigned need) {
-    const uint64_t t0 = tc::globaltimer_ns();
-    unsigned ns = 32;
-    while (true) {
-        const unsigned v = ld_acquire(done);
-        if (v & kPoison) return false;
-        if (v >= need) return true;
-        if (tc::globaltimer_ns() - t0 > kWaitNs) return false;
-        __nanosleep(ns);
-        if (ns < 1024) ns <<= 1;
-    }
-}
-
-// Persistent.  Two-kernel form (FUSED = false): block i computes units i,
-// i + gridDim.x, ... (unit = bh * nchunks + c) and leaves each chunk's image
-// for chunk_chain_kernel.  Fused form: units come from a ticket counter in
-// chunk-major order (unit = c * B*H + bh), and each unit also takes the
-// chain step itself: it waits (bounded) until its head's previous chunk has
-// published S_c, forms [S_c;S_c] [-Phi'^T;Qt]^T on the tensor core, writes
-// S_{c+1} to the head's ring slot, publishes it, and writes its outputs.  A
-// unit only ever waits for a smaller ticket, which a running block holds,
-// so the hand-off cannot deadlock.  Either way the inputs of the next unit
-// load while the block computes one.
-template <bool FUSED>
+// Persistent: block i computes units i, i + gridDim.x, ... (unit = bh *
+// nchunks + c), the inputs of its next unit loading while it computes one.
 __global__ void __launch_bounds__(NTH1, 2)
-    chunk_local_kernel(FwdParams p, const __grid_constant__ SplitMaps maps, uint8_t *img_ws, float *gc_ws,
-                       ChainRing ring) {
+    chunk_local_kernel(FwdParams p, const __grid_constant__ SplitMaps maps, uint8_t *img_ws, float *gc_ws) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = tc::smem_u32(smem_raw);
     uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -325,13 +279,7 @@ __global__ void __launch_bounds__(NTH1, 2)
     const bool reg = p.variant == F1;
     const int L = p.L;
     const int nch = (L + CH - 1) / CH;
-    const int BH = p.B * p.H;
-    const int units = BH * nch;
-    auto ubh_of = [&](int u) { return FUSED ? u % BH : u / nch; };
-    auto uc_of = [&](int u) { return FUSED ? u / BH : u % nch; };
-    // [2] the next unit, written by thread 0 before a barrier and read after
-    // it (the prologue's in slot 0, iteration n's in slot (n + 1) & 1)
-    unsigned *s_tick = reinterpret_cast<unsigned *>(sm + L_BAR + 32);
+    const int units = p.B * p.H * nch;
     LDBG_INIT();
     LBLK(0);
     LTIM(0);
@@ -340,7 +288,7 @@ __global__ void __launch_bounds__(NTH1, 2)
     // the prefix pair, key c0+t under the same-step pair; the key before the
     // sequence start and rows past its end read as zeros), q, v
     auto load_unit = [&](int u, int k) {
-        const int ubh = ubh_of(u), uc0 = uc_of(u) * CH;
+        const int ubh = u / nch, uc0 = (u - ubh * nch) * CH;
         const uint32_t o = sbase + (uint32_t)k * L_SET;
         tc::mbar_arrive_expect_tx(&tbar[k], 3 * TILE);
         tc::tma_load_3d(o, &maps.k, 0, p.pairing == 0 ? uc0 - 1 : uc0, ubh, &tbar[k]);
@@ -352,7 +300,7 @@ __global__ void __launch_bounds__(NTH1, 2)
         braw = __float2bfloat16_rn(0.f);
         lraw = 0.f;
         if (u >= units) return;
-        const int ubh = ubh_of(u), uc0 = uc_of(u) * CH;
+        const int ubh = u / nch, uc0 = (u - ubh * nch) * CH;
         // token t = tid / 4 on the first of the four threads of sample row t
         if ((tid & 3) == 0) {
             if (uc0 + (tid >> 2) < L) braw = static_cast<const __nv_bfloat16 *>(p.beta)[(size_t)ubh * L + uc0 + (tid >> 2)];
@@ -366,10 +314,8 @@ __global__ void __launch_bounds__(NTH1, 2)
         tc::mbar_init(&tbar[0], 1);
         tc::mbar_init(&tbar[1], 1);
         tc::fence_mbar_init();
-        const int first = FUSED ? (int)atomicAdd(ring.ticket, 1u) : (int)blockIdx.x;
-        s_tick[0] = (unsigned)first;
-        if (first < units) {
-            load_unit(first, 0);
+        if ((int)blockIdx.x < units) {
+            load_unit(blockIdx.x, 0);
             loads0 = 1;
         }
     }
@@ -378,13 +324,12 @@ __global__ void __launch_bounds__(NTH1, 2)
         tc::tmem_alloc(tmem_slot, TMEM1);
         tc::tmem_relinquish();
     }
+    __nv_bfloat16 beta_raw;
+    float lam_raw;
+    load_scalars(blockIdx.x, beta_raw, lam_raw);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const int u_first = (int)s_tick[0];
-    __nv_bfloat16 beta_raw;
-    float lam_raw;
-    load_scalars(u_first, beta_raw, lam_raw);
     const uint32_t tbase = *tmem_slot;
     const uint32_t tlane = tbase + ((uint32_t)(quarter * 32) << 16);  // this warp's lanes
     LTIM(1);
@@ -392,29 +337,26 @@ __global__ void __launch_bounds__(NTH1, 2)
     bool ok = true;
     uint32_t phase = 0;  // MMA-completion parity
     int n = 0;
-    int u = u_first, un = units;
-    for (; u < units; u = un, ++n) {
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
     const int set = n & 1;
     const uint32_t oX = (uint32_t)set * L_SET, oQ = oX + TILE, oV = oX + 2 * TILE;
     float *Zf = reinterpret_cast<float *>(sm + oX);  // inverse scratch over the consumed samples
+    const int un = u + gridDim.x;
     if (tid == 0) {
         // the previous image (the other set's tiles and B over M) has been
         // read out of shared memory: both may be written again
-        if (!FUSED) tc::bulk_wait_read();
-        const int nx = FUSED ? (int)atomicAdd(ring.ticket, 1u) : u + (int)gridDim.x;
-        s_tick[(n + 1) & 1] = (unsigned)nx;
-        if (nx < units) {
-            load_unit(nx, set ^ 1);
+        tc::bulk_wait_read();
+        if (un < units) {
+            load_unit(un, set ^ 1);
             if (set) ++loads0; else ++loads1;
         }
     }
-
-    ok = tc::mbar_wait_timeout(&tbar[set], (n >> 1) & 1, kWaitNs);
-    ok = __syncthreads_and(ok);
-    un = (int)s_tick[(n + 1) & 1];
     __nv_bfloat16 beta_next;
     float lam_next;
     load_scalars(un, beta_next, lam_next);
+
+    ok = tc::mbar_wait_timeout(&tbar[set], (n >> 1) & 1, kWaitNs);
+    ok = __syncthreads_and(ok);
     if (!ok) break;
     LTIM(2);
     {
@@ -424,13 +366,13 @@ __global__ void __launch_bounds__(NTH1, 2)
         {
             const int r = tid >> 2, part = tid & 3;
             // x of a continued segment's first token is the carried phi(k), as given
-            const bool carried = r == 0 && p.x_prev != nullptr && uc_of(u) == 0;
+            const bool carried = r == 0 && p.x_prev != nullptr && u % nch == 0;
             float xr[16];
             float ss = 0.f;
 #pragma unroll
             for (int c16 = 0; c16 < 2; ++c16) {
                 if (carried) {
-                    const float *xp = p.x_prev + (size_t)ubh_of(u) * DD + part * 16 + c16 * 8;
+                    const float *xp = p.x_prev + (size_t)(u / nch) * DD + part * 16 + c16 * 8;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) xr[c16 * 8 + e] = xp[e];
                 } else {
@@ -501,8 +443,7 @@ __global__ void __launch_bounds__(NTH1, 2)
             v_c[t] = __expf(Gt - Gr);
             v_b[t] = eta * __expf(Gr - Gt);
             if (t == 0) {
-                if (FUSED) v_sc[2] = __expf(GC);
-                else gc_ws[u] = __expf(GC);
+                gc_ws[u] = __expf(GC);
                 v_sc[1] = GC > kFactorMinLogDecay ? 1.f : 0.f;
             }
         } else if (warp >= 4) {
@@ -764,7 +705,7 @@ __global__ void __launch_bounds__(NTH1, 2)
         if (quarter < 2) {  // O0^T -> over T (bf16), B -> over [U0^T;W^T]; both [col/8][row][8]
             const int j = row;
 #pragma unroll
-            for (int part = 0; part < (FUSED ? 1 : 2); ++part) {  // (fused: B stays in tensor memory)
+            for (int part = 0; part < 2; ++part) {
                 const uint32_t dst = part ? L_MF : oV;
 #pragma unroll
                 for (int k2 = 0; k2 < 2; ++k2) {
@@ -780,7 +721,7 @@ __global__ void __launch_bounds__(NTH1, 2)
         tc::fence_proxy_async();  // staged image -> the bulk-copy engine
         __syncthreads();
         LTIM(12);
-        if (!FUSED && tid == 0) {
+        if (tid == 0) {
             uint8_t *dst = img_ws + (size_t)u * IMG;
             if (reg)
                 tc::bulk_store(dst, sbase + oX, 3 * TILE);  // -Phi'^T | Qt | O0^T
@@ -790,96 +731,6 @@ __global__ void __launch_bounds__(NTH1, 2)
             tc::bulk_commit();
         }
         LTIM(13);
-    }
-    if (FUSED && ok) {
-        // ---- the chain step of this unit: wait for S_c, then [S_c;S_c] [-Phi'^T;Qt]^T
-        //      (inner product: [S_c;S_c] Qt^T), S_{c+1} = g_C S_c - S_c Phi' + B, outputs
-        const int ubh = ubh_of(u), uc = uc_of(u);
-        bool go = true;
-        if (tid == 0 && uc > 0) go = wait_done(&ring.done[ubh], (unsigned)uc);
-        ok = __syncthreads_and(go);
-        float S[32];
-        if (ok && quarter < 2) {
-            // S_c row j, this thread's 32 columns: the ring slot (L2; another block wrote it),
-            // a continued segment's initial state, or zeros
-            const int j = row;
-            const float *src = uc > 0 ? ring.slots + (((size_t)ubh * 2 + (uc & 1)) * DD + j) * DD + chalf * 32
-                                      : (p.init_state ? p.init_state + ((size_t)ubh * DD + j) * DD + chalf * 32
-                                                      : nullptr);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-                const float4 v4 = src ? __ldcg(reinterpret_cast<const float4 *>(src) + q4)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-                S[q4 * 4] = v4.x; S[q4 * 4 + 1] = v4.y; S[q4 * 4 + 2] = v4.z; S[q4 * 4 + 3] = v4.w;
-            }
-            // its bf16 copy into both halves of the [S;S] operand, over [Y^T;(D_a X)^T]
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-                const uint4 u4 = pack8(&S[g8 * 8]);
-                *reinterpret_cast<uint4 *>(sm + L_XT + tc::sw128(j, chalf * 4 + g8)) = u4;
-                *reinterpret_cast<uint4 *>(sm + L_XT + TILE + tc::sw128(j, chalf * 4 + g8)) = u4;
-            }
-        }
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
-        ok = __syncthreads_and(ok);
-        if (ok) {
-            if (tid == ISSUER1) {
-                tc::fence_after_sync();
-                if (reg)
-                    issue_gemm(tbase, sbase + L_XT, sbase + oX, 128, false);  // [-S Phi' | (Qt S^T)^T]
-                else
-                    issue_gemm(tbase, sbase + L_XT, sbase + oQ, 64, false);   // (Qt S^T)^T
-                tc::mma_commit(bar);
-            }
-            ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
-            phase ^= 1;
-            ok = __syncthreads_and(ok);
-        }
-        if (ok) {
-            tc::fence_after_sync();
-            if (quarter < 2) {
-                const int j = row;
-                float bv[32], ds[32];
-                tc::tmem_ld32(tlane + C_G4 + 64 + chalf * 32, bv);  // B, fp32
-                if (reg) tc::tmem_ld32(tlane + chalf * 32, ds);      // -S_c Phi'
-                tc::tmem_wait_ld();
-                const float g = v_sc[2];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) S[i] = g * S[i] + (reg ? ds[i] : 0.f) + bv[i];
-                float *dst = uc + 1 < nch
-                                 ? ring.slots + (((size_t)ubh * 2 + ((uc + 1) & 1)) * DD + j) * DD + chalf * 32
-                                 : (p.final_state ? p.final_state + ((size_t)ubh * DD + j) * DD + chalf * 32 : nullptr);
-                if (dst) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4)
-                        __stcg(reinterpret_cast<float4 *>(dst) + q4,
-                               make_float4(S[q4 * 4], S[q4 * 4 + 1], S[q4 * 4 + 2], S[q4 * 4 + 3]));
-                }
-                tc::named_sync(3, 128);  // the four state warps' stores are issued
-                if (tid == 0) {
-                    __threadfence();
-                    st_release(&ring.done[ubh], (unsigned)(uc + 1));
-                }
-            } else {
-                // outputs of the chunk: O^T = (Qt S_c^T)^T + O0^T -> out[c0 + t][j]
-                const int j = row - 64;
-                float ov[32], o0[32];
-                tc::tmem_ld32(tlane + (reg ? 64 : 0) + chalf * 32, ov);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8)
-                    unpack8(*reinterpret_cast<const uint4 *>(sm + oV + rowmajor8(j, chalf * 4 + g8)), &o0[g8 * 8]);
-                const int c0 = uc * CH, nt = min(CH, L - c0);
-                __nv_bfloat16 *ko = static_cast<__nv_bfloat16 *>(p.out) + ((size_t)ubh * L + c0) * DD;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int t = chalf * 32 + i;
-                    if (t < nt) ko[(size_t)t * DD + j] = __float2bfloat16_rn(ov[i] + o0[i]);
-                }
-            }
-        }
-        LTIM(15);
     }
     if (!ok) break;
     beta_raw = beta_next;
@@ -892,10 +743,6 @@ __global__ void __launch_bounds__(NTH1, 2)
         tc::bulk_wait_read();  // the last images have been read out of shared memory
         if (!ok) {
             atomicAdd(&g_split_wait_timeouts, 1u);
-            if (FUSED) {  // the heads of this unit and of the one it prefetched get no state from here on
-                if (u < units) atomicOr(&ring.done[ubh_of(u)], kPoison);
-                if (un < units) atomicOr(&ring.done[ubh_of(un)], kPoison);
-            }
             // loads still in flight must land before the block leaves
             if (loads0 > 0) (void)tc::mbar_wait_timeout(&tbar[0], (loads0 - 1) & 1, kWaitNs);
             if (loads1 > 0) (void)tc::mbar_wait_timeout(&tbar[1], (loads1 - 1) & 1, kWaitNs);
@@ -1227,27 +1074,12 @@ bool split_chunk_covers(const FwdParams &p) {
     return (size_t)p.B * p.H * ((p.L + CH - 1) / CH) <= 0x7fffffffu;
 }
 
-size_t split_chunk_images_ws_bytes(const FwdParams &p) {
+size_t split_chunk_ws_bytes(const FwdParams &p) {
     const size_t units = (size_t)p.B * p.H * ((p.L + CH - 1) / CH);
     return units * IMG + units * sizeof(float);
 }
 
-namespace {
-
-size_t al256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
-
-// fused form: the ticket counter (256 bytes), the heads' published-chunk
-// counts, then the two-slot state ring of every head
-size_t fused_ws_bytes(const FwdParams &p) {
-    const size_t BH = (size_t)p.B * p.H;
-    return 256 + al256(BH * sizeof(unsigned)) + BH * 2 * DD * DD * sizeof(float);
-}
-
-}  // namespace
-
-size_t split_chunk_ws_bytes(const FwdParams &p) {
-    return p.states_out ? split_chunk_images_ws_bytes(p) : fused_ws_bytes(p);
-}
+size_t split_chunk_images_ws_bytes(const FwdParams &p) { return split_chunk_ws_bytes(p); }
 
 int launch_split_chunk(const FwdParams &p, cudaStream_t s) {
     auto al16 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
@@ -1263,35 +1095,17 @@ int launch_split_chunk(const FwdParams &p, cudaStream_t s) {
     const size_t units = (size_t)BH * nch;
     const int wrc = ws_acquire(p.ws_given, p.ws, p.ws_bytes, split_chunk_ws_bytes(p), s, &ws, &owned);
     if (wrc) return wrc;
+    uint8_t *img = static_cast<uint8_t *>(ws);
+    float *gc = reinterpret_cast<float *>(img + units * IMG);
     static bool attrs_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attrs_set[dev]) {
-        cudaFuncSetAttribute(chunk_local_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L_SMEM);
-        cudaFuncSetAttribute(chunk_local_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L_SMEM);
+        cudaFuncSetAttribute(chunk_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L_SMEM);
         cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_SMEM);
         if (dev >= 0 && dev < 64) attrs_set[dev] = true;
     }
-    const unsigned grid = (unsigned)std::min<size_t>(units, (size_t)2 * sm_count());
-    if (!p.states_out) {
-        // fused form: one kernel, the chain steps handed between blocks through the ring
-        uint8_t *b8 = static_cast<uint8_t *>(ws);
-        ChainRing ring;
-        ring.ticket = reinterpret_cast<unsigned *>(b8);
-        ring.done = reinterpret_cast<unsigned *>(b8 + 256);
-        ring.slots = reinterpret_cast<float *>(b8 + 256 + al256((size_t)BH * sizeof(unsigned)));
-        cudaError_t e = cudaMemsetAsync(b8, 0, 256 + al256((size_t)BH * sizeof(unsigned)), s);
-        if (e == cudaSuccess) {
-            chunk_local_kernel<true><<<grid, NTH1, L_SMEM, s>>>(p, maps, nullptr, nullptr, ring);
-            e = cudaGetLastError();
-        }
-        ws_release(ws, owned, s);
-        return e == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
-    }
-    // two-kernel form (the backward needs every chunk's image and entering state)
-    uint8_t *img = static_cast<uint8_t *>(ws);
-    float *gc = reinterpret_cast<float *>(img + units * IMG);
-    chunk_local_kernel<false><<<grid, NTH1, L_SMEM, s>>>(p, maps, img, gc, ChainRing{nullptr, nullptr, nullptr});
+    chunk_local_kernel<<<(unsigned)std::min<size_t>(units, (size_t)2 * sm_count()), NTH1, L_SMEM, s>>>(p, maps, img, gc);
     // the chain kernel as a programmatic dependent launch (see griddepcontrol in both kernels)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(BH);

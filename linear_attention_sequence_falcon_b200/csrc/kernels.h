@@ -21,8 +21,8 @@ template <typename T> int launch_span_masked(const FwdParams &p, cudaStream_t s)
 int launch_split_chunk(const FwdParams &p, cudaStream_t s);
 // true when the shape is one the split kernels take (pointer alignment aside)
 bool split_chunk_covers(const FwdParams &p);
-// the workspace of the call (the fused form's 3 MB-class ring, or with
-// states_out the two-kernel form's per-chunk images), and the latter alone
+// the workspace of the call: the per-chunk images and g_C (the backward
+// keeps them, through split_chunk_images_ws_bytes, for its reverse chain)
 size_t split_chunk_ws_bytes(const FwdParams &p);
 size_t split_chunk_images_ws_bytes(const FwdParams &p);
 // Number of tensor-core thread blocks that gave up on a bounded wait.

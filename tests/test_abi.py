@@ -57,7 +57,8 @@ def test_validation_codes(lib):
     assert _fwd(lib, chunk=100) == -4
     assert _fwd(lib, chunk=128, variant=1) == -4          # chunk 128: Falcon-1/1A only,
     assert _fwd(lib, chunk=128, dtype=0) == -4            # with bf16 inputs
-    assert _fwd(lib, chunk=128, dk=32, dv=32) == -4       # and d = 64
+    assert _fwd(lib, chunk=128, dk=128, dv=128) == -4     # and d = 32 or 64
+    assert _fwd(lib, chunk=128, dk=32, dv=64) == -4
     assert _fwd(lib, chunk=256) == -4
     assert _fwd(lib, variant=2, window=0) == -6
     assert _fwd(lib, variant=5, window=9) == -6
@@ -134,13 +135,9 @@ def test_workspace_size_query(lib):
     """The size query is host-only: the tensor-core chunk paths and the masked
     form need a workspace, every other path none."""
     lib.falcon_fwd_workspace_size.restype = ctypes.c_int
-    # Falcon-1/1A chunk 64, bf16, d = 64 (one fused kernel): a 256-byte ticket
-    # counter, one published-chunk count per head (padded to 256 bytes) and a
-    # two-slot fp32 state ring per head
-    BH = 8 * 12
-    fused = 256 + ((BH * 4 + 255) // 256) * 256 + BH * 2 * 64 * 64 * 4
-    assert _size(lib) == (0, fused)
-    assert _size(lib, variant=3) == (0, fused)
+    units = 8 * 12 * 32
+    assert _size(lib) == (0, units * 32 * 1024 + units * 4)          # Falcon-1 chunk, bf16, d = 64
+    assert _size(lib, variant=3) == (0, units * 32 * 1024 + units * 4)  # Falcon-1A
     assert _size(lib, dtype=0) == (0, 0)                              # fp32: the span kernel, no workspace
     assert _size(lib, chunk=32) == (0, 0)
     assert _size(lib, variant=1, B=4, H=16, L=4096, dk=128, dv=128) == (0, 0)  # Falcon-2: one block per head
