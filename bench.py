@@ -301,13 +301,18 @@ def run_ours(args):
               for var in w["variants"]}
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
+    # the caller-owned workspace of each forward (falcon_fwd_ws), allocated
+    # once: no stream-ordered allocation runs inside the timed region
+    ws = {var: torch.empty(F.fwd_workspace_size(var, "chunk", torch.bfloat16, w["B"], w["H"], w["L"], w["dk"],
+                                                w["dv"], chunk=w["chunk"]), dtype=torch.uint8, device="cuda")
+          for var in w["variants"]}
 
     def step(ev=None):
         for var in w["variants"]:
             if ev is not None:
                 ev[var][0].record(stream)
             F.fwd(var, "chunk", q, k, v, beta, lam, d["eps"], chunk=w["chunk"], out=outs[var],
-                  final_state=states[var], stream=stream)
+                  final_state=states[var], stream=stream, workspace=ws[var])
             if ev is not None:
                 ev[var][1].record(stream)
 
@@ -662,8 +667,8 @@ def run_backward(args):
         tok = B * H * L
         ab = tok * (dk + dk + dv + nb + dv) * 2 + tok * (dk + dk + dv + nb) * 4 + B * H * dv * dk * 4
         gbs = ab / (t / 1e3) / 1e9
-        kern = ("bwd_prep_kernel + chunk_local_kernel + chunk_chain_kernel + bwd_rchain_kernel + bwd_chunk_kernel"
-                " + bwd_decay_kernel + bwd_key_kernel" if args.bwd_form == "chunk" else
+        kern = ("chunk_local_kernel + chunk_chain_kernel + bwd_rchain_kernel + bwd_chunk_kernel"
+                if args.bwd_form == "chunk" else
                 "bwd_prep_kernel + bwd_sweep_kernel + bwd_decay_kernel + bwd_key_kernel")
         line = {"backward": var, "form": args.bwd_form, "workload": w["name"], "ms": t,
                 "tokens_per_s": B * L / (t / 1e3), "kernels": kern,

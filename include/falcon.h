@@ -111,7 +111,10 @@ enum {
  * multiple of `chunk`.  Three paths need a workspace, drawn stream-ordered
  * on `stream` from the device's current memory pool (FALCON_ERR_ALLOC if
  * that fails; falcon_fwd_ws takes it from the caller instead):
- * FALCON_MASKED (about B*H*L*(window*d_v+2*d_v) floats), the bf16
+ * FALCON_MASKED (about B*H*L*(window*d_v+2*d_v) floats on the CUDA cores;
+ * Falcon-1/1A with bf16 inputs, d_k = d_v = 64 and L <= 65536 run on the
+ * tensor cores, keeping 16 KiB per (b, h, 64-token block), and take the
+ * larger of the two so that misaligned pointers can fall back), the bf16
  * tensor-core chunk path of Falcon-1/1A with d_k = d_v = 64 and chunk 64
  * (32 KiB + 4 bytes per (b, h, chunk): the chunk-local results that the
  * second of its two kernels chains across chunks) and that of Falcon-2A
@@ -321,9 +324,12 @@ int falcon_bwd(falcon_variant variant, falcon_dtype dtype, falcon_pairing pairin
  *         cores) runs first and keeps the state entering every chunk; a
  *         reverse chain per head then carries dL/dS across chunk boundaries,
  *         G_c = g_C G_{c+1} - G_{c+1} Phi'_c^T + dO_c^T Qt_c, with the
- *         forward's per-chunk operators; every chunk's gradients then come at
+ *         forward's per-chunk operators; every chunk's gradients (through
+ *         the steps, the decays and the key normalisation too) then come at
  *         once from its inputs, its entering state and G_{c+1} (matrix form,
- *         TF32 tensor-core products, fp32 accumulation).  The inputs must be
+ *         TF32 tensor-core products with truncated operands, fp32
+ *         accumulation; dlambda summed with float atomics, so its last bits
+ *         may differ between runs).  q, k, v, dout, dq, dk and dv must be
  *         16-byte aligned (FALCON_ERR_UNSUPPORTED otherwise).
  *         FALCON_MASKED: FALCON_ERR_UNSUPPORTED.
  *   chunk 64 for FALCON_CHUNK; ignored otherwise
@@ -421,8 +427,12 @@ int falcon_decode_carry_from_prefill_ex(falcon_variant variant, falcon_dtype dty
  * memory budget.  falcon_fwd's masked form draws its scratch from
  * a stream-ordered pool; this one uses a fixed array of
  * FALCON_NOALLOC_SCRATCH_BYTES inside the library instead, which every GPU
- * that loads the library holds until the process exits.  Arguments, layouts
- * and results are those of falcon_fwd with form = FALCON_MASKED.
+ * that loads the library holds until the process exits.  Arguments and
+ * layouts are those of falcon_fwd with form = FALCON_MASKED; it always runs
+ * the CUDA-core masked kernel, so its results are bit for bit those of
+ * falcon_fwd's masked form wherever that form runs on the CUDA cores too
+ * (every shape but Falcon-1/1A with bf16 inputs and d_k = d_v = 64, which
+ * falcon_fwd runs on the tensor cores: equal there within rounding).
  *  - The problem must fit: B*H*L*(window_eff*d_v + 2*d_v) floats, window_eff
  *    = window for Falcon-3/3A and 1 otherwise, at most
  *    FALCON_NOALLOC_SCRATCH_BYTES/4; larger problems return

@@ -3,6 +3,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "../../include/falcon.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -68,7 +70,13 @@ FwdParams shape_params(int variant, int form, int pairing, int phi, int window, 
 // Falcon-2A at d = 128, chunk 64) and the masked-parallel form; 0 otherwise.
 size_t fwd_ws_need(const FwdParams &p, int dtype) {
     if ((size_t)p.B * p.H * p.L == 0) return 0;
-    if (p.form == FALCON_MASKED) return sizeof(float) * (masked_ws_r_floats(p) + 2 * masked_ws_eg_floats(p));
+    if (p.form == FALCON_MASKED) {
+        // the CUDA-core kernel's scratch; the tensor-core kernel (Falcon-1/1A,
+        // bf16, d = 64) takes its own, the larger of the two (misaligned
+        // pointers send that call to the CUDA-core kernel)
+        const size_t span = sizeof(float) * (masked_ws_r_floats(p) + 2 * masked_ws_eg_floats(p));
+        return dtype == FALCON_BF16 && masked_tc_covers(p) ? std::max(span, masked_tc_ws_bytes(p)) : span;
+    }
     if (p.form != FALCON_CHUNK || dtype != FALCON_BF16) return 0;
     if (split_chunk_covers(p)) return split_chunk_ws_bytes(p);
     if (pc_chunk_covers(p)) return pc_chunk_ws_bytes(p);
@@ -123,16 +131,21 @@ int fwd_impl(falcon_variant variant, falcon_form form, falcon_dtype dtype, falco
         }
         return launched(bf16 ? launch_span_chunk<__nv_bfloat16>(p, stream) : launch_span_chunk<float>(p, stream));
     }
-    // masked-parallel: scratch for the solved unknowns, the steps and Gamma
-    const size_t nr = masked_ws_r_floats(p), neg = masked_ws_eg_floats(p);
+    // masked-parallel: the tensor-core kernel (Falcon-1/1A, bf16, d = 64), else
+    // the CUDA-core kernel with scratch for the solved unknowns, the steps and Gamma
     void *ws = nullptr;
     bool owned = false;
-    rc = ws_acquire(ws_given, ws_ptr, ws_bytes, sizeof(float) * (nr + 2 * neg), stream, &ws, &owned);
+    rc = ws_acquire(ws_given, ws_ptr, ws_bytes, fwd_ws_need(p, dtype), stream, &ws, &owned);
     if (rc) return rc;
-    p.ws_r = static_cast<float *>(ws);
-    p.ws_eta = p.ws_r + nr;
-    p.ws_gam = p.ws_eta + neg;
-    rc = launched(bf16 ? launch_span_masked<__nv_bfloat16>(p, stream) : launch_span_masked<float>(p, stream));
+    int mrc = bf16 ? launch_masked_tc(p, ws, stream) : 1;
+    if (mrc == 1) {
+        const size_t nr = masked_ws_r_floats(p), neg = masked_ws_eg_floats(p);
+        p.ws_r = static_cast<float *>(ws);
+        p.ws_eta = p.ws_r + nr;
+        p.ws_gam = p.ws_eta + neg;
+        mrc = bf16 ? launch_span_masked<__nv_bfloat16>(p, stream) : launch_span_masked<float>(p, stream);
+    }
+    rc = launched(mrc);
     ws_release(ws, owned, stream);
     return rc;
 }
@@ -364,7 +377,8 @@ extern "C" int falcon_bwd_ws(falcon_variant variant, falcon_form form, falcon_dt
 
 extern "C" int falcon_device_wait_timeouts(unsigned int *count) {
     if (!count) return FALCON_ERR_NULL;
-    *count = split_wait_timeouts() + pc_wait_timeouts() + f2_wait_timeouts() + w_wait_timeouts();
+    *count = split_wait_timeouts() + pc_wait_timeouts() + f2_wait_timeouts() + w_wait_timeouts() +
+             masked_wait_timeouts();
     return cudaGetLastError() == cudaSuccess ? FALCON_OK : FALCON_ERR_LAUNCH;
 }
 

@@ -1167,17 +1167,15 @@ __global__ void __launch_bounds__(256, 1) bwd_sweep_reg_rsw_kernel(BwdParams p, 
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float *ns, const float *etas,
                                                        const float *alphas, const float *dga, const float *dgb,
-                                                       const float *dgx, float *deta) {
+                                                       float *deta) {
     constexpr int PER = 8, TS = 256 * PER;
     __shared__ float wsum[8];
     __shared__ float wlam[8];
     const int nch = (p.variant == F2A || p.variant == F2) ? p.dv : 1;
     const size_t bh = blockIdx.x / nch;
     const int ch = (int)(blockIdx.x % nch), L = p.L, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // the regression family's recurrent sweeps give dL/dalpha directly; the
-    // chunk-parallel backward (dgx != NULL) gives dL/dlog alpha whole in dga
-    const bool direct = dgx != nullptr;
-    const bool reg = (p.variant == F1 || p.variant == F2 || p.variant == F3) && !direct;
+    // the regression family's sweeps give dL/dalpha directly
+    const bool reg = p.variant == F1 || p.variant == F2 || p.variant == F3;
     const float lam = p.lambda[bh % p.H];
     const T *beta = static_cast<const T *>(p.beta) + bh * (size_t)L * nch;
     float carry = 0.f, dlam = 0.f;
@@ -1188,7 +1186,7 @@ __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float
         for (int k = 0; k < PER; ++k) {
             const int t = base + k;
             const size_t i = (bh * L + t) * nch + ch;
-            v[k] = (t < t1 && !reg && !direct) ? dga[i] - dgb[i] : 0.f;
+            v[k] = (t < t1 && !reg) ? dga[i] - dgb[i] : 0.f;
         }
         float run = 0.f;
 #pragma unroll
@@ -1220,7 +1218,7 @@ __global__ void __launch_bounds__(256) bwd_decay_kernel(BwdParams p, const float
             const size_t i = (bh * L + t) * nch + ch;
             const float a = alphas[i], eta = etas[i], n = ns[bh * L + t];
             // the regression family's sweep gives dL/dalpha directly
-            const float dalpha = reg ? dga[i] : direct ? dga[i] / a : (sfx[k] + later) / a;
+            const float dalpha = reg ? dga[i] : (sfx[k] + later) / a;
             float d = deta[i];
             if (1.f - eta * lam > kAlphaFloor) {
                 d -= lam * dalpha;
@@ -1345,9 +1343,7 @@ size_t bwd_ck_offset(const BwdParams &p) {
 size_t bwd_ws_bytes(const BwdParams &p) {
     const size_t BH = (size_t)p.B * p.H, ntile = (p.L + TT - 1) / TT;
     if (BH * p.L == 0) return 0;
-    if (bwd_chunk_covers(p))  // the per-token arrays, dgx, then the chunk path's own
-        return bwd_ck_offset(p) * sizeof(float) + ((BH * p.L * sizeof(float) + 255) & ~static_cast<size_t>(255)) +
-               bwd_chunk_ws_bytes(p);
+    if (bwd_chunk_covers(p)) return bwd_chunk_ws_bytes(p);
     const size_t nreg = regression(p.variant) ? BH * (ntile + TT) * p.dk * p.dk : 0;
     return (bwd_ck_offset(p) + nreg) * sizeof(float);
 }
@@ -1357,38 +1353,34 @@ int launch_bwd(const BwdParams &p, cudaStream_t s) {
     const int D = p.dk, nch = channels(p);
     const size_t rows = (size_t)p.B * p.H * p.L;
     if (rows == 0) return 0;
-    const size_t BH = (size_t)p.B * p.H, ntile = (p.L + TT - 1) / TT;
-    const size_t off_ck = bwd_ck_offset(p);
     void *ws = nullptr;
     bool owned = false;
     const int wrc = ws_acquire(p.ws_given, p.ws, p.ws_bytes, bwd_ws_bytes(p), s, &ws, &owned);
     if (wrc) return wrc;
+    if (p.dlambda) cudaMemsetAsync(p.dlambda, 0, sizeof(float) * p.H, s);
+    if (bwd_chunk_covers(p)) {
+        // chunk-parallel: every gradient comes from the per-chunk kernel
+        int rc = launch_bwd_chunk(p, ws, s);
+        if (rc == 1) rc = -9;  // FALCON_ERR_UNSUPPORTED: misaligned pointers
+        ws_release(ws, owned, s);
+        return rc;
+    }
+    const size_t BH = (size_t)p.B * p.H, ntile = (p.L + TT - 1) / TT;
     float *xs = static_cast<float *>(ws), *dx = xs + rows * D, *ns = dx + rows * D;
     float *etas = ns + rows, *alphas = etas + rows * nch, *dga = alphas + rows * nch, *dgb = dga + rows * nch;
     float *deta = dgb + rows * nch;
-    float *ck = xs + off_ck, *ts = ck + BH * ntile * D * D;
+    float *ck = xs + bwd_ck_offset(p), *ts = ck + BH * ntile * D * D;
     const unsigned wblocks = (unsigned)((rows * 32 + 255) / 256);
     bwd_prep_kernel<T><<<wblocks, 256, 0, s>>>(p, xs, ns, etas, alphas);
-    float *dgx = nullptr;
-    int rc;
-    if (bwd_chunk_covers(p)) {
-        // chunk-parallel: dgx after the per-token arrays, then the chunk path's workspace
-        dgx = xs + off_ck;
-        uint8_t *cws = reinterpret_cast<uint8_t *>(dgx) + ((rows * sizeof(float) + 255) & ~static_cast<size_t>(255));
-        rc = launch_bwd_chunk(p, cws, xs, etas, alphas, dga, dgb, dgx, deta, dx, s);
-        if (rc == 1) rc = -9;  // FALCON_ERR_UNSUPPORTED: the forward's tensor-core path refused the pointers
-    } else {
-        rc = D == 32 ? launch_sweep<T, 32>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
-           : D == 64 ? launch_sweep<T, 64>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
-                     : launch_sweep<T, 128>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s);
-    }
+    const int rc = D == 32 ? launch_sweep<T, 32>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
+                 : D == 64 ? launch_sweep<T, 64>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s)
+                           : launch_sweep<T, 128>(p, xs, etas, alphas, dga, dgb, deta, dx, ck, ts, s);
     if (rc != 0) {
         ws_release(ws, owned, s);
         return rc;
     }
     const size_t chans = (size_t)p.B * p.H * nch;
-    if (p.dlambda) cudaMemsetAsync(p.dlambda, 0, sizeof(float) * p.H, s);
-    bwd_decay_kernel<T><<<(unsigned)chans, 256, 0, s>>>(p, ns, etas, alphas, dga, dgb, dgx, deta);
+    bwd_decay_kernel<T><<<(unsigned)chans, 256, 0, s>>>(p, ns, etas, alphas, dga, dgb, deta);
     bwd_key_kernel<T><<<wblocks, 256, 0, s>>>(p, xs, deta, dx);
     const cudaError_t e = cudaGetLastError();
     ws_release(ws, owned, s);

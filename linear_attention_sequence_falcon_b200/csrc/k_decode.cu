@@ -170,13 +170,20 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
 // dot products need only log2(LPR) shuffle steps; 1/(eps+n), beta and the
 // shared sample are staged once per block, never per row.  A block serves
 // HPB (n,h) pairs so that the whole grid is resident at once (one wave).
+// (n,h) pairs and warps per block of decode1_kernel: at d = 128 one pair per
+// block of four warps (eight blocks per SM, so the blocks spread evenly over
+// the SMs), below two pairs per block of eight warps (four per SM); either
+// way the grid of the decode shapes is resident at once
+__host__ __device__ constexpr int decode1_hpb(int dk) { return dk >= 128 ? 1 : 2; }
+__host__ __device__ constexpr int decode1_warps(int dk) { return dk >= 128 ? 4 : 8; }
+
 template <typename T, int DK>
-__global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
-    constexpr int HPB = 2;
+__global__ void __launch_bounds__(32 * decode1_warps(DK), DK >= 128 ? 8 : 4) decode1_kernel(DecodeParams p) {
+    constexpr int HPB = decode1_hpb(DK);
     constexpr int LPR = DK >= 32 ? 8 : DK / 4;
     constexpr int NV4 = DK / (4 * LPR);  // float4 per lane per row
     constexpr int RPW = 32 / LPR;        // rows per warp per pass
-    constexpr int NW = 8;
+    constexpr int NW = decode1_warps(DK);
     __shared__ __align__(16) float xs[HPB][DK];
     __shared__ __align__(16) float qs[HPB][DK];
     __shared__ float ks[HPB][DK];
@@ -190,6 +197,22 @@ __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
     const int nh0 = blockIdx.x * HPB;
     const int nheads = min(HPB, nh_total - nh0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // below d = 128 the first row of the state is requested before anything
+    // else (the staging below then runs under its latency; at d = 128 the
+    // row's 16 registers would spill across the staging)
+    const int sl = lane % LPR, rsub = warp * RPW + lane / LPR;
+    const int total = nheads * dv, stride = NW * RPW;
+    float4 cur[NV4], nxt[NV4];
+    auto load_row = [&](int r, float4(&dst)[NV4]) {
+        if (r < total) {
+            const int hh = r / dv, row = r - hh * dv;
+            const float4 *Srow = reinterpret_cast<const float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
+#pragma unroll
+            for (int i = 0; i < NV4; ++i) dst[i] = Srow[sl + LPR * i];
+        }
+    };
+    if constexpr (NV4 <= 2) load_row(rsub, cur);
 
     // stage each pair's sample x = x_prev (prefix pair) or k, normalised
     // below (same-step pair), q, k, v and beta
@@ -244,20 +267,9 @@ __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
         __syncthreads();
     }
 
-    const int sl = lane % LPR, rsub = warp * RPW + lane / LPR;
-    const int total = nheads * dv, stride = NW * RPW;
     // the next row's state is loaded before this row is reduced, so two rows'
     // loads are in flight per lane (the step waits on HBM, not on issue)
-    float4 cur[NV4], nxt[NV4];
-    auto load_row = [&](int r, float4(&dst)[NV4]) {
-        if (r < total) {
-            const int hh = r / dv, row = r - hh * dv;
-            const float4 *Srow = reinterpret_cast<const float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
-#pragma unroll
-            for (int i = 0; i < NV4; ++i) dst[i] = Srow[sl + LPR * i];
-        }
-    };
-    load_row(rsub, cur);
+    if constexpr (NV4 > 2) load_row(rsub, cur);
     for (int r = rsub; r < total; r += stride) {
         load_row(r + stride, nxt);
         const int hh = r / dv, row = r - hh * dv;  // uniform across a row's lanes
@@ -303,6 +315,170 @@ __global__ void __launch_bounds__(256, 4) decode1_kernel(DecodeParams p) {
     }
 }
 
+// Window variants (Falcon-3/3A, W = 2..8 samples per update), laid out as
+// decode1_kernel: LPR lanes per row of S, HPB (n,h) pairs per block so the
+// whole grid is resident at once, and the first rows of the state requested
+// before the block stages its window.  Per row: W + 1 dot products (S_j.x_m,
+// S_j.q) reduced together, e_m = y_m - S_j.x_m (inner product: y_m), and
+// S_j <- alpha S_j + eta sum_m e_m x_m^T, o_j = alpha S_j.q + eta sum_m e_m (x_m.q).
+template <typename T, int DK, int W>
+__global__ void __launch_bounds__(256, 2) decodew_kernel(DecodeParams p) {
+    constexpr int HPB = 4;
+    constexpr int LPR = DK >= 32 ? 8 : DK / 4;
+    constexpr int NV4 = DK / (4 * LPR);  // float4 per lane per row
+    constexpr int RPW = 32 / LPR;        // rows per warp per pass
+    constexpr int NW = 8;
+    __shared__ __align__(16) float xs[HPB][W][DK];  // samples, oldest first; slot W-1 the current one
+    __shared__ __align__(16) float qs[HPB][DK];
+    __shared__ float ks[HPB][DK];
+    __shared__ float ys[HPB][W][128];
+    __shared__ float red[HPB][W + 1][2];  // per sample |x_m|^2 and x_m.q; then |k|^2
+    __shared__ float hsc[HPB][W + 3];     // eta, alpha, 1/|k|, x_m.q for m < W
+
+    const bool reg = variant_info(p.variant, W).regression;
+    const int nh_total = p.N * p.H, dv = p.dv;
+    const int nh0 = blockIdx.x * HPB;
+    const int nheads = min(HPB, nh_total - nh0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool same = p.pairing != 0;  // same-step pair: the current sample is (phi(k_t), v_t)
+
+    const int sl = lane % LPR, rsub = warp * RPW + lane / LPR;
+    const int total = nheads * dv, stride = NW * RPW;
+    float4 cur[NV4], nxt[NV4];
+    auto load_row = [&](int r, float4(&dst)[NV4]) {
+        if (r < total) {
+            const int hh = r / dv, row = r - hh * dv;
+            const float4 *Srow = reinterpret_cast<const float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
+#pragma unroll
+            for (int i = 0; i < NV4; ++i) dst[i] = Srow[sl + LPR * i];
+        }
+    };
+    load_row(rsub, cur);
+    load_row(rsub + stride, nxt);
+
+    // stage the window (oldest first), the current sample (x_prev, or k to be
+    // normalised under the same-step pair), q and k
+    for (int hh = 0; hh < nheads; ++hh) {
+        const int nh = nh0 + hh;
+        const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
+        const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
+        const T *v = static_cast<const T *>(p.v) + (size_t)nh * dv;
+        const float *xp = p.x_prev ? p.x_prev + (size_t)nh * DK : nullptr;
+        const float *win = p.win + (size_t)nh * (W - 1) * (DK + dv);
+        for (int i = threadIdx.x; i < DK; i += blockDim.x) {
+            const float kv = to_f32(k[i]);
+            qs[hh][i] = to_f32(q[i]);
+            ks[hh][i] = kv;
+            xs[hh][W - 1][i] = same ? kv : xp[i];
+        }
+        for (int i = threadIdx.x; i < dv; i += blockDim.x) ys[hh][W - 1][i] = to_f32(v[i]);
+        for (int i = threadIdx.x; i < (W - 1) * (DK + dv); i += blockDim.x) {
+            const int m = i / (DK + dv), c = i % (DK + dv);
+            const float val = win[i];
+            if (c < DK) xs[hh][m][c] = val; else ys[hh][m][c - DK] = val;
+        }
+    }
+    __syncthreads();
+    // one warp per (pair, sample): |x_m|^2 and x_m.q; job m = W: |k|^2
+    for (int job = warp; job < nheads * (W + 1); job += NW) {
+        const int hh = job / (W + 1), m = job % (W + 1);
+        const float *x = m < W ? xs[hh][m] : ks[hh];
+        float a = 0.f, b = 0.f;
+        for (int c = lane; c < DK; c += 32) {
+            a += x[c] * x[c];
+            b += x[c] * qs[hh][c];
+        }
+        a = group_sum<32>(a);
+        b = group_sum<32>(b);
+        if (lane == 0) { red[hh][m][0] = a; red[hh][m][1] = b; }
+    }
+    __syncthreads();
+    if (threadIdx.x < nheads) {
+        const int hh = threadIdx.x;
+        const float knorm = red[hh][W][0];
+        const float kinv = knorm > 0.f ? rsqrtf(knorm) : 0.f;
+        float n = 0.f;
+#pragma unroll
+        for (int m = 0; m < W; ++m) {
+            float e2 = red[hh][m][0], xq = red[hh][m][1];
+            if (same && m == W - 1) {  // x = k / |k|
+                e2 *= kinv * kinv;
+                xq *= kinv;
+            }
+            n += e2;
+            hsc[hh][3 + m] = xq;
+        }
+        const float lam = p.lambda[(nh0 + hh) % p.H];
+        float eta, alpha;
+        step_and_decay(to_f32(static_cast<const T *>(p.beta)[nh0 + hh]), n, p.eps, lam, eta, alpha);
+        hsc[hh][0] = eta;
+        hsc[hh][1] = alpha;
+        hsc[hh][2] = kinv;
+    }
+    __syncthreads();
+    if (same) {
+        for (int hh = 0; hh < nheads; ++hh)
+            for (int i = threadIdx.x; i < DK; i += blockDim.x) xs[hh][W - 1][i] *= hsc[hh][2];
+        __syncthreads();
+    }
+
+    for (int r = rsub; r < total; r += stride) {
+        const int hh = r / dv, row = r - hh * dv;  // uniform across a row's lanes
+        float4 *Srow = reinterpret_cast<float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
+        float sq = 0.f, sx[W];
+#pragma unroll
+        for (int m = 0; m < W; ++m) sx[m] = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) {
+            const float4 q4 = *reinterpret_cast<const float4 *>(&qs[hh][4 * (sl + LPR * i)]);
+            sq += cur[i].x * q4.x + cur[i].y * q4.y + cur[i].z * q4.z + cur[i].w * q4.w;
+            if (reg) {
+#pragma unroll
+                for (int m = 0; m < W; ++m) {
+                    const float4 x4 = *reinterpret_cast<const float4 *>(&xs[hh][m][4 * (sl + LPR * i)]);
+                    sx[m] += cur[i].x * x4.x + cur[i].y * x4.y + cur[i].z * x4.z + cur[i].w * x4.w;
+                }
+            }
+        }
+        sq = group_sum<LPR>(sq);
+        const float eta = hsc[hh][0], alpha = hsc[hh][1];
+        float ge[W], gq = 0.f;
+#pragma unroll
+        for (int m = 0; m < W; ++m) {
+            const float e = reg ? ys[hh][m][row] - group_sum<LPR>(sx[m]) : ys[hh][m][row];
+            ge[m] = eta * e;
+            gq += ge[m] * hsc[hh][3 + m];
+        }
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) {
+            float4 o;
+            o.x = alpha * cur[i].x; o.y = alpha * cur[i].y; o.z = alpha * cur[i].z; o.w = alpha * cur[i].w;
+#pragma unroll
+            for (int m = 0; m < W; ++m) {
+                const float4 x4 = *reinterpret_cast<const float4 *>(&xs[hh][m][4 * (sl + LPR * i)]);
+                o.x += ge[m] * x4.x; o.y += ge[m] * x4.y; o.z += ge[m] * x4.z; o.w += ge[m] * x4.w;
+            }
+            Srow[sl + LPR * i] = o;
+        }
+        if (sl == 0) static_cast<T *>(p.out)[(size_t)(nh0 + hh) * dv + row] = from_f32<T>(alpha * sq + gq);
+#pragma unroll
+        for (int i = 0; i < NV4; ++i) cur[i] = nxt[i];
+        load_row(r + 2 * stride, nxt);
+    }
+    // carry: x_prev <- phi(k_t); the window drops its oldest sample and
+    // appends the current one
+    for (int hh = 0; hh < nheads; ++hh) {
+        const int nh = nh0 + hh;
+        if (p.x_prev)
+            for (int i = threadIdx.x; i < DK; i += blockDim.x) p.x_prev[(size_t)nh * DK + i] = ks[hh][i] * hsc[hh][2];
+        float *win = p.win + (size_t)nh * (W - 1) * (DK + dv);
+        for (int i = threadIdx.x; i < (W - 1) * (DK + dv); i += blockDim.x) {
+            const int m = i / (DK + dv), c = i % (DK + dv);
+            win[i] = c < DK ? xs[hh][m + 1][c] : ys[hh][m + 1][c - DK];
+        }
+    }
+}
+
 template <typename T, int DK>
 __global__ void __launch_bounds__(128) carry_kernel(CarryParams p) {
     const VariantInfo vi = variant_info(p.variant, p.window);
@@ -335,12 +511,24 @@ __global__ void __launch_bounds__(128) carry_kernel(CarryParams p) {
     }
 }
 
+template <typename T, int DK, int W>
+static void launch_decodew(const DecodeParams &p, cudaStream_t s) {
+    decodew_kernel<T, DK, W><<<(p.N * p.H + 3) / 4, 256, 0, s>>>(p);
+}
+
 template <typename T, int DK>
 static void launch_decode_dk(const DecodeParams &p, cudaStream_t s) {
-    if (variant_info(p.variant, p.window).window == 1)
-        decode1_kernel<T, DK><<<(p.N * p.H + 1) / 2, 256, 0, s>>>(p);
-    else
-        decode_kernel<T, DK><<<p.N * p.H, 256, 0, s>>>(p);
+    switch (variant_info(p.variant, p.window).window) {
+        case 1: {
+            constexpr int hpb = decode1_hpb(DK);
+            decode1_kernel<T, DK><<<(p.N * p.H + hpb - 1) / hpb, 32 * decode1_warps(DK), 0, s>>>(p);
+            return;
+        }
+        case 2: launch_decodew<T, DK, 2>(p, s); return;
+        case 3: launch_decodew<T, DK, 3>(p, s); return;
+        case 4: launch_decodew<T, DK, 4>(p, s); return;
+        default: decode_kernel<T, DK><<<p.N * p.H, 256, 0, s>>>(p); return;  // windows 5-8
+    }
 }
 
 template <typename T>

@@ -1,0 +1,617 @@
+// k_masked_tc.cu -- the masked-parallel form of Falcon-1 and Falcon-1A on the
+// tcgen05 tensor cores (bf16 inputs, d_k = d_v = 64, S_0 = 0).
+//
+// Method: "masked-parallel: every step at once through a causal mask" (page
+// "Fast Weight Attention for Continual Learning", 方法/计算形式与数值稳定;
+// page "Fast Weight Attention：用于持续学习的快速权重注意力", 核心方法 3).  With
+// Gamma_t = sum_{r<=t} log alpha_r over the sequence, the regression family
+// solves the unrolled system
+//   r_t = y_t - sum_{s<t} e^{Gamma_{t-1}-Gamma_s} eta_s (x_t . x_s) r_s,
+//   o_t = sum_{s<=t} e^{Gamma_t-Gamma_s} eta_s (q_t . x_s) r_s
+// (inner product: r = y), and the final state is
+//   S_L = sum_s e^{Gamma_L-Gamma_s} eta_s r_s x_s^T.
+// No state is formed on the way: the kernel walks row blocks I of 64 tokens
+// in causal order and, for every earlier column block J, forms the pairwise
+// tiles [X_I; Q_I] X_J^T on the tensor core and applies them to the solved
+// residuals of block J:
+//   [R_I; O_I] -= / += gamma_IJ [X_I X_J^T; Q_I X_J^T] E~_J,
+// with E~_J = diag(e^{Gamma_Jend-Gamma_s} eta_s) r_J (kept, bf16, per block)
+// and gamma_IJ = e^{Gamma_{I0-1}-Gamma_Jend}.  The decay of a pair splits at
+// the block boundaries into a row factor e^{Gamma_{t-1}-Gamma_{I0-1}} (or
+// e^{Gamma_t-...}), gamma_IJ and the column factor, each <= 1.  The diagonal
+// block then solves its own triangle: R_I = Y_I - D_a (accumulated), E_I =
+// (I + M_II)^{-1} R_I, O_I = D_c (accumulated) + (P o Dm)_II E_I.
+//
+// One block per (b, h).  The pair products run on tcgen05 (bf16 operands in
+// 128-byte-swizzled shared memory, fp32 accumulators in tensor memory): P1 =
+// [X_I; Q_I] X_J^T into one of two accumulators while the previous pair's
+// P1 is scaled and rounded into the operand of P2 = [gA; gP] E~_J, which
+// accumulates [R; O] over J.  X_J and E~_J come back from the workspace by
+// bulk copies, each through a ring of four slots.  The diagonal block works on the
+// CUDA cores and the TF32 warp MMAs: T = (I + M_II)^{-1} from its 16 x 16
+// diagonal blocks (D) and K = D M_o, T = (I - K + K^2 - K^3) D.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_sm100.cuh"
+#include "warp_tf32.cuh"
+
+namespace falcon {
+
+namespace {
+
+constexpr int BM = 64;         // tokens per block; d_k = d_v = 64
+constexpr int NTHM = 256;
+constexpr int LDM = 72;        // fp32 row stride of the CUDA-core tiles
+constexpr int TFM = BM * LDM;  // floats per fp32 tile
+constexpr uint32_t TB = 8192;  // one bf16 64 x 64 tile (128-byte rows, 128-byte swizzle)
+constexpr int NRING = 4;       // slots of each operand ring
+constexpr int NGMAX = 1024;    // row blocks per sequence (L <= 65536)
+constexpr uint64_t kWaitNsM = 2000000000ull;  // bounded waits: two seconds
+
+// shared memory (bytes from a 1024-aligned base)
+constexpr uint32_t M_AQ = 0;                           // [X_I; Q_I] bf16: A of P1; rows 0-63 also B of the diagonal
+constexpr uint32_t M_RING = 2 * TB;                    // NRING slots of X_J bf16 (B of P1) ...
+constexpr uint32_t M_ERING = M_RING + NRING * TB;      // ... and NRING slots of E~_J^T bf16 (B of P2)
+constexpr uint32_t M_AOP = M_ERING + NRING * TB;       // two [gA; gP] bf16 operands of P2
+constexpr uint32_t M_LOOPEND = M_AOP + 2 * 2 * TB;
+constexpr uint32_t M_XF = M_LOOPEND;                   // fp32: X_I
+constexpr uint32_t M_YF = M_XF + TFM * 4;              // fp32: Y_I, then R_I, then E_I
+constexpr uint32_t M_MT = M_YF + TFM * 4;              // fp32: M_II (with the steps)
+constexpr uint32_t M_PD = M_MT + TFM * 4;              // fp32: (P o Dm)_II (with the steps)
+constexpr uint32_t M_OF = M_PD + TFM * 4;              // fp32: D_c (accumulated O)
+constexpr uint32_t M_ET = M_OF + TFM * 4;              // bf16: E~_I^T, staged for the workspace
+constexpr uint32_t M_VEC = M_ET + TB;                  // per-token vectors
+constexpr uint32_t M_GAM = M_VEC + 6 * BM * 4;        // gamma_IJ of the row block, J < I
+constexpr uint32_t M_BAR = M_GAM + NGMAX * 4;
+constexpr uint32_t M_SMEM = M_BAR + 128 + 1024;        // + alignment slack
+// the inverse's fp32 tiles D, K, K^2, T over the loop region (idle in the diagonal step)
+static_assert(4 * TFM * 4 <= M_LOOPEND - M_RING, "inverse scratch must fit over the pair buffers");
+static_assert(M_SMEM <= 227 * 1024, "shared memory of one block");
+// tensor memory: P1 accumulators at columns 0 and 64, [R; O] at 128
+constexpr uint32_t TM_COLS = 256, TM_P1 = 0, TM_ACC = 128;
+
+__device__ unsigned int g_masked_wait_timeouts;
+
+#ifdef FALCON_TC_DEBUG
+// block 0, threads 0 (the issuer) and 32: SM cycles per phase summed over the row blocks
+__device__ long long *g_masked_tim;
+#define MT_INIT()                    \
+    long long mt_acc_[16] = {0};     \
+    long long mt_prev_ = clock64();  \
+    const bool mt_on_ = blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == 32)
+#define MT(k)                                    \
+    do {                                         \
+        if (mt_on_) {                            \
+            const long long n_ = clock64();      \
+            mt_acc_[k] += n_ - mt_prev_;         \
+            mt_prev_ = n_;                       \
+        }                                        \
+    } while (0)
+#define MT_END()                                                                                    \
+    do {                                                                                            \
+        if (mt_on_ && g_masked_tim)                                                                 \
+            for (int i_ = 0; i_ < 16; ++i_) g_masked_tim[(threadIdx.x ? 16 : 0) + i_] = mt_acc_[i_]; \
+    } while (0)
+#else
+#define MT_INIT()
+#define MT(k)
+#define MT_END()
+#endif
+
+// D = A B^T over K = 64 (four K=16 slices), both operands K-major and
+// 128-byte swizzled; M = 128, N = 64.
+__device__ __forceinline__ void issue_128x64(uint32_t d_tmem, uint32_t a_saddr, uint32_t b_saddr, bool accumulate) {
+    const uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = tc::sdesc_sw128(a_saddr + kk * 32, 16, 1024);
+        const uint64_t bd = tc::sdesc_sw128(b_saddr + kk * 32, 16, 1024);
+        tc::mma_bf16(d_tmem, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+template <bool TA, bool TB, bool SK = false>
+__device__ __forceinline__ void mma64(const float *A, const float *B, float (&acc)[4][4], int kb, int ke,
+                                      const float *sk = nullptr) {
+    wt::mma64<LDM, TA, TB, SK>(A, B, acc, kb, ke, sk);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(NTHM, 1)
+    masked_tc_kernel(FwdParams p, uint8_t *xs_ws, uint8_t *es_ws, float *gend_ws) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = tc::smem_u32(smem_raw);
+    uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sb = tc::smem_u32(sm);
+    float *XF = reinterpret_cast<float *>(sm + M_XF), *YF = reinterpret_cast<float *>(sm + M_YF);
+    float *MT = reinterpret_cast<float *>(sm + M_MT), *PD = reinterpret_cast<float *>(sm + M_PD);
+    float *OF = reinterpret_cast<float *>(sm + M_OF);
+    float *DI = reinterpret_cast<float *>(sm + M_RING), *KI = DI + TFM, *K2 = KI + TFM, *TI = K2 + TFM;
+    float *vec = reinterpret_cast<float *>(sm + M_VEC);
+    float *vG = vec, *veta = vec + BM, *vla = vec + 2 * BM, *va = vec + 3 * BM, *vc = vec + 4 * BM,
+          *vb = vec + 5 * BM;
+    float *vgam = reinterpret_cast<float *>(sm + M_GAM);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + M_BAR);
+    uint64_t *txb = bar, *teb = bar + NRING, *bp1 = bar + 2 * NRING, *bp2 = bp1 + 2, *bd = bp2 + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bd + 1);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int quarter = warp & 3, chalf = warp >> 2;
+    const int row = quarter * 32 + lane;  // tensor-memory lane of this thread
+    const bool reg = p.variant == F1;
+    const int L = p.L, nb = (L + BM - 1) / BM;
+    const size_t bh = blockIdx.x;
+    const float lam = p.lambda[bh % p.H];
+    const __nv_bfloat16 *kh = static_cast<const __nv_bfloat16 *>(p.k) + bh * (size_t)L * BM;
+    const __nv_bfloat16 *qh = static_cast<const __nv_bfloat16 *>(p.q) + bh * (size_t)L * BM;
+    const __nv_bfloat16 *vh = static_cast<const __nv_bfloat16 *>(p.v) + bh * (size_t)L * BM;
+    const __nv_bfloat16 *bth = static_cast<const __nv_bfloat16 *>(p.beta) + bh * (size_t)L;
+    __nv_bfloat16 *oh = static_cast<__nv_bfloat16 *>(p.out) + bh * (size_t)L * BM;
+    uint8_t *xs = xs_ws + bh * (size_t)nb * TB;
+    uint8_t *es = es_ws + bh * (size_t)nb * TB;
+    float *gend = gend_ws + bh * (size_t)nb;
+
+    if (tid == 0) {
+        for (int i = 0; i < 2 * NRING + 5; ++i) tc::mbar_init(&bar[i], 1);
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, TM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tlane = tbase + ((uint32_t)(quarter * 32) << 16);
+
+    // completion counts: every thread tracks the MMA barriers alike; thread 0
+    // alone tracks the rings (loads issued and consumed per slot)
+    uint32_t n1[2] = {0u, 0u}, n2[2] = {0u, 0u}, ndg = 0u;
+    uint32_t lx[NRING] = {0u, 0u, 0u, 0u}, cx[NRING] = {0u, 0u, 0u, 0u};
+    uint32_t le[NRING] = {0u, 0u, 0u, 0u}, ce[NRING] = {0u, 0u, 0u, 0u};
+    bool ok = true;
+    float Gprev = 0.f;  // Gamma_{I0-1}
+    MT_INIT();
+    float sacc[4][4];   // S (this warp's 16 x 32 block), e^{...} relative to the last block's end
+    wt::zero(sacc);
+
+    // thread 0: X_J into its ring slot, E~_J^T into its own; the waits for them
+    auto load_x = [&](int J) {
+        const int s = J % NRING;
+        tc::mbar_arrive_expect_tx(&txb[s], TB);
+        tc::bulk_load(sb + M_RING + (uint32_t)s * TB, xs + (size_t)J * TB, TB, &txb[s]);
+        ++lx[s];
+    };
+    auto load_e = [&](int J) {
+        const int s = J % NRING;
+        tc::mbar_arrive_expect_tx(&teb[s], TB);
+        tc::bulk_load(sb + M_ERING + (uint32_t)s * TB, es + (size_t)J * TB, TB, &teb[s]);
+        ++le[s];
+    };
+    auto wait_x = [&](int J) {
+        const int s = J % NRING;
+        const bool r = tc::mbar_wait_timeout(&txb[s], cx[s] & 1u, kWaitNsM);
+        ++cx[s];
+        return r;
+    };
+    auto wait_e = [&](int J) {
+        const int s = J % NRING;
+        const bool r = tc::mbar_wait_timeout(&teb[s], ce[s] & 1u, kWaitNsM);
+        ++ce[s];
+        return r;
+    };
+    auto issue_p1 = [&](int J) {  // P1(J) = [X_I; Q_I] X_J^T into accumulator J & 1
+        issue_128x64(tbase + TM_P1 + (uint32_t)(J & 1) * 64, sb + M_AQ, sb + M_RING + (uint32_t)(J % NRING) * TB,
+                     false);
+        tc::mma_commit(&bp1[J & 1]);
+    };
+
+    for (int I = 0; I < nb; ++I) {
+        const int I0 = I * BM, n = min(BM, L - I0);
+        // ---- the block's inputs: samples x_t = phi(k_{t-1}) (prefix pair;
+        //      phi(k_t) same-step), q, v, the steps and the decays
+        if (tid == 0) tc::bulk_wait_read();  // the stores of the last block have read AQ and ET
+        __syncthreads();
+        {
+            uint4 lq[2], lv[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int e = tid + NTHM * j;  // 16-byte piece: row e / 8, columns 8 (e % 8)..
+                const bool in = (e >> 3) < n;
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                lq[j] = in ? wt::ld16(qh + (size_t)I0 * BM + 8 * e) : z;
+                lv[j] = in ? wt::ld16(vh + (size_t)I0 * BM + 8 * e) : z;
+            }
+            uint32_t kw[8];
+            float bv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = warp * 8 + i, t = I0 + r, kr = p.pairing == 0 ? t - 1 : t;
+                kw[i] = (r < n && kr >= 0) ? *reinterpret_cast<const uint32_t *>(kh + (size_t)kr * BM + 2 * lane) : 0u;
+                bv[i] = r < n ? __bfloat162float(bth[t]) : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = warp * 8 + i;
+                const float x0 = __uint_as_float(kw[i] << 16), x1 = __uint_as_float(kw[i] & 0xffff0000u);
+                const float ss = group_sum<32>(x0 * x0 + x1 * x1);
+                const float inv = p.phi != 0 ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
+                const float y0 = x0 * inv, y1 = x1 * inv;
+                *reinterpret_cast<float2 *>(XF + r * LDM + 2 * lane) = make_float2(y0, y1);
+                *reinterpret_cast<uint32_t *>(sm + M_AQ + tc::sw128(r, lane >> 2) + (lane & 3) * 4) = pack2(y0, y1);
+                if (lane == 0) {
+                    const float nn = ss * inv * inv;  // the sample's energy (0: no sample)
+                    float eta = 0.f, alpha = 1.f;
+                    if (r < n) step_and_decay(bv[i], nn, p.eps, lam, eta, alpha);
+                    veta[r] = eta;
+                    vla[r] = __logf(alpha);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int e = tid + NTHM * j, r = e >> 3, c = e & 7;
+                *reinterpret_cast<uint4 *>(sm + M_AQ + tc::sw128(64 + r, c)) = lq[j];
+                wt::st8(YF + r * LDM + 8 * c, lv[j]);
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {  // block-local cumulative log decay G_t
+            float la[2] = {vla[lane], vla[lane + 32]};
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const float y = __shfl_up_sync(0xffffffffu, la[h2], o);
+                    if (lane >= o) la[h2] += y;
+                }
+            }
+            la[1] += __shfl_sync(0xffffffffu, la[0], 31);
+            vG[lane] = la[0];
+            vG[lane + 32] = la[1];
+        }
+        __syncthreads();
+        const float GE = vG[BM - 1];
+        if (tid < BM) {
+            const int t = tid;
+            va[t] = __expf(t > 0 ? vG[t - 1] : 0.f);   // e^{Gamma_{t-1} - Gamma_{I0-1}}
+            vc[t] = __expf(vG[t]);                      // e^{Gamma_t - Gamma_{I0-1}}
+            vb[t] = __expf(GE - vG[t]) * veta[t];       // e^{Gamma_Iend - Gamma_t} eta_t
+        }
+        if (tid == 0) gend[I] = Gprev + GE;
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        if (tid == 0) {  // X_I for the later row blocks
+            tc::bulk_store(xs + (size_t)I * TB, sb + M_AQ, TB);
+            tc::bulk_commit();
+        }
+        MT(0);
+
+        // ---- the pairs (I, J < I).  P1 runs two pairs ahead of the pair whose
+        //      operand is being formed; X_J is loaded four pairs ahead, E~_J three
+        if (I > 0) {
+            if (tid == 0) {
+                // every earlier X_J and E~_J has landed in the workspace (the
+                // store of X_I, the newest group, may still be in flight)
+                asm volatile("cp.async.bulk.wait_group 1;" ::: "memory");
+                for (int J = 0; J < min(NRING, I); ++J) load_x(J);
+                for (int J = 0; J < min(NRING - 1, I); ++J) load_e(J);
+                bool r = wait_x(0);
+                if (r) issue_p1(0);
+                if (r && I > 1) {
+                    r = wait_x(1);
+                    if (r) issue_p1(1);
+                }
+                ok = r;
+            }
+            for (int J = tid; J < I; J += NTHM) vgam[J] = __expf(Gprev - gend[J]);
+            ok = __syncthreads_and(ok);
+            MT(1);
+            for (int J = 0; J < I && ok; ++J) {
+                const int b = J & 1;
+                // P1(J) -> this thread's 32 columns of its lane
+                bool w = tc::mbar_wait_timeout(&bp1[b], n1[b] & 1u, kWaitNsM);
+                ++n1[b];
+                __syncwarp();
+                tc::fence_after_sync();
+                float v[32];
+                tc::tmem_ld32(tlane + TM_P1 + b * 64 + chalf * 32, v);
+                tc::tmem_wait_ld();
+                MT(2);
+                // [gA; gP] of this pair into operand b once P2(J-2) has read it
+                const float g = vgam[J];
+                if (J >= 2) {
+                    w = tc::mbar_wait_timeout(&bp2[b], n2[b] & 1u, kWaitNsM) && w;
+                    ++n2[b];
+                }
+                const uint32_t aop = M_AOP + (uint32_t)b * 2 * TB;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint4 u;
+                    u.x = pack2(g * v[c4 * 8 + 0], g * v[c4 * 8 + 1]);
+                    u.y = pack2(g * v[c4 * 8 + 2], g * v[c4 * 8 + 3]);
+                    u.z = pack2(g * v[c4 * 8 + 4], g * v[c4 * 8 + 5]);
+                    u.w = pack2(g * v[c4 * 8 + 6], g * v[c4 * 8 + 7]);
+                    *reinterpret_cast<uint4 *>(sm + aop + tc::sw128(row, chalf * 4 + c4)) = u;
+                }
+                tc::fence_proxy_async();
+                tc::fence_before_sync();
+                MT(3);
+                // every thread has read accumulator b and written operand b
+                ok = __syncthreads_and(w && ok);
+                if (!ok) break;
+                tc::fence_after_sync();
+                MT(4);
+                if (tid == 0) {
+                    // P2(J): [R; O] += [gA; gP] E~_J
+                    bool r = wait_e(J);
+                    if (r) {
+                        issue_128x64(tbase + TM_ACC, sb + aop, sb + M_ERING + (uint32_t)(J % NRING) * TB, J > 0);
+                        tc::mma_commit(&bp2[b]);
+                    }
+                    // P1(J+2) into accumulator b, read out above
+                    if (r && J + 2 < I) {
+                        r = wait_x(J + 2);
+                        if (r) issue_p1(J + 2);
+                    }
+                    // X_{J+4} into the slot of X_J (P1(J) is done)
+                    if (r && J + NRING < I) load_x(J + NRING);
+                    // E~_{J+3} into the slot of E~_{J-1} once P2(J-1) is done: the
+                    // newest product of accumulator b ^ 1, waited on here without
+                    // consuming the completion the other threads count
+                    if (r && J + NRING - 1 < I) {
+                        if (J >= 1) r = tc::mbar_wait_timeout(&bp2[b ^ 1], n2[b ^ 1] & 1u, kWaitNsM);
+                        if (r) load_e(J + NRING - 1);
+                    }
+                    if (!r) ok = false;
+                }
+                MT(5);
+            }
+            if (ok) {
+                // the last two P2 (the others have been counted)
+                for (int J = max(0, I - 2); J < I && ok; ++J) {
+                    const int b = J & 1;
+                    ok = tc::mbar_wait_timeout(&bp2[b], n2[b] & 1u, kWaitNsM);
+                    ++n2[b];
+                }
+            }
+            ok = __syncthreads_and(ok);
+            if (!ok) break;
+            MT(6);
+        }
+
+        // ---- the diagonal block: [A_II; P_II] = [X_I; Q_I] X_I^T
+        if (tid == 0) {
+            tc::fence_after_sync();
+            issue_128x64(tbase + TM_P1, sb + M_AQ, sb + M_AQ, false);
+            tc::mma_commit(bd);
+        }
+        {
+            const bool w = tc::mbar_wait_timeout(bd, ndg & 1u, kWaitNsM);
+            ++ndg;
+            ok = __syncthreads_and(w);
+            if (!ok) break;
+        }
+        tc::fence_after_sync();
+        {
+            float v[32], r[32];
+            tc::tmem_ld32(tlane + TM_P1 + chalf * 32, v);
+            if (I > 0) tc::tmem_ld32(tlane + TM_ACC + chalf * 32, r);
+            tc::tmem_wait_ld();
+            if (I == 0) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = 0.f;
+            }
+            if (quarter < 2) {  // rows 0-63 (regression): M_II (with the steps), R = Y - D_a (accumulated)
+                if (reg) {
+                    const int t = row;
+                    const float gm = t > 0 ? vG[t - 1] : 0.f, a = va[t];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int s = chalf * 32 + i;
+                        MT[t * LDM + s] = s < t ? __expf(gm - vG[s]) * veta[s] * v[i] : 0.f;
+                        YF[t * LDM + s] -= a * r[i];
+                    }
+                }
+            } else {  // rows 64-127: (P o Dm)_II (with the steps) and D_c (accumulated)
+                const int t = row - 64;
+                const float gt = vG[t], c = vc[t];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int s = chalf * 32 + i;
+                    PD[t * LDM + s] = s <= t ? __expf(gt - vG[s]) * veta[s] * v[i] : 0.f;
+                    OF[t * LDM + s] = c * r[i];
+                }
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        MT(7);
+        const int rb = (warp & 3) * 16, cb = (warp >> 2) * 32;
+        float acc[4][4];
+        if (reg) {
+            // ---- T = (I + M_II)^{-1}: D, the diagonal 16 x 16 blocks' inverses
+            //      (one column of a block per thread, threads 0-63); zeros elsewhere
+            if (tid < 64) {
+                const int o = (tid >> 4) * 16, j = tid & 15;
+                float col[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float s = i == j ? 1.f : 0.f;
+#pragma unroll
+                    for (int s2 = 0; s2 < i; ++s2) s -= MT[(o + i) * LDM + o + s2] * col[s2];
+                    col[i] = s;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) DI[(o + i) * LDM + o + j] = col[i];
+            } else {
+                for (int e = tid - 64; e < BM * BM; e += NTHM - 64) {
+                    const int r2 = e >> 6, s = e & 63;
+                    if ((r2 >> 4) != (s >> 4)) DI[r2 * LDM + s] = 0.f;
+                }
+            }
+            __syncthreads();
+            // K = D M_o: D M on the blocks below the diagonal (D reads its own block only)
+            wt::zero(acc);
+            mma64<false, false>(DI, MT, acc, rb, rb + 16);
+            wt::each(acc, [&](int r2, int s, float &val) { KI[r2 * LDM + s] = (s >> 4) < (r2 >> 4) ? val : 0.f; });
+            __syncthreads();
+            wt::zero(acc);
+            if (rb > 0) mma64<false, false>(KI, KI, acc, 0, rb);
+            wt::each(acc, [&](int r2, int s, float &val) { K2[r2 * LDM + s] = val; });
+            __syncthreads();
+            wt::zero(acc);
+            if (rb > 0) mma64<false, false>(KI, K2, acc, 0, rb);
+            wt::each(acc, [&](int r2, int s, float &val) {
+                TI[r2 * LDM + s] = (r2 == s ? 1.f : 0.f) - KI[r2 * LDM + s] + K2[r2 * LDM + s] - val;
+            });
+            __syncthreads();
+            // T = (I - K + K^2 - K^3) D: each warp reads only the block of the sum it writes
+            wt::zero(acc);
+            {
+                const int ke = min(cb + 32, rb + 16);
+                if (ke > cb) mma64<false, false>(TI, DI, acc, cb, ke);
+            }
+            __syncwarp();
+            wt::each(acc, [&](int r2, int s, float &val) { TI[r2 * LDM + s] = val; });
+            __syncthreads();
+            // E = T R (T lower: k <= r)
+            wt::zero(acc);
+            mma64<false, false>(TI, YF, acc, 0, rb + 16);
+            __syncthreads();
+            wt::each(acc, [&](int r2, int j, float &val) { YF[r2 * LDM + j] = val; });
+            __syncthreads();
+        }
+        MT(8);
+        // ---- O_I = D_c (accumulated) + (P o Dm)_II E_I
+        wt::zero(acc);
+        mma64<false, false>(PD, YF, acc, 0, rb + 16);
+        {
+            const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int r2 = rb + g + 8 * h2, j = cb + nt * 8 + 2 * t4;
+                    if (r2 < n) {
+                        const float o0 = acc[nt][2 * h2] + OF[r2 * LDM + j];
+                        const float o1 = acc[nt][2 * h2 + 1] + OF[r2 * LDM + j + 1];
+                        *reinterpret_cast<uint32_t *>(oh + (size_t)(I0 + r2) * BM + j) = pack2(o0, o1);
+                    }
+                }
+        }
+        // ---- E~_I^T (bf16, swizzled: row j holds b_s E[s][j] over s) for the later
+        //      row blocks, and S <- e^{G_Iend} S + E~_I^T X_I
+        {
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int e = tid + NTHM * k2, j = e >> 3, c = e & 7;
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = vb[8 * c + i] * YF[(8 * c + i) * LDM + j];
+                uint4 u;
+                u.x = pack2(f[0], f[1]);
+                u.y = pack2(f[2], f[3]);
+                u.z = pack2(f[4], f[5]);
+                u.w = pack2(f[6], f[7]);
+                *reinterpret_cast<uint4 *>(sm + M_ET + tc::sw128(j, c)) = u;
+            }
+            const float gI = __expf(GE);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc[nt][e] *= gI;
+            mma64<true, false, true>(YF, XF, sacc, 0, 64, vb);
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            tc::bulk_store(es + (size_t)I * TB, sb + M_ET, TB);
+            tc::bulk_commit();
+        }
+        Gprev += GE;
+        MT(9);
+    }
+
+    MT_END();
+    if (p.final_state && ok)
+        wt::each(sacc, [&](int j, int i, float &val) { p.final_state[(bh * BM + j) * BM + i] = val; });
+    if (tid == 0) {
+        tc::bulk_wait_all();
+        if (!ok) {
+            atomicAdd(&g_masked_wait_timeouts, 1u);
+            // loads still in flight must land before the block leaves
+            for (int s = 0; s < NRING; ++s) {
+                if (lx[s] > cx[s]) (void)tc::mbar_wait_timeout(&txb[s], (lx[s] - 1u) & 1u, kWaitNsM);
+                if (le[s] > ce[s]) (void)tc::mbar_wait_timeout(&teb[s], (le[s] - 1u) & 1u, kWaitNsM);
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, TM_COLS);
+}
+
+// ------------------------------------------------------------ launcher
+namespace {
+
+size_t al256m(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+bool al16m(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+bool masked_tc_covers(const FwdParams &p) {
+    return (p.variant == F1 || p.variant == F1A) && p.dk == BM && p.dv == BM && p.form == 1 && p.L > 0 &&
+           (p.L + BM - 1) / BM <= NGMAX;
+}
+
+size_t masked_tc_ws_bytes(const FwdParams &p) {
+    const size_t BH = (size_t)p.B * p.H, nb = (p.L + BM - 1) / BM;
+    return 2 * al256m(BH * nb * TB) + al256m(BH * nb * sizeof(float));
+}
+
+// 1: not covered (the caller takes the CUDA-core path); 0 launched; < 0 an error
+int launch_masked_tc(const FwdParams &p, void *ws, cudaStream_t s) {
+    if (!masked_tc_covers(p)) return 1;
+    if (!al16m(p.q) || !al16m(p.k) || !al16m(p.v) || !al16m(p.out)) return 1;
+    const size_t BH = (size_t)p.B * p.H, nb = (p.L + BM - 1) / BM;
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    uint8_t *xs = base, *es = base + al256m(BH * nb * TB);
+    float *gend = reinterpret_cast<float *>(es + al256m(BH * nb * TB));
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr[dev]) {
+        cudaFuncSetAttribute(masked_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)M_SMEM);
+        if (dev >= 0 && dev < 64) attr[dev] = true;
+    }
+    masked_tc_kernel<<<(unsigned)BH, NTHM, M_SMEM, s>>>(p, xs, es, gend);
+    return cudaGetLastError() == cudaSuccess ? 0 : -7;
+}
+
+#ifdef FALCON_TC_DEBUG
+extern "C" int falcon_masked_debug_timer_set(long long *ptr) {
+    return cudaMemcpyToSymbol(g_masked_tim, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;
+}
+#endif
+
+unsigned int masked_wait_timeouts() {
+    unsigned int v = 0;
+    cudaMemcpyFromSymbol(&v, g_masked_wait_timeouts, sizeof(v));
+    return v;
+}
+
+}  // namespace falcon

@@ -55,12 +55,11 @@ template <typename T> int launch_decode(const DecodeParams &p, cudaStream_t s);
 template <typename T> int launch_bwd(const BwdParams &p, cudaStream_t s);
 size_t bwd_ws_bytes(const BwdParams &p);
 // The chunk-parallel backward (k_bwd_chunk.cu): the shapes it takes, its
-// share of the workspace, and its launch (forward with chunk states, reverse
-// chain, per-chunk gradients) over the per-token arrays of launch_bwd.
+// workspace, and its launch (forward with chunk states, reverse chain,
+// per-chunk gradients: dq, dk, dv, dbeta and dlambda whole).
 bool bwd_chunk_covers(const BwdParams &p);
 size_t bwd_chunk_ws_bytes(const BwdParams &p);
-int launch_bwd_chunk(const BwdParams &p, void *ws, const float *xs, const float *etas, const float *alphas,
-                     float *dga, float *dgb, float *dgx, float *deta, float *dx, cudaStream_t s);
+int launch_bwd_chunk(const BwdParams &p, void *ws, cudaStream_t s);
 template <typename T> int launch_carry(const CarryParams &p, cudaStream_t s);
 
 // Stream-ordered scratch from the device's current memory pool
@@ -86,6 +85,13 @@ int validate_fwd(int variant, int form, int dtype, int pairing, int phi, int win
                  int d_v, int chunk);
 
 // Scratch sizes (floats) of the masked-parallel form.
+// The masked-parallel form of Falcon-1/1A (bf16, d = 64) on the tensor cores
+// (k_masked_tc.cu): covered shapes, workspace, launch (1: not covered or
+// misaligned pointers, the CUDA-core kernel takes it), give-ups of its waits.
+bool masked_tc_covers(const FwdParams &p);
+size_t masked_tc_ws_bytes(const FwdParams &p);
+int launch_masked_tc(const FwdParams &p, void *ws, cudaStream_t s);
+unsigned int masked_wait_timeouts();
 size_t masked_ws_r_floats(const FwdParams &p);
 size_t masked_ws_eg_floats(const FwdParams &p);
 

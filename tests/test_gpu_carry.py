@@ -80,6 +80,13 @@ def test_carry_tensor_core_path(F, variant, chunk):
     check_segment(F, variant, "chunk", "bf16", 2, 3, 200, 64, 64, chunk, 31)
 
 
+@pytest.mark.parametrize("d,chunk", [(32, 128), (128, 16), (128, 64)])
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_carry_tensor_core_widths(F, variant, d, chunk):
+    """A continued segment through the per-head chunk kernel at d = 32 and 128."""
+    check_segment(F, variant, "chunk", "bf16", 1, 2, 200, d, d, chunk, 33)
+
+
 @pytest.mark.parametrize("variant", ["F1", "F2", "F3", "F1A", "F2A", "F3A"])
 @pytest.mark.parametrize("form,chunk", [("recurrent", 64), ("chunk", 32), ("chunk", 64)])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

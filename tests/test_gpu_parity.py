@@ -121,6 +121,19 @@ def test_tensor_core_chunk_lengths_options(F, variant, chunk):
     check(F, d, variant, "chunk", chunk=chunk, phi="identity")
 
 
+@pytest.mark.parametrize("d_,chunk", [(32, 16), (32, 32), (32, 64), (32, 128), (128, 16), (128, 32), (128, 64)])
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_tensor_core_chunk_widths(F, variant, d_, chunk):
+    """The per-head tensor-core chunk kernel at d = 32 and d = 128: one token,
+    a ragged tail and many chunks, with the same-step pair and strong
+    forgetting on the longest case."""
+    for L in (1, 100, 300):
+        d = gen.draw(variant, 2, 2, L, d_, d_, seed=320 + L + chunk + d_, dtype="bf16")
+        check(F, d, variant, "chunk", chunk=chunk)
+    d = gen.draw(variant, 1, 2, 300, d_, d_, seed=330 + chunk + d_, dtype="bf16", lam=0.999, key_scale=0.125)
+    check(F, d, variant, "chunk", chunk=chunk, pairing="same_step")
+
+
 @pytest.mark.parametrize("w", [1, 2, 5, 8])
 @pytest.mark.parametrize("variant", ["F3", "F3A"])
 @pytest.mark.parametrize("form", ["recurrent", "masked", "chunk"])
@@ -196,6 +209,59 @@ def test_workload2_chunk_full(F, variant):
     """8x12x2048x64 bf16, chunk 64, every (b,h) unit against the oracle."""
     d = gen.workload_inputs(2, variant)
     check(F, d, variant, "chunk", chunk=64)
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_workload2_masked_tensor_core(F, variant):
+    """8x12x2048x64 bf16 in the masked-parallel form (the tensor-core pair
+    products): sampled units against the oracle, and every unit against the
+    chunk-parallel form on the GPU (the same function computed two ways)."""
+    d = gen.workload_inputs(2, variant)
+    check(F, d, variant, "masked", units=[(0, 0), (3, 7), (7, 11)])
+    om, Sm = gpu_fwd(F, d, variant, "masked")
+    oc, Sc = gpu_fwd(F, d, variant, "chunk")
+    assert rel(om, oc) <= 2e-2 and rel(Sm, Sc) <= 2e-2
+
+
+@pytest.mark.parametrize("L", [1, 63, 64, 65, 200, 700])
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_masked_tensor_core_lengths(F, variant, L):
+    """The masked-parallel tensor-core kernel (bf16, d = 64): one block, a
+    ragged block, exact multiples and many row blocks."""
+    d = gen.draw(variant, 2, 2, L, 64, 64, seed=340 + L, dtype="bf16")
+    check(F, d, variant, "masked")
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_masked_tensor_core_options(F, variant):
+    """The same kernel with the same-step pair and the identity map, strong
+    forgetting, and the decay floor."""
+    d = gen.draw(variant, 1, 2, 300, 64, 64, seed=350, dtype="bf16", key_scale=0.125)
+    check(F, d, variant, "masked", pairing="same_step", phi="identity")
+    d = gen.draw(variant, 1, 3, 400, 64, 64, seed=351, dtype="bf16", lam=0.999)
+    check(F, d, variant, "masked")
+    d = gen.draw(variant, 1, 2, 300, 64, 64, seed=352, dtype="bf16", lam=0.9, key_scale=0.05)
+    check(F, d, variant, "masked", phi="identity")
+
+
+@pytest.mark.parametrize("variant", ["F1", "F1A"])
+def test_masked_misaligned_inputs_take_the_cuda_core_kernel(F, variant):
+    """Inputs that are not 16-byte aligned (a view one element into its
+    storage) are refused by the tensor-core kernel and computed by the
+    CUDA-core one: same results within the tolerance."""
+    d = gen.draw(variant, 1, 2, 130, 64, 64, seed=353, dtype="bf16")
+    a = []
+    for n in ("q", "k", "v", "beta", "lam"):
+        x = dev(d, n)
+        if n != "lam":
+            buf = torch.empty(x.numel() + 1, dtype=x.dtype, device=x.device)
+            buf[1:].copy_(x.reshape(-1))
+            x = buf[1:].view(x.shape)
+        a.append(x)
+    out, S = F.fwd(variant, "masked", *a, d["eps"])
+    torch.cuda.synchronize()
+    oo, oS = oracle_fwd(d, variant)
+    assert rel(out.double().cpu().numpy(), oo) <= TOL["bf16"] and rel(S.double().cpu().numpy(), oS) <= TOL["bf16"]
 
 
 def test_workload3_falcon2_chunk_sampled(F):
@@ -302,6 +368,30 @@ def test_decode_odd_pair_count(F, variant, dk, dv):
     """An odd number of (n, h) pairs leaves the last decode block one pair short."""
     d, outs, S = _decode_chain(F, variant, 3, 3, dk, dv, 20, 5, "f32", 1)
     oo, oS = oracle_fwd(d, variant, 1)
+    assert rel(outs, oo[:, :, 20:]) <= 1e-4
+    assert rel(S, oS) <= 1e-4
+
+
+@pytest.mark.parametrize("pairing", ["prefix", "same_step"])
+@pytest.mark.parametrize("variant,w,dk,dv,dtype", [("F3", 2, 64, 64, "f32"), ("F3A", 3, 32, 16, "f32"),
+                                                   ("F3", 4, 128, 128, "bf16"), ("F3A", 4, 16, 32, "bf16"),
+                                                   ("F3", 5, 64, 32, "f32"), ("F3", 8, 32, 32, "f32")])
+def test_decode_window_paths(F, variant, w, dk, dv, dtype, pairing):
+    """The window decode kernels (windows 2-4 templated on the window, 5-8 the
+    general one) at several widths, with 2 x 5 = 10 (n, h) pairs: the last
+    block of four is half full."""
+    d, outs, S = _decode_chain(F, variant, 2, 5, dk, dv, 30, 6, dtype, w, pairing=pairing)
+    oo, oS = oracle_fwd(d, variant, w, pairing=pairing)
+    tol = TOL[dtype]
+    assert rel(outs, oo[:, :, 30:]) <= tol
+    assert rel(S, oS) <= tol
+
+
+@pytest.mark.parametrize("N,H", [(2, 5), (1, 4), (3, 1)])
+def test_decode_d128_pair_counts(F, N, H):
+    """d = 128 decode blocks take three (n, h) pairs: 10, 4 and 3 pairs."""
+    d, outs, S = _decode_chain(F, "F2A", N, H, 128, 128, 20, 5, "f32", 1)
+    oo, oS = oracle_fwd(d, "F2A", 1)
     assert rel(outs, oo[:, :, 20:]) <= 1e-4
     assert rel(S, oS) <= 1e-4
 
