@@ -167,16 +167,12 @@ struct SplitMaps {
 };
 
 // D = A B^T over K = 64 (four K=16 slices), both operands K-major and
-// 128-byte swizzled; M = 128, N = 64 or 128.
+// 128-byte swizzled; M = 128, N = 64 or 128.  Each descriptor is built once
+// and advanced per slice.
 __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_saddr, uint32_t b_saddr, int N,
                                            bool accumulate) {
-    const uint32_t idesc = tc::idesc_bf16(128, N, 0, 0);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = tc::sdesc_sw128(a_saddr + kk * 32, 16, 1024);
-        const uint64_t bd = tc::sdesc_sw128(b_saddr + kk * 32, 16, 1024);
-        tc::mma_bf16(d_tmem, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
-    }
+    tc::mma_k64(d_tmem, tc::sdesc_sw128(a_saddr, 16, 1024), tc::sdesc_sw128(b_saddr, 16, 1024),
+                tc::idesc_bf16(128, N, 0, 0), accumulate);
 }
 
 // One warp: C (16 x 8) = A (16 x K, rows of stride lda) * B (K x 8, rows of

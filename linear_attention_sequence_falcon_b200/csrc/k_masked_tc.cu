@@ -22,7 +22,8 @@
 // block then solves its own triangle: R_I = Y_I - D_a (accumulated), E_I =
 // (I + M_II)^{-1} R_I, O_I = D_c (accumulated) + (P o Dm)_II E_I.
 //
-// One block per (b, h).  The pair products run on tcgen05 (bf16 operands in
+// One block per (b, h): eight compute warps and an issuing warp.  The pair
+// products run on tcgen05 (bf16 operands in
 // 128-byte-swizzled shared memory, fp32 accumulators in tensor memory): P1 =
 // [X_I; Q_I] X_J^T into one of two accumulators while the previous pair's
 // P1 is scaled and rounded into the operand of P2 = [gA; gP] E~_J, which
@@ -43,7 +44,8 @@ namespace falcon {
 namespace {
 
 constexpr int BM = 64;         // tokens per block; d_k = d_v = 64
-constexpr int NTHM = 256;
+constexpr int NTHC = 256;              // eight compute warps
+constexpr int NTHM = NTHC + 32;        // and one warp whose lane 0 issues the products and copies
 constexpr int LDM = 72;        // fp32 row stride of the CUDA-core tiles
 constexpr int TFM = BM * LDM;  // floats per fp32 tile
 constexpr uint32_t TB = 8192;  // one bf16 64 x 64 tile (128-byte rows, 128-byte swizzle)
@@ -66,7 +68,7 @@ constexpr uint32_t M_ET = M_OF + TFM * 4;              // bf16: E~_I^T, staged f
 constexpr uint32_t M_VEC = M_ET + TB;                  // per-token vectors
 constexpr uint32_t M_GAM = M_VEC + 6 * BM * 4;        // gamma_IJ of the row block, J < I
 constexpr uint32_t M_BAR = M_GAM + NGMAX * 4;
-constexpr uint32_t M_SMEM = M_BAR + 128 + 1024;        // + alignment slack
+constexpr uint32_t M_SMEM = M_BAR + 192 + 1024;        // + alignment slack
 // the inverse's fp32 tiles D, K, K^2, T over the loop region (idle in the diagonal step)
 static_assert(4 * TFM * 4 <= M_LOOPEND - M_RING, "inverse scratch must fit over the pair buffers");
 static_assert(M_SMEM <= 227 * 1024, "shared memory of one block");
@@ -76,12 +78,12 @@ constexpr uint32_t TM_COLS = 256, TM_P1 = 0, TM_ACC = 128;
 __device__ unsigned int g_masked_wait_timeouts;
 
 #ifdef FALCON_TC_DEBUG
-// block 0, threads 0 (the issuer) and 32: SM cycles per phase summed over the row blocks
+// block 0, threads 0 (compute) and 256 (the issuer): SM cycles per phase summed over the row blocks
 __device__ long long *g_masked_tim;
 #define MT_INIT()                    \
     long long mt_acc_[16] = {0};     \
     long long mt_prev_ = clock64();  \
-    const bool mt_on_ = blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == 32)
+    const bool mt_on_ = blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == 256)
 #define MT(k)                                    \
     do {                                         \
         if (mt_on_) {                            \
@@ -101,16 +103,23 @@ __device__ long long *g_masked_tim;
 #define MT_END()
 #endif
 
-// D = A B^T over K = 64 (four K=16 slices), both operands K-major and
-// 128-byte swizzled; M = 128, N = 64.
-__device__ __forceinline__ void issue_128x64(uint32_t d_tmem, uint32_t a_saddr, uint32_t b_saddr, bool accumulate) {
-    const uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = tc::sdesc_sw128(a_saddr + kk * 32, 16, 1024);
-        const uint64_t bd = tc::sdesc_sw128(b_saddr + kk * 32, 16, 1024);
-        tc::mma_bf16(d_tmem, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
-    }
+// every product here: M = 128, N = 64, K = 64, both operands K-major
+constexpr uint32_t kIdesc = tc::idesc_bf16(128, 64, 0, 0);
+// descriptor units (16 bytes) of one bf16 tile
+constexpr uint32_t kTileDesc = TB >> 4;
+
+// barrier `id` over the first n threads of the block; true when pred holds on all of them
+__device__ __forceinline__ bool named_sync_and(uint32_t id, uint32_t n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -141,12 +150,13 @@ __global__ void __launch_bounds__(NTHM, 1)
           *vb = vec + 5 * BM;
     float *vgam = reinterpret_cast<float *>(sm + M_GAM);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + M_BAR);
-    uint64_t *txb = bar, *teb = bar + NRING, *bp1 = bar + 2 * NRING, *bp2 = bp1 + 2, *bd = bp2 + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bd + 1);
+    uint64_t *txb = bar, *teb = bar + NRING, *bp1 = bar + 2 * NRING, *bp2 = bp1 + 2, *bd = bp2 + 2, *bao = bd + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bao + 2);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool compute = tid < NTHC, issuer = tid == NTHC;  // warps 0-7 compute; warp 8 lane 0 issues
     const int quarter = warp & 3, chalf = warp >> 2;
-    const int row = quarter * 32 + lane;  // tensor-memory lane of this thread
+    const int row = quarter * 32 + lane;  // tensor-memory lane of a compute thread
     const bool reg = p.variant == F1;
     const int L = p.L, nb = (L + BM - 1) / BM;
     const size_t bh = blockIdx.x;
@@ -160,8 +170,10 @@ __global__ void __launch_bounds__(NTHM, 1)
     uint8_t *es = es_ws + bh * (size_t)nb * TB;
     float *gend = gend_ws + bh * (size_t)nb;
 
-    if (tid == 0) {
+    if (issuer) {
         for (int i = 0; i < 2 * NRING + 5; ++i) tc::mbar_init(&bar[i], 1);
+        tc::mbar_init(&bao[0], NTHC);
+        tc::mbar_init(&bao[1], NTHC);
         tc::fence_mbar_init();
     }
     if (warp == 0) {
@@ -174,18 +186,20 @@ __global__ void __launch_bounds__(NTHM, 1)
     const uint32_t tbase = *tmem_slot;
     const uint32_t tlane = tbase + ((uint32_t)(quarter * 32) << 16);
 
-    // completion counts: every thread tracks the MMA barriers alike; thread 0
-    // alone tracks the rings (loads issued and consumed per slot)
+    // completion counts.  The compute threads count the product barriers
+    // (P1, P2, the diagonal product); the issuer counts the operand
+    // hand-offs, the P2 issued per accumulator and the ring loads.
     uint32_t n1[2] = {0u, 0u}, n2[2] = {0u, 0u}, ndg = 0u;
+    uint32_t na[2] = {0u, 0u}, i2[2] = {0u, 0u};
     uint32_t lx[NRING] = {0u, 0u, 0u, 0u}, cx[NRING] = {0u, 0u, 0u, 0u};
     uint32_t le[NRING] = {0u, 0u, 0u, 0u}, ce[NRING] = {0u, 0u, 0u, 0u};
     bool ok = true;
     float Gprev = 0.f;  // Gamma_{I0-1}
-    MT_INIT();
-    float sacc[4][4];   // S (this warp's 16 x 32 block), e^{...} relative to the last block's end
+    float sacc[4][4];   // S (this compute warp's 16 x 32 block), relative to the last block's end
     wt::zero(sacc);
+    MT_INIT();
 
-    // thread 0: X_J into its ring slot, E~_J^T into its own; the waits for them
+    // issuer: X_J into its ring slot, E~_J^T into its own; the waits for them
     auto load_x = [&](int J) {
         const int s = J % NRING;
         tc::mbar_arrive_expect_tx(&txb[s], TB);
@@ -210,9 +224,14 @@ __global__ void __launch_bounds__(NTHM, 1)
         ++ce[s];
         return r;
     };
+    // the operand descriptors, built once
+    const uint64_t dAQ = tc::sdesc_sw128(sb + M_AQ, 16, 1024);
+    const uint64_t dX0 = tc::sdesc_sw128(sb + M_RING, 16, 1024);
+    const uint64_t dE0 = tc::sdesc_sw128(sb + M_ERING, 16, 1024);
+    const uint64_t dA0 = tc::sdesc_sw128(sb + M_AOP, 16, 1024);
     auto issue_p1 = [&](int J) {  // P1(J) = [X_I; Q_I] X_J^T into accumulator J & 1
-        issue_128x64(tbase + TM_P1 + (uint32_t)(J & 1) * 64, sb + M_AQ, sb + M_RING + (uint32_t)(J % NRING) * TB,
-                     false);
+        tc::mma_k64(tbase + TM_P1 + (uint32_t)(J & 1) * 64, dAQ, dX0 + (uint64_t)(J % NRING) * kTileDesc, kIdesc,
+                    false);
         tc::mma_commit(&bp1[J & 1]);
     };
 
@@ -220,13 +239,13 @@ __global__ void __launch_bounds__(NTHM, 1)
         const int I0 = I * BM, n = min(BM, L - I0);
         // ---- the block's inputs: samples x_t = phi(k_{t-1}) (prefix pair;
         //      phi(k_t) same-step), q, v, the steps and the decays
-        if (tid == 0) tc::bulk_wait_read();  // the stores of the last block have read AQ and ET
+        if (issuer) tc::bulk_wait_read();  // the stores of the last block have read AQ and ET
         __syncthreads();
-        {
+        if (compute) {
             uint4 lq[2], lv[2];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const int e = tid + NTHM * j;  // 16-byte piece: row e / 8, columns 8 (e % 8)..
+                const int e = tid + NTHC * j;  // 16-byte piece: row e / 8, columns 8 (e % 8)..
                 const bool in = (e >> 3) < n;
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
                 lq[j] = in ? wt::ld16(qh + (size_t)I0 * BM + 8 * e) : z;
@@ -259,49 +278,52 @@ __global__ void __launch_bounds__(NTHM, 1)
             }
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const int e = tid + NTHM * j, r = e >> 3, c = e & 7;
+                const int e = tid + NTHC * j, r = e >> 3, c = e & 7;
                 *reinterpret_cast<uint4 *>(sm + M_AQ + tc::sw128(64 + r, c)) = lq[j];
                 wt::st8(YF + r * LDM + 8 * c, lv[j]);
             }
-        }
-        __syncthreads();
-        if (warp == 0) {  // block-local cumulative log decay G_t
-            float la[2] = {vla[lane], vla[lane + 32]};
+            tc::named_sync(1, NTHC);
+            if (warp == 0) {  // block-local cumulative log decay G_t
+                float la[2] = {vla[lane], vla[lane + 32]};
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
+                for (int o = 1; o < 32; o <<= 1) {
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const float y = __shfl_up_sync(0xffffffffu, la[h2], o);
-                    if (lane >= o) la[h2] += y;
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const float y = __shfl_up_sync(0xffffffffu, la[h2], o);
+                        if (lane >= o) la[h2] += y;
+                    }
                 }
+                la[1] += __shfl_sync(0xffffffffu, la[0], 31);
+                vG[lane] = la[0];
+                vG[lane + 32] = la[1];
             }
-            la[1] += __shfl_sync(0xffffffffu, la[0], 31);
-            vG[lane] = la[0];
-            vG[lane + 32] = la[1];
+            tc::named_sync(1, NTHC);
+            const float GE = vG[BM - 1];
+            if (tid < BM) {
+                const int t = tid;
+                va[t] = __expf(t > 0 ? vG[t - 1] : 0.f);   // e^{Gamma_{t-1} - Gamma_{I0-1}}
+                vc[t] = __expf(vG[t]);                      // e^{Gamma_t - Gamma_{I0-1}}
+                vb[t] = __expf(GE - vG[t]) * veta[t];       // e^{Gamma_Iend - Gamma_t} eta_t
+            }
+            if (tid == 0) gend[I] = Gprev + GE;
+            tc::fence_proxy_async();
         }
-        __syncthreads();
-        const float GE = vG[BM - 1];
-        if (tid < BM) {
-            const int t = tid;
-            va[t] = __expf(t > 0 ? vG[t - 1] : 0.f);   // e^{Gamma_{t-1} - Gamma_{I0-1}}
-            vc[t] = __expf(vG[t]);                      // e^{Gamma_t - Gamma_{I0-1}}
-            vb[t] = __expf(GE - vG[t]) * veta[t];       // e^{Gamma_Iend - Gamma_t} eta_t
-        }
-        if (tid == 0) gend[I] = Gprev + GE;
-        tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
-        if (tid == 0) {  // X_I for the later row blocks
+        const float GE = vG[BM - 1];
+        if (issuer) {  // X_I for the later row blocks
             tc::bulk_store(xs + (size_t)I * TB, sb + M_AQ, TB);
             tc::bulk_commit();
         }
         MT(0);
 
-        // ---- the pairs (I, J < I).  P1 runs two pairs ahead of the pair whose
-        //      operand is being formed; X_J is loaded four pairs ahead, E~_J three
+        // ---- the pairs (I, J < I).  The compute warps turn P1(J) into the
+        //      operand [gA; gP] of P2(J) and hand it over through an mbarrier;
+        //      the issuer runs P2(J) and P1 two pairs ahead, and keeps X_J
+        //      four pairs and E~_J three pairs ahead in their rings
         if (I > 0) {
-            if (tid == 0) {
+            if (issuer) {
                 // every earlier X_J and E~_J has landed in the workspace (the
                 // store of X_I, the newest group, may still be in flight)
                 asm volatile("cp.async.bulk.wait_group 1;" ::: "memory");
@@ -314,76 +336,86 @@ __global__ void __launch_bounds__(NTHM, 1)
                     if (r) issue_p1(1);
                 }
                 ok = r;
+            } else if (compute) {
+                for (int J = tid; J < I; J += NTHC) vgam[J] = __expf(Gprev - gend[J]);
             }
-            for (int J = tid; J < I; J += NTHM) vgam[J] = __expf(Gprev - gend[J]);
             ok = __syncthreads_and(ok);
             MT(1);
-            for (int J = 0; J < I && ok; ++J) {
-                const int b = J & 1;
-                // P1(J) -> this thread's 32 columns of its lane
-                bool w = tc::mbar_wait_timeout(&bp1[b], n1[b] & 1u, kWaitNsM);
-                ++n1[b];
-                __syncwarp();
-                tc::fence_after_sync();
-                float v[32];
-                tc::tmem_ld32(tlane + TM_P1 + b * 64 + chalf * 32, v);
-                tc::tmem_wait_ld();
-                MT(2);
-                // [gA; gP] of this pair into operand b once P2(J-2) has read it
-                const float g = vgam[J];
-                if (J >= 2) {
-                    w = tc::mbar_wait_timeout(&bp2[b], n2[b] & 1u, kWaitNsM) && w;
-                    ++n2[b];
-                }
-                const uint32_t aop = M_AOP + (uint32_t)b * 2 * TB;
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint4 u;
-                    u.x = pack2(g * v[c4 * 8 + 0], g * v[c4 * 8 + 1]);
-                    u.y = pack2(g * v[c4 * 8 + 2], g * v[c4 * 8 + 3]);
-                    u.z = pack2(g * v[c4 * 8 + 4], g * v[c4 * 8 + 5]);
-                    u.w = pack2(g * v[c4 * 8 + 6], g * v[c4 * 8 + 7]);
-                    *reinterpret_cast<uint4 *>(sm + aop + tc::sw128(row, chalf * 4 + c4)) = u;
-                }
-                tc::fence_proxy_async();
-                tc::fence_before_sync();
-                MT(3);
-                // every thread has read accumulator b and written operand b
-                ok = __syncthreads_and(w && ok);
-                if (!ok) break;
-                tc::fence_after_sync();
-                MT(4);
-                if (tid == 0) {
-                    // P2(J): [R; O] += [gA; gP] E~_J
-                    bool r = wait_e(J);
-                    if (r) {
-                        issue_128x64(tbase + TM_ACC, sb + aop, sb + M_ERING + (uint32_t)(J % NRING) * TB, J > 0);
-                        tc::mma_commit(&bp2[b]);
+            if (compute) {
+                for (int J = 0; J < I && ok; ++J) {
+                    const int b = J & 1;
+                    // P1(J) -> this thread's 32 columns of its lane
+                    bool w = tc::mbar_wait_timeout(&bp1[b], n1[b] & 1u, kWaitNsM);
+                    ++n1[b];
+                    __syncwarp();
+                    tc::fence_after_sync();
+                    float v[32];
+                    tc::tmem_ld32(tlane + TM_P1 + b * 64 + chalf * 32, v);
+                    tc::tmem_wait_ld();
+                    MT(2);
+                    // [gA; gP] of this pair into operand b once P2(J-2) has read it
+                    const float g = vgam[J];
+                    if (J >= 2) {
+                        w = tc::mbar_wait_timeout(&bp2[b], n2[b] & 1u, kWaitNsM) && w;
+                        ++n2[b];
                     }
-                    // P1(J+2) into accumulator b, read out above
+                    const uint32_t aop = M_AOP + (uint32_t)b * 2 * TB;
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint4 u;
+                        u.x = pack2(g * v[c4 * 8 + 0], g * v[c4 * 8 + 1]);
+                        u.y = pack2(g * v[c4 * 8 + 2], g * v[c4 * 8 + 3]);
+                        u.z = pack2(g * v[c4 * 8 + 4], g * v[c4 * 8 + 5]);
+                        u.w = pack2(g * v[c4 * 8 + 6], g * v[c4 * 8 + 7]);
+                        *reinterpret_cast<uint4 *>(sm + aop + tc::sw128(row, chalf * 4 + c4)) = u;
+                    }
+                    tc::fence_proxy_async();
+                    tc::fence_before_sync();
+                    // accumulator b is read and operand b written: hand both over
+                    tc::mbar_arrive(&bao[b]);
+                    ok = w;
+                    MT(3);
+                }
+                if (ok) {
+                    // the last two P2 (the others have been counted)
+                    for (int J = max(0, I - 2); J < I && ok; ++J) {
+                        const int b = J & 1;
+                        ok = tc::mbar_wait_timeout(&bp2[b], n2[b] & 1u, kWaitNsM);
+                        ++n2[b];
+                    }
+                }
+            } else if (issuer) {
+                for (int J = 0; J < I && ok; ++J) {
+                    const int b = J & 1;
+                    bool r = tc::mbar_wait_timeout(&bao[b], na[b] & 1u, kWaitNsM);
+                    ++na[b];
+                    tc::fence_after_sync();
+                    MT(4);
+                    // P2(J): [R; O] += [gA; gP] E~_J
+                    r = r && wait_e(J);
+                    if (r) {
+                        tc::mma_k64(tbase + TM_ACC, dA0 + (uint64_t)b * 2 * kTileDesc,
+                                    dE0 + (uint64_t)(J % NRING) * kTileDesc, kIdesc, J > 0);
+                        tc::mma_commit(&bp2[b]);
+                        ++i2[b];
+                    }
+                    MT(10);
+                    // P1(J+2) into accumulator b, read out by every compute thread
                     if (r && J + 2 < I) {
                         r = wait_x(J + 2);
                         if (r) issue_p1(J + 2);
                     }
+                    MT(11);
                     // X_{J+4} into the slot of X_J (P1(J) is done)
                     if (r && J + NRING < I) load_x(J + NRING);
-                    // E~_{J+3} into the slot of E~_{J-1} once P2(J-1) is done: the
-                    // newest product of accumulator b ^ 1, waited on here without
-                    // consuming the completion the other threads count
+                    // E~_{J+3} into the slot of E~_{J-1} once P2(J-1), the newest
+                    // product of accumulator b ^ 1, is done
                     if (r && J + NRING - 1 < I) {
-                        if (J >= 1) r = tc::mbar_wait_timeout(&bp2[b ^ 1], n2[b ^ 1] & 1u, kWaitNsM);
+                        if (J >= 1) r = tc::mbar_wait_timeout(&bp2[b ^ 1], (i2[b ^ 1] - 1u) & 1u, kWaitNsM);
                         if (r) load_e(J + NRING - 1);
                     }
+                    MT(5);
                     if (!r) ok = false;
-                }
-                MT(5);
-            }
-            if (ok) {
-                // the last two P2 (the others have been counted)
-                for (int J = max(0, I - 2); J < I && ok; ++J) {
-                    const int b = J & 1;
-                    ok = tc::mbar_wait_timeout(&bp2[b], n2[b] & 1u, kWaitNsM);
-                    ++n2[b];
                 }
             }
             ok = __syncthreads_and(ok);
@@ -392,19 +424,18 @@ __global__ void __launch_bounds__(NTHM, 1)
         }
 
         // ---- the diagonal block: [A_II; P_II] = [X_I; Q_I] X_I^T
-        if (tid == 0) {
-            tc::fence_after_sync();
-            issue_128x64(tbase + TM_P1, sb + M_AQ, sb + M_AQ, false);
+        if (issuer) {
+            tc::mma_k64(tbase + TM_P1, dAQ, dAQ, kIdesc, false);
             tc::mma_commit(bd);
         }
-        {
-            const bool w = tc::mbar_wait_timeout(bd, ndg & 1u, kWaitNsM);
-            ++ndg;
-            ok = __syncthreads_and(w);
-            if (!ok) break;
-        }
-        tc::fence_after_sync();
-        {
+        if (compute) {
+            {
+                const bool w = tc::mbar_wait_timeout(bd, ndg & 1u, kWaitNsM);
+                ++ndg;
+                __syncwarp();
+                tc::fence_after_sync();
+                ok = w;
+            }
             float v[32], r[32];
             tc::tmem_ld32(tlane + TM_P1 + chalf * 32, v);
             if (I > 0) tc::tmem_ld32(tlane + TM_ACC + chalf * 32, r);
@@ -419,9 +450,9 @@ __global__ void __launch_bounds__(NTHM, 1)
                     const float gm = t > 0 ? vG[t - 1] : 0.f, a = va[t];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const int s = chalf * 32 + i;
-                        MT[t * LDM + s] = s < t ? __expf(gm - vG[s]) * veta[s] * v[i] : 0.f;
-                        YF[t * LDM + s] -= a * r[i];
+                        const int s2 = chalf * 32 + i;
+                        MT[t * LDM + s2] = s2 < t ? __expf(gm - vG[s2]) * veta[s2] * v[i] : 0.f;
+                        YF[t * LDM + s2] -= a * r[i];
                     }
                 }
             } else {  // rows 64-127: (P o Dm)_II (with the steps) and D_c (accumulated)
@@ -429,94 +460,94 @@ __global__ void __launch_bounds__(NTHM, 1)
                 const float gt = vG[t], c = vc[t];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int s = chalf * 32 + i;
-                    PD[t * LDM + s] = s <= t ? __expf(gt - vG[s]) * veta[s] * v[i] : 0.f;
-                    OF[t * LDM + s] = c * r[i];
+                    const int s2 = chalf * 32 + i;
+                    PD[t * LDM + s2] = s2 <= t ? __expf(gt - vG[s2]) * veta[s2] * v[i] : 0.f;
+                    OF[t * LDM + s2] = c * r[i];
                 }
             }
+            tc::fence_before_sync();
+            ok = named_sync_and(1, NTHC, ok);
         }
-        tc::fence_before_sync();
-        __syncthreads();
         MT(7);
-        const int rb = (warp & 3) * 16, cb = (warp >> 2) * 32;
-        float acc[4][4];
-        if (reg) {
-            // ---- T = (I + M_II)^{-1}: D, the diagonal 16 x 16 blocks' inverses
-            //      (one column of a block per thread, threads 0-63); zeros elsewhere
-            if (tid < 64) {
-                const int o = (tid >> 4) * 16, j = tid & 15;
-                float col[16];
+        if (compute && ok) {
+            const int rb = (warp & 3) * 16, cb = (warp >> 2) * 32;
+            float acc[4][4];
+            if (reg) {
+                // ---- T = (I + M_II)^{-1}: D, the diagonal 16 x 16 blocks' inverses
+                //      (one column of a block per thread, threads 0-63); zeros elsewhere
+                if (tid < 64) {
+                    const int o = (tid >> 4) * 16, j = tid & 15;
+                    float col[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float s = i == j ? 1.f : 0.f;
+                    for (int i = 0; i < 16; ++i) {
+                        float sv = i == j ? 1.f : 0.f;
 #pragma unroll
-                    for (int s2 = 0; s2 < i; ++s2) s -= MT[(o + i) * LDM + o + s2] * col[s2];
-                    col[i] = s;
-                }
+                        for (int s2 = 0; s2 < i; ++s2) sv -= MT[(o + i) * LDM + o + s2] * col[s2];
+                        col[i] = sv;
+                    }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) DI[(o + i) * LDM + o + j] = col[i];
-            } else {
-                for (int e = tid - 64; e < BM * BM; e += NTHM - 64) {
-                    const int r2 = e >> 6, s = e & 63;
-                    if ((r2 >> 4) != (s >> 4)) DI[r2 * LDM + s] = 0.f;
-                }
-            }
-            __syncthreads();
-            // K = D M_o: D M on the blocks below the diagonal (D reads its own block only)
-            wt::zero(acc);
-            mma64<false, false>(DI, MT, acc, rb, rb + 16);
-            wt::each(acc, [&](int r2, int s, float &val) { KI[r2 * LDM + s] = (s >> 4) < (r2 >> 4) ? val : 0.f; });
-            __syncthreads();
-            wt::zero(acc);
-            if (rb > 0) mma64<false, false>(KI, KI, acc, 0, rb);
-            wt::each(acc, [&](int r2, int s, float &val) { K2[r2 * LDM + s] = val; });
-            __syncthreads();
-            wt::zero(acc);
-            if (rb > 0) mma64<false, false>(KI, K2, acc, 0, rb);
-            wt::each(acc, [&](int r2, int s, float &val) {
-                TI[r2 * LDM + s] = (r2 == s ? 1.f : 0.f) - KI[r2 * LDM + s] + K2[r2 * LDM + s] - val;
-            });
-            __syncthreads();
-            // T = (I - K + K^2 - K^3) D: each warp reads only the block of the sum it writes
-            wt::zero(acc);
-            {
-                const int ke = min(cb + 32, rb + 16);
-                if (ke > cb) mma64<false, false>(TI, DI, acc, cb, ke);
-            }
-            __syncwarp();
-            wt::each(acc, [&](int r2, int s, float &val) { TI[r2 * LDM + s] = val; });
-            __syncthreads();
-            // E = T R (T lower: k <= r)
-            wt::zero(acc);
-            mma64<false, false>(TI, YF, acc, 0, rb + 16);
-            __syncthreads();
-            wt::each(acc, [&](int r2, int j, float &val) { YF[r2 * LDM + j] = val; });
-            __syncthreads();
-        }
-        MT(8);
-        // ---- O_I = D_c (accumulated) + (P o Dm)_II E_I
-        wt::zero(acc);
-        mma64<false, false>(PD, YF, acc, 0, rb + 16);
-        {
-            const int g = lane >> 2, t4 = lane & 3;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const int r2 = rb + g + 8 * h2, j = cb + nt * 8 + 2 * t4;
-                    if (r2 < n) {
-                        const float o0 = acc[nt][2 * h2] + OF[r2 * LDM + j];
-                        const float o1 = acc[nt][2 * h2 + 1] + OF[r2 * LDM + j + 1];
-                        *reinterpret_cast<uint32_t *>(oh + (size_t)(I0 + r2) * BM + j) = pack2(o0, o1);
+                    for (int i = 0; i < 16; ++i) DI[(o + i) * LDM + o + j] = col[i];
+                } else {
+                    for (int e = tid - 64; e < BM * BM; e += NTHC - 64) {
+                        const int r2 = e >> 6, s2 = e & 63;
+                        if ((r2 >> 4) != (s2 >> 4)) DI[r2 * LDM + s2] = 0.f;
                     }
                 }
-        }
-        // ---- E~_I^T (bf16, swizzled: row j holds b_s E[s][j] over s) for the later
-        //      row blocks, and S <- e^{G_Iend} S + E~_I^T X_I
-        {
+                tc::named_sync(1, NTHC);
+                // K = D M_o: D M on the blocks below the diagonal (D reads its own block only)
+                wt::zero(acc);
+                mma64<false, false>(DI, MT, acc, rb, rb + 16);
+                wt::each(acc, [&](int r2, int s2, float &val) { KI[r2 * LDM + s2] = (s2 >> 4) < (r2 >> 4) ? val : 0.f; });
+                tc::named_sync(1, NTHC);
+                wt::zero(acc);
+                if (rb > 0) mma64<false, false>(KI, KI, acc, 0, rb);
+                wt::each(acc, [&](int r2, int s2, float &val) { K2[r2 * LDM + s2] = val; });
+                tc::named_sync(1, NTHC);
+                wt::zero(acc);
+                if (rb > 0) mma64<false, false>(KI, K2, acc, 0, rb);
+                wt::each(acc, [&](int r2, int s2, float &val) {
+                    TI[r2 * LDM + s2] = (r2 == s2 ? 1.f : 0.f) - KI[r2 * LDM + s2] + K2[r2 * LDM + s2] - val;
+                });
+                tc::named_sync(1, NTHC);
+                // T = (I - K + K^2 - K^3) D: each warp reads only the block of the sum it writes
+                wt::zero(acc);
+                {
+                    const int ke = min(cb + 32, rb + 16);
+                    if (ke > cb) mma64<false, false>(TI, DI, acc, cb, ke);
+                }
+                __syncwarp();
+                wt::each(acc, [&](int r2, int s2, float &val) { TI[r2 * LDM + s2] = val; });
+                tc::named_sync(1, NTHC);
+                // E = T R (T lower: k <= r)
+                wt::zero(acc);
+                mma64<false, false>(TI, YF, acc, 0, rb + 16);
+                tc::named_sync(1, NTHC);
+                wt::each(acc, [&](int r2, int j, float &val) { YF[r2 * LDM + j] = val; });
+                tc::named_sync(1, NTHC);
+            }
+            MT(8);
+            // ---- O_I = D_c (accumulated) + (P o Dm)_II E_I
+            wt::zero(acc);
+            mma64<false, false>(PD, YF, acc, 0, rb + 16);
+            {
+                const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int r2 = rb + g + 8 * h2, j = cb + nt * 8 + 2 * t4;
+                        if (r2 < n) {
+                            const float o0 = acc[nt][2 * h2] + OF[r2 * LDM + j];
+                            const float o1 = acc[nt][2 * h2 + 1] + OF[r2 * LDM + j + 1];
+                            *reinterpret_cast<uint32_t *>(oh + (size_t)(I0 + r2) * BM + j) = pack2(o0, o1);
+                        }
+                    }
+            }
+            // ---- E~_I^T (bf16, swizzled: row j holds b_s E[s][j] over s) for the later
+            //      row blocks, and S <- e^{G_Iend} S + E~_I^T X_I
 #pragma unroll
             for (int k2 = 0; k2 < 2; ++k2) {
-                const int e = tid + NTHM * k2, j = e >> 3, c = e & 7;
+                const int e = tid + NTHC * k2, j = e >> 3, c = e & 7;
                 float f[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) f[i] = vb[8 * c + i] * YF[(8 * c + i) * LDM + j];
@@ -533,11 +564,12 @@ __global__ void __launch_bounds__(NTHM, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sacc[nt][e] *= gI;
             mma64<true, false, true>(YF, XF, sacc, 0, 64, vb);
+            tc::fence_proxy_async();
         }
-        tc::fence_proxy_async();
         tc::fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        if (issuer) {
             tc::bulk_store(es + (size_t)I * TB, sb + M_ET, TB);
             tc::bulk_commit();
         }
@@ -546,16 +578,16 @@ __global__ void __launch_bounds__(NTHM, 1)
     }
 
     MT_END();
-    if (p.final_state && ok)
+    if (p.final_state && ok && compute)
         wt::each(sacc, [&](int j, int i, float &val) { p.final_state[(bh * BM + j) * BM + i] = val; });
-    if (tid == 0) {
+    if (issuer) {
         tc::bulk_wait_all();
         if (!ok) {
             atomicAdd(&g_masked_wait_timeouts, 1u);
             // loads still in flight must land before the block leaves
-            for (int s = 0; s < NRING; ++s) {
-                if (lx[s] > cx[s]) (void)tc::mbar_wait_timeout(&txb[s], (lx[s] - 1u) & 1u, kWaitNsM);
-                if (le[s] > ce[s]) (void)tc::mbar_wait_timeout(&teb[s], (le[s] - 1u) & 1u, kWaitNsM);
+            for (int s2 = 0; s2 < NRING; ++s2) {
+                if (lx[s2] > cx[s2]) (void)tc::mbar_wait_timeout(&txb[s2], (lx[s2] - 1u) & 1u, kWaitNsM);
+                if (le[s2] > ce[s2]) (void)tc::mbar_wait_timeout(&teb[s2], (le[s2] - 1u) & 1u, kWaitNsM);
             }
         }
     }

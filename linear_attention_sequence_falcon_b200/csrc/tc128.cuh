@@ -60,12 +60,8 @@ __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a, uint32_t
                                            uint32_t b_step, int nk, int N) {
     const uint32_t idesc = tc::idesc_bf16(128, N, 0, 0);
     for (int kt = 0; kt < nk; ++kt)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = tc::sdesc_sw128(a + kt * a_step + kk * 32, 16, 1024);
-            const uint64_t bd = tc::sdesc_sw128(b + kt * b_step + kk * 32, 16, 1024);
-            tc::mma_bf16(d_tmem, ad, bd, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
-        }
+        tc::mma_k64(d_tmem, tc::sdesc_sw128(a + kt * a_step, 16, 1024), tc::sdesc_sw128(b + kt * b_step, 16, 1024),
+                    idesc, kt > 0);
 }
 
 // Transposed copy of four 8x8 blocks of a 64-row bf16 tile (128-byte rows,

@@ -224,6 +224,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
+// D (+)= A B^T over K = 64 bf16 (four K=16 slices) from the descriptors of
+// the K-major, 128-byte-swizzled tiles A and B: a slice starts 32 bytes
+// further in, i.e. 2 more in the descriptors' 16-byte address units (tile
+// bases below 256 KB, so the start field cannot carry).  The descriptors are
+// built once by the caller; the slices only add.
+__device__ __forceinline__ void mma_k64(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (accumulate || kk > 0) ? 1u : 0u);
+}
+
 // Arrive on `bar` once every MMA issued so far by this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
