@@ -77,6 +77,22 @@ def algorithmic_bytes_fwd(B, H, L, dk, dv, per_channel=False, elt=2):
     return tok * (2 * dk + dv + (dv if per_channel else 1) + dv) * elt + B * H * dv * dk * 4 + H * 4
 
 
+# fp32 CUDA-core peak of a B200 at its maximum clock: 148 SMs x 128 FP32 lanes
+# x 2 flop (one FMA) x 1965 MHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def window_walk_flops(B, H, L, C, w, dv):
+    """Flops of the chunk form's per-token solve for the C*B_w window errors
+    of the regression family (Falcon-3), on the CUDA cores: token t of a
+    chunk, window slot m and value channel j take the dot product of row
+    t+m of the sample Gram with the per-row sums of the errors solved so far,
+    which cover rows 0 .. t+B_w-2 (2 (t + B_w - 1) flops), plus 8 flops for
+    the rest of the update.  Summed over full chunks."""
+    per_chunk = dv * w * sum(2 * (t + w - 1) + 8 for t in range(C))
+    return B * H * ((L + C - 1) // C) * per_chunk
+
+
 def algorithmic_bytes_decode(N, H, dk, dv, per_channel=True, elt=2):
     """Per decode step: state read + write (fp32), x_prev read + write (fp32),
     q, k, v, beta in, out."""
@@ -603,6 +619,13 @@ def run_workloads(args):
                 "ms": t, "tokens_per_s": w["B"] * w["L"] / (t / 1e3),
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                              "peak_source": peak_src, "algorithmic_bytes_per_launch": ab}}
+        if form == "chunk" and var == "F3":
+            # the per-token window solve runs on the CUDA cores: its fp32 roofline
+            fl = window_walk_flops(w["B"], w["H"], w["L"], w["chunk"], w["window"], w["dv"])
+            tfs = fl / (t / 1e3) / 1e12
+            line["roofline_alu"] = {"bound": "alu", "achieved": tfs, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                                    "frac": tfs / FP32_ALU_TFLOPS, "flops_per_launch": fl,
+                                    "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
         if not args.no_cpu_baseline:
             line["cpu_oracle"] = workload_oracle_rate(d, var, form, w)
         print(json.dumps(line), flush=True)

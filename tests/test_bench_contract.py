@@ -33,6 +33,23 @@ def test_algorithmic_bytes_of_the_bench_workload(bench):
         10 * (128 * 4 + 128) * 2 + 128 * 128 * 4 + 4
 
 
+def test_window_walk_flops_count_each_dot_product(bench):
+    """The Falcon-3 window solve's flop count against a direct loop over
+    tokens, window slots and value channels: the dot product of token t,
+    slot m covers the rows 0 .. t+B_w-2 finished so far (two flops per row),
+    plus eight for the rest of the update; a partial last chunk counts as
+    full."""
+    C, w, dv = 8, 3, 5
+    direct = 0
+    for t in range(C):
+        for m in range(w):
+            for j in range(dv):
+                direct += 2 * (t + w - 1) + 8
+    assert bench.window_walk_flops(1, 1, C, C, w, dv) == direct
+    assert bench.window_walk_flops(2, 3, 2 * C + 1, C, w, dv) == 2 * 3 * 3 * direct
+    assert abs(bench.FP32_ALU_TFLOPS - 74.44992) < 1e-6
+
+
 def test_profiled_traffic_follows_the_sources(bench, monkeypatch, tmp_path):
     """A summary's traffic figure counts while the captured kernel's sources
     hash to the value it records, and not after any of them changes."""
