@@ -378,7 +378,7 @@ extern "C" int falcon_bwd_ws(falcon_variant variant, falcon_form form, falcon_dt
 extern "C" int falcon_device_wait_timeouts(unsigned int *count) {
     if (!count) return FALCON_ERR_NULL;
     *count = split_wait_timeouts() + pc_wait_timeouts() + f2_wait_timeouts() + w_wait_timeouts() +
-             masked_wait_timeouts();
+             masked_wait_timeouts() + decode_wait_timeouts();
     return cudaGetLastError() == cudaSuccess ? FALCON_OK : FALCON_ERR_LAUNCH;
 }
 

@@ -13,6 +13,7 @@
 // the window) is updated in place without races.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_sm100.cuh"
 
 namespace falcon {
 
@@ -315,6 +316,170 @@ __global__ void __launch_bounds__(32 * decode1_warps(DK), DK >= 128 ? 8 : 4) dec
     }
 }
 
+// Window-1 decode at d = 64 with the state streamed through shared memory:
+// one block of four warps per (n,h) pair.  Thread 0 bulk-copies the pair's
+// state (16 KB) in four stages of 16 rows, all issued before the block stages
+// its token vectors; the lanes read their row from shared memory and store
+// the new row straight to HBM.  At d = 64 a pair's rows are few, so
+// decode1_kernel's two rows in flight per lane left the step latency-bound
+// (15.9 us against 14.3 us here on N = 64, H = 16).  At d = 128 this layout
+// measured no faster than decode1_kernel (31.9 against 31.2 us: there the
+// step is bound by the HBM read/write mix, not by loads in flight), so d = 128
+// keeps decode1_kernel.  The row arithmetic is decode1_kernel's.  Every wait
+// is bounded; a give-up leaves the pair's outputs incomplete and is counted.
+__device__ unsigned int g_decode_wait_timeouts;
+
+template <typename T, int DK>
+__global__ void __launch_bounds__(128, 8) decode1r_kernel(DecodeParams p) {
+    constexpr int LPR = 8, NV4 = DK / (4 * LPR), RPW = 32 / LPR, NW = 4;
+    constexpr int RPS = NW * RPW;  // rows per stage: 16
+    constexpr int NST = 4;  // with d_v <= 64 rows, a pair's whole state
+    __shared__ __align__(128) float ring[NST][RPS * DK];
+    __shared__ __align__(8) uint64_t bars[NST];
+    __shared__ __align__(16) float xs[DK];
+    __shared__ __align__(16) float qs[DK];
+    __shared__ float ks[DK];
+    __shared__ float ys[128];
+    __shared__ float bs[128];
+    __shared__ float red[3][NW];
+    __shared__ float hsc[5];  // inv_den, xq, lambda, |k|^2, 1/|k| (same-step pair)
+
+    const VariantInfo vi = variant_info(p.variant, 1);
+    const int nh = blockIdx.x, dv = p.dv;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nstage = (dv + RPS - 1) / RPS;
+    float *S = p.state + (size_t)nh * dv * DK;
+    int issued = 0;  // stages issued (thread 0)
+    auto issue = [&](int st) {
+        const int rows = min(RPS, dv - st * RPS);
+        const uint32_t bytes = (uint32_t)(rows * DK * 4);
+        uint64_t *b = &bars[st % NST];
+        tc::mbar_arrive_expect_tx(b, bytes);
+        tc::bulk_load(tc::smem_u32(ring[st % NST]), S + (size_t)st * RPS * DK, bytes, b);
+        ++issued;
+    };
+    if (tid == 0) {
+        for (int i = 0; i < NST; ++i) tc::mbar_init(&bars[i], 1);
+        tc::fence_mbar_init();
+        for (int st = 0; st < min(NST, nstage); ++st) issue(st);
+    }
+
+    // stage the sample x = x_prev (prefix pair) or k, normalised below
+    // (same-step pair), q, k, v and beta
+    const bool same = p.pairing != 0;
+    const T *q = static_cast<const T *>(p.q) + (size_t)nh * DK;
+    const T *k = static_cast<const T *>(p.k) + (size_t)nh * DK;
+    const T *v = static_cast<const T *>(p.v) + (size_t)nh * dv;
+    const T *beta = static_cast<const T *>(p.beta) + (size_t)nh * (vi.per_channel ? dv : 1);
+    {
+        const float *xp = same ? nullptr : p.x_prev + (size_t)nh * DK;
+        float px = 0.f, pq = 0.f, pk = 0.f;
+        for (int i = tid; i < DK; i += blockDim.x) {
+            const float qv = to_f32(q[i]), kv = to_f32(k[i]), xv = same ? kv : xp[i];
+            xs[i] = xv;
+            qs[i] = qv;
+            ks[i] = kv;
+            px += xv * xv;
+            pq += xv * qv;
+            pk += kv * kv;
+        }
+        for (int i = tid; i < dv; i += blockDim.x) {
+            ys[i] = to_f32(v[i]);
+            bs[i] = to_f32(beta[vi.per_channel ? i : 0]);
+        }
+        px = group_sum<32>(px);
+        pq = group_sum<32>(pq);
+        pk = group_sum<32>(pk);
+        if (lane == 0) { red[0][warp] = px; red[1][warp] = pq; red[2][warp] = pk; }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float n = 0.f, xq = 0.f, knorm = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) { n += red[0][w]; xq += red[1][w]; knorm += red[2][w]; }
+        if (same) {  // x = k / |k|: its energy and its product with q
+            const float inv = knorm > 0.f ? rsqrtf(knorm) : 0.f;
+            n *= inv * inv;
+            xq *= inv;
+            hsc[4] = inv;
+        }
+        hsc[0] = n > 0.f ? 1.f / (p.eps + n) : 0.f;  // eta = beta * inv_den
+        hsc[1] = xq;
+        hsc[2] = p.lambda[nh % p.H];
+        hsc[3] = knorm;
+    }
+    __syncthreads();
+    if (same) {
+        for (int i = tid; i < DK; i += blockDim.x) xs[i] *= hsc[4];
+        __syncthreads();
+    }
+
+    const int sl = lane % LPR, rsub = warp * RPW + lane / LPR;
+    float4 xr[NV4], qr[NV4];
+#pragma unroll
+    for (int i = 0; i < NV4; ++i) {
+        xr[i] = *reinterpret_cast<const float4 *>(&xs[4 * (sl + LPR * i)]);
+        qr[i] = *reinterpret_cast<const float4 *>(&qs[4 * (sl + LPR * i)]);
+    }
+    const float inv_den = hsc[0], xq = hsc[1], lam = hsc[2];
+    bool ok = true;
+    int first_bad = nstage;  // the first stage whose wait gave up
+    for (int st = 0; st < nstage; ++st) {
+        const int slot = st % NST;
+        if (ok) {
+            ok = tc::mbar_wait_timeout(&bars[slot], (uint32_t)(st / NST) & 1u, 2000000000ull);
+            if (!ok) first_bad = st;
+        }
+        const int row = st * RPS + rsub;
+        if (ok && row < dv) {
+            const float4 *src = reinterpret_cast<const float4 *>(&ring[slot][rsub * DK]);
+            float4 cur[NV4];
+#pragma unroll
+            for (int i = 0; i < NV4; ++i) cur[i] = src[sl + LPR * i];
+            float sq = 0.f, sx = 0.f;
+#pragma unroll
+            for (int i = 0; i < NV4; ++i) {
+                sq += cur[i].x * qr[i].x + cur[i].y * qr[i].y + cur[i].z * qr[i].z + cur[i].w * qr[i].w;
+                sx += cur[i].x * xr[i].x + cur[i].y * xr[i].y + cur[i].z * xr[i].z + cur[i].w * xr[i].w;
+            }
+            sq = group_sum<LPR>(sq);
+            if (vi.regression) sx = group_sum<LPR>(sx);
+            const float eta = bs[row] * inv_den;
+            const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
+            const float y = ys[row];
+            const float ge = eta * (vi.regression ? y - sx : y);
+            float4 *dst = reinterpret_cast<float4 *>(S + (size_t)row * DK);
+#pragma unroll
+            for (int i = 0; i < NV4; ++i) {
+                float4 o;
+                o.x = alpha * cur[i].x + ge * xr[i].x;
+                o.y = alpha * cur[i].y + ge * xr[i].y;
+                o.z = alpha * cur[i].z + ge * xr[i].z;
+                o.w = alpha * cur[i].w + ge * xr[i].w;
+                dst[sl + LPR * i] = o;
+            }
+            if (sl == 0) static_cast<T *>(p.out)[(size_t)nh * dv + row] = from_f32<T>(alpha * sq + ge * xq);
+        }
+        // every thread has read the stage: it may be written again
+        tc::fence_proxy_async();
+        __syncthreads();
+        if (tid == 0 && ok && st + NST < nstage) issue(st + NST);
+    }
+    // carry: x_prev <- phi(k_t) (the same-step pair may leave it out)
+    if (p.x_prev) {
+        const float kn = hsc[3];
+        const float kinv = kn > 0.f ? rsqrtf(kn) : 0.f;
+        for (int i = tid; i < DK; i += blockDim.x) p.x_prev[(size_t)nh * DK + i] = ks[i] * kinv;
+    }
+    if (tid == 0 && !ok) {
+        atomicAdd(&g_decode_wait_timeouts, 1u);
+        // copies still in flight (from the stage that gave up on) must land
+        // before the block leaves
+        for (int st = first_bad; st < issued; ++st)
+            (void)tc::mbar_wait_timeout(&bars[st % NST], (uint32_t)(st / NST) & 1u, 2000000000ull);
+    }
+}
+
 // Window variants (Falcon-3/3A, W = 2..8 samples per update), laid out as
 // decode1_kernel: LPR lanes per row of S, HPB (n,h) pairs per block so the
 // whole grid is resident at once, and the first rows of the state requested
@@ -520,6 +685,14 @@ template <typename T, int DK>
 static void launch_decode_dk(const DecodeParams &p, cudaStream_t s) {
     switch (variant_info(p.variant, p.window).window) {
         case 1: {
+            if constexpr (DK == 64) {
+                // bulk copies need a 16-byte aligned state; more than 64 value
+                // rows would need more stages than the ring holds
+                if ((reinterpret_cast<uintptr_t>(p.state) & 15u) == 0 && p.dv <= 64) {
+                    decode1r_kernel<T, DK><<<p.N * p.H, 128, 0, s>>>(p);
+                    return;
+                }
+            }
             constexpr int hpb = decode1_hpb(DK);
             decode1_kernel<T, DK><<<(p.N * p.H + hpb - 1) / hpb, 32 * decode1_warps(DK), 0, s>>>(p);
             return;
@@ -551,6 +724,12 @@ int launch_carry(const CarryParams &p, cudaStream_t s) {
         case 128: carry_kernel<T, 128><<<p.B * p.H, 128, 0, s>>>(p); return 0;
     }
     return -3;
+}
+
+unsigned int decode_wait_timeouts() {
+    unsigned int v = 0;
+    cudaMemcpyFromSymbol(&v, g_decode_wait_timeouts, sizeof(v));
+    return v;
 }
 
 template int launch_decode<float>(const DecodeParams &, cudaStream_t);

@@ -27,6 +27,7 @@ size_t split_chunk_ws_bytes(const FwdParams &p);
 size_t split_chunk_images_ws_bytes(const FwdParams &p);
 // Number of tensor-core thread blocks that gave up on a bounded wait.
 unsigned int split_wait_timeouts();
+unsigned int decode_wait_timeouts();
 // bf16 Falcon-2A chunk-parallel forward, d_k = d_v = 128, chunk 64, on
 // tcgen05 (dS per chunk, state scan, outputs); returns 1 for shapes it does
 // not cover.
