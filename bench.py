@@ -589,7 +589,7 @@ def run_workloads(args):
         if args.only and n != args.only:
             continue
         forms = list(w["forms"])
-        if n == 2:
+        if n in (2, 4):  # the parallel forms beside the recurrent kernel on the same inputs
             forms = ["chunk", "masked", "recurrent"]
         for var in w["variants"]:
             for form in forms:

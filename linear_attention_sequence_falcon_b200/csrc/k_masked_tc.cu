@@ -66,7 +66,7 @@ constexpr uint32_t M_PD = M_MT + TFM * 4;              // fp32: (P o Dm)_II (wit
 constexpr uint32_t M_OF = M_PD + TFM * 4;              // fp32: D_c (accumulated O)
 constexpr uint32_t M_ET = M_OF + TFM * 4;              // bf16: E~_I^T, staged for the workspace
 constexpr uint32_t M_VEC = M_ET + TB;                  // per-token vectors
-constexpr uint32_t M_GAM = M_VEC + 6 * BM * 4;        // gamma_IJ of the row block, J < I
+constexpr uint32_t M_GAM = M_VEC + 9 * BM * 4;        // gamma_IJ of the row block, J < I
 constexpr uint32_t M_BAR = M_GAM + NGMAX * 4;
 constexpr uint32_t M_SMEM = M_BAR + 192 + 1024;        // + alignment slack
 // the inverse's fp32 tiles D, K, K^2, T over the loop region (idle in the diagonal step)
@@ -135,8 +135,11 @@ __device__ __forceinline__ void mma64(const float *A, const float *B, float (&ac
 
 }  // namespace
 
+template <int W>
 __global__ void __launch_bounds__(NTHM, 1)
     masked_tc_kernel(FwdParams p, uint8_t *xs_ws, uint8_t *es_ws, float *gend_ws) {
+    // tokens per row block: its samples (the window reaches W - 1 back) fill the 64 rows
+    constexpr int TOK = BM + 1 - W;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = tc::smem_u32(smem_raw);
     uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -147,7 +150,10 @@ __global__ void __launch_bounds__(NTHM, 1)
     float *DI = reinterpret_cast<float *>(sm + M_RING), *KI = DI + TFM, *K2 = KI + TFM, *TI = K2 + TFM;
     float *vec = reinterpret_cast<float *>(sm + M_VEC);
     float *vG = vec, *veta = vec + BM, *vla = vec + 2 * BM, *va = vec + 3 * BM, *vc = vec + 4 * BM,
-          *vb = vec + 5 * BM;
+          *vb = vec + 5 * BM, *vsq = vec + 6 * BM, *vbeta = vec + 7 * BM, *valpha = vec + 8 * BM;
+    // window system (W > 1): the sample Gram, the token-sample scores, the
+    // accumulated pair terms per sample row and the block's residual sums
+    float *AT = MT, *PT = PD, *VT = DI, *RT = KI;
     float *vgam = reinterpret_cast<float *>(sm + M_GAM);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + M_BAR);
     uint64_t *txb = bar, *teb = bar + NRING, *bp1 = bar + 2 * NRING, *bp2 = bp1 + 2, *bd = bp2 + 2, *bao = bd + 1;
@@ -157,8 +163,8 @@ __global__ void __launch_bounds__(NTHM, 1)
     const bool compute = tid < NTHC, issuer = tid == NTHC;  // warps 0-7 compute; warp 8 lane 0 issues
     const int quarter = warp & 3, chalf = warp >> 2;
     const int row = quarter * 32 + lane;  // tensor-memory lane of a compute thread
-    const bool reg = p.variant == F1;
-    const int L = p.L, nb = (L + BM - 1) / BM;
+    const bool reg = p.variant == F1 || p.variant == F3;
+    const int L = p.L, nb = (L + TOK - 1) / TOK;
     const size_t bh = blockIdx.x;
     const float lam = p.lambda[bh % p.H];
     const __nv_bfloat16 *kh = static_cast<const __nv_bfloat16 *>(p.k) + bh * (size_t)L * BM;
@@ -236,28 +242,33 @@ __global__ void __launch_bounds__(NTHM, 1)
     };
 
     for (int I = 0; I < nb; ++I) {
-        const int I0 = I * BM, n = min(BM, L - I0);
-        // ---- the block's inputs: samples x_t = phi(k_{t-1}) (prefix pair;
-        //      phi(k_t) same-step), q, v, the steps and the decays
+        const int I0 = I * TOK, n = min(TOK, L - I0);
+        // sample row r holds sample i0 + r (the window of token I0 + tau covers
+        // rows tau .. tau + W - 1); rows from nsr on, and samples before the
+        // sequence, are empty
+        const int i0 = I0 - (W - 1), nsr = n + W - 1;
+        // ---- the block's inputs: samples x_i = phi(k_{i-1}) (prefix pair;
+        //      phi(k_i) same-step) with their targets y_i = v_i, q, the window
+        //      energies, the steps and the decays
         if (issuer) tc::bulk_wait_read();  // the stores of the last block have read AQ and ET
         __syncthreads();
         if (compute) {
             uint4 lq[2], lv[2];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const int e = tid + NTHC * j;  // 16-byte piece: row e / 8, columns 8 (e % 8)..
-                const bool in = (e >> 3) < n;
+                const int e = tid + NTHC * j, r = e >> 3, c = e & 7;  // 16-byte piece: row r, columns 8c..
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                lq[j] = in ? wt::ld16(qh + (size_t)I0 * BM + 8 * e) : z;
-                lv[j] = in ? wt::ld16(vh + (size_t)I0 * BM + 8 * e) : z;
+                lq[j] = r < n ? wt::ld16(qh + (size_t)(I0 + r) * BM + 8 * c) : z;
+                lv[j] = (r < nsr && i0 + r >= 0) ? wt::ld16(vh + (size_t)(i0 + r) * BM + 8 * c) : z;
             }
             uint32_t kw[8];
             float bv[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int r = warp * 8 + i, t = I0 + r, kr = p.pairing == 0 ? t - 1 : t;
-                kw[i] = (r < n && kr >= 0) ? *reinterpret_cast<const uint32_t *>(kh + (size_t)kr * BM + 2 * lane) : 0u;
-                bv[i] = r < n ? __bfloat162float(bth[t]) : 0.f;
+                const int r = warp * 8 + i, si = i0 + r, kr = p.pairing == 0 ? si - 1 : si;
+                kw[i] = (r < nsr && si >= 0 && kr >= 0)
+                            ? *reinterpret_cast<const uint32_t *>(kh + (size_t)kr * BM + 2 * lane) : 0u;
+                bv[i] = r < n ? __bfloat162float(bth[I0 + r]) : 0.f;
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -269,11 +280,8 @@ __global__ void __launch_bounds__(NTHM, 1)
                 *reinterpret_cast<float2 *>(XF + r * LDM + 2 * lane) = make_float2(y0, y1);
                 *reinterpret_cast<uint32_t *>(sm + M_AQ + tc::sw128(r, lane >> 2) + (lane & 3) * 4) = pack2(y0, y1);
                 if (lane == 0) {
-                    const float nn = ss * inv * inv;  // the sample's energy (0: no sample)
-                    float eta = 0.f, alpha = 1.f;
-                    if (r < n) step_and_decay(bv[i], nn, p.eps, lam, eta, alpha);
-                    veta[r] = eta;
-                    vla[r] = __logf(alpha);
+                    vsq[r] = ss * inv * inv;  // the sample's energy (0: no sample)
+                    vbeta[r] = bv[i];
                 }
             }
 #pragma unroll
@@ -281,6 +289,18 @@ __global__ void __launch_bounds__(NTHM, 1)
                 const int e = tid + NTHC * j, r = e >> 3, c = e & 7;
                 *reinterpret_cast<uint4 *>(sm + M_AQ + tc::sw128(64 + r, c)) = lq[j];
                 wt::st8(YF + r * LDM + 8 * c, lv[j]);
+            }
+            tc::named_sync(1, NTHC);
+            if (tid < BM) {  // token tau: its window's energy, step and decay
+                const int t = tid;
+                float nn = 0.f;
+#pragma unroll
+                for (int m = 0; m < W; ++m) nn += vsq[min(t + m, BM - 1)];
+                float eta = 0.f, alpha = 1.f;
+                if (t < n) step_and_decay(vbeta[t], nn, p.eps, lam, eta, alpha);
+                veta[t] = eta;
+                valpha[t] = alpha;
+                vla[t] = __logf(alpha);
             }
             tc::named_sync(1, NTHC);
             if (warp == 0) {  // block-local cumulative log decay G_t
@@ -444,7 +464,27 @@ __global__ void __launch_bounds__(NTHM, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) r[i] = 0.f;
             }
-            if (quarter < 2) {  // rows 0-63 (regression): M_II (with the steps), R = Y - D_a (accumulated)
+            if (W > 1) {
+                // window system: the sample Gram and V (rows 0-63, regression),
+                // the token-sample scores and D_c (accumulated O) (rows 64-127)
+                if (quarter < 2) {
+                    if (reg) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            AT[row * LDM + chalf * 32 + i] = v[i];
+                            VT[row * LDM + chalf * 32 + i] = r[i];
+                        }
+                    }
+                } else {
+                    const int t = row - 64;
+                    const float c = vc[t];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        PT[t * LDM + chalf * 32 + i] = v[i];
+                        OF[t * LDM + chalf * 32 + i] = c * r[i];
+                    }
+                }
+            } else if (quarter < 2) {  // rows 0-63 (regression): M_II (with the steps), R = Y - D_a (accumulated)
                 if (reg) {
                     const int t = row;
                     const float gm = t > 0 ? vG[t - 1] : 0.f, a = va[t];
@@ -469,7 +509,7 @@ __global__ void __launch_bounds__(NTHM, 1)
             ok = named_sync_and(1, NTHC, ok);
         }
         MT(7);
-        if (compute && ok) {
+        if (compute && ok && W == 1) {
             const int rb = (warp & 3) * 16, cb = (warp >> 2) * 32;
             float acc[4][4];
             if (reg) {
@@ -566,6 +606,83 @@ __global__ void __launch_bounds__(NTHM, 1)
             mma64<true, false, true>(YF, XF, sacc, 0, 64, vb);
             tc::fence_proxy_async();
         }
+        if (compute && ok && W > 1) {
+            // ---- the window system in token order.  Thread (j, q): value
+            //      channel j, sample rows 16q..16q+15 of the running sums
+            //        R[r] = sum_{s <= t} e^{G_t - G_s} eta_s r_{s, r}   (r in W_s),
+            //      R <- alpha_t R + eta_t r_t after token t.  Token t's residuals
+            //        r_{t, rho} = y_rho - a_t V[rho] - (A R)[rho], rho = t .. t+W-1
+            //      (inner product: r = y), and o_t = D_c (accumulated) + P[t] R.
+            //      After the last token R is the block's residual sum per sample
+            //      row, weighted to the block's end.
+            const int jc = tid >> 2, qr = tid & 3;
+            float racc[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) racc[q] = 0.f;
+            for (int t = 0; t < n; ++t) {
+                const float a = va[t], eta = veta[t], alpha = valpha[t];
+                float rm[W];
+#pragma unroll
+                for (int m = 0; m < W; ++m) {
+                    const int rho = t + m;
+                    float res = YF[rho * LDM + jc];
+                    if (reg) {
+                        const float4 *ar = reinterpret_cast<const float4 *>(AT + rho * LDM + 16 * qr);
+                        float d = 0.f;
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 av = ar[q4];
+                            d += av.x * racc[4 * q4] + av.y * racc[4 * q4 + 1] + av.z * racc[4 * q4 + 2] +
+                                 av.w * racc[4 * q4 + 3];
+                        }
+                        d += __shfl_xor_sync(0xffffffffu, d, 1);
+                        d += __shfl_xor_sync(0xffffffffu, d, 2);
+                        res -= a * VT[rho * LDM + jc] + d;
+                    }
+                    rm[m] = res;
+                }
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    float add = 0.f;
+#pragma unroll
+                    for (int m = 0; m < W; ++m) add += (16 * qr + q == t + m) ? rm[m] : 0.f;
+                    racc[q] = alpha * racc[q] + eta * add;
+                }
+                const float4 *pr = reinterpret_cast<const float4 *>(PT + t * LDM + 16 * qr);
+                float o = 0.f;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 pv = pr[q4];
+                    o += pv.x * racc[4 * q4] + pv.y * racc[4 * q4 + 1] + pv.z * racc[4 * q4 + 2] +
+                         pv.w * racc[4 * q4 + 3];
+                }
+                o += __shfl_xor_sync(0xffffffffu, o, 1);
+                o += __shfl_xor_sync(0xffffffffu, o, 2);
+                if (qr == 0) oh[(size_t)(I0 + t) * BM + jc] = __float2bfloat16_rn(OF[t * LDM + jc] + o);
+            }
+            // the block's residual sums: fp32 for the state, bf16 (row j, sample
+            // rows along K) for the later row blocks
+#pragma unroll
+            for (int q = 0; q < 16; ++q) RT[(16 * qr + q) * LDM + jc] = racc[q];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint4 u;
+                u.x = pack2(racc[8 * h2 + 0], racc[8 * h2 + 1]);
+                u.y = pack2(racc[8 * h2 + 2], racc[8 * h2 + 3]);
+                u.z = pack2(racc[8 * h2 + 4], racc[8 * h2 + 5]);
+                u.w = pack2(racc[8 * h2 + 6], racc[8 * h2 + 7]);
+                *reinterpret_cast<uint4 *>(sm + M_ET + tc::sw128(jc, 2 * qr + h2)) = u;
+            }
+            tc::named_sync(1, NTHC);
+            // S <- e^{G_Iend} S + R^T X
+            const float gI = __expf(GE);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc[nt][e] *= gI;
+            mma64<true, false>(RT, XF, sacc, 0, 64);
+            tc::fence_proxy_async();
+        }
         tc::fence_before_sync();
         ok = __syncthreads_and(ok);
         if (!ok) break;
@@ -605,21 +722,32 @@ bool al16m(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; 
 
 }  // namespace
 
-bool masked_tc_covers(const FwdParams &p) {
-    return (p.variant == F1 || p.variant == F1A) && p.dk == BM && p.dv == BM && p.form == 1 && p.L > 0 &&
-           (p.L + BM - 1) / BM <= NGMAX;
+// samples per update the kernel runs with: 1 (Falcon-1/1A, or a window of
+// one), 2-4 (Falcon-3/3A); 0: not covered
+int masked_tc_window(const FwdParams &p) {
+    if (p.dk != BM || p.dv != BM || p.form != 1 || p.L <= 0) return 0;
+    int w = 0;
+    if (p.variant == F1 || p.variant == F1A) w = 1;
+    if ((p.variant == F3 || p.variant == F3A) && p.window >= 1 && p.window <= 4) w = p.window;
+    if (w == 0) return 0;
+    const int tok = BM + 1 - w;
+    return (p.L + tok - 1) / tok <= NGMAX ? w : 0;
 }
 
+bool masked_tc_covers(const FwdParams &p) { return masked_tc_window(p) != 0; }
+
 size_t masked_tc_ws_bytes(const FwdParams &p) {
-    const size_t BH = (size_t)p.B * p.H, nb = (p.L + BM - 1) / BM;
+    const int w = masked_tc_window(p);
+    const size_t BH = (size_t)p.B * p.H, nb = (p.L + BM - w) / (BM + 1 - (w ? w : 1));
     return 2 * al256m(BH * nb * TB) + al256m(BH * nb * sizeof(float));
 }
 
-// 1: not covered (the caller takes the CUDA-core path); 0 launched; < 0 an error
-int launch_masked_tc(const FwdParams &p, void *ws, cudaStream_t s) {
-    if (!masked_tc_covers(p)) return 1;
-    if (!al16m(p.q) || !al16m(p.k) || !al16m(p.v) || !al16m(p.out)) return 1;
-    const size_t BH = (size_t)p.B * p.H, nb = (p.L + BM - 1) / BM;
+namespace {
+
+template <int W>
+int launch_w(const FwdParams &p, void *ws, cudaStream_t s) {
+    constexpr int TOK = BM + 1 - W;
+    const size_t BH = (size_t)p.B * p.H, nb = (p.L + TOK - 1) / TOK;
     uint8_t *base = static_cast<uint8_t *>(ws);
     uint8_t *xs = base, *es = base + al256m(BH * nb * TB);
     float *gend = reinterpret_cast<float *>(es + al256m(BH * nb * TB));
@@ -627,18 +755,27 @@ int launch_masked_tc(const FwdParams &p, void *ws, cudaStream_t s) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr[dev]) {
-        cudaFuncSetAttribute(masked_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)M_SMEM);
+        cudaFuncSetAttribute(masked_tc_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)M_SMEM);
         if (dev >= 0 && dev < 64) attr[dev] = true;
     }
-    masked_tc_kernel<<<(unsigned)BH, NTHM, M_SMEM, s>>>(p, xs, es, gend);
+    masked_tc_kernel<W><<<(unsigned)BH, NTHM, M_SMEM, s>>>(p, xs, es, gend);
     return cudaGetLastError() == cudaSuccess ? 0 : -7;
 }
 
-#ifdef FALCON_TC_DEBUG
-extern "C" int falcon_masked_debug_timer_set(long long *ptr) {
-    return cudaMemcpyToSymbol(g_masked_tim, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;
+}  // namespace
+
+// 1: not covered (the caller takes the CUDA-core path); 0 launched; < 0 an error
+int launch_masked_tc(const FwdParams &p, void *ws, cudaStream_t s) {
+    const int w = masked_tc_window(p);
+    if (w == 0) return 1;
+    if (!al16m(p.q) || !al16m(p.k) || !al16m(p.v) || !al16m(p.out)) return 1;
+    switch (w) {
+        case 1: return launch_w<1>(p, ws, s);
+        case 2: return launch_w<2>(p, ws, s);
+        case 3: return launch_w<3>(p, ws, s);
+        default: return launch_w<4>(p, ws, s);
+    }
 }
-#endif
 
 unsigned int masked_wait_timeouts() {
     unsigned int v = 0;

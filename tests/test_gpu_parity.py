@@ -244,6 +244,29 @@ def test_masked_tensor_core_options(F, variant):
     check(F, d, variant, "masked", phi="identity")
 
 
+@pytest.mark.parametrize("L", [1, 60, 61, 62, 122, 123, 300])
+@pytest.mark.parametrize("w", [2, 3, 4])
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+def test_masked_tensor_core_windows(F, variant, w, L):
+    """The masked tensor-core kernel with windows (bf16, d = 64): row blocks
+    of 65 - B_w tokens whose window samples fill 64 rows; one token, block
+    edges and many blocks."""
+    d = gen.draw(variant, 2, 2, L, 64, 64, seed=360 + L + 7 * w, dtype="bf16")
+    check(F, d, variant, "masked", window=w)
+
+
+@pytest.mark.parametrize("variant", ["F3", "F3A"])
+def test_masked_tensor_core_window_options(F, variant):
+    """Windowed masked form with the same-step pair and the identity map,
+    strong forgetting, and the decay floor."""
+    d = gen.draw(variant, 1, 2, 250, 64, 64, seed=370, dtype="bf16", key_scale=0.125)
+    check(F, d, variant, "masked", window=3, pairing="same_step", phi="identity")
+    d = gen.draw(variant, 1, 3, 300, 64, 64, seed=371, dtype="bf16", lam=0.999)
+    check(F, d, variant, "masked", window=4)
+    d = gen.draw(variant, 1, 2, 200, 64, 64, seed=372, dtype="bf16", lam=0.9, key_scale=0.05)
+    check(F, d, variant, "masked", window=2, phi="identity")
+
+
 @pytest.mark.parametrize("variant", ["F1", "F1A"])
 def test_masked_misaligned_inputs_take_the_cuda_core_kernel(F, variant):
     """Inputs that are not 16-byte aligned (a view one element into its
