@@ -1,5 +1,5 @@
-// k_masked_tc.cu -- the masked-parallel form of Falcon-1 and Falcon-1A on the
-// tcgen05 tensor cores (bf16 inputs, d_k = d_v = 64, S_0 = 0).
+// k_masked_tc.cu -- the masked-parallel form of Falcon-1/1A and Falcon-3/3A (windows
+// of 1-4 samples) on the tcgen05 tensor cores (bf16 inputs, d_k = d_v = 64, S_0 = 0).
 //
 // Method: "masked-parallel: every step at once through a causal mask" (page
 // "Fast Weight Attention for Continual Learning", 方法/计算形式与数值稳定;
@@ -21,6 +21,17 @@
 // e^{Gamma_t-...}), gamma_IJ and the column factor, each <= 1.  The diagonal
 // block then solves its own triangle: R_I = Y_I - D_a (accumulated), E_I =
 // (I + M_II)^{-1} R_I, O_I = D_c (accumulated) + (P o Dm)_II E_I.
+//
+// Windows (Falcon-3/3A, B_w samples per update): token t's unknowns are the
+// residuals r_{t,i} of the samples i in its window W_t, and the sums above run
+// over the window's samples as well.  A row block then holds 65 - B_w tokens,
+// so that the samples their windows reach fill the same 64 rows; the pair
+// products apply, per sample row, each earlier block's residual sums
+//   R~_J[i] = sum_{s in J, i in W_s} e^{Gamma_Jend-Gamma_s} eta_s r_{s,i},
+// and the diagonal block walks its C*B_w system token by token with the
+// decayed running sums R <- alpha_t R + eta_t r_t (every factor <= 1):
+//   r_{t,i} = y_i - a_t V[i] - (A_II R)[i],  o_t = c_t (accumulated) + P_II[t] R,
+// and R after its last token is the block's R~.
 //
 // One block per (b, h): eight compute warps and an issuing warp.  The pair
 // products run on tcgen05 (bf16 operands in
@@ -619,46 +630,63 @@ __global__ void __launch_bounds__(NTHM, 1)
             float racc[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q) racc[q] = 0.f;
-            for (int t = 0; t < n; ++t) {
-                const float a = va[t], eta = veta[t], alpha = valpha[t];
-                float rm[W];
+            // tokens in groups of 16 (t = 16 g + v, v unrolled): token t's rows
+            // t + m fall in this thread's rows 16 qr .. 16 qr + 15 at the fixed
+            // index v + m when qr == g, or v + m - 16 when qr == g + 1
+            for (int g = 0; 16 * g < n; ++g) {
 #pragma unroll
-                for (int m = 0; m < W; ++m) {
-                    const int rho = t + m;
-                    float res = YF[rho * LDM + jc];
-                    if (reg) {
-                        const float4 *ar = reinterpret_cast<const float4 *>(AT + rho * LDM + 16 * qr);
-                        float d = 0.f;
+                for (int v = 0; v < 16; ++v) {
+                    const int t = 16 * g + v;
+                    if (t >= n) break;
+                    const float a = va[t], eta = veta[t], alpha = valpha[t];
+                    float rm[W];
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const float4 av = ar[q4];
-                            d += av.x * racc[4 * q4] + av.y * racc[4 * q4 + 1] + av.z * racc[4 * q4 + 2] +
-                                 av.w * racc[4 * q4 + 3];
+                    for (int m = 0; m < W; ++m) {
+                        const int rho = t + m;
+                        float res = YF[rho * LDM + jc];
+                        if (reg) {
+                            const float4 *ar = reinterpret_cast<const float4 *>(AT + rho * LDM + 16 * qr);
+                            float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; q4 += 2) {
+                                const float4 av = ar[q4], aw = ar[q4 + 1];
+                                d0 += av.x * racc[4 * q4] + av.y * racc[4 * q4 + 1] + av.z * racc[4 * q4 + 2] +
+                                      av.w * racc[4 * q4 + 3];
+                                d1 += aw.x * racc[4 * q4 + 4] + aw.y * racc[4 * q4 + 5] +
+                                      aw.z * racc[4 * q4 + 6] + aw.w * racc[4 * q4 + 7];
+                            }
+                            float d = d0 + d1;
+                            d += __shfl_xor_sync(0xffffffffu, d, 1);
+                            d += __shfl_xor_sync(0xffffffffu, d, 2);
+                            res -= a * VT[rho * LDM + jc] + d;
                         }
-                        d += __shfl_xor_sync(0xffffffffu, d, 1);
-                        d += __shfl_xor_sync(0xffffffffu, d, 2);
-                        res -= a * VT[rho * LDM + jc] + d;
+                        rm[m] = eta * res;
                     }
-                    rm[m] = res;
-                }
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    float add = 0.f;
+                    for (int q = 0; q < 16; ++q) racc[q] *= alpha;
 #pragma unroll
-                    for (int m = 0; m < W; ++m) add += (16 * qr + q == t + m) ? rm[m] : 0.f;
-                    racc[q] = alpha * racc[q] + eta * add;
-                }
-                const float4 *pr = reinterpret_cast<const float4 *>(PT + t * LDM + 16 * qr);
-                float o = 0.f;
+                    for (int m = 0; m < W; ++m) {
+                        if (v + m < 16) {
+                            if (qr == g) racc[v + m] += rm[m];
+                        } else {
+                            if (qr == g + 1) racc[v + m - 16] += rm[m];
+                        }
+                    }
+                    const float4 *pr = reinterpret_cast<const float4 *>(PT + t * LDM + 16 * qr);
+                    float o0 = 0.f, o1 = 0.f;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 pv = pr[q4];
-                    o += pv.x * racc[4 * q4] + pv.y * racc[4 * q4 + 1] + pv.z * racc[4 * q4 + 2] +
-                         pv.w * racc[4 * q4 + 3];
+                    for (int q4 = 0; q4 < 4; q4 += 2) {
+                        const float4 pv = pr[q4], pw = pr[q4 + 1];
+                        o0 += pv.x * racc[4 * q4] + pv.y * racc[4 * q4 + 1] + pv.z * racc[4 * q4 + 2] +
+                              pv.w * racc[4 * q4 + 3];
+                        o1 += pw.x * racc[4 * q4 + 4] + pw.y * racc[4 * q4 + 5] + pw.z * racc[4 * q4 + 6] +
+                              pw.w * racc[4 * q4 + 7];
+                    }
+                    float o = o0 + o1;
+                    o += __shfl_xor_sync(0xffffffffu, o, 1);
+                    o += __shfl_xor_sync(0xffffffffu, o, 2);
+                    if (qr == 0) oh[(size_t)(I0 + t) * BM + jc] = __float2bfloat16_rn(OF[t * LDM + jc] + o);
                 }
-                o += __shfl_xor_sync(0xffffffffu, o, 1);
-                o += __shfl_xor_sync(0xffffffffu, o, 2);
-                if (qr == 0) oh[(size_t)(I0 + t) * BM + jc] = __float2bfloat16_rn(OF[t * LDM + jc] + o);
             }
             // the block's residual sums: fp32 for the state, bf16 (row j, sample
             // rows along K) for the later row blocks
