@@ -424,6 +424,7 @@ __global__ void __launch_bounds__(NTHM, 1)
                     MT(4);
                     // P2(J): [R; O] += [gA; gP] E~_J
                     r = r && wait_e(J);
+                    MT(12);
                     if (r) {
                         tc::mma_k64(tbase + TM_ACC, dA0 + (uint64_t)b * 2 * kTileDesc,
                                     dE0 + (uint64_t)(J % NRING) * kTileDesc, kIdesc, J > 0);
@@ -804,6 +805,12 @@ int launch_masked_tc(const FwdParams &p, void *ws, cudaStream_t s) {
         default: return launch_w<4>(p, ws, s);
     }
 }
+
+#ifdef FALCON_TC_DEBUG
+extern "C" int falcon_masked_debug_timer_set(long long *ptr) {
+    return cudaMemcpyToSymbol(g_masked_tim, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 unsigned int masked_wait_timeouts() {
     unsigned int v = 0;
