@@ -26,8 +26,9 @@
 //
 // One block per (b, h) walks the chunks; S stays in fp32 registers (thread:
 // row j, 64 columns) with its bf16 copy in shared memory as the operand of
-// S_0 [X;Q]^T.  The per-channel systems are solved by forward substitution,
-// one thread per channel.
+// S_0 [X;Q]^T.  The per-channel systems are solved by forward substitution
+// in blocks of 8 tokens, two threads (lanes of one warp) per channel: each
+// forms half of a block's sums over the earlier tokens, and both walk it.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -246,95 +247,116 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
         __syncthreads();
         F2T(4);
         tc::fence_after_sync();
-        // ---- per-channel systems (warps 0-3, thread = channel jj = tensor-memory lane)
-        if (tid < DD) {
-            const int jj = tid;
+        // ---- per-channel systems.  Two threads per channel, both lanes of one
+        //      warp: warp w takes channels 32 (w & 3) + 16 (w >> 2) .. +15 (inside
+        //      its tensor-memory lanes), lane l channel ... + l / 2.  Each thread
+        //      of a pair forms four of the eight sums over the rows before a
+        //      block of 8 tokens; the pair swaps them and both walk the block.
+        if (!unsafe) {
+            const int part = lane & 1, src = 16 * (warp >> 2) + (lane >> 1);
+            const int jj = 32 * quarter + src;
             const float gc = gcv[jj];
             float Z[64];
 #pragma unroll
             for (int s = 0; s < 64; ++s) Z[s] = 0.f;
-            if (!unsafe) {
-                // in blocks of 8 tokens: the sums over the rows before a block are one
-                // batch of independent dot products, the rows inside it a short walk
-                float Gprev = 0.f;
+            float Gprev = 0.f;
 #pragma unroll
-                for (int tb = 0; tb < 4; ++tb) {
-                    float xs[16];
-                    tc::tmem_ld16(tl + C_S + tb * 16, xs);
-                    tc::tmem_wait_ld();
+            for (int tb = 0; tb < 4; ++tb) {
+                float xs[16];
+                tc::tmem_ld16(tl + C_S + tb * 16, xs);
+                tc::tmem_wait_ld();
 #pragma unroll
-                    for (int hb = 0; hb < 2; ++hb) {
-                        const int t0 = tb * 16 + hb * 8;
-                        float r[8], kap[8], cr[8];
+                for (int i = 0; i < 16; ++i) xs[i] = __shfl_sync(0xffffffffu, xs[i], src);  // channel jj's row
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int t = t0 + i;
-                            const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
-                            const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
-                            const float G = Gt[gidx(t, jj)];
-                            r[i] = __expf(gc - G) * eta * (pair_get(sm, F_V, t, jj) - __expf(Gprev) * xs[hb * 8 + i]);
-                            kap[i] = __fdividef(eta, alpha);
-                            cr[i] = 0.f;
-                            Gprev = G;
-                        }
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int t0 = tb * 16 + hb * 8;
+                    float r[8], kap[8], cr[8];
 #pragma unroll
-                        for (int s = 0; s < t0; s += 4) {
+                    for (int i = 0; i < 8; ++i) {
+                        const int t = t0 + i;
+                        const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
+                        const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
+                        const float G = Gt[gidx(t, jj)];
+                        r[i] = __expf(gc - G) * eta * (pair_get(sm, F_V, t, jj) - __expf(Gprev) * xs[hb * 8 + i]);
+                        kap[i] = __fdividef(eta, alpha);
+                        Gprev = G;
+                    }
+                    // rows t0 + 4 part .. + 3 of this thread, then the partner's four
+                    float cm[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float *arow = At + (t0 + 4 * part) * LDA;
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const float4 a = *reinterpret_cast<const float4 *>(At + (t0 + i) * LDA + s);
-                                cr[i] = fmaf(a.x, Z[s], fmaf(a.y, Z[s + 1], fmaf(a.z, Z[s + 2], fmaf(a.w, Z[s + 3], cr[i]))));
-                            }
-                        }
+                    for (int s = 0; s < t0; s += 4) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            float acc = cr[i];
-#pragma unroll
-                            for (int s = t0; s < t0 + i; ++s) acc = fmaf(At[(t0 + i) * LDA + s], Z[s], acc);
-                            Z[t0 + i] = r[i] - kap[i] * acc;
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 a = *reinterpret_cast<const float4 *>(arow + i * LDA + s);
+                            cm[i] = fmaf(a.x, Z[s], fmaf(a.y, Z[s + 1], fmaf(a.z, Z[s + 2], fmaf(a.w, Z[s + 3], cm[i]))));
                         }
                     }
-                }
-            } else {
-                // F_s = eta_s E_s with one exponential per term (every exponent <= 0),
-                // the outputs from it, then Z_s = e^{G_C-G_s} F_s
-                float xs[64], F[64];
 #pragma unroll
-                for (int tb = 0; tb < 4; ++tb) {
-                    float v[16];
-                    tc::tmem_ld16(tl + C_S + tb * 16, v);
-                    tc::tmem_wait_ld();
+                    for (int i = 0; i < 4; ++i) {
+                        const float other = __shfl_xor_sync(0xffffffffu, cm[i], 1);
+                        cr[i] = part ? other : cm[i];
+                        cr[4 + i] = part ? cm[i] : other;
+                    }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) xs[tb * 16 + i] = v[i];
-                }
-                float Gprev = 0.f;
-#pragma unroll 1
-                for (int t = 0; t < CH; ++t) {
-                    const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
-                    float a = 0.f;
-                    for (int s = 0; s < t; ++s) a += __expf(Gprev - Gt[gidx(s, jj)]) * At[t * LDA + s] * F[s];
-                    F[t] = eta * (pair_get(sm, F_V, t, jj) - __expf(Gprev) * xs[t] - a);
-                    Gprev = Gt[gidx(t, jj)];
-                }
+                    for (int i = 0; i < 8; ++i) {
+                        float acc = cr[i];
 #pragma unroll
-                for (int tb = 0; tb < 4; ++tb) {
-                    float v[16];
-                    tc::tmem_ld16(tl + C_S + 64 + tb * 16, v);  // (S_0 Q^T)[j][t]
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) xs[tb * 16 + i] = v[i];
+                        for (int s = t0; s < t0 + i; ++s) acc = fmaf(At[(t0 + i) * LDA + s], Z[s], acc);
+                        Z[t0 + i] = r[i] - kap[i] * acc;
+                    }
                 }
-#pragma unroll 1
-                for (int t = 0; t < nt; ++t) {
-                    const float G = Gt[gidx(t, jj)];
-                    float o = __expf(G) * xs[t];
-                    for (int s = 0; s <= t; ++s) o += __expf(G - Gt[gidx(s, jj)]) * pm_get(sm, t, s) * F[s];
-                    static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + jj] = __float2bfloat16_rn(o);
-                }
-#pragma unroll 1
-                for (int s = 0; s < CH; ++s) F[s] *= __expf(gc - Gt[gidx(s, jj)]);
-#pragma unroll
-                for (int s = 0; s < 64; ++s) Z[s] = F[s];
             }
+            // Z^T row jj: each thread of the pair half of it
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const uint4 lo = pack8(&Z[c4 * 8]), hi = pack8(&Z[32 + c4 * 8]);
+                *reinterpret_cast<uint4 *>(sm + F_ZT + tc::sw128(jj, part * 4 + c4)) = part ? hi : lo;
+            }
+        } else if (tid < DD) {
+            // (warps 0-3, thread = channel jj = tensor-memory lane)
+            const int jj = tid;
+            const float gc = gcv[jj];
+            float Z[64];
+            // F_s = eta_s E_s with one exponential per term (every exponent <= 0),
+            // the outputs from it, then Z_s = e^{G_C-G_s} F_s
+            float xs[64], F[64];
+#pragma unroll
+            for (int tb = 0; tb < 4; ++tb) {
+                float v[16];
+                tc::tmem_ld16(tl + C_S + tb * 16, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) xs[tb * 16 + i] = v[i];
+            }
+            float Gprev = 0.f;
+#pragma unroll 1
+            for (int t = 0; t < CH; ++t) {
+                const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
+                float a = 0.f;
+                for (int s = 0; s < t; ++s) a += __expf(Gprev - Gt[gidx(s, jj)]) * At[t * LDA + s] * F[s];
+                F[t] = eta * (pair_get(sm, F_V, t, jj) - __expf(Gprev) * xs[t] - a);
+                Gprev = Gt[gidx(t, jj)];
+            }
+#pragma unroll
+            for (int tb = 0; tb < 4; ++tb) {
+                float v[16];
+                tc::tmem_ld16(tl + C_S + 64 + tb * 16, v);  // (S_0 Q^T)[j][t]
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) xs[tb * 16 + i] = v[i];
+            }
+#pragma unroll 1
+            for (int t = 0; t < nt; ++t) {
+                const float G = Gt[gidx(t, jj)];
+                float o = __expf(G) * xs[t];
+                for (int s = 0; s <= t; ++s) o += __expf(G - Gt[gidx(s, jj)]) * pm_get(sm, t, s) * F[s];
+                static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + jj] = __float2bfloat16_rn(o);
+            }
+#pragma unroll 1
+            for (int s = 0; s < CH; ++s) F[s] *= __expf(gc - Gt[gidx(s, jj)]);
+#pragma unroll
+            for (int s = 0; s < 64; ++s) Z[s] = F[s];
             // Z^T row jj
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8)
