@@ -259,7 +259,6 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
             float Z[64];
 #pragma unroll
             for (int s = 0; s < 64; ++s) Z[s] = 0.f;
-            float Gprev = 0.f;
 #pragma unroll
             for (int tb = 0; tb < 4; ++tb) {
                 float xs[16];
@@ -269,17 +268,28 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
                 for (int i = 0; i < 16; ++i) xs[i] = __shfl_sync(0xffffffffu, xs[i], src);  // channel jj's row
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb) {
-                    const int t0 = tb * 16 + hb * 8;
-                    float r[8], kap[8], cr[8];
+                    const int t0 = tb * 16 + hb * 8, tp = t0 + 4 * part;  // this thread's four tokens
+                    float r[8], kap[8], cr[8], rm[4], km[4];
+                    float Gp = tp > 0 ? Gt[gidx(tp - 1, jj)] : 0.f;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int t = t0 + i;
+                    for (int i = 0; i < 4; ++i) {
+                        const int t = tp + i;
                         const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
                         const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
                         const float G = Gt[gidx(t, jj)];
-                        r[i] = __expf(gc - G) * eta * (pair_get(sm, F_V, t, jj) - __expf(Gprev) * xs[hb * 8 + i]);
-                        kap[i] = __fdividef(eta, alpha);
-                        Gprev = G;
+                        const float x = part ? xs[hb * 8 + 4 + i] : xs[hb * 8 + i];
+                        rm[i] = __expf(gc - G) * eta * (pair_get(sm, F_V, t, jj) - __expf(Gp) * x);
+                        km[i] = __fdividef(eta, alpha);
+                        Gp = G;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float ro = __shfl_xor_sync(0xffffffffu, rm[i], 1);
+                        const float ko = __shfl_xor_sync(0xffffffffu, km[i], 1);
+                        r[i] = part ? ro : rm[i];
+                        r[4 + i] = part ? rm[i] : ro;
+                        kap[i] = part ? ko : km[i];
+                        kap[4 + i] = part ? km[i] : ko;
                     }
                     // rows t0 + 4 part .. + 3 of this thread, then the partner's four
                     float cm[4] = {0.f, 0.f, 0.f, 0.f};
