@@ -1,9 +1,9 @@
 // host.cu -- falcon_fwd_host: the forward on host buffers.  The batch is cut
-// into slices; each slice's inputs go host -> device on a copy-in stream, its
-// forward (every requested variant) runs on the caller's stream, and its
-// outputs go device -> host on a copy-out stream, so that the copies of one
-// slice overlap the compute and the opposite-direction copies of its
-// neighbours.  Events order the three streams; the device buffers are one
+// into slices; the slices' inputs go host -> device on a copy-in stream (all
+// of them enqueued first), each slice's forward (every requested variant)
+// runs on the caller's stream once its inputs have landed, and its outputs go
+// device -> host on a copy-out stream, so that the copies of one slice
+// overlap the compute and the opposite-direction copies of its neighbours.  Events order the three streams; the device buffers are one
 // block: the caller's workspace (falcon_fwd_host_ws), or stream-ordered
 // memory freed on the caller's stream once every copy has been joined back
 // into it (falcon_fwd_host).
@@ -195,16 +195,21 @@ int fwd_host_impl(int n_variants, const falcon_variant *variants, falcon_form fo
     if (rc == FALCON_OK) ok(cudaStreamWaitEvent(s_in, ev_start, 0));
     if (rc == FALCON_OK) ok(cudaStreamWaitEvent(s_out, ev_start, 0));
     if (L > 0) copy(dev + o_l, lambda, (size_t)H * sizeof(float), s_in);
+    // every slice's inputs are enqueued first, so that the copy-in stream
+    // never waits for the host to enqueue a slice's forward
     for (int i = 0; i < ns && rc == FALCON_OK; ++i) {
         const int b0 = (int)((long long)i * B / ns), b1 = (int)((long long)(i + 1) * B / ns), nb = b1 - b0;
-        cudaEvent_t ev_in = evs.ev[2 * i], ev_comp = evs.ev[2 * i + 1];
         if (L > 0) {
             copy(dev + b0 * bq, hq + b0 * bq, nb * bq, s_in);
             copy(dev + o_k + b0 * bq, hk + b0 * bq, nb * bq, s_in);
             copy(dev + o_v + b0 * bv, hv + b0 * bv, nb * bv, s_in);
             copy(dev + o_b + b0 * bb, hb + b0 * bb, nb * bb, s_in);
         }
-        if (rc == FALCON_OK) ok(cudaEventRecord(ev_in, s_in));
+        if (rc == FALCON_OK) ok(cudaEventRecord(evs.ev[2 * i], s_in));
+    }
+    for (int i = 0; i < ns && rc == FALCON_OK; ++i) {
+        const int b0 = (int)((long long)i * B / ns), b1 = (int)((long long)(i + 1) * B / ns), nb = b1 - b0;
+        cudaEvent_t ev_in = evs.ev[2 * i], ev_comp = evs.ev[2 * i + 1];
         if (rc == FALCON_OK) ok(cudaStreamWaitEvent(stream, ev_in, 0));
         for (int j = 0; j < n_variants && rc == FALCON_OK; ++j) {
             const bool st = final_state && final_state[j];
