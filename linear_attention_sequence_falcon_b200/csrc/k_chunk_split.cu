@@ -514,6 +514,17 @@ __global__ void __launch_bounds__(NTH1, 2)
                     *reinterpret_cast<uint4 *>(sm + L_A3 + tc::sw128(t, cs * 2 + 1)) = pack8(&m[8]);
                 }
             }
+        } else {
+            // inner-product family, rows 0-63: no M; Qt = D_g Q in place (G1 has read Q)
+            const float g = v_gt[t];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float q8[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm + oQ + tc::sw128(t, chalf * 4 + cc)), q8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q8[i] *= g;
+                *reinterpret_cast<uint4 *>(sm + oQ + tc::sw128(t, chalf * 4 + cc)) = pack8(q8);
+            }
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
@@ -668,16 +679,6 @@ __global__ void __launch_bounds__(NTH1, 2)
             }
         }
         a4 = sbase + L_MF;
-    } else if (ok && quarter < 2) {  // inner-product family: Qt = D_g Q in place
-        const float g = v_gt[row];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            float q8[8];
-            unpack8(*reinterpret_cast<const uint4 *>(sm + oQ + tc::sw128(row, chalf * 4 + cc)), q8);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) q8[i] *= g;
-            *reinterpret_cast<uint4 *>(sm + oQ + tc::sw128(row, chalf * 4 + cc)) = pack8(q8);
-        }
     }
     tc::fence_proxy_async();
     tc::fence_before_sync();
