@@ -680,9 +680,11 @@ __global__ void __launch_bounds__(NTH1, 2)
         }
         a4 = sbase + L_MF;
     }
-    tc::fence_proxy_async();
-    tc::fence_before_sync();
-    ok = __syncthreads_and(ok);
+    if (reg) {  // (the inner-product family's G4 operands were complete at the last barrier)
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        ok = __syncthreads_and(ok);
+    }
     LTIM(10);
 
     if (ok && !reg) {  // (the regression family issued G4 with G3)
