@@ -209,8 +209,9 @@ __global__ void __launch_bounds__(32 * decode1_warps(DK), DK >= 128 ? 8 : 4) dec
         if (r < total) {
             const int hh = r / dv, row = r - hh * dv;
             const float4 *Srow = reinterpret_cast<const float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
+            // read once per step: evict-first (the row is written back below)
 #pragma unroll
-            for (int i = 0; i < NV4; ++i) dst[i] = Srow[sl + LPR * i];
+            for (int i = 0; i < NV4; ++i) dst[i] = __ldcs(Srow + sl + LPR * i);
         }
     };
     if constexpr (NV4 <= 2) load_row(rsub, cur);
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(32 * decode1_warps(DK), DK >= 128 ? 8 : 4) dec
             o.y = alpha * cur[i].y + ge * xr[i].y;
             o.z = alpha * cur[i].z + ge * xr[i].z;
             o.w = alpha * cur[i].w + ge * xr[i].w;
-            Srow[sl + LPR * i] = o;
+            __stcs(Srow + sl + LPR * i, o);  // (streaming: not read again this step)
         }
         if (sl == 0)
             static_cast<T *>(p.out)[(size_t)(nh0 + hh) * dv + row] = from_f32<T>(alpha * sq + ge * hsc[hh][1]);
