@@ -85,33 +85,43 @@ __device__ __forceinline__ void mma64(const float *A, const float *B, float (&ac
     wt::mma64<LD, TA, TB, SK, NT>(A, B, acc, kb, ke, sk);
 }
 
-// the reverse chain's 16 x 16 block per warp (columns 16 w): acc(r, n) +=
+// The reverse chain's 16 x 16 block per warp (columns 16 w): acc(r, n) +=
 // sum_{k < 64} op(A)(r, k) B[k][n], op(A)(r, k) = TA ? A[k][r] : A[r][k]
-// (row stride lda), B of row stride LD
+// (fp32, row stride lda), B a bf16 64 x 64 tile of the forward's image read
+// as it is (128-byte rows, 128-byte swizzle, B[k][n] in row k): ldmatrix.trans
+// hands each lane B[k0+2t][n] and B[k0+2t+1][n] packed, exactly the TF32
+// fragment in the k-slot order of the A side (slot t <- k0+2t, t+4 <- k0+2t+1),
+// for two k-steps and both n-tiles in one instruction.
 template <bool TA>
-__device__ __forceinline__ void mma16(const float *A, int lda, const float *B, float (&acc)[2][4]) {
+__device__ __forceinline__ void mma16b(const float *A, int lda, uint32_t Bt, float (&acc)[2][4]) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
     const int cb = warp * 16;
-#pragma unroll 4
-    for (int k0 = 0; k0 < 64; k0 += 8) {
-        const int ka = k0 + 2 * t;
-        float a0, a1, a2, a3;
-        if (TA) {
-            a0 = A[ka * lda + g];
-            a1 = A[ka * lda + g + 8];
-            a2 = A[(ka + 1) * lda + g];
-            a3 = A[(ka + 1) * lda + g + 8];
-        } else {
-            const float2 u0 = *reinterpret_cast<const float2 *>(A + g * lda + ka);
-            const float2 u1 = *reinterpret_cast<const float2 *>(A + (g + 8) * lda + ka);
-            a0 = u0.x; a2 = u0.y; a1 = u1.x; a3 = u1.y;
-        }
-        const uint32_t a[4] = {tf(a0), tf(a1), tf(a2), tf(a3)};
+    const int mi = lane >> 3, ri = lane & 7;  // the 8 x 8 matrix this lane addresses, and its row
+#pragma unroll 2
+    for (int k0 = 0; k0 < 64; k0 += 16) {
+        uint32_t bb[4];  // matrix m: k-half m >> 1, n-tile m & 1
+        tc::ldsm_x4_trans(Bt + tc::sw128(k0 + (mi >> 1) * 8 + ri, (cb >> 3) + (mi & 1)), bb);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int n = cb + nt * 8 + g;
-            const uint32_t b[2] = {tf(B[ka * LD + n]), tf(B[(ka + 1) * LD + n])};
-            tc::mma_tf32(acc[nt], a, b);
+        for (int kh = 0; kh < 2; ++kh) {
+            const int ka = k0 + kh * 8 + 2 * t;
+            float a0, a1, a2, a3;
+            if (TA) {
+                a0 = A[ka * lda + g];
+                a1 = A[ka * lda + g + 8];
+                a2 = A[(ka + 1) * lda + g];
+                a3 = A[(ka + 1) * lda + g + 8];
+            } else {
+                const float2 u0 = *reinterpret_cast<const float2 *>(A + g * lda + ka);
+                const float2 u1 = *reinterpret_cast<const float2 *>(A + (g + 8) * lda + ka);
+                a0 = u0.x; a2 = u0.y; a1 = u1.x; a3 = u1.y;
+            }
+            const uint32_t a[4] = {tf(a0), tf(a1), tf(a2), tf(a3)};
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const uint32_t w = bb[kh * 2 + nt];
+                const uint32_t b[2] = {w << 16, w & 0xffff0000u};
+                tc::mma_tf32(acc[nt], a, b);
+            }
         }
     }
 }
@@ -134,10 +144,10 @@ __global__ void __launch_bounds__(NTHR)
     bwd_rchain_kernel(BwdParams p, const uint8_t *img, const float *gc, const float *states,
                       const float *final_state, float *gend, float *bnd, int nch) {
     extern __shared__ __align__(16) float smr[];
-    float *Gh = smr;            // 16 x LD: this block's rows of G^
-    float *Ph = Gh + 16 * LD;   // 64 x LD: -Phi'^T of the chunk (regression)
-    float *Qt = Ph + TF;        // 64 x LD: Qt of the chunk
-    float *dOc = Qt + TF;       // 64 x LDC: dO of the chunk, this block's 16 columns
+    float *Gh = smr;                 // 16 x LD: this block's rows of G^
+    float *dOc = Gh + 16 * LD;       // 64 x LDC: dO of the chunk, this block's 16 columns
+    uint8_t *Pb = reinterpret_cast<uint8_t *>(dOc + 64 * LDC);  // bf16 -Phi'^T of the chunk, as in the image
+    uint8_t *Qb = Pb + TILE_B;                                   // bf16 Qt of the chunk, as in the image
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const bool reg = p.variant == F1;
     const size_t bh = blockIdx.x / RQ;
@@ -171,14 +181,13 @@ __global__ void __launch_bounds__(NTHR)
     };
     auto step = [&](int c, Ops &o) {
         const size_t u = bh * nch + c;
-        __syncthreads();  // the previous products are done with Ph, Qt, dOc; G^ is current
-        // the chunk's operands to shared memory (piece j of a tile: row j / 8,
-        // stored 16-byte piece j % 8 = logical piece (j % 8) ^ (row % 8))
+        __syncthreads();  // the previous products are done with Pb, Qb, dOc; G^ is current
+        // the chunk's image tiles to shared memory as they are (16-byte pieces)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int pc = tid + NTHR * j, r = pc >> 3, lp = (pc & 7) ^ (r & 7);
-            if (reg) st8(Ph + r * LD + 8 * lp, o.p[j]);
-            st8(Qt + r * LD + 8 * lp, o.q[j]);
+            const int pc = tid + NTHR * j;
+            if (reg) *reinterpret_cast<uint4 *>(Pb + pc * 16) = o.p[j];
+            *reinterpret_cast<uint4 *>(Qb + pc * 16) = o.q[j];
         }
         st8(dOc + (tid >> 1) * LDC + 8 * (tid & 1), o.d);
         // G^_{c+1} out, and <G^_{c+1}, S_{c+1}> over these rows
@@ -196,8 +205,8 @@ __global__ void __launch_bounds__(NTHR)
         if (c >= 2) fetch(c - 2, o);
         __syncthreads();
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        if (reg) mma16<false>(Gh, LD, Ph, acc);  // G^ (-Phi'^T)
-        mma16<true>(dOc, LDC, Qt, acc);          // dO^T Qt
+        if (reg) mma16b<false>(Gh, LD, tc::smem_u32(Pb), acc);  // G^ (-Phi'^T)
+        mma16b<true>(dOc, LDC, tc::smem_u32(Qb), acc);          // dO^T Qt
         const int gq = lane >> 2, tq = lane & 3;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
@@ -661,7 +670,7 @@ int launch_bwd_chunk(const BwdParams &p, void *ws, cudaStream_t s) {
     f.states_out = states;
     const int frc = launch_split_chunk(f, s);
     if (frc != 0) return frc;  // 1: the forward's tensor-core path refused the pointers
-    const size_t rbytes = (16 * (size_t)LD + 2 * (size_t)TF + 64 * (size_t)LDC) * sizeof(float);
+    const size_t rbytes = (16 * (size_t)LD + 64 * (size_t)LDC) * sizeof(float) + 2 * (size_t)TILE_B;
     const size_t cbytes = ((size_t)NTILE * TF + NVEC) * sizeof(float);
     static_assert(((size_t)NTILE * TF + NVEC) * sizeof(float) <= 227 * 1024, "shared memory of one block");
     static bool attrs[64] = {false};
