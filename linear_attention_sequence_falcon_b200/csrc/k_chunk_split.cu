@@ -115,6 +115,11 @@ __device__ long long *g_split_tim;
     do {                                                                                   \
         if (dbg_tim_ && dbg_w_ >= 0 && threadIdx.x == 0) dbg_tim_[dbg_w_ * 32 + (k)] = clock64(); \
     } while (0)
+// the same by thread t_ (the product windows: issued by ISSUER1, seen by thread 64)
+#define LTIMX(t_, k)                                                                         \
+    do {                                                                                     \
+        if (dbg_tim_ && dbg_w_ >= 0 && threadIdx.x == (t_)) dbg_tim_[dbg_w_ * 32 + (k)] = clock64(); \
+    } while (0)
 #define LBLK(k)                                                                      \
     do {                                                                             \
         if (dbg_tim_ && threadIdx.x == 0 && blockIdx.x < 4096) {                     \
@@ -134,6 +139,7 @@ __device__ long long *g_split_tim;
 #define LDBG_INIT()
 #define CDBG_INIT()
 #define LTIM(k)
+#define LTIMX(t_, k)
 #define LBLK(k)
 #define CTIM(c, k)
 #endif
@@ -411,6 +417,7 @@ __global__ void __launch_bounds__(NTH1, 2)
         // ---- G1 [X;Q] X^T -> A (lanes 0-63), P (lanes 64-127), while the decays are formed
         if (tid == ISSUER1) {
             tc::fence_after_sync();
+            LTIMX(ISSUER1, 24);
             issue_gemm(tbase + C_G1, sbase + oX, sbase + oX, 64, false);
             tc::mma_commit(bar);
         }
@@ -452,6 +459,7 @@ __global__ void __launch_bounds__(NTH1, 2)
         }
         LTIM(16);
         ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        LTIMX(64, 28);
         phase ^= 1;
         ok = __syncthreads_and(ok);
         LTIM(4);
@@ -614,10 +622,12 @@ __global__ void __launch_bounds__(NTH1, 2)
         // ---- G2: [Y^T;(D_a X)^T] T^T -> U0^T (lanes 0-63), W^T (lanes 64-127)
         if (tid == ISSUER1) {
             tc::fence_after_sync();
+            LTIMX(ISSUER1, 25);
             issue_gemm(tbase + C_G2, sbase + L_XT, sbase + oV, 64, false);
             tc::mma_commit(bar);
         }
         ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        LTIMX(64, 29);
         phase ^= 1;
         ok = __syncthreads_and(ok);
         if (ok) {
@@ -641,11 +651,13 @@ __global__ void __launch_bounds__(NTH1, 2)
             //      G4: [U0^T;W^T] [P o Dm;(D_w X)^T]^T -> [O0^T | B] (lanes 0-63), at once
             if (tid == ISSUER1) {
                 tc::fence_after_sync();
+                LTIMX(ISSUER1, 26);
                 issue_gemm(tbase + C_G3, sbase + L_A3, sbase + L_MF + TILE, 64, false);
                 issue_gemm(tbase + C_G4, sbase + L_MF, sbase + L_A3, 128, false);
                 tc::mma_commit(bar);
             }
             ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+            LTIMX(64, 30);
             phase ^= 1;
             ok = __syncthreads_and(ok);
             LTIM(9);
@@ -691,10 +703,12 @@ __global__ void __launch_bounds__(NTH1, 2)
         // ---- G4: [Y^T; .] [P o Dm; (D_w X)^T]^T -> [O0^T | B] (lanes 0-63)
         if (tid == ISSUER1) {
             tc::fence_after_sync();
+            LTIMX(ISSUER1, 27);
             issue_gemm(tbase + C_G4, a4, sbase + L_A3, 128, false);
             tc::mma_commit(bar);
         }
         ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        LTIMX(64, 31);
         phase ^= 1;
         ok = __syncthreads_and(ok);
         LTIM(11);
