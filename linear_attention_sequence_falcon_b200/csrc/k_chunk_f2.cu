@@ -24,11 +24,17 @@
 // The output form needs G_C > -80 in every channel; a chunk below that
 // solves for eta_s E_s with one exponential per term instead.
 //
-// One block per (b, h) walks the chunks; S stays in fp32 registers (thread:
-// row j, 64 columns) with its bf16 copy in shared memory as the operand of
-// S_0 [X;Q]^T.  The per-channel systems are solved by forward substitution
-// in blocks of 8 tokens, two threads (lanes of one warp) per channel: each
-// forms half of a block's sums over the earlier tokens, and both walk it.
+// Rows of S never mix, so a head's channels can be shared out: one block per
+// (b, h) walks the chunks for all 128 channels, or, when twice the heads fit
+// on the SMs, two blocks per head take 64 channels each (the sample
+// normalisation and the key products are then done by both).  S stays in
+// fp32 registers (thread: row j, a segment of its columns) with its bf16
+// copy in shared memory as the operand of S_0 [X;Q]^T; with 64 channels the
+// copy fills both halves of the 128-row operand, so every tensor-memory lane
+// quarter holds channel rows.  The per-channel systems are solved by forward
+// substitution in blocks of 8 tokens, two threads (lanes of one warp) per
+// channel with 128 channels, four with 64: each forms its share of a block's
+// sums over the earlier tokens, and all walk it.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -92,10 +98,29 @@ constexpr float kMinLogDecay = -80.f;
 // fp32 G table: row t, column j ^ (t mod 32) (conflict-free along either index)
 __device__ __forceinline__ int gidx(int t, int j) { return t * DD + (j ^ (t & 31)); }
 
-__device__ __forceinline__ void store_state_image(uint8_t *sm, int j, int half, const float *S) {
+// bf16 copy of this thread's state columns seg * SC .. + SC - 1 of row j
+// (SC = 64 with 128 channels, 32 with 64 channels, whose rows go to both
+// halves of the operand)
+template <int NJ>
+__device__ __forceinline__ void store_state_image(uint8_t *sm, int j, int seg, const float *S) {
+    constexpr int SC = 128 / (256 / NJ);
+    const int half = (seg * SC) >> 6, ch0 = ((seg * SC) & 63) >> 3;
 #pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8)
-        *reinterpret_cast<uint4 *>(sm + F_S + half * 2 * TILE + tc::sw128(j, c8)) = pack8(&S[c8 * 8]);
+    for (int c8 = 0; c8 < SC / 8; ++c8) {
+        const uint4 u = pack8(&S[c8 * 8]);
+        *reinterpret_cast<uint4 *>(sm + F_S + half * 2 * TILE + tc::sw128(j, ch0 + c8)) = u;
+        if (NJ == 64) *reinterpret_cast<uint4 *>(sm + F_S + half * 2 * TILE + tc::sw128(j + 64, ch0 + c8)) = u;
+    }
+}
+
+// a[part * STRIDE] for a compile-time array position a and a runtime part < TPC
+template <int TPC, int STRIDE>
+__device__ __forceinline__ float pick(const float *a, int part) {
+    if constexpr (TPC == 2) {
+        return part ? a[STRIDE] : a[0];
+    } else {
+        return (part & 2) ? ((part & 1) ? a[3 * STRIDE] : a[2 * STRIDE]) : ((part & 1) ? a[STRIDE] : a[0]);
+    }
 }
 
 // bf16 element (t, s) of the 64-row P o mask tile
@@ -106,7 +131,12 @@ __device__ __forceinline__ float pm_get(const uint8_t *sm, int t, int s) {
 
 }  // namespace
 
+template <int NJ>
 __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __grid_constant__ PcMaps maps) {
+    constexpr int NSPLIT = DD / NJ;  // blocks per head
+    constexpr int NSEG = 256 / NJ;   // threads per channel in the solve and the epilogue
+    constexpr int SC = DD / NSEG;    // state columns per thread
+    constexpr bool DUP = NJ == 64;   // channel rows in both halves of the 128-row operands
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = tc::smem_u32(smem_raw);
     uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -123,19 +153,29 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, chalf = warp >> 2, row = quarter * 32 + lane;
-    const int bh = blockIdx.x, L = p.L, nch = (L + CH - 1) / CH;
+    // this thread's tensor-memory lane holds channel jl (of the block's NJ);
+    // its segment of that channel's tokens and state columns is seg
+    const int jl = row & (NJ - 1), seg = DUP ? 2 * (quarter >> 1) + chalf : chalf;
+    const int bh = blockIdx.x / NSPLIT, J0 = (blockIdx.x % NSPLIT) * NJ;
+    const int L = p.L, nch = (L + CH - 1) / CH;
     const float lam = p.lambda[bh % p.H];
 
-    // keys (rows c0-1 .. under the prefix pair) and q as [X;Q] per K half, v, beta
+    // keys (rows c0-1 .. under the prefix pair) and q as [X;Q] per K half, then
+    // the block's columns of v and beta (both halves, or the one of its channels)
     auto load_chunk = [&](int c) {
         const int c0 = c * CH, krow = p.pairing == 0 ? c0 - 1 : c0;
-        tc::mbar_arrive_expect_tx(tbar, 8 * TILE);
+        tc::mbar_arrive_expect_tx(tbar, (4 + 2 * (NJ / 64)) * TILE);
         tc::tma_load_3d(sbase + F_IN, &maps.k, 0, krow, bh, tbar);
         tc::tma_load_3d(sbase + F_IN + TILE, &maps.q, 0, c0, bh, tbar);
         tc::tma_load_3d(sbase + F_IN + 2 * TILE, &maps.k, 64, krow, bh, tbar);
         tc::tma_load_3d(sbase + F_IN + 3 * TILE, &maps.q, 64, c0, bh, tbar);
-        load_pair(sbase + F_V, &maps.v, c0, bh, tbar);
-        load_pair(sbase + F_B, &maps.beta, c0, bh, tbar);
+        if constexpr (NJ == DD) {
+            load_pair(sbase + F_V, &maps.v, c0, bh, tbar);
+            load_pair(sbase + F_B, &maps.beta, c0, bh, tbar);
+        } else {
+            tc::tma_load_3d(sbase + F_V, &maps.v, J0, c0, bh, tbar);
+            tc::tma_load_3d(sbase + F_B, &maps.beta, J0, c0, bh, tbar);
+        }
     };
     int issued = 0;  // chunk loads issued (thread 0)
     if (tid == 0) {
@@ -152,12 +192,12 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
         tc::tmem_alloc(tmem_slot, 512);
         tc::tmem_relinquish();
     }
-    // S in fp32 registers: thread = (row j, column half chalf)
-    float S[64];
+    // S in fp32 registers: thread = (row J0 + jl, columns seg * SC ..)
+    float S[SC];
 #pragma unroll
-    for (int e = 0; e < 64; ++e)
-        S[e] = p.init_state ? p.init_state[((size_t)bh * DD + row) * DD + chalf * 64 + e] : 0.f;
-    store_state_image(sm, row, chalf, S);
+    for (int e = 0; e < SC; ++e)
+        S[e] = p.init_state ? p.init_state[((size_t)bh * DD + J0 + jl) * DD + seg * SC + e] : 0.f;
+    store_state_image<NJ>(sm, jl, seg, S);
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
@@ -186,31 +226,38 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
             issue_gemm(tbase + C_S, sbase + F_S, 2 * TILE, sbase + F_IN, 2 * TILE, 2, 128);
             tc::mma_commit(bar);
         }
-        // ---- log decays: thread (half h, channel jj), 32 running sums in registers; X^T
+        // ---- log decays: thread (token group h, channel jj), TG running sums in registers; X^T
         {
-            const int h = tid >> 7, jj = tid & (DD - 1);
-            float Gl[32];
+            constexpr int NG = 256 / NJ, TG = CH / NG;
+            const int h = tid / NJ, jj = tid % NJ;
+            float Gl[TG];
             float acc = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int t = h * 32 + i;
+            for (int i = 0; i < TG; ++i) {
+                const int t = h * TG + i;
                 const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
                 acc += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
                 Gl[i] = acc;
             }
-            hsum[h * DD + jj] = acc;
+            hsum[h * NJ + jj] = acc;
             for (int g = warp; g < 32; g += NTH / 32) {
                 const int half = g >> 4, rb = (g >> 1) & 7, cb0 = (g & 1) * 4;
                 transpose4(sbase + F_IN + half * 2 * TILE, rb, cb0, sbase + F_XT, half * 64);
             }
             __syncthreads();
-            const float base = h ? hsum[jj] : 0.f;
+            float base = 0.f, tot = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) Gt[gidx(h * 32 + i, jj)] = base + Gl[i];
-            if (h == 0) gcv[jj] = hsum[jj] + hsum[DD + jj];
+            for (int h2 = 0; h2 < NG; ++h2) {
+                const float hs = hsum[h2 * NJ + jj];
+                if (h2 < h) base += hs;
+                tot += hs;
+            }
+#pragma unroll
+            for (int i = 0; i < TG; ++i) Gt[gidx(h * TG + i, jj)] = base + Gl[i];
+            if (h == 0) gcv[jj] = tot;
         }
         __syncthreads();
-        const bool unsafe = __syncthreads_or(tid < DD && !(gcv[tid] > kMinLogDecay)) != 0;
+        const bool unsafe = __syncthreads_or(tid < NJ && !(gcv[tid] > kMinLogDecay)) != 0;
         F2T(2);
         ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
         phase ^= 1;
@@ -247,14 +294,20 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
         __syncthreads();
         F2T(4);
         tc::fence_after_sync();
-        // ---- per-channel systems.  Two threads per channel, both lanes of one
-        //      warp: warp w takes channels 32 (w & 3) + 16 (w >> 2) .. +15 (inside
-        //      its tensor-memory lanes), lane l channel ... + l / 2.  Each thread
-        //      of a pair forms four of the eight sums over the rows before a
-        //      block of 8 tokens; the pair swaps them and both walk the block.
+        // ---- per-channel systems.  TPC threads per channel, lanes of one warp.
+        //      128 channels: warp w takes channels 32 (w & 3) + 16 (w >> 2) .. +15
+        //      (inside its tensor-memory lanes), lane l channel ... + l / 2.  64
+        //      channels (rows in both lane halves): the four warps of lane
+        //      quarters q and q ^ 2 take 8 channels each of 32 (q & 1) .. +31, lane
+        //      l channel ... + l / 4.  Each thread of a channel forms 8 / TPC of
+        //      the eight sums over the rows before a block of 8 tokens; the
+        //      threads swap them and all walk the block.
         if (!unsafe) {
-            const int part = lane & 1, src = 16 * (warp >> 2) + (lane >> 1);
-            const int jj = 32 * quarter + src;
+            constexpr int TPC = NSEG, PT = 8 / TPC;
+            const int part = lane & (TPC - 1);
+            const int slot = DUP ? (warp >> 2) + 2 * (quarter >> 1) : (warp >> 2);
+            const int src = (32 / TPC) * slot + lane / TPC;  // the channel's lane inside this quarter
+            const int jj = 32 * (DUP ? (quarter & 1) : quarter) + src;
             const float gc = gcv[jj];
             float Z[64];
 #pragma unroll
@@ -268,45 +321,65 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
                 for (int i = 0; i < 16; ++i) xs[i] = __shfl_sync(0xffffffffu, xs[i], src);  // channel jj's row
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb) {
-                    const int t0 = tb * 16 + hb * 8, tp = t0 + 4 * part;  // this thread's four tokens
-                    float r[8], kap[8], cr[8], rm[4], km[4];
+                    const int t0 = tb * 16 + hb * 8, tp = t0 + PT * part;  // this thread's PT tokens
+                    float r[8], kap[8], cr[8], rm[PT], km[PT];
                     float Gp = tp > 0 ? Gt[gidx(tp - 1, jj)] : 0.f;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < PT; ++i) {
                         const int t = tp + i;
                         const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
                         const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
                         const float G = Gt[gidx(t, jj)];
-                        const float x = part ? xs[hb * 8 + 4 + i] : xs[hb * 8 + i];
+                        const float x = pick<TPC, PT>(&xs[hb * 8 + i], part);
                         rm[i] = __expf(gc - G) * eta * (pair_get(sm, F_V, t, jj) - __expf(Gp) * x);
                         km[i] = __fdividef(eta, alpha);
                         Gp = G;
                     }
+                    if constexpr (TPC == 2) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float ro = __shfl_xor_sync(0xffffffffu, rm[i], 1);
-                        const float ko = __shfl_xor_sync(0xffffffffu, km[i], 1);
-                        r[i] = part ? ro : rm[i];
-                        r[4 + i] = part ? rm[i] : ro;
-                        kap[i] = part ? ko : km[i];
-                        kap[4 + i] = part ? km[i] : ko;
+                        for (int i = 0; i < 4; ++i) {
+                            const float ro = __shfl_xor_sync(0xffffffffu, rm[i], 1);
+                            const float ko = __shfl_xor_sync(0xffffffffu, km[i], 1);
+                            r[i] = part ? ro : rm[i];
+                            r[4 + i] = part ? rm[i] : ro;
+                            kap[i] = part ? ko : km[i];
+                            kap[4 + i] = part ? km[i] : ko;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q2 = 0; q2 < TPC; ++q2)
+#pragma unroll
+                            for (int i = 0; i < PT; ++i) {
+                                r[q2 * PT + i] = __shfl_sync(0xffffffffu, rm[i], (lane & ~(TPC - 1)) | q2);
+                                kap[q2 * PT + i] = __shfl_sync(0xffffffffu, km[i], (lane & ~(TPC - 1)) | q2);
+                            }
                     }
-                    // rows t0 + 4 part .. + 3 of this thread, then the partner's four
-                    float cm[4] = {0.f, 0.f, 0.f, 0.f};
-                    const float *arow = At + (t0 + 4 * part) * LDA;
+                    // rows t0 + PT part .. + PT - 1 of this thread, then the others'
+                    float cm[PT];
+#pragma unroll
+                    for (int i = 0; i < PT; ++i) cm[i] = 0.f;
+                    const float *arow = At + (t0 + PT * part) * LDA;
 #pragma unroll
                     for (int s = 0; s < t0; s += 4) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
+                        for (int i = 0; i < PT; ++i) {
                             const float4 a = *reinterpret_cast<const float4 *>(arow + i * LDA + s);
                             cm[i] = fmaf(a.x, Z[s], fmaf(a.y, Z[s + 1], fmaf(a.z, Z[s + 2], fmaf(a.w, Z[s + 3], cm[i]))));
                         }
                     }
+                    if constexpr (TPC == 2) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float other = __shfl_xor_sync(0xffffffffu, cm[i], 1);
-                        cr[i] = part ? other : cm[i];
-                        cr[4 + i] = part ? cm[i] : other;
+                        for (int i = 0; i < 4; ++i) {
+                            const float other = __shfl_xor_sync(0xffffffffu, cm[i], 1);
+                            cr[i] = part ? other : cm[i];
+                            cr[4 + i] = part ? cm[i] : other;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q2 = 0; q2 < TPC; ++q2)
+#pragma unroll
+                            for (int i = 0; i < PT; ++i)
+                                cr[q2 * PT + i] = __shfl_sync(0xffffffffu, cm[i], (lane & ~(TPC - 1)) | q2);
                     }
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -317,14 +390,26 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
                     }
                 }
             }
-            // Z^T row jj: each thread of the pair half of it
+            // Z^T row jj (and its copy in lanes 64-127 with 64 channels): each
+            // thread of the channel 64 / TPC of its columns
+            if constexpr (TPC == 2) {
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const uint4 lo = pack8(&Z[c4 * 8]), hi = pack8(&Z[32 + c4 * 8]);
-                *reinterpret_cast<uint4 *>(sm + F_ZT + tc::sw128(jj, part * 4 + c4)) = part ? hi : lo;
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint4 lo = pack8(&Z[c4 * 8]), hi = pack8(&Z[32 + c4 * 8]);
+                    *reinterpret_cast<uint4 *>(sm + F_ZT + tc::sw128(jj, part * 4 + c4)) = part ? hi : lo;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const uint4 u0 = pack8(&Z[8 * e]), u1 = pack8(&Z[16 + 8 * e]), u2 = pack8(&Z[32 + 8 * e]),
+                                u3 = pack8(&Z[48 + 8 * e]);
+                    const uint4 u = (part & 2) ? ((part & 1) ? u3 : u2) : ((part & 1) ? u1 : u0);
+                    *reinterpret_cast<uint4 *>(sm + F_ZT + tc::sw128(jj, part * 2 + e)) = u;
+                    *reinterpret_cast<uint4 *>(sm + F_ZT + tc::sw128(jj + 64, part * 2 + e)) = u;
+                }
             }
-        } else if (tid < DD) {
-            // (warps 0-3, thread = channel jj = tensor-memory lane)
+        } else if (tid < NJ) {
+            // (thread = channel jj = tensor-memory lane)
             const int jj = tid;
             const float gc = gcv[jj];
             float Z[64];
@@ -361,16 +446,19 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
                 const float G = Gt[gidx(t, jj)];
                 float o = __expf(G) * xs[t];
                 for (int s = 0; s <= t; ++s) o += __expf(G - Gt[gidx(s, jj)]) * pm_get(sm, t, s) * F[s];
-                static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + jj] = __float2bfloat16_rn(o);
+                static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + J0 + jj] = __float2bfloat16_rn(o);
             }
 #pragma unroll 1
             for (int s = 0; s < CH; ++s) F[s] *= __expf(gc - Gt[gidx(s, jj)]);
 #pragma unroll
             for (int s = 0; s < 64; ++s) Z[s] = F[s];
-            // Z^T row jj
+            // Z^T row jj (and its copy)
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8)
-                *reinterpret_cast<uint4 *>(sm + F_ZT + tc::sw128(jj, c8)) = pack8(&Z[c8 * 8]);
+            for (int c8 = 0; c8 < 8; ++c8) {
+                const uint4 u = pack8(&Z[c8 * 8]);
+                *reinterpret_cast<uint4 *>(sm + F_ZT + tc::sw128(jj, c8)) = u;
+                if (DUP) *reinterpret_cast<uint4 *>(sm + F_ZT + tc::sw128(jj + 64, c8)) = u;
+            }
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
@@ -393,13 +481,14 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
         if (!ok) break;
         F2T(6);
         tc::fence_after_sync();
-        const float gcj = gcv[row];
+        const float gcj = gcv[jl];
         if (!unsafe) {
-            // o_t[j] for t in 32 chalf .. 32 chalf + 31
+            // o_t[J0 + jl] for the segment's tokens t = seg * TPS ..
+            constexpr int TPS = CH / NSEG;
             const float ig = __expf(-gcj);
 #pragma unroll
-            for (int k2 = 0; k2 < 2; ++k2) {
-                const int t0 = chalf * 32 + k2 * 16;
+            for (int k2 = 0; k2 < TPS / 16; ++k2) {
+                const int t0 = seg * TPS + k2 * 16;
                 float iv[16], av[16];
                 tc::tmem_ld16(tl + C_S + 64 + t0, iv);
                 tc::tmem_ld16(tl + C_I + t0, av);
@@ -407,25 +496,25 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int t = t0 + i;
-                    const float o = __expf(Gt[gidx(t, row)]) * fmaf(ig, av[i], iv[i]);
+                    const float o = __expf(Gt[gidx(t, jl)]) * fmaf(ig, av[i], iv[i]);
                     if (t < nt)
-                        static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + row] =
+                        static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + J0 + jl] =
                             __float2bfloat16_rn(o);
                 }
             }
         }
-        // S_end = diag(e^{G_C}) S_0 + Z^T X
+        // S_end = diag(e^{G_C}) S_0 + Z^T X, this thread's columns
         {
             const float g = __expf(gcj);
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
+            for (int k4 = 0; k4 < SC / 16; ++k4) {
                 float dv[16];
-                tc::tmem_ld16(tl + C_DS + chalf * 64 + k4 * 16, dv);
+                tc::tmem_ld16(tl + C_DS + seg * SC + k4 * 16, dv);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) S[k4 * 16 + i] = fmaf(g, S[k4 * 16 + i], dv[i]);
             }
-            store_state_image(sm, row, chalf, S);
+            store_state_image<NJ>(sm, jl, seg, S);
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
@@ -435,7 +524,7 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
     F2T_END();
     if (ok && p.final_state) {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) p.final_state[((size_t)bh * DD + row) * DD + chalf * 64 + e] = S[e];
+        for (int e = 0; e < SC; ++e) p.final_state[((size_t)bh * DD + J0 + jl) * DD + seg * SC + e] = S[e];
     }
     if (!ok && tid == 0) {
         atomicAdd(&g_f2_wait_timeouts, 1u);
@@ -459,13 +548,26 @@ int launch_f2_chunk(const FwdParams &p, cudaStream_t s) {
         !make_map(&maps.beta, p.beta, BH, p.L))
         return 1;
     static bool attr_set[64] = {false};
+    static int sm_count[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        cudaFuncSetAttribute(f2_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)F_SMEM);
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    int sms = 148;
+    if (dev >= 0 && dev < 64 && attr_set[dev]) {
+        sms = sm_count[dev];
+    } else {
+        cudaFuncSetAttribute(f2_chunk_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)F_SMEM);
+        cudaFuncSetAttribute(f2_chunk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)F_SMEM);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+        if (dev >= 0 && dev < 64) {
+            sm_count[dev] = sms;
+            attr_set[dev] = true;
+        }
     }
-    f2_chunk_kernel<<<(unsigned)BH, NTH, F_SMEM, s>>>(p, maps);
+    // one block per SM: two blocks per head while they all fit at once
+    if (2 * BH <= sms)
+        f2_chunk_kernel<64><<<(unsigned)(2 * BH), NTH, F_SMEM, s>>>(p, maps);
+    else
+        f2_chunk_kernel<DD><<<(unsigned)BH, NTH, F_SMEM, s>>>(p, maps);
     return cudaGetLastError() == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
 }
 

@@ -481,9 +481,9 @@ def test_falcon2a_d128_decay_floor(F):
 
 @pytest.mark.parametrize("L", [64, 200, 513])
 def test_falcon2_d128_tensor_core_path(F, L):
-    """bf16 Falcon-2, d_k = d_v = 128, chunk 64: one block per head, the
-    per-channel systems by forward substitution, the products on tcgen05;
-    one chunk, a ragged tail, many chunks."""
+    """bf16 Falcon-2, d_k = d_v = 128, chunk 64: two blocks of 64 channels
+    per head, the per-channel systems by forward substitution, the products
+    on tcgen05; one chunk, a ragged tail, many chunks."""
     d = gen.draw("F2", 2, 3, L, 128, 128, seed=80 + L, dtype="bf16", lam=0.02)
     check(F, d, "F2", "chunk", chunk=64)
 
@@ -507,6 +507,16 @@ def test_falcon2_d128_decay_floor(F):
     for eta E with one exponential per term."""
     d = gen.draw("F2", 1, 2, 130, 128, 128, seed=86, dtype="bf16", lam=0.9, key_scale=0.03)
     check(F, d, "F2", "chunk", chunk=64, phi="identity")
+
+
+@pytest.mark.parametrize("lam,key_scale,phi", [(0.02, 1.0, "l2"), (0.9, 0.03, "identity")])
+def test_falcon2_d128_one_block_per_head(F, lam, key_scale, phi):
+    """B*H = 80 heads: twice that many blocks would not fit on the SMs at
+    once, so each head runs as one block over all 128 channels (two threads
+    per channel in the solve) instead of two blocks of 64 channels; with and
+    without the decay floor."""
+    d = gen.draw("F2", 5, 16, 130, 128, 128, seed=87, dtype="bf16", lam=lam, key_scale=key_scale)
+    check(F, d, "F2", "chunk", chunk=64, phi=phi)
 
 
 # --------------------------------------------------------------- the windowed (Falcon-3/3A, d = 64) tensor-core path
