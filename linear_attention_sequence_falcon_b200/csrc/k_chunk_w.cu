@@ -439,27 +439,26 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
 #pragma unroll
                     for (int hb = 0; hb < 2; ++hb) {
                         const int t0 = tb * 16 + hb * NB;
-                        float cr[NB][BW];
+                        // rows r' < t0 are final (in shared memory): the sum over them
+                        // of A[t+m][r'] Zacc[r'] depends on t+m only, one sum per row
+                        float crr[RB];
 #pragma unroll
-                        for (int i = 0; i < NB; ++i)
-#pragma unroll
-                            for (int m = 0; m < BW; ++m) cr[i][m] = 0.f;
+                        for (int rr = 0; rr < RB; ++rr) crr[rr] = 0.f;
                         if (reg) {
-                            // rows r' < t0: final, in shared memory
                             for (int q = 0; q < (t0 >> 2); ++q) {
                                 const float4 z4 = *reinterpret_cast<const float4 *>(za + q * 4);
 #pragma unroll
                                 for (int rr = 0; rr < RB; ++rr) {
                                     const float4 a4 = *reinterpret_cast<const float4 *>(At + (t0 + rr) * LDA + q * 4);
-                                    const float d = fmaf(a4.x, z4.x, fmaf(a4.y, z4.y, fmaf(a4.z, z4.z, a4.w * z4.w)));
-#pragma unroll
-                                    for (int i = 0; i < NB; ++i)
-#pragma unroll
-                                        for (int m = 0; m < BW; ++m)
-                                            if (i + m == rr) cr[i][m] += d;
+                                    crr[rr] = fmaf(a4.x, z4.x, fmaf(a4.y, z4.y, fmaf(a4.z, z4.z, fmaf(a4.w, z4.w, crr[rr]))));
                                 }
                             }
                         }
+                        float cr[NB][BW];
+#pragma unroll
+                        for (int i = 0; i < NB; ++i)
+#pragma unroll
+                            for (int m = 0; m < BW; ++m) cr[i][m] = crr[i + m];
 #pragma unroll
                         for (int i = 0; i < NB; ++i) {
                             const int t = t0 + i;
