@@ -486,7 +486,11 @@ def measure_decode(F, gen, stream, flush, hbm, args, profile=False, variant=None
     if window > 1:  # the window carry is read and written too
         ab += N * H * (window - 1) * (dk + dv) * 4 * 2
     gbs = ab / (t / 1e3) / 1e9
-    kernel = "decode1_kernel" if window == 1 else "decode_kernel"
+    # the kernel the library picks for this shape
+    if window == 1:
+        kernel = "decode1r_kernel" if dk == 64 and dv <= 64 else "decode1_kernel"
+    else:
+        kernel = "decodew_kernel" if window <= 4 else "decode_kernel"
     return {"workload": "%s-decode-bf16-N%dxH%d-state%dx%d-fp32%s" % (
                 variant.replace("F", "falcon"), N, H, dv, dk, "-window%d" % window if window > 1 else ""),
             "kernel": kernel, "us_per_step": t * 1e3, "tokens_per_s": N / (t / 1e3), "steps": steps,

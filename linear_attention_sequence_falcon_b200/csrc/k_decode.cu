@@ -487,13 +487,19 @@ __global__ void __launch_bounds__(128, 8) decode1r_kernel(DecodeParams p) {
 // before the block stages its window.  Per row: W + 1 dot products (S_j.x_m,
 // S_j.q) reduced together, e_m = y_m - S_j.x_m (inner product: y_m), and
 // S_j <- alpha S_j + eta sum_m e_m x_m^T, o_j = alpha S_j.q + eta sum_m e_m (x_m.q).
+// At d = 128 one pair per block of four warps, seven blocks per SM (so the
+// blocks spread evenly and 32 warps per SM keep rows in flight); below, four
+// pairs per block of eight warps, two blocks per SM.
+__host__ __device__ constexpr int decodew_hpb(int dk) { return dk >= 128 ? 1 : 4; }
+__host__ __device__ constexpr int decodew_warps(int dk) { return dk >= 128 ? 4 : 8; }
+
 template <typename T, int DK, int W>
-__global__ void __launch_bounds__(256, 2) decodew_kernel(DecodeParams p) {
-    constexpr int HPB = 4;
+__global__ void __launch_bounds__(32 * decodew_warps(DK), DK >= 128 ? 7 : 2) decodew_kernel(DecodeParams p) {
+    constexpr int HPB = decodew_hpb(DK);
     constexpr int LPR = DK >= 32 ? 8 : DK / 4;
     constexpr int NV4 = DK / (4 * LPR);  // float4 per lane per row
     constexpr int RPW = 32 / LPR;        // rows per warp per pass
-    constexpr int NW = 8;
+    constexpr int NW = decodew_warps(DK);
     __shared__ __align__(16) float xs[HPB][W][DK];  // samples, oldest first; slot W-1 the current one
     __shared__ __align__(16) float qs[HPB][DK];
     __shared__ float ks[HPB][DK];
@@ -516,7 +522,7 @@ __global__ void __launch_bounds__(256, 2) decodew_kernel(DecodeParams p) {
             const int hh = r / dv, row = r - hh * dv;
             const float4 *Srow = reinterpret_cast<const float4 *>(p.state + ((size_t)(nh0 + hh) * dv + row) * DK);
 #pragma unroll
-            for (int i = 0; i < NV4; ++i) dst[i] = Srow[sl + LPR * i];
+            for (int i = 0; i < NV4; ++i) dst[i] = __ldcs(Srow + sl + LPR * i);  // read once: evict first
         }
     };
     load_row(rsub, cur);
@@ -624,7 +630,7 @@ __global__ void __launch_bounds__(256, 2) decodew_kernel(DecodeParams p) {
                 const float4 x4 = *reinterpret_cast<const float4 *>(&xs[hh][m][4 * (sl + LPR * i)]);
                 o.x += ge[m] * x4.x; o.y += ge[m] * x4.y; o.z += ge[m] * x4.z; o.w += ge[m] * x4.w;
             }
-            Srow[sl + LPR * i] = o;
+            __stcs(Srow + sl + LPR * i, o);  // streaming store
         }
         if (sl == 0) static_cast<T *>(p.out)[(size_t)(nh0 + hh) * dv + row] = from_f32<T>(alpha * sq + gq);
 #pragma unroll
@@ -679,7 +685,8 @@ __global__ void __launch_bounds__(128) carry_kernel(CarryParams p) {
 
 template <typename T, int DK, int W>
 static void launch_decodew(const DecodeParams &p, cudaStream_t s) {
-    decodew_kernel<T, DK, W><<<(p.N * p.H + 3) / 4, 256, 0, s>>>(p);
+    constexpr int hpb = decodew_hpb(DK);
+    decodew_kernel<T, DK, W><<<(p.N * p.H + hpb - 1) / hpb, 32 * decodew_warps(DK), 0, s>>>(p);
 }
 
 template <typename T, int DK>
