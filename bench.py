@@ -340,7 +340,9 @@ def run_ours(args):
         return
     if args.profile_decode:
         args.steps = max(args.steps, 1)
-        measure_decode(F, gen, stream, flush, peaks()[0], args, profile=True)
+        wdw = args.decode_window
+        measure_decode(F, gen, stream, flush, peaks()[0], args, profile=True,
+                       variant="F3" if wdw > 1 else None, window=wdw)
         return
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
@@ -757,6 +759,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="leave out the chunk sweep and backward keys")
     ap.add_argument("--profile-decode", action="store_true",
                     help="run only warmup+steps decode steps (no flush or JSON), for ncu")
+    ap.add_argument("--decode-window", type=int, default=1,
+                    help="with --profile-decode: the Falcon-3 window decode of this window (2-8) instead")
     ap.add_argument("--workloads", action="store_true",
                     help="time every workload and form of the workloads table, one JSON line each")
     ap.add_argument("--only", type=int, default=0, help="with --workloads or --backward: just this workload number")
