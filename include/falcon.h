@@ -187,7 +187,7 @@ int falcon_fwd_ws(falcon_variant variant, falcon_form form, falcon_dtype dtype,
  *   final_state  NULL, or an array of n_variants host pointers (entries may
  *                be NULL), final_state[i] [B,H,d_v,d_k] fp32
  *   slices       number of slices, clamped to [1, min(B, 64)]; 0 lets the
- *                library choose (about one per 4 MiB of input, at most 8)
+ *                library choose (about one per 16 MiB of input, at most 8)
  *   every other argument as in falcon_fwd_ex.
  * The call returns once the work is enqueued.  The host buffers must stay
  * valid, and the inputs unchanged, until `stream` has passed the call's work;
