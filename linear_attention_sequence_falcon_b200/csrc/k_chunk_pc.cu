@@ -53,8 +53,8 @@ constexpr uint32_t D_WT = D_X;
 constexpr uint32_t D_V = 2 * TILE;     // values -> W[s][j] = e^{G_C-G_s} eta y in place (tile pair)
 constexpr uint32_t D_B = 4 * TILE;     // per-channel beta -> E[s][j] = e^{G_s} in place (tile pair)
 constexpr uint32_t D_XT = 6 * TILE;    // X^T: 128 rows i x 64 s
-constexpr uint32_t D_VEC = 8 * TILE;   // |x_s|^2 [64], 1/(eps+|x_s|^2) [64], half-chunk log-decay sums [2][128]
-constexpr uint32_t D_BAR = D_VEC + (64 + 64 + 2 * DD) * 4;
+constexpr uint32_t D_VEC = 8 * TILE;   // |x_s|^2 [64], 1/(eps+|x_s|^2) [64], quarter-chunk log-decay sums [4][128]
+constexpr uint32_t D_BAR = D_VEC + (64 + 64 + 4 * DD) * 4;
 constexpr uint32_t D_SMEM = D_BAR + 64 + 1024;
 constexpr uint32_t WTIMG = 2 * TILE;   // W^T image handed to pc_out_kernel
 constexpr uint32_t EIMG = 2 * TILE;    // e^{G_t} tile pair handed to pc_out_kernel
@@ -78,9 +78,10 @@ __host__ __device__ inline PcWs pc_ws(void *base, size_t units) {
 }  // namespace
 
 // One block per unit (b*H + h, chunk); blockIdx.x = bh * nchunks + c.
-// The decays are taken by one thread per (channel j, half of the chunk):
-// 32 log-decays summed in registers, the two halves joined through shared
-// memory.  Outputs: dS (bf16 image, the layout of the state operand), g =
+// The decays are taken by one thread per (pair of adjacent channels, quarter
+// of the chunk), so that every shared-memory access moves a bf16 pair: 16
+// log-decays per channel summed in registers, the quarters joined through
+// shared memory.  Outputs: dS (bf16 image, the layout of the state operand), g =
 // e^{G_C}, and for pc_out_kernel W^T (its intra-chunk operand) and e^{G_t}.
 __global__ void __launch_bounds__(NTH, 3) pc_delta_kernel(FwdParams p, const __grid_constant__ PcMaps maps, PcWs ws) {
     extern __shared__ uint8_t smem_raw[];
@@ -122,19 +123,23 @@ __global__ void __launch_bounds__(NTH, 3) pc_delta_kernel(FwdParams p, const __g
     if (ok) {
         samples_pair(sm, D_X, TILE, p, bh, c0 == 0, sqn, rinv);
         __syncthreads();
-        // channel j, tokens 32h .. 32h+31: the running sums of log alpha
-        const int h = tid >> 7, j = tid & (DD - 1);
-        float Gl[32];
+        // channels j0, j0+1, tokens 16 hq .. 16 hq + 15: the running sums of log alpha
+        const int hq = tid >> 6, j0 = 2 * (tid & 63);
+        float Gl0[16], Gl1[16];
         {
-            float acc = 0.f;
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int s_ = h * 32 + i;
-                const float eta = pair_get(sm, D_B, s_, j) * rinv[s_];
-                acc += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
-                Gl[i] = acc;
+            for (int i = 0; i < 16; ++i) {
+                const int s_ = hq * 16 + i;
+                const float2 b2 =
+                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + D_B + pair_off(s_, j0)));
+                const float ri = rinv[s_];
+                a0 += __logf(fmaxf(1.f - b2.x * ri * lam, kAlphaFloor));
+                a1 += __logf(fmaxf(1.f - b2.y * ri * lam, kAlphaFloor));
+                Gl0[i] = a0;
+                Gl1[i] = a1;
             }
-            hsum[h * DD + j] = acc;
+            *reinterpret_cast<float2 *>(hsum + hq * DD + j0) = make_float2(a0, a1);
         }
         // X^T, four 8x8 groups per warp
         for (int g = warp; g < 32; g += NTH / 32) {
@@ -143,20 +148,34 @@ __global__ void __launch_bounds__(NTH, 3) pc_delta_kernel(FwdParams p, const __g
         }
         __syncthreads();
         {
-            // G_{s,j} = (h ? S0_j : 0) + Gl, G_C = S0_j + S1_j; every exponent below is <= 0
-            const float s0 = hsum[j], s1 = hsum[DD + j];
-            const float base = h ? s0 : 0.f, tail = h ? s1 : s0 + s1;  // G_C - base
+            // G_{s,j} = base_j + Gl (base: the quarters before), G_C = the sum of
+            // all four; every exponent below is <= 0
+            float base0 = 0.f, base1 = 0.f, tot0 = 0.f, tot1 = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int s_ = h * 32 + i;
-                const uint32_t off = pair_off(s_, j);
-                __nv_bfloat16 *bp = reinterpret_cast<__nv_bfloat16 *>(sm + D_B + off);
-                __nv_bfloat16 *vp = reinterpret_cast<__nv_bfloat16 *>(sm + D_V + off);
-                const float eta = __bfloat162float(*bp) * rinv[s_];
-                *vp = __float2bfloat16_rn(__expf(tail - Gl[i]) * eta * __bfloat162float(*vp));
-                *bp = __float2bfloat16_rn(__expf(base + Gl[i]));
+            for (int q = 0; q < 4; ++q) {
+                const float2 hs = *reinterpret_cast<const float2 *>(hsum + q * DD + j0);
+                if (q < hq) {
+                    base0 += hs.x;
+                    base1 += hs.y;
+                }
+                tot0 += hs.x;
+                tot1 += hs.y;
             }
-            if (h == 0) ws.g[(size_t)u * DD + j] = __expf(s0 + s1);
+            const float tail0 = tot0 - base0, tail1 = tot1 - base1;  // G_C - base
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int s_ = hq * 16 + i;
+                const uint32_t off = pair_off(s_, j0);
+                __nv_bfloat162 *bp = reinterpret_cast<__nv_bfloat162 *>(sm + D_B + off);
+                __nv_bfloat162 *vp = reinterpret_cast<__nv_bfloat162 *>(sm + D_V + off);
+                const float2 b2 = __bfloat1622float2(*bp), v2 = __bfloat1622float2(*vp);
+                const float ri = rinv[s_];
+                *vp = __floats2bfloat162_rn(__expf(tail0 - Gl0[i]) * (b2.x * ri) * v2.x,
+                                            __expf(tail1 - Gl1[i]) * (b2.y * ri) * v2.y);
+                *bp = __floats2bfloat162_rn(__expf(base0 + Gl0[i]), __expf(base1 + Gl1[i]));
+            }
+            if (hq == 0)
+                *reinterpret_cast<float2 *>(ws.g + (size_t)u * DD + j0) = make_float2(__expf(tot0), __expf(tot1));
         }
         __syncthreads();
         transpose_pair(sbase + D_V, sbase + D_WT);
