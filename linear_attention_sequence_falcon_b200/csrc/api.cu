@@ -66,8 +66,9 @@ FwdParams shape_params(int variant, int form, int pairing, int phi, int window, 
 }
 
 // Bytes of workspace the call with these shapes needs: the bf16 tensor-core
-// paths that hand per-chunk results between kernels (Falcon-1/1A at d = 64,
-// Falcon-2A at d = 128, chunk 64) and the masked-parallel form; 0 otherwise.
+// paths that hand per-chunk results between kernels (Falcon-1/1A and
+// Falcon-3A at d = 64, Falcon-2A at d = 128, chunk 64) and the
+// masked-parallel form; 0 otherwise.
 size_t fwd_ws_need(const FwdParams &p, int dtype) {
     if ((size_t)p.B * p.H * p.L == 0) return 0;
     if (p.form == FALCON_MASKED) {
@@ -80,6 +81,7 @@ size_t fwd_ws_need(const FwdParams &p, int dtype) {
     if (p.form != FALCON_CHUNK || dtype != FALCON_BF16) return 0;
     if (split_chunk_covers(p)) return split_chunk_ws_bytes(p);
     if (pc_chunk_covers(p)) return pc_chunk_ws_bytes(p);
+    if (w_local_covers(p)) return w_local_ws_bytes(p);
     return 0;
 }
 

@@ -1120,8 +1120,25 @@ int launch_split_chunk(const FwdParams &p, cudaStream_t s) {
     }
     chunk_local_kernel<<<(unsigned)std::min<size_t>(units, (size_t)2 * sm_count()), NTH1, L_SMEM, s>>>(p, maps, img, gc);
     // the chain kernel as a programmatic dependent launch (see griddepcontrol in both kernels)
+    if (cudaGetLastError() != cudaSuccess) {
+        ws_release(ws, owned, s);
+        return -7;  // FALCON_ERR_LAUNCH
+    }
+    const int crc = launch_chain_images(p, img, gc, s);
+    ws_release(ws, owned, s);
+    return crc;
+}
+
+int launch_chain_images(const FwdParams &p, const uint8_t *img, const float *gc, cudaStream_t s) {
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_SMEM);
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(BH);
+    cfg.gridDim = dim3(p.B * p.H);
     cfg.blockDim = dim3(NTH2);
     cfg.dynamicSmemBytes = S_SMEM;
     cfg.stream = s;
@@ -1130,14 +1147,9 @@ int launch_split_chunk(const FwdParams &p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const uint8_t *cimg = img;
-    const float *cgc = gc;
-    cudaLaunchKernelEx(&cfg, chunk_chain_kernel, p, cimg, cgc);
-    const cudaError_t e = cudaGetLastError();
-    ws_release(ws, owned, s);
-    return e == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
+    cudaLaunchKernelEx(&cfg, chunk_chain_kernel, p, img, gc);
+    return cudaGetLastError() == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
 }
-
 #ifdef FALCON_TC_DEBUG
 extern "C" int falcon_split_debug_timer_set(long long *ptr) {
     return cudaMemcpyToSymbol(g_split_tim, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;

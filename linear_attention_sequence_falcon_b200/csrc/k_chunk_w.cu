@@ -130,6 +130,9 @@ __device__ __forceinline__ void unpack8(uint4 u, float *f) {
     }
 }
 
+// byte offset of 8-column group g8 of row r in a 64-row [col/8][row][8] bf16 tile
+__device__ __forceinline__ uint32_t rowmajor8(int r, int g8) { return (uint32_t)((g8 * 64 + r) * 16); }
+
 // bf16 element (r, c) of a 128-byte-row swizzled tile
 __device__ __forceinline__ float tile_get(const uint8_t *sm, uint32_t off, int r, int c) {
     return __bfloat162float(
@@ -647,6 +650,366 @@ __global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __gr
     if (warp == 0) tc::tmem_dealloc(tbase, 512);
 }
 
+
+// ============================================================ Falcon-3A: per-chunk images
+namespace {
+// shared memory of w_local_kernel (bytes from a 1024-aligned base): only the
+// inner-product tiles, so that two blocks share an SM.  The Zt^T operands
+// are 128-row A tiles of which rows 64-127 (tensor-memory lanes nobody
+// reads) fall on the P o mask tile that follows each.
+constexpr uint32_t U_XE = 0;            // sample rows x_r (128 rows); then the image staging
+constexpr uint32_t U_VE = 2 * TILE;     // sample rows y_r (128 rows)
+constexpr uint32_t U_Q = 4 * TILE;      // q rows t (64 rows; rows 64-127 only read as unused A rows)
+constexpr uint32_t U_XT0 = 6 * TILE;    // X^T: rows c, samples 0-63
+constexpr uint32_t U_XT1 = 7 * TILE;    // X^T: rows c, samples 64-79
+constexpr uint32_t U_ZT0 = 8 * TILE;    // Zt^T: rows j, samples 0-63
+constexpr uint32_t U_PM0 = 9 * TILE;    // P o (r <= t): rows t, samples 0-63
+constexpr uint32_t U_ZT1 = 10 * TILE;   // Zt^T: rows j, samples 64-79
+constexpr uint32_t U_PM1 = 11 * TILE;   // rows t, samples 64-79
+constexpr uint32_t U_VEC = 12 * TILE;   // scalars (the V_* layout)
+constexpr uint32_t U_BAR = U_VEC + V_END * 4;
+constexpr uint32_t U_SMEM = U_BAR + 64 + 1024;
+static_assert(2 * (U_SMEM + 1024) <= 228 * 1024, "two blocks per SM");
+// tensor memory (256 columns): the band terms; P, whose columns the two
+// last products reuse once it has been read out
+constexpr uint32_t U_G = 0, U_P = 64, U_DS = 64, U_I = 128;
+}  // namespace
+
+// The inner-product family has no state in its increments, so a chunk
+// entered with S_0 gives, exactly,
+//   O = Qt S_0^T + O0,   S_end = g_C S_0 + B,   Qt = D_g Q,
+//   O0[t] = e^{G_t - G_C} (sum_{r<=t} P[t][r] Zt[r] + band_t),   B = Zt^T X,
+// and every term but the S_0 ones is formed for all (head, chunk) units at
+// once here, one block per unit; the chain kernel of the split Falcon-1A
+// path then walks the chunks of a head (the image layout is its own:
+// [unused | Qt (K-major, swizzled) | O0^T | B ([col/8][row][8])] and g_C).
+// A chunk whose G_C is -80 or below sums O0 with one exponential per term.
+template <int BW>
+__global__ void __launch_bounds__(NTH, 2)
+    w_local_kernel(FwdParams p, const __grid_constant__ WMaps maps, uint8_t *img_ws, float *gc_ws) {
+    constexpr int MM = CH + BW - 1;  // sample rows of a chunk
+    constexpr uint32_t IMG = 4 * TILE;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = tc::smem_u32(smem_raw);
+    uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = tc::smem_u32(sm);
+    float *vec = reinterpret_cast<float *>(sm + U_VEC);
+    float *sqn = vec + V_SQN, *vbeta = vec + V_BETA, *veta = vec + V_ETA, *valpha = vec + V_ALPHA, *vG = vec + V_G,
+          *vw = vec + V_W, *pband = vec + V_PB, *misc = vec + V_MISC;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + U_BAR);
+    uint64_t *tbar = bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, chalf = warp >> 2, row = quarter * 32 + lane;
+    const int L = p.L, nch = (L + CH - 1) / CH;
+    const int u = blockIdx.x, bh = u / nch, c = u - bh * nch, c0 = c * CH, nt = min(CH, L - c0);
+    const float lam = p.lambda[bh % p.H];
+    const __nv_bfloat16 *betap = static_cast<const __nv_bfloat16 *>(p.beta) + (size_t)bh * L;
+
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::mbar_init(tbar, 1);
+        tc::fence_mbar_init();
+        // sample row r holds sample i = c0 - BW + 1 + r: key row i-1 (prefix
+        // pair) or i (same-step pair), value row i
+        const int r0 = c0 - BW + 1, krow = p.pairing == 0 ? r0 - 1 : r0;
+        tc::mbar_arrive_expect_tx(tbar, 5 * TILE);
+        tc::tma_load_3d(sbase + U_XE, &maps.k, 0, krow, bh, tbar);
+        tc::tma_load_3d(sbase + U_XE + TILE, &maps.k, 0, krow + 64, bh, tbar);
+        tc::tma_load_3d(sbase + U_VE, &maps.v, 0, r0, bh, tbar);
+        tc::tma_load_3d(sbase + U_VE + TILE, &maps.v, 0, r0 + 64, bh, tbar);
+        tc::tma_load_3d(sbase + U_Q, &maps.q, 0, c0, bh, tbar);
+    }
+    __syncwarp();
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 256);
+        tc::tmem_relinquish();
+    }
+    if (tid < CH) vbeta[tid] = tid < nt ? __bfloat162float(betap[c0 + tid]) : 0.f;
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
+    bool ok = tc::mbar_wait_timeout(tbar, 0, kWaitNs);
+    ok = __syncthreads_and(ok);
+    uint32_t phase = 0;
+    if (ok) {
+        // ---- samples: rows r < MM normalised in place (four threads per row), rows MM..NR-1 zero
+        for (int rr = tid >> 2; rr < NR; rr += NTH / 4) {  // a warp's lanes share the trip count
+            const int part = tid & 3, i = c0 - BW + 1 + rr;
+            float xr[16];
+            bool given = false;  // a carried sample, used as given
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xr[e] = 0.f;
+            if (rr < MM) {
+                // a continued segment: sample 0 (prefix pair) is the carried phi(k); samples
+                // before it come from the carried window, values included
+                const bool cx = i == 0 && p.pairing == 0 && p.x_prev != nullptr;
+                const float *cw = (i < 0 && i >= -(BW - 1) && p.win)
+                                      ? p.win + ((size_t)bh * (BW - 1) + (i + BW - 1)) * (DD + DD)
+                                      : nullptr;
+                given = cx || cw;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int cc = part * 16 + h2 * 8;
+                    if (cx) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) xr[h2 * 8 + e] = p.x_prev[(size_t)bh * DD + cc + e];
+                    } else if (cw) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) xr[h2 * 8 + e] = cw[cc + e];
+                    } else {
+                        unpack8(*reinterpret_cast<const uint4 *>(sm + U_XE + tc::sw128(rr, part * 2 + h2)), &xr[h2 * 8]);
+                    }
+                }
+                if (cw) {
+                    float yv[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) yv[e] = cw[DD + part * 16 + e];
+                    *reinterpret_cast<uint4 *>(sm + U_VE + tc::sw128(rr, part * 2)) = pack8(&yv[0]);
+                    *reinterpret_cast<uint4 *>(sm + U_VE + tc::sw128(rr, part * 2 + 1)) = pack8(&yv[8]);
+                }
+            }
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ss += xr[e] * xr[e];
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            const float inv = (given || p.phi != 0) ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xr[e] *= inv;
+            if (part == 0) sqn[rr] = ss * inv * inv;
+            *reinterpret_cast<uint4 *>(sm + U_XE + tc::sw128(rr, part * 2)) = pack8(&xr[0]);
+            *reinterpret_cast<uint4 *>(sm + U_XE + tc::sw128(rr, part * 2 + 1)) = pack8(&xr[8]);
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        // ---- P = Q X^T over the sample rows
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_k(tbase + U_P, sbase + U_Q, sbase + U_XE, NR);
+            tc::mma_commit(bar);
+        }
+        // ---- per-token steps and decays (warps 0-1), X^T (warps 2-7)
+        if (tid < CH) {
+            const int t = tid;
+            float n = 0.f;
+#pragma unroll
+            for (int m = 0; m < BW; ++m) n += sqn[t + m];
+            float eta, alpha;
+            step_and_decay(vbeta[t], n, p.eps, lam, eta, alpha);
+            float run = __logf(alpha);  // inclusive sum over the warp
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, run, o);
+                if (lane >= o) run += y;
+            }
+            if (lane == 31) misc[warp] = run;
+            veta[t] = eta;
+            valpha[t] = alpha;
+            vG[t] = run;  // warp-local; warp 1 adds warp 0's total below
+        } else {
+            for (int g = warp - 2; g < 20; g += 6) {
+                const int srb = g >> 1, cb0 = (g & 1) * 4;
+                transpose_blk(sbase + U_XE, srb, cb0, srb < 8 ? sbase + U_XT0 : sbase + U_XT1, srb & 7);
+            }
+        }
+        __syncthreads();
+        if (tid < CH) {
+            const int t = tid;
+            const float G = vG[t] + (t >= 32 ? misc[0] : 0.f);
+            const float GC = misc[0] + misc[1];
+            vw[t] = __expf(GC - G) * veta[t];
+            __syncwarp();
+            vG[t] = G;
+            if (t == 0) misc[2] = GC;
+        }
+        __syncthreads();
+        ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        phase ^= 1;
+        ok = __syncthreads_and(ok);
+    }
+    const float GC = misc[2];
+    const bool unsafe = !(GC > kMinLogDecay);
+    if (ok) {
+        tc::fence_after_sync();
+        // ---- P (lanes 0-63) -> P o (r <= t) bf16 and the band P[t][t+k], k = 1 .. BW-1
+        if (quarter < 2) {
+            const int t = row;
+            for (int g = chalf; g < 5; g += 2) {
+                float v[16];
+                tc::tmem_ld16(tl + U_P + g * 16, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int r = g * 16 + i, k = r - t;
+                    if (k >= 1 && k < BW) pband[t * 4 + k] = v[i];
+                    v[i] = r <= t ? v[i] : 0.f;
+                }
+                const uint32_t dst = g < 4 ? U_PM0 : U_PM1;
+                const int ch0 = g < 4 ? g * 2 : 0;
+                *reinterpret_cast<uint4 *>(sm + dst + tc::sw128(t, ch0)) = pack8(&v[0]);
+                *reinterpret_cast<uint4 *>(sm + dst + tc::sw128(t, ch0 + 1)) = pack8(&v[8]);
+            }
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        // ---- Zt[r] = sum over the tokens whose window holds row r of w_t y_r, and
+        //      the band terms sum_k P[t][t+k] Zacc_{t+1}[t+k] (warps 0-1: thread =
+        //      channel j = lane), in blocks of 8 tokens as in w_chunk_kernel
+        if (tid < DD) {
+            const int j = tid;
+            constexpr int NB = 8, RB = NB + BW - 1;  // tokens and rows of a block
+            float zb[RB];                            // rows t0 .. t0+RB-1
+#pragma unroll
+            for (int k = 0; k < RB; ++k) zb[k] = 0.f;
+#pragma unroll 1
+            for (int tb = 0; tb < 4; ++tb) {
+                float bnd[16];
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int t0 = tb * 16 + hb * NB;
+#pragma unroll
+                    for (int i = 0; i < NB; ++i) {
+                        const int t = t0 + i;
+                        const float wt = vw[t];
+                        // z_{t,m} lands on row t+m
+#pragma unroll
+                        for (int m = 0; m < BW; ++m) zb[i + m] += wt * tile_get(sm, U_VE, t + m, j);
+                        float bsum = 0.f;
+#pragma unroll
+                        for (int k = 1; k < BW; ++k) bsum = fmaf(pband[t * 4 + k], zb[i + k], bsum);
+                        bnd[hb * NB + i] = bsum;
+                    }
+                    // rows t0 .. t0+7 are final (bf16 Zt^T row j, 16-byte chunk t0 / 8);
+                    // rows t0+8 .. carry into the next block
+                    *reinterpret_cast<uint4 *>(sm + U_ZT0 + tc::sw128(j, t0 >> 3)) = pack8(zb);
+#pragma unroll
+                    for (int k = 0; k < RB; ++k) zb[k] = k + NB < RB ? zb[k + NB] : 0.f;
+                }
+                tc::tmem_st16(tl + U_G + tb * 16, bnd);
+            }
+            // rows 64 .. 64+BW-2 end the chunk in registers; samples beyond are zero
+            float zt[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) zt[k] = k < BW - 1 ? zb[k] : 0.f;
+            *reinterpret_cast<uint4 *>(sm + U_ZT1 + tc::sw128(j, 0)) = pack8(&zt[0]);
+            *reinterpret_cast<uint4 *>(sm + U_ZT1 + tc::sw128(j, 1)) = pack8(&zt[8]);
+            tc::tmem_wait_st();
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_k(tbase + U_DS, sbase + U_ZT0, sbase + U_XT0, DD, sbase + U_ZT1, sbase + U_XT1, 1);  // Zt^T X
+            issue_k(tbase + U_I, sbase + U_ZT0, sbase + U_PM0, CH, sbase + U_ZT1, sbase + U_PM1, 1);   // Zt^T (P o m)^T
+            tc::mma_commit(bar);
+        }
+        ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        phase ^= 1;
+        ok = __syncthreads_and(ok);
+    }
+    if (ok) {
+        tc::fence_after_sync();
+        // ---- the image, staged over the consumed sample tiles: Qt at 0, O0^T at
+        //      TILE, B at 2 TILE (stage offsets; image offsets one TILE more)
+        uint8_t *stg = sm + U_XE;
+        // Qt = D_g Q: rows t (t >= nt: zero rows of the tile, kept)
+        for (int e = tid; e < CH * 8; e += NTH) {
+            const int t = e >> 3, c16 = e & 7;
+            float q8[8];
+            unpack8(*reinterpret_cast<const uint4 *>(sm + U_Q + tc::sw128(t, c16)), q8);
+            const float g = __expf(vG[t]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) q8[i] *= g;
+            *reinterpret_cast<uint4 *>(stg + tc::sw128(t, c16)) = pack8(q8);
+        }
+        if (quarter < 2) {
+            const int j = row;
+            // O0^T row j, tokens 32 chalf .. + 31
+            if (!unsafe) {
+                const float ig = __expf(-GC);
+#pragma unroll
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    const int t0 = chalf * 32 + k2 * 16;
+                    float iv[16], bv[16], o[16];
+                    tc::tmem_ld16(tl + U_I + t0, iv);
+                    tc::tmem_ld16(tl + U_G + t0, bv);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o[i] = t0 + i < nt ? __expf(vG[t0 + i]) * (ig * (iv[i] + bv[i])) : 0.f;
+                    *reinterpret_cast<uint4 *>(stg + TILE + rowmajor8(j, t0 >> 3)) = pack8(&o[0]);
+                    *reinterpret_cast<uint4 *>(stg + TILE + rowmajor8(j, (t0 >> 3) + 1)) = pack8(&o[8]);
+                }
+            } else {
+                // O0[t][j] = sum_{s<=t} e^{G_t-G_s} eta_s sum_m P[t][s+m] y_{s+m}[j], one
+                // exponential per term (every exponent <= 0); P from the masked tile
+                // (r <= t) and the band (r = t+1 .. t+BW-1)
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    float o[8];
+                    for (int i = 0; i < 8; ++i) {
+                        const int t = chalf * 32 + g8 * 8 + i;
+                        float acc = 0.f;
+                        if (t < nt) {
+                            const float Gt = vG[t];
+                            for (int s = 0; s <= t; ++s) {
+                                float a = 0.f;
+#pragma unroll
+                                for (int m = 0; m < BW; ++m) {
+                                    const int r = s + m;
+                                    const float pr = r <= t ? tile_get(sm, r < 64 ? U_PM0 : U_PM1, t, r & 63)
+                                                            : pband[t * 4 + (r - t)];
+                                    a = fmaf(pr, tile_get(sm, U_VE, r, j), a);
+                                }
+                                acc = fmaf(__expf(Gt - vG[s]) * veta[s], a, acc);
+                            }
+                        }
+                        o[i] = acc;
+                    }
+                    *reinterpret_cast<uint4 *>(stg + TILE + rowmajor8(j, chalf * 4 + g8)) = pack8(o);
+                }
+            }
+        }
+        // B is staged over the value tile, which the branch above may still read
+        __syncthreads();
+        if (quarter < 2) {
+            const int j = row;
+            // B row j = (Zt^T X)[j][.], columns 32 chalf .. + 31
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int i0 = chalf * 32 + k2 * 16;
+                float dv[16];
+                tc::tmem_ld16(tl + U_DS + i0, dv);
+                tc::tmem_wait_ld();
+                *reinterpret_cast<uint4 *>(stg + 2 * TILE + rowmajor8(j, i0 >> 3)) = pack8(&dv[0]);
+                *reinterpret_cast<uint4 *>(stg + 2 * TILE + rowmajor8(j, (i0 >> 3) + 1)) = pack8(&dv[8]);
+            }
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            gc_ws[u] = __expf(GC);
+            tc::bulk_store(img_ws + (size_t)u * IMG + TILE, sbase + U_XE, 3 * TILE);
+            tc::bulk_commit();
+            tc::bulk_wait_all();
+        }
+    } else if (tid == 0) {
+        atomicAdd(&g_w_wait_timeouts, 1u);
+        (void)tc::mbar_wait_timeout(tbar, 0, kWaitNs);  // the load must land before the block leaves
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 256);
+}
+
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -693,7 +1056,42 @@ int launch_w(const FwdParams &p, const WMaps &maps, cudaStream_t s) {
     return cudaGetLastError() == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
 }
 
+// Falcon-3A: the per-chunk images, then the chain kernel of the split path
+template <int BW>
+int launch_wl(const FwdParams &p, const WMaps &maps, cudaStream_t s) {
+    const size_t units = (size_t)p.B * p.H * ((p.L + CH - 1) / CH);
+    void *ws = nullptr;
+    bool owned = false;
+    const int wrc = ws_acquire(p.ws_given, p.ws, p.ws_bytes, w_local_ws_bytes(p), s, &ws, &owned);
+    if (wrc) return wrc;
+    uint8_t *img = static_cast<uint8_t *>(ws);
+    float *gc = reinterpret_cast<float *>(img + units * 4 * TILE);
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        cudaFuncSetAttribute(w_local_kernel<BW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)U_SMEM);
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    w_local_kernel<BW><<<(unsigned)units, NTH, U_SMEM, s>>>(p, maps, img, gc);
+    int rc = cudaGetLastError() == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
+    if (rc == 0) rc = launch_chain_images(p, img, gc, s);
+    ws_release(ws, owned, s);
+    return rc;
+}
+
 }  // namespace
+
+bool w_local_covers(const FwdParams &p) {
+    if (!(p.variant == F3A && p.dk == DD && p.dv == DD && p.chunk == CH && p.window >= 2 && p.window <= 4))
+        return false;
+    return (size_t)p.B * p.H * ((p.L + CH - 1) / CH) <= 0x7fffffffu;
+}
+
+size_t w_local_ws_bytes(const FwdParams &p) {
+    const size_t units = (size_t)p.B * p.H * ((p.L + CH - 1) / CH);
+    return units * 4 * TILE + units * sizeof(float);
+}
 
 int launch_w_chunk(const FwdParams &p, cudaStream_t s) {
     const bool shape_ok = (p.variant == F3 || p.variant == F3A) && p.dk == DD && p.dv == DD && p.chunk == CH &&
@@ -705,6 +1103,13 @@ int launch_w_chunk(const FwdParams &p, cudaStream_t s) {
     WMaps maps;
     if (!make_map(&maps.q, p.q, BH, p.L) || !make_map(&maps.k, p.k, BH, p.L) || !make_map(&maps.v, p.v, BH, p.L))
         return 1;
+    if (w_local_covers(p)) {
+        switch (p.window) {
+            case 2: return launch_wl<2>(p, maps, s);
+            case 3: return launch_wl<3>(p, maps, s);
+            default: return launch_wl<4>(p, maps, s);
+        }
+    }
     switch (p.window) {
         case 2: return launch_w<2>(p, maps, s);
         case 3: return launch_w<3>(p, maps, s);
