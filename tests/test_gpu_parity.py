@@ -419,6 +419,34 @@ def test_decode_d128_pair_counts(F, N, H):
     assert rel(S, oS) <= 1e-4
 
 
+@pytest.mark.parametrize("variant", ["F1", "F2A"])
+def test_decode_d128_state_16_byte_aligned(F, variant):
+    """d = 128 decode on a state that is only 16-byte aligned (a view into a
+    larger buffer) and on an aligned one, both against the fp64 recurrence
+    after the same prefill: the row accesses need 16-byte alignment only."""
+    N, H, dk, L0, steps = 2, 3, 128, 20, 5
+    d = gen.draw(variant, N, H, L0 + steps, dk, dk, seed=606, dtype="f32", lam=0.02)
+    pre = {n: d[n][:, :, :L0].contiguous() for n in ("q", "k", "v", "beta")}
+    _, S = F.fwd(variant, "chunk", *(pre[n].cuda() for n in ("q", "k", "v", "beta")), d["lam"].cuda(), d["eps"],
+                 chunk=64)
+    oo, oS = oracle_fwd(d, variant, 1)
+    tok = {n: d[n][:, :, L0:].movedim(2, 0).contiguous().cuda() for n in ("q", "k", "v", "beta")}
+    for shift in (0, 4):  # floats: 0 keeps torch's alignment, 4 leaves 16 bytes
+        buf = torch.zeros(S.numel() + 8, dtype=torch.float32, device="cuda")
+        Sx = buf[shift:shift + S.numel()].view(S.shape)
+        Sx.copy_(S)
+        assert (Sx.data_ptr() % 32 == 0) == (shift == 0)
+        x_prev, _ = F.carry_from_prefill(variant, pre["k"].cuda(), pre["v"].cuda(), 1)
+        outs = torch.empty((steps, N, H, dk), dtype=torch.float32, device="cuda")
+        for i in range(steps):
+            F.decode_step(variant, tok["q"][i], tok["k"][i], tok["v"][i], tok["beta"][i], d["lam"].cuda(), d["eps"],
+                          1, Sx, x_prev, None, out=outs[i])
+        torch.cuda.synchronize()
+        o = outs.movedim(0, 2).double().cpu().numpy()
+        assert rel(o, oo[:, :, L0:]) <= 1e-4, shift
+        assert rel(Sx.double().cpu().numpy(), oS) <= 1e-4, shift
+
+
 # --------------------------------------------------------------- tensor-core path options and extremes
 
 @pytest.mark.parametrize("pairing,phi", [("same_step", "l2"), ("prefix", "identity"), ("same_step", "identity")])
