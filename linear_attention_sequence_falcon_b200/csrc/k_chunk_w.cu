@@ -25,8 +25,11 @@
 // a chunk below that runs its tokens one by one (the recurrence itself, S in
 // registers).
 //
-// One block per (b, h) walks the chunks; S stays in fp32 registers (thread:
-// row j, 32 columns) with its bf16 copy as the operand of S_0 X^T and S_0 Q^T.
+// Falcon-3: one block per (b, h) walks the chunks (w_chunk_kernel); S stays
+// in fp32 registers (thread: row j, 32 columns) with its bf16 copy as the
+// operand of S_0 X^T and S_0 Q^T.  Falcon-3A has no state in its increments:
+// w_local_kernel forms every (head, chunk) unit's image at once and the
+// chain kernel of the split Falcon-1A path walks the chunks (below).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
