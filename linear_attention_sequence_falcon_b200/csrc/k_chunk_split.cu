@@ -807,7 +807,7 @@ __global__ void __launch_bounds__(NTH2, 1)
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool reg = p.variant == F1;
+    const bool reg = p.variant == F1 || p.variant == F3;  // a -Phi'^T tile in the image
     const int L = p.L, nch = (L + CH - 1) / CH;
     const int bh = blockIdx.x;
     const uint8_t *imgs = img_ws + (size_t)bh * nch * IMG;

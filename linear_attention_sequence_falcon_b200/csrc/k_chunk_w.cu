@@ -33,6 +33,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -1013,6 +1014,527 @@ __global__ void __launch_bounds__(NTH, 2)
     if (warp == 0) tc::tmem_dealloc(tbase, 256);
 }
 
+
+// ============================================================ Falcon-3: per-chunk images
+// The chunk's map S_0 -> (O, S_end) is affine.  Running the chunk's
+// computation with S_0 = 0 over the real values gives O0 and B, and with
+// S_0 = I and zero values it gives Qt and the transition T:
+//   O = Qt S_0^T + O0,   S_end = S_0 T + B.
+// w_reg_local_kernel does both at once, one block per (head, chunk), on 128
+// rows: rows 0-63 are the value channels (S_0 = 0), rows 64-127 the rows of
+// the identity (values zero), so the windowed system is walked for 128
+// right-hand sides by warps 0-3 (every tensor-memory lane quarter).  It
+// writes the chain kernel's image [(T - g_C I)^T | Qt | O0^T | B] and g_C,
+// and the chain of the Falcon-1 path walks the chunks of a head.  A chunk
+// whose G_C is -80 or below runs the recurrence token by token on the 128
+// rows instead.
+namespace {
+// two sets of input tiles, so that a block prefetches its next unit while it
+// computes this one; each set's x and y rows are then its image staging area
+constexpr uint32_t R_XE0 = 0;            // sample rows x_r (128 rows)
+constexpr uint32_t R_VE0 = 2 * TILE;     // sample rows y_r (128 rows)
+constexpr uint32_t R_Q0 = 4 * TILE;      // q rows t (64 rows; the P product reads the next 64 as unused A rows)
+constexpr uint32_t R_XE1 = 5 * TILE, R_VE1 = 7 * TILE, R_Q1 = 9 * TILE;
+constexpr uint32_t R_XT0 = 10 * TILE;   // X^T: rows c, samples 0-63
+constexpr uint32_t R_XT1 = 11 * TILE;   // X^T: rows c, samples 64-79
+constexpr uint32_t R_ZT0 = 12 * TILE;   // Zt^T: 128 rows, samples 0-63
+constexpr uint32_t R_ZT1 = 14 * TILE;   // Zt^T: 128 rows, samples 64-79
+constexpr uint32_t R_PM0 = 16 * TILE;   // P o (r <= t): rows t, samples 0-63
+constexpr uint32_t R_PM1 = 17 * TILE;   // rows t, samples 64-79
+constexpr uint32_t R_A = 18 * TILE;                   // fp32 A[r][r'], r < 68
+constexpr uint32_t R_ZA = R_A + 68 * LDA * 4;         // fp32 Zacc[row][r], 128 rows (token path: outputs)
+constexpr uint32_t R_VEC = R_ZA + 2 * DD * LDZ * 4;   // scalars: the V_* layout up to the band, then
+constexpr int RV_RED = V_RED, RV_MISC = V_RED + 2 * 4 * 2 * DD, RV_END = RV_MISC + 16;  // red over 128 rows
+constexpr uint32_t R_BAR = R_VEC + RV_END * 4;  // MMA barrier, one load barrier per set
+constexpr uint32_t R_SMEM = R_BAR + 64 + 1024;
+static_assert(R_SMEM <= 227 * 1024, "shared memory");
+static_assert(2 * DD * CH <= 2 * DD * LDZ, "token-path outputs fit over Zacc");
+// tensor memory (512 columns)
+constexpr uint32_t RC_G = 0;     // Gram: lanes r, columns r' (80); then the band terms, lanes row, columns t
+constexpr uint32_t RC_P = 96;    // P: lanes t, columns r (80)
+constexpr uint32_t RC_DS = 192;  // Zt^T X: lanes row, columns c (64)
+constexpr uint32_t RC_I = 256;   // Zt^T (P o mask)^T: lanes row, columns t (64)
+}  // namespace
+
+template <int BW>
+__global__ void __launch_bounds__(NTH, 1)
+    w_reg_local_kernel(FwdParams p, const __grid_constant__ WMaps maps, uint8_t *img_ws, float *gc_ws) {
+    constexpr int MM = CH + BW - 1;  // sample rows of a chunk
+    constexpr uint32_t IMG = 4 * TILE;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = tc::smem_u32(smem_raw);
+    uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = tc::smem_u32(sm);
+    float *At = reinterpret_cast<float *>(sm + R_A);
+    float *Za = reinterpret_cast<float *>(sm + R_ZA);
+    float *vec = reinterpret_cast<float *>(sm + R_VEC);
+    float *sqn = vec + V_SQN, *vbeta = vec + V_BETA, *veta = vec + V_ETA, *valpha = vec + V_ALPHA, *vG = vec + V_G,
+          *vw = vec + V_W, *vkap = vec + V_KAP, *vgm1 = vec + V_GM1, *pband = vec + V_PB, *red = vec + RV_RED,
+          *misc = vec + RV_MISC;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + R_BAR);
+    uint64_t *tbar = bar + 1;  // [2] the loads of input set 0 / 1
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 3);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, chalf = warp >> 2, row = quarter * 32 + lane;  // row: 0-127
+    const int L = p.L, nch = (L + CH - 1) / CH;
+    const int units = p.B * p.H * nch;
+
+    // unit w's inputs into set st: sample row r holds sample i = c0 - BW + 1 + r,
+    // key row i-1 (prefix pair) or i (same-step pair), value row i
+    auto load_unit = [&](int w, int st) {
+        const int wbh = w / nch, wc0 = (w - wbh * nch) * CH;
+        const int r0 = wc0 - BW + 1, krow = p.pairing == 0 ? r0 - 1 : r0;
+        const uint32_t xe = st ? R_XE1 : R_XE0, ve = st ? R_VE1 : R_VE0, qq = st ? R_Q1 : R_Q0;
+        tc::mbar_arrive_expect_tx(&tbar[st], 5 * TILE);
+        tc::tma_load_3d(sbase + xe, &maps.k, 0, krow, wbh, &tbar[st]);
+        tc::tma_load_3d(sbase + xe + TILE, &maps.k, 0, krow + 64, wbh, &tbar[st]);
+        tc::tma_load_3d(sbase + ve, &maps.v, 0, r0, wbh, &tbar[st]);
+        tc::tma_load_3d(sbase + ve + TILE, &maps.v, 0, r0 + 64, wbh, &tbar[st]);
+        tc::tma_load_3d(sbase + qq, &maps.q, 0, wc0, wbh, &tbar[st]);
+    };
+    int loads = 0;  // loads issued (thread 0)
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::mbar_init(&tbar[0], 1);
+        tc::mbar_init(&tbar[1], 1);
+        tc::fence_mbar_init();
+        if ((int)blockIdx.x < units) {
+            load_unit(blockIdx.x, 0);
+            loads = 1;
+        }
+    }
+    __syncwarp();
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    // X^T beyond sample 79 only pads its tile
+    for (int e = tid; e < TILE / 16; e += NTH)
+        *reinterpret_cast<uint4 *>(sm + R_XT1 + e * 16) = make_uint4(0, 0, 0, 0);
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
+    uint32_t phase = 0;  // MMA-completion parity
+    bool ok = true;
+    int n = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
+    const int set = n & 1;
+    const uint32_t R_XE = set ? R_XE1 : R_XE0, R_VE = set ? R_VE1 : R_VE0, R_Q = set ? R_Q1 : R_Q0;
+    const int bh = u / nch, c = u - bh * nch, c0 = c * CH, nt = min(CH, L - c0);
+    const float lam = p.lambda[bh % p.H];
+    const __nv_bfloat16 *betap = static_cast<const __nv_bfloat16 *>(p.beta) + (size_t)bh * L;
+    if (tid == 0 && u + (int)gridDim.x < units) {
+        // the other set's last image has been read out by its bulk store
+        tc::bulk_wait_read();
+        load_unit(u + gridDim.x, set ^ 1);
+        ++loads;
+    }
+    if (tid < CH) vbeta[tid] = tid < nt ? __bfloat162float(betap[c0 + tid]) : 0.f;
+    ok = tc::mbar_wait_timeout(&tbar[set], (uint32_t)((n >> 1) & 1), kWaitNs);
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    if (ok) {
+        // ---- samples: rows r < MM normalised in place (four threads per row), rows MM..NR-1 zero
+        for (int rr = tid >> 2; rr < NR; rr += NTH / 4) {  // a warp's lanes share the trip count
+            const int part = tid & 3, i = c0 - BW + 1 + rr;
+            float xr[16];
+            bool given = false;  // a carried sample, used as given
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xr[e] = 0.f;
+            if (rr < MM) {
+                const bool cx = i == 0 && p.pairing == 0 && p.x_prev != nullptr;
+                const float *cw = (i < 0 && i >= -(BW - 1) && p.win)
+                                      ? p.win + ((size_t)bh * (BW - 1) + (i + BW - 1)) * (DD + DD)
+                                      : nullptr;
+                given = cx || cw;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int cc = part * 16 + h2 * 8;
+                    if (cx) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) xr[h2 * 8 + e] = p.x_prev[(size_t)bh * DD + cc + e];
+                    } else if (cw) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) xr[h2 * 8 + e] = cw[cc + e];
+                    } else {
+                        unpack8(*reinterpret_cast<const uint4 *>(sm + R_XE + tc::sw128(rr, part * 2 + h2)), &xr[h2 * 8]);
+                    }
+                }
+                if (cw) {
+                    float yv[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) yv[e] = cw[DD + part * 16 + e];
+                    *reinterpret_cast<uint4 *>(sm + R_VE + tc::sw128(rr, part * 2)) = pack8(&yv[0]);
+                    *reinterpret_cast<uint4 *>(sm + R_VE + tc::sw128(rr, part * 2 + 1)) = pack8(&yv[8]);
+                }
+            }
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ss += xr[e] * xr[e];
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            const float inv = (given || p.phi != 0) ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xr[e] *= inv;
+            if (part == 0) sqn[rr] = ss * inv * inv;
+            *reinterpret_cast<uint4 *>(sm + R_XE + tc::sw128(rr, part * 2)) = pack8(&xr[0]);
+            *reinterpret_cast<uint4 *>(sm + R_XE + tc::sw128(rr, part * 2 + 1)) = pack8(&xr[8]);
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        // ---- the Gram and P over the sample rows
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_k(tbase + RC_G, sbase + R_XE, sbase + R_XE, NR);
+            issue_k(tbase + RC_P, sbase + R_Q, sbase + R_XE, NR);
+            tc::mma_commit(bar);
+        }
+        // ---- per-token steps and decays (warps 0-1), X^T (warps 2-7)
+        if (tid < CH) {
+            const int t = tid;
+            float n = 0.f;
+#pragma unroll
+            for (int m = 0; m < BW; ++m) n += sqn[t + m];
+            float eta, alpha;
+            step_and_decay(vbeta[t], n, p.eps, lam, eta, alpha);
+            float run = __logf(alpha);  // inclusive sum over the warp
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, run, o);
+                if (lane >= o) run += y;
+            }
+            if (lane == 31) misc[warp] = run;
+            veta[t] = eta;
+            valpha[t] = alpha;
+            vG[t] = run;  // warp-local; warp 1 adds warp 0's total below
+        } else {
+            for (int g = warp - 2; g < 20; g += 6) {
+                const int srb = g >> 1, cb0 = (g & 1) * 4;
+                transpose_blk(sbase + R_XE, srb, cb0, srb < 8 ? sbase + R_XT0 : sbase + R_XT1, srb & 7);
+            }
+        }
+        __syncthreads();
+        if (tid < CH) {
+            const int t = tid;
+            const float G = vG[t] + (t >= 32 ? misc[0] : 0.f);
+            const float GC = misc[0] + misc[1];
+            const float Gm = G - __logf(valpha[t]);  // G_{t-1}
+            const float eta = veta[t];
+            vw[t] = __expf(GC - G) * eta;
+            vkap[t] = __fdividef(eta, valpha[t]);
+            vgm1[t] = __expf(Gm);
+            __syncwarp();
+            vG[t] = G;
+            if (t == 0) misc[2] = GC;
+        }
+        __syncthreads();
+        ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        phase ^= 1;
+        ok = __syncthreads_and(ok);
+    }
+    const float GC = misc[2];
+    const bool unsafe = !(GC > kMinLogDecay);
+    uint8_t *stg = sm + R_XE;  // the image, staged over the consumed sample tiles
+    if (ok && !unsafe) {
+        tc::fence_after_sync();
+        // ---- Gram rows r < 68 (lanes 0-79) -> fp32; P (lanes 0-63) -> P o (r <= t) bf16 and the band
+        if (quarter < 3) {
+            const int r = row;
+            for (int g = chalf; g < 5; g += 2) {
+                float v[16];
+                tc::tmem_ld16(tl + RC_G + g * 16, v);
+                tc::tmem_wait_ld();
+                if (r < LDA) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (g * 16 + i < LDA) At[r * LDA + g * 16 + i] = v[i];
+                }
+            }
+        }
+        if (quarter < 2) {
+            const int t = row;
+            for (int g = chalf; g < 5; g += 2) {
+                float v[16];
+                tc::tmem_ld16(tl + RC_P + g * 16, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int r = g * 16 + i, k = r - t;
+                    if (k >= 1 && k < BW) pband[t * 4 + k] = v[i];
+                    v[i] = r <= t ? v[i] : 0.f;
+                }
+                const uint32_t dst = g < 4 ? R_PM0 : R_PM1;
+                const int ch0 = g < 4 ? g * 2 : 0;
+                *reinterpret_cast<uint4 *>(sm + dst + tc::sw128(t, ch0)) = pack8(&v[0]);
+                *reinterpret_cast<uint4 *>(sm + dst + tc::sw128(t, ch0 + 1)) = pack8(&v[8]);
+            }
+        }
+        if (tid < 2 * DD) {
+#pragma unroll
+            for (int q4 = 0; q4 < NR / 4; ++q4)
+                *reinterpret_cast<float4 *>(Za + tid * LDZ + q4 * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        // ---- the chunk's system in token order for 128 right-hand sides (warps
+        //      0-3: thread = row = lane): rows 0-63 the value channels (S_0 = 0),
+        //      rows 64-127 the rows of the identity (values zero, (S_0 x_r) = x_r[c]);
+        //      in blocks of 8 tokens as in w_chunk_kernel
+        if (tid < 2 * DD) {
+            const int rw = tid;
+            const bool vrow = rw < DD;  // a value channel; else identity row c = rw - 64
+            float *za = Za + rw * LDZ;
+            auto yv = [&](int r) { return vrow ? tile_get(sm, R_VE, r, rw) : 0.f; };
+            auto sxv = [&](int r) { return vrow ? 0.f : tile_get(sm, R_XE, r, rw - DD); };
+            constexpr int NB = 8, RB = NB + BW - 1;  // tokens and rows of a block
+            float zb[RB];                            // rows t0 .. t0+RB-1
+#pragma unroll
+            for (int k = 0; k < RB; ++k) zb[k] = 0.f;
+#pragma unroll 1
+            for (int tb = 0; tb < 4; ++tb) {
+                float bnd[16];
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int t0 = tb * 16 + hb * NB;
+                    // rows r' < t0 are final (in shared memory): the sum over them
+                    // of A[t+m][r'] Zacc[r'] depends on t+m only, one sum per row
+                    float crr[RB];
+#pragma unroll
+                    for (int rr = 0; rr < RB; ++rr) crr[rr] = 0.f;
+                    for (int q = 0; q < (t0 >> 2); ++q) {
+                        const float4 z4 = *reinterpret_cast<const float4 *>(za + q * 4);
+#pragma unroll
+                        for (int rr = 0; rr < RB; ++rr) {
+                            const float4 a4 = *reinterpret_cast<const float4 *>(At + (t0 + rr) * LDA + q * 4);
+                            crr[rr] = fmaf(a4.x, z4.x, fmaf(a4.y, z4.y, fmaf(a4.z, z4.z, fmaf(a4.w, z4.w, crr[rr]))));
+                        }
+                    }
+                    float cr[NB][BW];
+#pragma unroll
+                    for (int i = 0; i < NB; ++i)
+#pragma unroll
+                        for (int m = 0; m < BW; ++m) cr[i][m] = crr[i + m];
+#pragma unroll
+                    for (int i = 0; i < NB; ++i) {
+                        const int t = t0 + i;
+                        const float wt = vw[t], gm = vgm1[t], kt = vkap[t];
+#pragma unroll
+                        for (int m = 0; m < BW; ++m) {
+                            float acc = cr[i][m];
+                            // rows t0 .. t+BW-2 still accumulating: registers
+#pragma unroll
+                            for (int k = 0; k < i + BW - 1; ++k) acc = fmaf(At[(t + m) * LDA + t0 + k], zb[k], acc);
+                            const int r = t + m;
+                            cr[i][m] = wt * (yv(r) - gm * sxv(r)) - kt * acc;
+                        }
+                        // z_{t,m} lands on row t+m only after every slot of token t used the old sums
+#pragma unroll
+                        for (int m = 0; m < BW; ++m) zb[i + m] += cr[i][m];
+                        float bsum = 0.f;
+#pragma unroll
+                        for (int k = 1; k < BW; ++k) bsum = fmaf(pband[t * 4 + k], zb[i + k], bsum);
+                        bnd[hb * NB + i] = bsum;
+                    }
+                    // rows t0 .. t0+7 are final; rows t0+8 .. carry into the next block
+#pragma unroll
+                    for (int k = 0; k < NB; ++k) za[t0 + k] = zb[k];
+#pragma unroll
+                    for (int k = 0; k < RB; ++k) zb[k] = k + NB < RB ? zb[k + NB] : 0.f;
+                }
+                tc::tmem_st16(tl + RC_G + tb * 16, bnd);
+            }
+            // rows 64 .. 64+BW-2 end the chunk in registers; samples beyond are zero
+#pragma unroll
+            for (int k = 0; k < BW - 1; ++k) za[CH + k] = zb[k];
+            tc::tmem_wait_st();
+            float zr[NR];
+#pragma unroll
+            for (int q4 = 0; q4 < NR / 4; ++q4) {
+                const float4 z4 = *reinterpret_cast<const float4 *>(za + q4 * 4);
+                zr[q4 * 4] = z4.x; zr[q4 * 4 + 1] = z4.y; zr[q4 * 4 + 2] = z4.z; zr[q4 * 4 + 3] = z4.w;
+            }
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8)
+                *reinterpret_cast<uint4 *>(sm + R_ZT0 + tc::sw128(rw, c8)) = pack8(&zr[c8 * 8]);
+#pragma unroll
+            for (int c8 = 0; c8 < 2; ++c8)
+                *reinterpret_cast<uint4 *>(sm + R_ZT1 + tc::sw128(rw, c8)) = pack8(&zr[64 + c8 * 8]);
+        }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == ISSUER) {
+            tc::fence_after_sync();
+            issue_k(tbase + RC_DS, sbase + R_ZT0, sbase + R_XT0, DD, sbase + R_ZT1, sbase + R_XT1, 1);  // Zt^T X
+            issue_k(tbase + RC_I, sbase + R_ZT0, sbase + R_PM0, CH, sbase + R_ZT1, sbase + R_PM1, 1);   // Zt^T (P o m)^T
+            tc::mma_commit(bar);
+        }
+        ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
+        phase ^= 1;
+        ok = __syncthreads_and(ok);
+        if (ok) {
+            tc::fence_after_sync();
+            // ---- the image, every thread one row (0-127) and half of the tokens
+            //      and columns: value rows give O0^T and B, identity rows Qt and
+            //      T - g_C I (transposed as they are stored)
+            const bool vrow = row < DD;
+            const int cc = row - DD;
+            const float ig = __expf(-GC);
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int t0 = chalf * 32 + k2 * 16;
+                float iv[16], bv[16], o[16];
+                tc::tmem_ld16(tl + RC_I + t0, iv);
+                tc::tmem_ld16(tl + RC_G + t0, bv);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int t = t0 + i;
+                    const float sq = vrow ? 0.f : tile_get(sm, R_Q, t, cc);
+                    o[i] = t < nt ? __expf(vG[t]) * fmaf(ig, iv[i] + bv[i], sq) : 0.f;
+                }
+                if (vrow) {
+                    *reinterpret_cast<uint4 *>(stg + 2 * TILE + rowmajor8(row, t0 >> 3)) = pack8(&o[0]);
+                    *reinterpret_cast<uint4 *>(stg + 2 * TILE + rowmajor8(row, (t0 >> 3) + 1)) = pack8(&o[8]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        *reinterpret_cast<__nv_bfloat16 *>(stg + TILE + tc::sw128(t0 + i, cc >> 3) + (uint32_t)(cc & 7) * 2) =
+                            __float2bfloat16_rn(o[i]);
+                }
+            }
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int i0 = chalf * 32 + k2 * 16;
+                float dv[16];
+                tc::tmem_ld16(tl + RC_DS + i0, dv);
+                tc::tmem_wait_ld();
+                if (vrow) {
+                    *reinterpret_cast<uint4 *>(stg + 3 * TILE + rowmajor8(row, i0 >> 3)) = pack8(&dv[0]);
+                    *reinterpret_cast<uint4 *>(stg + 3 * TILE + rowmajor8(row, (i0 >> 3) + 1)) = pack8(&dv[8]);
+                } else {
+                    // (T - g_C I)[c][i] = (Zt^T X)[64 + c][i], stored at row i, column c
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        *reinterpret_cast<__nv_bfloat16 *>(stg + tc::sw128(i0 + i, cc >> 3) + (uint32_t)(cc & 7) * 2) =
+                            __float2bfloat16_rn(dv[i]);
+                }
+            }
+        }
+    } else if (ok) {
+        // ---- a chunk whose decay leaves the fp32 range of the factorised form:
+        //      the recurrence token by token on the 128 rows, R_t = alpha_t R_{t-1}
+        //      + eta_t sum_m (y_{t+m} - R_{t-1} x_{t+m}) x_{t+m}^T (values zero on
+        //      the identity rows), o_t = R_t q_t; thread (row, 32 columns), partial
+        //      dot products meeting in `red`, the outputs in fp32 over Zacc
+        float *outb = Za;  // [row][t]
+        for (int e = tid; e < 2 * DD * CH; e += NTH) outb[e] = 0.f;
+        float S[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) S[e] = (row >= DD && chalf * 32 + e == row - DD) ? 1.f : 0.f;
+        __syncthreads();
+        for (int t = 0; t < nt; ++t) {
+            float xm[BW][32];
+#pragma unroll
+            for (int m = 0; m < BW; ++m) {
+                float part = 0.f;
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + R_XE + tc::sw128(t + m, chalf * 4 + c8)), &xm[m][c8 * 8]);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) part = fmaf(S[c8 * 8 + i], xm[m][c8 * 8 + i], part);
+                }
+                red[(chalf * 4 + m) * 2 * DD + row] = part;
+            }
+            __syncthreads();
+            {
+                float e[BW];
+#pragma unroll
+                for (int m = 0; m < BW; ++m) {
+                    const float sxm = red[m * 2 * DD + row] + red[(4 + m) * 2 * DD + row];
+                    const float y = row < DD ? tile_get(sm, R_VE, t + m, row) : 0.f;
+                    e[m] = y - sxm;
+                }
+                const float eta = veta[t], alpha = valpha[t];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float u2 = 0.f;
+#pragma unroll
+                    for (int m = 0; m < BW; ++m) u2 = fmaf(e[m], xm[m][i], u2);
+                    S[i] = fmaf(alpha, S[i], eta * u2);
+                }
+            }
+            __syncthreads();
+            {
+                float part = 0.f;
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    float q8[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + R_Q + tc::sw128(t, chalf * 4 + c8)), q8);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) part = fmaf(S[c8 * 8 + i], q8[i], part);
+                }
+                red[(chalf * 4) * 2 * DD + row] = part;
+            }
+            __syncthreads();
+            if (chalf == 0) outb[row * CH + t] = red[row] + red[4 * 2 * DD + row];
+            __syncthreads();
+        }
+        // the image over the consumed sample tiles
+        const bool vrow = row < DD;
+        const int cc = row - DD;
+        const float g = __expf(GC);
+        if (vrow) {
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+                // B row j, columns 32 chalf .. ; O0^T row j, tokens 32 chalf ..
+                *reinterpret_cast<uint4 *>(stg + 3 * TILE + rowmajor8(row, chalf * 4 + g8)) = pack8(&S[g8 * 8]);
+                *reinterpret_cast<uint4 *>(stg + 2 * TILE + rowmajor8(row, chalf * 4 + g8)) =
+                    pack8(&outb[row * CH + chalf * 32 + g8 * 8]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int col = chalf * 32 + i;  // (T - g_C I)[c][col] at row col, column c
+                *reinterpret_cast<__nv_bfloat16 *>(stg + tc::sw128(col, cc >> 3) + (uint32_t)(cc & 7) * 2) =
+                    __float2bfloat16_rn(S[i] - (col == cc ? g : 0.f));
+                const int t = chalf * 32 + i;    // Qt[t][c] = (T_t q_t)[c]
+                *reinterpret_cast<__nv_bfloat16 *>(stg + TILE + tc::sw128(t, cc >> 3) + (uint32_t)(cc & 7) * 2) =
+                    __float2bfloat16_rn(outb[row * CH + t]);
+            }
+        }
+    }
+    if (!ok) break;
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+        gc_ws[u] = __expf(GC);
+        tc::bulk_store(img_ws + (size_t)u * IMG, sbase + R_XE, IMG);
+        tc::bulk_commit();
+    }
+    }  // units
+    if (tid == 0) {
+        tc::bulk_wait_all();
+        if (!ok) {
+            atomicAdd(&g_w_wait_timeouts, 1u);
+            // every load issued must land before the block leaves
+            for (int k = max(0, loads - 2); k < loads; ++k)
+                (void)tc::mbar_wait_timeout(&tbar[k & 1], (uint32_t)((k >> 1) & 1), kWaitNs);
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 512);
+}
+
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -1059,7 +1581,20 @@ int launch_w(const FwdParams &p, const WMaps &maps, cudaStream_t s) {
     return cudaGetLastError() == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
 }
 
-// Falcon-3A: the per-chunk images, then the chain kernel of the split path
+int w_sm_count() {
+    static int counts[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (counts[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
+// Falcon-3 / Falcon-3A: the per-chunk images, then the chain kernel of the split path
 template <int BW>
 int launch_wl(const FwdParams &p, const WMaps &maps, cudaStream_t s) {
     const size_t units = (size_t)p.B * p.H * ((p.L + CH - 1) / CH);
@@ -1074,9 +1609,14 @@ int launch_wl(const FwdParams &p, const WMaps &maps, cudaStream_t s) {
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
         cudaFuncSetAttribute(w_local_kernel<BW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)U_SMEM);
+        cudaFuncSetAttribute(w_reg_local_kernel<BW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)R_SMEM);
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    w_local_kernel<BW><<<(unsigned)units, NTH, U_SMEM, s>>>(p, maps, img, gc);
+    if (p.variant == F3)  // persistent: one block per SM
+        w_reg_local_kernel<BW><<<(unsigned)std::min<size_t>(units, (size_t)w_sm_count()), NTH, R_SMEM, s>>>(p, maps,
+                                                                                                       img, gc);
+    else
+        w_local_kernel<BW><<<(unsigned)units, NTH, U_SMEM, s>>>(p, maps, img, gc);
     int rc = cudaGetLastError() == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
     if (rc == 0) rc = launch_chain_images(p, img, gc, s);
     ws_release(ws, owned, s);
@@ -1086,7 +1626,7 @@ int launch_wl(const FwdParams &p, const WMaps &maps, cudaStream_t s) {
 }  // namespace
 
 bool w_local_covers(const FwdParams &p) {
-    if (!(p.variant == F3A && p.dk == DD && p.dv == DD && p.chunk == CH && p.window >= 2 && p.window <= 4))
+    if (!((p.variant == F3 || p.variant == F3A) && p.dk == DD && p.dv == DD && p.chunk == CH && p.window >= 2 && p.window <= 4))
         return false;
     return (size_t)p.B * p.H * ((p.L + CH - 1) / CH) <= 0x7fffffffu;
 }

@@ -41,13 +41,13 @@ unsigned int pc_wait_timeouts();
 // (one block per head, per-channel forward substitution); returns 1 for
 // shapes it does not cover.
 int launch_f2_chunk(const FwdParams &p, cudaStream_t s);
-// Falcon-3A (bf16, d = 64, chunk 64, window 2-4): per-chunk images, then the
-// split path's chain kernel on them
+// Falcon-3 / Falcon-3A (bf16, d = 64, chunk 64, window 2-4): per-chunk
+// images, then the split path's chain kernel on them
 bool w_local_covers(const FwdParams &p);
 size_t w_local_ws_bytes(const FwdParams &p);
-// the chain kernel of the split path over per-chunk images [unused | Qt |
-// O0^T | B] (32 KB each, per (b*H + h, chunk)) and g_C, in stream order
-// after the kernel that wrote them (inner-product family)
+// the chain kernel of the split path over per-chunk images [-Phi'^T (the
+// regression family) | Qt | O0^T | B] (32 KB each, per (b*H + h, chunk)) and
+// g_C, in stream order after the kernel that wrote them
 int launch_chain_images(const FwdParams &p, const uint8_t *img, const float *gc, cudaStream_t s);
 unsigned int f2_wait_timeouts();
 // bf16 Falcon-3/3A chunk-parallel forward, d_k = d_v = 64, chunk 64, window

@@ -50,9 +50,9 @@ def test_host_chunk_falcon1_pair(F, slices):
 
 @pytest.mark.parametrize("slices", [0, 3])
 def test_host_chunk_falcon3_pair_window(F, slices):
-    """Falcon-3 (one block per head) and Falcon-3A (per-chunk images and the
-    chain kernel, in the workspace the host call sizes) from one set of host
-    inputs, window 4, B = 4 in 1 or 3 slices."""
+    """Falcon-3 and Falcon-3A (per-chunk images and the chain kernel, in the
+    workspace the host call sizes) from one set of host inputs, window 4,
+    B = 4 in 1 or 3 slices."""
     d = gen.draw("F3", 4, 3, 150, 64, 64, seed=302, dtype="bf16")
     outs, states = on_host(F, ["F3", "F3A"], "chunk", d, chunk=64, window=4, slices=slices)
     for i, var in enumerate(["F3", "F3A"]):

@@ -553,10 +553,11 @@ def test_falcon2_d128_one_block_per_head(F, lam, key_scale, phi):
 @pytest.mark.parametrize("variant", ["F3", "F3A"])
 @pytest.mark.parametrize("L", [1, 5, 64, 65, 200])
 def test_window_tensor_core_path(F, variant, w, L):
-    """bf16 Falcon-3/3A, d_k = d_v = 64, chunk 64: Falcon-3 one block per
-    head with the windowed system in token order, Falcon-3A one block per
-    (head, chunk) writing images for the chain kernel; the products on
-    tcgen05; one chunk and a ragged tail over several chunks."""
+    """bf16 Falcon-3/3A, d_k = d_v = 64, chunk 64: per-chunk images written
+    for the chain kernel (Falcon-3: the windowed system walked for the value
+    channels and the rows of the identity, Falcon-3A: for the value channels
+    alone); the products on tcgen05; one chunk and a ragged tail over several
+    chunks."""
     d = gen.draw(variant, 2, 3, L, 64, 64, seed=100 + 10 * w + L, dtype="bf16")
     check(F, d, variant, "chunk", chunk=64, window=w)
 
@@ -573,9 +574,10 @@ def test_window_tensor_core_strong_forgetting(F, variant):
 @pytest.mark.parametrize("variant", ["F3", "F3A"])
 def test_window_tensor_core_decay_floor(F, variant, w):
     """Tiny keys under the identity map with lambda = 0.9: alpha on the 2^-20
-    floor, chunk log-decays far below -80; those chunks run token by token
-    (Falcon-3), or sum their intra-chunk outputs with one exponential per
-    term (Falcon-3A)."""
+    floor, chunk log-decays far below -80; those chunks run the recurrence
+    token by token on the value channels and the identity rows (Falcon-3),
+    or sum their intra-chunk outputs with one exponential per term
+    (Falcon-3A)."""
     d = gen.draw(variant, 1, 2, 150, 64, 64, seed=132 + w, dtype="bf16", lam=0.9, key_scale=0.03)
     check(F, d, variant, "chunk", chunk=64, window=w, phi="identity")
 
