@@ -22,14 +22,15 @@
 //   o_t   = e^{G_t} ((S_0 Q^T)[j][t] + e^{-G_C} (sum_{r<=t} P[t][r] Zt[r]
 //                                             + sum_{k=1}^{B_w-1} P[t][t+k] Zacc_{t+1}[t+k])),
 // P = Q X^T.  Every coefficient stays inside the fp32 range while G_C > -80;
-// a chunk below that runs its tokens one by one (the recurrence itself, S in
-// registers).
+// a chunk below that runs its tokens one by one (the recurrence itself).
 //
-// Falcon-3: one block per (b, h) walks the chunks (w_chunk_kernel); S stays
-// in fp32 registers (thread: row j, 32 columns) with its bf16 copy as the
-// operand of S_0 X^T and S_0 Q^T.  Falcon-3A has no state in its increments:
-// w_local_kernel forms every (head, chunk) unit's image at once and the
-// chain kernel of the split Falcon-1A path walks the chunks (below).
+// Both variants form every (head, chunk) unit's effect on the state at once
+// and hand it, as a per-chunk image, to the chain kernel of the split
+// Falcon-1/1A path, which walks the chunks of each head: w_reg_local_kernel
+// (Falcon-3) solves the system for the value channels with S_0 = 0 and for
+// the rows of the identity with zero values, giving O0, B, Qt and the
+// transition; w_local_kernel (Falcon-3A, no state in its increments) walks
+// the value channels alone.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -55,61 +56,13 @@ constexpr float kMinLogDecay = -80.f;
 
 __device__ unsigned int g_w_wait_timeouts;
 
-#ifdef FALCON_TC_DEBUG
-// block 0, thread 0: SM cycles per phase summed over the chunks
-__device__ long long *g_w_tim;
-#define WT_INIT()                    \
-    long long wt_acc_[8] = {0};      \
-    long long wt_prev_ = clock64();  \
-    const bool wt_on_ = blockIdx.x == 0 && threadIdx.x == 0
-#define WT(k)                                  \
-    do {                                       \
-        if (wt_on_) {                          \
-            const long long n_ = clock64();    \
-            wt_acc_[k] += n_ - wt_prev_;       \
-            wt_prev_ = n_;                     \
-        }                                      \
-    } while (0)
-#define WT_END()                                                         \
-    do {                                                                 \
-        if (wt_on_ && g_w_tim)                                           \
-            for (int i_ = 0; i_ < 8; ++i_) g_w_tim[i_] = wt_acc_[i_];     \
-    } while (0)
-#else
-#define WT_INIT()
-#define WT(k)
-#define WT_END()
-#endif
 
-// shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t W_XE = 0;            // sample rows x_r (128 rows; rows >= 64+B_w-1 zero up to NR)
-constexpr uint32_t W_VE = 2 * TILE;     // sample rows y_r (128 rows)
-constexpr uint32_t W_Q = 4 * TILE;      // q rows t (64 rows; the next 64 are only read as unused A rows)
-constexpr uint32_t W_S = 6 * TILE;      // bf16 S_0 rows j (64 rows), then 64 zero rows
-constexpr uint32_t W_XT0 = 8 * TILE;    // X^T: rows c, samples 0-63
-constexpr uint32_t W_XT1 = 9 * TILE;    // X^T: rows c, samples 64-79 (two 16-byte chunks per row)
-constexpr uint32_t W_ZT0 = 10 * TILE;   // Zt^T: rows j, samples 0-63 (128 rows, 64-127 zero)
-constexpr uint32_t W_ZT1 = 12 * TILE;   // Zt^T: rows j, samples 64-79
-constexpr uint32_t W_PM0 = 14 * TILE;   // P o (r <= t): rows t, samples 0-63
-constexpr uint32_t W_PM1 = 15 * TILE;   // rows t, samples 64-79
 constexpr int LDA = 68;                 // fp32 Gram rows (samples 0-67)
-constexpr int LDZ = 84;                 // fp32 per-channel rows: conflict-free float4 along the channel
-constexpr uint32_t W_A = 16 * TILE;                         // fp32 A[r][r'], r < 68
-constexpr uint32_t W_SX = W_A + 68 * LDA * 4;              // fp32 (S_0 X^T)[j][r]
-constexpr uint32_t W_ZA = W_SX + DD * LDZ * 4;              // fp32 Zacc[j][r]
-constexpr uint32_t W_VEC = W_ZA + DD * LDZ * 4;             // scalars
-// vec: sqn[80] beta[64] eta[64] alpha[64] G[64] w[64] kappa[64] gm1[64] pband[64*4] red[2*4*64] misc[16]
+constexpr int LDZ = 84;                 // fp32 per-row sums: conflict-free float4 along the row
+// per-token scalars (floats): sqn[80] beta[64] eta[64] alpha[64] G[64] w[64]
+// kappa[64] gm1[64] pband[64*4], then red and misc (each kernel's own size)
 constexpr int V_SQN = 0, V_BETA = 80, V_ETA = 144, V_ALPHA = 208, V_G = 272, V_W = 336, V_KAP = 400,
               V_GM1 = 464, V_PB = 528, V_RED = 784, V_MISC = 1296, V_END = 1312;
-constexpr uint32_t W_BAR = W_VEC + V_END * 4;
-constexpr uint32_t W_SMEM = W_BAR + 64 + 1024;
-// tensor memory (512 columns)
-constexpr uint32_t C_G = 0;      // Gram: lanes r, columns r' (80); then the band terms, lanes j, columns t
-constexpr uint32_t C_P = 96;     // P: lanes t, columns r (80)
-constexpr uint32_t C_SX = 192;   // S_0 X^T: lanes j, columns r (80)
-constexpr uint32_t C_SQ = 288;   // S_0 Q^T: lanes j, columns t (64)
-constexpr uint32_t C_DS = 352;   // Zt^T X: lanes j, columns c (64)
-constexpr uint32_t C_I = 416;    // Zt^T (P o mask)^T: lanes j, columns t (64)
 
 __device__ __forceinline__ uint4 pack8(const float *f) {
     __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]);
@@ -172,488 +125,6 @@ struct WMaps {
 };
 
 }  // namespace
-
-template <int BW>
-__global__ void __launch_bounds__(NTH, 1) w_chunk_kernel(FwdParams p, const __grid_constant__ WMaps maps) {
-    constexpr int MM = CH + BW - 1;  // sample rows of a chunk
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_s = tc::smem_u32(smem_raw);
-    uint8_t *sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
-    const uint32_t sbase = tc::smem_u32(sm);
-    float *At = reinterpret_cast<float *>(sm + W_A);
-    float *SXt = reinterpret_cast<float *>(sm + W_SX);
-    float *Za = reinterpret_cast<float *>(sm + W_ZA);
-    float *vec = reinterpret_cast<float *>(sm + W_VEC);
-    float *sqn = vec + V_SQN, *vbeta = vec + V_BETA, *veta = vec + V_ETA, *valpha = vec + V_ALPHA, *vG = vec + V_G,
-          *vw = vec + V_W, *vkap = vec + V_KAP, *vgm1 = vec + V_GM1, *pband = vec + V_PB, *red = vec + V_RED,
-          *misc = vec + V_MISC;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + W_BAR);
-    uint64_t *tbar = bar + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quarter = warp & 3, chalf = warp >> 2, row = quarter * 32 + lane;
-    const int bh = blockIdx.x, L = p.L, nch = (L + CH - 1) / CH;
-    const float lam = p.lambda[bh % p.H];
-    const bool reg = p.variant == F3;
-    const __nv_bfloat16 *betap = static_cast<const __nv_bfloat16 *>(p.beta) + (size_t)bh * L;
-
-    // sample row r of chunk c holds sample i = c0 - BW + 1 + r: key row i-1
-    // (prefix pair) or i (same-step pair), value row i
-    auto load_chunk = [&](int c) {
-        const int c0 = c * CH, r0 = c0 - BW + 1, krow = p.pairing == 0 ? r0 - 1 : r0;
-        tc::mbar_arrive_expect_tx(tbar, 5 * TILE);
-        tc::tma_load_3d(sbase + W_XE, &maps.k, 0, krow, bh, tbar);
-        tc::tma_load_3d(sbase + W_XE + TILE, &maps.k, 0, krow + 64, bh, tbar);
-        tc::tma_load_3d(sbase + W_VE, &maps.v, 0, r0, bh, tbar);
-        tc::tma_load_3d(sbase + W_VE + TILE, &maps.v, 0, r0 + 64, bh, tbar);
-        tc::tma_load_3d(sbase + W_Q, &maps.q, 0, c0, bh, tbar);
-    };
-    int issued = 0;
-    if (tid == 0) {
-        tc::mbar_init(bar, 1);
-        tc::mbar_init(tbar, 1);
-        tc::fence_mbar_init();
-        if (nch > 0) {
-            load_chunk(0);
-            issued = 1;
-        }
-    }
-    __syncwarp();
-    if (warp == 0) {
-        tc::tmem_alloc(tmem_slot, 512);
-        tc::tmem_relinquish();
-    }
-    // zero rows that only pad the 128-row operands: S rows 64-127, Zt^T rows 64-127
-    for (int e = tid; e < 4 * TILE / 16; e += NTH) {
-        const int part = e / (TILE / 16), o = e % (TILE / 16);
-        const uint32_t base = part == 0 ? W_S + TILE : part == 1 ? W_ZT0 + TILE : part == 2 ? W_ZT1 + TILE : W_XT1;
-        *reinterpret_cast<uint4 *>(sm + base + o * 16) = make_uint4(0, 0, 0, 0);
-    }
-    // S in fp32 registers: warps 0,1,4,5, thread = (row j, 32 columns)
-    const bool sthr = quarter < 2;
-    float S[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-        S[e] = (sthr && p.init_state) ? p.init_state[((size_t)bh * DD + row) * DD + chalf * 32 + e] : 0.f;
-    if (sthr) {
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8)
-            *reinterpret_cast<uint4 *>(sm + W_S + tc::sw128(row, chalf * 4 + c8)) = pack8(&S[c8 * 8]);
-    }
-    float beta_next = 0.f;
-    if (tid < CH && nch > 0) beta_next = tid < L ? __bfloat162float(betap[tid]) : 0.f;
-    tc::fence_proxy_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tbase = *tmem_slot;
-    const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
-
-    bool ok = true;
-    uint32_t phase = 0;
-    WT_INIT();
-    for (int c = 0; c < nch; ++c) {
-        const int c0 = c * CH, nt = min(CH, L - c0);
-        if (tid < CH) {
-            vbeta[tid] = beta_next;
-            beta_next = (c + 1 < nch && c0 + CH + tid < L) ? __bfloat162float(betap[c0 + CH + tid]) : 0.f;
-        }
-        ok = tc::mbar_wait_timeout(tbar, (uint32_t)(c & 1), kWaitNs);
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
-        WT(0);
-        // ---- samples: rows r < MM normalised in place (four threads per row), rows MM..NR-1 zero
-        for (int rr = tid >> 2; rr < NR; rr += NTH / 4) {  // a warp's lanes share the trip count
-            const int part = tid & 3, i = c0 - BW + 1 + rr;
-            float xr[16];
-            bool given = false;  // a carried sample, used as given
-#pragma unroll
-            for (int e = 0; e < 16; ++e) xr[e] = 0.f;
-            if (rr < MM) {
-                // a continued segment: sample 0 (prefix pair) is the carried phi(k); samples
-                // before it come from the carried window, values included
-                const bool cx = i == 0 && p.pairing == 0 && p.x_prev != nullptr;
-                const float *cw = (i < 0 && i >= -(BW - 1) && p.win)
-                                      ? p.win + ((size_t)bh * (BW - 1) + (i + BW - 1)) * (DD + DD)
-                                      : nullptr;
-                given = cx || cw;
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const int cc = part * 16 + h2 * 8;
-                    if (cx) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) xr[h2 * 8 + e] = p.x_prev[(size_t)bh * DD + cc + e];
-                    } else if (cw) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) xr[h2 * 8 + e] = cw[cc + e];
-                    } else {
-                        unpack8(*reinterpret_cast<const uint4 *>(sm + W_XE + tc::sw128(rr, part * 2 + h2)), &xr[h2 * 8]);
-                    }
-                }
-                if (cw) {
-                    float yv[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) yv[e] = cw[DD + part * 16 + e];
-                    *reinterpret_cast<uint4 *>(sm + W_VE + tc::sw128(rr, part * 2)) = pack8(&yv[0]);
-                    *reinterpret_cast<uint4 *>(sm + W_VE + tc::sw128(rr, part * 2 + 1)) = pack8(&yv[8]);
-                }
-            }
-            float ss = 0.f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) ss += xr[e] * xr[e];
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-            const float inv = (given || p.phi != 0) ? 1.f : (ss > 0.f ? rsqrtf(ss) : 0.f);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) xr[e] *= inv;
-            if (part == 0) sqn[rr] = ss * inv * inv;
-            *reinterpret_cast<uint4 *>(sm + W_XE + tc::sw128(rr, part * 2)) = pack8(&xr[0]);
-            *reinterpret_cast<uint4 *>(sm + W_XE + tc::sw128(rr, part * 2 + 1)) = pack8(&xr[8]);
-        }
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
-        __syncthreads();
-        WT(1);
-        // ---- products: Gram and P over the sample rows, S_0 X^T, S_0 Q^T
-        if (tid == ISSUER) {
-            tc::fence_after_sync();
-            issue_k(tbase + C_G, sbase + W_XE, sbase + W_XE, NR);
-            issue_k(tbase + C_P, sbase + W_Q, sbase + W_XE, NR);
-            issue_k(tbase + C_SX, sbase + W_S, sbase + W_XE, NR);
-            issue_k(tbase + C_SQ, sbase + W_S, sbase + W_Q, CH);
-            tc::mma_commit(bar);
-        }
-        // ---- per-token steps and decays (warps 0-1), X^T (warps 2-7)
-        if (tid < CH) {
-            const int t = tid;
-            float n = 0.f;
-#pragma unroll
-            for (int m = 0; m < BW; ++m) n += sqn[t + m];
-            float eta, alpha;
-            step_and_decay(vbeta[t], n, p.eps, lam, eta, alpha);
-            const float la = __logf(alpha);
-            float run = la;  // inclusive sum over the warp
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, run, o);
-                if (lane >= o) run += y;
-            }
-            if (lane == 31) misc[warp] = run;
-            veta[t] = eta;
-            valpha[t] = alpha;
-            vG[t] = run;  // warp-local; warp 1 adds warp 0's total below
-        } else {
-            // X^T: 10 source row blocks x 2 chunk groups over warps 2-7
-            for (int g = warp - 2; g < 20; g += 6) {
-                const int srb = g >> 1, cb0 = (g & 1) * 4;
-                transpose_blk(sbase + W_XE, srb, cb0, srb < 8 ? sbase + W_XT0 : sbase + W_XT1, srb & 7);
-            }
-        }
-        __syncthreads();
-        if (tid < CH) {
-            const int t = tid;
-            const float G = vG[t] + (t >= 32 ? misc[0] : 0.f);
-            const float GC = misc[0] + misc[1];
-            const float Gm = G - __logf(valpha[t]);  // G_{t-1}
-            const float eta = veta[t];
-            vw[t] = __expf(GC - G) * eta;
-            vkap[t] = __fdividef(eta, valpha[t]);
-            vgm1[t] = __expf(Gm);
-            __syncwarp();
-            vG[t] = G;
-            if (t == 0) misc[2] = GC;
-        }
-        __syncthreads();
-        const float GC = misc[2];
-        const bool unsafe = !(GC > kMinLogDecay);
-        WT(2);
-        ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
-        phase ^= 1;
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
-        WT(3);
-        tc::fence_after_sync();
-        if (!unsafe) {
-            // ---- Gram rows r < 68 (lanes 0-79) -> fp32; P (lanes 0-63) -> P o (r <= t) bf16 and the band
-            if (quarter < 3) {
-                const int r = row;
-                for (int g = chalf; g < 5; g += 2) {
-                    float v[16];
-                    tc::tmem_ld16(tl + C_G + g * 16, v);
-                    tc::tmem_wait_ld();
-                    if (r < LDA) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (g * 16 + i < LDA) At[r * LDA + g * 16 + i] = v[i];
-                    }
-                }
-            }
-            if (quarter < 2) {
-                const int t = row;
-                for (int g = chalf; g < 5; g += 2) {
-                    float v[16];
-                    tc::tmem_ld16(tl + C_P + g * 16, v);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int r = g * 16 + i, k = r - t;
-                        if (k >= 1 && k < BW) pband[t * 4 + k] = v[i];
-                        v[i] = r <= t ? v[i] : 0.f;
-                    }
-                    const uint32_t dst = g < 4 ? W_PM0 : W_PM1;
-                    const int ch0 = g < 4 ? g * 2 : 0;
-                    *reinterpret_cast<uint4 *>(sm + dst + tc::sw128(t, ch0)) = pack8(&v[0]);
-                    *reinterpret_cast<uint4 *>(sm + dst + tc::sw128(t, ch0 + 1)) = pack8(&v[8]);
-                }
-            }
-            // S_0 X^T rows j -> fp32 (the solving threads' own rows)
-            if (tid < DD) {
-#pragma unroll
-                for (int g = 0; g < 5; ++g) {
-                    float v[16];
-                    tc::tmem_ld16(tl + C_SX + g * 16, v);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        *reinterpret_cast<float4 *>(SXt + tid * LDZ + g * 16 + q4 * 4) =
-                            make_float4(v[q4 * 4], v[q4 * 4 + 1], v[q4 * 4 + 2], v[q4 * 4 + 3]);
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < NR / 4; ++q4)
-                    *reinterpret_cast<float4 *>(Za + tid * LDZ + q4 * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            tc::fence_proxy_async();
-            tc::fence_before_sync();
-            __syncthreads();
-            WT(4);
-            tc::fence_after_sync();
-            // ---- the chunk's system in token order (warps 0-1: thread = channel j = lane),
-            //      in blocks of 8 tokens: the sums over rows final before a block are one
-            //      batch of independent dot products; only the rows the block itself
-            //      still adds to (t0 .. t0+7+BW-1, in registers) are walked token by token
-            if (tid < DD) {
-                const int j = tid;
-                float *za = Za + j * LDZ;
-                const float *sx = SXt + j * LDZ;
-                constexpr int NB = 8, RB = NB + BW - 1;  // tokens and rows of a block
-                float zb[RB];                            // rows t0 .. t0+RB-1
-#pragma unroll
-                for (int k = 0; k < RB; ++k) zb[k] = 0.f;
-#pragma unroll 1
-                for (int tb = 0; tb < 4; ++tb) {
-                    float bnd[16];
-#pragma unroll
-                    for (int hb = 0; hb < 2; ++hb) {
-                        const int t0 = tb * 16 + hb * NB;
-                        // rows r' < t0 are final (in shared memory): the sum over them
-                        // of A[t+m][r'] Zacc[r'] depends on t+m only, one sum per row
-                        float crr[RB];
-#pragma unroll
-                        for (int rr = 0; rr < RB; ++rr) crr[rr] = 0.f;
-                        if (reg) {
-                            for (int q = 0; q < (t0 >> 2); ++q) {
-                                const float4 z4 = *reinterpret_cast<const float4 *>(za + q * 4);
-#pragma unroll
-                                for (int rr = 0; rr < RB; ++rr) {
-                                    const float4 a4 = *reinterpret_cast<const float4 *>(At + (t0 + rr) * LDA + q * 4);
-                                    crr[rr] = fmaf(a4.x, z4.x, fmaf(a4.y, z4.y, fmaf(a4.z, z4.z, fmaf(a4.w, z4.w, crr[rr]))));
-                                }
-                            }
-                        }
-                        float cr[NB][BW];
-#pragma unroll
-                        for (int i = 0; i < NB; ++i)
-#pragma unroll
-                            for (int m = 0; m < BW; ++m) cr[i][m] = crr[i + m];
-#pragma unroll
-                        for (int i = 0; i < NB; ++i) {
-                            const int t = t0 + i;
-                            const float wt = vw[t], gm = vgm1[t], kt = vkap[t];
-#pragma unroll
-                            for (int m = 0; m < BW; ++m) {
-                                float acc = cr[i][m];
-                                if (reg) {
-                                    // rows t0 .. t+BW-2 still accumulating: registers
-#pragma unroll
-                                    for (int k = 0; k < i + BW - 1; ++k)
-                                        acc = fmaf(At[(t + m) * LDA + t0 + k], zb[k], acc);
-                                }
-                                const int r = t + m;
-                                const float y = tile_get(sm, W_VE, r, j);
-                                cr[i][m] = reg ? wt * (y - gm * sx[r]) - kt * acc : wt * y;
-                            }
-                            // z_{t,m} lands on row t+m only after every slot of token t used the old sums
-#pragma unroll
-                            for (int m = 0; m < BW; ++m) zb[i + m] += cr[i][m];
-                            float bsum = 0.f;
-#pragma unroll
-                            for (int k = 1; k < BW; ++k) bsum = fmaf(pband[t * 4 + k], zb[i + k], bsum);
-                            bnd[hb * NB + i] = bsum;
-                        }
-                        // rows t0 .. t0+7 are final; rows t0+8 .. carry into the next block
-#pragma unroll
-                        for (int k = 0; k < NB; ++k) za[t0 + k] = zb[k];
-#pragma unroll
-                        for (int k = 0; k < RB; ++k) zb[k] = k + NB < RB ? zb[k + NB] : 0.f;
-                    }
-                    tc::tmem_st16(tl + C_G + tb * 16, bnd);
-                }
-                // rows 64 .. 64+BW-2 end the chunk in registers
-#pragma unroll
-                for (int k = 0; k < BW - 1; ++k) za[CH + k] = zb[k];
-                tc::tmem_wait_st();
-                // Zt^T row j
-                float zr[NR];
-#pragma unroll
-                for (int q4 = 0; q4 < NR / 4; ++q4) {
-                    const float4 z4 = *reinterpret_cast<const float4 *>(za + q4 * 4);
-                    zr[q4 * 4] = z4.x; zr[q4 * 4 + 1] = z4.y; zr[q4 * 4 + 2] = z4.z; zr[q4 * 4 + 3] = z4.w;
-                }
-#pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8)
-                    *reinterpret_cast<uint4 *>(sm + W_ZT0 + tc::sw128(j, c8)) = pack8(&zr[c8 * 8]);
-#pragma unroll
-                for (int c8 = 0; c8 < 2; ++c8)
-                    *reinterpret_cast<uint4 *>(sm + W_ZT1 + tc::sw128(j, c8)) = pack8(&zr[64 + c8 * 8]);
-            }
-            tc::fence_proxy_async();
-            tc::fence_before_sync();
-            __syncthreads();
-            WT(5);
-            if (tid == 0 && c + 1 < nch) {
-                load_chunk(c + 1);
-                ++issued;
-            }
-            if (tid == ISSUER) {
-                tc::fence_after_sync();
-                issue_k(tbase + C_DS, sbase + W_ZT0, sbase + W_XT0, DD, sbase + W_ZT1, sbase + W_XT1, 1);  // Zt^T X
-                issue_k(tbase + C_I, sbase + W_ZT0, sbase + W_PM0, CH, sbase + W_ZT1, sbase + W_PM1, 1);   // Zt^T (P o m)^T
-                tc::mma_commit(bar);
-            }
-            ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
-            phase ^= 1;
-            ok = __syncthreads_and(ok);
-            if (!ok) break;
-            WT(6);
-            tc::fence_after_sync();
-            if (sthr) {
-                const int j = row;
-                const float ig = __expf(-GC);
-                // o_t[j] for t in 32 chalf .. 32 chalf + 31
-#pragma unroll
-                for (int k2 = 0; k2 < 2; ++k2) {
-                    const int t0 = chalf * 32 + k2 * 16;
-                    float sq[16], iv[16], bv[16];
-                    tc::tmem_ld16(tl + C_SQ + t0, sq);
-                    tc::tmem_ld16(tl + C_I + t0, iv);
-                    tc::tmem_ld16(tl + C_G + t0, bv);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int t = t0 + i;
-                        const float o = __expf(vG[t]) * fmaf(ig, iv[i] + bv[i], sq[i]);
-                        if (t < nt)
-                            static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + j] =
-                                __float2bfloat16_rn(o);
-                    }
-                }
-                // S_end = e^{G_C} S_0 + Zt^T X
-                const float g = __expf(GC);
-#pragma unroll
-                for (int k2 = 0; k2 < 2; ++k2) {
-                    float dv[16];
-                    tc::tmem_ld16(tl + C_DS + chalf * 32 + k2 * 16, dv);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) S[k2 * 16 + i] = fmaf(g, S[k2 * 16 + i], dv[i]);
-                }
-            }
-        } else {
-            // ---- a chunk whose decay leaves the fp32 range of the factorised form:
-            //      its tokens one by one, S_t = alpha_t S_{t-1} + eta_t sum_m e_{t,m} x^T, o_t = S_t q_t
-            //      (thread (j, 32 columns) of warps 0,1,4,5; partial dot products meet in `red`)
-            for (int t = 0; t < nt; ++t) {
-                float xm[BW][32];
-                float e[BW];
-#pragma unroll
-                for (int m = 0; m < BW; ++m) {
-                    float part = 0.f;
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        unpack8(*reinterpret_cast<const uint4 *>(sm + W_XE + tc::sw128(t + m, chalf * 4 + c8)),
-                                &xm[m][c8 * 8]);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) part = fmaf(S[c8 * 8 + i], xm[m][c8 * 8 + i], part);
-                    }
-                    if (sthr) red[(chalf * 4 + m) * DD + row] = part;
-                }
-                __syncthreads();
-                if (sthr) {
-#pragma unroll
-                    for (int m = 0; m < BW; ++m) {
-                        const float sxm = red[m * DD + row] + red[(4 + m) * DD + row];
-                        const float y = tile_get(sm, W_VE, t + m, row);
-                        e[m] = reg ? y - sxm : y;
-                    }
-                    const float eta = veta[t], alpha = valpha[t];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        float u = 0.f;
-#pragma unroll
-                        for (int m = 0; m < BW; ++m) u = fmaf(e[m], xm[m][i], u);
-                        S[i] = fmaf(alpha, S[i], eta * u);
-                    }
-                }
-                __syncthreads();
-                if (sthr) {
-                    float part = 0.f;
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        float q8[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(sm + W_Q + tc::sw128(t, chalf * 4 + c8)), q8);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) part = fmaf(S[c8 * 8 + i], q8[i], part);
-                    }
-                    red[(chalf * 4) * DD + row] = part;
-                }
-                __syncthreads();
-                if (sthr && chalf == 0) {
-                    const float o = red[row] + red[4 * DD + row];
-                    static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + row] = __float2bfloat16_rn(o);
-                }
-                __syncthreads();
-            }
-            if (tid == 0 && c + 1 < nch) {
-                load_chunk(c + 1);
-                ++issued;
-            }
-        }
-        // bf16 copy of the new state
-        if (sthr) {
-#pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8)
-                *reinterpret_cast<uint4 *>(sm + W_S + tc::sw128(row, chalf * 4 + c8)) = pack8(&S[c8 * 8]);
-        }
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
-        __syncthreads();
-        WT(7);
-    }
-    WT_END();
-    if (ok && sthr && p.final_state) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) p.final_state[((size_t)bh * DD + row) * DD + chalf * 32 + e] = S[e];
-    }
-    if (!ok && tid == 0) {
-        atomicAdd(&g_w_wait_timeouts, 1u);
-        if (issued > 0) (void)tc::mbar_wait_timeout(tbar, (uint32_t)((issued - 1) & 1), kWaitNs);
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tbase, 512);
-}
-
 
 // ============================================================ Falcon-3A: per-chunk images
 namespace {
@@ -866,7 +337,9 @@ __global__ void __launch_bounds__(NTH, 2)
         tc::fence_after_sync();
         // ---- Zt[r] = sum over the tokens whose window holds row r of w_t y_r, and
         //      the band terms sum_k P[t][t+k] Zacc_{t+1}[t+k] (warps 0-1: thread =
-        //      channel j = lane), in blocks of 8 tokens as in w_chunk_kernel
+        //      channel j = lane), in blocks of 8 tokens: the sums over rows final
+        //      before a block are one batch of dot products, one per row of the
+        //      block's windows; only the block's own rows are walked token by token
         if (tid < DD) {
             const int j = tid;
             constexpr int NB = 8, RB = NB + BW - 1;  // tokens and rows of a block
@@ -1286,7 +759,10 @@ __global__ void __launch_bounds__(NTH, 1)
         // ---- the chunk's system in token order for 128 right-hand sides (warps
         //      0-3: thread = row = lane): rows 0-63 the value channels (S_0 = 0),
         //      rows 64-127 the rows of the identity (values zero, (S_0 x_r) = x_r[c]);
-        //      in blocks of 8 tokens as in w_chunk_kernel
+        //      in blocks of 8 tokens: the sums over rows final before a block are
+        //      one batch of dot products, one per row of the block's windows (every
+        //      (token, slot) pair that reads a row starts from its sum); only the
+        //      block's own rows, in registers, are walked token by token
         if (tid < 2 * DD) {
             const int rw = tid;
             const bool vrow = rw < DD;  // a value channel; else identity row c = rw - 64
@@ -1568,19 +1044,6 @@ bool make_map(CUtensorMap *m, const void *base, int BH, int L) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BW>
-int launch_w(const FwdParams &p, const WMaps &maps, cudaStream_t s) {
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        cudaFuncSetAttribute(w_chunk_kernel<BW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)W_SMEM);
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
-    w_chunk_kernel<BW><<<(unsigned)(p.B * p.H), NTH, W_SMEM, s>>>(p, maps);
-    return cudaGetLastError() == cudaSuccess ? 0 : -7;  // FALCON_ERR_LAUNCH
-}
-
 int w_sm_count() {
     static int counts[64] = {0};
     int dev = 0;
@@ -1646,25 +1109,13 @@ int launch_w_chunk(const FwdParams &p, cudaStream_t s) {
     WMaps maps;
     if (!make_map(&maps.q, p.q, BH, p.L) || !make_map(&maps.k, p.k, BH, p.L) || !make_map(&maps.v, p.v, BH, p.L))
         return 1;
-    if (w_local_covers(p)) {
-        switch (p.window) {
-            case 2: return launch_wl<2>(p, maps, s);
-            case 3: return launch_wl<3>(p, maps, s);
-            default: return launch_wl<4>(p, maps, s);
-        }
-    }
+    if (!w_local_covers(p)) return 1;
     switch (p.window) {
-        case 2: return launch_w<2>(p, maps, s);
-        case 3: return launch_w<3>(p, maps, s);
-        default: return launch_w<4>(p, maps, s);
+        case 2: return launch_wl<2>(p, maps, s);
+        case 3: return launch_wl<3>(p, maps, s);
+        default: return launch_wl<4>(p, maps, s);
     }
 }
-
-#ifdef FALCON_TC_DEBUG
-extern "C" int falcon_w_debug_timer_set(long long *ptr) {
-    return cudaMemcpyToSymbol(g_w_tim, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;
-}
-#endif
 
 unsigned int w_wait_timeouts() {
     unsigned int v = 0;
