@@ -56,6 +56,33 @@ constexpr float kMinLogDecay = -80.f;
 
 __device__ unsigned int g_w_wait_timeouts;
 
+#ifdef FALCON_TC_DEBUG
+// w_reg_local_kernel, block 0, threads 0 and 128: SM cycles per phase summed
+// over the block's units
+__device__ long long *g_wr_tim;
+#define WRT_INIT()                  \
+    long long wrt_acc_[8] = {0};    \
+    long long wrt_prev_ = clock64(); \
+    const bool wrt_on_ = blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == 128)
+#define WRT(k)                                      \
+    do {                                            \
+        if (wrt_on_) {                              \
+            const long long n_ = clock64();         \
+            wrt_acc_[k] += n_ - wrt_prev_;          \
+            wrt_prev_ = n_;                         \
+        }                                           \
+    } while (0)
+#define WRT_END()                                                                              \
+    do {                                                                                       \
+        if (wrt_on_ && g_wr_tim)                                                               \
+            for (int i_ = 0; i_ < 8; ++i_) g_wr_tim[(threadIdx.x ? 8 : 0) + i_] = wrt_acc_[i_]; \
+    } while (0)
+#else
+#define WRT_INIT()
+#define WRT(k)
+#define WRT_END()
+#endif
+
 
 constexpr int LDA = 68;                 // fp32 Gram rows (samples 0-67)
 constexpr int LDZ = 84;                 // fp32 per-row sums: conflict-free float4 along the row
@@ -594,6 +621,7 @@ __global__ void __launch_bounds__(NTH, 1)
     uint32_t phase = 0;  // MMA-completion parity
     bool ok = true;
     int n = 0;
+    WRT_INIT();
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
     const int set = n & 1;
     const uint32_t R_XE = set ? R_XE1 : R_XE0, R_VE = set ? R_VE1 : R_VE0, R_Q = set ? R_Q1 : R_Q0;
@@ -609,6 +637,7 @@ __global__ void __launch_bounds__(NTH, 1)
     if (tid < CH) vbeta[tid] = tid < nt ? __bfloat162float(betap[c0 + tid]) : 0.f;
     ok = tc::mbar_wait_timeout(&tbar[set], (uint32_t)((n >> 1) & 1), kWaitNs);
     ok = __syncthreads_and(ok);
+    WRT(0);
     if (!ok) break;
     if (ok) {
         // ---- samples: rows r < MM normalised in place (four threads per row), rows MM..NR-1 zero
@@ -660,6 +689,7 @@ __global__ void __launch_bounds__(NTH, 1)
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        WRT(1);
         // ---- the Gram and P over the sample rows
         if (tid == ISSUER) {
             tc::fence_after_sync();
@@ -692,6 +722,7 @@ __global__ void __launch_bounds__(NTH, 1)
             }
         }
         __syncthreads();
+        WRT(2);
         if (tid < CH) {
             const int t = tid;
             const float G = vG[t] + (t >= 32 ? misc[0] : 0.f);
@@ -709,6 +740,7 @@ __global__ void __launch_bounds__(NTH, 1)
         ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
         phase ^= 1;
         ok = __syncthreads_and(ok);
+        WRT(3);
     }
     const float GC = misc[2];
     const bool unsafe = !(GC > kMinLogDecay);
@@ -755,6 +787,7 @@ __global__ void __launch_bounds__(NTH, 1)
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        WRT(4);
         tc::fence_after_sync();
         // ---- the chunk's system in token order for 128 right-hand sides (warps
         //      0-3: thread = row = lane): rows 0-63 the value channels (S_0 = 0),
@@ -762,15 +795,20 @@ __global__ void __launch_bounds__(NTH, 1)
         //      in blocks of 8 tokens: the sums over rows final before a block are
         //      one batch of dot products, one per row of the block's windows (every
         //      (token, slot) pair that reads a row starts from its sum); only the
-        //      block's own rows, in registers, are walked token by token
+        //      block's own rows, in registers, are walked token by token.  Warps
+        //      4-7 form each block's sums over the rows final before the block
+        //      ahead of it, while warps 0-3 walk that block; warps 0-3 then add
+        //      the rows of the block just walked (the same order of additions)
+        constexpr int NB = 8, RB = NB + BW - 1;  // tokens and rows of a block
+        static_assert(2 * RB * 2 * DD * 4 <= 4 * TILE, "the sums fit over the Zt^T tiles");
+        float *psum = reinterpret_cast<float *>(sm + R_ZT0);  // [2][RB][128] the sums, by block parity
         if (tid < 2 * DD) {
             const int rw = tid;
             const bool vrow = rw < DD;  // a value channel; else identity row c = rw - 64
             float *za = Za + rw * LDZ;
             auto yv = [&](int r) { return vrow ? tile_get(sm, R_VE, r, rw) : 0.f; };
             auto sxv = [&](int r) { return vrow ? 0.f : tile_get(sm, R_XE, r, rw - DD); };
-            constexpr int NB = 8, RB = NB + BW - 1;  // tokens and rows of a block
-            float zb[RB];                            // rows t0 .. t0+RB-1
+            float zb[RB];  // rows t0 .. t0+RB-1
 #pragma unroll
             for (int k = 0; k < RB; ++k) zb[k] = 0.f;
 #pragma unroll 1
@@ -778,13 +816,17 @@ __global__ void __launch_bounds__(NTH, 1)
                 float bnd[16];
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb) {
-                    const int t0 = tb * 16 + hb * NB;
+                    const int t0 = tb * 16 + hb * NB, blk = tb * 2 + hb;
                     // rows r' < t0 are final (in shared memory): the sum over them
-                    // of A[t+m][r'] Zacc[r'] depends on t+m only, one sum per row
+                    // of A[t+m][r'] Zacc[r'] depends on t+m only, one sum per row;
+                    // rows r' < t0 - NB were summed by warps 4-7 during the last block
+                    tc::named_sync(1, NTH);
                     float crr[RB];
 #pragma unroll
-                    for (int rr = 0; rr < RB; ++rr) crr[rr] = 0.f;
-                    for (int q = 0; q < (t0 >> 2); ++q) {
+                    for (int rr = 0; rr < RB; ++rr) crr[rr] = blk > 0 ? psum[((blk & 1) * RB + rr) * 2 * DD + rw] : 0.f;
+#pragma unroll
+                    for (int q = (t0 >> 2) - NB / 4; q < (t0 >> 2); ++q) {
+                        if (q < 0) continue;
                         const float4 z4 = *reinterpret_cast<const float4 *>(za + q * 4);
 #pragma unroll
                         for (int rr = 0; rr < RB; ++rr) {
@@ -797,25 +839,40 @@ __global__ void __launch_bounds__(NTH, 1)
                     for (int i = 0; i < NB; ++i)
 #pragma unroll
                         for (int m = 0; m < BW; ++m) cr[i][m] = crr[i + m];
+                    // the block's rows of the right-hand side: y_r on a value row,
+                    // (S_0 x_r) = x_r[c] on an identity row
+                    float ev[RB];
+#pragma unroll
+                    for (int rr = 0; rr < RB; ++rr) ev[rr] = vrow ? yv(t0 + rr) : sxv(t0 + rr);
 #pragma unroll
                     for (int i = 0; i < NB; ++i) {
                         const int t = t0 + i;
-                        const float wt = vw[t], gm = vgm1[t], kt = vkap[t];
+                        const float wt = vw[t], kt = vkap[t];
+                        const float cf = vrow ? wt : -(wt * vgm1[t]);  // w_t, or -w_t e^{G_{t-1}}
 #pragma unroll
                         for (int m = 0; m < BW; ++m) {
                             float acc = cr[i][m];
-                            // rows t0 .. t+BW-2 still accumulating: registers
+                            // rows t0 .. t+BW-2 still accumulating: registers, their
+                            // Gram entries four at a time
+                            const float *arow = At + (t + m) * LDA + t0;
 #pragma unroll
-                            for (int k = 0; k < i + BW - 1; ++k) acc = fmaf(At[(t + m) * LDA + t0 + k], zb[k], acc);
-                            const int r = t + m;
-                            cr[i][m] = wt * (yv(r) - gm * sxv(r)) - kt * acc;
+                            for (int k4 = 0; k4 < (i + BW - 1 + 3) / 4; ++k4) {
+                                const float4 a4 = *reinterpret_cast<const float4 *>(arow + k4 * 4);
+                                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    if (k4 * 4 + e < i + BW - 1) acc = fmaf(av[e], zb[k4 * 4 + e], acc);
+                            }
+                            cr[i][m] = cf * ev[i + m] - kt * acc;
                         }
                         // z_{t,m} lands on row t+m only after every slot of token t used the old sums
 #pragma unroll
                         for (int m = 0; m < BW; ++m) zb[i + m] += cr[i][m];
+                        const float4 pb4 = *reinterpret_cast<const float4 *>(pband + t * 4);
+                        const float pbv[4] = {pb4.x, pb4.y, pb4.z, pb4.w};
                         float bsum = 0.f;
 #pragma unroll
-                        for (int k = 1; k < BW; ++k) bsum = fmaf(pband[t * 4 + k], zb[i + k], bsum);
+                        for (int k = 1; k < BW; ++k) bsum = fmaf(pbv[k], zb[i + k], bsum);
                         bnd[hb * NB + i] = bsum;
                     }
                     // rows t0 .. t0+7 are final; rows t0+8 .. carry into the next block
@@ -836,16 +893,43 @@ __global__ void __launch_bounds__(NTH, 1)
                 const float4 z4 = *reinterpret_cast<const float4 *>(za + q4 * 4);
                 zr[q4 * 4] = z4.x; zr[q4 * 4 + 1] = z4.y; zr[q4 * 4 + 2] = z4.z; zr[q4 * 4 + 3] = z4.w;
             }
+            tc::named_sync(2, 2 * DD);  // every row's last sums read before Zt^T covers them
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8)
                 *reinterpret_cast<uint4 *>(sm + R_ZT0 + tc::sw128(rw, c8)) = pack8(&zr[c8 * 8]);
 #pragma unroll
             for (int c8 = 0; c8 < 2; ++c8)
                 *reinterpret_cast<uint4 *>(sm + R_ZT1 + tc::sw128(rw, c8)) = pack8(&zr[64 + c8 * 8]);
+        } else {
+            // warps 4-7, one thread per row: at each block's start, the sums for
+            // the next block over the rows final now (its t0 - NB rows)
+            const int rw = tid - 2 * DD;
+            const float *za = Za + rw * LDZ;
+#pragma unroll 1
+            for (int blk = 0; blk < CH / NB; ++blk) {
+                const int t0 = blk * NB;
+                tc::named_sync(1, NTH);
+                if (blk + 1 < CH / NB) {
+                    float crr[RB];
+#pragma unroll
+                    for (int rr = 0; rr < RB; ++rr) crr[rr] = 0.f;
+                    for (int q = 0; q < (t0 >> 2); ++q) {
+                        const float4 z4 = *reinterpret_cast<const float4 *>(za + q * 4);
+#pragma unroll
+                        for (int rr = 0; rr < RB; ++rr) {
+                            const float4 a4 = *reinterpret_cast<const float4 *>(At + (t0 + NB + rr) * LDA + q * 4);
+                            crr[rr] = fmaf(a4.x, z4.x, fmaf(a4.y, z4.y, fmaf(a4.z, z4.z, fmaf(a4.w, z4.w, crr[rr]))));
+                        }
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < RB; ++rr) psum[(((blk + 1) & 1) * RB + rr) * 2 * DD + rw] = crr[rr];
+                }
+            }
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        WRT(5);
         if (tid == ISSUER) {
             tc::fence_after_sync();
             issue_k(tbase + RC_DS, sbase + R_ZT0, sbase + R_XT0, DD, sbase + R_ZT1, sbase + R_XT1, 1);  // Zt^T X
@@ -855,6 +939,7 @@ __global__ void __launch_bounds__(NTH, 1)
         ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
         phase ^= 1;
         ok = __syncthreads_and(ok);
+        WRT(6);
         if (ok) {
             tc::fence_after_sync();
             // ---- the image, every thread one row (0-127) and half of the tokens
@@ -991,6 +1076,7 @@ __global__ void __launch_bounds__(NTH, 1)
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
+    WRT(7);
     if (tid == 0) {
         gc_ws[u] = __expf(GC);
         tc::bulk_store(img_ws + (size_t)u * IMG, sbase + R_XE, IMG);
@@ -1008,6 +1094,7 @@ __global__ void __launch_bounds__(NTH, 1)
     }
     tc::fence_before_sync();
     __syncthreads();
+    WRT_END();
     if (warp == 0) tc::tmem_dealloc(tbase, 512);
 }
 
@@ -1116,6 +1203,12 @@ int launch_w_chunk(const FwdParams &p, cudaStream_t s) {
         default: return launch_wl<4>(p, maps, s);
     }
 }
+
+#ifdef FALCON_TC_DEBUG
+extern "C" int falcon_wr_debug_timer_set(long long *ptr) {
+    return cudaMemcpyToSymbol(g_wr_tim, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 unsigned int w_wait_timeouts() {
     unsigned int v = 0;
