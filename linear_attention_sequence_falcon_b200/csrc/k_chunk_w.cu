@@ -62,6 +62,7 @@ __device__ unsigned int g_w_wait_timeouts;
 __device__ long long *g_wr_tim;
 #define WRT_INIT()                  \
     long long wrt_acc_[8] = {0};    \
+    long long wrt_bar_ = 0, wrs_[2] = {0, 0}, wrs0_ = 0; \
     long long wrt_prev_ = clock64(); \
     const bool wrt_on_ = blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == 128)
 #define WRT(k)                                      \
@@ -76,8 +77,33 @@ __device__ long long *g_wr_tim;
     do {                                                                                       \
         if (wrt_on_ && g_wr_tim)                                                               \
             for (int i_ = 0; i_ < 8; ++i_) g_wr_tim[(threadIdx.x ? 8 : 0) + i_] = wrt_acc_[i_]; \
+        if (wrt_on_ && g_wr_tim) g_wr_tim[16 + (threadIdx.x ? 1 : 0)] = wrt_bar_;                 \
+        if (wrt_on_ && g_wr_tim)                                                               \
+            for (int i_ = 0; i_ < 2; ++i_) g_wr_tim[18 + (threadIdx.x ? 2 : 0) + i_] = wrs_[i_];    \
+    } while (0)
+// cycles a walk thread spends in its per-block barrier
+#define WRB(stmt)                                       \
+    do {                                                \
+        const long long b0_ = wrt_on_ ? clock64() : 0;  \
+        stmt;                                           \
+        if (wrt_on_) wrt_bar_ += clock64() - b0_;       \
+    } while (0)
+#define WRS_B()                          \
+    do {                                 \
+        if (wrt_on_) wrs0_ = clock64();  \
+    } while (0)
+#define WRS_E(k)                                  \
+    do {                                          \
+        if (wrt_on_) {                            \
+            const long long n_ = clock64();       \
+            wrs_[k] += n_ - wrs0_;                \
+            wrs0_ = n_;                           \
+        }                                         \
     } while (0)
 #else
+#define WRS_B()
+#define WRS_E(k)
+#define WRB(stmt) stmt
 #define WRT_INIT()
 #define WRT(k)
 #define WRT_END()
@@ -621,20 +647,21 @@ __global__ void __launch_bounds__(NTH, 1)
     uint32_t phase = 0;  // MMA-completion parity
     bool ok = true;
     int n = 0;
+    // beta of a unit's tokens (threads t < CH), read a unit ahead
+    auto beta_of = [&](int w) {
+        const int wbh = w / nch, wc0 = (w - wbh * nch) * CH;
+        return tid < min(CH, L - wc0)
+                   ? __bfloat162float(static_cast<const __nv_bfloat16 *>(p.beta)[(size_t)wbh * L + wc0 + tid])
+                   : 0.f;
+    };
+    float bnext = tid < CH && (int)blockIdx.x < units ? beta_of(blockIdx.x) : 0.f;
     WRT_INIT();
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
     const int set = n & 1;
     const uint32_t R_XE = set ? R_XE1 : R_XE0, R_VE = set ? R_VE1 : R_VE0, R_Q = set ? R_Q1 : R_Q0;
     const int bh = u / nch, c = u - bh * nch, c0 = c * CH, nt = min(CH, L - c0);
     const float lam = p.lambda[bh % p.H];
-    const __nv_bfloat16 *betap = static_cast<const __nv_bfloat16 *>(p.beta) + (size_t)bh * L;
-    if (tid == 0 && u + (int)gridDim.x < units) {
-        // the other set's last image has been read out by its bulk store
-        tc::bulk_wait_read();
-        load_unit(u + gridDim.x, set ^ 1);
-        ++loads;
-    }
-    if (tid < CH) vbeta[tid] = tid < nt ? __bfloat162float(betap[c0 + tid]) : 0.f;
+    if (tid < CH) vbeta[tid] = bnext;
     ok = tc::mbar_wait_timeout(&tbar[set], (uint32_t)((n >> 1) & 1), kWaitNs);
     ok = __syncthreads_and(ok);
     WRT(0);
@@ -741,6 +768,13 @@ __global__ void __launch_bounds__(NTH, 1)
         phase ^= 1;
         ok = __syncthreads_and(ok);
         WRT(3);
+        if (tid == 0 && u + (int)gridDim.x < units) {
+            // the other set's last image has been read out by its bulk store
+            tc::bulk_wait_read();
+            load_unit(u + gridDim.x, set ^ 1);
+            ++loads;
+        }
+        if (tid < CH && u + (int)gridDim.x < units) bnext = beta_of(u + gridDim.x);
     }
     const float GC = misc[2];
     const bool unsafe = !(GC > kMinLogDecay);
@@ -800,8 +834,8 @@ __global__ void __launch_bounds__(NTH, 1)
         //      ahead of it, while warps 0-3 walk that block; warps 0-3 then add
         //      the rows of the block just walked (the same order of additions)
         constexpr int NB = 8, RB = NB + BW - 1;  // tokens and rows of a block
-        static_assert(2 * RB * 2 * DD * 4 <= 4 * TILE, "the sums fit over the Zt^T tiles");
-        float *psum = reinterpret_cast<float *>(sm + R_ZT0);  // [2][RB][128] the sums, by block parity
+        static_assert(2 * 2 * RB * 2 * DD * 4 <= 4 * TILE, "the sums fit over the Zt^T tiles");
+        float *psum = reinterpret_cast<float *>(sm + R_ZT0);  // [2][2][RB][128] the sums, by block parity and half
         if (tid < 2 * DD) {
             const int rw = tid;
             const bool vrow = rw < DD;  // a value channel; else identity row c = rw - 64
@@ -811,6 +845,7 @@ __global__ void __launch_bounds__(NTH, 1)
             float zb[RB];  // rows t0 .. t0+RB-1
 #pragma unroll
             for (int k = 0; k < RB; ++k) zb[k] = 0.f;
+            WRS_B();
 #pragma unroll 1
             for (int tb = 0; tb < 4; ++tb) {
                 float bnd[16];
@@ -820,10 +855,13 @@ __global__ void __launch_bounds__(NTH, 1)
                     // rows r' < t0 are final (in shared memory): the sum over them
                     // of A[t+m][r'] Zacc[r'] depends on t+m only, one sum per row;
                     // rows r' < t0 - NB were summed by warps 4-7 during the last block
-                    tc::named_sync(1, NTH);
+                    WRB(tc::named_sync(1, NTH));
                     float crr[RB];
 #pragma unroll
-                    for (int rr = 0; rr < RB; ++rr) crr[rr] = blk > 0 ? psum[((blk & 1) * RB + rr) * 2 * DD + rw] : 0.f;
+                    for (int rr = 0; rr < RB; ++rr)
+                        crr[rr] = blk > 0 ? psum[((blk & 1) * 2 * RB + rr) * 2 * DD + rw] +
+                                                psum[(((blk & 1) * 2 + 1) * RB + rr) * 2 * DD + rw]
+                                          : 0.f;
 #pragma unroll
                     for (int q = (t0 >> 2) - NB / 4; q < (t0 >> 2); ++q) {
                         if (q < 0) continue;
@@ -834,40 +872,53 @@ __global__ void __launch_bounds__(NTH, 1)
                             crr[rr] = fmaf(a4.x, z4.x, fmaf(a4.y, z4.y, fmaf(a4.z, z4.z, fmaf(a4.w, z4.w, crr[rr]))));
                         }
                     }
-                    float cr[NB][BW];
-#pragma unroll
-                    for (int i = 0; i < NB; ++i)
-#pragma unroll
-                        for (int m = 0; m < BW; ++m) cr[i][m] = crr[i + m];
                     // the block's rows of the right-hand side: y_r on a value row,
                     // (S_0 x_r) = x_r[c] on an identity row
                     float ev[RB];
 #pragma unroll
                     for (int rr = 0; rr < RB; ++rr) ev[rr] = vrow ? yv(t0 + rr) : sxv(t0 + rr);
+                    // crr[R]: the sum for row t0+R over the rows final so far; each
+                    // row of the block adds its term once it is final
 #pragma unroll
                     for (int i = 0; i < NB; ++i) {
                         const int t = t0 + i;
                         const float wt = vw[t], kt = vkap[t];
                         const float cf = vrow ? wt : -(wt * vgm1[t]);  // w_t, or -w_t e^{G_{t-1}}
+                        float cri[BW];
 #pragma unroll
                         for (int m = 0; m < BW; ++m) {
-                            float acc = cr[i][m];
-                            // rows t0 .. t+BW-2 still accumulating: registers, their
-                            // Gram entries four at a time
+                            // rows t0+i .. t+BW-2 still accumulating: registers, their
+                            // Gram entries read four at a time
                             const float *arow = At + (t + m) * LDA + t0;
+                            float acc = crr[i + m];
 #pragma unroll
-                            for (int k4 = 0; k4 < (i + BW - 1 + 3) / 4; ++k4) {
+                            for (int k4 = i / 4; k4 <= (i + BW - 2) / 4; ++k4) {
                                 const float4 a4 = *reinterpret_cast<const float4 *>(arow + k4 * 4);
                                 const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    if (k4 * 4 + e < i + BW - 1) acc = fmaf(av[e], zb[k4 * 4 + e], acc);
+                                for (int e = 0; e < 4; ++e) {
+                                    const int k = k4 * 4 + e;
+                                    if (k >= i && k <= i + BW - 2) acc = fmaf(av[e], zb[k], acc);
+                                }
                             }
-                            cr[i][m] = cf * ev[i + m] - kt * acc;
+                            cri[m] = cf * ev[i + m] - kt * acc;
                         }
                         // z_{t,m} lands on row t+m only after every slot of token t used the old sums
 #pragma unroll
-                        for (int m = 0; m < BW; ++m) zb[i + m] += cr[i][m];
+                        for (int m = 0; m < BW; ++m) zb[i + m] += cri[m];
+                        // row t0+i is final: its term into the sums of the block's later
+                        // rows (the Gram is symmetric: row t0+i, columns t0+R)
+                        const float *acol = At + t * LDA + t0;
+#pragma unroll
+                        for (int k4 = (i + 1) / 4; k4 * 4 < RB; ++k4) {
+                            const float4 a4 = *reinterpret_cast<const float4 *>(acol + k4 * 4);
+                            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int R = k4 * 4 + e;
+                                if (R > i && R < RB) crr[R] = fmaf(av[e], zb[i], crr[R]);
+                            }
+                        }
                         const float4 pb4 = *reinterpret_cast<const float4 *>(pband + t * 4);
                         const float pbv[4] = {pb4.x, pb4.y, pb4.z, pb4.w};
                         float bsum = 0.f;
@@ -883,6 +934,7 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 tc::tmem_st16(tl + RC_G + tb * 16, bnd);
             }
+            WRS_E(0);
             // rows 64 .. 64+BW-2 end the chunk in registers; samples beyond are zero
 #pragma unroll
             for (int k = 0; k < BW - 1; ++k) za[CH + k] = zb[k];
@@ -894,6 +946,7 @@ __global__ void __launch_bounds__(NTH, 1)
                 zr[q4 * 4] = z4.x; zr[q4 * 4 + 1] = z4.y; zr[q4 * 4 + 2] = z4.z; zr[q4 * 4 + 3] = z4.w;
             }
             tc::named_sync(2, 2 * DD);  // every row's last sums read before Zt^T covers them
+            WRS_E(1);
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8)
                 *reinterpret_cast<uint4 *>(sm + R_ZT0 + tc::sw128(rw, c8)) = pack8(&zr[c8 * 8]);
@@ -901,30 +954,42 @@ __global__ void __launch_bounds__(NTH, 1)
             for (int c8 = 0; c8 < 2; ++c8)
                 *reinterpret_cast<uint4 *>(sm + R_ZT1 + tc::sw128(rw, c8)) = pack8(&zr[64 + c8 * 8]);
         } else {
-            // warps 4-7, one thread per row: at each block's start, the sums for
-            // the next block over the rows final now (its t0 - NB rows)
-            const int rw = tid - 2 * DD;
-            const float *za = Za + rw * LDZ;
+            // warps 4-7: at each block's start, the sums for the next block over
+            // the rows final now (its t0 - NB rows); a thread takes two rows (rw,
+            // rw + 64), warps 4-5 the first half of those rows and warps 6-7 the
+            // second, so that each Gram row read serves two right-hand sides
+            const int h = tid - 2 * DD, qh = h >> 6, rw = h & (DD - 1);
+            const float *za0 = Za + rw * LDZ, *za1 = Za + (rw + DD) * LDZ;
+            WRS_B();
 #pragma unroll 1
             for (int blk = 0; blk < CH / NB; ++blk) {
                 const int t0 = blk * NB;
-                tc::named_sync(1, NTH);
+                WRB(tc::named_sync(1, NTH));
                 if (blk + 1 < CH / NB) {
-                    float crr[RB];
+                    float c0r[RB], c1r[RB];
 #pragma unroll
-                    for (int rr = 0; rr < RB; ++rr) crr[rr] = 0.f;
-                    for (int q = 0; q < (t0 >> 2); ++q) {
-                        const float4 z4 = *reinterpret_cast<const float4 *>(za + q * 4);
+                    for (int rr = 0; rr < RB; ++rr) c0r[rr] = c1r[rr] = 0.f;
+                    const int q0 = qh ? (t0 >> 3) : 0, q1 = qh ? (t0 >> 2) : (t0 >> 3);
+#pragma unroll 2
+                    for (int q = q0; q < q1; ++q) {
+                        const float4 z0 = *reinterpret_cast<const float4 *>(za0 + q * 4);
+                        const float4 z1 = *reinterpret_cast<const float4 *>(za1 + q * 4);
 #pragma unroll
                         for (int rr = 0; rr < RB; ++rr) {
                             const float4 a4 = *reinterpret_cast<const float4 *>(At + (t0 + NB + rr) * LDA + q * 4);
-                            crr[rr] = fmaf(a4.x, z4.x, fmaf(a4.y, z4.y, fmaf(a4.z, z4.z, fmaf(a4.w, z4.w, crr[rr]))));
+                            c0r[rr] = fmaf(a4.x, z0.x, fmaf(a4.y, z0.y, fmaf(a4.z, z0.z, fmaf(a4.w, z0.w, c0r[rr]))));
+                            c1r[rr] = fmaf(a4.x, z1.x, fmaf(a4.y, z1.y, fmaf(a4.z, z1.z, fmaf(a4.w, z1.w, c1r[rr]))));
                         }
                     }
+                    float *ps = psum + ((((blk + 1) & 1) * 2 + qh) * RB) * 2 * DD;
 #pragma unroll
-                    for (int rr = 0; rr < RB; ++rr) psum[(((blk + 1) & 1) * RB + rr) * 2 * DD + rw] = crr[rr];
+                    for (int rr = 0; rr < RB; ++rr) {
+                        ps[rr * 2 * DD + rw] = c0r[rr];
+                        ps[rr * 2 * DD + rw + DD] = c1r[rr];
+                    }
                 }
             }
+            WRS_E(0);
         }
         tc::fence_proxy_async();
         tc::fence_before_sync();
