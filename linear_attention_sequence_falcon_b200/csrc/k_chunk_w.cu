@@ -62,7 +62,7 @@ __device__ unsigned int g_w_wait_timeouts;
 __device__ long long *g_wr_tim;
 #define WRT_INIT()                  \
     long long wrt_acc_[8] = {0};    \
-    long long wrt_bar_ = 0, wrs_[2] = {0, 0}, wrs0_ = 0; \
+    long long wrt_bar_ = 0, wrs_[6] = {0, 0, 0, 0, 0, 0}, wrs0_ = 0; \
     long long wrt_prev_ = clock64(); \
     const bool wrt_on_ = blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == 128)
 #define WRT(k)                                      \
@@ -79,7 +79,7 @@ __device__ long long *g_wr_tim;
             for (int i_ = 0; i_ < 8; ++i_) g_wr_tim[(threadIdx.x ? 8 : 0) + i_] = wrt_acc_[i_]; \
         if (wrt_on_ && g_wr_tim) g_wr_tim[16 + (threadIdx.x ? 1 : 0)] = wrt_bar_;                 \
         if (wrt_on_ && g_wr_tim)                                                               \
-            for (int i_ = 0; i_ < 2; ++i_) g_wr_tim[18 + (threadIdx.x ? 2 : 0) + i_] = wrs_[i_];    \
+            for (int i_ = 0; i_ < 6; ++i_) g_wr_tim[24 + (threadIdx.x ? 6 : 0) + i_] = wrs_[i_];    \
     } while (0)
 // cycles a walk thread spends in its per-block barrier
 #define WRB(stmt)                                       \
@@ -570,7 +570,7 @@ constexpr uint32_t R_PM1 = 17 * TILE;   // rows t, samples 64-79
 constexpr uint32_t R_A = 18 * TILE;                   // fp32 A[r][r'], r < 68
 constexpr uint32_t R_ZA = R_A + 68 * LDA * 4;         // fp32 Zacc[row][r], 128 rows (token path: outputs)
 constexpr uint32_t R_VEC = R_ZA + 2 * DD * LDZ * 4;   // scalars: the V_* layout up to the band, then
-constexpr int RV_RED = V_RED, RV_MISC = V_RED + 2 * 4 * 2 * DD, RV_END = RV_MISC + 16;  // red over 128 rows
+constexpr int RV_RED = V_RED, RV_MISC = V_RED + 2 * 4 * 2 * DD, RV_EG = RV_MISC + 16, RV_END = RV_EG + CH;  // red over 128 rows; e^{G_t}
 constexpr uint32_t R_BAR = R_VEC + RV_END * 4;  // MMA barrier, one load barrier per set
 constexpr uint32_t R_SMEM = R_BAR + 64 + 1024;
 static_assert(R_SMEM <= 227 * 1024, "shared memory");
@@ -596,7 +596,7 @@ __global__ void __launch_bounds__(NTH, 1)
     float *vec = reinterpret_cast<float *>(sm + R_VEC);
     float *sqn = vec + V_SQN, *vbeta = vec + V_BETA, *veta = vec + V_ETA, *valpha = vec + V_ALPHA, *vG = vec + V_G,
           *vw = vec + V_W, *vkap = vec + V_KAP, *vgm1 = vec + V_GM1, *pband = vec + V_PB, *red = vec + RV_RED,
-          *misc = vec + RV_MISC;
+          *misc = vec + RV_MISC, *veg = vec + RV_EG;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + R_BAR);
     uint64_t *tbar = bar + 1;  // [2] the loads of input set 0 / 1
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 3);
@@ -647,21 +647,21 @@ __global__ void __launch_bounds__(NTH, 1)
     uint32_t phase = 0;  // MMA-completion parity
     bool ok = true;
     int n = 0;
-    // beta of a unit's tokens (threads t < CH), read a unit ahead
+    // beta of a unit's tokens (threads t < CH), read a unit ahead and widened
+    // only when it is stored, so that no thread waits for the load
     auto beta_of = [&](int w) {
         const int wbh = w / nch, wc0 = (w - wbh * nch) * CH;
-        return tid < min(CH, L - wc0)
-                   ? __bfloat162float(static_cast<const __nv_bfloat16 *>(p.beta)[(size_t)wbh * L + wc0 + tid])
-                   : 0.f;
+        return tid < min(CH, L - wc0) ? static_cast<const __nv_bfloat16 *>(p.beta)[(size_t)wbh * L + wc0 + tid]
+                                      : __float2bfloat16_rn(0.f);
     };
-    float bnext = tid < CH && (int)blockIdx.x < units ? beta_of(blockIdx.x) : 0.f;
+    __nv_bfloat16 bnext = tid < CH && (int)blockIdx.x < units ? beta_of(blockIdx.x) : __float2bfloat16_rn(0.f);
     WRT_INIT();
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
     const int set = n & 1;
     const uint32_t R_XE = set ? R_XE1 : R_XE0, R_VE = set ? R_VE1 : R_VE0, R_Q = set ? R_Q1 : R_Q0;
     const int bh = u / nch, c = u - bh * nch, c0 = c * CH, nt = min(CH, L - c0);
     const float lam = p.lambda[bh % p.H];
-    if (tid < CH) vbeta[tid] = bnext;
+    if (tid < CH) vbeta[tid] = __bfloat162float(bnext);
     ok = tc::mbar_wait_timeout(&tbar[set], (uint32_t)((n >> 1) & 1), kWaitNs);
     ok = __syncthreads_and(ok);
     WRT(0);
@@ -761,6 +761,7 @@ __global__ void __launch_bounds__(NTH, 1)
             vgm1[t] = __expf(Gm);
             __syncwarp();
             vG[t] = G;
+            veg[t] = __expf(G);
             if (t == 0) misc[2] = GC;
         }
         __syncthreads();
@@ -1007,6 +1008,7 @@ __global__ void __launch_bounds__(NTH, 1)
         WRT(6);
         if (ok) {
             tc::fence_after_sync();
+            WRS_B();
             // ---- the image, every thread one row (0-127) and half of the tokens
             //      and columns: value rows give O0^T and B, identity rows Qt and
             //      T - g_C I (transposed as they are stored)
@@ -1020,11 +1022,12 @@ __global__ void __launch_bounds__(NTH, 1)
                 tc::tmem_ld16(tl + RC_I + t0, iv);
                 tc::tmem_ld16(tl + RC_G + t0, bv);
                 tc::tmem_wait_ld();
+                WRS_E(5);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int t = t0 + i;
                     const float sq = vrow ? 0.f : tile_get(sm, R_Q, t, cc);
-                    o[i] = t < nt ? __expf(vG[t]) * fmaf(ig, iv[i] + bv[i], sq) : 0.f;
+                    o[i] = t < nt ? veg[t] * fmaf(ig, iv[i] + bv[i], sq) : 0.f;
                 }
                 if (vrow) {
                     *reinterpret_cast<uint4 *>(stg + 2 * TILE + rowmajor8(row, t0 >> 3)) = pack8(&o[0]);
@@ -1035,6 +1038,7 @@ __global__ void __launch_bounds__(NTH, 1)
                         *reinterpret_cast<__nv_bfloat16 *>(stg + TILE + tc::sw128(t0 + i, cc >> 3) + (uint32_t)(cc & 7) * 2) =
                             __float2bfloat16_rn(o[i]);
                 }
+                WRS_E(2);
             }
 #pragma unroll
             for (int k2 = 0; k2 < 2; ++k2) {
@@ -1053,6 +1057,7 @@ __global__ void __launch_bounds__(NTH, 1)
                             __float2bfloat16_rn(dv[i]);
                 }
             }
+            WRS_E(3);
         }
     } else if (ok) {
         // ---- a chunk whose decay leaves the fp32 range of the factorised form:
@@ -1141,6 +1146,7 @@ __global__ void __launch_bounds__(NTH, 1)
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
+    WRS_E(4);
     WRT(7);
     if (tid == 0) {
         gc_ws[u] = __expf(GC);
