@@ -224,6 +224,7 @@ __global__ void __launch_bounds__(NTH, 2)
     float *vec = reinterpret_cast<float *>(sm + U_VEC);
     float *sqn = vec + V_SQN, *vbeta = vec + V_BETA, *veta = vec + V_ETA, *valpha = vec + V_ALPHA, *vG = vec + V_G,
           *vw = vec + V_W, *pband = vec + V_PB, *misc = vec + V_MISC;
+    float *veg = vec + V_KAP;  // e^{G_t} (the slot of the regression family's eta/alpha)
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + U_BAR);
     uint64_t *tbar = bar + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
@@ -354,6 +355,7 @@ __global__ void __launch_bounds__(NTH, 2)
             vw[t] = __expf(GC - G) * veta[t];
             __syncwarp();
             vG[t] = G;
+            veg[t] = __expf(G);
             if (t == 0) misc[2] = GC;
         }
         __syncthreads();
@@ -456,7 +458,7 @@ __global__ void __launch_bounds__(NTH, 2)
             const int t = e >> 3, c16 = e & 7;
             float q8[8];
             unpack8(*reinterpret_cast<const uint4 *>(sm + U_Q + tc::sw128(t, c16)), q8);
-            const float g = __expf(vG[t]);
+            const float g = veg[t];
 #pragma unroll
             for (int i = 0; i < 8; ++i) q8[i] *= g;
             *reinterpret_cast<uint4 *>(stg + tc::sw128(t, c16)) = pack8(q8);
@@ -474,7 +476,7 @@ __global__ void __launch_bounds__(NTH, 2)
                     tc::tmem_ld16(tl + U_G + t0, bv);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) o[i] = t0 + i < nt ? __expf(vG[t0 + i]) * (ig * (iv[i] + bv[i])) : 0.f;
+                    for (int i = 0; i < 16; ++i) o[i] = t0 + i < nt ? veg[t0 + i] * (ig * (iv[i] + bv[i])) : 0.f;
                     *reinterpret_cast<uint4 *>(stg + TILE + rowmajor8(j, t0 >> 3)) = pack8(&o[0]);
                     *reinterpret_cast<uint4 *>(stg + TILE + rowmajor8(j, (t0 >> 3) + 1)) = pack8(&o[8]);
                 }
