@@ -85,8 +85,9 @@ constexpr uint32_t F_PM = 16 * TILE;  // P o mask (s <= t): 64 rows t x 64 s
 constexpr uint32_t F_G = 17 * TILE;   // fp32 G[t][j] at gidx(t, j)
 constexpr int LDA = 68;               // fp32 row stride of A (16-byte rows, conflict-free stores)
 constexpr uint32_t F_A = F_G + CH * DD * 4;     // fp32 A[t][s] for s < t, zero above
-constexpr uint32_t F_VEC = F_A + CH * LDA * 4;  // |x|^2 [64], 1/(eps+|x|^2) [64], half sums [256], G_C [128]
-constexpr uint32_t F_BAR = F_VEC + (64 + 64 + 2 * DD + DD) * 4;
+constexpr uint32_t F_VEC = F_A + CH * LDA * 4;  // |x|^2 [64], 1/(eps+|x|^2) [64], group log sums [256], G_C [128],
+                                                // group products [256]
+constexpr uint32_t F_BAR = F_VEC + (64 + 64 + 2 * DD + DD + 2 * DD) * 4;
 constexpr uint32_t F_SMEM = F_BAR + 64 + 1024;
 // tensor memory (512 columns)
 constexpr uint32_t C_PA = 0;    // [X;Q] X^T: A rows t (lanes 0-63), P rows t (lanes 64-127); 64 columns
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
     float *rinv = sqn + 64;
     float *hsum = rinv + 64;
     float *gcv = hsum + 2 * DD;
+    float *hprod = gcv + DD;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + F_BAR);
     uint64_t *tbar = bar + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
@@ -226,38 +228,48 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
             issue_gemm(tbase + C_S, sbase + F_S, 2 * TILE, sbase + F_IN, 2 * TILE, 2, 128);
             tc::mma_commit(bar);
         }
-        // ---- log decays: thread (token group h, channel jj), TG running sums in registers; X^T
+        // ---- decays: thread (token group h, channel jj), TG running log sums and
+        //      products in registers; X^T.  F_G then holds e^{G_t} (as products of
+        //      the factors), or G_t itself in a chunk whose G_C is -80 or below
+        bool unsafe;
         {
             constexpr int NG = 256 / NJ, TG = CH / NG;
             const int h = tid / NJ, jj = tid % NJ;
-            float Gl[TG];
-            float acc = 0.f;
+            float Gl[TG], Pl[TG];
+            float acc = 0.f, prod = 1.f;
 #pragma unroll
             for (int i = 0; i < TG; ++i) {
                 const int t = h * TG + i;
                 const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
-                acc += __logf(fmaxf(1.f - eta * lam, kAlphaFloor));
+                const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
+                acc += __logf(alpha);
+                prod *= alpha;
                 Gl[i] = acc;
+                Pl[i] = prod;
             }
             hsum[h * NJ + jj] = acc;
+            hprod[h * NJ + jj] = prod;
             for (int g = warp; g < 32; g += NTH / 32) {
                 const int half = g >> 4, rb = (g >> 1) & 7, cb0 = (g & 1) * 4;
                 transpose4(sbase + F_IN + half * 2 * TILE, rb, cb0, sbase + F_XT, half * 64);
             }
             __syncthreads();
-            float base = 0.f, tot = 0.f;
+            float base = 0.f, tot = 0.f, pbase = 1.f;
 #pragma unroll
             for (int h2 = 0; h2 < NG; ++h2) {
                 const float hs = hsum[h2 * NJ + jj];
-                if (h2 < h) base += hs;
+                if (h2 < h) {
+                    base += hs;
+                    pbase *= hprod[h2 * NJ + jj];
+                }
                 tot += hs;
             }
+            unsafe = __syncthreads_or(!(tot > kMinLogDecay)) != 0;
 #pragma unroll
-            for (int i = 0; i < TG; ++i) Gt[gidx(h * TG + i, jj)] = base + Gl[i];
+            for (int i = 0; i < TG; ++i) Gt[gidx(h * TG + i, jj)] = unsafe ? base + Gl[i] : pbase * Pl[i];
             if (h == 0) gcv[jj] = tot;
         }
         __syncthreads();
-        const bool unsafe = __syncthreads_or(tid < NJ && !(gcv[tid] > kMinLogDecay)) != 0;
         F2T(2);
         ok = tc::mbar_wait_timeout(bar, phase, kWaitNs);
         phase ^= 1;
@@ -308,7 +320,7 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
             const int slot = DUP ? (warp >> 2) + 2 * (quarter >> 1) : (warp >> 2);
             const int src = (32 / TPC) * slot + lane / TPC;  // the channel's lane inside this quarter
             const int jj = 32 * (DUP ? (quarter & 1) : quarter) + src;
-            const float gc = gcv[jj];
+            const float egc = Gt[gidx(CH - 1, jj)];  // e^{G_C}
             float Z[64];
 #pragma unroll
             for (int s = 0; s < 64; ++s) Z[s] = 0.f;
@@ -323,17 +335,17 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
                 for (int hb = 0; hb < 2; ++hb) {
                     const int t0 = tb * 16 + hb * 8, tp = t0 + PT * part;  // this thread's PT tokens
                     float r[8], kap[8], cr[8], rm[PT], km[PT];
-                    float Gp = tp > 0 ? Gt[gidx(tp - 1, jj)] : 0.f;
+                    float egp = tp > 0 ? Gt[gidx(tp - 1, jj)] : 1.f;  // e^{G_{t-1}}
 #pragma unroll
                     for (int i = 0; i < PT; ++i) {
                         const int t = tp + i;
                         const float eta = pair_get(sm, F_B, t, jj) * rinv[t];
                         const float alpha = fmaxf(1.f - eta * lam, kAlphaFloor);
-                        const float G = Gt[gidx(t, jj)];
+                        const float eg = Gt[gidx(t, jj)];
                         const float x = pick<TPC, PT>(&xs[hb * 8 + i], part);
-                        rm[i] = __expf(gc - G) * eta * (pair_get(sm, F_V, t, jj) - __expf(Gp) * x);
+                        rm[i] = __fdividef(egc, eg) * eta * (pair_get(sm, F_V, t, jj) - egp * x);
                         km[i] = __fdividef(eta, alpha);
-                        Gp = G;
+                        egp = eg;
                     }
                     if constexpr (TPC == 2) {
 #pragma unroll
@@ -496,7 +508,7 @@ __global__ void __launch_bounds__(NTH, 1) f2_chunk_kernel(FwdParams p, const __g
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int t = t0 + i;
-                    const float o = __expf(Gt[gidx(t, jl)]) * fmaf(ig, av[i], iv[i]);
+                    const float o = Gt[gidx(t, jl)] * fmaf(ig, av[i], iv[i]);
                     if (t < nt)
                         static_cast<__nv_bfloat16 *>(p.out)[((size_t)bh * L + c0 + t) * DD + J0 + jl] =
                             __float2bfloat16_rn(o);
