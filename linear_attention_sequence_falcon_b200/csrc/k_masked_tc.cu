@@ -335,6 +335,7 @@ __global__ void __launch_bounds__(NTHM, 1)
                 va[t] = __expf(t > 0 ? vG[t - 1] : 0.f);   // e^{Gamma_{t-1} - Gamma_{I0-1}}
                 vc[t] = __expf(vG[t]);                      // e^{Gamma_t - Gamma_{I0-1}}
                 vb[t] = __expf(GE - vG[t]) * veta[t];       // e^{Gamma_Iend - Gamma_t} eta_t
+                vla[t] = __expf(-vG[t]) * veta[t];          // e^{Gamma_{I0-1} - Gamma_t} eta_t (the logs are read)
             }
             if (tid == 0) gend[I] = Gprev + GE;
             tc::fence_proxy_async();
@@ -343,6 +344,7 @@ __global__ void __launch_bounds__(NTHM, 1)
         __syncthreads();
         tc::fence_after_sync();
         const float GE = vG[BM - 1];
+        const bool fact = GE > -80.f;  // every e^{-G_t} of the block inside the fp32 range
         if (issuer) {  // X_I for the later row blocks
             tc::bulk_store(xs + (size_t)I * TB, sb + M_AQ, TB);
             tc::bulk_commit();
@@ -503,7 +505,9 @@ __global__ void __launch_bounds__(NTHM, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int s2 = chalf * 32 + i;
-                        MT[t * LDM + s2] = s2 < t ? __expf(gm - vG[s2]) * veta[s2] * v[i] : 0.f;
+                        // e^{G_{t-1} - G_s} eta_s: factorised while the block's G stays above -80
+                        const float f = fact ? a * vla[s2] : __expf(gm - vG[s2]) * veta[s2];
+                        MT[t * LDM + s2] = s2 < t ? f * v[i] : 0.f;
                         YF[t * LDM + s2] -= a * r[i];
                     }
                 }
@@ -513,7 +517,8 @@ __global__ void __launch_bounds__(NTHM, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int s2 = chalf * 32 + i;
-                    PD[t * LDM + s2] = s2 <= t ? __expf(gt - vG[s2]) * veta[s2] * v[i] : 0.f;
+                    const float f = fact ? c * vla[s2] : __expf(gt - vG[s2]) * veta[s2];
+                    PD[t * LDM + s2] = s2 <= t ? f * v[i] : 0.f;
                     OF[t * LDM + s2] = c * r[i];
                 }
             }
